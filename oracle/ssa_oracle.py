@@ -1,0 +1,303 @@
+"""Plain fp64 CPU oracle of SSA dual-stream attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline / reference legs of ``bench.py`` may import this module.  It
+shares no code with the CUDA path (``block_sparse_full_b200``) and never
+imports it; its inputs come from ``block_sparse_full_b200.inputs`` (random
+draws only) or from hand-written fixtures.
+
+Everything here is the plain definition of what one SSA attention layer
+computes, written out in float64 with numpy (a matmul is the only library
+primitive used).  No blocking, online softmax or fusion: each quantity is
+formed directly from its definition so it can be checked by eye against the
+method as the SSA pages describe it.
+
+Sources (page title, section):
+
+* "Sintesi Tecnica: SSA (Sparse Sparse Attention)", gist.science (Italian
+  technical summary), section 2 "Metodologia": the sparse-attention stream is
+  block-sparse attention, the full-attention stream is ordinary (causal)
+  softmax attention that gives gradient to every token; the counterpart
+  output of the opposite mode is computed only for alignment; the alignment
+  loss has two parts, L_sparsity (full output imitates sparse output, which
+  lowers the discarded attention mass delta(t)) and L_commit (sparse output
+  stays near the full output); the total objective adds alpha * L_align.
+* Same page, section 1 "Definizione del Problema": sparse training normalises
+  only over the selected subset; the approximation error grows linearly with
+  the discarded attention mass (weight on tokens the sparse rule did not
+  select).
+* Same page, section 4 "Risultati Sperimentali", "Efficienza": at inference SSA
+  runs the same operations as MoBA (mean-pooled key blocks scored against the
+  query block, top-k blocks, the current block always attended).
+* "Résumé technique : SSA", gist.science (French), sections 1, 2 and 4: the
+  same statements.
+
+Readings where the pages are silent (each restated in the design doc):
+
+* pooling: mean of the keys of a block and mean of the queries of a query
+  block; score s_ij = Qbar_i . Kbar_j (equal to the mean over the block's
+  queries of q_t . Kbar_j, by linearity);
+* query-block size equals key-block size; selection is per query block;
+* the diagonal (current) block is always selected and counts inside the
+  budget k; block 0 is forced only with ``force_sink`` (also inside k);
+* candidates rank by (score descending, block index ascending); with fewer
+  causal blocks than k all are taken; indices are emitted ascending, padded
+  with -1;
+* L_sparsity = L_commit = mean over all B*H*T*d elements of
+  (h_full - h_sparse)^2; L_sparsity sends gradient only to h_full, L_commit
+  only to h_sparse (stop-gradient on the opposite stream); the weights
+  w_s, w_c absorb alpha;
+* no gradient flows through block selection or through delta(t).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "f64", "pool_blocks", "block_scores", "select_blocks", "block_selection_matrix",
+    "attn_fwd_dual", "align_loss", "alignment_upstream", "attn_bwd",
+]
+
+
+def f64(x) -> np.ndarray:
+    """Exact float64 copy of a torch tensor or array (bf16/f32 -> f64 is exact)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------
+# Block selection (sparse-attention stream's block-sparse rule)
+# --------------------------------------------------------------------------
+
+def pool_blocks(x: np.ndarray, block: int) -> np.ndarray:
+    """Mean of each run of ``block`` consecutive rows of x [T, d] -> [T/block, d].
+
+    MoBA-identical block representation ("Efficienza", section 4).  With
+    bf16/f32 inputs the block sums are exact in float64, and division by a
+    power-of-two block is exact too, so this value is the same whatever the
+    summation order.
+    """
+    T, d = x.shape
+    n = T // block
+    return x[: n * block].reshape(n, block, d).sum(axis=1) / float(block)
+
+
+def block_scores(q: np.ndarray, k: np.ndarray, block: int) -> np.ndarray:
+    """s[i, j] = Qbar_i . Kbar_j for one (batch, head); q, k are [T, d]."""
+    return pool_blocks(q, block) @ pool_blocks(k, block).T
+
+
+def select_blocks(q, k, block: int, topk: int, force_sink: bool = False):
+    """Per query block i: the set S_i of key blocks the sparse stream attends.
+
+    S_i = forced_i  u  top-(k - |forced_i|) of the remaining causal blocks
+    j < i by (score descending, j ascending), all of them if fewer remain.
+    forced_i = {i}, plus {0} when ``force_sink`` and i > 0.
+
+    q, k: [B, H, T, d].  Returns
+      idx    int32  [B, H, n, topk]  ascending block indices, -1 padded
+      cnt    int32  [B, H, n]        |S_i|
+      mask   uint32 [B, H, n, ceil(n/32)]  bit j of S_i
+      margin float64 [B, H, n]  score gap between the last selected and the
+             first rejected candidate (inf when nothing was rejected); a GPU
+             selection may only differ from this one where it is ~0.
+    """
+    q, k = f64(q), f64(k)
+    B, H, T, _ = q.shape
+    n = T // block
+    words = (n + 31) // 32
+    idx = np.full((B, H, n, topk), -1, dtype=np.int32)
+    cnt = np.zeros((B, H, n), dtype=np.int32)
+    mask = np.zeros((B, H, n, words), dtype=np.uint32)
+    margin = np.full((B, H, n), np.inf)
+    for b in range(B):
+        for h in range(H):
+            s = block_scores(q[b, h], k[b, h], block)
+            for i in range(n):
+                forced = [i] + ([0] if (force_sink and i > 0) else [])
+                cand = [j for j in range(i) if j not in forced]
+                r = max(topk - len(forced), 0)
+                ranked = sorted(cand, key=lambda j: (-s[i, j], j))
+                chosen = sorted(set(forced) | set(ranked[:r]))
+                if 0 < r < len(ranked):
+                    margin[b, h, i] = s[i, ranked[r - 1]] - s[i, ranked[r]]
+                cnt[b, h, i] = len(chosen)
+                idx[b, h, i, : len(chosen)] = chosen
+                for j in chosen:
+                    mask[b, h, i, j // 32] |= np.uint32(1 << (j % 32))
+    return idx, cnt, mask, margin
+
+
+def block_selection_matrix(idx: np.ndarray, cnt: np.ndarray) -> np.ndarray:
+    """Boolean [.., n, n] with [i, j] = (j in S_i), from idx/cnt [.., n, k]."""
+    lead = idx.shape[:-2]
+    n = idx.shape[-2]
+    sel = np.zeros(lead + (n, n), dtype=bool)
+    for pos in np.ndindex(*lead, n):
+        c = int(cnt[pos])
+        sel[pos][idx[pos][:c]] = True
+    return sel
+
+
+# --------------------------------------------------------------------------
+# Forward: both streams, discarded mass, log-sum-exps
+# --------------------------------------------------------------------------
+
+def _fwd_rows(q, k, v, blocksel, block, sm_scale, rows):
+    """Both attention outputs for query rows ``rows`` of one (batch, head)."""
+    tmax = int(rows.max()) + 1
+    s = np.arange(tmax)
+    x = sm_scale * (q[rows] @ k[:tmax].T)                 # logits  [r, tmax]
+    causal = s[None, :] <= rows[:, None]
+    in_sel = blocksel[rows // block][:, s // block]        # s's block in S_i
+    sel = causal & in_sel
+    uns = causal & ~in_sel
+    m = np.where(causal, x, -np.inf).max(axis=1)
+    p = np.where(causal, np.exp(x - m[:, None]), 0.0)     # unnormalised weights
+    p_sel = np.where(sel, p, 0.0)
+    p_uns = np.where(uns, p, 0.0)
+    l_sel = p_sel.sum(axis=1)
+    l_uns = p_uns.sum(axis=1)
+    o_sel = p_sel @ v[:tmax]
+    o_uns = p_uns @ v[:tmax]
+    l_all = l_sel + l_uns
+    h_full = (o_sel + o_uns) / l_all[:, None]             # softmax over all s <= t
+    h_sparse = o_sel / l_sel[:, None]                     # softmax over selected s only
+    with np.errstate(invalid="ignore", divide="ignore"):
+        h_unsel = np.where(l_uns[:, None] > 0, o_uns / l_uns[:, None], 0.0)
+    return {
+        "h_full": h_full,
+        "h_sparse": h_sparse,
+        "h_unsel": h_unsel,
+        "delta": l_uns / l_all,
+        "lse_full": m + np.log(l_all),
+        "lse_sparse": m + np.log(l_sel),
+        "sqdiff": ((h_full - h_sparse) ** 2).sum(axis=1),
+    }
+
+
+def attn_fwd_dual(q, k, v, idx, cnt, block: int, sm_scale: float, rows=None,
+                  max_elems: int = 1 << 23):
+    """Full-attention and block-sparse outputs of the same Q, K, V.
+
+    For query t (block i) and every key s <= t, with x = sm_scale * q_t . k_s:
+      h_full(t)   = sum_s softmax_{s<=t}(x) v_s
+      h_sparse(t) = sum_{s: block(s) in S_i} softmax over those s of x, times v_s
+      delta(t)    = full-softmax mass on keys whose block is not in S_i
+      lse_full    = log sum_{s<=t} e^x,  lse_sparse = log sum_{selected} e^x
+      sqdiff(t)   = sum_c (h_full - h_sparse)_c^2
+    (sections 1 and 2 of the technical summaries; the sparse stream
+    normalises over the selected subset only).
+
+    q, k, v: [B, H, T, d]; idx, cnt from ``select_blocks``.  ``rows``
+    optionally restricts the query rows (same rows for every batch/head);
+    outputs then have T' = len(rows) rows.  Extra output ``h_unsel`` is the
+    softmax average of v over the unselected keys (0 where there are none).
+    """
+    q, k, v = f64(q), f64(k), f64(v)
+    B, H, T, d = q.shape
+    rows = np.arange(T) if rows is None else np.asarray(sorted(rows), dtype=np.int64)
+    R = len(rows)
+    blocksel = block_selection_matrix(idx, cnt)
+    dv = v.shape[-1]  # value width (equal to d in the layer; tests may widen it)
+    out = {name: np.zeros((B, H, R, dv)) for name in ("h_full", "h_sparse", "h_unsel")}
+    for name in ("delta", "lse_full", "lse_sparse", "sqdiff"):
+        out[name] = np.zeros((B, H, R))
+    for b in range(B):
+        for h in range(H):
+            step = max(1, max_elems // T)
+            for start in range(0, R, step):
+                chunk = rows[start:start + step]
+                res = _fwd_rows(q[b, h], k[b, h], v[b, h], blocksel[b, h], block,
+                                sm_scale, chunk)
+                for name, val in res.items():
+                    out[name][b, h, start:start + step] = val
+    return out
+
+
+def align_loss(h_full, h_sparse, w_sparsity: float = 1.0, w_commit: float = 1.0):
+    """(w_s * L_sparsity, w_c * L_commit), both the mean squared difference of
+    the two outputs over all elements (section 2, "Allineamento
+    Bidirezionale"; the distance is the reading stated in the module header)."""
+    hf, hs = f64(h_full), f64(h_sparse)
+    L = float(np.mean((hf - hs) ** 2))
+    return w_sparsity * L, w_commit * L
+
+
+def alignment_upstream(h_full, h_sparse, dh_full, dh_sparse, w_s, w_c, n_total):
+    """Gradients reaching each output: the caller's upstream plus the
+    alignment terms with stop-gradient on the opposite stream.
+
+    d(w_s L_sparsity)/d h_full   = w_s * 2/N * (h_full - h_sparse)   (h_sparse held fixed)
+    d(w_c L_commit)/d h_sparse   = w_c * 2/N * (h_sparse - h_full)   (h_full held fixed)
+    """
+    hf, hs = f64(h_full), f64(h_sparse)
+    g_full = f64(dh_full) + w_s * (2.0 / n_total) * (hf - hs)
+    g_sparse = f64(dh_sparse) + w_c * (2.0 / n_total) * (hs - hf)
+    return g_full, g_sparse
+
+
+# --------------------------------------------------------------------------
+# Backward through both streams
+# --------------------------------------------------------------------------
+
+def _bwd_head(q, k, v, blocksel, block, sm_scale, g_full, g_sparse):
+    """dq, dk, dv of  sum(g_full * h_full) + sum(g_sparse * h_sparse)  for one
+    (batch, head), selection held fixed.  Written with the explicit softmax
+    Jacobian: for P = softmax(x) over a key set and upstream dP = g v^T,
+    dx = P * (dP - rowsum(P * dP))."""
+    T = q.shape[0]
+    t = np.arange(T)
+    x = sm_scale * (q @ k.T)
+    causal = t[None, :] <= t[:, None]
+    in_sel = blocksel[t // block][:, t // block]
+    sel = causal & in_sel
+
+    def softmax_over(allowed):
+        xm = np.where(allowed, x, -np.inf)
+        m = xm.max(axis=1, keepdims=True)
+        e = np.where(allowed, np.exp(xm - m), 0.0)
+        return e / e.sum(axis=1, keepdims=True)
+
+    p_full = softmax_over(causal)       # full-attention stream: every s <= t
+    p_sparse = softmax_over(sel)        # sparse stream: selected blocks only
+    dv = p_full.T @ g_full + p_sparse.T @ g_sparse
+    dp_full = g_full @ v.T
+    dp_sparse = g_sparse @ v.T
+    dx = p_full * (dp_full - (p_full * dp_full).sum(axis=1, keepdims=True))
+    dx += p_sparse * (dp_sparse - (p_sparse * dp_sparse).sum(axis=1, keepdims=True))
+    dq = sm_scale * dx @ k
+    dk = sm_scale * dx.T @ q
+    return dq, dk, dv
+
+
+def attn_bwd(q, k, v, idx, cnt, block: int, sm_scale: float, dh_full, dh_sparse,
+             w_sparsity: float = 0.0, w_commit: float = 0.0, n_total=None):
+    """Gradients of  <dh_full, h_full> + <dh_sparse, h_sparse>
+    + w_s * L_sparsity + w_c * L_commit  with respect to q, k, v.
+
+    The full stream carries gradient to every causal key (section 2, "Full
+    Attention Stream"); the sparse stream only to selected keys; the
+    alignment terms follow ``alignment_upstream``.  ``n_total`` is the
+    element count N of the whole layer output (defaults to q.size) so that a
+    caller may pass a slice of heads.  Returns (dq, dk, dv) float64.
+    """
+    q, k, v = f64(q), f64(k), f64(v)
+    B, H, T, d = q.shape
+    n_total = q.size if n_total is None else n_total
+    fw = attn_fwd_dual(q, k, v, idx, cnt, block, sm_scale)
+    g_full, g_sparse = alignment_upstream(fw["h_full"], fw["h_sparse"], dh_full,
+                                          dh_sparse, w_sparsity, w_commit, n_total)
+    blocksel = block_selection_matrix(idx, cnt)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            dq[b, h], dk[b, h], dv[b, h] = _bwd_head(
+                q[b, h], k[b, h], v[b, h], blocksel[b, h], block, sm_scale,
+                g_full[b, h], g_sparse[b, h])
+    return dq, dk, dv

@@ -1,0 +1,74 @@
+"""The pins must be sharp: plant a plausible mistake in a copy of the oracle
+(on the CPU) and check that at least one pin fails.  Each mutation edits one
+line of the oracle's source and loads the result as a separate module; the
+real oracle is untouched."""
+import importlib.util
+import os
+import types
+
+import pytest
+
+import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "ssa_oracle.py")
+
+# (original text, planted mistake)
+MUTATIONS = {
+    "drop_causal_mask": ("causal = s[None, :] <= rows[:, None]",
+                         "causal = s[None, :] <= rows[:, None] + 1"),
+    "sparse_normalised_over_all": ("h_sparse = o_sel / l_sel[:, None]",
+                                   "h_sparse = o_sel / l_all[:, None]"),
+    "delta_of_selected_mass": ("\"delta\": l_uns / l_all,", "\"delta\": l_sel / l_all,"),
+    "lse_missing_max": ("\"lse_full\": m + np.log(l_all),", "\"lse_full\": np.log(l_all),"),
+    "pool_first_half_only": ("return x[: n * block].reshape(n, block, d).sum(axis=1) / float(block)",
+                             "return x[: n * block].reshape(n, block, d)[:, : block // 2].sum(axis=1) / float(block)"),
+    "scores_transposed": ("return pool_blocks(q, block) @ pool_blocks(k, block).T",
+                          "return pool_blocks(k, block) @ pool_blocks(q, block).T"),
+    "ties_to_higher_index": ("ranked = sorted(cand, key=lambda j: (-s[i, j], j))",
+                             "ranked = sorted(cand, key=lambda j: (-s[i, j], -j))"),
+    "diagonal_outside_budget": ("r = max(topk - len(forced), 0)",
+                                "r = max(topk - len(forced) + 1, 0)"),
+    "commit_gradient_sign": ("g_sparse = f64(dh_sparse) + w_c * (2.0 / n_total) * (hs - hf)",
+                             "g_sparse = f64(dh_sparse) + w_c * (2.0 / n_total) * (hf - hs)"),
+    "bwd_missing_scale": ("dk = sm_scale * dx.T @ q", "dk = dx.T @ q"),
+    "bwd_dv_sparse_dropped": ("dv = p_full.T @ g_full + p_sparse.T @ g_sparse",
+                              "dv = p_full.T @ g_full"),
+    "loss_sum_not_mean": ("L = float(np.mean((hf - hs) ** 2))", "L = float(np.sum((hf - hs) ** 2))"),
+}
+
+PIN_TESTS = [
+    lambda: pins.test_worked_example_closed_form(),
+    lambda: pins.test_worked_example_sink_flag(),
+    lambda: pins.test_pooling_closed_forms(),
+    lambda: pins.test_scores_are_mean_of_per_query_scores(),
+    lambda: pins.test_topk_ties_go_to_lower_block_index(),
+    lambda: pins.test_mask_words_beyond_32_blocks(),
+    lambda: pins.test_full_budget_reduces_to_causal_attention(),
+    lambda: pins.test_streams_match_library_attention_with_masks(),
+    lambda: pins.test_lse_against_library_logsumexp(),
+    lambda: pins.test_align_loss_is_library_mse(),
+    lambda: pins.test_bwd_central_finite_differences(40.0, 25.0),
+    lambda: pins.test_bwd_matches_library_autograd(),
+]
+
+
+def _mutant(name):
+    before, after = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor not unique/present: {name}"
+    mod = types.ModuleType(f"ssa_oracle_mutant_{name}")
+    exec(compile(src.replace(before, after), SRC, "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, monkeypatch):
+    monkeypatch.setattr(pins, "O", _mutant(name))
+    caught = 0
+    for t in PIN_TESTS:
+        try:
+            t()
+        except (AssertionError, ValueError, IndexError):
+            caught += 1
+    assert caught > 0, f"no pin detects the planted mistake {name!r}"
