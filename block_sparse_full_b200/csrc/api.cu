@@ -1,0 +1,226 @@
+// Host side of the C ABI declared in include/ssa.h: argument validation,
+// workspace sizing, kernel-path choice and status reporting.  Every compute
+// step runs in the kernels of the sibling .cu files.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <cmath>
+
+#include "ssa_internal.h"
+
+namespace ssa {
+
+namespace {
+thread_local char g_last_error[512] = "";
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape/method checks shared by every entry point.
+int validate(const ssa_params_t* p) {
+    if (!p) return fail(SSA_ERR_INVALID_ARG, "params is NULL");
+    if (p->B <= 0 || p->H <= 0 || p->T <= 0 || p->D <= 0)
+        return fail(SSA_ERR_INVALID_ARG, "B, H, T, D must be positive (got %d, %d, %d, %d)", p->B,
+                    p->H, p->T, p->D);
+    if (p->dtype != SSA_F32 && p->dtype != SSA_BF16)
+        return fail(SSA_ERR_INVALID_ARG, "unknown dtype %d", p->dtype);
+    if (p->block != 64 && p->block != 128)
+        return fail(SSA_ERR_UNSUPPORTED, "block must be 64 or 128 (got %d)", p->block);
+    if (p->T % p->block != 0)
+        return fail(SSA_ERR_INVALID_ARG, "T (%d) must be a multiple of block (%d)", p->T, p->block);
+    if (p->D != 64 && p->D != 128)
+        return fail(SSA_ERR_UNSUPPORTED, "head dim D must be 64 or 128 (got %d)", p->D);
+    const int n = p->T / p->block;
+    if (p->topk < 1 || p->topk > n)
+        return fail(SSA_ERR_INVALID_ARG, "topk must be in [1, T/block = %d] (got %d)", n, p->topk);
+    if ((p->flags & SSA_FLAG_FORCE_SINK) && p->topk < 2)
+        return fail(SSA_ERR_INVALID_ARG, "FORCE_SINK needs topk >= 2 (got %d)", p->topk);
+    if (p->flags & ~(unsigned)(SSA_FLAG_FORCE_SINK | SSA_FLAG_FORCE_SIMT))
+        return fail(SSA_ERR_INVALID_ARG, "unknown flag bits 0x%x", p->flags);
+    if (!(p->sm_scale > 0.f) || !std::isfinite(p->sm_scale))
+        return fail(SSA_ERR_INVALID_ARG, "sm_scale must be positive and finite");
+    if ((double)p->B * p->H * p->T * p->D > 9.0e15)
+        return fail(SSA_ERR_INVALID_ARG, "tensor too large");
+    return SSA_OK;
+}
+
+int need_ptr(const void* ptr, const char* name) {
+    if (!ptr) return fail(SSA_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(ptr)) return fail(SSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return SSA_OK;
+}
+
+int opt_ptr(const void* ptr, const char* name) {
+    if (ptr && !aligned16(ptr)) return fail(SSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return SSA_OK;
+}
+
+int need_ws(void* ws, size_t have, size_t need, const char* what) {
+    if (need == 0) return SSA_OK;
+    if (have < need)
+        return fail(SSA_ERR_WORKSPACE, "%s needs %zu workspace bytes, got %zu", what, need, have);
+    if (!ws) return fail(SSA_ERR_WORKSPACE, "%s: workspace pointer is NULL", what);
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+        return fail(SSA_ERR_INVALID_ARG, "%s: workspace must be 256-byte aligned", what);
+    return SSA_OK;
+}
+
+bool use_tc(const ssa_params_t& p) {
+    return !(p.flags & SSA_FLAG_FORCE_SIMT) && fwd_tc_supported(p);
+}
+
+size_t fwd_workspace(const ssa_params_t& p) { return use_tc(p) ? fwd_tc_workspace(p) : 0; }
+
+}  // namespace
+
+int fail(int status, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int check_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return SSA_OK;
+}
+
+}  // namespace ssa
+
+using namespace ssa;
+
+#define SSA_TRY(expr)              \
+    do {                           \
+        int _st = (expr);          \
+        if (_st != SSA_OK) return _st; \
+    } while (0)
+
+extern "C" {
+
+size_t ssa_workspace_size(const ssa_params_t* p, int which) {
+    if (validate(p) != SSA_OK) return (size_t)-1;
+    switch (which) {
+        case SSA_WS_SELECT: return select_workspace(*p);
+        case SSA_WS_FWD: return fwd_workspace(*p);
+        case SSA_WS_LOSS: return loss_workspace(*p);
+        case SSA_WS_BWD: return bwd_simt_workspace(*p);
+        default: fail(SSA_ERR_INVALID_ARG, "unknown workspace id %d", which); return (size_t)-1;
+    }
+}
+
+int ssa_select_blocks(const ssa_params_t* p, const void* q, const void* k, int32_t* idx,
+                      int32_t* cnt, uint32_t* mask, void* ws, size_t ws_bytes, void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(validate(p));
+    SSA_TRY(need_ptr(q, "q"));
+    SSA_TRY(need_ptr(k, "k"));
+    SSA_TRY(need_ptr(idx, "idx"));
+    SSA_TRY(need_ptr(cnt, "cnt"));
+    SSA_TRY(need_ptr(mask, "mask"));
+    SSA_TRY(need_ws(ws, ws_bytes, select_workspace(*p), "ssa_select_blocks"));
+    return launch_select(*p, q, k, idx, cnt, mask, ws, static_cast<cudaStream_t>(stream));
+}
+
+int ssa_attn_fwd_dual(const ssa_params_t* p, const void* q, const void* k, const void* v,
+                      const int32_t* idx, const int32_t* cnt, const uint32_t* mask,
+                      void* h_full, void* h_sparse, float* delta, float* lse_full,
+                      float* lse_sparse, float* sqdiff, void* ws, size_t ws_bytes,
+                      void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(validate(p));
+    SSA_TRY(need_ptr(q, "q"));
+    SSA_TRY(need_ptr(k, "k"));
+    SSA_TRY(need_ptr(v, "v"));
+    SSA_TRY(opt_ptr(idx, "idx"));
+    SSA_TRY(opt_ptr(cnt, "cnt"));
+    SSA_TRY(need_ptr(mask, "mask"));
+    SSA_TRY(need_ptr(h_full, "h_full"));
+    SSA_TRY(need_ptr(h_sparse, "h_sparse"));
+    SSA_TRY(need_ptr(delta, "delta"));
+    SSA_TRY(need_ptr(lse_full, "lse_full"));
+    SSA_TRY(need_ptr(lse_sparse, "lse_sparse"));
+    SSA_TRY(need_ptr(sqdiff, "sqdiff_rows"));
+    SSA_TRY(need_ws(ws, ws_bytes, fwd_workspace(*p), "ssa_attn_fwd_dual"));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (use_tc(*p))
+        return launch_fwd_tc(*p, q, k, v, mask, h_full, h_sparse, delta, lse_full, lse_sparse,
+                             sqdiff, ws, s);
+    return launch_fwd_simt(*p, q, k, v, mask, h_full, h_sparse, delta, lse_full, lse_sparse,
+                           sqdiff, s);
+}
+
+int ssa_align_loss(const ssa_params_t* p, const float* sqdiff, float w_s, float w_c,
+                   float* loss_out, void* ws, size_t ws_bytes, void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(validate(p));
+    SSA_TRY(need_ptr(sqdiff, "sqdiff_rows"));
+    SSA_TRY(need_ptr(loss_out, "loss_out"));
+    if (!std::isfinite(w_s) || !std::isfinite(w_c))
+        return fail(SSA_ERR_INVALID_ARG, "loss weights must be finite");
+    SSA_TRY(need_ws(ws, ws_bytes, loss_workspace(*p), "ssa_align_loss"));
+    return launch_loss(*p, sqdiff, w_s, w_c, loss_out, ws, static_cast<cudaStream_t>(stream));
+}
+
+int ssa_attn_bwd(const ssa_params_t* p, const void* q, const void* k, const void* v,
+                 const int32_t* idx, const int32_t* cnt, const uint32_t* mask,
+                 const void* h_full, const void* h_sparse, const float* lse_full,
+                 const float* lse_sparse, const void* dh_full, const void* dh_sparse,
+                 float w_s, float w_c, void* dq, void* dk, void* dv, void* ws,
+                 size_t ws_bytes, void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(validate(p));
+    SSA_TRY(need_ptr(q, "q"));
+    SSA_TRY(need_ptr(k, "k"));
+    SSA_TRY(need_ptr(v, "v"));
+    SSA_TRY(opt_ptr(idx, "idx"));
+    SSA_TRY(opt_ptr(cnt, "cnt"));
+    SSA_TRY(need_ptr(mask, "mask"));
+    SSA_TRY(need_ptr(h_full, "h_full"));
+    SSA_TRY(need_ptr(h_sparse, "h_sparse"));
+    SSA_TRY(need_ptr(lse_full, "lse_full"));
+    SSA_TRY(need_ptr(lse_sparse, "lse_sparse"));
+    SSA_TRY(opt_ptr(dh_full, "dh_full"));
+    SSA_TRY(opt_ptr(dh_sparse, "dh_sparse"));
+    SSA_TRY(need_ptr(dq, "dq"));
+    SSA_TRY(need_ptr(dk, "dk"));
+    SSA_TRY(need_ptr(dv, "dv"));
+    if (!std::isfinite(w_s) || !std::isfinite(w_c))
+        return fail(SSA_ERR_INVALID_ARG, "loss weights must be finite");
+    SSA_TRY(need_ws(ws, ws_bytes, bwd_simt_workspace(*p), "ssa_attn_bwd"));
+    return launch_bwd_simt(*p, q, k, v, mask, h_full, h_sparse, lse_full, lse_sparse, dh_full,
+                           dh_sparse, w_s, w_c, dq, dk, dv, ws, static_cast<cudaStream_t>(stream));
+}
+
+int ssa_device_status(void* stream) {
+    g_last_error[0] = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+    int st = fwd_tc_take_status(s);
+    if (st != SSA_OK) return st;
+    return check_launch("pending");
+}
+
+const char* ssa_status_string(int status) {
+    switch (status) {
+        case SSA_OK: return "ok";
+        case SSA_ERR_INVALID_ARG: return "invalid argument";
+        case SSA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case SSA_ERR_WORKSPACE: return "workspace too small or missing";
+        case SSA_ERR_CUDA: return "CUDA error";
+        case SSA_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+const char* ssa_last_error(void) { return g_last_error; }
+
+int ssa_kernel_path(const ssa_params_t* p) {
+    if (validate(p) != SSA_OK) return -1;
+    return use_tc(*p) ? 1 : 0;
+}
+
+int ssa_version(void) { return (1 << 16) | 0; }
+
+}  // extern "C"

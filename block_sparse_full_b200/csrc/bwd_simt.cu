@@ -1,0 +1,322 @@
+// Backward through both SSA attention streams on CUDA cores (float32
+// arithmetic).  Used for float32 inputs, bf16 with D = 64 and under
+// SSA_FLAG_FORCE_SIMT.
+//
+// Upstream reaching each output ("Sintesi Tecnica: SSA", section 2: the
+// full stream gives gradient to every token; L_sparsity pulls h_full toward
+// h_sparse, L_commit pulls h_sparse toward h_full, each with stop-gradient
+// on the other stream):
+//   G_f = dh_full   + w_s * 2/N * (h_full - h_sparse)
+//   G_s = dh_sparse + w_c * 2/N * (h_sparse - h_full)
+// For query t, key s <= t, x = sigma q_t.k_s:
+//   P_f = exp(x - lse_full(t)),  P_s = exp(x - lse_sparse(t)) on selected s
+//   dS  = P_f (G_f(t).v_s - D_f(t)) + [sel] P_s (G_s(t).v_s - D_s(t))
+//   with D_f = G_f.h_full and D_s = G_s.h_sparse (row dots),
+//   dq_t = sigma sum_s dS k_s,  dk_s = sigma sum_t dS q_t,
+//   dv_s = sum_t P_f G_f(t) + [sel] P_s G_s(t).
+// Three kernels: a row preprocess (G_f, G_s, D_f, D_s into the workspace), a
+// dq kernel over query tiles and a dk/dv kernel over key tiles; no atomics,
+// so results are bitwise repeatable.
+#include "device_util.cuh"
+#include "ssa_internal.h"
+
+namespace ssa {
+namespace {
+
+constexpr int kTile = 32;
+constexpr int kThreads = 128;
+constexpr int kRowsPerWarp = kTile / (kThreads / 32);
+
+struct BwdWs {
+    float* gf;
+    float* gs;
+    float* df;
+    float* ds;
+};
+
+BwdWs carve(const ssa_params_t& p, void* ws) {
+    const size_t big = align_up(num_elems(p) * sizeof(float), 256);
+    const size_t small = align_up(num_rows(p) * sizeof(float), 256);
+    char* b = static_cast<char*>(ws);
+    return {reinterpret_cast<float*>(b), reinterpret_cast<float*>(b + big),
+            reinterpret_cast<float*>(b + 2 * big), reinterpret_cast<float*>(b + 2 * big + small)};
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+bwd_pre_kernel(const T* __restrict__ hf, const T* __restrict__ hs, const T* __restrict__ dhf,
+               const T* __restrict__ dhs, size_t rows, int D, float cf, float cs, BwdWs w) {
+    const size_t row = (size_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float sf = 0.f, ss = 0.f;
+    for (int c = lane; c < D; c += 32) {
+        const size_t e = row * D + c;
+        const float f = to_f32(hf[e]), s = to_f32(hs[e]);
+        const float gf = (dhf ? to_f32(dhf[e]) : 0.f) + cf * (f - s);
+        const float gs = (dhs ? to_f32(dhs[e]) : 0.f) + cs * (s - f);
+        w.gf[e] = gf;
+        w.gs[e] = gs;
+        sf = fmaf(gf, f, sf);
+        ss = fmaf(gs, s, ss);
+    }
+    sf = warp_sum(sf);
+    ss = warp_sum(ss);
+    if (lane == 0) {
+        w.df[row] = sf;
+        w.ds[row] = ss;
+    }
+}
+
+template <int D>
+struct DqSmem {
+    float q[kTile][D], gf[kTile][D], gs[kTile][D];
+    float k[kTile][D + 1], v[kTile][D + 1];
+    float lf[kTile], ls[kTile], df[kTile], ds[kTile];
+    uint32_t mrow[256];
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+              const uint32_t* __restrict__ mask, const float* __restrict__ lse_f,
+              const float* __restrict__ lse_s, BwdWs w, int BH, int T_, int block, int words,
+              float sm_scale, T* __restrict__ dq) {
+    constexpr int DPL = D / 32;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    DqSmem<D>& sm = *reinterpret_cast<DqSmem<D>*>(smem_raw);
+    const int ntiles = T_ / kTile;
+    const int tile = ntiles - 1 - (int)(blockIdx.x / BH);
+    const size_t bh = blockIdx.x % BH;
+    const int t0 = tile * kTile;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t base = bh * (size_t)T_ * D;
+    const size_t rbase = bh * (size_t)T_ + t0;
+
+    for (int e = tid; e < kTile * D; e += kThreads) {
+        const size_t g = base + (size_t)t0 * D + e;
+        sm.q[e / D][e % D] = to_f32(q[g]);
+        sm.gf[e / D][e % D] = w.gf[g];
+        sm.gs[e / D][e % D] = w.gs[g];
+    }
+    if (tid < kTile) {
+        sm.lf[tid] = lse_f[rbase + tid];
+        sm.ls[tid] = lse_s[rbase + tid];
+        sm.df[tid] = w.df[rbase + tid];
+        sm.ds[tid] = w.ds[rbase + tid];
+    }
+    const uint32_t* mrow = mask + (bh * (T_ / block) + t0 / block) * (size_t)words;
+    for (int i = tid; i < words; i += kThreads) sm.mrow[i] = mrow[i];
+
+    float acc[kRowsPerWarp][DPL];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+#pragma unroll
+        for (int u = 0; u < DPL; ++u) acc[r][u] = 0.f;
+
+    for (int s0 = 0; s0 < t0 + kTile; s0 += kTile) {
+        __syncthreads();
+        for (int e = tid; e < kTile * D; e += kThreads) {
+            const size_t g = base + (size_t)s0 * D + e;
+            sm.k[e / D][e % D] = to_f32(k[g]);
+            sm.v[e / D][e % D] = to_f32(v[g]);
+        }
+        __syncthreads();
+        const bool sel = mask_bit(sm.mrow, s0 / block);
+#pragma unroll 1
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int rr = warp * kRowsPerWarp + r;
+            const int t = t0 + rr;
+            const bool valid = s0 + lane <= t;
+            float x = 0.f, dpf = 0.f, dps = 0.f;
+#pragma unroll 16
+            for (int c = 0; c < D; ++c) {
+                x = fmaf(sm.q[rr][c], sm.k[lane][c], x);
+                dpf = fmaf(sm.gf[rr][c], sm.v[lane][c], dpf);
+            }
+            x *= sm_scale;
+            const float pf = valid ? expf(x - sm.lf[rr]) : 0.f;
+            float dsv = pf * (dpf - sm.df[rr]);
+            if (sel) {
+#pragma unroll 16
+                for (int c = 0; c < D; ++c) dps = fmaf(sm.gs[rr][c], sm.v[lane][c], dps);
+                const float lsr = sm.ls[rr];
+                const float ps = (valid && lsr > -INFINITY) ? expf(x - lsr) : 0.f;
+                dsv += ps * (dps - sm.ds[rr]);
+            }
+#pragma unroll 8
+            for (int j = 0; j < kTile; ++j) {
+                const float dj = __shfl_sync(0xffffffffu, dsv, j);
+#pragma unroll
+                for (int u = 0; u < DPL; ++u) acc[r][u] = fmaf(dj, sm.k[j][lane + 32 * u], acc[r][u]);
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+        const size_t row = rbase + warp * kRowsPerWarp + r;
+#pragma unroll
+        for (int u = 0; u < DPL; ++u) dq[row * D + lane + 32 * u] = from_f32<T>(sm_scale * acc[r][u]);
+    }
+}
+
+template <int D>
+struct DkvSmem {
+    float k[kTile][D], v[kTile][D];
+    float q[kTile][D + 1], gf[kTile][D + 1], gs[kTile][D + 1];
+    float lf[kTile], ls[kTile], df[kTile], ds[kTile];
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+bwd_dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                const uint32_t* __restrict__ mask, const float* __restrict__ lse_f,
+                const float* __restrict__ lse_s, BwdWs w, int BH, int T_, int block, int words,
+                float sm_scale, T* __restrict__ dk, T* __restrict__ dv) {
+    constexpr int DPL = D / 32;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    DkvSmem<D>& sm = *reinterpret_cast<DkvSmem<D>*>(smem_raw);
+    const int tile = (int)(blockIdx.x / BH);  // key tile 0 sees every query: first
+    const size_t bh = blockIdx.x % BH;
+    const int s_base = tile * kTile;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t base = bh * (size_t)T_ * D;
+    const int n = T_ / block;
+    const int kblk = s_base / block;
+
+    for (int e = tid; e < kTile * D; e += kThreads) {
+        const size_t g = base + (size_t)s_base * D + e;
+        sm.k[e / D][e % D] = to_f32(k[g]);
+        sm.v[e / D][e % D] = to_f32(v[g]);
+    }
+    float adk[kRowsPerWarp][DPL], adv[kRowsPerWarp][DPL];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+#pragma unroll
+        for (int u = 0; u < DPL; ++u) adk[r][u] = adv[r][u] = 0.f;
+
+    for (int t0 = s_base; t0 < T_; t0 += kTile) {
+        __syncthreads();
+        for (int e = tid; e < kTile * D; e += kThreads) {
+            const size_t g = base + (size_t)t0 * D + e;
+            sm.q[e / D][e % D] = to_f32(q[g]);
+            sm.gf[e / D][e % D] = w.gf[g];
+            sm.gs[e / D][e % D] = w.gs[g];
+        }
+        if (tid < kTile) {
+            const size_t rr = bh * (size_t)T_ + t0 + tid;
+            sm.lf[tid] = lse_f[rr];
+            sm.ls[tid] = lse_s[rr];
+            sm.df[tid] = w.df[rr];
+            sm.ds[tid] = w.ds[rr];
+        }
+        __syncthreads();
+        const uint32_t* mrow = mask + (bh * n + t0 / block) * (size_t)words;
+        const bool sel = mask_bit(mrow, kblk);
+        const int t = t0 + lane;
+#pragma unroll 1
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int rr = warp * kRowsPerWarp + r;
+            const int s = s_base + rr;
+            const bool valid = t >= s;
+            float x = 0.f, dpf = 0.f, dps = 0.f;
+#pragma unroll 16
+            for (int c = 0; c < D; ++c) {
+                x = fmaf(sm.q[lane][c], sm.k[rr][c], x);
+                dpf = fmaf(sm.gf[lane][c], sm.v[rr][c], dpf);
+            }
+            x *= sm_scale;
+            const float pf = valid ? expf(x - sm.lf[lane]) : 0.f;
+            float dsv = pf * (dpf - sm.df[lane]);
+            float ps = 0.f;
+            if (sel) {
+#pragma unroll 16
+                for (int c = 0; c < D; ++c) dps = fmaf(sm.gs[lane][c], sm.v[rr][c], dps);
+                const float lsr = sm.ls[lane];
+                ps = (valid && lsr > -INFINITY) ? expf(x - lsr) : 0.f;
+                dsv += ps * (dps - sm.ds[lane]);
+            }
+#pragma unroll 4
+            for (int j = 0; j < kTile; ++j) {
+                const float pfj = __shfl_sync(0xffffffffu, pf, j);
+                const float psj = __shfl_sync(0xffffffffu, ps, j);
+                const float dj = __shfl_sync(0xffffffffu, dsv, j);
+#pragma unroll
+                for (int u = 0; u < DPL; ++u) {
+                    const int c = lane + 32 * u;
+                    adv[r][u] = fmaf(pfj, sm.gf[j][c], fmaf(psj, sm.gs[j][c], adv[r][u]));
+                    adk[r][u] = fmaf(dj, sm.q[j][c], adk[r][u]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+        const size_t row = bh * (size_t)T_ + s_base + warp * kRowsPerWarp + r;
+#pragma unroll
+        for (int u = 0; u < DPL; ++u) {
+            dk[row * D + lane + 32 * u] = from_f32<T>(sm_scale * adk[r][u]);
+            dv[row * D + lane + 32 * u] = from_f32<T>(adv[r][u]);
+        }
+    }
+}
+
+template <typename T, int D>
+int launch_typed(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                 const uint32_t* mask, const void* hf, const void* hs, const float* lf,
+                 const float* ls, const void* dhf, const void* dhs, float w_s, float w_c,
+                 void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
+    const BwdWs w = carve(p, ws);
+    const size_t rows = num_rows(p);
+    const double two_over_n = 2.0 / (double)num_elems(p);
+    bwd_pre_kernel<T><<<(unsigned)((rows + 3) / 4), kThreads, 0, s>>>(
+        static_cast<const T*>(hf), static_cast<const T*>(hs), static_cast<const T*>(dhf),
+        static_cast<const T*>(dhs), rows, D, (float)(w_s * two_over_n), (float)(w_c * two_over_n), w);
+    int st = check_launch("bwd_pre_kernel");
+    if (st != SSA_OK) return st;
+
+    const int BH = p.B * p.H;
+    const unsigned grid = (unsigned)((size_t)BH * (p.T / kTile));
+    size_t smem = sizeof(DqSmem<D>);
+    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<T, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "bwd_dq: smem attribute: %s", cudaGetErrorString(e));
+    bwd_dq_kernel<T, D><<<grid, kThreads, smem, s>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), mask, lf, ls,
+        w, BH, p.T, p.block, mask_words(p), p.sm_scale, static_cast<T*>(dq));
+    st = check_launch("bwd_dq_kernel");
+    if (st != SSA_OK) return st;
+
+    smem = sizeof(DkvSmem<D>);
+    e = cudaFuncSetAttribute(bwd_dkdv_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "bwd_dkdv: smem attribute: %s", cudaGetErrorString(e));
+    bwd_dkdv_kernel<T, D><<<grid, kThreads, smem, s>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), mask, lf, ls,
+        w, BH, p.T, p.block, mask_words(p), p.sm_scale, static_cast<T*>(dk), static_cast<T*>(dv));
+    return check_launch("bwd_dkdv_kernel");
+}
+
+}  // namespace
+
+size_t bwd_simt_workspace(const ssa_params_t& p) {
+    return 2 * align_up(num_elems(p) * sizeof(float), 256) +
+           2 * align_up(num_rows(p) * sizeof(float), 256);
+}
+
+int launch_bwd_simt(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                    const uint32_t* mask, const void* hf, const void* hs, const float* lf,
+                    const float* ls, const void* dhf, const void* dhs, float w_s, float w_c,
+                    void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
+    if (mask_words(p) > 256) return fail(SSA_ERR_UNSUPPORTED, "bwd_simt: more than 8192 blocks");
+    if ((size_t)p.B * p.H * (p.T / kTile) > 0x7fffffffull)
+        return fail(SSA_ERR_UNSUPPORTED, "bwd_simt: grid too large");
+    const bool bf = p.dtype == SSA_BF16;
+#define SSA_BWD_ARGS p, q, k, v, mask, hf, hs, lf, ls, dhf, dhs, w_s, w_c, dq, dk, dv, ws, s
+    if (p.D == 64)
+        return bf ? launch_typed<__nv_bfloat16, 64>(SSA_BWD_ARGS) : launch_typed<float, 64>(SSA_BWD_ARGS);
+    return bf ? launch_typed<__nv_bfloat16, 128>(SSA_BWD_ARGS) : launch_typed<float, 128>(SSA_BWD_ARGS);
+#undef SSA_BWD_ARGS
+}
+
+}  // namespace ssa

@@ -1,0 +1,526 @@
+// Fused dual-stream forward on the sm_100a tensor cores (bf16 in, fp32
+// accumulate, head dim 128): one pass over the causal K/V of a 128-row query
+// tile produces the full-attention output, the block-sparse output, the
+// discarded mass delta(t) and both log-sum-exps ("Sintesi Tecnica: SSA",
+// section 2: the sparse stream and its full-attention counterpart of the
+// same layer; section 1: the sparse stream normalises over the selected
+// subset only).
+//
+// CTA = (query tile of 128 rows, batch*head), 256 threads:
+//   warp 0      TMA producer: Q once, then K_j and V_j into 2-stage rings
+//   warp 1      TMEM owner and MMA issuer (one thread):
+//                 S_j = Q K_j^T          (tcgen05 SS, into S buffer j%2)
+//                 O_sel/O_uns += P_j V_j  (tcgen05 TS, P read from TMEM)
+//   warps 4..7  softmax: thread = query row = TMEM lane.  Reads S_j, keeps
+//               one running max for both streams, splits the row sum into
+//               l_sel / l_uns by the selection mask and writes P_j (bf16)
+//               back into the S buffer for the PV product.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O_sel [256,384) O_uns [384,512).
+//
+// A 128-key tile holds one or two key blocks and the 128 query rows one or
+// two query blocks.  For each 64-key half the selection is read for both
+// query blocks; when they agree the half's PV goes to one accumulator, when
+// they differ ("mixed") P is written twice with complementary rows zeroed
+// and both accumulators receive one MMA each.
+//
+// The running max is only raised (and O rescaled) when a row's tile max
+// exceeds it by more than 2^8; the final normalisation divides by sums taken
+// against the same stale max, so the result is unchanged.
+//
+// Every mbarrier wait is bounded (wall-clock limit); on expiry the kernel
+// records SSA_ERR_TIMEOUT in a device status word, the other roles stop,
+// in-flight tensor-core work is drained and TMEM is released.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "ssa_internal.h"
+#include "tc_util.cuh"
+
+namespace ssa {
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;  // query rows per tile
+constexpr int BN = 128;  // keys per tile
+constexpr int HD = 128;  // head dim
+constexpr int kThreads = 256;
+constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB
+constexpr uint32_t HALF_BYTES = 128 * 128;    // [128 rows x 64 cols] bf16 box, 16 KB
+constexpr int kMaxWords = 256;                // mask words per query block (n <= 8192)
+
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + TILE_BYTES;
+constexpr uint32_t OFF_V = OFF_K + 2 * TILE_BYTES;
+constexpr uint32_t OFF_BAR = OFF_V + 2 * TILE_BYTES;
+constexpr int NBAR = 16;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // [0] tmem base, [1] abort flag
+constexpr uint32_t OFF_MASK = OFF_MISC + 16;       // mask rows of the two query blocks
+constexpr uint32_t SMEM_USED = OFF_MASK + 2 * kMaxWords * 4;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+
+enum : int {
+    B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7,
+    B_SREADY = 9, B_PREADY = 11, B_PVDONE = 13, B_DRAIN = 14
+};
+
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_OSEL = 256, TM_OUNS = 384;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kLn2 = 0.693147180559945309f;
+
+__device__ unsigned int g_fwd_tc_status;
+
+struct FwdArgs {
+    __nv_bfloat16* h_full;
+    __nv_bfloat16* h_sparse;
+    float* delta;
+    float* lse_full;
+    float* lse_sparse;
+    float* sqdiff;
+    const uint32_t* mask;
+    int BH, T, block, words, n_blocks;
+    float scale_log2;  // sm_scale * log2(e)
+    unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ bool bit(const uint32_t* row, int j) {
+    return (row[j >> 5] >> (j & 31)) & 1u;
+}
+
+// Selection of key-tile J, half h, for the tile's two query blocks (rows
+// 0-63 and 64-127), with don't-care rows made to agree: query rows that see
+// none of the half's keys (diagonal tile, block 64, h = 1) and rows past T.
+__device__ __forceinline__ void half_sel(const uint32_t* mrow, int J, int I, int h, int block,
+                                         bool ragged1, bool& s0, bool& s1) {
+    const int kb = (J * BN + 64 * h) / block;
+    s0 = bit(mrow, kb);
+    s1 = bit(mrow + kMaxWords, kb);
+    if (block == 64 && J == I && h == 1) s0 = s1;
+    if (ragged1) s1 = s0;
+}
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > limit_ns) return false;
+    return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
+    uint32_t* mrow = reinterpret_cast<uint32_t*>(gbase + OFF_MASK);
+    unsigned int* status = &g_fwd_tc_status;
+    const uint64_t lim = a.timeout_ns;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntq = (a.T + BM - 1) / BM;
+    const int I = ntq - 1 - (int)(blockIdx.x / a.BH);  // longest rows first
+    const int bh = (int)(blockIdx.x % a.BH);
+    const int t0 = I * BM;
+    const int ntk = I + 1;
+    const bool ragged1 = t0 + 64 >= a.T;
+    const int qb0 = t0 / a.block;
+    const int qb1 = ragged1 ? qb0 : (t0 + 64) / a.block;
+    auto BAR = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_QFULL), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(BAR(B_KFULL + s), 1);
+            mbar_init(BAR(B_KEMPTY + s), 1);
+            mbar_init(BAR(B_VFULL + s), 1);
+            mbar_init(BAR(B_VEMPTY + s), 1);
+            mbar_init(BAR(B_SREADY + s), 1);
+            mbar_init(BAR(B_PREADY + s), 128);
+        }
+        mbar_init(BAR(B_PVDONE), 1);
+        mbar_init(BAR(B_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    {
+        const uint32_t* m0 = a.mask + ((size_t)bh * a.n_blocks + qb0) * a.words;
+        const uint32_t* m1 = a.mask + ((size_t)bh * a.n_blocks + qb1) * a.words;
+        for (int w = threadIdx.x; w < a.words; w += kThreads) {
+            mrow[w] = m0[w];
+            mrow[kMaxWords + w] = m1[w];
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(base + OFF_MISC, 512);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            mbar_expect_tx(BAR(B_QFULL), TILE_BYTES);
+            tma_load_3d(base + OFF_Q, &tm_q, BAR(B_QFULL), 0, t0, bh);
+            tma_load_3d(base + OFF_Q + HALF_BYTES, &tm_q, BAR(B_QFULL), 64, t0, bh);
+            int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
+            for (int j = 0; j < ntk; ++j) {
+                const int s = j & 1;
+                const uint32_t ph = ((j >> 1) + 1) & 1;
+                const uint32_t kdst = base + OFF_K + s * TILE_BYTES;
+                const uint32_t vdst = base + OFF_V + s * TILE_BYTES;
+                if (j >= 2 && !mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, status, lim)) break;
+                mbar_expect_tx(BAR(B_KFULL + s), TILE_BYTES);
+                tma_load_3d(kdst, &tm_k, BAR(B_KFULL + s), 0, j * BN, bh);
+                tma_load_3d(kdst + HALF_BYTES, &tm_k, BAR(B_KFULL + s), 64, j * BN, bh);
+                issued_k[s] = j;
+                if (j >= 2 && !mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, status, lim)) break;
+                mbar_expect_tx(BAR(B_VFULL + s), TILE_BYTES);
+                tma_load_3d(vdst, &tm_v, BAR(B_VFULL + s), 0, j * BN, bh);
+                tma_load_3d(vdst + HALF_BYTES, &tm_v, BAR(B_VFULL + s), 64, j * BN, bh);
+                issued_v[s] = j;
+            }
+            if (*abort_flag) {  // let copies in flight land before the CTA exits
+                for (int s = 0; s < 2; ++s) {
+                    if (issued_k[s] >= 0) wait_drain(BAR(B_KFULL + s), (issued_k[s] >> 1) & 1, lim);
+                    if (issued_v[s] >= 0) wait_drain(BAR(B_VFULL + s), (issued_v[s] >> 1) & 1, lim);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, status, lim);
+            auto issue_pv = [&](int i) -> bool {
+                const int b = i & 1;
+                const uint32_t ph = (i >> 1) & 1;
+                if (!mbar_wait(BAR(B_PREADY + b), ph, abort_flag, status, lim)) return false;
+                if (!mbar_wait(BAR(B_VFULL + b), ph, abort_flag, status, lim)) return false;
+                fence_after_sync();
+                const uint32_t vbase = base + OFF_V + b * TILE_BYTES;
+                const uint32_t sb = tmem + (b ? TM_S1 : TM_S0);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    bool s0, s1;
+                    half_sel(mrow, i, I, h, a.block, ragged1, s0, s1);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        // V is MN-major: 64-wide column boxes LBO = 16 KB apart,
+                        // 8-key row groups SBO = 1 KB apart; 16 keys per MMA
+                        const uint64_t bd = smem_desc_sw128(vbase + (4 * h + kk) * 2048, HALF_BYTES, 1024);
+                        const uint32_t pa = sb + 32 * h + 8 * kk;
+                        if (s0 == s1) {
+                            mma_ts(tmem + (s0 ? TM_OSEL : TM_OUNS), pa, bd, idesc_pv, 1);
+                        } else {
+                            mma_ts(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
+                            mma_ts(tmem + TM_OUNS, pa + 64, bd, idesc_pv, 1);
+                        }
+                    }
+                }
+                mma_commit(BAR(B_VEMPTY + b));
+                mma_commit(BAR(B_PVDONE));
+                return true;
+            };
+            for (int j = 0; ok && j < ntk; ++j) {
+                const int s = j & 1;
+                if (!mbar_wait(BAR(B_KFULL + s), (j >> 1) & 1, abort_flag, status, lim)) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t kbase = base + OFF_K + s * TILE_BYTES;
+                const uint32_t sd = tmem + (s ? TM_S1 : TM_S0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    // K-major, 128B swizzle: 16 bf16 of d = 32 bytes per MMA step
+                    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+                    mma_ss(sd, smem_desc_sw128(base + OFF_Q + off, 16, 1024),
+                           smem_desc_sw128(kbase + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(B_SREADY + s));
+                mma_commit(BAR(B_KEMPTY + s));
+                if (j >= 1 && !issue_pv(j - 1)) ok = false;
+            }
+            if (ok) issue_pv(ntk - 1);
+            mma_commit(BAR(B_DRAIN));  // all MMAs of this thread complete before teardown
+            wait_drain(BAR(B_DRAIN), 0, lim);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------ softmax warpgroup
+        const int sw = warp - 4;
+        const int r = sw * 32 + lane;  // row of the tile == TMEM lane
+        const uint32_t lane_base = (uint32_t)(sw * 32) << 16;
+        const uint32_t trow = tmem + lane_base;
+        {
+            uint32_t z[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) z[i] = 0u;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                tmem_st32(trow + TM_OSEL + 32 * c, z);
+                tmem_st32(trow + TM_OUNS + 32 * c, z);
+            }
+            tmem_wait_st();
+        }
+        const float sl2 = a.scale_log2;
+        float m2 = -INFINITY, lsel = 0.f, luns = 0.f;
+        bool ok = true;
+        for (int j = 0; j < ntk; ++j) {
+            const int b = j & 1;
+            // warp-uniform outcome: the TMEM loads below are warp-collective
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(BAR(B_SREADY + b), (j >> 1) & 1, abort_flag, status, lim))) {
+                ok = false;
+                break;
+            }
+            fence_after_sync();
+            const uint32_t sb = trow + (b ? TM_S1 : TM_S0);
+            float s[128];
+            {
+                uint32_t u0[32], u1[32], u2[32], u3[32];
+                tmem_ld32(sb, u0);
+                tmem_ld32(sb + 32, u1);
+                tmem_ld32(sb + 64, u2);
+                tmem_ld32(sb + 96, u3);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    s[c] = __uint_as_float(u0[c]);
+                    s[32 + c] = __uint_as_float(u1[c]);
+                    s[64 + c] = __uint_as_float(u2[c]);
+                    s[96 + c] = __uint_as_float(u3[c]);
+                }
+            }
+            if (j == I) {  // diagonal tile: keys after the row are masked (and keys >= T)
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c > r) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            const float mnew = mx * sl2;
+            if (j == 0) {
+                m2 = mnew;
+            } else {
+                const bool need = mnew > m2 + kRescaleThreshold;
+                if (__any_sync(0xffffffffu, need)) {
+                    // PV_{j-1} must have landed in O before it is rescaled
+                    if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (j - 1) & 1, abort_flag,
+                                                           status, lim))) {
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
+                    const float mup = fmaxf(m2, mnew);
+                    const float alpha = ex2(m2 - mup);
+                    m2 = mup;
+                    lsel *= alpha;
+                    luns *= alpha;
+#pragma unroll 1
+                    for (int c = 0; c < 8; ++c) {
+                        const uint32_t col = (c < 4 ? TM_OSEL : TM_OUNS) + 32 * (c & 3);
+                        uint32_t u[32];
+                        tmem_ld32(trow + col, u);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+                        tmem_st32(trow + col, u);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            const float negm = -m2;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                bool s0, s1;
+                half_sel(mrow, j, I, h, a.block, ragged1, s0, s1);
+                const bool mixed = s0 != s1;
+                const bool row_sel = mixed ? ((r < 64 || a.block == 128) ? s0 : s1) : s0;
+                float sum = 0.f;
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2(fmaf(s[64 * h + 2 * c], sl2, negm));
+                    const float p1 = ex2(fmaf(s[64 * h + 2 * c + 1], sl2, negm));
+                    sum += p0 + p1;
+                    pk[c] = pack_bf16(p0, p1);
+                }
+                if (!mixed) {
+                    tmem_st32(sb + 32 * h, pk);
+                } else {
+                    uint32_t main_[32], alt[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        main_[c] = row_sel ? pk[c] : 0u;
+                        alt[c] = row_sel ? 0u : pk[c];
+                    }
+                    tmem_st32(sb + 32 * h, main_);
+                    tmem_st32(sb + 64 + 32 * h, alt);
+                }
+                if (row_sel) lsel += sum;
+                else luns += sum;
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(BAR(B_PREADY + b));
+        }
+        if (ok)
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(BAR(B_PVDONE), (ntk - 1) & 1, abort_flag, status, lim));
+        if (ok) {
+            fence_after_sync();
+            const int t = t0 + r;
+            const bool valid = t < a.T;
+            const size_t row = (size_t)bh * a.T + (valid ? t : 0);
+            const float l = lsel + luns;
+            const float inv_l = 1.f / l;
+            const float inv_ls = lsel > 0.f ? 1.f / lsel : 0.f;
+            float sq = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t os[32], ou[32];
+                tmem_ld32(trow + TM_OSEL + 32 * c, os);
+                tmem_ld32(trow + TM_OUNS + 32 * c, ou);
+                tmem_wait_ld();
+                uint32_t hf[16], hs[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float sa = __uint_as_float(os[2 * e]), sb2 = __uint_as_float(os[2 * e + 1]);
+                    const float ua = __uint_as_float(ou[2 * e]), ub = __uint_as_float(ou[2 * e + 1]);
+                    const float fa = (sa + ua) * inv_l, fb = (sb2 + ub) * inv_l;
+                    const float pa = sa * inv_ls, pb = sb2 * inv_ls;
+                    sq = fmaf(fa - pa, fa - pa, sq);
+                    sq = fmaf(fb - pb, fb - pb, sq);
+                    hf[e] = pack_bf16(fa, fb);
+                    hs[e] = pack_bf16(pa, pb);
+                }
+                if (valid) {
+                    uint4* df = reinterpret_cast<uint4*>(a.h_full + row * HD + 32 * c);
+                    uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * HD + 32 * c);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        df[v4] = make_uint4(hf[4 * v4], hf[4 * v4 + 1], hf[4 * v4 + 2], hf[4 * v4 + 3]);
+                        ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
+                    }
+                }
+            }
+            if (valid) {
+                a.delta[row] = luns * inv_l;
+                a.lse_full[row] = (m2 + log2f(l)) * kLn2;
+                a.lse_sparse[row] = lsel > 0.f ? (m2 + log2f(lsel)) * kLn2 : -INFINITY;
+                a.sqdiff[row] = sq;
+            }
+        }
+    }
+
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// [BH, T, 128] bf16 viewed as a 3-D tensor (d, t, bh); box = 64 d x 128 t,
+// 128-byte swizzle; rows past T are zero-filled by the TMA unit.
+int make_map(CUtensorMap* m, const void* ptr, int BH, int T) {
+    auto fn = encode_fn();
+    if (!fn) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)T * HD * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)BM, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SSA_OK;
+}
+
+}  // namespace
+
+bool fwd_tc_supported(const ssa_params_t& p) {
+    return p.dtype == SSA_BF16 && p.D == HD && (p.block == 64 || p.block == 128) &&
+           mask_words(p) <= kMaxWords && (size_t)p.B * p.H * ((p.T + BM - 1) / BM) <= 0x7fffffffull;
+}
+
+size_t fwd_tc_workspace(const ssa_params_t&) { return 0; }
+
+int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                  const uint32_t* mask, void* hf, void* hs, float* delta, float* lf, float* ls,
+                  float* sq, void*, cudaStream_t s) {
+    const int BH = p.B * p.H;
+    CUtensorMap mq, mk, mv;
+    int st = make_map(&mq, q, BH, p.T);
+    if (st == SSA_OK) st = make_map(&mk, k, BH, p.T);
+    if (st == SSA_OK) st = make_map(&mv, v, BH, p.T);
+    if (st != SSA_OK) return st;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(SSA_ERR_CUDA, "fwd_tc: smem attribute: %s", cudaGetErrorString(attr_err));
+    FwdArgs a;
+    a.h_full = static_cast<__nv_bfloat16*>(hf);
+    a.h_sparse = static_cast<__nv_bfloat16*>(hs);
+    a.delta = delta;
+    a.lse_full = lf;
+    a.lse_sparse = ls;
+    a.sqdiff = sq;
+    a.mask = mask;
+    a.BH = BH;
+    a.T = p.T;
+    a.block = p.block;
+    a.words = mask_words(p);
+    a.n_blocks = num_blocks(p);
+    a.scale_log2 = p.sm_scale * 1.4426950408889634f;
+    a.timeout_ns = 2000000000ull;
+    const unsigned grid = (unsigned)((size_t)BH * ((p.T + BM - 1) / BM));
+    fwd_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, a);
+    return check_launch("fwd_tc_kernel");
+}
+
+int fwd_tc_take_status(cudaStream_t) {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_fwd_tc_status, sizeof v);
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (v) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_fwd_tc_status, &zero, sizeof zero);
+        return fail(SSA_ERR_TIMEOUT, "fwd_tc_kernel: a bounded mbarrier wait expired");
+    }
+    return SSA_OK;
+}
+
+}  // namespace ssa

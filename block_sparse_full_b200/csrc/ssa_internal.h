@@ -1,0 +1,61 @@
+// Internal declarations shared by the host-side translation units of libssa.
+// Kernels live in their own .cu files; each exposes one host launcher here.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ssa.h"
+
+namespace ssa {
+
+// Records a detail message for ssa_last_error() and returns `status`.
+int fail(int status, const char* fmt, ...);
+
+// Turns a pending launch/runtime error into SSA_ERR_CUDA (with detail).
+int check_launch(const char* what);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline size_t num_rows(const ssa_params_t& p) {
+    return (size_t)p.B * p.H * p.T;
+}
+inline size_t num_elems(const ssa_params_t& p) { return num_rows(p) * p.D; }
+inline int num_blocks(const ssa_params_t& p) { return p.T / p.block; }
+inline int mask_words(const ssa_params_t& p) { return (num_blocks(p) + 31) / 32; }
+
+// ---- selection (select.cu)
+size_t select_workspace(const ssa_params_t& p);
+int launch_select(const ssa_params_t& p, const void* q, const void* k, int32_t* idx,
+                  int32_t* cnt, uint32_t* mask, void* ws, cudaStream_t s);
+
+// ---- forward, CUDA-core path (fwd_simt.cu)
+int launch_fwd_simt(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                    const uint32_t* mask, void* h_full, void* h_sparse, float* delta,
+                    float* lse_full, float* lse_sparse, float* sqdiff, cudaStream_t s);
+
+// ---- forward, tcgen05 path (fwd_tc.cu)
+bool fwd_tc_supported(const ssa_params_t& p);
+size_t fwd_tc_workspace(const ssa_params_t& p);
+int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                  const uint32_t* mask, void* h_full, void* h_sparse, float* delta,
+                  float* lse_full, float* lse_sparse, float* sqdiff, void* ws,
+                  cudaStream_t s);
+int fwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
+
+// ---- alignment loss (loss.cu)
+size_t loss_workspace(const ssa_params_t& p);
+int launch_loss(const ssa_params_t& p, const float* sqdiff, float w_s, float w_c,
+                float* loss_out, void* ws, cudaStream_t s);
+
+// ---- backward, CUDA-core path (bwd_simt.cu)
+size_t bwd_simt_workspace(const ssa_params_t& p);
+int launch_bwd_simt(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                    const uint32_t* mask, const void* h_full, const void* h_sparse,
+                    const float* lse_full, const float* lse_sparse, const void* dh_full,
+                    const void* dh_sparse, float w_s, float w_c, void* dq, void* dk,
+                    void* dv, void* ws, cudaStream_t s);
+
+}  // namespace ssa

@@ -1,0 +1,188 @@
+/*
+ * ssa.h -- C ABI of libssa: the per-layer dual-stream causal attention of
+ * SSA ("SSA: Sparse Sparse Attention by Aligning Full and Sparse Attention
+ * Outputs in Feature Space", arXiv 2511.20102) on NVIDIA B200 (sm_100a).
+ *
+ * For one layer and the same Q, K, V the library computes
+ *   - the full-attention output h_full (causal softmax over every past token),
+ *   - the block-sparse output h_sparse (softmax over the selected key blocks
+ *     only; the sparse stream normalises over its own subset),
+ *   - the discarded attention mass delta(t) (full-softmax weight on keys the
+ *     sparse rule did not select),
+ *   - the alignment losses L_sparsity and L_commit,
+ *   - and the backward pass through both streams.
+ * Sources: gist.science technical summaries of the paper (Italian
+ * "Sintesi Tecnica", French "Resume technique"), section 1 (problem
+ * statement: normalisation over the selected subset, error linear in the
+ * discarded mass), section 2 (methodology: sparse and full streams,
+ * counterpart output computed only for alignment, L_sparsity and L_commit,
+ * total objective E_mode[L_ce] + alpha L_align), section 4 ("Efficienza":
+ * inference runs the same operations as MoBA).
+ *
+ * Conventions for every entry point
+ *   - Tensors are row-major contiguous [B, H, T, D] (q, k, v, h_*, dh_*, d*),
+ *     in the element type given by params->dtype.  Row statistics (delta,
+ *     lse_*, sqdiff_rows) are float32 [B, H, T].  Selection outputs are
+ *     idx int32 [B, H, n, topk], cnt int32 [B, H, n] and mask uint32
+ *     [B, H, n, ceil(n/32)] with n = T / block.
+ *   - Every pointer except `params` is DEVICE memory owned by the caller.
+ *     The library allocates nothing.  Scratch memory is passed as `ws`
+ *     (device, 256-byte aligned) of at least ssa_workspace_size(...) bytes;
+ *     it may be NULL when that size is 0.  The library keeps no pointer
+ *     after a call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are returned synchronously before
+ *     anything is launched; launch errors return SSA_ERR_CUDA.  A kernel
+ *     whose bounded wait expired records SSA_ERR_TIMEOUT in a device status
+ *     word that ssa_device_status() reports after synchronising.
+ *   - Alignment: every device pointer 16-byte aligned; the bf16 tensor-core
+ *     path additionally requires D == 128.
+ */
+#ifndef SSA_H
+#define SSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSA_OK = 0,
+    SSA_ERR_INVALID_ARG = -1, /* null pointer, bad shape, misaligned pointer */
+    SSA_ERR_UNSUPPORTED = -2, /* valid but not implemented (dtype/D/block)   */
+    SSA_ERR_WORKSPACE = -3,   /* ws smaller than ssa_workspace_size()        */
+    SSA_ERR_CUDA = -4,        /* a CUDA runtime call or launch failed         */
+    SSA_ERR_TIMEOUT = -5      /* a device-side bounded wait gave up           */
+} ssa_status_t;
+
+typedef enum { SSA_F32 = 0, SSA_BF16 = 1 } ssa_dtype_t;
+
+/* SSA_FLAG_FORCE_SINK: block 0 (the "sink") is always selected; it counts
+ * inside topk.
+ * SSA_FLAG_FORCE_SIMT: run the CUDA-core (SIMT) kernels even where the
+ * tcgen05 tensor-core kernels apply; a slower comparator with the same
+ * results up to float32 rounding order. */
+enum { SSA_FLAG_FORCE_SINK = 1u, SSA_FLAG_FORCE_SIMT = 2u };
+
+/*
+ * Layer shape and method parameters.
+ *   B, H, T, D : batch, heads, tokens, head dim.  T % block == 0.
+ *                D in {64, 128}.
+ *   block      : tokens per query block and per key block, 64 or 128.
+ *   topk       : selected key blocks per query block, counting the always
+ *                selected current block (and block 0 under FORCE_SINK);
+ *                1 <= topk <= n, topk >= 2 with FORCE_SINK.
+ *   dtype      : ssa_dtype_t of every [B,H,T,D] tensor.
+ *   sm_scale   : softmax scale sigma (logit = sigma * q.k), > 0.
+ *   flags      : OR of SSA_FLAG_*.
+ */
+typedef struct {
+    int B, H, T, D, block, topk;
+    int dtype;
+    float sm_scale;
+    unsigned flags;
+} ssa_params_t;
+
+enum {
+    SSA_WS_SELECT = 0,
+    SSA_WS_FWD = 1,
+    SSA_WS_LOSS = 2,
+    SSA_WS_BWD = 3
+};
+
+/* Bytes of scratch the named entry point needs for these params (0 if none,
+ * (size_t)-1 if the params are invalid). */
+size_t ssa_workspace_size(const ssa_params_t* params, int which);
+
+/*
+ * Block selection of the sparse stream (section 2, "Sparse Attention
+ * Stream": block-sparse attention; section 4: MoBA-identical operations).
+ * Per (b, h, query block i):
+ *   Qbar_i = mean of q over block i, Kbar_j = mean of k over block j,
+ *   score s_ij = Qbar_i . Kbar_j, formed in float64 (block sums are exact);
+ *   S_i = {i} (plus {0} under FORCE_SINK) and the best topk - |forced|
+ *   blocks j < i by (score descending, j ascending), or all j < i if fewer.
+ * Writes idx (S_i ascending, -1 padded), cnt (|S_i|) and mask (bit j%32 of
+ * word j/32 set iff j in S_i).  Workspace: SSA_WS_SELECT.
+ */
+int ssa_select_blocks(const ssa_params_t* params, const void* q, const void* k,
+                      int32_t* idx, int32_t* cnt, uint32_t* mask,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Both attention streams in one pass over K/V (section 2: the full stream
+ * and the counterpart sparse output of the same layer).  For query t in
+ * block i, keys s <= t, x = sm_scale * q_t . k_s, sel(t,s) = block(s) in S_i
+ * (read from `mask`; idx/cnt may be NULL and are not read):
+ *   h_full   = sum_s e^x v_s / sum_s e^x
+ *   h_sparse = sum_{sel} e^x v_s / sum_{sel} e^x
+ *   delta    = sum_{not sel} e^x / sum_s e^x
+ *   lse_full = log sum_s e^x,   lse_sparse = log sum_{sel} e^x
+ *   sqdiff_rows[t] = sum_c (h_full - h_sparse)_c^2 from the float32 values
+ *                    before rounding to dtype.
+ * Accumulation is float32.  Workspace: SSA_WS_FWD.
+ */
+int ssa_attn_fwd_dual(const ssa_params_t* params, const void* q, const void* k,
+                      const void* v, const int32_t* idx, const int32_t* cnt,
+                      const uint32_t* mask, void* h_full, void* h_sparse,
+                      float* delta, float* lse_full, float* lse_sparse,
+                      float* sqdiff_rows, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Alignment losses (section 2, "Allineamento Bidirezionale"): with
+ * N = B*H*T*D and L = sum(sqdiff_rows) / N (the mean squared difference of
+ * the two outputs), writes loss_out[0] = w_sparsity * L (L_sparsity) and
+ * loss_out[1] = w_commit * L (L_commit), float32, device memory.  The sum
+ * is a fixed-order float64 reduction: repeated calls give identical bits.
+ * Workspace: SSA_WS_LOSS.
+ */
+int ssa_align_loss(const ssa_params_t* params, const float* sqdiff_rows,
+                   float w_sparsity, float w_commit, float* loss_out,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward of  <dh_full, h_full> + <dh_sparse, h_sparse>
+ *            + w_sparsity * L_sparsity + w_commit * L_commit
+ * with respect to q, k, v; L_sparsity reaches h_full only and L_commit
+ * h_sparse only (stop-gradient on the opposite stream); no gradient flows
+ * through selection or delta.  The full stream carries gradient to every
+ * causal key (section 2, "Full Attention Stream").  h_full, h_sparse,
+ * lse_full and lse_sparse are the forward's outputs for the same inputs.
+ * dh_full / dh_sparse may be NULL (read as zero).  dq, dk, dv are written
+ * (not accumulated).  Workspace: SSA_WS_BWD.
+ */
+int ssa_attn_bwd(const ssa_params_t* params, const void* q, const void* k,
+                 const void* v, const int32_t* idx, const int32_t* cnt,
+                 const uint32_t* mask, const void* h_full, const void* h_sparse,
+                 const float* lse_full, const float* lse_sparse,
+                 const void* dh_full, const void* dh_sparse,
+                 float w_sparsity, float w_commit,
+                 void* dq, void* dk, void* dv,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns SSA_ERR_TIMEOUT if any kernel since the
+ * previous call recorded an expired wait (and clears the record), else
+ * SSA_ERR_CUDA on a pending CUDA error, else SSA_OK. */
+int ssa_device_status(void* stream);
+
+/* Static text for a status code. */
+const char* ssa_status_string(int status);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char* ssa_last_error(void);
+
+/* Which kernel family the params select: 0 = CUDA-core (SIMT) kernels
+ * (float32, bf16 with D = 64, or SSA_FLAG_FORCE_SIMT), 1 = bf16 tcgen05
+ * tensor-core kernels (D = 128), -1 = invalid or unsupported params. */
+int ssa_kernel_path(const ssa_params_t* params);
+
+/* ABI version, (major << 16) | minor. */
+int ssa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H */

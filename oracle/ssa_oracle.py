@@ -246,33 +246,37 @@ def alignment_upstream(h_full, h_sparse, dh_full, dh_sparse, w_s, w_c, n_total):
 # Backward through both streams
 # --------------------------------------------------------------------------
 
-def _bwd_head(q, k, v, blocksel, block, sm_scale, g_full, g_sparse):
+def _bwd_head(q, k, v, blocksel, block, sm_scale, g_full, g_sparse, max_elems=1 << 23):
     """dq, dk, dv of  sum(g_full * h_full) + sum(g_sparse * h_sparse)  for one
     (batch, head), selection held fixed.  Written with the explicit softmax
     Jacobian: for P = softmax(x) over a key set and upstream dP = g v^T,
-    dx = P * (dP - rowsum(P * dP))."""
+    dx = P * (dP - rowsum(P * dP)).  Query rows are independent, so they are
+    taken a slice at a time; dk and dv sum the slices' contributions."""
     T = q.shape[0]
-    t = np.arange(T)
-    x = sm_scale * (q @ k.T)
-    causal = t[None, :] <= t[:, None]
-    in_sel = blocksel[t // block][:, t // block]
-    sel = causal & in_sel
+    s = np.arange(T)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
 
-    def softmax_over(allowed):
+    def softmax_over(x, allowed):
         xm = np.where(allowed, x, -np.inf)
         m = xm.max(axis=1, keepdims=True)
         e = np.where(allowed, np.exp(xm - m), 0.0)
         return e / e.sum(axis=1, keepdims=True)
 
-    p_full = softmax_over(causal)       # full-attention stream: every s <= t
-    p_sparse = softmax_over(sel)        # sparse stream: selected blocks only
-    dv = p_full.T @ g_full + p_sparse.T @ g_sparse
-    dp_full = g_full @ v.T
-    dp_sparse = g_sparse @ v.T
-    dx = p_full * (dp_full - (p_full * dp_full).sum(axis=1, keepdims=True))
-    dx += p_sparse * (dp_sparse - (p_sparse * dp_sparse).sum(axis=1, keepdims=True))
-    dq = sm_scale * dx @ k
-    dk = sm_scale * dx.T @ q
+    step = max(1, max_elems // T)
+    for t0 in range(0, T, step):
+        t = np.arange(t0, min(T, t0 + step))
+        x = sm_scale * (q[t] @ k.T)
+        causal = s[None, :] <= t[:, None]
+        sel = causal & blocksel[t // block][:, s // block]
+        p_full = softmax_over(x, causal)    # full-attention stream: every s <= t
+        p_sparse = softmax_over(x, sel)     # sparse stream: selected blocks only
+        dv += p_full.T @ g_full[t] + p_sparse.T @ g_sparse[t]
+        dp_full = g_full[t] @ v.T
+        dp_sparse = g_sparse[t] @ v.T
+        dx = p_full * (dp_full - (p_full * dp_full).sum(axis=1, keepdims=True))
+        dx += p_sparse * (dp_sparse - (p_sparse * dp_sparse).sum(axis=1, keepdims=True))
+        dq[t] = sm_scale * dx @ k
+        dk += sm_scale * dx.T @ q[t]
     return dq, dk, dv
 
 

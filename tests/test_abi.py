@@ -1,0 +1,116 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol the
+header declares, and rejects bad arguments on the host before launching."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_full_b200 import ssa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssa.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssa_\w+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(ssa.LIB_PATH)
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(ssa.EXPORTS) == names
+
+
+def test_exports_are_c_symbols():
+    # plain C names, no C++ mangling
+    out = os.popen(f"nm -D --defined-only {ssa.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}$", out, flags=re.M), name
+
+
+def test_version_and_status_strings():
+    assert ssa.ssa_version() >> 16 == 1
+    assert ssa.ssa_status_string(0) == "ok"
+    assert "timed out" in ssa.ssa_status_string(ssa.SSA_ERR_TIMEOUT)
+    assert ssa.ssa_status_string(12345) == "unknown status"
+
+
+GOOD = dict(B=1, H=2, T=1024, D=128, block=64, topk=4, dtype=ssa.SSA_BF16)
+
+
+def P(**kw):
+    a = {**GOOD, **kw}
+    return ssa.make_params(a["B"], a["H"], a["T"], a["D"], a["block"], a["topk"], a["dtype"],
+                           kw.get("sm_scale"), kw.get("flags", 0))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=1000), ssa.SSA_ERR_INVALID_ARG),           # T % block
+    (dict(block=32), ssa.SSA_ERR_UNSUPPORTED),
+    (dict(D=96), ssa.SSA_ERR_UNSUPPORTED),
+    (dict(topk=0), ssa.SSA_ERR_INVALID_ARG),
+    (dict(topk=17), ssa.SSA_ERR_INVALID_ARG),          # > T/block
+    (dict(topk=1, flags=ssa.SSA_FLAG_FORCE_SINK), ssa.SSA_ERR_INVALID_ARG),
+    (dict(flags=8), ssa.SSA_ERR_INVALID_ARG),
+    (dict(dtype=7), ssa.SSA_ERR_INVALID_ARG),
+    (dict(B=0), ssa.SSA_ERR_INVALID_ARG),
+    (dict(sm_scale=-1.0), ssa.SSA_ERR_INVALID_ARG),
+    (dict(sm_scale=float("inf")), ssa.SSA_ERR_INVALID_ARG),
+])
+def test_bad_params_rejected_before_launch(kw, code):
+    p = P(**kw)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    st = ssa.ssa_select_blocks(p, fake, fake, fake, fake, fake, fake, 1 << 30, None)
+    assert st == code, ssa.ssa_last_error()
+    assert ssa.ssa_last_error()
+    assert ssa.ssa_workspace_size(p, 0) == ctypes.c_size_t(-1).value
+    assert ssa.ssa_kernel_path(p) == -1
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = P()
+    a = 1 << 20
+    assert ssa.ssa_select_blocks(p, None, a, a, a, a, a, 1 << 30, None) == ssa.SSA_ERR_INVALID_ARG
+    assert "q is NULL" in ssa.ssa_last_error()
+    assert ssa.ssa_select_blocks(p, a + 2, a, a, a, a, a, 1 << 30, None) == ssa.SSA_ERR_INVALID_ARG
+    assert "aligned" in ssa.ssa_last_error()
+    st = ssa.ssa_attn_fwd_dual(p, a, a, a, None, None, None, a, a, a, a, a, a, a, 1 << 30, None)
+    assert st == ssa.SSA_ERR_INVALID_ARG and "mask" in ssa.ssa_last_error()
+    st = ssa.ssa_attn_bwd(p, a, a, a, None, None, a, a, a, a, a, None, None, 0.0, 0.0,
+                          a, a, None, a, 1 << 40, None)
+    assert st == ssa.SSA_ERR_INVALID_ARG and "dv" in ssa.ssa_last_error()
+    st = ssa.ssa_align_loss(p, a, float("nan"), 1.0, a, a, 1 << 20, None)
+    assert st == ssa.SSA_ERR_INVALID_ARG
+
+
+def test_workspace_too_small_rejected():
+    p = P()
+    need = ssa.ssa_workspace_size(p, ssa.SSA_WS_SELECT)
+    assert need > 0
+    a = 1 << 20
+    st = ssa.ssa_select_blocks(p, a, a, a, a, a, a, need - 1, None)
+    assert st == ssa.SSA_ERR_WORKSPACE
+    st = ssa.ssa_select_blocks(p, a, a, a, a, a, None, need, None)
+    assert st == ssa.SSA_ERR_WORKSPACE
+    st = ssa.ssa_select_blocks(p, a, a, a, a, a, a + 16, need, None)  # not 256-aligned
+    assert st == ssa.SSA_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_scale_with_shape():
+    small, big = P(T=1024), P(T=4096, topk=4)
+    for w in (ssa.SSA_WS_SELECT, ssa.SSA_WS_LOSS, ssa.SSA_WS_BWD):
+        assert ssa.ssa_workspace_size(big, w) >= ssa.ssa_workspace_size(small, w)
+    # select: Qbar and Kbar in float64
+    assert ssa.ssa_workspace_size(small, 0) == 2 * 1 * 2 * 16 * 128 * 8
+
+
+def test_kernel_path_choice():
+    assert ssa.ssa_kernel_path(P(dtype=ssa.SSA_F32)) == 0
+    assert ssa.ssa_kernel_path(P(D=64)) == 0
+    assert ssa.ssa_kernel_path(P(flags=ssa.SSA_FLAG_FORCE_SIMT)) == 0

@@ -31,9 +31,9 @@ MUTATIONS = {
                                 "r = max(topk - len(forced) + 1, 0)"),
     "commit_gradient_sign": ("g_sparse = f64(dh_sparse) + w_c * (2.0 / n_total) * (hs - hf)",
                              "g_sparse = f64(dh_sparse) + w_c * (2.0 / n_total) * (hf - hs)"),
-    "bwd_missing_scale": ("dk = sm_scale * dx.T @ q", "dk = dx.T @ q"),
-    "bwd_dv_sparse_dropped": ("dv = p_full.T @ g_full + p_sparse.T @ g_sparse",
-                              "dv = p_full.T @ g_full"),
+    "bwd_missing_scale": ("dk += sm_scale * dx.T @ q[t]", "dk += dx.T @ q[t]"),
+    "bwd_dv_sparse_dropped": ("dv += p_full.T @ g_full[t] + p_sparse.T @ g_sparse[t]",
+                              "dv += p_full.T @ g_full[t]"),
     "loss_sum_not_mean": ("L = float(np.mean((hf - hs) ** 2))", "L = float(np.sum((hf - hs) ** 2))"),
 }
 
