@@ -1,0 +1,473 @@
+"""Benchmark of the SSA dual-stream attention layer on B200.
+
+One step = the whole hot path over one batch of synthetic input, through the
+C ABI: block selection -> fused dual-stream forward -> alignment loss ->
+backward of both streams (upstream N(0,1) gradients on both outputs plus
+both alignment terms).  Default workload: B=1, H=16, T=8192, d=128, bf16,
+block 64, top-k 16 with planted hot blocks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is algorithmic TFLOP/s of the step
+(forward 4*d*P_full, backward 10*d*P_full + 4*d*P_sel per head, P_full =
+T(T+1)/2 causal pairs, P_sel = selected causal pairs) summed over all ranks,
+divided by the slowest rank's device time; inputs are resident in HBM and L2
+is flushed before every timed step.  Under torchrun each rank runs its own
+copy of the workload (independent (batch, head) units, no data-path
+collective): weak scaling.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded slice of the
+same workload on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from datetime import timedelta
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_full_b200.inputs import WORKLOADS, make_inputs, upstream_grads  # noqa: E402
+
+DEFAULT_WORKLOAD = "bf16_T8192_H16_hot"
+METRIC = "dual-stream SSA attention fwd(+bwd) TFLOP/s and % bf16 tensor peak at T=8192"
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+FP32_LANES_PER_SM = 128
+NUM_SMS = 148
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def pair_counts(w, idx, cnt):
+    """Causal pairs per (b, h): full = T(T+1)/2 and selected (from idx/cnt)."""
+    T, blk = w.T, w.block
+    p_full = T * (T + 1) // 2
+    idx = idx.reshape(-1, w.n_blocks, idx.shape[-1])
+    cnt = cnt.reshape(-1, w.n_blocks)
+    p_sel = 0
+    for bh in range(idx.shape[0]):
+        for i in range(w.n_blocks):
+            js = idx[bh, i, :cnt[bh, i]]
+            # rows of block i see all keys of earlier selected blocks and the
+            # causal triangle of block i itself
+            p_sel += blk * blk * int((js < i).sum()) + blk * (blk + 1) // 2
+    return p_full, p_sel / idx.shape[0]
+
+
+def step_flops(w, p_full, p_sel):
+    BH = w.B * w.H
+    f_fwd = 4 * w.D * p_full * BH
+    f_bwd = (10 * w.D * p_full + 4 * w.D * p_sel) * BH
+    return f_fwd, f_bwd
+
+
+def source_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "block_sparse_full_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch recorded from an ncu capture of this kernel,
+    or None when no capture exists or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    e = table.get(kernel_key)
+    if not e or e.get("source_sha") != source_sha(*e["sources"]):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return None
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[4:8]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Layer:
+    """Preallocated device buffers and raw C-ABI calls for one step."""
+
+    def __init__(self, w, inp, grads, dev):
+        from block_sparse_full_b200 import ssa
+        self.ssa, self.w, self.dev = ssa, w, dev
+        self.q, self.k, self.v = (inp[n].to(dev) for n in "qkv")
+        self.dhf, self.dhs = grads["dh_full"].to(dev), grads["dh_sparse"].to(dev)
+        self.p = ssa.params_for(self.q, w.block, w.topk, w.sm_scale, w.flags)
+        n, words = w.n_blocks, (w.n_blocks + 31) // 32
+        B, H, T = w.B, w.H, w.T
+        self.idx = torch.empty((B, H, n, w.topk), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((B, H, n), dtype=torch.int32, device=dev)
+        self.mask = torch.empty((B, H, n, words), dtype=torch.int32, device=dev)
+        self.hf, self.hs = torch.empty_like(self.q), torch.empty_like(self.q)
+        self.rows = {k: torch.empty((B, H, T), dtype=torch.float32, device=dev)
+                     for k in ("delta", "lse_f", "lse_s", "sqd")}
+        self.loss = torch.empty(2, dtype=torch.float32, device=dev)
+        self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
+        self.ws = {i: ssa.workspace(self.p, i, dev) for i in range(4)}
+        self.w_s = self.w_c = 1.0
+        self.path = ssa.ssa_kernel_path(self.p)
+
+    def launches_per_step(self):
+        # select: pool + score; fwd: 1; loss: 2; bwd (CUDA-core): pre + dq + dkdv
+        return 2 + 1 + 2 + 3
+
+    def run(self, stream, events=None):
+        s, ssa, P = stream.cuda_stream, self.ssa, self.p
+        ptr = lambda t: t.data_ptr()
+        ev = events or [None] * 5
+        if ev[0] is not None:
+            ev[0].record(stream)
+        st = ssa.ssa_select_blocks(P, ptr(self.q), ptr(self.k), ptr(self.idx), ptr(self.cnt),
+                                   ptr(self.mask), ptr(self.ws[0]), self.ws[0].numel(), s)
+        ssa.check(st, "select")
+        if ev[1] is not None:
+            ev[1].record(stream)
+        r = self.rows
+        st = ssa.ssa_attn_fwd_dual(P, ptr(self.q), ptr(self.k), ptr(self.v), None, None,
+                                   ptr(self.mask), ptr(self.hf), ptr(self.hs), ptr(r["delta"]),
+                                   ptr(r["lse_f"]), ptr(r["lse_s"]), ptr(r["sqd"]),
+                                   ptr(self.ws[1]), self.ws[1].numel(), s)
+        ssa.check(st, "fwd")
+        if ev[2] is not None:
+            ev[2].record(stream)
+        st = ssa.ssa_align_loss(P, ptr(r["sqd"]), self.w_s, self.w_c, ptr(self.loss),
+                                ptr(self.ws[2]), self.ws[2].numel(), s)
+        ssa.check(st, "loss")
+        if ev[3] is not None:
+            ev[3].record(stream)
+        st = ssa.ssa_attn_bwd(P, ptr(self.q), ptr(self.k), ptr(self.v), None, None,
+                              ptr(self.mask), ptr(self.hf), ptr(self.hs), ptr(r["lse_f"]),
+                              ptr(r["lse_s"]), ptr(self.dhf), ptr(self.dhs), self.w_s, self.w_c,
+                              ptr(self.dq), ptr(self.dk), ptr(self.dv), ptr(self.ws[3]),
+                              self.ws[3].numel(), s)
+        ssa.check(st, "bwd")
+        if ev[4] is not None:
+            ev[4].record(stream)
+
+
+def run_ours(args, rank, world, dev, peaks, peak_src):
+    w = WORKLOADS[args.workload]
+    torch.cuda.set_device(dev)
+    inp = make_inputs(w)
+    grads = upstream_grads(w)
+    layer = Layer(w, inp, grads, dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    for _ in range(args.warmup):
+        layer.run(stream)
+    torch.cuda.synchronize(dev)
+    layer.ssa.device_status()
+    p_full, p_sel = pair_counts(w, layer.idx.cpu().numpy(), layer.cnt.cpu().numpy())
+    f_fwd, f_bwd = step_flops(w, p_full, p_sel)
+
+    names = ("select", "fwd", "loss", "bwd")
+    per_call = {n: 0.0 for n in names}
+    step_ms = []
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush.zero_()  # evict L2 between timed steps (outside the events)
+            layer.run(stream, evs[i])
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    layer.ssa.device_status()
+    for e in evs:
+        step_ms.append(e[0].elapsed_time(e[4]))
+        for j, n in enumerate(names):
+            per_call[n] += e[j].elapsed_time(e[j + 1])
+    total_ms = sum(step_ms)
+    max_ms = reduce_max(total_ms, world, dev)
+    ms_per_step = max_ms / args.steps
+    value = (f_fwd + f_bwd) * world / (ms_per_step * 1e-3) / 1e12
+
+    # dominant ABI call and its roofline
+    avg = {n: per_call[n] / args.steps for n in names}
+    dom = max(("fwd", "bwd"), key=lambda n: avg[n])
+    sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    if dom == "fwd" and layer.path == 1:
+        achieved = f_fwd / (avg["fwd"] * 1e-3) / 1e12
+        roof = {"kernel": "fwd_tc_kernel", "bound": "tensor", "peak": sustained,
+                "unit": "TFLOP/s", "peak_kind": f"{peak_src} bf16 dense, sustained",
+                "traffic": ncu_traffic("fwd_tc_kernel")}
+    else:
+        flops = f_fwd if dom == "fwd" else f_bwd
+        achieved = flops / (avg[dom] * 1e-3) / 1e12
+        fp32 = NUM_SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        roof = {"kernel": f"{dom}_simt", "bound": "alu", "peak": round(fp32, 1),
+                "unit": "TFLOP/s", "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock",
+                "traffic": ncu_traffic(f"{dom}_simt")}
+    roof["achieved"] = round(achieved, 2)
+    roof["frac"] = round(achieved / roof["peak"], 4)
+    roof["ms_per_launch"] = round(avg[dom], 4)
+    roof["flops_per_launch"] = f_fwd if dom == "fwd" else f_bwd
+
+    fwd_tflops = f_fwd / (avg["fwd"] * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(d) with planted hot key blocks)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "block": w.block,
+                   "topk": w.topk, "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": f"replicas x{world} (independent batch*head units)",
+                   "l2": "flushed before every timed step", "kernel_path": layer.path},
+        "roofline": roof,
+        "breakdown_ms": {n: round(avg[n], 4) for n in names},
+        "fwd_tflops": round(fwd_tflops, 2),
+        "fwd_frac_sustained": round(fwd_tflops / sustained, 4),
+        "fwd_frac_burst": round(fwd_tflops / peaks.get("bf16_tflops", 1590.0), 4),
+        "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd, "P_full": p_full, "P_sel": p_sel},
+        "gpu_launches": layer.launches_per_step() * args.steps,
+        "clocks": clk.summary(),
+        "peaks": {"source": peak_src, "bf16_tflops": peaks.get("bf16_tflops"),
+                  "bf16_tflops_sustained": sustained, "hbm_gbs": peaks.get("hbm_gbs")},
+    }
+    if args.e2e:
+        out["e2e"] = run_e2e(args, layer, inp, grads, f_fwd + f_bwd, world, dev)
+    return out
+
+
+def run_e2e(args, layer, inp, grads, flops, world, dev):
+    """Same metric with host buffers: pinned host -> device copies of the
+    step's inputs and a device -> host read of the loss inside the timing."""
+    host = {n: inp[n].pin_memory() for n in "qkv"}
+    host["dh_full"] = grads["dh_full"].pin_memory()
+    host["dh_sparse"] = grads["dh_sparse"].pin_memory()
+    loss_h = torch.empty(2, dtype=torch.float32).pin_memory()
+    dst = {"q": layer.q, "k": layer.k, "v": layer.v, "dh_full": layer.dhf, "dh_sparse": layer.dhs}
+    stream = torch.cuda.current_stream(dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+
+    def step():
+        for n, t in host.items():
+            dst[n].copy_(t, non_blocking=True)
+        layer.run(stream)
+        loss_h.copy_(layer.loss, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
+    return {"value": round(flops * world / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": loss_h.numel() * loss_h.element_size()}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def oracle_slice(w, inp, grads, sel, row_slice):
+    """Oracle select + forward + loss + backward for head (0, 0) restricted
+    to the query rows ``row_slice``; returns (algorithmic flops, seconds)."""
+    from oracle import ssa_oracle as O
+    q, k, v = (inp[n][:1, :1] for n in "qkv")
+    rows = np.arange(row_slice.start, row_slice.stop)
+    t0 = time.perf_counter()
+    idx, cnt, _, _ = O.select_blocks(q, k, w.block, w.topk)
+    fw = O.attn_fwd_dual(q, k, v, idx, cnt, w.block, w.sm_scale, rows=rows)
+    O.align_loss(fw["h_full"], fw["h_sparse"])
+    O.attn_bwd(q, k, v, idx, cnt, w.block, w.sm_scale, grads["dh_full"][:1, :1],
+               grads["dh_sparse"][:1, :1], 1.0, 1.0, n_total=inp["q"].numel(), rows=rows)
+    dt = time.perf_counter() - t0
+    blocksel = O.block_selection_matrix(idx, cnt)[0, 0]
+    pf = int((rows + 1).sum())
+    ps = 0
+    for t in rows:
+        i = t // w.block
+        ps += int(blocksel[i, :i].sum()) * w.block + (t - i * w.block + 1)
+    flops = 4 * w.D * pf + 10 * w.D * pf + 4 * w.D * ps
+    return flops, dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, inp, grads, slices=8, rows_per_slice=1024):
+    flops = secs = 0.0
+    for s in range(slices):
+        hi = w.T - s * rows_per_slice
+        f, t = oracle_slice(w, inp, grads, None, range(hi - rows_per_slice, hi))
+        flops += f
+        secs += t
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle", "seconds": round(secs, 2),
+            "sample": f"fp64 numpy oracle, head (0,0) of {w.name}, query rows "
+                      f"[{w.T - slices * rows_per_slice}, {w.T}): select + fwd + loss + bwd"}
+
+
+def run_reference(args, world):
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    grads = upstream_grads(w)
+    rows = 512
+    for _ in range(args.warmup):
+        oracle_slice(w, inp, grads, None, range(w.T - rows, w.T))
+    flops = secs = 0.0
+    for _ in range(args.steps):
+        f, t = oracle_slice(w, inp, grads, None, range(w.T - rows, w.T))
+        flops += f
+        secs += t
+    value = flops / secs / 1e12
+    cores = blas_threads()
+    sample = (f"fp64 numpy oracle, head (0,0) of {w.name}, query rows [{w.T - rows}, {w.T}) "
+              f"per step: select + fwd + loss + bwd")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D,
+                   "block": w.block, "topk": w.topk},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def reduce_max(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world)), flush=True)
+        return 0
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                             device_id=dev)
+    peaks, src = load_peaks()
+    out = run_ours(args, rank, world, dev, peaks, src)
+    if rank == 0:
+        if world == 1 and args.cpu_baseline:
+            w = WORKLOADS[args.workload]
+            out["cpu_baseline"] = cpu_baseline(w, make_inputs(w), upstream_grads(w))
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

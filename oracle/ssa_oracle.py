@@ -246,7 +246,8 @@ def alignment_upstream(h_full, h_sparse, dh_full, dh_sparse, w_s, w_c, n_total):
 # Backward through both streams
 # --------------------------------------------------------------------------
 
-def _bwd_head(q, k, v, blocksel, block, sm_scale, g_full, g_sparse, max_elems=1 << 23):
+def _bwd_head(q, k, v, blocksel, block, sm_scale, g_full, g_sparse, max_elems=1 << 23,
+              rows=None):
     """dq, dk, dv of  sum(g_full * h_full) + sum(g_sparse * h_sparse)  for one
     (batch, head), selection held fixed.  Written with the explicit softmax
     Jacobian: for P = softmax(x) over a key set and upstream dP = g v^T,
@@ -262,9 +263,10 @@ def _bwd_head(q, k, v, blocksel, block, sm_scale, g_full, g_sparse, max_elems=1 
         e = np.where(allowed, np.exp(xm - m), 0.0)
         return e / e.sum(axis=1, keepdims=True)
 
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
     step = max(1, max_elems // T)
-    for t0 in range(0, T, step):
-        t = np.arange(t0, min(T, t0 + step))
+    for c0 in range(0, len(rows), step):
+        t = rows[c0:c0 + step]
         x = sm_scale * (q[t] @ k.T)
         causal = s[None, :] <= t[:, None]
         sel = causal & blocksel[t // block][:, s // block]
@@ -281,7 +283,7 @@ def _bwd_head(q, k, v, blocksel, block, sm_scale, g_full, g_sparse, max_elems=1 
 
 
 def attn_bwd(q, k, v, idx, cnt, block: int, sm_scale: float, dh_full, dh_sparse,
-             w_sparsity: float = 0.0, w_commit: float = 0.0, n_total=None):
+             w_sparsity: float = 0.0, w_commit: float = 0.0, n_total=None, rows=None):
     """Gradients of  <dh_full, h_full> + <dh_sparse, h_sparse>
     + w_s * L_sparsity + w_c * L_commit  with respect to q, k, v.
 
@@ -289,19 +291,31 @@ def attn_bwd(q, k, v, idx, cnt, block: int, sm_scale: float, dh_full, dh_sparse,
     Attention Stream"); the sparse stream only to selected keys; the
     alignment terms follow ``alignment_upstream``.  ``n_total`` is the
     element count N of the whole layer output (defaults to q.size) so that a
-    caller may pass a slice of heads.  Returns (dq, dk, dv) float64.
+    caller may pass a slice of heads.  ``rows`` optionally keeps only the
+    terms of those query rows (dq of other rows is then 0 and dk, dv hold
+    those rows' share); used to time a bounded slice.  Returns (dq, dk, dv)
+    float64.
     """
     q, k, v = f64(q), f64(k), f64(v)
     B, H, T, d = q.shape
     n_total = q.size if n_total is None else n_total
-    fw = attn_fwd_dual(q, k, v, idx, cnt, block, sm_scale)
-    g_full, g_sparse = alignment_upstream(fw["h_full"], fw["h_sparse"], dh_full,
-                                          dh_sparse, w_sparsity, w_commit, n_total)
+    sel_rows = None if rows is None else np.asarray(sorted(rows), dtype=np.int64)
+    fw = attn_fwd_dual(q, k, v, idx, cnt, block, sm_scale, rows=sel_rows)
+    dhf, dhs = f64(dh_full), f64(dh_sparse)
+    if sel_rows is not None:
+        dhf, dhs = dhf[:, :, sel_rows], dhs[:, :, sel_rows]
+    g_rows = alignment_upstream(fw["h_full"], fw["h_sparse"], dhf, dhs, w_sparsity,
+                                w_commit, n_total)
+    if sel_rows is None:
+        g_full, g_sparse = g_rows
+    else:  # scatter the listed rows' upstream into full-length arrays
+        g_full, g_sparse = np.zeros_like(q), np.zeros_like(q)
+        g_full[:, :, sel_rows], g_sparse[:, :, sel_rows] = g_rows
     blocksel = block_selection_matrix(idx, cnt)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     for b in range(B):
         for h in range(H):
             dq[b, h], dk[b, h], dv[b, h] = _bwd_head(
                 q[b, h], k[b, h], v[b, h], blocksel[b, h], block, sm_scale,
-                g_full[b, h], g_sparse[b, h])
+                g_full[b, h], g_sparse[b, h], rows=sel_rows)
     return dq, dk, dv
