@@ -31,7 +31,8 @@ SSA_WS_SELECT, SSA_WS_FWD, SSA_WS_LOSS, SSA_WS_BWD = 0, 1, 2, 3
 
 # every symbol include/ssa.h declares
 EXPORTS = (
-    "ssa_workspace_size", "ssa_select_blocks", "ssa_attn_fwd_dual", "ssa_align_loss",
+    "ssa_workspace_size", "ssa_select_blocks", "ssa_select_blocks_noalloc",
+    "ssa_attn_fwd_dual", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
     "ssa_kernel_path", "ssa_version",
 )
@@ -57,6 +58,8 @@ _SIGNATURES = {
     "ssa_workspace_size": (c_size_t, [_P, c_int]),
     "ssa_select_blocks": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_size_t, c_void_p]),
+    "ssa_select_blocks_noalloc": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                          c_void_p]),
     "ssa_attn_fwd_dual": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -101,6 +104,11 @@ def ssa_workspace_size(params, which):
 def ssa_select_blocks(params, q, k, idx, cnt, mask, ws, ws_bytes, stream):
     return _lib.ssa_select_blocks(ctypes.byref(params), q, k, idx, cnt, mask, ws, ws_bytes,
                                   stream)
+
+
+def ssa_select_blocks_noalloc(params, q, k, idx, cnt, mask, stream):
+    """Selection with the library's built-in scratch (no workspace argument)."""
+    return _lib.ssa_select_blocks_noalloc(ctypes.byref(params), q, k, idx, cnt, mask, stream)
 
 
 def ssa_attn_fwd_dual(params, q, k, v, idx, cnt, mask, h_full, h_sparse, delta, lse_full,

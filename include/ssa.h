@@ -112,6 +112,28 @@ int ssa_select_blocks(const ssa_params_t* params, const void* q, const void* k,
                       void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * ssa_select_blocks without a workspace argument, for callers that cannot
+ * allocate device memory where they run selection (for example a plugin
+ * inside a serving process whose memory pool owns all device memory, or a
+ * latency-critical loop that must not call cudaMalloc after start-up).  The
+ * paper has no counterpart; this is a packaging variant of the call above
+ * with identical results.
+ *   - Scratch comes from a 16 MiB array in the library's own device memory,
+ *     held by every GPU that loads the library until the process exits.
+ *     Shapes needing more (B*H*(T/block)*D > 1,048,576) are rejected with
+ *     SSA_ERR_UNSUPPORTED before anything is launched.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race and give undefined results; order
+ *     them on one stream.  Nothing in the array needs clearing between calls.
+ */
+int ssa_select_blocks_noalloc(const ssa_params_t* params, const void* q, const void* k,
+                              int32_t* idx, int32_t* cnt, uint32_t* mask, void* stream);
+
+/*
  * Both attention streams in one pass over K/V (section 2: the full stream
  * and the counterpart sparse output of the same layer).  For query t in
  * block i, keys s <= t, x = sm_scale * q_t . k_s, sel(t,s) = block(s) in S_i
