@@ -184,7 +184,7 @@ class Layer:
         self.path = ssa.ssa_kernel_path(self.p)
 
     def launches_per_step(self):
-        # select: pool + score; fwd: 1; loss: 2; bwd (CUDA-core): pre + dq + dkdv
+        # select: pool + score; fwd: 1; loss: 2; bwd: pre + dk/dv + dq (either path)
         return 2 + 1 + 2 + 3
 
     def run(self, stream, events=None):
@@ -263,11 +263,13 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
     avg = {n: per_call[n] / args.steps for n in names}
     dom = max(("fwd", "bwd"), key=lambda n: avg[n])
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    if dom == "fwd" and layer.path == 1:
-        achieved = f_fwd / (avg["fwd"] * 1e-3) / 1e12
-        roof = {"kernel": "fwd_tc_kernel", "bound": "tensor", "peak": sustained,
+    if layer.path == 1:
+        flops = f_fwd if dom == "fwd" else f_bwd
+        achieved = flops / (avg[dom] * 1e-3) / 1e12
+        name = "fwd_tc_kernel" if dom == "fwd" else "bwd_tc (pre + dkdv + dq kernels)"
+        roof = {"kernel": name, "bound": "tensor", "peak": sustained,
                 "unit": "TFLOP/s", "peak_kind": f"{peak_src} bf16 dense, sustained",
-                "traffic": ncu_traffic("fwd_tc_kernel")}
+                "traffic": ncu_traffic("fwd_tc_kernel" if dom == "fwd" else "bwd_tc")}
     else:
         flops = f_fwd if dom == "fwd" else f_bwd
         achieved = flops / (avg[dom] * 1e-3) / 1e12

@@ -65,10 +65,13 @@ int need_ws(void* ws, size_t have, size_t need, const char* what) {
 }
 
 bool use_tc(const ssa_params_t& p) {
-    return !(p.flags & SSA_FLAG_FORCE_SIMT) && fwd_tc_supported(p);
+    return !(p.flags & SSA_FLAG_FORCE_SIMT) && fwd_tc_supported(p) && bwd_tc_supported(p);
 }
 
 size_t fwd_workspace(const ssa_params_t& p) { return use_tc(p) ? fwd_tc_workspace(p) : 0; }
+size_t bwd_workspace(const ssa_params_t& p) {
+    return use_tc(p) ? bwd_tc_workspace(p) : bwd_simt_workspace(p);
+}
 
 }  // namespace
 
@@ -104,7 +107,7 @@ size_t ssa_workspace_size(const ssa_params_t* p, int which) {
         case SSA_WS_SELECT: return select_workspace(*p);
         case SSA_WS_FWD: return fwd_workspace(*p);
         case SSA_WS_LOSS: return loss_workspace(*p);
-        case SSA_WS_BWD: return bwd_simt_workspace(*p);
+        case SSA_WS_BWD: return bwd_workspace(*p);
         default: fail(SSA_ERR_INVALID_ARG, "unknown workspace id %d", which); return (size_t)-1;
     }
 }
@@ -187,9 +190,13 @@ int ssa_attn_bwd(const ssa_params_t* p, const void* q, const void* k, const void
     SSA_TRY(need_ptr(dv, "dv"));
     if (!std::isfinite(w_s) || !std::isfinite(w_c))
         return fail(SSA_ERR_INVALID_ARG, "loss weights must be finite");
-    SSA_TRY(need_ws(ws, ws_bytes, bwd_simt_workspace(*p), "ssa_attn_bwd"));
+    SSA_TRY(need_ws(ws, ws_bytes, bwd_workspace(*p), "ssa_attn_bwd"));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (use_tc(*p))
+        return launch_bwd_tc(*p, q, k, v, mask, h_full, h_sparse, lse_full, lse_sparse, dh_full,
+                             dh_sparse, w_s, w_c, dq, dk, dv, ws, s);
     return launch_bwd_simt(*p, q, k, v, mask, h_full, h_sparse, lse_full, lse_sparse, dh_full,
-                           dh_sparse, w_s, w_c, dq, dk, dv, ws, static_cast<cudaStream_t>(stream));
+                           dh_sparse, w_s, w_c, dq, dk, dv, ws, s);
 }
 
 int ssa_device_status(void* stream) {
@@ -198,6 +205,7 @@ int ssa_device_status(void* stream) {
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
     int st = fwd_tc_take_status(s);
+    if (st == SSA_OK) st = bwd_tc_take_status(s);
     if (st != SSA_OK) return st;
     return check_launch("pending");
 }

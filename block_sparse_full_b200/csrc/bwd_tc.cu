@@ -1,0 +1,842 @@
+// Backward through both SSA attention streams on the sm_100a tensor cores
+// (bf16 operands, fp32 accumulate, head dim 128).
+//
+// Math ("Sintesi Tecnica: SSA", section 2: the full stream carries gradient
+// to every token; L_sparsity and L_commit with stop-gradient on the opposite
+// stream).  For query t, key s <= t, x = sigma q_t.k_s:
+//   P_f = exp(x - lse_full(t));  P_s = c_t P_f on selected (t,s), else 0,
+//   with c_t = exp(lse_full(t) - lse_sparse(t)) (the sparse stream's own
+//   normaliser);
+//   dS  = P_f (G_f(t).v_s - D_f(t)) + P_s (G_s(t).v_s - D_s(t))
+//   dv_s = sum_t P_f G_f(t) + P_s G_s(t),  dk_s = sigma sum_t dS q_t,
+//   dq_t = sigma sum_s dS k_s,
+// where G_f, G_s are the upstream gradients of h_full, h_sparse plus the
+// alignment terms and D_f = G_f.h_full, D_s = G_s.h_sparse.
+//
+// Three kernels, no atomics (bitwise repeatable):
+//   bwd_tc_pre_kernel   one warp per row: G_f, G_s rounded to bf16, D_f and
+//                       D_s from the rounded values, lse_full*log2(e), c_t.
+//   bwd_dkdv_tc_kernel  CTA = 128 keys; steps of 64 queries.  Per step:
+//                       S^T = K Q^T, dP_f^T = V G_f^T, dP_s^T = V G_s^T
+//                       (tcgen05 SS, N = 64), the compute warpgroup forms
+//                       P_f^T, P_s^T, dS^T (bf16, written back to TMEM), then
+//                       dV += P_f^T G_f + P_s^T G_s and dK += dS^T Q (TS).
+//                       TMEM: dV | dK | S^T x2 | dP_f^T | dP_s^T = 512 cols.
+//   bwd_dq_tc_kernel    CTA = 128 queries; steps of 64 keys: S = Q K^T,
+//                       dP_f = G_f V^T, dP_s = G_s V^T, dS, dQ += dS K.
+//                       TMEM: dQ | S x2 | (dP_f, dP_s) x2 = 512 cols.
+// The sparse-stream MMAs are skipped on steps where no (query block, key
+// block) pair is selected.  Every wait is bounded; an expiry sets a device
+// status word and the CTA drains its tensor-core work and frees TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "ssa_internal.h"
+#include "tc_util.cuh"
+
+namespace ssa {
+namespace {
+
+using namespace tc;
+
+constexpr int HD = 128;
+constexpr int TILE = 128;  // keys per dK/dV CTA, queries per dQ CTA
+constexpr int STEP = 64;   // queries per dK/dV step, keys per dQ step
+constexpr int kThreads = 256;
+constexpr int kMaxWords = 256;
+constexpr int kMaxBlocks = kMaxWords * 32;
+constexpr uint32_t BOX_T = TILE * 128;  // [128 rows x 64 d] bf16 = 16 KB
+constexpr uint32_t BOX_S = STEP * 128;  // [64 rows x 64 d] bf16 = 8 KB
+constexpr uint32_t TILE_BYTES = 2 * BOX_T;
+constexpr uint32_t STEP_BYTES = 2 * BOX_S;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ unsigned int g_bwd_tc_status;
+
+struct BwdArgs {
+    __nv_bfloat16* dq;
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    const float* lse2;  // lse_full * log2(e)
+    const float* cfac;  // exp(lse_full - lse_sparse), 0 where the sparse mass is 0
+    const float* Df;
+    const float* Ds;
+    const uint32_t* mask;
+    int BH, T, block, words, n_blocks;
+    float scale_log2;  // sigma * log2(e)
+    float sm_scale;
+    unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ bool bit(const uint32_t* row, int j) {
+    return (row[j >> 5] >> (j & 31)) & 1u;
+}
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > limit_ns) return false;
+    return true;
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+// K-major SW128 operand of R rows x 128 d (two 64-column boxes of R*128
+// bytes): descriptor of MMA k-step kk (16 d per step).
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, uint32_t box_bytes, int kk) {
+    return smem_desc_sw128(base + (kk >> 2) * box_bytes + (kk & 3) * 32, 16, 1024);
+}
+// The same tile read as an MN-major B operand (N = d): k-step kk covers 16
+// rows (2 swizzle atoms of 8 rows); the two d-halves are box_bytes apart.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, uint32_t box_bytes, int kk) {
+    return smem_desc_sw128(base + kk * 2048, box_bytes, 1024);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+// Writes a TMEM accumulator row (128 fp32 columns at `col`) scaled by `mul`
+// as bf16 to global memory.
+__device__ __forceinline__ void store_row(uint32_t trow_col, float mul, __nv_bfloat16* dst,
+                                          bool valid) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        uint32_t u[32];
+        tmem_ld32(trow_col + 32 * c, u);
+        tmem_wait_ld();
+        uint32_t o[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            o[e] = pack_bf16(__uint_as_float(u[2 * e]) * mul, __uint_as_float(u[2 * e + 1]) * mul);
+        if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+                d4[v4] = make_uint4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
+        }
+    }
+}
+
+// ============================================================ preprocess
+// One warp per row, lane owns 4 consecutive columns.
+__global__ void __launch_bounds__(256)
+bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __restrict__ hs,
+                  const __nv_bfloat16* __restrict__ dhf, const __nv_bfloat16* __restrict__ dhs,
+                  const float* __restrict__ lse_f, const float* __restrict__ lse_s, size_t rows,
+                  float cf, float cs, __nv_bfloat16* __restrict__ gf, __nv_bfloat16* __restrict__ gs,
+                  float* __restrict__ lse2, float* __restrict__ cfac, float* __restrict__ Df,
+                  float* __restrict__ Ds) {
+    const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const size_t e = row * HD + 4 * lane;
+    auto ld4 = [](const __nv_bfloat16* p, float (&o)[4]) {
+        const uint2 u = *reinterpret_cast<const uint2*>(p);
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+        o[0] = __low2float(a); o[1] = __high2float(a); o[2] = __low2float(b); o[3] = __high2float(b);
+    };
+    float f[4], s[4], uf[4] = {0, 0, 0, 0}, us[4] = {0, 0, 0, 0};
+    ld4(hf + e, f);
+    ld4(hs + e, s);
+    if (dhf) ld4(dhf + e, uf);
+    if (dhs) ld4(dhs + e, us);
+    float sf = 0.f, ss = 0.f;
+    uint32_t pf[2], ps[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float gf0 = uf[2 * i] + cf * (f[2 * i] - s[2 * i]);
+        const float gf1 = uf[2 * i + 1] + cf * (f[2 * i + 1] - s[2 * i + 1]);
+        const float gs0 = us[2 * i] + cs * (s[2 * i] - f[2 * i]);
+        const float gs1 = us[2 * i + 1] + cs * (s[2 * i + 1] - f[2 * i + 1]);
+        pf[i] = pack_bf16(gf0, gf1);
+        ps[i] = pack_bf16(gs0, gs1);
+        // D from the rounded values the tensor cores will see
+        const __nv_bfloat162 rf = *reinterpret_cast<__nv_bfloat162*>(&pf[i]);
+        const __nv_bfloat162 rs = *reinterpret_cast<__nv_bfloat162*>(&ps[i]);
+        sf = fmaf(__low2float(rf), f[2 * i], fmaf(__high2float(rf), f[2 * i + 1], sf));
+        ss = fmaf(__low2float(rs), s[2 * i], fmaf(__high2float(rs), s[2 * i + 1], ss));
+    }
+    *reinterpret_cast<uint2*>(gf + e) = make_uint2(pf[0], pf[1]);
+    *reinterpret_cast<uint2*>(gs + e) = make_uint2(ps[0], ps[1]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        sf += __shfl_xor_sync(0xffffffffu, sf, o);
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    }
+    if (lane == 0) {
+        const float lf = lse_f[row], ls = lse_s[row];
+        lse2[row] = lf * kLog2e;
+        cfac[row] = ls > -INFINITY ? expf(lf - ls) : 0.f;
+        Df[row] = sf;
+        Ds[row] = ss;
+    }
+}
+
+// ============================================================ dK / dV
+namespace kv {
+constexpr uint32_t OFF_K = 0;
+constexpr uint32_t OFF_V = TILE_BYTES;
+constexpr uint32_t OFF_STAGE = 2 * TILE_BYTES;
+constexpr uint32_t ST_Q = 0, ST_GF = STEP_BYTES, ST_GS = 2 * STEP_BYTES, ST_ROWS = 3 * STEP_BYTES;
+constexpr uint32_t STAGE_BYTES = (3 * STEP_BYTES + 4 * STEP * 4 + 1023) / 1024 * 1024;
+constexpr uint32_t OFF_BAR = OFF_STAGE + 2 * STAGE_BYTES;
+constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
+constexpr uint32_t OFF_SEL = OFF_MISC + 16;  // one byte per query block
+constexpr uint32_t SMEM_BYTES = OFF_SEL + kMaxBlocks + 1024;
+enum : int { B_KV = 0, B_FULL = 1, B_EMPTY = 3, B_READY = 5, B_PREADY = 6, B_DONE = 7, B_DRAIN = 8 };
+constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_S0 = 256, TM_S1 = 320, TM_DPF = 384, TM_DPS = 448;
+}  // namespace kv
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_gf,
+                   const __grid_constant__ CUtensorMap tm_gs, const BwdArgs a) {
+    using namespace kv;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
+    uint8_t* selb = gbase + OFF_SEL;
+    unsigned int* status = &g_bwd_tc_status;
+    const uint64_t lim = a.timeout_ns;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int J = (int)(blockIdx.x / a.BH);  // key tile; J = 0 has the most steps: first
+    const int bh = (int)(blockIdx.x % a.BH);
+    const int s0 = J * TILE;
+    const int ns = (a.T - s0) / STEP;
+    const int kb0 = s0 / a.block;
+    const int kb1 = (s0 + 64 < a.T) ? (s0 + 64) / a.block : kb0;
+    const int qb_first = s0 / a.block;
+    auto BAR = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
+    const size_t rowbase = (size_t)bh * a.T;
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_KV), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(BAR(B_FULL + s), 1);
+            mbar_init(BAR(B_EMPTY + s), 1);
+        }
+        mbar_init(BAR(B_READY), 1);
+        mbar_init(BAR(B_PREADY), 128);
+        mbar_init(BAR(B_DONE), 1);
+        mbar_init(BAR(B_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // selection of this tile's key blocks for every later query block
+    for (int qb = qb_first + (int)threadIdx.x; qb < a.n_blocks; qb += kThreads) {
+        const uint32_t* m = a.mask + ((size_t)bh * a.n_blocks + qb) * a.words;
+        selb[qb] = (uint8_t)(bit(m, kb0) | (bit(m, kb1) << 1));
+    }
+    if (warp == 1) {
+        tmem_alloc(base + OFF_MISC, 512);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    auto step_qb = [&](int i) { return (s0 + STEP * i) / a.block; };
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---------------------------------------- TMA producer
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_gf);
+            prefetch_tmap(&tm_gs);
+            mbar_expect_tx(BAR(B_KV), 2 * TILE_BYTES);
+            tma_load_3d(base + OFF_K, &tm_k, BAR(B_KV), 0, s0, bh);
+            tma_load_3d(base + OFF_K + BOX_T, &tm_k, BAR(B_KV), 64, s0, bh);
+            tma_load_3d(base + OFF_V, &tm_v, BAR(B_KV), 0, s0, bh);
+            tma_load_3d(base + OFF_V + BOX_T, &tm_v, BAR(B_KV), 64, s0, bh);
+            int issued[2] = {-1, -1};
+            for (int i = 0; i < ns; ++i) {
+                const int s = i & 1;
+                if (i >= 2 && !mbar_wait(BAR(B_EMPTY + s), ((i >> 1) + 1) & 1, abort_flag, status, lim))
+                    break;
+                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                const int t0 = s0 + STEP * i;
+                mbar_expect_tx(BAR(B_FULL + s), 3 * STEP_BYTES + 4 * STEP * 4);
+                tma_load_3d(st + ST_Q, &tm_q, BAR(B_FULL + s), 0, t0, bh);
+                tma_load_3d(st + ST_Q + BOX_S, &tm_q, BAR(B_FULL + s), 64, t0, bh);
+                tma_load_3d(st + ST_GF, &tm_gf, BAR(B_FULL + s), 0, t0, bh);
+                tma_load_3d(st + ST_GF + BOX_S, &tm_gf, BAR(B_FULL + s), 64, t0, bh);
+                tma_load_3d(st + ST_GS, &tm_gs, BAR(B_FULL + s), 0, t0, bh);
+                tma_load_3d(st + ST_GS + BOX_S, &tm_gs, BAR(B_FULL + s), 64, t0, bh);
+                const size_t r0 = rowbase + t0;
+                bulk_load(st + ST_ROWS, a.lse2 + r0, STEP * 4, BAR(B_FULL + s));
+                bulk_load(st + ST_ROWS + STEP * 4, a.cfac + r0, STEP * 4, BAR(B_FULL + s));
+                bulk_load(st + ST_ROWS + 2 * STEP * 4, a.Df + r0, STEP * 4, BAR(B_FULL + s));
+                bulk_load(st + ST_ROWS + 3 * STEP * 4, a.Ds + r0, STEP * 4, BAR(B_FULL + s));
+                issued[s] = i;
+            }
+            wait_drain(BAR(B_KV), 0, lim);
+            if (*abort_flag)
+                for (int s = 0; s < 2; ++s)
+                    if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] >> 1) & 1, lim);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // ---------------------------------------- MMA issuer
+            constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S^T, dP^T
+            constexpr uint32_t id_a = idesc_bf16_f32(TILE, HD, true);     // dV, dK
+            bool ok = mbar_wait(BAR(B_KV), 0, abort_flag, status, lim);
+            auto sparse = [&](int i) { return selb[step_qb(i)] != 0; };
+            auto issue_s = [&](int i) {
+                const uint32_t st = base + OFF_STAGE + (i & 1) * STAGE_BYTES;
+                const uint32_t d = tmem + ((i & 1) ? TM_S1 : TM_S0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(d, kmajor_desc(base + OFF_K, BOX_T, kk), kmajor_desc(st + ST_Q, BOX_S, kk),
+                           id_s, kk > 0);
+            };
+            auto issue_dp = [&](int i) {
+                const uint32_t st = base + OFF_STAGE + (i & 1) * STAGE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmem + TM_DPF, kmajor_desc(base + OFF_V, BOX_T, kk),
+                           kmajor_desc(st + ST_GF, BOX_S, kk), id_s, kk > 0);
+                if (sparse(i)) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(tmem + TM_DPS, kmajor_desc(base + OFF_V, BOX_T, kk),
+                               kmajor_desc(st + ST_GS, BOX_S, kk), id_s, kk > 0);
+                }
+            };
+            if (ok && ns > 0) {
+                ok = mbar_wait(BAR(B_FULL), 0, abort_flag, status, lim);
+                if (ok) {
+                    fence_after_sync();
+                    issue_s(0);
+                    issue_dp(0);
+                    mma_commit(BAR(B_READY));
+                }
+            }
+            for (int i = 0; ok && i < ns; ++i) {
+                const int s = i & 1;
+                if (i + 1 < ns) {
+                    if (!mbar_wait(BAR(B_FULL + ((i + 1) & 1)), ((i + 1) >> 1) & 1, abort_flag, status,
+                                   lim)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
+                    issue_s(i + 1);
+                }
+                if (!mbar_wait(BAR(B_PREADY), i & 1, abort_flag, status, lim)) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                const uint32_t sb = tmem + (s ? TM_S1 : TM_S0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // dV += P_f^T G_f
+                    mma_ts(tmem + TM_DV, sb + 8 * kk, mnmajor_desc(st + ST_GF, BOX_S, kk), id_a,
+                           (i > 0 || kk > 0) ? 1u : 0u);
+                if (sparse(i)) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // dV += P_s^T G_s
+                        mma_ts(tmem + TM_DV, tmem + TM_DPS + 8 * kk, mnmajor_desc(st + ST_GS, BOX_S, kk),
+                               id_a, 1u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
+                    mma_ts(tmem + TM_DK, tmem + TM_DPF + 8 * kk, mnmajor_desc(st + ST_Q, BOX_S, kk),
+                           id_a, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(BAR(B_EMPTY + s));
+                if (i + 1 < ns) {
+                    issue_dp(i + 1);
+                    mma_commit(BAR(B_READY));
+                }
+            }
+            mma_commit(BAR(B_DONE));
+            mma_commit(BAR(B_DRAIN));
+            wait_drain(BAR(B_DRAIN), 0, lim);
+        }
+    } else if (warp >= 4) {
+        // -------------------------------------------------- compute warpgroup
+        const int sw = warp - 4;
+        const int r = sw * 32 + lane;  // key row of the tile == TMEM lane
+        const int s_tok = s0 + r;
+        const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
+        const float sl2 = a.scale_log2;
+        const bool in_kb1 = r >= 64 && a.block == 64;
+        bool ok = true;
+        for (int i = 0; i < ns; ++i) {
+            if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_READY), i & 1, abort_flag, status, lim))) {
+                ok = false;
+                break;
+            }
+            const int s = i & 1;
+            // the stage's row vectors (bulk copies) are read directly: observe their barrier
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(BAR(B_FULL + s), (i >> 1) & 1, abort_flag, status, lim))) {
+                ok = false;
+                break;
+            }
+            fence_after_sync();
+            const float* rows = reinterpret_cast<const float*>(gbase + OFF_STAGE + s * STAGE_BYTES + ST_ROWS);
+            const int t0 = s0 + STEP * i;
+            const uint8_t sb2 = selb[step_qb(i)];
+            const bool sparse = sb2 != 0;
+            const bool my_sel = in_kb1 ? (sb2 >> 1) & 1 : sb2 & 1;
+            const bool diag = t0 < s0 + TILE;
+            const uint32_t sbuf = trow + (s ? TM_S1 : TM_S0);
+#pragma unroll 1
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t su[32], fu[32], pu[32];
+                tmem_ld32(sbuf + 32 * ch, su);
+                tmem_ld32(trow + TM_DPF + 32 * ch, fu);
+                if (sparse) tmem_ld32(trow + TM_DPS + 32 * ch, pu);
+                tmem_wait_ld();
+                uint32_t pfk[16], psk[16], dsk[16];
+#pragma unroll
+                for (int j2 = 0; j2 < 16; ++j2) {
+                    float pf2[2], ps2[2], ds2[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int col = 32 * ch + 2 * j2 + h;
+                        const float x = fmaf(__uint_as_float(su[2 * j2 + h]), sl2, -rows[col]);
+                        float pf = ex2(x);
+                        if (diag && t0 + col < s_tok) pf = 0.f;
+                        float ds = pf * (__uint_as_float(fu[2 * j2 + h]) - rows[2 * STEP + col]);
+                        float ps = 0.f;
+                        if (sparse && my_sel) {
+                            ps = pf * rows[STEP + col];
+                            ds = fmaf(ps, __uint_as_float(pu[2 * j2 + h]) - rows[3 * STEP + col], ds);
+                        }
+                        pf2[h] = pf;
+                        ps2[h] = ps;
+                        ds2[h] = ds;
+                    }
+                    pfk[j2] = pack_bf16(pf2[0], pf2[1]);
+                    psk[j2] = pack_bf16(ps2[0], ps2[1]);
+                    dsk[j2] = pack_bf16(ds2[0], ds2[1]);
+                }
+                tmem_st16(sbuf + 16 * ch, pfk);                  // P_f^T
+                if (sparse) tmem_st16(trow + TM_DPS + 16 * ch, psk);  // P_s^T
+                tmem_st16(trow + TM_DPF + 16 * ch, dsk);         // dS^T
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(BAR(B_PREADY));
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim));
+        if (ok) {
+            fence_after_sync();
+            const bool valid = s_tok < a.T;
+            const size_t row = rowbase + (valid ? s_tok : 0);
+            store_row(trow + TM_DV, 1.f, a.dv + row * HD, valid);
+            store_row(trow + TM_DK, a.sm_scale, a.dk + row * HD, valid);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ============================================================ dQ
+namespace qk {
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_GF = TILE_BYTES;
+constexpr uint32_t OFF_GS = 2 * TILE_BYTES;
+constexpr uint32_t OFF_STAGE = 3 * TILE_BYTES;
+constexpr int NSTAGE = 3;
+constexpr uint32_t ST_K = 0, ST_V = STEP_BYTES;
+constexpr uint32_t STAGE_BYTES = 2 * STEP_BYTES;
+constexpr uint32_t OFF_BAR = OFF_STAGE + NSTAGE * STAGE_BYTES;
+constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
+constexpr uint32_t OFF_MASK = OFF_MISC + 16;
+constexpr uint32_t SMEM_BYTES = OFF_MASK + 2 * kMaxWords * 4 + 1024;
+enum : int { B_QG = 0, B_FULL = 1, B_EMPTY = 4, B_READY = 7, B_PREADY = 9, B_DONE = 11, B_DRAIN = 12 };
+constexpr uint32_t TM_DQ = 0, TM_S0 = 128, TM_S1 = 192, TM_DP0 = 256, TM_DP1 = 384;  // DP: f | s
+}  // namespace qk
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_gf,
+                 const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
+    using namespace qk;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
+    uint32_t* mrow = reinterpret_cast<uint32_t*>(gbase + OFF_MASK);
+    unsigned int* status = &g_bwd_tc_status;
+    const uint64_t lim = a.timeout_ns;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntq = (a.T + TILE - 1) / TILE;
+    const int I = ntq - 1 - (int)(blockIdx.x / a.BH);  // longest rows first
+    const int bh = (int)(blockIdx.x % a.BH);
+    const int t0 = I * TILE;
+    const int last = min(t0 + TILE, a.T);      // keys needed: [0, last)
+    const int ns = (last + STEP - 1) / STEP;
+    const bool ragged1 = t0 + 64 >= a.T;
+    const int qb0 = t0 / a.block;
+    const int qb1 = ragged1 ? qb0 : (t0 + 64) / a.block;
+    auto BAR = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
+    const size_t rowbase = (size_t)bh * a.T;
+
+    if (threadIdx.x == 0) {
+        mbar_init(BAR(B_QG), 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(BAR(B_FULL + s), 1);
+            mbar_init(BAR(B_EMPTY + s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR(B_READY + b), 1);
+            mbar_init(BAR(B_PREADY + b), 128);
+        }
+        mbar_init(BAR(B_DONE), 1);
+        mbar_init(BAR(B_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    {
+        const uint32_t* m0 = a.mask + ((size_t)bh * a.n_blocks + qb0) * a.words;
+        const uint32_t* m1 = a.mask + ((size_t)bh * a.n_blocks + qb1) * a.words;
+        for (int w = threadIdx.x; w < a.words; w += kThreads) {
+            mrow[w] = m0[w];
+            mrow[kMaxWords + w] = m1[w];
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc(base + OFF_MISC, 512);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    // key block of step i and whether either query block selects it
+    auto step_kb = [&](int i) { return (STEP * i) / a.block; };
+    auto sparse = [&](int i) {
+        const int kb = step_kb(i);
+        return bit(mrow, kb) || bit(mrow + kMaxWords, kb);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {  // ---------------------------------------- TMA producer
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_gf);
+            prefetch_tmap(&tm_gs);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            mbar_expect_tx(BAR(B_QG), 3 * TILE_BYTES);
+            tma_load_3d(base + OFF_Q, &tm_q, BAR(B_QG), 0, t0, bh);
+            tma_load_3d(base + OFF_Q + BOX_T, &tm_q, BAR(B_QG), 64, t0, bh);
+            tma_load_3d(base + OFF_GF, &tm_gf, BAR(B_QG), 0, t0, bh);
+            tma_load_3d(base + OFF_GF + BOX_T, &tm_gf, BAR(B_QG), 64, t0, bh);
+            tma_load_3d(base + OFF_GS, &tm_gs, BAR(B_QG), 0, t0, bh);
+            tma_load_3d(base + OFF_GS + BOX_T, &tm_gs, BAR(B_QG), 64, t0, bh);
+            int issued[NSTAGE] = {-1, -1, -1};
+            for (int i = 0; i < ns; ++i) {
+                const int s = i % NSTAGE;
+                if (i >= NSTAGE &&
+                    !mbar_wait(BAR(B_EMPTY + s), ((i / NSTAGE) + 1) & 1, abort_flag, status, lim))
+                    break;
+                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                mbar_expect_tx(BAR(B_FULL + s), 2 * STEP_BYTES);
+                tma_load_3d(st + ST_K, &tm_k, BAR(B_FULL + s), 0, STEP * i, bh);
+                tma_load_3d(st + ST_K + BOX_S, &tm_k, BAR(B_FULL + s), 64, STEP * i, bh);
+                tma_load_3d(st + ST_V, &tm_v, BAR(B_FULL + s), 0, STEP * i, bh);
+                tma_load_3d(st + ST_V + BOX_S, &tm_v, BAR(B_FULL + s), 64, STEP * i, bh);
+                issued[s] = i;
+            }
+            wait_drain(BAR(B_QG), 0, lim);
+            if (*abort_flag)
+                for (int s = 0; s < NSTAGE; ++s)
+                    if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, lim);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // ---------------------------------------- MMA issuer
+            constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S, dP
+            constexpr uint32_t id_q = idesc_bf16_f32(TILE, HD, true);     // dQ
+            bool ok = mbar_wait(BAR(B_QG), 0, abort_flag, status, lim);
+            auto issue_front = [&](int i) -> bool {  // S_i, dP_f_i, dP_s_i
+                const int s = i % NSTAGE, b = i & 1;
+                if (!mbar_wait(BAR(B_FULL + s), (i / NSTAGE) & 1, abort_flag, status, lim)) return false;
+                fence_after_sync();
+                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                const uint32_t sd = tmem + (b ? TM_S1 : TM_S0);
+                const uint32_t dp = tmem + (b ? TM_DP1 : TM_DP0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(sd, kmajor_desc(base + OFF_Q, BOX_T, kk), kmajor_desc(st + ST_K, BOX_S, kk),
+                           id_s, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(dp, kmajor_desc(base + OFF_GF, BOX_T, kk), kmajor_desc(st + ST_V, BOX_S, kk),
+                           id_s, kk > 0);
+                if (sparse(i)) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(dp + 64, kmajor_desc(base + OFF_GS, BOX_T, kk),
+                               kmajor_desc(st + ST_V, BOX_S, kk), id_s, kk > 0);
+                }
+                mma_commit(BAR(B_READY + b));
+                return true;
+            };
+            for (int i = 0; ok && i < ns && i < 2; ++i) ok = issue_front(i);
+            for (int i = 0; ok && i < ns; ++i) {
+                const int s = i % NSTAGE, b = i & 1;
+                if (!mbar_wait(BAR(B_PREADY + b), (i >> 1) & 1, abort_flag, status, lim)) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                const uint32_t sd = tmem + (b ? TM_S1 : TM_S0);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)  // dQ += dS K
+                    mma_ts(tmem + TM_DQ, sd + 8 * kk, mnmajor_desc(st + ST_K, BOX_S, kk), id_q,
+                           (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(BAR(B_EMPTY + s));
+                if (i + 2 < ns && !issue_front(i + 2)) ok = false;
+            }
+            mma_commit(BAR(B_DONE));
+            mma_commit(BAR(B_DRAIN));
+            wait_drain(BAR(B_DRAIN), 0, lim);
+        }
+    } else if (warp >= 4) {
+        // -------------------------------------------------- compute warpgroup
+        const int sw = warp - 4;
+        const int r = sw * 32 + lane;  // query row of the tile == TMEM lane
+        const int t = t0 + r;
+        const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
+        const size_t row = rowbase + (t < a.T ? t : a.T - 1);
+        const float my_lse2 = a.lse2[row], my_c = a.cfac[row], my_df = a.Df[row], my_ds = a.Ds[row];
+        const uint32_t* myrow = (r < 64 || a.block == 128 || ragged1) ? mrow : mrow + kMaxWords;
+        const float sl2 = a.scale_log2;
+        bool ok = true;
+        for (int i = 0; i < ns; ++i) {
+            const int b = i & 1;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(BAR(B_READY + b), (i >> 1) & 1, abort_flag, status, lim))) {
+                ok = false;
+                break;
+            }
+            fence_after_sync();
+            const bool sp = sparse(i);
+            const bool my_sel = bit(myrow, step_kb(i));
+            const int k0 = STEP * i;
+            const bool diag = k0 + STEP - 1 > t0;
+            const uint32_t sbuf = trow + (b ? TM_S1 : TM_S0);
+            const uint32_t dp = trow + (b ? TM_DP1 : TM_DP0);
+#pragma unroll 1
+            for (int ch = 0; ch < 2; ++ch) {
+                uint32_t su[32], fu[32], pu[32];
+                tmem_ld32(sbuf + 32 * ch, su);
+                tmem_ld32(dp + 32 * ch, fu);
+                if (sp) tmem_ld32(dp + 64 + 32 * ch, pu);
+                tmem_wait_ld();
+                uint32_t dsk[16];
+#pragma unroll
+                for (int j2 = 0; j2 < 16; ++j2) {
+                    float ds2[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int col = 32 * ch + 2 * j2 + h;
+                        float pf = ex2(fmaf(__uint_as_float(su[2 * j2 + h]), sl2, -my_lse2));
+                        if (diag && k0 + col > t) pf = 0.f;
+                        float ds = pf * (__uint_as_float(fu[2 * j2 + h]) - my_df);
+                        if (sp && my_sel)
+                            ds = fmaf(pf * my_c, __uint_as_float(pu[2 * j2 + h]) - my_ds, ds);
+                        ds2[h] = ds;
+                    }
+                    dsk[j2] = pack_bf16(ds2[0], ds2[1]);
+                }
+                tmem_st16(sbuf + 16 * ch, dsk);  // dS (bf16) over the consumed S columns
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(BAR(B_PREADY + b));
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim));
+        if (ok) {
+            fence_after_sync();
+            const bool valid = t < a.T;
+            store_row(trow + TM_DQ, a.sm_scale, a.dq + (valid ? row : rowbase) * HD, valid);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ============================================================ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// [BH, T, 128] bf16 as a 3-D tensor (d, t, bh); box 64 d x `rows` t; 128B swizzle.
+int make_map(CUtensorMap* m, const void* ptr, int BH, int T, int rows) {
+    auto fn = encode_fn();
+    if (!fn) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)T * HD * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return SSA_OK;
+}
+
+struct TcWs {
+    __nv_bfloat16* gf;
+    __nv_bfloat16* gs;
+    float *lse2, *cfac, *Df, *Ds;
+};
+
+TcWs carve(const ssa_params_t& p, void* ws) {
+    const size_t big = align_up(num_elems(p) * 2, 256);
+    const size_t small = align_up(num_rows(p) * 4, 256);
+    char* b = static_cast<char*>(ws);
+    TcWs w;
+    w.gf = reinterpret_cast<__nv_bfloat16*>(b);
+    w.gs = reinterpret_cast<__nv_bfloat16*>(b + big);
+    w.lse2 = reinterpret_cast<float*>(b + 2 * big);
+    w.cfac = reinterpret_cast<float*>(b + 2 * big + small);
+    w.Df = reinterpret_cast<float*>(b + 2 * big + 2 * small);
+    w.Ds = reinterpret_cast<float*>(b + 2 * big + 3 * small);
+    return w;
+}
+
+}  // namespace
+
+bool bwd_tc_supported(const ssa_params_t& p) {
+    return p.dtype == SSA_BF16 && p.D == HD && (p.block == 64 || p.block == 128) &&
+           mask_words(p) <= kMaxWords && num_blocks(p) <= kMaxBlocks &&
+           (size_t)p.B * p.H * ((p.T + TILE - 1) / TILE) <= 0x7fffffffull;
+}
+
+size_t bwd_tc_workspace(const ssa_params_t& p) {
+    return 2 * align_up(num_elems(p) * 2, 256) + 4 * align_up(num_rows(p) * 4, 256);
+}
+
+int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                  const uint32_t* mask, const void* hf, const void* hs, const float* lf,
+                  const float* ls, const void* dhf, const void* dhs, float w_s, float w_c,
+                  void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
+    const int BH = p.B * p.H;
+    const TcWs w = carve(p, ws);
+    const size_t rows = num_rows(p);
+    const double two_over_n = 2.0 / (double)num_elems(p);
+    bwd_tc_pre_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(hf), static_cast<const __nv_bfloat16*>(hs),
+        static_cast<const __nv_bfloat16*>(dhf), static_cast<const __nv_bfloat16*>(dhs), lf, ls, rows,
+        (float)(w_s * two_over_n), (float)(w_c * two_over_n), w.gf, w.gs, w.lse2, w.cfac, w.Df, w.Ds);
+    int st = check_launch("bwd_tc_pre_kernel");
+    if (st != SSA_OK) return st;
+
+    CUtensorMap k128, v128, q64, gf64, gs64, q128, gf128, gs128, k64, v64;
+    const void* srcs[5] = {q, k, v, w.gf, w.gs};
+    CUtensorMap* m128[5] = {&q128, &k128, &v128, &gf128, &gs128};
+    CUtensorMap* m64[5] = {&q64, &k64, &v64, &gf64, &gs64};
+    for (int i = 0; i < 5 && st == SSA_OK; ++i) {
+        st = make_map(m128[i], srcs[i], BH, p.T, TILE);
+        if (st == SSA_OK) st = make_map(m64[i], srcs[i], BH, p.T, STEP);
+    }
+    if (st != SSA_OK) return st;
+
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(bwd_dkdv_tc_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv::SMEM_BYTES);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(bwd_dq_tc_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)qk::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess)
+        return fail(SSA_ERR_CUDA, "bwd_tc: smem attribute: %s", cudaGetErrorString(attr_err));
+
+    BwdArgs a;
+    a.dq = static_cast<__nv_bfloat16*>(dq);
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.lse2 = w.lse2;
+    a.cfac = w.cfac;
+    a.Df = w.Df;
+    a.Ds = w.Ds;
+    a.mask = mask;
+    a.BH = BH;
+    a.T = p.T;
+    a.block = p.block;
+    a.words = mask_words(p);
+    a.n_blocks = num_blocks(p);
+    a.scale_log2 = p.sm_scale * kLog2e;
+    a.sm_scale = p.sm_scale;
+    a.timeout_ns = 2000000000ull;
+    const unsigned grid = (unsigned)((size_t)BH * ((p.T + TILE - 1) / TILE));
+    bwd_dkdv_tc_kernel<<<grid, kThreads, kv::SMEM_BYTES, s>>>(k128, v128, q64, gf64, gs64, a);
+    st = check_launch("bwd_dkdv_tc_kernel");
+    if (st != SSA_OK) return st;
+    bwd_dq_tc_kernel<<<grid, kThreads, qk::SMEM_BYTES, s>>>(q128, gf128, gs128, k64, v64, a);
+    return check_launch("bwd_dq_tc_kernel");
+}
+
+int bwd_tc_take_status(cudaStream_t) {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_bwd_tc_status, sizeof v);
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (v) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_bwd_tc_status, &zero, sizeof zero);
+        return fail(SSA_ERR_TIMEOUT, "bwd tcgen05 kernels: a bounded mbarrier wait expired");
+    }
+    return SSA_OK;
+}
+
+}  // namespace ssa

@@ -58,4 +58,14 @@ int launch_bwd_simt(const ssa_params_t& p, const void* q, const void* k, const v
                     const void* dh_sparse, float w_s, float w_c, void* dq, void* dk,
                     void* dv, void* ws, cudaStream_t s);
 
+// ---- backward, tcgen05 path (bwd_tc.cu)
+bool bwd_tc_supported(const ssa_params_t& p);
+size_t bwd_tc_workspace(const ssa_params_t& p);
+int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                  const uint32_t* mask, const void* h_full, const void* h_sparse,
+                  const float* lse_full, const float* lse_sparse, const void* dh_full,
+                  const void* dh_sparse, float w_s, float w_c, void* dq, void* dk, void* dv,
+                  void* ws, cudaStream_t s);
+int bwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
+
 }  // namespace ssa
