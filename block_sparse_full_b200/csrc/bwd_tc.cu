@@ -44,7 +44,8 @@ using namespace tc;
 constexpr int HD = 128;
 constexpr int TILE = 128;  // keys per dK/dV CTA, queries per dQ CTA
 constexpr int STEP = 64;   // queries per dK/dV step, keys per dQ step
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // warps 0-1 roles, 2-3 idle, 4-11 two compute warpgroups
+constexpr int kCompute = 256;
 constexpr int kMaxWords = 256;
 constexpr int kMaxBlocks = kMaxWords * 32;
 constexpr uint32_t BOX_T = TILE * 128;  // [128 rows x 64 d] bf16 = 16 KB
@@ -100,6 +101,10 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, uint32_t box_byt
     return smem_desc_sw128(base + kk * 2048, box_bytes, 1024);
 }
 
+// bf16 A operand of 64 K-columns written as two 32-wide halves, each half at
+// the start of its own 32-column fp32 source range: k-step kk (16 columns).
+__device__ __forceinline__ uint32_t split_acol(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
@@ -119,12 +124,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
-// Writes a TMEM accumulator row (128 fp32 columns at `col`) scaled by `mul`
-// as bf16 to global memory.
-__device__ __forceinline__ void store_row(uint32_t trow_col, float mul, __nv_bfloat16* dst,
-                                          bool valid) {
+// Writes 64 fp32 columns of a TMEM accumulator row (from `trow_col`) scaled
+// by `mul` as bf16 to global memory at dst.
+__device__ __forceinline__ void store_half_row(uint32_t trow_col, float mul, __nv_bfloat16* dst,
+                                               bool valid) {
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
         uint32_t u[32];
         tmem_ld32(trow_col + 32 * c, u);
         tmem_wait_ld();
@@ -245,7 +250,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             mbar_init(BAR(B_EMPTY + s), 1);
         }
         mbar_init(BAR(B_READY), 1);
-        mbar_init(BAR(B_PREADY), 128);
+        mbar_init(BAR(B_PREADY), kCompute);
         mbar_init(BAR(B_DONE), 1);
         mbar_init(BAR(B_DRAIN), 1);
         *abort_flag = 0;
@@ -266,8 +271,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const uint32_t tmem = *tmem_slot;
     auto step_qb = [&](int i) { return (s0 + STEP * i) / a.block; };
 
+    const unsigned FULL = 0xffffffffu;
     if (warp == 0) {
-        if (lane == 0) {  // ---------------------------------------- TMA producer
+        // -------------------------------------------- TMA producer (whole warp)
+        if (elect_one()) {
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_q);
@@ -278,13 +285,17 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tma_load_3d(base + OFF_K + BOX_T, &tm_k, BAR(B_KV), 64, s0, bh);
             tma_load_3d(base + OFF_V, &tm_v, BAR(B_KV), 0, s0, bh);
             tma_load_3d(base + OFF_V + BOX_T, &tm_v, BAR(B_KV), 64, s0, bh);
-            int issued[2] = {-1, -1};
-            for (int i = 0; i < ns; ++i) {
-                const int s = i & 1;
-                if (i >= 2 && !mbar_wait(BAR(B_EMPTY + s), ((i >> 1) + 1) & 1, abort_flag, status, lim))
-                    break;
-                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
-                const int t0 = s0 + STEP * i;
+        }
+        __syncwarp();
+        int issued[2] = {-1, -1};
+        for (int i = 0; i < ns; ++i) {
+            const int s = i & 1;
+            if (i >= 2 &&
+                !__all_sync(FULL, mbar_wait(BAR(B_EMPTY + s), ((i >> 1) + 1) & 1, abort_flag, status, lim)))
+                break;
+            const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+            const int t0 = s0 + STEP * i;
+            if (elect_one()) {
                 mbar_expect_tx(BAR(B_FULL + s), 3 * STEP_BYTES + 4 * STEP * 4);
                 tma_load_3d(st + ST_Q, &tm_q, BAR(B_FULL + s), 0, t0, bh);
                 tma_load_3d(st + ST_Q + BOX_S, &tm_q, BAR(B_FULL + s), 64, t0, bh);
@@ -297,61 +308,62 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 bulk_load(st + ST_ROWS + STEP * 4, a.cfac + r0, STEP * 4, BAR(B_FULL + s));
                 bulk_load(st + ST_ROWS + 2 * STEP * 4, a.Df + r0, STEP * 4, BAR(B_FULL + s));
                 bulk_load(st + ST_ROWS + 3 * STEP * 4, a.Ds + r0, STEP * 4, BAR(B_FULL + s));
-                issued[s] = i;
             }
-            wait_drain(BAR(B_KV), 0, lim);
-            if (*abort_flag)
-                for (int s = 0; s < 2; ++s)
-                    if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] >> 1) & 1, lim);
+            __syncwarp();
+            issued[s] = i;
         }
+        wait_drain(BAR(B_KV), 0, lim);
+        if (*abort_flag)
+            for (int s = 0; s < 2; ++s)
+                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] >> 1) & 1, lim);
     } else if (warp == 1) {
-        if (lane == 0) {  // ---------------------------------------- MMA issuer
+        {  // ------------------------------------------ MMA issuer (whole warp)
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S^T, dP^T
             constexpr uint32_t id_a = idesc_bf16_f32(TILE, HD, true);     // dV, dK
-            bool ok = mbar_wait(BAR(B_KV), 0, abort_flag, status, lim);
+            bool ok = __all_sync(FULL, mbar_wait(BAR(B_KV), 0, abort_flag, status, lim));
             auto sparse = [&](int i) { return selb[step_qb(i)] != 0; };
             auto issue_s = [&](int i) {
                 const uint32_t st = base + OFF_STAGE + (i & 1) * STAGE_BYTES;
                 const uint32_t d = tmem + ((i & 1) ? TM_S1 : TM_S0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(d, kmajor_desc(base + OFF_K, BOX_T, kk), kmajor_desc(st + ST_Q, BOX_S, kk),
+                    mma_ss_w(d, kmajor_desc(base + OFF_K, BOX_T, kk), kmajor_desc(st + ST_Q, BOX_S, kk),
                            id_s, kk > 0);
             };
             auto issue_dp = [&](int i) {
                 const uint32_t st = base + OFF_STAGE + (i & 1) * STAGE_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + TM_DPF, kmajor_desc(base + OFF_V, BOX_T, kk),
+                    mma_ss_w(tmem + TM_DPF, kmajor_desc(base + OFF_V, BOX_T, kk),
                            kmajor_desc(st + ST_GF, BOX_S, kk), id_s, kk > 0);
                 if (sparse(i)) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + TM_DPS, kmajor_desc(base + OFF_V, BOX_T, kk),
+                        mma_ss_w(tmem + TM_DPS, kmajor_desc(base + OFF_V, BOX_T, kk),
                                kmajor_desc(st + ST_GS, BOX_S, kk), id_s, kk > 0);
                 }
             };
             if (ok && ns > 0) {
-                ok = mbar_wait(BAR(B_FULL), 0, abort_flag, status, lim);
+                ok = __all_sync(FULL, mbar_wait(BAR(B_FULL), 0, abort_flag, status, lim));
                 if (ok) {
                     fence_after_sync();
                     issue_s(0);
                     issue_dp(0);
-                    mma_commit(BAR(B_READY));
+                    mma_commit_w(BAR(B_READY));
                 }
             }
             for (int i = 0; ok && i < ns; ++i) {
                 const int s = i & 1;
                 if (i + 1 < ns) {
-                    if (!mbar_wait(BAR(B_FULL + ((i + 1) & 1)), ((i + 1) >> 1) & 1, abort_flag, status,
-                                   lim)) {
+                    if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + ((i + 1) & 1)), ((i + 1) >> 1) & 1,
+                                                    abort_flag, status, lim))) {
                         ok = false;
                         break;
                     }
                     fence_after_sync();
                     issue_s(i + 1);
                 }
-                if (!mbar_wait(BAR(B_PREADY), i & 1, abort_flag, status, lim)) {
+                if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY), i & 1, abort_flag, status, lim))) {
                     ok = false;
                     break;
                 }
@@ -360,36 +372,38 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const uint32_t sb = tmem + (s ? TM_S1 : TM_S0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // dV += P_f^T G_f
-                    mma_ts(tmem + TM_DV, sb + 8 * kk, mnmajor_desc(st + ST_GF, BOX_S, kk), id_a,
+                    mma_ts_w(tmem + TM_DV, sb + split_acol(kk), mnmajor_desc(st + ST_GF, BOX_S, kk), id_a,
                            (i > 0 || kk > 0) ? 1u : 0u);
                 if (sparse(i)) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // dV += P_s^T G_s
-                        mma_ts(tmem + TM_DV, tmem + TM_DPS + 8 * kk, mnmajor_desc(st + ST_GS, BOX_S, kk),
-                               id_a, 1u);
+                        mma_ts_w(tmem + TM_DV, tmem + TM_DPS + split_acol(kk),
+                               mnmajor_desc(st + ST_GS, BOX_S, kk), id_a, 1u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-                    mma_ts(tmem + TM_DK, tmem + TM_DPF + 8 * kk, mnmajor_desc(st + ST_Q, BOX_S, kk),
+                    mma_ts_w(tmem + TM_DK, tmem + TM_DPF + split_acol(kk), mnmajor_desc(st + ST_Q, BOX_S, kk),
                            id_a, (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(BAR(B_EMPTY + s));
+                mma_commit_w(BAR(B_EMPTY + s));
                 if (i + 1 < ns) {
                     issue_dp(i + 1);
-                    mma_commit(BAR(B_READY));
+                    mma_commit_w(BAR(B_READY));
                 }
             }
-            mma_commit(BAR(B_DONE));
-            mma_commit(BAR(B_DRAIN));
+            mma_commit_w(BAR(B_DONE));
+            mma_commit_w(BAR(B_DRAIN));
             wait_drain(BAR(B_DRAIN), 0, lim);
         }
     } else if (warp >= 4) {
-        // -------------------------------------------------- compute warpgroup
-        const int sw = warp - 4;
+        // ------------------------------------------ two compute warpgroups
+        // warpgroup wg handles columns [32 wg, 32 wg + 32) of every step
+        const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
         const int r = sw * 32 + lane;  // key row of the tile == TMEM lane
         const int s_tok = s0 + r;
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
         const float sl2 = a.scale_log2;
         const bool in_kb1 = r >= 64 && a.block == 64;
+        const int c0 = 32 * wg;
         bool ok = true;
         for (int i = 0; i < ns; ++i) {
             if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_READY), i & 1, abort_flag, status, lim))) {
@@ -404,48 +418,55 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 break;
             }
             fence_after_sync();
-            const float* rows = reinterpret_cast<const float*>(gbase + OFF_STAGE + s * STAGE_BYTES + ST_ROWS);
+            const float4* rows4 = reinterpret_cast<const float4*>(
+                gbase + OFF_STAGE + s * STAGE_BYTES + ST_ROWS);  // lse2 | c | Df | Ds, 64 each
             const int t0 = s0 + STEP * i;
             const uint8_t sb2 = selb[step_qb(i)];
             const bool sparse = sb2 != 0;
             const bool my_sel = in_kb1 ? (sb2 >> 1) & 1 : sb2 & 1;
+            const bool use_s = sparse && my_sel;
             const bool diag = t0 < s0 + TILE;
             const uint32_t sbuf = trow + (s ? TM_S1 : TM_S0);
-#pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t su[32], fu[32], pu[32];
-                tmem_ld32(sbuf + 32 * ch, su);
-                tmem_ld32(trow + TM_DPF + 32 * ch, fu);
-                if (sparse) tmem_ld32(trow + TM_DPS + 32 * ch, pu);
-                tmem_wait_ld();
-                uint32_t pfk[16], psk[16], dsk[16];
+            uint32_t su[32], fu[32], pu[32];
+            tmem_ld32(sbuf + c0, su);
+            tmem_ld32(trow + TM_DPF + c0, fu);
+            if (sparse) tmem_ld32(trow + TM_DPS + c0, pu);
+            tmem_wait_ld();
+            uint32_t pfk[16], psk[16], dsk[16];
 #pragma unroll
-                for (int j2 = 0; j2 < 16; ++j2) {
-                    float pf2[2], ps2[2], ds2[2];
+            for (int j4 = 0; j4 < 8; ++j4) {
+                const int col = c0 + 4 * j4;
+                const float4 L = rows4[col >> 2], C = rows4[(STEP + col) >> 2];
+                const float4 F = rows4[(2 * STEP + col) >> 2], S = rows4[(3 * STEP + col) >> 2];
+                const float lv[4] = {L.x, L.y, L.z, L.w}, cv[4] = {C.x, C.y, C.z, C.w};
+                const float fv[4] = {F.x, F.y, F.z, F.w}, sv[4] = {S.x, S.y, S.z, S.w};
+                float pf[4], ps[4], ds[4];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int col = 32 * ch + 2 * j2 + h;
-                        const float x = fmaf(__uint_as_float(su[2 * j2 + h]), sl2, -rows[col]);
-                        float pf = ex2(x);
-                        if (diag && t0 + col < s_tok) pf = 0.f;
-                        float ds = pf * (__uint_as_float(fu[2 * j2 + h]) - rows[2 * STEP + col]);
-                        float ps = 0.f;
-                        if (sparse && my_sel) {
-                            ps = pf * rows[STEP + col];
-                            ds = fmaf(ps, __uint_as_float(pu[2 * j2 + h]) - rows[3 * STEP + col], ds);
-                        }
-                        pf2[h] = pf;
-                        ps2[h] = ps;
-                        ds2[h] = ds;
+                for (int h = 0; h < 4; ++h) {
+                    const int j = 4 * j4 + h;
+                    float p = ex2(fmaf(__uint_as_float(su[j]), sl2, -lv[h]));
+                    if (diag && t0 + col + h < s_tok) p = 0.f;
+                    float d = p * (__uint_as_float(fu[j]) - fv[h]);
+                    float q2 = 0.f;
+                    if (use_s) {
+                        q2 = p * cv[h];
+                        d = fmaf(q2, __uint_as_float(pu[j]) - sv[h], d);
                     }
-                    pfk[j2] = pack_bf16(pf2[0], pf2[1]);
-                    psk[j2] = pack_bf16(ps2[0], ps2[1]);
-                    dsk[j2] = pack_bf16(ds2[0], ds2[1]);
+                    pf[h] = p;
+                    ps[h] = q2;
+                    ds[h] = d;
                 }
-                tmem_st16(sbuf + 16 * ch, pfk);                  // P_f^T
-                if (sparse) tmem_st16(trow + TM_DPS + 16 * ch, psk);  // P_s^T
-                tmem_st16(trow + TM_DPF + 16 * ch, dsk);         // dS^T
+                pfk[2 * j4] = pack_bf16_alu(pf[0], pf[1]);
+                pfk[2 * j4 + 1] = pack_bf16_alu(pf[2], pf[3]);
+                psk[2 * j4] = pack_bf16_alu(ps[0], ps[1]);
+                psk[2 * j4 + 1] = pack_bf16_alu(ps[2], ps[3]);
+                dsk[2 * j4] = pack_bf16_alu(ds[0], ds[1]);
+                dsk[2 * j4 + 1] = pack_bf16_alu(ds[2], ds[3]);
             }
+            // bf16 results go to the first 16 columns of this warpgroup's own range
+            tmem_st16(sbuf + c0, pfk);                       // P_f^T
+            if (sparse) tmem_st16(trow + TM_DPS + c0, psk);  // P_s^T
+            tmem_st16(trow + TM_DPF + c0, dsk);              // dS^T
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PREADY));
@@ -455,8 +476,8 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             fence_after_sync();
             const bool valid = s_tok < a.T;
             const size_t row = rowbase + (valid ? s_tok : 0);
-            store_row(trow + TM_DV, 1.f, a.dv + row * HD, valid);
-            store_row(trow + TM_DK, a.sm_scale, a.dk + row * HD, valid);
+            store_half_row(trow + TM_DV + 64 * wg, 1.f, a.dv + row * HD + 64 * wg, valid);
+            store_half_row(trow + TM_DK + 64 * wg, a.sm_scale, a.dk + row * HD + 64 * wg, valid);
         }
     }
     fence_before_sync();
@@ -520,7 +541,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR(B_READY + b), 1);
-            mbar_init(BAR(B_PREADY + b), 128);
+            mbar_init(BAR(B_PREADY + b), kCompute);
         }
         mbar_init(BAR(B_DONE), 1);
         mbar_init(BAR(B_DRAIN), 1);
@@ -550,8 +571,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         return bit(mrow, kb) || bit(mrow + kMaxWords, kb);
     };
 
+    const unsigned FULL = 0xffffffffu;
     if (warp == 0) {
-        if (lane == 0) {  // ---------------------------------------- TMA producer
+        // -------------------------------------------- TMA producer (whole warp)
+        if (elect_one()) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_gf);
             prefetch_tmap(&tm_gs);
@@ -564,58 +587,64 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tma_load_3d(base + OFF_GF + BOX_T, &tm_gf, BAR(B_QG), 64, t0, bh);
             tma_load_3d(base + OFF_GS, &tm_gs, BAR(B_QG), 0, t0, bh);
             tma_load_3d(base + OFF_GS + BOX_T, &tm_gs, BAR(B_QG), 64, t0, bh);
-            int issued[NSTAGE] = {-1, -1, -1};
-            for (int i = 0; i < ns; ++i) {
-                const int s = i % NSTAGE;
-                if (i >= NSTAGE &&
-                    !mbar_wait(BAR(B_EMPTY + s), ((i / NSTAGE) + 1) & 1, abort_flag, status, lim))
-                    break;
-                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+        }
+        __syncwarp();
+        int issued[NSTAGE] = {-1, -1, -1};
+        for (int i = 0; i < ns; ++i) {
+            const int s = i % NSTAGE;
+            if (i >= NSTAGE &&
+                !__all_sync(FULL, mbar_wait(BAR(B_EMPTY + s), ((i / NSTAGE) + 1) & 1, abort_flag, status,
+                                            lim)))
+                break;
+            const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+            if (elect_one()) {
                 mbar_expect_tx(BAR(B_FULL + s), 2 * STEP_BYTES);
                 tma_load_3d(st + ST_K, &tm_k, BAR(B_FULL + s), 0, STEP * i, bh);
                 tma_load_3d(st + ST_K + BOX_S, &tm_k, BAR(B_FULL + s), 64, STEP * i, bh);
                 tma_load_3d(st + ST_V, &tm_v, BAR(B_FULL + s), 0, STEP * i, bh);
                 tma_load_3d(st + ST_V + BOX_S, &tm_v, BAR(B_FULL + s), 64, STEP * i, bh);
-                issued[s] = i;
             }
-            wait_drain(BAR(B_QG), 0, lim);
-            if (*abort_flag)
-                for (int s = 0; s < NSTAGE; ++s)
-                    if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, lim);
+            __syncwarp();
+            issued[s] = i;
         }
+        wait_drain(BAR(B_QG), 0, lim);
+        if (*abort_flag)
+            for (int s = 0; s < NSTAGE; ++s)
+                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, lim);
     } else if (warp == 1) {
-        if (lane == 0) {  // ---------------------------------------- MMA issuer
+        {  // ------------------------------------------ MMA issuer (whole warp)
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S, dP
             constexpr uint32_t id_q = idesc_bf16_f32(TILE, HD, true);     // dQ
-            bool ok = mbar_wait(BAR(B_QG), 0, abort_flag, status, lim);
+            bool ok = __all_sync(FULL, mbar_wait(BAR(B_QG), 0, abort_flag, status, lim));
             auto issue_front = [&](int i) -> bool {  // S_i, dP_f_i, dP_s_i
                 const int s = i % NSTAGE, b = i & 1;
-                if (!mbar_wait(BAR(B_FULL + s), (i / NSTAGE) & 1, abort_flag, status, lim)) return false;
+                if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + s), (i / NSTAGE) & 1, abort_flag, status, lim)))
+                    return false;
                 fence_after_sync();
                 const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
                 const uint32_t sd = tmem + (b ? TM_S1 : TM_S0);
                 const uint32_t dp = tmem + (b ? TM_DP1 : TM_DP0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(sd, kmajor_desc(base + OFF_Q, BOX_T, kk), kmajor_desc(st + ST_K, BOX_S, kk),
+                    mma_ss_w(sd, kmajor_desc(base + OFF_Q, BOX_T, kk), kmajor_desc(st + ST_K, BOX_S, kk),
                            id_s, kk > 0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(dp, kmajor_desc(base + OFF_GF, BOX_T, kk), kmajor_desc(st + ST_V, BOX_S, kk),
+                    mma_ss_w(dp, kmajor_desc(base + OFF_GF, BOX_T, kk), kmajor_desc(st + ST_V, BOX_S, kk),
                            id_s, kk > 0);
                 if (sparse(i)) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(dp + 64, kmajor_desc(base + OFF_GS, BOX_T, kk),
+                        mma_ss_w(dp + 64, kmajor_desc(base + OFF_GS, BOX_T, kk),
                                kmajor_desc(st + ST_V, BOX_S, kk), id_s, kk > 0);
                 }
-                mma_commit(BAR(B_READY + b));
+                mma_commit_w(BAR(B_READY + b));
                 return true;
             };
             for (int i = 0; ok && i < ns && i < 2; ++i) ok = issue_front(i);
             for (int i = 0; ok && i < ns; ++i) {
                 const int s = i % NSTAGE, b = i & 1;
-                if (!mbar_wait(BAR(B_PREADY + b), (i >> 1) & 1, abort_flag, status, lim)) {
+                if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY + b), (i >> 1) & 1, abort_flag, status, lim))) {
                     ok = false;
                     break;
                 }
@@ -624,18 +653,19 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const uint32_t sd = tmem + (b ? TM_S1 : TM_S0);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)  // dQ += dS K
-                    mma_ts(tmem + TM_DQ, sd + 8 * kk, mnmajor_desc(st + ST_K, BOX_S, kk), id_q,
+                    mma_ts_w(tmem + TM_DQ, sd + split_acol(kk), mnmajor_desc(st + ST_K, BOX_S, kk), id_q,
                            (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(BAR(B_EMPTY + s));
+                mma_commit_w(BAR(B_EMPTY + s));
                 if (i + 2 < ns && !issue_front(i + 2)) ok = false;
             }
-            mma_commit(BAR(B_DONE));
-            mma_commit(BAR(B_DRAIN));
+            mma_commit_w(BAR(B_DONE));
+            mma_commit_w(BAR(B_DRAIN));
             wait_drain(BAR(B_DRAIN), 0, lim);
         }
     } else if (warp >= 4) {
-        // -------------------------------------------------- compute warpgroup
-        const int sw = warp - 4;
+        // ------------------------------------------ two compute warpgroups
+        // warpgroup wg handles key columns [32 wg, 32 wg + 32) of every step
+        const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
         const int r = sw * 32 + lane;  // query row of the tile == TMEM lane
         const int t = t0 + r;
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
@@ -643,6 +673,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float my_lse2 = a.lse2[row], my_c = a.cfac[row], my_df = a.Df[row], my_ds = a.Ds[row];
         const uint32_t* myrow = (r < 64 || a.block == 128 || ragged1) ? mrow : mrow + kMaxWords;
         const float sl2 = a.scale_log2;
+        const int c0 = 32 * wg;
         bool ok = true;
         for (int i = 0; i < ns; ++i) {
             const int b = i & 1;
@@ -653,36 +684,32 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             fence_after_sync();
             const bool sp = sparse(i);
-            const bool my_sel = bit(myrow, step_kb(i));
-            const int k0 = STEP * i;
-            const bool diag = k0 + STEP - 1 > t0;
+            const bool use_s = sp && bit(myrow, step_kb(i));
+            const int k0 = STEP * i + c0;
+            const bool diag = k0 + 31 > t0;
             const uint32_t sbuf = trow + (b ? TM_S1 : TM_S0);
             const uint32_t dp = trow + (b ? TM_DP1 : TM_DP0);
-#pragma unroll 1
-            for (int ch = 0; ch < 2; ++ch) {
-                uint32_t su[32], fu[32], pu[32];
-                tmem_ld32(sbuf + 32 * ch, su);
-                tmem_ld32(dp + 32 * ch, fu);
-                if (sp) tmem_ld32(dp + 64 + 32 * ch, pu);
-                tmem_wait_ld();
-                uint32_t dsk[16];
+            uint32_t su[32], fu[32], pu[32];
+            tmem_ld32(sbuf + c0, su);
+            tmem_ld32(dp + c0, fu);
+            if (sp) tmem_ld32(dp + 64 + c0, pu);
+            tmem_wait_ld();
+            uint32_t dsk[16];
 #pragma unroll
-                for (int j2 = 0; j2 < 16; ++j2) {
-                    float ds2[2];
+            for (int j2 = 0; j2 < 16; ++j2) {
+                float ds2[2];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int col = 32 * ch + 2 * j2 + h;
-                        float pf = ex2(fmaf(__uint_as_float(su[2 * j2 + h]), sl2, -my_lse2));
-                        if (diag && k0 + col > t) pf = 0.f;
-                        float ds = pf * (__uint_as_float(fu[2 * j2 + h]) - my_df);
-                        if (sp && my_sel)
-                            ds = fmaf(pf * my_c, __uint_as_float(pu[2 * j2 + h]) - my_ds, ds);
-                        ds2[h] = ds;
-                    }
-                    dsk[j2] = pack_bf16(ds2[0], ds2[1]);
+                for (int h = 0; h < 2; ++h) {
+                    const int j = 2 * j2 + h;
+                    float pf = ex2(fmaf(__uint_as_float(su[j]), sl2, -my_lse2));
+                    if (diag && k0 + j > t) pf = 0.f;
+                    float ds = pf * (__uint_as_float(fu[j]) - my_df);
+                    if (use_s) ds = fmaf(pf * my_c, __uint_as_float(pu[j]) - my_ds, ds);
+                    ds2[h] = ds;
                 }
-                tmem_st16(sbuf + 16 * ch, dsk);  // dS (bf16) over the consumed S columns
+                dsk[j2] = pack_bf16_alu(ds2[0], ds2[1]);
             }
+            tmem_st16(sbuf + c0, dsk);  // dS (bf16) over this warpgroup's consumed S columns
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PREADY + b));
@@ -691,7 +718,8 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (ok) {
             fence_after_sync();
             const bool valid = t < a.T;
-            store_row(trow + TM_DQ, a.sm_scale, a.dq + (valid ? row : rowbase) * HD, valid);
+            store_half_row(trow + TM_DQ + 64 * wg, a.sm_scale,
+                           a.dq + (valid ? row : rowbase) * HD + 64 * wg, valid);
         }
     }
     fence_before_sync();

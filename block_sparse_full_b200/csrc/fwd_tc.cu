@@ -46,7 +46,8 @@ using namespace tc;
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int HD = 128;  // head dim
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;  // warps 0-1 roles, 2-3 idle, 4-11 two softmax warpgroups
+constexpr int kSoftmax = 256;
 constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB
 constexpr uint32_t HALF_BYTES = 128 * 128;    // [128 rows x 64 cols] bf16 box, 16 KB
 constexpr int kMaxWords = 256;                // mask words per query block (n <= 8192)
@@ -58,7 +59,11 @@ constexpr uint32_t OFF_BAR = OFF_V + 2 * TILE_BYTES;
 constexpr int NBAR = 16;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // [0] tmem base, [1] abort flag
 constexpr uint32_t OFF_MASK = OFF_MISC + 16;       // mask rows of the two query blocks
-constexpr uint32_t SMEM_USED = OFF_MASK + 2 * kMaxWords * 4;
+// warpgroup exchange area, 1024 f32: row maxima [parity][wg][row] (512), then in
+// the epilogue l_sel/l_uns [wg][2][row] (512) and squared-difference sums [wg][row]
+// at offset 512 (256)
+constexpr uint32_t OFF_XCH = OFF_MASK + 2 * kMaxWords * 4;
+constexpr uint32_t SMEM_USED = OFF_XCH + 1024 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 
 enum : int {
@@ -68,6 +73,7 @@ enum : int {
 
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_OSEL = 256, TM_OUNS = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kPolyLane = 3;  // pairs c with c % 4 == 3 use the FMA-pipe exponential
 constexpr float kLn2 = 0.693147180559945309f;
 
 __device__ unsigned int g_fwd_tc_status;
@@ -140,7 +146,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(BAR(B_VFULL + s), 1);
             mbar_init(BAR(B_VEMPTY + s), 1);
             mbar_init(BAR(B_SREADY + s), 1);
-            mbar_init(BAR(B_PREADY + s), 128);
+            mbar_init(BAR(B_PREADY + s), kSoftmax);
         }
         mbar_init(BAR(B_PVDONE), 1);
         mbar_init(BAR(B_DRAIN), 1);
@@ -164,114 +170,145 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
+    // Roles 0 and 1 run their loops with the whole warp (warp-uniform address and
+    // descriptor arithmetic); one elected lane issues each TMA / tcgen05 op.
+    const unsigned FULL = 0xffffffffu;
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (elect_one()) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             mbar_expect_tx(BAR(B_QFULL), TILE_BYTES);
             tma_load_3d(base + OFF_Q, &tm_q, BAR(B_QFULL), 0, t0, bh);
             tma_load_3d(base + OFF_Q + HALF_BYTES, &tm_q, BAR(B_QFULL), 64, t0, bh);
-            int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
-            for (int j = 0; j < ntk; ++j) {
-                const int s = j & 1;
-                const uint32_t ph = ((j >> 1) + 1) & 1;
-                const uint32_t kdst = base + OFF_K + s * TILE_BYTES;
-                const uint32_t vdst = base + OFF_V + s * TILE_BYTES;
-                if (j >= 2 && !mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, status, lim)) break;
+        }
+        __syncwarp();
+        int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
+        for (int j = 0; j < ntk; ++j) {
+            const int s = j & 1;
+            const uint32_t ph = ((j >> 1) + 1) & 1;
+            const uint32_t kdst = base + OFF_K + s * TILE_BYTES;
+            const uint32_t vdst = base + OFF_V + s * TILE_BYTES;
+            if (j >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, status, lim)))
+                break;
+            if (elect_one()) {
                 mbar_expect_tx(BAR(B_KFULL + s), TILE_BYTES);
                 tma_load_3d(kdst, &tm_k, BAR(B_KFULL + s), 0, j * BN, bh);
                 tma_load_3d(kdst + HALF_BYTES, &tm_k, BAR(B_KFULL + s), 64, j * BN, bh);
-                issued_k[s] = j;
-                if (j >= 2 && !mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, status, lim)) break;
+            }
+            __syncwarp();
+            issued_k[s] = j;
+            if (j >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, status, lim)))
+                break;
+            if (elect_one()) {
                 mbar_expect_tx(BAR(B_VFULL + s), TILE_BYTES);
                 tma_load_3d(vdst, &tm_v, BAR(B_VFULL + s), 0, j * BN, bh);
                 tma_load_3d(vdst + HALF_BYTES, &tm_v, BAR(B_VFULL + s), 64, j * BN, bh);
-                issued_v[s] = j;
             }
-            if (*abort_flag) {  // let copies in flight land before the CTA exits
-                for (int s = 0; s < 2; ++s) {
-                    if (issued_k[s] >= 0) wait_drain(BAR(B_KFULL + s), (issued_k[s] >> 1) & 1, lim);
-                    if (issued_v[s] >= 0) wait_drain(BAR(B_VFULL + s), (issued_v[s] >> 1) & 1, lim);
-                }
+            __syncwarp();
+            issued_v[s] = j;
+        }
+        if (*abort_flag) {  // let copies in flight land before the CTA exits
+            for (int s = 0; s < 2; ++s) {
+                if (issued_k[s] >= 0) wait_drain(BAR(B_KFULL + s), (issued_k[s] >> 1) & 1, lim);
+                if (issued_v[s] >= 0) wait_drain(BAR(B_VFULL + s), (issued_v[s] >> 1) & 1, lim);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
-            bool ok = mbar_wait(BAR(B_QFULL), 0, abort_flag, status, lim);
-            auto issue_pv = [&](int i) -> bool {
-                const int b = i & 1;
-                const uint32_t ph = (i >> 1) & 1;
-                if (!mbar_wait(BAR(B_PREADY + b), ph, abort_flag, status, lim)) return false;
-                if (!mbar_wait(BAR(B_VFULL + b), ph, abort_flag, status, lim)) return false;
-                fence_after_sync();
-                const uint32_t vbase = base + OFF_V + b * TILE_BYTES;
-                const uint32_t sb = tmem + (b ? TM_S1 : TM_S0);
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+        bool ok = __all_sync(FULL, mbar_wait(BAR(B_QFULL), 0, abort_flag, status, lim));
+        auto issue_pv = [&](int i) -> bool {
+            const int b = i & 1;
+            const uint32_t ph = (i >> 1) & 1;
+            if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY + b), ph, abort_flag, status, lim))) return false;
+            if (!__all_sync(FULL, mbar_wait(BAR(B_VFULL + b), ph, abort_flag, status, lim))) return false;
+            fence_after_sync();
+            const uint32_t vbase = base + OFF_V + b * TILE_BYTES;
+            const uint32_t sb = tmem + (b ? TM_S1 : TM_S0);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    bool s0, s1;
-                    half_sel(mrow, i, I, h, a.block, ragged1, s0, s1);
+            for (int h = 0; h < 2; ++h) {
+                bool s0, s1;
+                half_sel(mrow, i, I, h, a.block, ragged1, s0, s1);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        // V is MN-major: 64-wide column boxes LBO = 16 KB apart,
-                        // 8-key row groups SBO = 1 KB apart; 16 keys per MMA
-                        const uint64_t bd = smem_desc_sw128(vbase + (4 * h + kk) * 2048, HALF_BYTES, 1024);
-                        const uint32_t pa = sb + 32 * h + 8 * kk;
-                        if (s0 == s1) {
-                            mma_ts(tmem + (s0 ? TM_OSEL : TM_OUNS), pa, bd, idesc_pv, 1);
-                        } else {
-                            mma_ts(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
-                            mma_ts(tmem + TM_OUNS, pa + 64, bd, idesc_pv, 1);
-                        }
+                for (int kk = 0; kk < 4; ++kk) {
+                    // V is MN-major: 64-wide column boxes LBO = 16 KB apart,
+                    // 8-key row groups SBO = 1 KB apart; 16 keys per MMA
+                    const uint64_t bd = smem_desc_sw128(vbase + (4 * h + kk) * 2048, HALF_BYTES, 1024);
+                    // half h's P sits in the first 32 columns of its own S range,
+                    // the complementary ("alt") copy of a mixed half in the next 32
+                    const uint32_t pa = sb + 64 * h + 8 * kk;
+                    if (s0 == s1) {
+                        mma_ts_w(tmem + (s0 ? TM_OSEL : TM_OUNS), pa, bd, idesc_pv, 1);
+                    } else {
+                        mma_ts_w(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
+                        mma_ts_w(tmem + TM_OUNS, pa + 32, bd, idesc_pv, 1);
                     }
                 }
-                mma_commit(BAR(B_VEMPTY + b));
-                mma_commit(BAR(B_PVDONE));
-                return true;
-            };
-            for (int j = 0; ok && j < ntk; ++j) {
-                const int s = j & 1;
-                if (!mbar_wait(BAR(B_KFULL + s), (j >> 1) & 1, abort_flag, status, lim)) {
-                    ok = false;
-                    break;
-                }
-                fence_after_sync();
-                const uint32_t kbase = base + OFF_K + s * TILE_BYTES;
-                const uint32_t sd = tmem + (s ? TM_S1 : TM_S0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // K-major, 128B swizzle: 16 bf16 of d = 32 bytes per MMA step
-                    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-                    mma_ss(sd, smem_desc_sw128(base + OFF_Q + off, 16, 1024),
-                           smem_desc_sw128(kbase + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(BAR(B_SREADY + s));
-                mma_commit(BAR(B_KEMPTY + s));
-                if (j >= 1 && !issue_pv(j - 1)) ok = false;
             }
-            if (ok) issue_pv(ntk - 1);
-            mma_commit(BAR(B_DRAIN));  // all MMAs of this thread complete before teardown
-            wait_drain(BAR(B_DRAIN), 0, lim);
+            mma_commit_w(BAR(B_VEMPTY + b));
+            mma_commit_w(BAR(B_PVDONE));
+            return true;
+        };
+        for (int j = 0; ok && j < ntk; ++j) {
+            const int s = j & 1;
+            if (!__all_sync(FULL, mbar_wait(BAR(B_KFULL + s), (j >> 1) & 1, abort_flag, status, lim))) {
+                ok = false;
+                break;
+            }
+            fence_after_sync();
+            const uint32_t kbase = base + OFF_K + s * TILE_BYTES;
+            const uint32_t sd = tmem + (s ? TM_S1 : TM_S0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                // K-major, 128B swizzle: 16 bf16 of d = 32 bytes per MMA step
+                const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+                mma_ss_w(sd, smem_desc_sw128(base + OFF_Q + off, 16, 1024),
+                         smem_desc_sw128(kbase + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit_w(BAR(B_SREADY + s));
+            mma_commit_w(BAR(B_KEMPTY + s));
+            if (j >= 1 && !issue_pv(j - 1)) ok = false;
         }
+        if (ok) issue_pv(ntk - 1);
+        mma_commit_w(BAR(B_DRAIN));  // all MMAs of this warp complete before teardown
+        wait_drain(BAR(B_DRAIN), 0, lim);
     } else if (warp >= 4) {
-        // ------------------------------------------------ softmax warpgroup
-        const int sw = warp - 4;
+        // ------------------------------------------- two softmax warpgroups
+        // Warpgroup h (= wg) owns keys [64h, 64h+64) of every tile and the
+        // columns [64h, 64h+64) of O_sel / O_uns.  The row max is combined
+        // through shared memory once per tile; l_sel / l_uns and the squared
+        // difference are combined in the epilogue.
+        const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
         const int r = sw * 32 + lane;  // row of the tile == TMEM lane
-        const uint32_t lane_base = (uint32_t)(sw * 32) << 16;
-        const uint32_t trow = tmem + lane_base;
+        const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
+        const int c0 = 64 * wg;
+        float* xch = reinterpret_cast<float*>(gbase + OFF_XCH);  // [parity][wg][row]
+        // named barrier of the two warpgroups; wg_vote also ORs a flag across them so
+        // that both always leave the tile loop at the same tile (same barrier count)
+        auto wg_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+        auto wg_vote = [](bool flag) -> bool {
+            uint32_t out;
+            asm volatile(
+                "{\n\t.reg .pred p, q;\n\t"
+                "setp.ne.u32 q, %1, 0;\n\t"
+                "bar.red.or.pred p, 1, 256, q;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(out)
+                : "r"((uint32_t)flag)
+                : "memory");
+            return out != 0;
+        };
         {
             uint32_t z[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) z[i] = 0u;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                tmem_st32(trow + TM_OSEL + 32 * c, z);
-                tmem_st32(trow + TM_OUNS + 32 * c, z);
-            }
+            tmem_st32(trow + TM_OSEL + c0, z);
+            tmem_st32(trow + TM_OSEL + c0 + 32, z);
+            tmem_st32(trow + TM_OUNS + c0, z);
+            tmem_st32(trow + TM_OUNS + c0 + 32, z);
             tmem_wait_st();
         }
         const float sl2 = a.scale_log2;
@@ -280,49 +317,58 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int j = 0; j < ntk; ++j) {
             const int b = j & 1;
             // warp-uniform outcome: the TMEM loads below are warp-collective
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(BAR(B_SREADY + b), (j >> 1) & 1, abort_flag, status, lim))) {
-                ok = false;
-                break;
-            }
-            fence_after_sync();
-            const uint32_t sb = trow + (b ? TM_S1 : TM_S0);
-            float s[128];
-            {
-                uint32_t u0[32], u1[32], u2[32], u3[32];
+            const bool got = __all_sync(
+                0xffffffffu, mbar_wait(BAR(B_SREADY + b), (j >> 1) & 1, abort_flag, status, lim));
+            const uint32_t sb = trow + (b ? TM_S1 : TM_S0) + c0;
+            float s[64];
+            if (got) {
+                fence_after_sync();
+                uint32_t u0[32], u1[32];
                 tmem_ld32(sb, u0);
                 tmem_ld32(sb + 32, u1);
-                tmem_ld32(sb + 64, u2);
-                tmem_ld32(sb + 96, u3);
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     s[c] = __uint_as_float(u0[c]);
                     s[32 + c] = __uint_as_float(u1[c]);
-                    s[64 + c] = __uint_as_float(u2[c]);
-                    s[96 + c] = __uint_as_float(u3[c]);
                 }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) s[c] = 0.f;
             }
             if (j == I) {  // diagonal tile: keys after the row are masked (and keys >= T)
 #pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c > r) s[c] = -INFINITY;
+                for (int c = 0; c < 64; ++c)
+                    if (c0 + c > r) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            float mx8[8];  // independent partial maxima (short dependency chains)
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            for (int k = 0; k < 8; ++k) {
+                mx8[k] = max3(s[k], s[8 + k], s[16 + k]);
+                mx8[k] = max3(mx8[k], s[24 + k], s[32 + k]);
+                mx8[k] = max3(mx8[k], s[40 + k], s[48 + k]);
+                mx8[k] = fmaxf(mx8[k], s[56 + k]);
+            }
+            float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]),
+                            fmaxf(mx8[6], mx8[7]));
+            float* xm = xch + (j & 1) * 256;
+            xm[wg * 128 + r] = mx;
+            if (wg_vote(!got || *abort_flag)) {  // a wait expired somewhere: both leave here
+                ok = false;
+                break;
+            }
+            mx = fmaxf(mx, xm[(1 - wg) * 128 + r]);
             const float mnew = mx * sl2;
             if (j == 0) {
                 m2 = mnew;
             } else {
                 const bool need = mnew > m2 + kRescaleThreshold;
-                if (__any_sync(0xffffffffu, need)) {
-                    // PV_{j-1} must have landed in O before it is rescaled
-                    if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (j - 1) & 1, abort_flag,
-                                                           status, lim))) {
-                        ok = false;
-                        break;
-                    }
+                // PV_{j-1} must have landed in O before it is rescaled.  If that wait
+                // expires the rescale is skipped and the abort flag ends the loop at
+                // the next vote.
+                if (__any_sync(0xffffffffu, need) &&
+                    __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (j - 1) & 1, abort_flag,
+                                                      status, lim))) {
                     fence_after_sync();
                     const float mup = fmaxf(m2, mnew);
                     const float alpha = ex2(m2 - mup);
@@ -330,8 +376,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     lsel *= alpha;
                     luns *= alpha;
 #pragma unroll 1
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t col = (c < 4 ? TM_OSEL : TM_OUNS) + 32 * (c & 3);
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t col = (c < 2 ? TM_OSEL : TM_OUNS) + c0 + 32 * (c & 1);
                         uint32_t u[32];
                         tmem_ld32(trow + col, u);
                         tmem_wait_ld();
@@ -343,36 +389,61 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             const float negm = -m2;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                bool s0, s1;
-                half_sel(mrow, j, I, h, a.block, ragged1, s0, s1);
-                const bool mixed = s0 != s1;
-                const bool row_sel = mixed ? ((r < 64 || a.block == 128) ? s0 : s1) : s0;
-                float sum = 0.f;
-                uint32_t pk[32];
+            bool s0, s1;
+            half_sel(mrow, j, I, wg, a.block, ragged1, s0, s1);
+            const bool mixed = s0 != s1;
+            const bool row_sel = mixed ? ((r < 64 || a.block == 128) ? s0 : s1) : s0;
+            // p = 2^(s*sigma*log2e - m), two columns at a time (packed f32x2).  Off
+            // the diagonal a quarter of the pairs take the FMA-pipe exponential so
+            // that the MUFU unit is not the limit; on the diagonal every pair uses
+            // the MUFU, whose 2^-inf = 0 keeps masked keys exact.
+            const f32x2 sl2x2 = mk2(sl2, sl2), nm2 = mk2(negm, negm);
+            f32x2 acc[4] = {mk2(0.f, 0.f), mk2(0.f, 0.f), mk2(0.f, 0.f), mk2(0.f, 0.f)};
+            uint32_t pk[32];
+            if (j == I) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const float p0 = ex2(fmaf(s[64 * h + 2 * c], sl2, negm));
-                    const float p1 = ex2(fmaf(s[64 * h + 2 * c + 1], sl2, negm));
-                    sum += p0 + p1;
-                    pk[c] = pack_bf16(p0, p1);
+                    float x0, x1;
+                    un2(fma2(mk2(s[2 * c], s[2 * c + 1]), sl2x2, nm2), x0, x1);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    acc[c & 3] = add2(acc[c & 3], mk2(p0, p1));
+                    pk[c] = pack_bf16_alu(p0, p1);
                 }
-                if (!mixed) {
-                    tmem_st32(sb + 32 * h, pk);
-                } else {
-                    uint32_t main_[32], alt[32];
+            } else {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        main_[c] = row_sel ? pk[c] : 0u;
-                        alt[c] = row_sel ? 0u : pk[c];
+                for (int c = 0; c < 32; ++c) {
+                    const f32x2 x2 = fma2(mk2(s[2 * c], s[2 * c + 1]), sl2x2, nm2);
+                    float p0, p1;
+                    if ((c & 3) == kPolyLane) {
+                        un2(exp2_poly2(x2), p0, p1);
+                    } else {
+                        float x0, x1;
+                        un2(x2, x0, x1);
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
                     }
-                    tmem_st32(sb + 32 * h, main_);
-                    tmem_st32(sb + 64 + 32 * h, alt);
+                    acc[c & 3] = add2(acc[c & 3], mk2(p0, p1));
+                    pk[c] = pack_bf16_alu(p0, p1);
                 }
-                if (row_sel) lsel += sum;
-                else luns += sum;
             }
+            float a0, a1, b0, b1;
+            un2(add2(acc[0], acc[1]), a0, a1);
+            un2(add2(acc[2], acc[3]), b0, b1);
+            const float sum = (a0 + a1) + (b0 + b1);
+            if (!mixed) {
+                tmem_st32(sb, pk);
+            } else {
+                uint32_t main_[32], alt[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    main_[c] = row_sel ? pk[c] : 0u;
+                    alt[c] = row_sel ? 0u : pk[c];
+                }
+                tmem_st32(sb, main_);
+                tmem_st32(sb + 32, alt);
+            }
+            if (row_sel) lsel += sum;
+            else luns += sum;
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PREADY + b));
@@ -380,20 +451,28 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (ok)
             ok = __all_sync(0xffffffffu,
                             mbar_wait(BAR(B_PVDONE), (ntk - 1) & 1, abort_flag, status, lim));
+        // both warpgroups take the same decision and the same barriers below
+        ok = !wg_vote(!ok || *abort_flag);
+        float* xl = xch;  // [wg][sel|uns][row] reuses the max exchange area
+        xl[(wg * 2) * 128 + r] = lsel;
+        xl[(wg * 2 + 1) * 128 + r] = luns;
+        wg_sync();
+        const float Ls = lsel + xl[((1 - wg) * 2) * 128 + r];
+        const float Lu = luns + xl[((1 - wg) * 2 + 1) * 128 + r];
+        float sq = 0.f;
+        const int t = t0 + r;
+        const bool valid = t < a.T;
+        const size_t row = (size_t)bh * a.T + (valid ? t : 0);
         if (ok) {
             fence_after_sync();
-            const int t = t0 + r;
-            const bool valid = t < a.T;
-            const size_t row = (size_t)bh * a.T + (valid ? t : 0);
-            const float l = lsel + luns;
+            const float l = Ls + Lu;
             const float inv_l = 1.f / l;
-            const float inv_ls = lsel > 0.f ? 1.f / lsel : 0.f;
-            float sq = 0.f;
+            const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t os[32], ou[32];
-                tmem_ld32(trow + TM_OSEL + 32 * c, os);
-                tmem_ld32(trow + TM_OUNS + 32 * c, ou);
+                tmem_ld32(trow + TM_OSEL + c0 + 32 * c, os);
+                tmem_ld32(trow + TM_OUNS + c0 + 32 * c, ou);
                 tmem_wait_ld();
                 uint32_t hf[16], hs[16];
 #pragma unroll
@@ -408,8 +487,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     hs[e] = pack_bf16(pa, pb);
                 }
                 if (valid) {
-                    uint4* df = reinterpret_cast<uint4*>(a.h_full + row * HD + 32 * c);
-                    uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * HD + 32 * c);
+                    uint4* df = reinterpret_cast<uint4*>(a.h_full + row * HD + c0 + 32 * c);
+                    uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * HD + c0 + 32 * c);
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
                         df[v4] = make_uint4(hf[4 * v4], hf[4 * v4 + 1], hf[4 * v4 + 2], hf[4 * v4 + 3]);
@@ -417,12 +496,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     }
                 }
             }
-            if (valid) {
-                a.delta[row] = luns * inv_l;
-                a.lse_full[row] = (m2 + log2f(l)) * kLn2;
-                a.lse_sparse[row] = lsel > 0.f ? (m2 + log2f(lsel)) * kLn2 : -INFINITY;
-                a.sqdiff[row] = sq;
-            }
+        }
+        float* xs = xch + 512;  // [wg][row] squared-difference partials
+        xs[wg * 128 + r] = sq;
+        wg_sync();
+        if (ok && wg == 0 && valid) {
+            const float l = Ls + Lu;
+            a.delta[row] = Lu / l;
+            a.lse_full[row] = (m2 + log2f(l)) * kLn2;
+            a.lse_sparse[row] = Ls > 0.f ? (m2 + log2f(Ls)) * kLn2 : -INFINITY;
+            a.sqdiff[row] = sq + xs[128 + r];
         }
     }
 

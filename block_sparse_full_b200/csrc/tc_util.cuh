@@ -106,6 +106,20 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// One lane of a converged warp (elect.sync).  The producer and MMA roles run
+// their loops with the whole warp, so that descriptor and address arithmetic
+// stays warp-uniform, and let the elected lane issue each TMA / tcgen05
+// instruction.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\t"
+        "elect.sync rx|px, 0xffffffff;\n\t"
+        "@px mov.s32 %0, 1;\n\t}"
+        : "+r"(pred));
+    return pred != 0;
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T  (kind::f16, one CTA)
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
@@ -124,11 +138,24 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
+// Warp-converged forms: every lane calls, one elected lane issues.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    if (elect_one()) mma_ss(d_tmem, a_desc, b_desc, idesc, accumulate);
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    if (elect_one()) mma_ts(d_tmem, a_tmem, b_desc, idesc, accumulate);
+}
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
         : "memory");
+}
+
+__device__ __forceinline__ void mma_commit_w(uint32_t bar) {
+    if (elect_one()) mma_commit(bar);
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread i gets lane (base + i).
@@ -190,6 +217,73 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Two floats -> two bf16 in one register (lo in the low half) without the
+// conversion unit: add half an ulp of bf16 to each bit pattern (rounds the
+// magnitude half-up: differs from round-to-nearest-even only on exact ties)
+// and keep the high halves with one byte permute.  Integer ALU only.
+__device__ __forceinline__ uint32_t pack_bf16_alu(float lo, float hi) {
+    const uint32_t a = __float_as_uint(lo) + 0x8000u;
+    const uint32_t b = __float_as_uint(hi) + 0x8000u;
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// ---------------------------------------------------------------- packed f32x2
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 mk2(float a, float b) {
+    f32x2 v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(a), "f"(b));
+    return v;
+}
+__device__ __forceinline__ void un2(f32x2 v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe, for x in [-125, 127] (smaller x
+// are clamped to -125, giving ~2^-125 instead of 0).  Split x = j + r with
+// j = round(x) by the 1.5 * 2^23 shifter (Cody and Waite style range
+// reduction), |r| <= 1/2; 2^r by a degree-3 polynomial whose coefficients
+// were fitted here (minimax relative error on [-1/2, 1/2] by Lawson's
+// iteratively reweighted least squares; measured max relative error 7.5e-5 in
+// float32 Horner form); 2^j is added to the exponent field.
+__device__ __forceinline__ f32x2 exp2_poly2(f32x2 x) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    constexpr float C0 = 0.9999280571937561f, C1 = 0.6932609677314758f;
+    constexpr float C2 = 0.2426111251115799f, C3 = 0.0551716685295105f;
+    float x0, x1;
+    un2(x, x0, x1);
+    x = mk2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const f32x2 t = add2(x, mk2(kShift, kShift));         // low mantissa bits hold round(x)
+    const f32x2 j = add2(t, mk2(-kShift, -kShift));
+    const f32x2 r = fma2(j, mk2(-1.f, -1.f), x);          // x - round(x), exact
+    f32x2 p = fma2(mk2(C3, C3), r, mk2(C2, C2));
+    p = fma2(p, r, mk2(C1, C1));
+    p = fma2(p, r, mk2(C0, C0));
+    float p0, p1, t0, t1;
+    un2(p, p0, p1);
+    un2(t, t0, t1);
+    // bits(t) << 23 == round(x) << 23 (the shifter's own bits shift out)
+    p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+    return mk2(p0, p1);
 }
 
 }  // namespace tc

@@ -34,7 +34,7 @@ EXPORTS = (
     "ssa_workspace_size", "ssa_select_blocks", "ssa_select_blocks_noalloc",
     "ssa_attn_fwd_dual", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
-    "ssa_kernel_path", "ssa_version",
+    "ssa_kernel_path", "ssa_selftest_math", "ssa_version",
 )
 
 
@@ -73,6 +73,7 @@ _SIGNATURES = {
     "ssa_status_string": (ctypes.c_char_p, [c_int]),
     "ssa_last_error": (ctypes.c_char_p, []),
     "ssa_kernel_path": (c_int, [_P]),
+    "ssa_selftest_math": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "ssa_version": (c_int, []),
 }
 
@@ -144,6 +145,10 @@ def ssa_last_error():
 
 def ssa_kernel_path(params):
     return _lib.ssa_kernel_path(ctypes.byref(params))
+
+
+def ssa_selftest_math(x, n, exp2_poly, exp2_mufu, bf16_alu, stream):
+    return _lib.ssa_selftest_math(x, n, exp2_poly, exp2_mufu, bf16_alu, stream)
 
 
 def ssa_version():

@@ -200,6 +200,13 @@ const char* ssa_last_error(void);
  * tensor-core kernels (D = 128), -1 = invalid or unsupported params. */
 int ssa_kernel_path(const ssa_params_t* params);
 
+/* Self-test of the element-wise arithmetic inside the tensor-core kernels
+ * (not part of the method; for tests).  For n device floats x, writes the
+ * FMA-pipe polynomial 2^x, the MUFU 2^x and the bf16 bit patterns produced
+ * by the integer-ALU packing, each exactly as the kernels compute them. */
+int ssa_selftest_math(const float* x, int n, float* exp2_poly, float* exp2_mufu,
+                      uint16_t* bf16_alu, void* stream);
+
 /* ABI version, (major << 16) | minor. */
 int ssa_version(void);
 
