@@ -90,30 +90,10 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
-// K-major SW128 operand of R rows x 128 d (two 64-column boxes of R*128
-// bytes): descriptor of MMA k-step kk (16 d per step).
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, uint32_t box_bytes, int kk) {
-    return smem_desc_sw128(base + (kk >> 2) * box_bytes + (kk & 3) * 32, 16, 1024);
-}
-// The same tile read as an MN-major B operand (N = d): k-step kk covers 16
-// rows (2 swizzle atoms of 8 rows); the two d-halves are box_bytes apart.
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, uint32_t box_bytes, int kk) {
-    return smem_desc_sw128(base + kk * 2048, box_bytes, 1024);
-}
-
 // bf16 A operand of 64 K-columns written as two 32-wide halves, each half at
 // the start of its own 32-column fp32 source range: k-step kk (16 columns).
 __device__ __forceinline__ uint32_t split_acol(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-        "%11, %12, %13, %14, %15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
@@ -318,38 +298,48 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] >> 1) & 1, lim);
     } else if (warp == 1) {
         {  // ------------------------------------------ MMA issuer (whole warp)
+            // descriptors formed once, advanced by constant offsets; each MMA group
+            // and its commits are issued by one elected lane
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S^T, dP^T
             constexpr uint32_t id_a = idesc_bf16_f32(TILE, HD, true);     // dV, dK
+            const uint64_t kdesc = smem_desc_sw128(base + OFF_K, 16, 1024);
+            const uint64_t vdesc = smem_desc_sw128(base + OFF_V, 16, 1024);
+            const uint64_t st_k0 = smem_desc_sw128(base + OFF_STAGE, 16, 1024);      // K-major
+            const uint64_t st_m0 = smem_desc_sw128(base + OFF_STAGE, BOX_S, 1024);   // MN-major
+            auto kq = [](int kk) { return (uint32_t)((kk >> 2) * BOX_T + (kk & 3) * 32); };
+            auto ks = [](int kk) { return (uint32_t)((kk >> 2) * BOX_S + (kk & 3) * 32); };
             bool ok = __all_sync(FULL, mbar_wait(BAR(B_KV), 0, abort_flag, status, lim));
             auto sparse = [&](int i) { return selb[step_qb(i)] != 0; };
-            auto issue_s = [&](int i) {
-                const uint32_t st = base + OFF_STAGE + (i & 1) * STAGE_BYTES;
+            auto issue_s = [&](int i) {  // elected lane only
+                const uint64_t qd = desc_add(st_k0, (i & 1) * STAGE_BYTES + ST_Q);
                 const uint32_t d = tmem + ((i & 1) ? TM_S1 : TM_S0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss_w(d, kmajor_desc(base + OFF_K, BOX_T, kk), kmajor_desc(st + ST_Q, BOX_S, kk),
-                           id_s, kk > 0);
+                    mma_ss(d, desc_add(kdesc, kq(kk)), desc_add(qd, ks(kk)), id_s, kk > 0);
             };
-            auto issue_dp = [&](int i) {
-                const uint32_t st = base + OFF_STAGE + (i & 1) * STAGE_BYTES;
+            auto issue_dp = [&](int i, bool sp) {  // elected lane only
+                const uint64_t gfd = desc_add(st_k0, (i & 1) * STAGE_BYTES + ST_GF);
+                const uint64_t gsd = desc_add(st_k0, (i & 1) * STAGE_BYTES + ST_GS);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_ss_w(tmem + TM_DPF, kmajor_desc(base + OFF_V, BOX_T, kk),
-                           kmajor_desc(st + ST_GF, BOX_S, kk), id_s, kk > 0);
-                if (sparse(i)) {
+                    mma_ss(tmem + TM_DPF, desc_add(vdesc, kq(kk)), desc_add(gfd, ks(kk)), id_s, kk > 0);
+                if (sp) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss_w(tmem + TM_DPS, kmajor_desc(base + OFF_V, BOX_T, kk),
-                               kmajor_desc(st + ST_GS, BOX_S, kk), id_s, kk > 0);
+                        mma_ss(tmem + TM_DPS, desc_add(vdesc, kq(kk)), desc_add(gsd, ks(kk)), id_s, kk > 0);
                 }
             };
             if (ok && ns > 0) {
                 ok = __all_sync(FULL, mbar_wait(BAR(B_FULL), 0, abort_flag, status, lim));
                 if (ok) {
                     fence_after_sync();
-                    issue_s(0);
-                    issue_dp(0);
-                    mma_commit_w(BAR(B_READY));
+                    const bool sp0 = sparse(0);
+                    if (elect_one()) {
+                        issue_s(0);
+                        issue_dp(0, sp0);
+                        mma_commit(BAR(B_READY));
+                    }
+                    __syncwarp();
                 }
             }
             for (int i = 0; ok && i < ns; ++i) {
@@ -361,37 +351,48 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         break;
                     }
                     fence_after_sync();
-                    issue_s(i + 1);
+                    if (elect_one()) issue_s(i + 1);
+                    __syncwarp();
                 }
                 if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY), i & 1, abort_flag, status, lim))) {
                     ok = false;
                     break;
                 }
                 fence_after_sync();
-                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
                 const uint32_t sb = tmem + (s ? TM_S1 : TM_S0);
+                const uint64_t gfm = desc_add(st_m0, s * STAGE_BYTES + ST_GF);
+                const uint64_t gsm = desc_add(st_m0, s * STAGE_BYTES + ST_GS);
+                const uint64_t qm = desc_add(st_m0, s * STAGE_BYTES + ST_Q);
+                const bool sp = sparse(i);
+                const bool sp_next = i + 1 < ns && sparse(i + 1);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // dV += P_f^T G_f
-                    mma_ts_w(tmem + TM_DV, sb + split_acol(kk), mnmajor_desc(st + ST_GF, BOX_S, kk), id_a,
-                           (i > 0 || kk > 0) ? 1u : 0u);
-                if (sparse(i)) {
+                    for (int kk = 0; kk < 4; ++kk)  // dV += P_f^T G_f
+                        mma_ts(tmem + TM_DV, sb + split_acol(kk), desc_add(gfm, kk * 2048), id_a,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                    if (sp) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // dV += P_s^T G_s
-                        mma_ts_w(tmem + TM_DV, tmem + TM_DPS + split_acol(kk),
-                               mnmajor_desc(st + ST_GS, BOX_S, kk), id_a, 1u);
+                        for (int kk = 0; kk < 4; ++kk)  // dV += P_s^T G_s
+                            mma_ts(tmem + TM_DV, tmem + TM_DPS + split_acol(kk), desc_add(gsm, kk * 2048),
+                                   id_a, 1u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
+                        mma_ts(tmem + TM_DK, tmem + TM_DPF + split_acol(kk), desc_add(qm, kk * 2048), id_a,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(BAR(B_EMPTY + s));
+                    if (i + 1 < ns) {
+                        issue_dp(i + 1, sp_next);
+                        mma_commit(BAR(B_READY));
+                    }
                 }
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-                    mma_ts_w(tmem + TM_DK, tmem + TM_DPF + split_acol(kk), mnmajor_desc(st + ST_Q, BOX_S, kk),
-                           id_a, (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit_w(BAR(B_EMPTY + s));
-                if (i + 1 < ns) {
-                    issue_dp(i + 1);
-                    mma_commit_w(BAR(B_READY));
-                }
+                __syncwarp();
             }
-            mma_commit_w(BAR(B_DONE));
-            mma_commit_w(BAR(B_DRAIN));
+            if (elect_one()) {
+                mma_commit(BAR(B_DONE));
+                mma_commit(BAR(B_DRAIN));
+            }
+            __syncwarp();
             wait_drain(BAR(B_DRAIN), 0, lim);
         }
     } else if (warp >= 4) {
@@ -615,30 +616,39 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         {  // ------------------------------------------ MMA issuer (whole warp)
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S, dP
             constexpr uint32_t id_q = idesc_bf16_f32(TILE, HD, true);     // dQ
+            const uint64_t qdesc = smem_desc_sw128(base + OFF_Q, 16, 1024);
+            const uint64_t gfdesc = smem_desc_sw128(base + OFF_GF, 16, 1024);
+            const uint64_t gsdesc = smem_desc_sw128(base + OFF_GS, 16, 1024);
+            const uint64_t st_k0 = smem_desc_sw128(base + OFF_STAGE, 16, 1024);      // K-major
+            const uint64_t st_m0 = smem_desc_sw128(base + OFF_STAGE, BOX_S, 1024);   // MN-major
+            auto kt = [](int kk) { return (uint32_t)((kk >> 2) * BOX_T + (kk & 3) * 32); };
+            auto ks = [](int kk) { return (uint32_t)((kk >> 2) * BOX_S + (kk & 3) * 32); };
             bool ok = __all_sync(FULL, mbar_wait(BAR(B_QG), 0, abort_flag, status, lim));
             auto issue_front = [&](int i) -> bool {  // S_i, dP_f_i, dP_s_i
                 const int s = i % NSTAGE, b = i & 1;
                 if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + s), (i / NSTAGE) & 1, abort_flag, status, lim)))
                     return false;
                 fence_after_sync();
-                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                const uint64_t kd = desc_add(st_k0, s * STAGE_BYTES + ST_K);
+                const uint64_t vd = desc_add(st_k0, s * STAGE_BYTES + ST_V);
                 const uint32_t sd = tmem + (b ? TM_S1 : TM_S0);
                 const uint32_t dp = tmem + (b ? TM_DP1 : TM_DP0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss_w(sd, kmajor_desc(base + OFF_Q, BOX_T, kk), kmajor_desc(st + ST_K, BOX_S, kk),
-                           id_s, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss_w(dp, kmajor_desc(base + OFF_GF, BOX_T, kk), kmajor_desc(st + ST_V, BOX_S, kk),
-                           id_s, kk > 0);
-                if (sparse(i)) {
+                const bool sp = sparse(i);
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss_w(dp + 64, kmajor_desc(base + OFF_GS, BOX_T, kk),
-                               kmajor_desc(st + ST_V, BOX_S, kk), id_s, kk > 0);
+                        mma_ss(sd, desc_add(qdesc, kt(kk)), desc_add(kd, ks(kk)), id_s, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ss(dp, desc_add(gfdesc, kt(kk)), desc_add(vd, ks(kk)), id_s, kk > 0);
+                    if (sp) {
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_ss(dp + 64, desc_add(gsdesc, kt(kk)), desc_add(vd, ks(kk)), id_s, kk > 0);
+                    }
+                    mma_commit(BAR(B_READY + b));
                 }
-                mma_commit_w(BAR(B_READY + b));
+                __syncwarp();
                 return true;
             };
             for (int i = 0; ok && i < ns && i < 2; ++i) ok = issue_front(i);
@@ -649,17 +659,23 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     break;
                 }
                 fence_after_sync();
-                const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
+                const uint64_t km = desc_add(st_m0, s * STAGE_BYTES + ST_K);
                 const uint32_t sd = tmem + (b ? TM_S1 : TM_S0);
+                if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)  // dQ += dS K
-                    mma_ts_w(tmem + TM_DQ, sd + split_acol(kk), mnmajor_desc(st + ST_K, BOX_S, kk), id_q,
-                           (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit_w(BAR(B_EMPTY + s));
+                    for (int kk = 0; kk < 4; ++kk)  // dQ += dS K
+                        mma_ts(tmem + TM_DQ, sd + split_acol(kk), desc_add(km, kk * 2048), id_q,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(BAR(B_EMPTY + s));
+                }
+                __syncwarp();
                 if (i + 2 < ns && !issue_front(i + 2)) ok = false;
             }
-            mma_commit_w(BAR(B_DONE));
-            mma_commit_w(BAR(B_DRAIN));
+            if (elect_one()) {
+                mma_commit(BAR(B_DONE));
+                mma_commit(BAR(B_DRAIN));
+            }
+            __syncwarp();
             wait_drain(BAR(B_DRAIN), 0, lim);
         }
     } else if (warp >= 4) {

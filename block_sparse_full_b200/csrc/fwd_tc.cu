@@ -217,8 +217,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
+        // Descriptors are formed once and advanced by constant offsets; each group
+        // of MMAs (and its commits) is issued by one elected lane.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+        const uint64_t qdesc = smem_desc_sw128(base + OFF_Q, 16, 1024);          // K-major Q
+        const uint64_t kdesc0 = smem_desc_sw128(base + OFF_K, 16, 1024);         // K-major K
+        // V is MN-major: 64-wide column boxes LBO = 16 KB apart, 8-key row groups
+        // SBO = 1 KB apart; 16 keys (2 KB) per MMA
+        const uint64_t vdesc0 = smem_desc_sw128(base + OFF_V, HALF_BYTES, 1024);
         bool ok = __all_sync(FULL, mbar_wait(BAR(B_QFULL), 0, abort_flag, status, lim));
         auto issue_pv = [&](int i) -> bool {
             const int b = i & 1;
@@ -226,30 +233,32 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY + b), ph, abort_flag, status, lim))) return false;
             if (!__all_sync(FULL, mbar_wait(BAR(B_VFULL + b), ph, abort_flag, status, lim))) return false;
             fence_after_sync();
-            const uint32_t vbase = base + OFF_V + b * TILE_BYTES;
+            const uint64_t vd = desc_add(vdesc0, b * TILE_BYTES);
             const uint32_t sb = tmem + (b ? TM_S1 : TM_S0);
+            bool s0[2], s1[2];
+            half_sel(mrow, i, I, 0, a.block, ragged1, s0[0], s1[0]);
+            half_sel(mrow, i, I, 1, a.block, ragged1, s0[1], s1[1]);
+            if (elect_one()) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                bool s0, s1;
-                half_sel(mrow, i, I, h, a.block, ragged1, s0, s1);
+                for (int h = 0; h < 2; ++h) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    // V is MN-major: 64-wide column boxes LBO = 16 KB apart,
-                    // 8-key row groups SBO = 1 KB apart; 16 keys per MMA
-                    const uint64_t bd = smem_desc_sw128(vbase + (4 * h + kk) * 2048, HALF_BYTES, 1024);
-                    // half h's P sits in the first 32 columns of its own S range,
-                    // the complementary ("alt") copy of a mixed half in the next 32
-                    const uint32_t pa = sb + 64 * h + 8 * kk;
-                    if (s0 == s1) {
-                        mma_ts_w(tmem + (s0 ? TM_OSEL : TM_OUNS), pa, bd, idesc_pv, 1);
-                    } else {
-                        mma_ts_w(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
-                        mma_ts_w(tmem + TM_OUNS, pa + 32, bd, idesc_pv, 1);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t bd = desc_add(vd, (4 * h + kk) * 2048);
+                        // half h's P sits in the first 32 columns of its own S range,
+                        // the complementary ("alt") copy of a mixed half in the next 32
+                        const uint32_t pa = sb + 64 * h + 8 * kk;
+                        if (s0[h] == s1[h]) {
+                            mma_ts(tmem + (s0[h] ? TM_OSEL : TM_OUNS), pa, bd, idesc_pv, 1);
+                        } else {
+                            mma_ts(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
+                            mma_ts(tmem + TM_OUNS, pa + 32, bd, idesc_pv, 1);
+                        }
                     }
                 }
+                mma_commit(BAR(B_VEMPTY + b));
+                mma_commit(BAR(B_PVDONE));
             }
-            mma_commit_w(BAR(B_VEMPTY + b));
-            mma_commit_w(BAR(B_PVDONE));
+            __syncwarp();
             return true;
         };
         for (int j = 0; ok && j < ntk; ++j) {
@@ -259,21 +268,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 break;
             }
             fence_after_sync();
-            const uint32_t kbase = base + OFF_K + s * TILE_BYTES;
+            const uint64_t kd = desc_add(kdesc0, s * TILE_BYTES);
             const uint32_t sd = tmem + (s ? TM_S1 : TM_S0);
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                // K-major, 128B swizzle: 16 bf16 of d = 32 bytes per MMA step
-                const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-                mma_ss_w(sd, smem_desc_sw128(base + OFF_Q + off, 16, 1024),
-                         smem_desc_sw128(kbase + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < 8; ++kk) {
+                    // K-major, 128B swizzle: 16 bf16 of d = 32 bytes per MMA step
+                    const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+                    mma_ss(sd, desc_add(qdesc, off), desc_add(kd, off), idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(BAR(B_SREADY + s));
+                mma_commit(BAR(B_KEMPTY + s));
             }
-            mma_commit_w(BAR(B_SREADY + s));
-            mma_commit_w(BAR(B_KEMPTY + s));
+            __syncwarp();
             if (j >= 1 && !issue_pv(j - 1)) ok = false;
         }
         if (ok) issue_pv(ntk - 1);
-        mma_commit_w(BAR(B_DRAIN));  // all MMAs of this warp complete before teardown
+        if (elect_one()) mma_commit(BAR(B_DRAIN));  // all MMAs complete before teardown
+        __syncwarp();
         wait_drain(BAR(B_DRAIN), 0, lim);
     } else if (warp >= 4) {
         // ------------------------------------------- two softmax warpgroups

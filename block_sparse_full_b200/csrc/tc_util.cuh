@@ -197,6 +197,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
+// A descriptor advanced by `bytes` (a multiple of 16): the start address is
+// the low field, and shared-memory addresses stay below 2^18, so the add never
+// carries out of it.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+    return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor of kind::f16: bf16 A and B, f32 accumulator.
 // b_mn_major: B stored MN-major (N contiguous) instead of K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
