@@ -257,7 +257,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
     total_ms = sum(step_ms)
     max_ms = reduce_max(total_ms, world, dev)
     ms_per_step = max_ms / args.steps
-    value = (f_fwd + f_bwd) * world / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tflops(f_fwd + f_bwd, world, ms_per_step)
 
     # dominant ABI call and its roofline
     avg = {n: per_call[n] / args.steps for n in names}
@@ -336,7 +336,7 @@ def run_e2e(args, layer, inp, grads, flops, world, dev):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms = reduce_max(e0.elapsed_time(e1), world, dev) / args.steps
-    return {"value": round(flops * world / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+    return {"value": round(whole_job_tflops(flops, world, ms), 3), "unit": "TFLOP/s",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": loss_h.numel() * loss_h.element_size()}
 
@@ -426,11 +426,18 @@ def barrier(world):
 
 
 def reduce_max(x, world, dev):
+    """Max of a per-rank value over all ranks (device time: the slowest rank)."""
     if world == 1:
         return x
     t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step, world, max_ms_per_step):
+    """Throughput of the whole job: every rank processes its own copy of the
+    workload, so units scale with the rank count; time is the slowest rank's."""
+    return flops_per_rank_step * world / (max_ms_per_step * 1e-3) / 1e12
 
 
 def main(argv=None):

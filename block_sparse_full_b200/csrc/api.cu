@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/ssa.h: argument validation,
 // workspace sizing, kernel-path choice and status reporting.  Every compute
 // step runs in the kernels of the sibling .cu files.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -12,6 +13,8 @@ namespace ssa {
 
 namespace {
 thread_local char g_last_error[512] = "";
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -74,6 +77,8 @@ size_t bwd_workspace(const ssa_params_t& p) {
 }
 
 }  // namespace
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 int fail(int status, const char* fmt, ...) {
     va_list ap;
@@ -206,6 +211,7 @@ int ssa_device_status(void* stream) {
     if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
     int st = fwd_tc_take_status(s);
     if (st == SSA_OK) st = bwd_tc_take_status(s);
+    if (st == SSA_OK) st = selftest_take_status();
     if (st != SSA_OK) return st;
     return check_launch("pending");
 }
@@ -230,5 +236,9 @@ int ssa_kernel_path(const ssa_params_t* p) {
 }
 
 int ssa_version(void) { return (1 << 16) | 0; }
+
+void ssa_debug_set_wait_limit_ns(unsigned long long ns) {
+    g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs, std::memory_order_relaxed);
+}
 
 }  // extern "C"

@@ -292,10 +292,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             __syncwarp();
             issued[s] = i;
         }
-        wait_drain(BAR(B_KV), 0, lim);
+        wait_drain(BAR(B_KV), 0, kDrainLimitNs);
         if (*abort_flag)
             for (int s = 0; s < 2; ++s)
-                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] >> 1) & 1, lim);
+                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] >> 1) & 1, kDrainLimitNs);
     } else if (warp == 1) {
         {  // ------------------------------------------ MMA issuer (whole warp)
             // descriptors formed once, advanced by constant offsets; each MMA group
@@ -393,7 +393,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 mma_commit(BAR(B_DRAIN));
             }
             __syncwarp();
-            wait_drain(BAR(B_DRAIN), 0, lim);
+            wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
         }
     } else if (warp >= 4) {
         // ------------------------------------------ two compute warpgroups
@@ -608,10 +608,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncwarp();
             issued[s] = i;
         }
-        wait_drain(BAR(B_QG), 0, lim);
+        wait_drain(BAR(B_QG), 0, kDrainLimitNs);
         if (*abort_flag)
             for (int s = 0; s < NSTAGE; ++s)
-                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, lim);
+                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
     } else if (warp == 1) {
         {  // ------------------------------------------ MMA issuer (whole warp)
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S, dP
@@ -676,7 +676,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mma_commit(BAR(B_DRAIN));
             }
             __syncwarp();
-            wait_drain(BAR(B_DRAIN), 0, lim);
+            wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
         }
     } else if (warp >= 4) {
         // ------------------------------------------ two compute warpgroups
@@ -862,7 +862,7 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     a.n_blocks = num_blocks(p);
     a.scale_log2 = p.sm_scale * kLog2e;
     a.sm_scale = p.sm_scale;
-    a.timeout_ns = 2000000000ull;
+    a.timeout_ns = wait_limit_ns();
     const unsigned grid = (unsigned)((size_t)BH * ((p.T + TILE - 1) / TILE));
     bwd_dkdv_tc_kernel<<<grid, kThreads, kv::SMEM_BYTES, s>>>(k128, v128, q64, gf64, gs64, a);
     st = check_launch("bwd_dkdv_tc_kernel");

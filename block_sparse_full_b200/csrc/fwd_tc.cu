@@ -211,8 +211,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         if (*abort_flag) {  // let copies in flight land before the CTA exits
             for (int s = 0; s < 2; ++s) {
-                if (issued_k[s] >= 0) wait_drain(BAR(B_KFULL + s), (issued_k[s] >> 1) & 1, lim);
-                if (issued_v[s] >= 0) wait_drain(BAR(B_VFULL + s), (issued_v[s] >> 1) & 1, lim);
+                if (issued_k[s] >= 0) wait_drain(BAR(B_KFULL + s), (issued_k[s] >> 1) & 1, kDrainLimitNs);
+                if (issued_v[s] >= 0) wait_drain(BAR(B_VFULL + s), (issued_v[s] >> 1) & 1, kDrainLimitNs);
             }
         }
     } else if (warp == 1) {
@@ -286,7 +286,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         if (ok) issue_pv(ntk - 1);
         if (elect_one()) mma_commit(BAR(B_DRAIN));  // all MMAs complete before teardown
         __syncwarp();
-        wait_drain(BAR(B_DRAIN), 0, lim);
+        wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
     } else if (warp >= 4) {
         // ------------------------------------------- two softmax warpgroups
         // Warpgroup h (= wg) owns keys [64h, 64h+64) of every tile and the
@@ -600,7 +600,7 @@ int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     a.words = mask_words(p);
     a.n_blocks = num_blocks(p);
     a.scale_log2 = p.sm_scale * 1.4426950408889634f;
-    a.timeout_ns = 2000000000ull;
+    a.timeout_ns = wait_limit_ns();
     const unsigned grid = (unsigned)((size_t)BH * ((p.T + BM - 1) / BM));
     fwd_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, a);
     return check_launch("fwd_tc_kernel");

@@ -26,8 +26,44 @@ __global__ void selftest_kernel(const float* __restrict__ x, int n, float* __res
     }
 }
 
+__device__ unsigned int g_selftest_status;
+
+// One thread waits, with the kernels' bounded wait, on an mbarrier that no
+// one ever arrives at: the wait must give up after `limit_ns` and record the
+// expiry in this file's device status word.
+__global__ void wait_timeout_kernel(unsigned long long limit_ns, int* __restrict__ gave_up) {
+    __shared__ __align__(8) unsigned long long bar;
+    __shared__ int abort_flag;
+    const uint32_t b = tc::smem_u32(&bar);
+    tc::mbar_init(b, 1);
+    tc::fence_mbar_init();
+    abort_flag = 0;
+    const bool ok = tc::mbar_wait(b, 0, &abort_flag, &g_selftest_status, limit_ns);
+    *gave_up = ok ? 0 : 1;
+}
+
 }  // namespace
+
+int selftest_take_status() {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_selftest_status, sizeof v);
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (v) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_selftest_status, &zero, sizeof zero);
+        return fail(SSA_ERR_TIMEOUT, "self-test: a bounded mbarrier wait expired");
+    }
+    return SSA_OK;
+}
+
 }  // namespace ssa
+
+extern "C" int ssa_selftest_wait_timeout(unsigned long long limit_ns, int* gave_up, void* stream) {
+    if (!gave_up || limit_ns == 0 || limit_ns > 10000000000ull)
+        return ssa::fail(SSA_ERR_INVALID_ARG, "ssa_selftest_wait_timeout: bad arguments");
+    ssa::wait_timeout_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, gave_up);
+    return ssa::check_launch("wait_timeout_kernel");
+}
 
 extern "C" int ssa_selftest_math(const float* x, int n, float* exp2_poly, float* exp2_mufu,
                                  uint16_t* bf16_alu, void* stream) {

@@ -19,6 +19,9 @@ int check_launch(const char* what);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Wall-clock limit of the kernels' bounded waits (default 2 s; tests shorten it).
+unsigned long long wait_limit_ns();
+
 inline size_t num_rows(const ssa_params_t& p) {
     return (size_t)p.B * p.H * p.T;
 }
@@ -67,5 +70,8 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
                   const void* dh_sparse, float w_s, float w_c, void* dq, void* dk, void* dv,
                   void* ws, cudaStream_t s);
 int bwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
+
+// ---- self-tests (selftest.cu)
+int selftest_take_status();  // SSA_ERR_TIMEOUT if the self-test wait expired
 
 }  // namespace ssa

@@ -48,26 +48,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase of parity `parity` to complete.  Gives up after
 // `limit_ns` of wall time, or as soon as *abort is set by another role;
 // on a timeout it sets *abort and ORs 1 into *status.  Returns false if it
-// gave up.
+// gave up.  After the first try each try sleeps at most min(limit, 1 ms).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           unsigned int* status, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;  // fast path: the phase is (nearly) done
+    const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
     const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0) {
-            if (*abort) return false;
-            if (globaltimer() - t0 > limit_ns) {
-                *abort = 1;
-                atomicOr(status, 1u);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_ns(bar, parity, hint)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > limit_ns) {
+            *abort = 1;
+            atomicOr(status, 1u);
+            return false;
         }
     }
 }
+
+// Limit for the teardown waits (copies and MMAs in flight must land before a
+// CTA frees its TMEM and exits); independent of the configurable wait limit.
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,

@@ -34,7 +34,8 @@ EXPORTS = (
     "ssa_workspace_size", "ssa_select_blocks", "ssa_select_blocks_noalloc",
     "ssa_attn_fwd_dual", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
-    "ssa_kernel_path", "ssa_selftest_math", "ssa_version",
+    "ssa_kernel_path", "ssa_selftest_math", "ssa_selftest_wait_timeout",
+    "ssa_debug_set_wait_limit_ns", "ssa_version",
 )
 
 
@@ -75,6 +76,8 @@ _SIGNATURES = {
     "ssa_kernel_path": (c_int, [_P]),
     "ssa_selftest_math": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "ssa_version": (c_int, []),
+    "ssa_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
+    "ssa_selftest_wait_timeout": (c_int, [ctypes.c_ulonglong, c_void_p, c_void_p]),
 }
 
 
@@ -149,6 +152,14 @@ def ssa_kernel_path(params):
 
 def ssa_selftest_math(x, n, exp2_poly, exp2_mufu, bf16_alu, stream):
     return _lib.ssa_selftest_math(x, n, exp2_poly, exp2_mufu, bf16_alu, stream)
+
+
+def ssa_selftest_wait_timeout(limit_ns, gave_up, stream):
+    return _lib.ssa_selftest_wait_timeout(limit_ns, gave_up, stream)
+
+
+def ssa_debug_set_wait_limit_ns(ns):
+    _lib.ssa_debug_set_wait_limit_ns(ns)
 
 
 def ssa_version():

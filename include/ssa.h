@@ -207,6 +207,21 @@ int ssa_kernel_path(const ssa_params_t* params);
 int ssa_selftest_math(const float* x, int n, float* exp2_poly, float* exp2_mufu,
                       uint16_t* bf16_alu, void* stream);
 
+/* Self-test of the bounded wait the tensor-core kernels use for every
+ * mbarrier (not part of the method; for tests): one thread waits on an
+ * mbarrier that nothing ever arrives at.  The wait gives up after limit_ns
+ * (1 ns .. 10 s), *gave_up (device int) is set to 1 and the expiry is
+ * recorded, so the next ssa_device_status returns SSA_ERR_TIMEOUT. */
+int ssa_selftest_wait_timeout(unsigned long long limit_ns, int* gave_up, void* stream);
+
+/* Test hook: wall-clock limit of every bounded wait inside the tensor-core
+ * kernels, in nanoseconds, for launches made after the call (0 restores the
+ * default of 2 s).  A wait that runs past it makes the kernel stop, let
+ * copies and MMAs in flight land, free TMEM and return; ssa_device_status
+ * then reports SSA_ERR_TIMEOUT and the outputs of that call are undefined.
+ * Process-wide; not synchronised with calls running on other threads. */
+void ssa_debug_set_wait_limit_ns(unsigned long long ns);
+
 /* ABI version, (major << 16) | minor. */
 int ssa_version(void);
 
