@@ -11,19 +11,24 @@
 //   dv_s = sum_t P_f G_f(t) + P_s G_s(t),  dk_s = sigma sum_t dS q_t,
 //   dq_t = sigma sum_s dS k_s,
 // where G_f, G_s are the upstream gradients of h_full, h_sparse plus the
-// alignment terms and D_f = G_f.h_full, D_s = G_s.h_sparse.
+// alignment terms and D_f = G_f.h_full, D_s = G_s.h_sparse.  Since P_s = c_t P_f
+// on selected pairs, the kernels use G_s' = c_t G_s and D_s' = c_t D_s:
+//   dS = P_f (G_f.v - D_f + sel (G_s'.v - D_s')),  dv_s += P_f (G_f + sel G_s'),
+// so c_t never appears past the preprocess and P_s^T is P_f^T with the
+// unselected key rows zeroed.
 //
 // Three kernels, no atomics (bitwise repeatable):
-//   bwd_tc_pre_kernel   one warp per row: G_f, G_s rounded to bf16, D_f and
-//                       D_s from the rounded values, lse_full*log2(e), c_t.
+//   bwd_tc_pre_kernel   one warp per row: G_f, G_s' rounded to bf16, D_f and
+//                       D_s' from the rounded values, lse_full*log2(e).
 //   bwd_dkdv_tc_kernel  CTA = 128 keys; steps of 64 queries.  Per step:
-//                       S^T = K Q^T, dP_f^T = V G_f^T, dP_s^T = V G_s^T
-//                       (tcgen05 SS, N = 64), the compute warpgroup forms
-//                       P_f^T, P_s^T, dS^T (bf16, written back to TMEM), then
-//                       dV += P_f^T G_f + P_s^T G_s and dK += dS^T Q (TS).
+//                       S^T = K Q^T, dP_f^T = V G_f^T, dP_s^T = V G_s'^T
+//                       (tcgen05 SS, N = 64), the compute warpgroups form
+//                       P_f^T (bf16, back to TMEM) and dS^T (bf16, to a
+//                       swizzled shared-memory tile), then
+//                       dV += P_f^T G_f + P_s^T G_s' (TS) and dK += dS^T Q (SS).
 //                       TMEM: dV | dK | S^T x2 | dP_f^T | dP_s^T = 512 cols.
 //   bwd_dq_tc_kernel    CTA = 128 queries; steps of 64 keys: S = Q K^T,
-//                       dP_f = G_f V^T, dP_s = G_s V^T, dS, dQ += dS K.
+//                       dP_f = G_f V^T, dP_s = G_s' V^T, dS, dQ += dS K.
 //                       TMEM: dQ | S x2 | (dP_f, dP_s) x2 = 512 cols.
 // The sparse-stream MMAs are skipped on steps where no (query block, key
 // block) pair is selected.  Every wait is bounded; an expiry sets a device
@@ -46,7 +51,7 @@ constexpr int TILE = 128;  // keys per dK/dV CTA, queries per dQ CTA
 constexpr int STEP = 64;   // queries per dK/dV step, keys per dQ step
 constexpr int kThreads = 384;  // warps 0-1 roles, 2-3 idle, 4-11 two compute warpgroups
 constexpr int kCompute = 256;
-constexpr int kMaxWords = 256;
+constexpr int kMaxWords = 128;  // mask words per query block: n <= 4096 blocks
 constexpr int kMaxBlocks = kMaxWords * 32;
 constexpr uint32_t BOX_T = TILE * 128;  // [128 rows x 64 d] bf16 = 16 KB
 constexpr uint32_t BOX_S = STEP * 128;  // [64 rows x 64 d] bf16 = 8 KB
@@ -61,9 +66,8 @@ struct BwdArgs {
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     const float* lse2;  // lse_full * log2(e)
-    const float* cfac;  // exp(lse_full - lse_sparse), 0 where the sparse mass is 0
     const float* Df;
-    const float* Ds;
+    const float* Ds;    // D_s of the c_t-scaled G_s
     const uint32_t* mask;
     int BH, T, block, words, n_blocks;
     float scale_log2;  // sigma * log2(e)
@@ -94,22 +98,50 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // the start of its own 32-column fp32 source range: k-step kk (16 columns).
 __device__ __forceinline__ uint32_t split_acol(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-        "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15])
-        : "memory");
+// TMEM row access of N consecutive 32-bit columns (32x32b shape: lane = row).
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 16 || N == 32, "16 or 32 columns");
+    if constexpr (N == 32) {
+        tmem_ld32(taddr, r);
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+            "%11, %12, %13, %14, %15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+              "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr)
+            : "memory");
+    }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]) {
+    static_assert(N == 8 || N == 16, "8 or 16 columns");
+    if constexpr (N == 16) {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+            "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+            "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+            "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+            "r"(r[15])
+            : "memory");
+    } else {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                taddr),
+            "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+            : "memory");
+    }
 }
 
-// Writes 64 fp32 columns of a TMEM accumulator row (from `trow_col`) scaled
-// by `mul` as bf16 to global memory at dst.
-__device__ __forceinline__ void store_half_row(uint32_t trow_col, float mul, __nv_bfloat16* dst,
+// Writes 32*NCH fp32 columns of a TMEM accumulator row (from `trow_col`)
+// scaled by `mul` as bf16 to global memory at dst.
+template <int NCH>
+__device__ __forceinline__ void store_row_cols(uint32_t trow_col, float mul, __nv_bfloat16* dst,
                                                bool valid) {
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
+    for (int c = 0; c < NCH; ++c) {
         uint32_t u[32];
         tmem_ld32(trow_col + 32 * c, u);
         tmem_wait_ld();
@@ -133,7 +165,7 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
                   const __nv_bfloat16* __restrict__ dhf, const __nv_bfloat16* __restrict__ dhs,
                   const float* __restrict__ lse_f, const float* __restrict__ lse_s, size_t rows,
                   float cf, float cs, __nv_bfloat16* __restrict__ gf, __nv_bfloat16* __restrict__ gs,
-                  float* __restrict__ lse2, float* __restrict__ cfac, float* __restrict__ Df,
+                  float* __restrict__ lse2, float* __restrict__ Df,
                   float* __restrict__ Ds) {
     const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -145,6 +177,10 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
         const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
         o[0] = __low2float(a); o[1] = __high2float(a); o[2] = __low2float(b); o[3] = __high2float(b);
     };
+    // c_t = exp(lse_full - lse_sparse) carries P_f to P_s on selected pairs; it is
+    // folded into G_s here (0 where the sparse stream has no mass)
+    const float lf = lse_f[row], ls = lse_s[row];
+    const float c = ls > -INFINITY ? expf(lf - ls) : 0.f;
     float f[4], s[4], uf[4] = {0, 0, 0, 0}, us[4] = {0, 0, 0, 0};
     ld4(hf + e, f);
     ld4(hs + e, s);
@@ -156,8 +192,8 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
     for (int i = 0; i < 2; ++i) {
         const float gf0 = uf[2 * i] + cf * (f[2 * i] - s[2 * i]);
         const float gf1 = uf[2 * i + 1] + cf * (f[2 * i + 1] - s[2 * i + 1]);
-        const float gs0 = us[2 * i] + cs * (s[2 * i] - f[2 * i]);
-        const float gs1 = us[2 * i + 1] + cs * (s[2 * i + 1] - f[2 * i + 1]);
+        const float gs0 = c * (us[2 * i] + cs * (s[2 * i] - f[2 * i]));
+        const float gs1 = c * (us[2 * i + 1] + cs * (s[2 * i + 1] - f[2 * i + 1]));
         pf[i] = pack_bf16(gf0, gf1);
         ps[i] = pack_bf16(gs0, gs1);
         // D from the rounded values the tensor cores will see
@@ -174,42 +210,76 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
         ss += __shfl_xor_sync(0xffffffffu, ss, o);
     }
     if (lane == 0) {
-        const float lf = lse_f[row], ls = lse_s[row];
         lse2[row] = lf * kLog2e;
-        cfac[row] = ls > -INFINITY ? expf(lf - ls) : 0.f;
         Df[row] = sf;
         Ds[row] = ss;
     }
 }
 
 // ============================================================ dK / dV
+#ifndef SSA_KV_WARPGROUPS
+#define SSA_KV_WARPGROUPS 2
+#endif
 namespace kv {
+constexpr int NWG = SSA_KV_WARPGROUPS;  // compute warpgroups; each owns COLS query columns of a step
+static_assert(NWG == 2 || NWG == 4, "2 or 4 compute warpgroups");
+constexpr int COLS = STEP / NWG;
+constexpr int kThr = 128 + 128 * NWG;  // warp 0 TMA, 1 MMA, 2-3 idle, then the compute warps
+constexpr int kComp = 128 * NWG;
 constexpr uint32_t OFF_K = 0;
 constexpr uint32_t OFF_V = TILE_BYTES;
 constexpr uint32_t OFF_STAGE = 2 * TILE_BYTES;
-constexpr uint32_t ST_Q = 0, ST_GF = STEP_BYTES, ST_GS = 2 * STEP_BYTES, ST_ROWS = 3 * STEP_BYTES;
-constexpr uint32_t STAGE_BYTES = (3 * STEP_BYTES + 4 * STEP * 4 + 1023) / 1024 * 1024;
-constexpr uint32_t OFF_BAR = OFF_STAGE + 2 * STAGE_BYTES;
+constexpr uint32_t ST_Q = 0, ST_GF = STEP_BYTES, ST_GS = 2 * STEP_BYTES;
+constexpr uint32_t STAGE_BYTES = 3 * STEP_BYTES;
+constexpr int NSTAGE = 3;
+// dS^T of the current step, bf16 [128 keys x 64 queries], K-major with
+// 128-byte swizzle: the A operand of dK += dS^T Q
+constexpr uint32_t OFF_DS = OFF_STAGE + NSTAGE * STAGE_BYTES;
+// per stage, fp32 over the step's 64 queries: lse_full*log2(e) | D_f | D_s
+constexpr uint32_t ROW_BYTES = 3 * STEP * 4;
+constexpr uint32_t OFF_ROWS = OFF_DS + 128 * 128;
+constexpr uint32_t OFF_BAR = OFF_ROWS + NSTAGE * ROW_BYTES;
+// TMEM slot, abort flag, then one selection word per stage (bit 0: the step's
+// query block selects key block kb0, bit 1: selects kb1)
 constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
-constexpr uint32_t OFF_SEL = OFF_MISC + 16;  // one byte per query block
-constexpr uint32_t SMEM_BYTES = OFF_SEL + kMaxBlocks + 1024;
-enum : int { B_KV = 0, B_FULL = 1, B_EMPTY = 3, B_READY = 5, B_PREADY = 6, B_DONE = 7, B_DRAIN = 8 };
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 32;
+static_assert(SMEM_BYTES <= 232448, "227 KB of shared memory per CTA");
+enum : int {  // barrier indices, derived from the ring depth
+    B_KV = 0, B_FULL = 1, B_EMPTY = B_FULL + NSTAGE, B_READY = B_EMPTY + NSTAGE,
+    B_PREADY = B_READY + 1, B_DONE = B_PREADY + 1, B_DRAIN = B_DONE + 1,
+    B_DPFREE = B_DRAIN + 1,  // compute has loaded dP_f^T / dP_s^T of the step (the buffers may be refilled)
+    B_DSFREE = B_DPFREE + 1,  // the dK MMAs have read the dS^T tile in shared memory
+    B_COUNT = B_DSFREE + 1
+};
+static_assert(B_COUNT <= 16, "barrier area holds 16");
 constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_S0 = 256, TM_S1 = 320, TM_DPF = 384, TM_DPS = 448;
+// bf16 P^T written by warpgroup w over the first COLS/2 of its own COLS fp32
+// S columns; the masked copy for the sparse stream follows at +COLS/2.
+// TMEM column of the A operand's k-step kk (16 queries):
+__device__ __forceinline__ uint32_t acol(int kk) {
+    return (uint32_t)(COLS * ((16 * kk) / COLS) + ((16 * kk) % COLS) / 2);
+}
 }  // namespace kv
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kv::kThr, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_gf,
                    const __grid_constant__ CUtensorMap tm_gs, const BwdArgs a) {
     using namespace kv;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* gbase = smem_raw + (base - raw);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t base = smem_u32(smem_raw);
+    unsigned int* status = &g_bwd_tc_status;
+    // the swizzled tiles need a 1024-byte aligned base and the layout leaves no
+    // room to realign: refuse (status bit 1) rather than misplace them
+    if (base & 1023u) {
+        if (threadIdx.x == 0) atomicOr(status, 2u);
+        return;
+    }
+    uint8_t* gbase = smem_raw;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
-    uint8_t* selb = gbase + OFF_SEL;
-    unsigned int* status = &g_bwd_tc_status;
+    uint32_t* flags = reinterpret_cast<uint32_t*>(gbase + OFF_MISC + 8);
+    const float* rows_s = reinterpret_cast<const float*>(gbase + OFF_ROWS);
     const uint64_t lim = a.timeout_ns;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -219,27 +289,23 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int ns = (a.T - s0) / STEP;
     const int kb0 = s0 / a.block;
     const int kb1 = (s0 + 64 < a.T) ? (s0 + 64) / a.block : kb0;
-    const int qb_first = s0 / a.block;
     auto BAR = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
     const size_t rowbase = (size_t)bh * a.T;
 
     if (threadIdx.x == 0) {
         mbar_init(BAR(B_KV), 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(BAR(B_FULL + s), 1);
             mbar_init(BAR(B_EMPTY + s), 1);
         }
         mbar_init(BAR(B_READY), 1);
-        mbar_init(BAR(B_PREADY), kCompute);
+        mbar_init(BAR(B_PREADY), kComp);
         mbar_init(BAR(B_DONE), 1);
         mbar_init(BAR(B_DRAIN), 1);
+        mbar_init(BAR(B_DPFREE), kComp);
+        mbar_init(BAR(B_DSFREE), 1);
         *abort_flag = 0;
         fence_mbar_init();
-    }
-    // selection of this tile's key blocks for every later query block
-    for (int qb = qb_first + (int)threadIdx.x; qb < a.n_blocks; qb += kThreads) {
-        const uint32_t* m = a.mask + ((size_t)bh * a.n_blocks + qb) * a.words;
-        selb[qb] = (uint8_t)(bit(m, kb0) | (bit(m, kb1) << 1));
     }
     if (warp == 1) {
         tmem_alloc(base + OFF_MISC, 512);
@@ -249,7 +315,6 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    auto step_qb = [&](int i) { return (s0 + STEP * i) / a.block; };
 
     const unsigned FULL = 0xffffffffu;
     if (warp == 0) {
@@ -267,35 +332,44 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tma_load_3d(base + OFF_V + BOX_T, &tm_v, BAR(B_KV), 64, s0, bh);
         }
         __syncwarp();
-        int issued[2] = {-1, -1};
+        int issued[NSTAGE];
+        for (int s = 0; s < NSTAGE; ++s) issued[s] = -1;
         for (int i = 0; i < ns; ++i) {
-            const int s = i & 1;
-            if (i >= 2 &&
-                !__all_sync(FULL, mbar_wait(BAR(B_EMPTY + s), ((i >> 1) + 1) & 1, abort_flag, status, lim)))
+            const int s = i % NSTAGE;
+            const int t0 = s0 + STEP * i;
+            // selection of the tile's key blocks by the step's query block
+            const uint32_t* m = a.mask + ((size_t)bh * a.n_blocks + t0 / a.block) * a.words;
+            const uint32_t fl = (uint32_t)bit(m, kb0) | ((uint32_t)bit(m, kb1) << 1);
+            if (i >= NSTAGE &&
+                !__all_sync(FULL, mbar_wait(BAR(B_EMPTY + s), ((i / NSTAGE) + 1) & 1, abort_flag, status,
+                                            lim)))
                 break;
             const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
-            const int t0 = s0 + STEP * i;
+            const uint32_t rw = base + OFF_ROWS + s * ROW_BYTES;
             if (elect_one()) {
-                mbar_expect_tx(BAR(B_FULL + s), 3 * STEP_BYTES + 4 * STEP * 4);
+                const bool sp = fl != 0u;
+                flags[s] = fl;  // published by the arrive below
+                mbar_expect_tx(BAR(B_FULL + s), 2 * STEP_BYTES + 2 * STEP * 4 +
+                                                    (sp ? STEP_BYTES + STEP * 4 : 0u));
                 tma_load_3d(st + ST_Q, &tm_q, BAR(B_FULL + s), 0, t0, bh);
                 tma_load_3d(st + ST_Q + BOX_S, &tm_q, BAR(B_FULL + s), 64, t0, bh);
                 tma_load_3d(st + ST_GF, &tm_gf, BAR(B_FULL + s), 0, t0, bh);
                 tma_load_3d(st + ST_GF + BOX_S, &tm_gf, BAR(B_FULL + s), 64, t0, bh);
-                tma_load_3d(st + ST_GS, &tm_gs, BAR(B_FULL + s), 0, t0, bh);
-                tma_load_3d(st + ST_GS + BOX_S, &tm_gs, BAR(B_FULL + s), 64, t0, bh);
-                const size_t r0 = rowbase + t0;
-                bulk_load(st + ST_ROWS, a.lse2 + r0, STEP * 4, BAR(B_FULL + s));
-                bulk_load(st + ST_ROWS + STEP * 4, a.cfac + r0, STEP * 4, BAR(B_FULL + s));
-                bulk_load(st + ST_ROWS + 2 * STEP * 4, a.Df + r0, STEP * 4, BAR(B_FULL + s));
-                bulk_load(st + ST_ROWS + 3 * STEP * 4, a.Ds + r0, STEP * 4, BAR(B_FULL + s));
+                bulk_load(rw, a.lse2 + rowbase + t0, STEP * 4, BAR(B_FULL + s));
+                bulk_load(rw + STEP * 4, a.Df + rowbase + t0, STEP * 4, BAR(B_FULL + s));
+                if (sp) {  // the sparse stream's operands only where it has work
+                    tma_load_3d(st + ST_GS, &tm_gs, BAR(B_FULL + s), 0, t0, bh);
+                    tma_load_3d(st + ST_GS + BOX_S, &tm_gs, BAR(B_FULL + s), 64, t0, bh);
+                    bulk_load(rw + 2 * STEP * 4, a.Ds + rowbase + t0, STEP * 4, BAR(B_FULL + s));
+                }
             }
             __syncwarp();
             issued[s] = i;
         }
         wait_drain(BAR(B_KV), 0, kDrainLimitNs);
         if (*abort_flag)
-            for (int s = 0; s < 2; ++s)
-                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] >> 1) & 1, kDrainLimitNs);
+            for (int s = 0; s < NSTAGE; ++s)
+                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
     } else if (warp == 1) {
         {  // ------------------------------------------ MMA issuer (whole warp)
             // descriptors formed once, advanced by constant offsets; each MMA group
@@ -309,17 +383,16 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             auto kq = [](int kk) { return (uint32_t)((kk >> 2) * BOX_T + (kk & 3) * 32); };
             auto ks = [](int kk) { return (uint32_t)((kk >> 2) * BOX_S + (kk & 3) * 32); };
             bool ok = __all_sync(FULL, mbar_wait(BAR(B_KV), 0, abort_flag, status, lim));
-            auto sparse = [&](int i) { return selb[step_qb(i)] != 0; };
             auto issue_s = [&](int i) {  // elected lane only
-                const uint64_t qd = desc_add(st_k0, (i & 1) * STAGE_BYTES + ST_Q);
+                const uint64_t qd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_Q);
                 const uint32_t d = tmem + ((i & 1) ? TM_S1 : TM_S0);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(d, desc_add(kdesc, kq(kk)), desc_add(qd, ks(kk)), id_s, kk > 0);
             };
             auto issue_dp = [&](int i, bool sp) {  // elected lane only
-                const uint64_t gfd = desc_add(st_k0, (i & 1) * STAGE_BYTES + ST_GF);
-                const uint64_t gsd = desc_add(st_k0, (i & 1) * STAGE_BYTES + ST_GS);
+                const uint64_t gfd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_GF);
+                const uint64_t gsd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_GS);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ss(tmem + TM_DPF, desc_add(vdesc, kq(kk)), desc_add(gfd, ks(kk)), id_s, kk > 0);
@@ -333,7 +406,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 ok = __all_sync(FULL, mbar_wait(BAR(B_FULL), 0, abort_flag, status, lim));
                 if (ok) {
                     fence_after_sync();
-                    const bool sp0 = sparse(0);
+                    const bool sp0 = flags[0] != 0u;
                     if (elect_one()) {
                         issue_s(0);
                         issue_dp(0, sp0);
@@ -342,10 +415,12 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     __syncwarp();
                 }
             }
+            const uint64_t dsd = smem_desc_sw128(base + OFF_DS, 16, 1024);  // K-major A
             for (int i = 0; ok && i < ns; ++i) {
-                const int s = i & 1;
+                const int s = i % NSTAGE, b = i & 1;
                 if (i + 1 < ns) {
-                    if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + ((i + 1) & 1)), ((i + 1) >> 1) & 1,
+                    // S^T of the next step: its buffer's P_f^T was read by dV of step i-1
+                    if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + (i + 1) % NSTAGE), ((i + 1) / NSTAGE) & 1,
                                                     abort_flag, status, lim))) {
                         ok = false;
                         break;
@@ -353,38 +428,49 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     fence_after_sync();
                     if (elect_one()) issue_s(i + 1);
                     __syncwarp();
+                    // dP^T of the next step as soon as the compute warps have loaded this one's
+                    if (!__all_sync(FULL, mbar_wait(BAR(B_DPFREE), i & 1, abort_flag, status, lim))) {
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
+                    const bool sp_next = flags[(i + 1) % NSTAGE] != 0u;
+                    if (elect_one()) {
+                        issue_dp(i + 1, sp_next);
+                        mma_commit(BAR(B_READY));
+                    }
+                    __syncwarp();
                 }
                 if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY), i & 1, abort_flag, status, lim))) {
                     ok = false;
                     break;
                 }
                 fence_after_sync();
-                const uint32_t sb = tmem + (s ? TM_S1 : TM_S0);
+                const uint32_t sb = tmem + (b ? TM_S1 : TM_S0);
                 const uint64_t gfm = desc_add(st_m0, s * STAGE_BYTES + ST_GF);
                 const uint64_t gsm = desc_add(st_m0, s * STAGE_BYTES + ST_GS);
                 const uint64_t qm = desc_add(st_m0, s * STAGE_BYTES + ST_Q);
-                const bool sp = sparse(i);
-                const bool sp_next = i + 1 < ns && sparse(i + 1);
+                const uint32_t fl = flags[s];
+                // P_s^T = P_f^T on selected key rows (c_t is folded into G_s); the
+                // masked copy is needed only when the tile's two key blocks differ
+                const uint32_t ps_off = (fl == 1u || fl == 2u) ? (uint32_t)(COLS / 2) : 0u;
                 if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // dV += P_f^T G_f
-                        mma_ts(tmem + TM_DV, sb + split_acol(kk), desc_add(gfm, kk * 2048), id_a,
+                    for (int kk = 0; kk < 4; ++kk)  // dV += P_f^T G_f  (P_f^T in TMEM)
+                        mma_ts(tmem + TM_DV, sb + acol(kk), desc_add(gfm, kk * 2048), id_a,
                                (i > 0 || kk > 0) ? 1u : 0u);
-                    if (sp) {
+                    if (fl != 0u) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)  // dV += P_s^T G_s
-                            mma_ts(tmem + TM_DV, tmem + TM_DPS + split_acol(kk), desc_add(gsm, kk * 2048),
-                                   id_a, 1u);
+                            mma_ts(tmem + TM_DV, sb + acol(kk) + ps_off, desc_add(gsm, kk * 2048), id_a,
+                                   1u);
                     }
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q
-                        mma_ts(tmem + TM_DK, tmem + TM_DPF + split_acol(kk), desc_add(qm, kk * 2048), id_a,
+                    for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q  (dS^T in smem)
+                        mma_ss(tmem + TM_DK, desc_add(dsd, kk * 32), desc_add(qm, kk * 2048), id_a,
                                (i > 0 || kk > 0) ? 1u : 0u);
                     mma_commit(BAR(B_EMPTY + s));
-                    if (i + 1 < ns) {
-                        issue_dp(i + 1, sp_next);
-                        mma_commit(BAR(B_READY));
-                    }
+                    mma_commit(BAR(B_DSFREE));
                 }
                 __syncwarp();
             }
@@ -396,89 +482,102 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
         }
     } else if (warp >= 4) {
-        // ------------------------------------------ two compute warpgroups
-        // warpgroup wg handles columns [32 wg, 32 wg + 32) of every step
+        // ------------------------------------------ compute warpgroups
+        // warpgroup wg handles query columns [COLS wg, COLS wg + COLS) of every step
         const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
         const int r = sw * 32 + lane;  // key row of the tile == TMEM lane
         const int s_tok = s0 + r;
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
         const float sl2 = a.scale_log2;
-        const bool in_kb1 = r >= 64 && a.block == 64;
-        const int c0 = 32 * wg;
+        const bool in_kb1 = r >= 64 && a.block == 64;  // warp-uniform
+        const int c0 = COLS * wg;
         bool ok = true;
         for (int i = 0; i < ns; ++i) {
-            if (!__all_sync(0xffffffffu, mbar_wait(BAR(B_READY), i & 1, abort_flag, status, lim))) {
-                ok = false;
-                break;
-            }
-            const int s = i & 1;
-            // the stage's row vectors (bulk copies) are read directly: observe their barrier
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(BAR(B_FULL + s), (i >> 1) & 1, abort_flag, status, lim))) {
+            const int t0 = s0 + STEP * i;
+            const int s = i % NSTAGE, b = i & 1;
+            // the stage's row vectors and selection word (already landed: the MMA
+            // warp waited for them before issuing this step's S^T)
+            if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + s), (i / NSTAGE) & 1, abort_flag, status, lim)) ||
+                !__all_sync(FULL, mbar_wait(BAR(B_READY), i & 1, abort_flag, status, lim))) {
                 ok = false;
                 break;
             }
             fence_after_sync();
-            const float4* rows4 = reinterpret_cast<const float4*>(
-                gbase + OFF_STAGE + s * STAGE_BYTES + ST_ROWS);  // lse2 | c | Df | Ds, 64 each
-            const int t0 = s0 + STEP * i;
-            const uint8_t sb2 = selb[step_qb(i)];
-            const bool sparse = sb2 != 0;
-            const bool my_sel = in_kb1 ? (sb2 >> 1) & 1 : sb2 & 1;
-            const bool use_s = sparse && my_sel;
+            const uint32_t fl = flags[s];
+            const bool use_s = in_kb1 ? (fl >> 1) & 1u : fl & 1u;
+            const bool mixed = fl == 1u || fl == 2u;
             const bool diag = t0 < s0 + TILE;
-            const uint32_t sbuf = trow + (s ? TM_S1 : TM_S0);
-            uint32_t su[32], fu[32], pu[32];
-            tmem_ld32(sbuf + c0, su);
-            tmem_ld32(trow + TM_DPF + c0, fu);
-            if (sparse) tmem_ld32(trow + TM_DPS + c0, pu);
+            const uint32_t sbuf = trow + (b ? TM_S1 : TM_S0);
+            uint32_t su[COLS], fu[COLS], pu[COLS];
+            tmem_ld<COLS>(sbuf + c0, su);
+            tmem_ld<COLS>(trow + TM_DPF + c0, fu);
+            if (use_s) tmem_ld<COLS>(trow + TM_DPS + c0, pu);
             tmem_wait_ld();
-            uint32_t pfk[16], psk[16], dsk[16];
+            fence_before_sync();
+            mbar_arrive(BAR(B_DPFREE));  // dP_f^T / dP_s^T may now be overwritten
+            const float4* L4 = reinterpret_cast<const float4*>(rows_s + s * (3 * STEP) + c0);
+            const float4* F4 = reinterpret_cast<const float4*>(rows_s + s * (3 * STEP) + STEP + c0);
+            const float4* S4 = reinterpret_cast<const float4*>(rows_s + s * (3 * STEP) + 2 * STEP + c0);
+            uint32_t pfk[COLS / 2], dsk[COLS / 2];
 #pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-                const int col = c0 + 4 * j4;
-                const float4 L = rows4[col >> 2], C = rows4[(STEP + col) >> 2];
-                const float4 F = rows4[(2 * STEP + col) >> 2], S = rows4[(3 * STEP + col) >> 2];
-                const float lv[4] = {L.x, L.y, L.z, L.w}, cv[4] = {C.x, C.y, C.z, C.w};
-                const float fv[4] = {F.x, F.y, F.z, F.w}, sv[4] = {S.x, S.y, S.z, S.w};
-                float pf[4], ps[4], ds[4];
+            for (int j4 = 0; j4 < COLS / 4; ++j4) {
+                const float4 L = L4[j4], F = F4[j4];
+                const float4 S = use_s ? S4[j4] : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float lv[4] = {L.x, L.y, L.z, L.w}, fv[4] = {F.x, F.y, F.z, F.w};
+                const float sv[4] = {S.x, S.y, S.z, S.w};
+                float pf[4], ds[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int j = 4 * j4 + h;
                     float p = ex2(fmaf(__uint_as_float(su[j]), sl2, -lv[h]));
-                    if (diag && t0 + col + h < s_tok) p = 0.f;
-                    float d = p * (__uint_as_float(fu[j]) - fv[h]);
-                    float q2 = 0.f;
-                    if (use_s) {
-                        q2 = p * cv[h];
-                        d = fmaf(q2, __uint_as_float(pu[j]) - sv[h], d);
-                    }
+                    if (diag && t0 + c0 + j < s_tok) p = 0.f;
+                    float g = __uint_as_float(fu[j]) - fv[h];
+                    if (use_s) g += __uint_as_float(pu[j]) - sv[h];
                     pf[h] = p;
-                    ps[h] = q2;
-                    ds[h] = d;
+                    ds[h] = p * g;
                 }
                 pfk[2 * j4] = pack_bf16_alu(pf[0], pf[1]);
                 pfk[2 * j4 + 1] = pack_bf16_alu(pf[2], pf[3]);
-                psk[2 * j4] = pack_bf16_alu(ps[0], ps[1]);
-                psk[2 * j4 + 1] = pack_bf16_alu(ps[2], ps[3]);
                 dsk[2 * j4] = pack_bf16_alu(ds[0], ds[1]);
                 dsk[2 * j4 + 1] = pack_bf16_alu(ds[2], ds[3]);
             }
-            // bf16 results go to the first 16 columns of this warpgroup's own range
-            tmem_st16(sbuf + c0, pfk);                       // P_f^T
-            if (sparse) tmem_st16(trow + TM_DPS + c0, psk);  // P_s^T
-            tmem_st16(trow + TM_DPF + c0, dsk);              // dS^T
+            // dS^T goes to shared memory, row r of a 128B-swizzled K-major tile,
+            // once the previous step's dK MMAs have read it
+            if (i > 0 && !__all_sync(FULL, mbar_wait(BAR(B_DSFREE), (i - 1) & 1, abort_flag, status, lim))) {
+                ok = false;
+                break;
+            }
+            // P_f^T (bf16) over this warpgroup's own consumed S columns; on a
+            // mixed step the sparse stream's copy, zero on unselected key rows
+            tmem_st<COLS / 2>(sbuf + c0, pfk);
+            if (mixed) {
+                if (!use_s)
+#pragma unroll
+                    for (int e = 0; e < COLS / 2; ++e) pfk[e] = 0u;
+                tmem_st<COLS / 2>(sbuf + c0 + COLS / 2, pfk);
+            }
+            {
+                const uint32_t rowoff = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
+#pragma unroll
+                for (int q4 = 0; q4 < COLS / 8; ++q4) {
+                    const uint32_t chunk = (uint32_t)((c0 >> 3) + q4) ^ (uint32_t)(r & 7);
+                    *reinterpret_cast<uint4*>(gbase + OFF_DS + rowoff + chunk * 16) =
+                        make_uint4(dsk[4 * q4], dsk[4 * q4 + 1], dsk[4 * q4 + 2], dsk[4 * q4 + 3]);
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the MMAs
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PREADY));
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim));
+        if (ok) ok = __all_sync(FULL, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim));
         if (ok) {
             fence_after_sync();
             const bool valid = s_tok < a.T;
             const size_t row = rowbase + (valid ? s_tok : 0);
-            store_half_row(trow + TM_DV + 64 * wg, 1.f, a.dv + row * HD + 64 * wg, valid);
-            store_half_row(trow + TM_DK + 64 * wg, a.sm_scale, a.dk + row * HD + 64 * wg, valid);
+            constexpr int OC = HD / NWG;  // output columns per warpgroup
+            store_row_cols<OC / 32>(trow + TM_DV + OC * wg, 1.f, a.dv + row * HD + OC * wg, valid);
+            store_row_cols<OC / 32>(trow + TM_DK + OC * wg, a.sm_scale, a.dk + row * HD + OC * wg, valid);
         }
     }
     fence_before_sync();
@@ -495,14 +594,18 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_GF = TILE_BYTES;
 constexpr uint32_t OFF_GS = 2 * TILE_BYTES;
 constexpr uint32_t OFF_STAGE = 3 * TILE_BYTES;
-constexpr int NSTAGE = 3;
+constexpr int NSTAGE = 4;
 constexpr uint32_t ST_K = 0, ST_V = STEP_BYTES;
 constexpr uint32_t STAGE_BYTES = 2 * STEP_BYTES;
 constexpr uint32_t OFF_BAR = OFF_STAGE + NSTAGE * STAGE_BYTES;
 constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
 constexpr uint32_t OFF_MASK = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = OFF_MASK + 2 * kMaxWords * 4 + 1024;
-enum : int { B_QG = 0, B_FULL = 1, B_EMPTY = 4, B_READY = 7, B_PREADY = 9, B_DONE = 11, B_DRAIN = 12 };
+enum : int {  // barrier indices, derived from the ring depth
+    B_QG = 0, B_FULL = 1, B_EMPTY = B_FULL + NSTAGE, B_READY = B_EMPTY + NSTAGE,
+    B_PREADY = B_READY + 2, B_DONE = B_PREADY + 2, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
+};
+static_assert(B_COUNT <= 16, "barrier area holds 16");
 constexpr uint32_t TM_DQ = 0, TM_S0 = 128, TM_S1 = 192, TM_DP0 = 256, TM_DP1 = 384;  // DP: f | s
 }  // namespace qk
 
@@ -590,7 +693,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tma_load_3d(base + OFF_GS + BOX_T, &tm_gs, BAR(B_QG), 64, t0, bh);
         }
         __syncwarp();
-        int issued[NSTAGE] = {-1, -1, -1};
+        int issued[NSTAGE] = {-1, -1, -1, -1};
         for (int i = 0; i < ns; ++i) {
             const int s = i % NSTAGE;
             if (i >= NSTAGE &&
@@ -686,7 +789,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int t = t0 + r;
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
         const size_t row = rowbase + (t < a.T ? t : a.T - 1);
-        const float my_lse2 = a.lse2[row], my_c = a.cfac[row], my_df = a.Df[row], my_ds = a.Ds[row];
+        const float my_lse2 = a.lse2[row], my_df = a.Df[row], my_ds = a.Ds[row];
         const uint32_t* myrow = (r < 64 || a.block == 128 || ragged1) ? mrow : mrow + kMaxWords;
         const float sl2 = a.scale_log2;
         const int c0 = 32 * wg;
@@ -708,7 +811,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             uint32_t su[32], fu[32], pu[32];
             tmem_ld32(sbuf + c0, su);
             tmem_ld32(dp + c0, fu);
-            if (sp) tmem_ld32(dp + 64 + c0, pu);
+            if (use_s) tmem_ld32(dp + 64 + c0, pu);  // warp-uniform: one query block per warp
             tmem_wait_ld();
             uint32_t dsk[16];
 #pragma unroll
@@ -719,13 +822,13 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const int j = 2 * j2 + h;
                     float pf = ex2(fmaf(__uint_as_float(su[j]), sl2, -my_lse2));
                     if (diag && k0 + j > t) pf = 0.f;
-                    float ds = pf * (__uint_as_float(fu[j]) - my_df);
-                    if (use_s) ds = fmaf(pf * my_c, __uint_as_float(pu[j]) - my_ds, ds);
-                    ds2[h] = ds;
+                    float g = __uint_as_float(fu[j]) - my_df;
+                    if (use_s) g += __uint_as_float(pu[j]) - my_ds;
+                    ds2[h] = pf * g;
                 }
                 dsk[j2] = pack_bf16_alu(ds2[0], ds2[1]);
             }
-            tmem_st16(sbuf + c0, dsk);  // dS (bf16) over this warpgroup's consumed S columns
+            tmem_st<16>(sbuf + c0, dsk);  // dS (bf16) over this warpgroup's consumed S columns
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PREADY + b));
@@ -734,7 +837,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (ok) {
             fence_after_sync();
             const bool valid = t < a.T;
-            store_half_row(trow + TM_DQ + 64 * wg, a.sm_scale,
+            store_row_cols<2>(trow + TM_DQ + 64 * wg, a.sm_scale,
                            a.dq + (valid ? row : rowbase) * HD + 64 * wg, valid);
         }
     }
@@ -779,7 +882,7 @@ int make_map(CUtensorMap* m, const void* ptr, int BH, int T, int rows) {
 struct TcWs {
     __nv_bfloat16* gf;
     __nv_bfloat16* gs;
-    float *lse2, *cfac, *Df, *Ds;
+    float *lse2, *Df, *Ds;
 };
 
 TcWs carve(const ssa_params_t& p, void* ws) {
@@ -790,9 +893,8 @@ TcWs carve(const ssa_params_t& p, void* ws) {
     w.gf = reinterpret_cast<__nv_bfloat16*>(b);
     w.gs = reinterpret_cast<__nv_bfloat16*>(b + big);
     w.lse2 = reinterpret_cast<float*>(b + 2 * big);
-    w.cfac = reinterpret_cast<float*>(b + 2 * big + small);
-    w.Df = reinterpret_cast<float*>(b + 2 * big + 2 * small);
-    w.Ds = reinterpret_cast<float*>(b + 2 * big + 3 * small);
+    w.Df = reinterpret_cast<float*>(b + 2 * big + small);
+    w.Ds = reinterpret_cast<float*>(b + 2 * big + 2 * small);
     return w;
 }
 
@@ -805,7 +907,7 @@ bool bwd_tc_supported(const ssa_params_t& p) {
 }
 
 size_t bwd_tc_workspace(const ssa_params_t& p) {
-    return 2 * align_up(num_elems(p) * 2, 256) + 4 * align_up(num_rows(p) * 4, 256);
+    return 2 * align_up(num_elems(p) * 2, 256) + 3 * align_up(num_rows(p) * 4, 256);
 }
 
 int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
@@ -819,7 +921,7 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     bwd_tc_pre_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(hf), static_cast<const __nv_bfloat16*>(hs),
         static_cast<const __nv_bfloat16*>(dhf), static_cast<const __nv_bfloat16*>(dhs), lf, ls, rows,
-        (float)(w_s * two_over_n), (float)(w_c * two_over_n), w.gf, w.gs, w.lse2, w.cfac, w.Df, w.Ds);
+        (float)(w_s * two_over_n), (float)(w_c * two_over_n), w.gf, w.gs, w.lse2, w.Df, w.Ds);
     int st = check_launch("bwd_tc_pre_kernel");
     if (st != SSA_OK) return st;
 
@@ -851,7 +953,6 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     a.dk = static_cast<__nv_bfloat16*>(dk);
     a.dv = static_cast<__nv_bfloat16*>(dv);
     a.lse2 = w.lse2;
-    a.cfac = w.cfac;
     a.Df = w.Df;
     a.Ds = w.Ds;
     a.mask = mask;
@@ -864,7 +965,7 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     a.sm_scale = p.sm_scale;
     a.timeout_ns = wait_limit_ns();
     const unsigned grid = (unsigned)((size_t)BH * ((p.T + TILE - 1) / TILE));
-    bwd_dkdv_tc_kernel<<<grid, kThreads, kv::SMEM_BYTES, s>>>(k128, v128, q64, gf64, gs64, a);
+    bwd_dkdv_tc_kernel<<<grid, kv::kThr, kv::SMEM_BYTES, s>>>(k128, v128, q64, gf64, gs64, a);
     st = check_launch("bwd_dkdv_tc_kernel");
     if (st != SSA_OK) return st;
     bwd_dq_tc_kernel<<<grid, kThreads, qk::SMEM_BYTES, s>>>(q128, gf128, gs128, k64, v64, a);
@@ -878,6 +979,8 @@ int bwd_tc_take_status(cudaStream_t) {
     if (v) {
         const unsigned int zero = 0;
         cudaMemcpyToSymbol(g_bwd_tc_status, &zero, sizeof zero);
+        if (v & 2u)
+            return fail(SSA_ERR_CUDA, "bwd tcgen05 kernels: dynamic shared memory not 1024-byte aligned");
         return fail(SSA_ERR_TIMEOUT, "bwd tcgen05 kernels: a bounded mbarrier wait expired");
     }
     return SSA_OK;

@@ -66,10 +66,11 @@ constexpr uint32_t OFF_XCH = OFF_MASK + 2 * kMaxWords * 4;
 constexpr uint32_t SMEM_USED = OFF_XCH + 1024 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 
-enum : int {
+enum : int {  // barrier indices (two-stage K / V rings, two S buffers)
     B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7,
-    B_SREADY = 9, B_PREADY = 11, B_PVDONE = 13, B_DRAIN = 14
+    B_SREADY = 9, B_PREADY = 11, B_PVDONE = 13, B_DRAIN = 14, B_COUNT = 15
 };
+static_assert(B_COUNT <= NBAR, "barrier area");
 
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_OSEL = 256, TM_OUNS = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
