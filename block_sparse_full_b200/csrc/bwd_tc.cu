@@ -49,8 +49,6 @@ using namespace tc;
 constexpr int HD = 128;
 constexpr int TILE = 128;  // keys per dK/dV CTA, queries per dQ CTA
 constexpr int STEP = 64;   // queries per dK/dV step, keys per dQ step
-constexpr int kThreads = 384;  // warps 0-1 roles, 2-3 idle, 4-11 two compute warpgroups
-constexpr int kCompute = 256;
 constexpr int kMaxWords = 128;  // mask words per query block: n <= 4096 blocks
 constexpr int kMaxBlocks = kMaxWords * 32;
 constexpr uint32_t BOX_T = TILE * 128;  // [128 rows x 64 d] bf16 = 16 KB
@@ -94,10 +92,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
-// bf16 A operand of 64 K-columns written as two 32-wide halves, each half at
-// the start of its own 32-column fp32 source range: k-step kk (16 columns).
-__device__ __forceinline__ uint32_t split_acol(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
-
 // TMEM row access of N consecutive 32-bit columns (32x32b shape: lane = row).
 template <int N>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]) {
@@ -117,8 +111,10 @@ __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]) {
 }
 template <int N>
 __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]) {
-    static_assert(N == 8 || N == 16, "8 or 16 columns");
-    if constexpr (N == 16) {
+    static_assert(N == 8 || N == 16 || N == 32, "8, 16 or 32 columns");
+    if constexpr (N == 32) {
+        tmem_st32(taddr, r);
+    } else if constexpr (N == 16) {
         asm volatile(
             "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
             "%10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
@@ -589,30 +585,53 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 }
 
 // ============================================================ dQ
+#ifndef SSA_DQ_WARPGROUPS
+#define SSA_DQ_WARPGROUPS 2
+#endif
 namespace qk {
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_GF = TILE_BYTES;
-constexpr uint32_t OFF_GS = 2 * TILE_BYTES;
-constexpr uint32_t OFF_STAGE = 3 * TILE_BYTES;
-constexpr int NSTAGE = 4;
+// K/V steps stream through a ring; Q, G_f, G_s' of the tile live in TMEM as the
+// A operands of S, dP_f, dP_s (TS form: only the 64-key B tile is read from
+// shared memory); dS goes to a double-buffered shared tile for dQ += dS K.
+// S and dP are handed over separately: the next step's S MMAs start once the
+// compute warps have read this step's S, while they still wait for its dP.
+constexpr int NWG = SSA_DQ_WARPGROUPS;  // compute warpgroups; each owns COLS key columns of a step
+static_assert(NWG == 2 || NWG == 4, "2 or 4 compute warpgroups");
+constexpr int COLS = STEP / NWG;
+constexpr int kThr = 128 + 128 * NWG;
+constexpr int kComp = 128 * NWG;
+constexpr int NSTAGE = 5;
 constexpr uint32_t ST_K = 0, ST_V = STEP_BYTES;
 constexpr uint32_t STAGE_BYTES = 2 * STEP_BYTES;
-constexpr uint32_t OFF_BAR = OFF_STAGE + NSTAGE * STAGE_BYTES;
-constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
+constexpr uint32_t OFF_STAGE = 0;
+// dS, bf16 [128 queries x 64 keys], K-major with 128-byte swizzle, x2
+constexpr uint32_t DS_BYTES = 128 * 128;
+constexpr uint32_t OFF_DS = OFF_STAGE + NSTAGE * STAGE_BYTES;
+constexpr uint32_t OFF_BAR = OFF_DS + 2 * DS_BYTES;
+constexpr int NBAR = 24;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t OFF_MASK = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = OFF_MASK + 2 * kMaxWords * 4 + 1024;
+static_assert(SMEM_BYTES <= 232448, "227 KB of shared memory per CTA");
 enum : int {  // barrier indices, derived from the ring depth
-    B_QG = 0, B_FULL = 1, B_EMPTY = B_FULL + NSTAGE, B_READY = B_EMPTY + NSTAGE,
-    B_PREADY = B_READY + 2, B_DONE = B_PREADY + 2, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
+    B_FULL = 0, B_EMPTY = B_FULL + NSTAGE,
+    B_OPS = B_EMPTY + NSTAGE,  // Q, G_f, G_s' are in TMEM
+    B_SREADY = B_OPS + 1,      // S of the step is in TMEM
+    B_PREADY = B_SREADY + 1,   // dP_f, dP_s of the step are in TMEM
+    B_SFREE = B_PREADY + 1,    // the compute warps have read S (may be overwritten)
+    B_PFREE = B_SFREE + 1,     // ... and dP
+    B_DSREADY = B_PFREE + 1,   // x2: dS buffer written
+    B_DSFREE = B_DSREADY + 2,  // x2: dS buffer read by the dQ MMAs
+    B_DONE = B_DSFREE + 2, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
 };
-static_assert(B_COUNT <= 16, "barrier area holds 16");
-constexpr uint32_t TM_DQ = 0, TM_S0 = 128, TM_S1 = 192, TM_DP0 = 256, TM_DP1 = 384;  // DP: f | s
+static_assert(B_COUNT <= NBAR, "barrier area");
+constexpr uint32_t TM_DQ = 0, TM_S = 128, TM_DPF = 192, TM_DPS = 256;
+constexpr uint32_t TM_Q = 320, TM_GF = 384, TM_GS = 448;  // bf16 A operands, 64 cols each
 }  // namespace qk
 
-__global__ void __launch_bounds__(kThreads, 1)
-bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_gf,
-                 const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
+__global__ void __launch_bounds__(qk::kThr, 1)
+bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gf,
+                 const __nv_bfloat16* __restrict__ gs, const BwdArgs a) {
     using namespace qk;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -638,14 +657,18 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const size_t rowbase = (size_t)bh * a.T;
 
     if (threadIdx.x == 0) {
-        mbar_init(BAR(B_QG), 1);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(BAR(B_FULL + s), 1);
             mbar_init(BAR(B_EMPTY + s), 1);
         }
+        mbar_init(BAR(B_OPS), kComp);
+        mbar_init(BAR(B_SREADY), 1);
+        mbar_init(BAR(B_PREADY), 1);
+        mbar_init(BAR(B_SFREE), kComp);
+        mbar_init(BAR(B_PFREE), kComp);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(BAR(B_READY + b), 1);
-            mbar_init(BAR(B_PREADY + b), kCompute);
+            mbar_init(BAR(B_DSREADY + b), kComp);
+            mbar_init(BAR(B_DSFREE + b), 1);
         }
         mbar_init(BAR(B_DONE), 1);
         mbar_init(BAR(B_DRAIN), 1);
@@ -655,7 +678,7 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     {
         const uint32_t* m0 = a.mask + ((size_t)bh * a.n_blocks + qb0) * a.words;
         const uint32_t* m1 = a.mask + ((size_t)bh * a.n_blocks + qb1) * a.words;
-        for (int w = threadIdx.x; w < a.words; w += kThreads) {
+        for (int w = threadIdx.x; w < a.words; w += kThr) {
             mrow[w] = m0[w];
             mrow[kMaxWords + w] = m1[w];
         }
@@ -679,21 +702,12 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (warp == 0) {
         // -------------------------------------------- TMA producer (whole warp)
         if (elect_one()) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_gf);
-            prefetch_tmap(&tm_gs);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            mbar_expect_tx(BAR(B_QG), 3 * TILE_BYTES);
-            tma_load_3d(base + OFF_Q, &tm_q, BAR(B_QG), 0, t0, bh);
-            tma_load_3d(base + OFF_Q + BOX_T, &tm_q, BAR(B_QG), 64, t0, bh);
-            tma_load_3d(base + OFF_GF, &tm_gf, BAR(B_QG), 0, t0, bh);
-            tma_load_3d(base + OFF_GF + BOX_T, &tm_gf, BAR(B_QG), 64, t0, bh);
-            tma_load_3d(base + OFF_GS, &tm_gs, BAR(B_QG), 0, t0, bh);
-            tma_load_3d(base + OFF_GS + BOX_T, &tm_gs, BAR(B_QG), 64, t0, bh);
         }
         __syncwarp();
-        int issued[NSTAGE] = {-1, -1, -1, -1};
+        int issued[NSTAGE];
+        for (int s = 0; s < NSTAGE; ++s) issued[s] = -1;
         for (int i = 0; i < ns; ++i) {
             const int s = i % NSTAGE;
             if (i >= NSTAGE &&
@@ -711,7 +725,6 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncwarp();
             issued[s] = i;
         }
-        wait_drain(BAR(B_QG), 0, kDrainLimitNs);
         if (*abort_flag)
             for (int s = 0; s < NSTAGE; ++s)
                 if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
@@ -719,60 +732,78 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         {  // ------------------------------------------ MMA issuer (whole warp)
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S, dP
             constexpr uint32_t id_q = idesc_bf16_f32(TILE, HD, true);     // dQ
-            const uint64_t qdesc = smem_desc_sw128(base + OFF_Q, 16, 1024);
-            const uint64_t gfdesc = smem_desc_sw128(base + OFF_GF, 16, 1024);
-            const uint64_t gsdesc = smem_desc_sw128(base + OFF_GS, 16, 1024);
             const uint64_t st_k0 = smem_desc_sw128(base + OFF_STAGE, 16, 1024);      // K-major
             const uint64_t st_m0 = smem_desc_sw128(base + OFF_STAGE, BOX_S, 1024);   // MN-major
-            auto kt = [](int kk) { return (uint32_t)((kk >> 2) * BOX_T + (kk & 3) * 32); };
+            const uint64_t ds_0 = smem_desc_sw128(base + OFF_DS, 16, 1024);          // K-major A
             auto ks = [](int kk) { return (uint32_t)((kk >> 2) * BOX_S + (kk & 3) * 32); };
-            bool ok = __all_sync(FULL, mbar_wait(BAR(B_QG), 0, abort_flag, status, lim));
-            auto issue_front = [&](int i) -> bool {  // S_i, dP_f_i, dP_s_i
-                const int s = i % NSTAGE, b = i & 1;
-                if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + s), (i / NSTAGE) & 1, abort_flag, status, lim)))
-                    return false;
+            auto wait = [&](int bar, uint32_t parity) {
+                const bool r = __all_sync(FULL, mbar_wait(BAR(bar), parity, abort_flag, status, lim));
                 fence_after_sync();
-                const uint64_t kd = desc_add(st_k0, s * STAGE_BYTES + ST_K);
-                const uint64_t vd = desc_add(st_k0, s * STAGE_BYTES + ST_V);
-                const uint32_t sd = tmem + (b ? TM_S1 : TM_S0);
-                const uint32_t dp = tmem + (b ? TM_DP1 : TM_DP0);
+                return r;
+            };
+            auto issue_s = [&](int i) {  // S = Q K^T
+                const uint64_t kd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_K);
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tmem + TM_S, tmem + TM_Q + 8 * kk, desc_add(kd, ks(kk)), id_s, kk > 0);
+                    mma_commit(BAR(B_SREADY));
+                }
+                __syncwarp();
+            };
+            auto issue_dp = [&](int i) {  // dP_f = G_f V^T, dP_s = G_s' V^T
+                const uint64_t vd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_V);
                 const bool sp = sparse(i);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(sd, desc_add(qdesc, kt(kk)), desc_add(kd, ks(kk)), id_s, kk > 0);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(dp, desc_add(gfdesc, kt(kk)), desc_add(vd, ks(kk)), id_s, kk > 0);
+                        mma_ts(tmem + TM_DPF, tmem + TM_GF + 8 * kk, desc_add(vd, ks(kk)), id_s, kk > 0);
                     if (sp) {
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_ss(dp + 64, desc_add(gsdesc, kt(kk)), desc_add(vd, ks(kk)), id_s, kk > 0);
+                            mma_ts(tmem + TM_DPS, tmem + TM_GS + 8 * kk, desc_add(vd, ks(kk)), id_s,
+                                   kk > 0);
                     }
-                    mma_commit(BAR(B_READY + b));
+                    mma_commit(BAR(B_PREADY));
                 }
                 __syncwarp();
-                return true;
             };
-            for (int i = 0; ok && i < ns && i < 2; ++i) ok = issue_front(i);
+            auto issue_dq = [&](int j) {  // dQ += dS_j K_j, then release stage and dS buffer
+                const uint64_t km = desc_add(st_m0, (j % NSTAGE) * STAGE_BYTES + ST_K);
+                const uint64_t dd = desc_add(ds_0, (j & 1) * DS_BYTES);
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tmem + TM_DQ, desc_add(dd, kk * 32), desc_add(km, kk * 2048), id_q,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(BAR(B_EMPTY + j % NSTAGE));
+                    mma_commit(BAR(B_DSFREE + (j & 1)));
+                }
+                __syncwarp();
+            };
+            bool ok = wait(B_OPS, 0) && wait(B_FULL, 0);
+            if (ok) {
+                issue_s(0);
+                issue_dp(0);
+            }
             for (int i = 0; ok && i < ns; ++i) {
-                const int s = i % NSTAGE, b = i & 1;
-                if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY + b), (i >> 1) & 1, abort_flag, status, lim))) {
+                if (i + 1 < ns) {
+                    if (!wait(B_FULL + (i + 1) % NSTAGE, ((i + 1) / NSTAGE) & 1) || !wait(B_SFREE, i & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    issue_s(i + 1);
+                    if (!wait(B_PFREE, i & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    issue_dp(i + 1);
+                }
+                if (!wait(B_DSREADY + (i & 1), (i >> 1) & 1)) {
                     ok = false;
                     break;
                 }
-                fence_after_sync();
-                const uint64_t km = desc_add(st_m0, s * STAGE_BYTES + ST_K);
-                const uint32_t sd = tmem + (b ? TM_S1 : TM_S0);
-                if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // dQ += dS K
-                        mma_ts(tmem + TM_DQ, sd + split_acol(kk), desc_add(km, kk * 2048), id_q,
-                               (i > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(BAR(B_EMPTY + s));
-                }
-                __syncwarp();
-                if (i + 2 < ns && !issue_front(i + 2)) ok = false;
+                issue_dq(i);
             }
             if (elect_one()) {
                 mma_commit(BAR(B_DONE));
@@ -782,63 +813,112 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
         }
     } else if (warp >= 4) {
-        // ------------------------------------------ two compute warpgroups
-        // warpgroup wg handles key columns [32 wg, 32 wg + 32) of every step
+        // ------------------------------------------ compute warpgroups
+        // warpgroup wg handles key columns [COLS wg, COLS wg + COLS) of every step
         const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
         const int r = sw * 32 + lane;  // query row of the tile == TMEM lane
         const int t = t0 + r;
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
         const size_t row = rowbase + (t < a.T ? t : a.T - 1);
+        bool ok = true;
+        {  // the tile's Q, G_f, G_s' rows (this warpgroup's HD/NWG columns) into TMEM
+            constexpr int W = HD / NWG / 2;  // 32-bit TMEM columns per warpgroup and operand
+            auto fill = [&](const __nv_bfloat16* src, uint32_t col) {
+                uint32_t u[W];
+                const uint4* p4 = reinterpret_cast<const uint4*>(src + row * HD + 2 * W * wg);
+#pragma unroll
+                for (int v4 = 0; v4 < W / 4; ++v4) {
+                    const uint4 x = t < a.T ? __ldg(p4 + v4) : make_uint4(0u, 0u, 0u, 0u);
+                    u[4 * v4] = x.x;
+                    u[4 * v4 + 1] = x.y;
+                    u[4 * v4 + 2] = x.z;
+                    u[4 * v4 + 3] = x.w;
+                }
+                tmem_st<W>(trow + col + W * wg, u);
+            };
+            fill(q, TM_Q);
+            fill(gf, TM_GF);
+            fill(gs, TM_GS);
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(BAR(B_OPS));
+        }
         const float my_lse2 = a.lse2[row], my_df = a.Df[row], my_ds = a.Ds[row];
         const uint32_t* myrow = (r < 64 || a.block == 128 || ragged1) ? mrow : mrow + kMaxWords;
         const float sl2 = a.scale_log2;
-        const int c0 = 32 * wg;
-        bool ok = true;
+        const int c0 = COLS * wg;
+        const uint32_t rowoff = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
+        auto wait = [&](int bar, uint32_t parity) {
+            const bool r2 = __all_sync(FULL, mbar_wait(BAR(bar), parity, abort_flag, status, lim));
+            fence_after_sync();
+            return r2;
+        };
         for (int i = 0; i < ns; ++i) {
             const int b = i & 1;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(BAR(B_READY + b), (i >> 1) & 1, abort_flag, status, lim))) {
+            if (!wait(B_SREADY, i & 1)) {
                 ok = false;
                 break;
             }
-            fence_after_sync();
-            const bool sp = sparse(i);
-            const bool use_s = sp && bit(myrow, step_kb(i));
             const int k0 = STEP * i + c0;
-            const bool diag = k0 + 31 > t0;
-            const uint32_t sbuf = trow + (b ? TM_S1 : TM_S0);
-            const uint32_t dp = trow + (b ? TM_DP1 : TM_DP0);
-            uint32_t su[32], fu[32], pu[32];
-            tmem_ld32(sbuf + c0, su);
-            tmem_ld32(dp + c0, fu);
-            if (use_s) tmem_ld32(dp + 64 + c0, pu);  // warp-uniform: one query block per warp
-            tmem_wait_ld();
-            uint32_t dsk[16];
+            const bool diag = k0 + COLS - 1 > t0;
+            float pf[COLS];
+            {
+                uint32_t su[COLS];
+                tmem_ld<COLS>(trow + TM_S + c0, su);
+                tmem_wait_ld();
+                fence_before_sync();
+                mbar_arrive(BAR(B_SFREE));  // S may now be overwritten by the next step
 #pragma unroll
-            for (int j2 = 0; j2 < 16; ++j2) {
+                for (int j = 0; j < COLS; ++j) {
+                    pf[j] = ex2(fmaf(__uint_as_float(su[j]), sl2, -my_lse2));
+                    if (diag && k0 + j > t) pf[j] = 0.f;
+                }
+            }
+            const bool use_s = sparse(i) && bit(myrow, step_kb(i));  // warp-uniform
+            if (!wait(B_PREADY, i & 1)) {
+                ok = false;
+                break;
+            }
+            uint32_t fu[COLS], pu[COLS];
+            tmem_ld<COLS>(trow + TM_DPF + c0, fu);
+            if (use_s) tmem_ld<COLS>(trow + TM_DPS + c0, pu);
+            tmem_wait_ld();
+            fence_before_sync();
+            mbar_arrive(BAR(B_PFREE));  // dP may now be overwritten by the next step
+            uint32_t dsk[COLS / 2];
+#pragma unroll
+            for (int j2 = 0; j2 < COLS / 2; ++j2) {
                 float ds2[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int j = 2 * j2 + h;
-                    float pf = ex2(fmaf(__uint_as_float(su[j]), sl2, -my_lse2));
-                    if (diag && k0 + j > t) pf = 0.f;
                     float g = __uint_as_float(fu[j]) - my_df;
                     if (use_s) g += __uint_as_float(pu[j]) - my_ds;
-                    ds2[h] = pf * g;
+                    ds2[h] = pf[j] * g;
                 }
                 dsk[j2] = pack_bf16_alu(ds2[0], ds2[1]);
             }
-            tmem_st<16>(sbuf + c0, dsk);  // dS (bf16) over this warpgroup's consumed S columns
-            tmem_wait_st();
-            fence_before_sync();
-            mbar_arrive(BAR(B_PREADY + b));
+            // dS row r into buffer b once the dQ MMAs of step i-2 have read it
+            if (i >= 2 && !wait(B_DSFREE + b, ((i >> 1) + 1) & 1)) {
+                ok = false;
+                break;
+            }
+            uint8_t* dsb = gbase + OFF_DS + b * DS_BYTES + rowoff;
+#pragma unroll
+            for (int q4 = 0; q4 < COLS / 8; ++q4) {
+                const uint32_t chunk = (uint32_t)((c0 >> 3) + q4) ^ (uint32_t)(r & 7);
+                *reinterpret_cast<uint4*>(dsb + chunk * 16) =
+                    make_uint4(dsk[4 * q4], dsk[4 * q4 + 1], dsk[4 * q4 + 2], dsk[4 * q4 + 3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the MMAs
+            mbar_arrive(BAR(B_DSREADY + b));
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim));
+        if (ok) ok = wait(B_DONE, 0);
         if (ok) {
-            fence_after_sync();
+            constexpr int OC = HD / NWG;  // output columns per warpgroup
             const bool valid = t < a.T;
-            store_row_cols<2>(trow + TM_DQ + 64 * wg, a.sm_scale,
-                           a.dq + (valid ? row : rowbase) * HD + 64 * wg, valid);
+            store_row_cols<OC / 32>(trow + TM_DQ + OC * wg, a.sm_scale,
+                                    a.dq + (valid ? row : rowbase) * HD + OC * wg, valid);
         }
     }
     fence_before_sync();
@@ -925,13 +1005,14 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     int st = check_launch("bwd_tc_pre_kernel");
     if (st != SSA_OK) return st;
 
-    CUtensorMap k128, v128, q64, gf64, gs64, q128, gf128, gs128, k64, v64;
-    const void* srcs[5] = {q, k, v, w.gf, w.gs};
-    CUtensorMap* m128[5] = {&q128, &k128, &v128, &gf128, &gs128};
-    CUtensorMap* m64[5] = {&q64, &k64, &v64, &gf64, &gs64};
-    for (int i = 0; i < 5 && st == SSA_OK; ++i) {
-        st = make_map(m128[i], srcs[i], BH, p.T, TILE);
-        if (st == SSA_OK) st = make_map(m64[i], srcs[i], BH, p.T, STEP);
+    CUtensorMap k128, v128, q64, gf64, gs64, k64, v64;
+    {
+        const void* srcs[5] = {k, v, q, w.gf, w.gs};
+        CUtensorMap* maps[5] = {&k128, &v128, &q64, &gf64, &gs64};
+        const int rows[5] = {TILE, TILE, STEP, STEP, STEP};
+        for (int i = 0; i < 5 && st == SSA_OK; ++i) st = make_map(maps[i], srcs[i], BH, p.T, rows[i]);
+        if (st == SSA_OK) st = make_map(&k64, k, BH, p.T, STEP);
+        if (st == SSA_OK) st = make_map(&v64, v, BH, p.T, STEP);
     }
     if (st != SSA_OK) return st;
 
@@ -968,7 +1049,8 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     bwd_dkdv_tc_kernel<<<grid, kv::kThr, kv::SMEM_BYTES, s>>>(k128, v128, q64, gf64, gs64, a);
     st = check_launch("bwd_dkdv_tc_kernel");
     if (st != SSA_OK) return st;
-    bwd_dq_tc_kernel<<<grid, kThreads, qk::SMEM_BYTES, s>>>(q128, gf128, gs128, k64, v64, a);
+    bwd_dq_tc_kernel<<<grid, qk::kThr, qk::SMEM_BYTES, s>>>(
+        k64, v64, static_cast<const __nv_bfloat16*>(q), w.gf, w.gs, a);
     return check_launch("bwd_dq_tc_kernel");
 }
 
