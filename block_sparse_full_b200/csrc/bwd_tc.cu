@@ -49,8 +49,6 @@ using namespace tc;
 constexpr int HD = 128;
 constexpr int TILE = 128;  // keys per dK/dV CTA, queries per dQ CTA
 constexpr int STEP = 64;   // queries per dK/dV step, keys per dQ step
-constexpr int kMaxWords = 128;  // mask words per query block: n <= 4096 blocks
-constexpr int kMaxBlocks = kMaxWords * 32;
 constexpr uint32_t BOX_T = TILE * 128;  // [128 rows x 64 d] bf16 = 16 KB
 constexpr uint32_t BOX_S = STEP * 128;  // [64 rows x 64 d] bf16 = 8 KB
 constexpr uint32_t TILE_BYTES = 2 * BOX_T;
@@ -68,6 +66,7 @@ struct BwdArgs {
     const float* Ds;    // D_s of the c_t-scaled G_s
     const uint32_t* mask;
     int BH, T, block, words, n_blocks;
+    int ds_blocks;  // dS^T blocks per (batch, head): one per (key tile, 64-query step)
     float scale_log2;  // sigma * log2(e)
     float sm_scale;
     unsigned long long timeout_ns;
@@ -217,23 +216,30 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
 #define SSA_KV_WARPGROUPS 2
 #endif
 namespace kv {
+// K stays in shared memory (A of S^T = K Q^T), V lives in TMEM (A of the dP^T
+// MMAs, TS form); Q, G_f, G_s' steps stream through a ring.  The compute
+// warps write P^T (and, on mixed steps, the sparse stream's row-masked copy)
+// and dS^T as swizzled bf16 tiles in shared memory: the A operands of
+// dV += P^T G and dK += dS^T Q.  S^T and dP^T are handed over separately as
+// soon as they have been read into registers.
 constexpr int NWG = SSA_KV_WARPGROUPS;  // compute warpgroups; each owns COLS query columns of a step
 static_assert(NWG == 2 || NWG == 4, "2 or 4 compute warpgroups");
 constexpr int COLS = STEP / NWG;
 constexpr int kThr = 128 + 128 * NWG;  // warp 0 TMA, 1 MMA, 2-3 idle, then the compute warps
 constexpr int kComp = 128 * NWG;
 constexpr uint32_t OFF_K = 0;
-constexpr uint32_t OFF_V = TILE_BYTES;
-constexpr uint32_t OFF_STAGE = 2 * TILE_BYTES;
+constexpr uint32_t OFF_STAGE = TILE_BYTES;
 constexpr uint32_t ST_Q = 0, ST_GF = STEP_BYTES, ST_GS = 2 * STEP_BYTES;
 constexpr uint32_t STAGE_BYTES = 3 * STEP_BYTES;
 constexpr int NSTAGE = 3;
-// dS^T of the current step, bf16 [128 keys x 64 queries], K-major with
-// 128-byte swizzle: the A operand of dK += dS^T Q
-constexpr uint32_t OFF_DS = OFF_STAGE + NSTAGE * STAGE_BYTES;
+// bf16 [128 keys x 64 queries] tiles, K-major with 128-byte swizzle
+constexpr uint32_t T_BYTES = 128 * 128;
+constexpr uint32_t OFF_DS = OFF_STAGE + NSTAGE * STAGE_BYTES;  // dS^T
+constexpr uint32_t OFF_PT = OFF_DS + T_BYTES;                  // P_f^T
+constexpr uint32_t OFF_PST = OFF_PT + T_BYTES;                 // P_s^T on mixed steps
 // per stage, fp32 over the step's 64 queries: lse_full*log2(e) | D_f | D_s
 constexpr uint32_t ROW_BYTES = 3 * STEP * 4;
-constexpr uint32_t OFF_ROWS = OFF_DS + 128 * 128;
+constexpr uint32_t OFF_ROWS = OFF_PST + T_BYTES;
 constexpr uint32_t OFF_BAR = OFF_ROWS + NSTAGE * ROW_BYTES;
 // TMEM slot, abort flag, then one selection word per stage (bit 0: the step's
 // query block selects key block kb0, bit 1: selects kb1)
@@ -241,26 +247,26 @@ constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 32;
 static_assert(SMEM_BYTES <= 232448, "227 KB of shared memory per CTA");
 enum : int {  // barrier indices, derived from the ring depth
-    B_KV = 0, B_FULL = 1, B_EMPTY = B_FULL + NSTAGE, B_READY = B_EMPTY + NSTAGE,
-    B_PREADY = B_READY + 1, B_DONE = B_PREADY + 1, B_DRAIN = B_DONE + 1,
-    B_DPFREE = B_DRAIN + 1,  // compute has loaded dP_f^T / dP_s^T of the step (the buffers may be refilled)
-    B_DSFREE = B_DPFREE + 1,  // the dK MMAs have read the dS^T tile in shared memory
-    B_COUNT = B_DSFREE + 1
+    B_FULL = 0, B_EMPTY = B_FULL + NSTAGE,
+    B_K = B_EMPTY + NSTAGE,  // K tile landed
+    B_OPS = B_K + 1,         // V is in TMEM
+    B_SREADY = B_OPS + 1,    // S^T of the step is in TMEM
+    B_PREADY = B_SREADY + 1, // dP_f^T, dP_s^T of the step are in TMEM
+    B_SFREE = B_PREADY + 1,  // the compute warps have read S^T (may be overwritten)
+    B_PFREE = B_SFREE + 1,   // ... and dP^T
+    B_TREADY = B_PFREE + 1,  // P^T / P_s^T / dS^T tiles written
+    B_TFREE = B_TREADY + 1,  // ... and read by the dV / dK MMAs and the dS^T store
+    B_DONE = B_TFREE + 1, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
 };
 static_assert(B_COUNT <= 16, "barrier area holds 16");
-constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_S0 = 256, TM_S1 = 320, TM_DPF = 384, TM_DPS = 448;
-// bf16 P^T written by warpgroup w over the first COLS/2 of its own COLS fp32
-// S columns; the masked copy for the sparse stream follows at +COLS/2.
-// TMEM column of the A operand's k-step kk (16 queries):
-__device__ __forceinline__ uint32_t acol(int kk) {
-    return (uint32_t)(COLS * ((16 * kk) / COLS) + ((16 * kk) % COLS) / 2);
-}
+constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_S = 256, TM_V = 320, TM_DPF = 384, TM_DPS = 448;
 }  // namespace kv
 
 __global__ void __launch_bounds__(kv::kThr, 1)
-bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_gf,
-                   const __grid_constant__ CUtensorMap tm_gs, const BwdArgs a) {
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_gf, const __grid_constant__ CUtensorMap tm_gs,
+                   const __grid_constant__ CUtensorMap tm_ds, const __nv_bfloat16* __restrict__ v,
+                   const BwdArgs a) {
     using namespace kv;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t base = smem_u32(smem_raw);
@@ -287,19 +293,24 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int kb1 = (s0 + 64 < a.T) ? (s0 + 64) / a.block : kb0;
     auto BAR = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
     const size_t rowbase = (size_t)bh * a.T;
+    // first dS^T block of this key tile: tiles J' < J hold (T - 128 J') / 64 blocks each
+    const int ds_blk0 = bh * a.ds_blocks + J * (a.T / STEP) - J * (J - 1);
 
     if (threadIdx.x == 0) {
-        mbar_init(BAR(B_KV), 1);
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(BAR(B_FULL + s), 1);
             mbar_init(BAR(B_EMPTY + s), 1);
         }
-        mbar_init(BAR(B_READY), 1);
-        mbar_init(BAR(B_PREADY), kComp);
+        mbar_init(BAR(B_K), 1);
+        mbar_init(BAR(B_OPS), kComp);
+        mbar_init(BAR(B_SREADY), 1);
+        mbar_init(BAR(B_PREADY), 1);
+        mbar_init(BAR(B_SFREE), kComp);
+        mbar_init(BAR(B_PFREE), kComp);
+        mbar_init(BAR(B_TREADY), kComp);
+        mbar_init(BAR(B_TFREE), 2);  // MMA commit + the dS^T store's source read
         mbar_init(BAR(B_DONE), 1);
         mbar_init(BAR(B_DRAIN), 1);
-        mbar_init(BAR(B_DPFREE), kComp);
-        mbar_init(BAR(B_DSFREE), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -313,19 +324,22 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const uint32_t tmem = *tmem_slot;
 
     const unsigned FULL = 0xffffffffu;
+    auto wait = [&](int bar, uint32_t parity) {
+        const bool r = __all_sync(FULL, mbar_wait(BAR(bar), parity, abort_flag, status, lim));
+        fence_after_sync();
+        return r;
+    };
     if (warp == 0) {
         // -------------------------------------------- TMA producer (whole warp)
         if (elect_one()) {
             prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_gf);
             prefetch_tmap(&tm_gs);
-            mbar_expect_tx(BAR(B_KV), 2 * TILE_BYTES);
-            tma_load_3d(base + OFF_K, &tm_k, BAR(B_KV), 0, s0, bh);
-            tma_load_3d(base + OFF_K + BOX_T, &tm_k, BAR(B_KV), 64, s0, bh);
-            tma_load_3d(base + OFF_V, &tm_v, BAR(B_KV), 0, s0, bh);
-            tma_load_3d(base + OFF_V + BOX_T, &tm_v, BAR(B_KV), 64, s0, bh);
+            prefetch_tmap(&tm_ds);
+            mbar_expect_tx(BAR(B_K), TILE_BYTES);
+            tma_load_3d(base + OFF_K, &tm_k, BAR(B_K), 0, s0, bh);
+            tma_load_3d(base + OFF_K + BOX_T, &tm_k, BAR(B_K), 64, s0, bh);
         }
         __syncwarp();
         int issued[NSTAGE];
@@ -362,7 +376,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             __syncwarp();
             issued[s] = i;
         }
-        wait_drain(BAR(B_KV), 0, kDrainLimitNs);
+        wait_drain(BAR(B_K), 0, kDrainLimitNs);
         if (*abort_flag)
             for (int s = 0; s < NSTAGE; ++s)
                 if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
@@ -373,415 +387,71 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S^T, dP^T
             constexpr uint32_t id_a = idesc_bf16_f32(TILE, HD, true);     // dV, dK
             const uint64_t kdesc = smem_desc_sw128(base + OFF_K, 16, 1024);
-            const uint64_t vdesc = smem_desc_sw128(base + OFF_V, 16, 1024);
             const uint64_t st_k0 = smem_desc_sw128(base + OFF_STAGE, 16, 1024);      // K-major
             const uint64_t st_m0 = smem_desc_sw128(base + OFF_STAGE, BOX_S, 1024);   // MN-major
+            const uint64_t dsd = smem_desc_sw128(base + OFF_DS, 16, 1024);           // K-major A
+            const uint64_t ptd = smem_desc_sw128(base + OFF_PT, 16, 1024);
+            const uint64_t pstd = smem_desc_sw128(base + OFF_PST, 16, 1024);
             auto kq = [](int kk) { return (uint32_t)((kk >> 2) * BOX_T + (kk & 3) * 32); };
             auto ks = [](int kk) { return (uint32_t)((kk >> 2) * BOX_S + (kk & 3) * 32); };
-            bool ok = __all_sync(FULL, mbar_wait(BAR(B_KV), 0, abort_flag, status, lim));
-            auto issue_s = [&](int i) {  // elected lane only
+            auto issue_s = [&](int i) {  // S^T = K Q^T
                 const uint64_t qd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_Q);
-                const uint32_t d = tmem + ((i & 1) ? TM_S1 : TM_S0);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(d, desc_add(kdesc, kq(kk)), desc_add(qd, ks(kk)), id_s, kk > 0);
-            };
-            auto issue_dp = [&](int i, bool sp) {  // elected lane only
-                const uint64_t gfd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_GF);
-                const uint64_t gsd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_GS);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmem + TM_DPF, desc_add(vdesc, kq(kk)), desc_add(gfd, ks(kk)), id_s, kk > 0);
-                if (sp) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + TM_DPS, desc_add(vdesc, kq(kk)), desc_add(gsd, ks(kk)), id_s, kk > 0);
-                }
-            };
-            if (ok && ns > 0) {
-                ok = __all_sync(FULL, mbar_wait(BAR(B_FULL), 0, abort_flag, status, lim));
-                if (ok) {
-                    fence_after_sync();
-                    const bool sp0 = flags[0] != 0u;
-                    if (elect_one()) {
-                        issue_s(0);
-                        issue_dp(0, sp0);
-                        mma_commit(BAR(B_READY));
-                    }
-                    __syncwarp();
-                }
-            }
-            const uint64_t dsd = smem_desc_sw128(base + OFF_DS, 16, 1024);  // K-major A
-            for (int i = 0; ok && i < ns; ++i) {
-                const int s = i % NSTAGE, b = i & 1;
-                if (i + 1 < ns) {
-                    // S^T of the next step: its buffer's P_f^T was read by dV of step i-1
-                    if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + (i + 1) % NSTAGE), ((i + 1) / NSTAGE) & 1,
-                                                    abort_flag, status, lim))) {
-                        ok = false;
-                        break;
-                    }
-                    fence_after_sync();
-                    if (elect_one()) issue_s(i + 1);
-                    __syncwarp();
-                    // dP^T of the next step as soon as the compute warps have loaded this one's
-                    if (!__all_sync(FULL, mbar_wait(BAR(B_DPFREE), i & 1, abort_flag, status, lim))) {
-                        ok = false;
-                        break;
-                    }
-                    fence_after_sync();
-                    const bool sp_next = flags[(i + 1) % NSTAGE] != 0u;
-                    if (elect_one()) {
-                        issue_dp(i + 1, sp_next);
-                        mma_commit(BAR(B_READY));
-                    }
-                    __syncwarp();
-                }
-                if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY), i & 1, abort_flag, status, lim))) {
-                    ok = false;
-                    break;
-                }
-                fence_after_sync();
-                const uint32_t sb = tmem + (b ? TM_S1 : TM_S0);
-                const uint64_t gfm = desc_add(st_m0, s * STAGE_BYTES + ST_GF);
-                const uint64_t gsm = desc_add(st_m0, s * STAGE_BYTES + ST_GS);
-                const uint64_t qm = desc_add(st_m0, s * STAGE_BYTES + ST_Q);
-                const uint32_t fl = flags[s];
-                // P_s^T = P_f^T on selected key rows (c_t is folded into G_s); the
-                // masked copy is needed only when the tile's two key blocks differ
-                const uint32_t ps_off = (fl == 1u || fl == 2u) ? (uint32_t)(COLS / 2) : 0u;
-                if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // dV += P_f^T G_f  (P_f^T in TMEM)
-                        mma_ts(tmem + TM_DV, sb + acol(kk), desc_add(gfm, kk * 2048), id_a,
-                               (i > 0 || kk > 0) ? 1u : 0u);
-                    if (fl != 0u) {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)  // dV += P_s^T G_s
-                            mma_ts(tmem + TM_DV, sb + acol(kk) + ps_off, desc_add(gsm, kk * 2048), id_a,
-                                   1u);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // dK += dS^T Q  (dS^T in smem)
-                        mma_ss(tmem + TM_DK, desc_add(dsd, kk * 32), desc_add(qm, kk * 2048), id_a,
-                               (i > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(BAR(B_EMPTY + s));
-                    mma_commit(BAR(B_DSFREE));
-                }
-                __syncwarp();
-            }
-            if (elect_one()) {
-                mma_commit(BAR(B_DONE));
-                mma_commit(BAR(B_DRAIN));
-            }
-            __syncwarp();
-            wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
-        }
-    } else if (warp >= 4) {
-        // ------------------------------------------ compute warpgroups
-        // warpgroup wg handles query columns [COLS wg, COLS wg + COLS) of every step
-        const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
-        const int r = sw * 32 + lane;  // key row of the tile == TMEM lane
-        const int s_tok = s0 + r;
-        const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
-        const float sl2 = a.scale_log2;
-        const bool in_kb1 = r >= 64 && a.block == 64;  // warp-uniform
-        const int c0 = COLS * wg;
-        bool ok = true;
-        for (int i = 0; i < ns; ++i) {
-            const int t0 = s0 + STEP * i;
-            const int s = i % NSTAGE, b = i & 1;
-            // the stage's row vectors and selection word (already landed: the MMA
-            // warp waited for them before issuing this step's S^T)
-            if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + s), (i / NSTAGE) & 1, abort_flag, status, lim)) ||
-                !__all_sync(FULL, mbar_wait(BAR(B_READY), i & 1, abort_flag, status, lim))) {
-                ok = false;
-                break;
-            }
-            fence_after_sync();
-            const uint32_t fl = flags[s];
-            const bool use_s = in_kb1 ? (fl >> 1) & 1u : fl & 1u;
-            const bool mixed = fl == 1u || fl == 2u;
-            const bool diag = t0 < s0 + TILE;
-            const uint32_t sbuf = trow + (b ? TM_S1 : TM_S0);
-            uint32_t su[COLS], fu[COLS], pu[COLS];
-            tmem_ld<COLS>(sbuf + c0, su);
-            tmem_ld<COLS>(trow + TM_DPF + c0, fu);
-            if (use_s) tmem_ld<COLS>(trow + TM_DPS + c0, pu);
-            tmem_wait_ld();
-            fence_before_sync();
-            mbar_arrive(BAR(B_DPFREE));  // dP_f^T / dP_s^T may now be overwritten
-            const float4* L4 = reinterpret_cast<const float4*>(rows_s + s * (3 * STEP) + c0);
-            const float4* F4 = reinterpret_cast<const float4*>(rows_s + s * (3 * STEP) + STEP + c0);
-            const float4* S4 = reinterpret_cast<const float4*>(rows_s + s * (3 * STEP) + 2 * STEP + c0);
-            uint32_t pfk[COLS / 2], dsk[COLS / 2];
-#pragma unroll
-            for (int j4 = 0; j4 < COLS / 4; ++j4) {
-                const float4 L = L4[j4], F = F4[j4];
-                const float4 S = use_s ? S4[j4] : make_float4(0.f, 0.f, 0.f, 0.f);
-                const float lv[4] = {L.x, L.y, L.z, L.w}, fv[4] = {F.x, F.y, F.z, F.w};
-                const float sv[4] = {S.x, S.y, S.z, S.w};
-                float pf[4], ds[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int j = 4 * j4 + h;
-                    float p = ex2(fmaf(__uint_as_float(su[j]), sl2, -lv[h]));
-                    if (diag && t0 + c0 + j < s_tok) p = 0.f;
-                    float g = __uint_as_float(fu[j]) - fv[h];
-                    if (use_s) g += __uint_as_float(pu[j]) - sv[h];
-                    pf[h] = p;
-                    ds[h] = p * g;
-                }
-                pfk[2 * j4] = pack_bf16_alu(pf[0], pf[1]);
-                pfk[2 * j4 + 1] = pack_bf16_alu(pf[2], pf[3]);
-                dsk[2 * j4] = pack_bf16_alu(ds[0], ds[1]);
-                dsk[2 * j4 + 1] = pack_bf16_alu(ds[2], ds[3]);
-            }
-            // dS^T goes to shared memory, row r of a 128B-swizzled K-major tile,
-            // once the previous step's dK MMAs have read it
-            if (i > 0 && !__all_sync(FULL, mbar_wait(BAR(B_DSFREE), (i - 1) & 1, abort_flag, status, lim))) {
-                ok = false;
-                break;
-            }
-            // P_f^T (bf16) over this warpgroup's own consumed S columns; on a
-            // mixed step the sparse stream's copy, zero on unselected key rows
-            tmem_st<COLS / 2>(sbuf + c0, pfk);
-            if (mixed) {
-                if (!use_s)
-#pragma unroll
-                    for (int e = 0; e < COLS / 2; ++e) pfk[e] = 0u;
-                tmem_st<COLS / 2>(sbuf + c0 + COLS / 2, pfk);
-            }
-            {
-                const uint32_t rowoff = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
-#pragma unroll
-                for (int q4 = 0; q4 < COLS / 8; ++q4) {
-                    const uint32_t chunk = (uint32_t)((c0 >> 3) + q4) ^ (uint32_t)(r & 7);
-                    *reinterpret_cast<uint4*>(gbase + OFF_DS + rowoff + chunk * 16) =
-                        make_uint4(dsk[4 * q4], dsk[4 * q4 + 1], dsk[4 * q4 + 2], dsk[4 * q4 + 3]);
-                }
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the MMAs
-            tmem_wait_st();
-            fence_before_sync();
-            mbar_arrive(BAR(B_PREADY));
-        }
-        if (ok) ok = __all_sync(FULL, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim));
-        if (ok) {
-            fence_after_sync();
-            const bool valid = s_tok < a.T;
-            const size_t row = rowbase + (valid ? s_tok : 0);
-            constexpr int OC = HD / NWG;  // output columns per warpgroup
-            store_row_cols<OC / 32>(trow + TM_DV + OC * wg, 1.f, a.dv + row * HD + OC * wg, valid);
-            store_row_cols<OC / 32>(trow + TM_DK + OC * wg, a.sm_scale, a.dk + row * HD + OC * wg, valid);
-        }
-    }
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 1) {
-        fence_after_sync();
-        tmem_dealloc(tmem, 512);
-    }
-}
-
-// ============================================================ dQ
-#ifndef SSA_DQ_WARPGROUPS
-#define SSA_DQ_WARPGROUPS 2
-#endif
-namespace qk {
-// K/V steps stream through a ring; Q, G_f, G_s' of the tile live in TMEM as the
-// A operands of S, dP_f, dP_s (TS form: only the 64-key B tile is read from
-// shared memory); dS goes to a double-buffered shared tile for dQ += dS K.
-// S and dP are handed over separately: the next step's S MMAs start once the
-// compute warps have read this step's S, while they still wait for its dP.
-constexpr int NWG = SSA_DQ_WARPGROUPS;  // compute warpgroups; each owns COLS key columns of a step
-static_assert(NWG == 2 || NWG == 4, "2 or 4 compute warpgroups");
-constexpr int COLS = STEP / NWG;
-constexpr int kThr = 128 + 128 * NWG;
-constexpr int kComp = 128 * NWG;
-constexpr int NSTAGE = 5;
-constexpr uint32_t ST_K = 0, ST_V = STEP_BYTES;
-constexpr uint32_t STAGE_BYTES = 2 * STEP_BYTES;
-constexpr uint32_t OFF_STAGE = 0;
-// dS, bf16 [128 queries x 64 keys], K-major with 128-byte swizzle, x2
-constexpr uint32_t DS_BYTES = 128 * 128;
-constexpr uint32_t OFF_DS = OFF_STAGE + NSTAGE * STAGE_BYTES;
-constexpr uint32_t OFF_BAR = OFF_DS + 2 * DS_BYTES;
-constexpr int NBAR = 24;
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr uint32_t OFF_MASK = OFF_MISC + 16;
-constexpr uint32_t SMEM_BYTES = OFF_MASK + 2 * kMaxWords * 4 + 1024;
-static_assert(SMEM_BYTES <= 232448, "227 KB of shared memory per CTA");
-enum : int {  // barrier indices, derived from the ring depth
-    B_FULL = 0, B_EMPTY = B_FULL + NSTAGE,
-    B_OPS = B_EMPTY + NSTAGE,  // Q, G_f, G_s' are in TMEM
-    B_SREADY = B_OPS + 1,      // S of the step is in TMEM
-    B_PREADY = B_SREADY + 1,   // dP_f, dP_s of the step are in TMEM
-    B_SFREE = B_PREADY + 1,    // the compute warps have read S (may be overwritten)
-    B_PFREE = B_SFREE + 1,     // ... and dP
-    B_DSREADY = B_PFREE + 1,   // x2: dS buffer written
-    B_DSFREE = B_DSREADY + 2,  // x2: dS buffer read by the dQ MMAs
-    B_DONE = B_DSFREE + 2, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
-};
-static_assert(B_COUNT <= NBAR, "barrier area");
-constexpr uint32_t TM_DQ = 0, TM_S = 128, TM_DPF = 192, TM_DPS = 256;
-constexpr uint32_t TM_Q = 320, TM_GF = 384, TM_GS = 448;  // bf16 A operands, 64 cols each
-}  // namespace qk
-
-__global__ void __launch_bounds__(qk::kThr, 1)
-bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gf,
-                 const __nv_bfloat16* __restrict__ gs, const BwdArgs a) {
-    using namespace qk;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* gbase = smem_raw + (base - raw);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
-    uint32_t* mrow = reinterpret_cast<uint32_t*>(gbase + OFF_MASK);
-    unsigned int* status = &g_bwd_tc_status;
-    const uint64_t lim = a.timeout_ns;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ntq = (a.T + TILE - 1) / TILE;
-    const int I = ntq - 1 - (int)(blockIdx.x / a.BH);  // longest rows first
-    const int bh = (int)(blockIdx.x % a.BH);
-    const int t0 = I * TILE;
-    const int last = min(t0 + TILE, a.T);      // keys needed: [0, last)
-    const int ns = (last + STEP - 1) / STEP;
-    const bool ragged1 = t0 + 64 >= a.T;
-    const int qb0 = t0 / a.block;
-    const int qb1 = ragged1 ? qb0 : (t0 + 64) / a.block;
-    auto BAR = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
-    const size_t rowbase = (size_t)bh * a.T;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < NSTAGE; ++s) {
-            mbar_init(BAR(B_FULL + s), 1);
-            mbar_init(BAR(B_EMPTY + s), 1);
-        }
-        mbar_init(BAR(B_OPS), kComp);
-        mbar_init(BAR(B_SREADY), 1);
-        mbar_init(BAR(B_PREADY), 1);
-        mbar_init(BAR(B_SFREE), kComp);
-        mbar_init(BAR(B_PFREE), kComp);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(BAR(B_DSREADY + b), kComp);
-            mbar_init(BAR(B_DSFREE + b), 1);
-        }
-        mbar_init(BAR(B_DONE), 1);
-        mbar_init(BAR(B_DRAIN), 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    {
-        const uint32_t* m0 = a.mask + ((size_t)bh * a.n_blocks + qb0) * a.words;
-        const uint32_t* m1 = a.mask + ((size_t)bh * a.n_blocks + qb1) * a.words;
-        for (int w = threadIdx.x; w < a.words; w += kThr) {
-            mrow[w] = m0[w];
-            mrow[kMaxWords + w] = m1[w];
-        }
-    }
-    if (warp == 1) {
-        tmem_alloc(base + OFF_MISC, 512);
-        tmem_relinquish();
-    }
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
-    // key block of step i and whether either query block selects it
-    auto step_kb = [&](int i) { return (STEP * i) / a.block; };
-    auto sparse = [&](int i) {
-        const int kb = step_kb(i);
-        return bit(mrow, kb) || bit(mrow + kMaxWords, kb);
-    };
-
-    const unsigned FULL = 0xffffffffu;
-    if (warp == 0) {
-        // -------------------------------------------- TMA producer (whole warp)
-        if (elect_one()) {
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-        }
-        __syncwarp();
-        int issued[NSTAGE];
-        for (int s = 0; s < NSTAGE; ++s) issued[s] = -1;
-        for (int i = 0; i < ns; ++i) {
-            const int s = i % NSTAGE;
-            if (i >= NSTAGE &&
-                !__all_sync(FULL, mbar_wait(BAR(B_EMPTY + s), ((i / NSTAGE) + 1) & 1, abort_flag, status,
-                                            lim)))
-                break;
-            const uint32_t st = base + OFF_STAGE + s * STAGE_BYTES;
-            if (elect_one()) {
-                mbar_expect_tx(BAR(B_FULL + s), 2 * STEP_BYTES);
-                tma_load_3d(st + ST_K, &tm_k, BAR(B_FULL + s), 0, STEP * i, bh);
-                tma_load_3d(st + ST_K + BOX_S, &tm_k, BAR(B_FULL + s), 64, STEP * i, bh);
-                tma_load_3d(st + ST_V, &tm_v, BAR(B_FULL + s), 0, STEP * i, bh);
-                tma_load_3d(st + ST_V + BOX_S, &tm_v, BAR(B_FULL + s), 64, STEP * i, bh);
-            }
-            __syncwarp();
-            issued[s] = i;
-        }
-        if (*abort_flag)
-            for (int s = 0; s < NSTAGE; ++s)
-                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
-    } else if (warp == 1) {
-        {  // ------------------------------------------ MMA issuer (whole warp)
-            constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S, dP
-            constexpr uint32_t id_q = idesc_bf16_f32(TILE, HD, true);     // dQ
-            const uint64_t st_k0 = smem_desc_sw128(base + OFF_STAGE, 16, 1024);      // K-major
-            const uint64_t st_m0 = smem_desc_sw128(base + OFF_STAGE, BOX_S, 1024);   // MN-major
-            const uint64_t ds_0 = smem_desc_sw128(base + OFF_DS, 16, 1024);          // K-major A
-            auto ks = [](int kk) { return (uint32_t)((kk >> 2) * BOX_S + (kk & 3) * 32); };
-            auto wait = [&](int bar, uint32_t parity) {
-                const bool r = __all_sync(FULL, mbar_wait(BAR(bar), parity, abort_flag, status, lim));
-                fence_after_sync();
-                return r;
-            };
-            auto issue_s = [&](int i) {  // S = Q K^T
-                const uint64_t kd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_K);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + TM_S, tmem + TM_Q + 8 * kk, desc_add(kd, ks(kk)), id_s, kk > 0);
+                        mma_ss(tmem + TM_S, desc_add(kdesc, kq(kk)), desc_add(qd, ks(kk)), id_s, kk > 0);
                     mma_commit(BAR(B_SREADY));
                 }
                 __syncwarp();
             };
-            auto issue_dp = [&](int i) {  // dP_f = G_f V^T, dP_s = G_s' V^T
-                const uint64_t vd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_V);
-                const bool sp = sparse(i);
+            auto issue_dp = [&](int i) {  // dP_f^T = V G_f^T, dP_s^T = V G_s'^T (V in TMEM)
+                const uint32_t s = i % NSTAGE;
+                const uint64_t gfd = desc_add(st_k0, s * STAGE_BYTES + ST_GF);
+                const uint64_t gsd = desc_add(st_k0, s * STAGE_BYTES + ST_GS);
+                const bool sp = flags[s] != 0u;
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + TM_DPF, tmem + TM_GF + 8 * kk, desc_add(vd, ks(kk)), id_s, kk > 0);
+                        mma_ts(tmem + TM_DPF, tmem + TM_V + 8 * kk, desc_add(gfd, ks(kk)), id_s, kk > 0);
                     if (sp) {
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk)
-                            mma_ts(tmem + TM_DPS, tmem + TM_GS + 8 * kk, desc_add(vd, ks(kk)), id_s,
+                            mma_ts(tmem + TM_DPS, tmem + TM_V + 8 * kk, desc_add(gsd, ks(kk)), id_s,
                                    kk > 0);
                     }
                     mma_commit(BAR(B_PREADY));
                 }
                 __syncwarp();
             };
-            auto issue_dq = [&](int j) {  // dQ += dS_j K_j, then release stage and dS buffer
-                const uint64_t km = desc_add(st_m0, (j % NSTAGE) * STAGE_BYTES + ST_K);
-                const uint64_t dd = desc_add(ds_0, (j & 1) * DS_BYTES);
+            auto issue_acc = [&](int i) {  // dV += P_f^T G_f + P_s^T G_s', dK += dS^T Q
+                const uint32_t s = i % NSTAGE;
+                const uint64_t gfm = desc_add(st_m0, s * STAGE_BYTES + ST_GF);
+                const uint64_t gsm = desc_add(st_m0, s * STAGE_BYTES + ST_GS);
+                const uint64_t qm = desc_add(st_m0, s * STAGE_BYTES + ST_Q);
+                const uint32_t fl = flags[s];
+                // P_s^T = P_f^T on selected key rows (c_t is folded into G_s'); the
+                // row-masked copy is needed only when the tile's two key blocks differ
+                const uint64_t psd = (fl == 1u || fl == 2u) ? pstd : ptd;
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + TM_DQ, desc_add(dd, kk * 32), desc_add(km, kk * 2048), id_q,
-                               (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(BAR(B_EMPTY + j % NSTAGE));
-                    mma_commit(BAR(B_DSFREE + (j & 1)));
+                        mma_ss(tmem + TM_DV, desc_add(ptd, kk * 32), desc_add(gfm, kk * 2048), id_a,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                    if (fl != 0u) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ss(tmem + TM_DV, desc_add(psd, kk * 32), desc_add(gsm, kk * 2048), id_a, 1u);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tmem + TM_DK, desc_add(dsd, kk * 32), desc_add(qm, kk * 2048), id_a,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(BAR(B_EMPTY + s));
+                    mma_commit(BAR(B_TFREE));
                 }
                 __syncwarp();
             };
-            bool ok = wait(B_OPS, 0) && wait(B_FULL, 0);
+            bool ok = wait(B_K, 0) && wait(B_OPS, 0) && wait(B_FULL, 0);
             if (ok) {
                 issue_s(0);
                 issue_dp(0);
@@ -799,11 +469,22 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     }
                     issue_dp(i + 1);
                 }
-                if (!wait(B_DSREADY + (i & 1), (i >> 1) & 1)) {
+                if (!wait(B_TREADY, i & 1)) {
                     ok = false;
                     break;
                 }
-                issue_dq(i);
+                // dS^T of the step to global memory for the dQ GEMM (lane 0 owns the
+                // bulk group), then the dV / dK MMAs on the same tiles
+                if (lane == 0) {
+                    tma_store_3d(&tm_ds, base + OFF_DS, 0, 0, ds_blk0 + i);
+                    bulk_commit_group();
+                }
+                issue_acc(i);
+                if (lane == 0) {
+                    bulk_wait_group_read0();
+                    mbar_arrive(BAR(B_TFREE));
+                }
+                __syncwarp();
             }
             if (elect_one()) {
                 mma_commit(BAR(B_DONE));
@@ -811,114 +492,139 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             }
             __syncwarp();
             wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
+            if (lane == 0) bulk_wait_group0();  // the dS^T stores are complete
         }
     } else if (warp >= 4) {
         // ------------------------------------------ compute warpgroups
-        // warpgroup wg handles key columns [COLS wg, COLS wg + COLS) of every step
+        // warpgroup wg handles query columns [COLS wg, COLS wg + COLS) of every step
         const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
-        const int r = sw * 32 + lane;  // query row of the tile == TMEM lane
-        const int t = t0 + r;
+        const int r = sw * 32 + lane;  // key row of the tile == TMEM lane
+        const int s_tok = s0 + r;
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
-        const size_t row = rowbase + (t < a.T ? t : a.T - 1);
+        const float sl2 = a.scale_log2;
+        const bool in_kb1 = r >= 64 && a.block == 64;  // warp-uniform
+        const bool key_ok = s_tok < a.T;
+        const int c0 = COLS * wg;
         bool ok = true;
-        {  // the tile's Q, G_f, G_s' rows (this warpgroup's HD/NWG columns) into TMEM
-            constexpr int W = HD / NWG / 2;  // 32-bit TMEM columns per warpgroup and operand
-            auto fill = [&](const __nv_bfloat16* src, uint32_t col) {
-                uint32_t u[W];
-                const uint4* p4 = reinterpret_cast<const uint4*>(src + row * HD + 2 * W * wg);
+        {  // V rows of the tile (this warpgroup's HD/NWG columns) into TMEM
+            constexpr int W = HD / NWG / 2;  // 32-bit TMEM columns per warpgroup
+            uint32_t u[W];
+            const uint4* p4 = reinterpret_cast<const uint4*>(v + (rowbase + (s_tok < a.T ? s_tok : 0)) * HD +
+                                                             2 * W * wg);
 #pragma unroll
-                for (int v4 = 0; v4 < W / 4; ++v4) {
-                    const uint4 x = t < a.T ? __ldg(p4 + v4) : make_uint4(0u, 0u, 0u, 0u);
-                    u[4 * v4] = x.x;
-                    u[4 * v4 + 1] = x.y;
-                    u[4 * v4 + 2] = x.z;
-                    u[4 * v4 + 3] = x.w;
-                }
-                tmem_st<W>(trow + col + W * wg, u);
-            };
-            fill(q, TM_Q);
-            fill(gf, TM_GF);
-            fill(gs, TM_GS);
+            for (int v4 = 0; v4 < W / 4; ++v4) {
+                const uint4 x = s_tok < a.T ? __ldg(p4 + v4) : make_uint4(0u, 0u, 0u, 0u);
+                u[4 * v4] = x.x;
+                u[4 * v4 + 1] = x.y;
+                u[4 * v4 + 2] = x.z;
+                u[4 * v4 + 3] = x.w;
+            }
+            tmem_st<W>(trow + TM_V + W * wg, u);
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_OPS));
         }
-        const float my_lse2 = a.lse2[row], my_df = a.Df[row], my_ds = a.Ds[row];
-        const uint32_t* myrow = (r < 64 || a.block == 128 || ragged1) ? mrow : mrow + kMaxWords;
-        const float sl2 = a.scale_log2;
-        const int c0 = COLS * wg;
         const uint32_t rowoff = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
-        auto wait = [&](int bar, uint32_t parity) {
-            const bool r2 = __all_sync(FULL, mbar_wait(BAR(bar), parity, abort_flag, status, lim));
-            fence_after_sync();
-            return r2;
+        auto put_row = [&](uint32_t tile, const uint32_t (&w)[COLS / 2]) {  // swizzled row r
+#pragma unroll
+            for (int q4 = 0; q4 < COLS / 8; ++q4) {
+                const uint32_t chunk = (uint32_t)((c0 >> 3) + q4) ^ (uint32_t)(r & 7);
+                *reinterpret_cast<uint4*>(gbase + tile + rowoff + chunk * 16) =
+                    make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+            }
         };
         for (int i = 0; i < ns; ++i) {
-            const int b = i & 1;
-            if (!wait(B_SREADY, i & 1)) {
+            const int t0 = s0 + STEP * i;
+            const int s = i % NSTAGE;
+            // the stage's row vectors and selection word (already landed: the MMA
+            // warp waited for them before issuing this step's S^T)
+            if (!wait(B_FULL + s, (i / NSTAGE) & 1) || !wait(B_SREADY, i & 1)) {
                 ok = false;
                 break;
             }
-            const int k0 = STEP * i + c0;
-            const bool diag = k0 + COLS - 1 > t0;
+            const uint32_t fl = flags[s];
+            const bool use_s = in_kb1 ? (fl >> 1) & 1u : fl & 1u;
+            const bool mixed = fl == 1u || fl == 2u;
+            const bool diag = t0 < s0 + TILE;
+            const float* rw = rows_s + s * (3 * STEP);
             float pf[COLS];
+            uint32_t pfk[COLS / 2];
             {
                 uint32_t su[COLS];
                 tmem_ld<COLS>(trow + TM_S + c0, su);
                 tmem_wait_ld();
                 fence_before_sync();
-                mbar_arrive(BAR(B_SFREE));  // S may now be overwritten by the next step
+                mbar_arrive(BAR(B_SFREE));  // S^T may now be overwritten by the next step
+                const float4* L4 = reinterpret_cast<const float4*>(rw + c0);
 #pragma unroll
-                for (int j = 0; j < COLS; ++j) {
-                    pf[j] = ex2(fmaf(__uint_as_float(su[j]), sl2, -my_lse2));
-                    if (diag && k0 + j > t) pf[j] = 0.f;
+                for (int j4 = 0; j4 < COLS / 4; ++j4) {
+                    const float4 L = L4[j4];
+                    const float lv[4] = {L.x, L.y, L.z, L.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const int j = 4 * j4 + h;
+                        float p = ex2(fmaf(__uint_as_float(su[j]), sl2, -lv[h]));
+                        if (diag && t0 + c0 + j < s_tok) p = 0.f;
+                        pf[j] = p;
+                    }
+                    pfk[2 * j4] = pack_bf16_alu(pf[4 * j4], pf[4 * j4 + 1]);
+                    pfk[2 * j4 + 1] = pack_bf16_alu(pf[4 * j4 + 2], pf[4 * j4 + 3]);
                 }
             }
-            const bool use_s = sparse(i) && bit(myrow, step_kb(i));  // warp-uniform
             if (!wait(B_PREADY, i & 1)) {
                 ok = false;
                 break;
             }
-            uint32_t fu[COLS], pu[COLS];
-            tmem_ld<COLS>(trow + TM_DPF + c0, fu);
-            if (use_s) tmem_ld<COLS>(trow + TM_DPS + c0, pu);
-            tmem_wait_ld();
-            fence_before_sync();
-            mbar_arrive(BAR(B_PFREE));  // dP may now be overwritten by the next step
             uint32_t dsk[COLS / 2];
+            {
+                uint32_t fu[COLS], pu[COLS];
+                tmem_ld<COLS>(trow + TM_DPF + c0, fu);
+                if (use_s) tmem_ld<COLS>(trow + TM_DPS + c0, pu);
+                tmem_wait_ld();
+                fence_before_sync();
+                mbar_arrive(BAR(B_PFREE));  // dP^T may now be overwritten by the next step
+                const float4* F4 = reinterpret_cast<const float4*>(rw + STEP + c0);
+                const float4* S4 = reinterpret_cast<const float4*>(rw + 2 * STEP + c0);
 #pragma unroll
-            for (int j2 = 0; j2 < COLS / 2; ++j2) {
-                float ds2[2];
+                for (int j4 = 0; j4 < COLS / 4; ++j4) {
+                    const float4 F = F4[j4];
+                    const float4 S = use_s ? S4[j4] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float fv[4] = {F.x, F.y, F.z, F.w}, sv[4] = {S.x, S.y, S.z, S.w};
+                    float ds[4];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int j = 2 * j2 + h;
-                    float g = __uint_as_float(fu[j]) - my_df;
-                    if (use_s) g += __uint_as_float(pu[j]) - my_ds;
-                    ds2[h] = pf[j] * g;
+                    for (int h = 0; h < 4; ++h) {
+                        const int j = 4 * j4 + h;
+                        float g = __uint_as_float(fu[j]) - fv[h];
+                        if (use_s) g += __uint_as_float(pu[j]) - sv[h];
+                        ds[h] = key_ok ? pf[j] * g : 0.f;  // stored dS^T rows past T stay zero
+                    }
+                    dsk[2 * j4] = pack_bf16_alu(ds[0], ds[1]);
+                    dsk[2 * j4 + 1] = pack_bf16_alu(ds[2], ds[3]);
                 }
-                dsk[j2] = pack_bf16_alu(ds2[0], ds2[1]);
             }
-            // dS row r into buffer b once the dQ MMAs of step i-2 have read it
-            if (i >= 2 && !wait(B_DSFREE + b, ((i >> 1) + 1) & 1)) {
+            // the tiles are single-buffered: wait for the previous step's dV / dK MMAs
+            if (i > 0 && !wait(B_TFREE, (i - 1) & 1)) {
                 ok = false;
                 break;
             }
-            uint8_t* dsb = gbase + OFF_DS + b * DS_BYTES + rowoff;
+            put_row(OFF_PT, pfk);
+            put_row(OFF_DS, dsk);
+            if (mixed) {  // the sparse stream's P^T: zero on unselected key rows
+                if (!use_s)
 #pragma unroll
-            for (int q4 = 0; q4 < COLS / 8; ++q4) {
-                const uint32_t chunk = (uint32_t)((c0 >> 3) + q4) ^ (uint32_t)(r & 7);
-                *reinterpret_cast<uint4*>(dsb + chunk * 16) =
-                    make_uint4(dsk[4 * q4], dsk[4 * q4 + 1], dsk[4 * q4 + 2], dsk[4 * q4 + 3]);
+                    for (int e = 0; e < COLS / 2; ++e) pfk[e] = 0u;
+                put_row(OFF_PST, pfk);
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the MMAs
-            mbar_arrive(BAR(B_DSREADY + b));
+            mbar_arrive(BAR(B_TREADY));
         }
         if (ok) ok = wait(B_DONE, 0);
         if (ok) {
+            const bool valid = s_tok < a.T;
+            const size_t row = rowbase + (valid ? s_tok : 0);
             constexpr int OC = HD / NWG;  // output columns per warpgroup
-            const bool valid = t < a.T;
-            store_row_cols<OC / 32>(trow + TM_DQ + OC * wg, a.sm_scale,
-                                    a.dq + (valid ? row : rowbase) * HD + OC * wg, valid);
+            store_row_cols<OC / 32>(trow + TM_DV + OC * wg, 1.f, a.dv + row * HD + OC * wg, valid);
+            store_row_cols<OC / 32>(trow + TM_DK + OC * wg, a.sm_scale, a.dk + row * HD + OC * wg, valid);
         }
     }
     fence_before_sync();
@@ -926,6 +632,147 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (warp == 1) {
         fence_after_sync();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// ============================================================ dQ
+// dQ = sigma dS K as a GEMM over the dS^T blocks the dK/dV kernel stored:
+// CTA = 128 queries (M), K-dim = keys in tiles of 128, N = head dim.  A is the
+// pair of [128 keys x 64 queries] dS^T blocks of the query tile (MN-major),
+// B the key tile (MN-major); both arrive by TMA into a 3-stage ring.
+namespace dq {
+constexpr int NSTAGE = 3;
+constexpr uint32_t BLK_BYTES = 128 * 128;            // one dS^T block
+constexpr uint32_t ST_B = 2 * BLK_BYTES;             // K tile after the two blocks
+constexpr uint32_t STAGE_BYTES = 2 * BLK_BYTES + TILE_BYTES;
+constexpr uint32_t OFF_BAR = NSTAGE * STAGE_BYTES;
+constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+static_assert(SMEM_BYTES <= 232448, "227 KB of shared memory per CTA");
+constexpr int kThr = 192;  // warp 0 TMA, 1 MMA, 2-5 epilogue
+enum : int {
+    B_FULL = 0, B_EMPTY = B_FULL + NSTAGE, B_DONE = B_EMPTY + NSTAGE, B_DRAIN = B_DONE + 1,
+    B_COUNT = B_DRAIN + 1
+};
+static_assert(B_COUNT <= 16, "barrier area holds 16");
+}  // namespace dq
+
+__global__ void __launch_bounds__(dq::kThr, 1)
+bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_k,
+                   const BwdArgs a) {
+    using namespace dq;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
+    unsigned int* status = &g_bwd_tc_status;
+    const uint64_t lim = a.timeout_ns;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntq = (a.T + TILE - 1) / TILE;
+    const int I = ntq - 1 - (int)(blockIdx.x / a.BH);  // longest rows first
+    const int bh = (int)(blockIdx.x % a.BH);
+    const int t0 = I * TILE;
+    const bool two = t0 + 64 < a.T;  // the tile's second 64-query step exists
+    const int nj = I + 1;            // key tiles 0..I
+    auto BAR = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
+    const size_t rowbase = (size_t)bh * a.T;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSTAGE; ++s) {
+            mbar_init(BAR(B_FULL + s), 1);
+            mbar_init(BAR(B_EMPTY + s), 1);
+        }
+        mbar_init(BAR(B_DONE), 1);
+        mbar_init(BAR(B_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(base + OFF_MISC, 128);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    const unsigned FULL = 0xffffffffu;
+    if (warp == 0) {
+        // -------------------------------------------- TMA producer (whole warp)
+        if (elect_one()) {
+            prefetch_tmap(&tm_ds);
+            prefetch_tmap(&tm_k);
+        }
+        __syncwarp();
+        int issued[NSTAGE];
+        for (int s = 0; s < NSTAGE; ++s) issued[s] = -1;
+        for (int j = 0; j < nj; ++j) {
+            const int s = j % NSTAGE;
+            if (j >= NSTAGE &&
+                !__all_sync(FULL, mbar_wait(BAR(B_EMPTY + s), ((j / NSTAGE) + 1) & 1, abort_flag, status,
+                                            lim)))
+                break;
+            const uint32_t st = base + s * STAGE_BYTES;
+            // blocks of key tile j for query steps 2(I - j) and 2(I - j) + 1
+            const int blk = bh * a.ds_blocks + j * (a.T / STEP) - j * (j - 1) + 2 * (I - j);
+            if (elect_one()) {
+                mbar_expect_tx(BAR(B_FULL + s), (two ? 2 : 1) * BLK_BYTES + TILE_BYTES);
+                tma_load_3d(st, &tm_ds, BAR(B_FULL + s), 0, 0, blk);
+                if (two) tma_load_3d(st + BLK_BYTES, &tm_ds, BAR(B_FULL + s), 0, 0, blk + 1);
+                tma_load_3d(st + ST_B, &tm_k, BAR(B_FULL + s), 0, TILE * j, bh);
+                tma_load_3d(st + ST_B + BOX_T, &tm_k, BAR(B_FULL + s), 64, TILE * j, bh);
+            }
+            __syncwarp();
+            issued[s] = j;
+        }
+        if (*abort_flag)
+            for (int s = 0; s < NSTAGE; ++s)
+                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
+    } else if (warp == 1) {
+        // ------------------------------------------ MMA issuer (whole warp)
+        constexpr uint32_t id = idesc_bf16_f32(TILE, HD, true, true);  // A and B MN-major
+        const uint64_t a0 = smem_desc_sw128(base, BLK_BYTES, 1024);
+        const uint64_t b0 = smem_desc_sw128(base + ST_B, BOX_T, 1024);
+        for (int j = 0; j < nj; ++j) {
+            const int s = j % NSTAGE;
+            if (!__all_sync(FULL, mbar_wait(BAR(B_FULL + s), (j / NSTAGE) & 1, abort_flag, status, lim)))
+                break;
+            fence_after_sync();
+            if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // 16 keys per k-step
+                    mma_ss(tmem, desc_add(a0, s * STAGE_BYTES + kk * 2048),
+                           desc_add(b0, s * STAGE_BYTES + kk * 2048), id, (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(BAR(B_EMPTY + s));
+            }
+            __syncwarp();
+        }
+        if (elect_one()) {
+            mma_commit(BAR(B_DONE));
+            mma_commit(BAR(B_DRAIN));
+        }
+        __syncwarp();
+        wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
+    } else {
+        // ------------------------------------------ epilogue: warps 2-5 cover TMEM lanes
+        const int sw = warp & 3;
+        const int r = sw * 32 + lane;
+        const int t = t0 + r;
+        const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
+        if (__all_sync(FULL, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim))) {
+            fence_after_sync();
+            const bool valid = t < a.T;
+            store_row_cols<4>(trow, a.sm_scale, a.dq + (rowbase + (valid ? t : 0)) * HD, valid);
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        fence_after_sync();
+        tmem_dealloc(tmem, 128);
     }
 }
 
@@ -959,10 +806,43 @@ int make_map(CUtensorMap* m, const void* ptr, int BH, int T, int rows) {
     return SSA_OK;
 }
 
+// dS^T blocks [128 keys x 64 queries] bf16 as a 3-D tensor (query, key, block);
+// box = one block; 128B swizzle (the layout the dK/dV kernel writes in smem).
+int make_ds_map(CUtensorMap* m, void* ptr, size_t nblk) {
+    auto fn = encode_fn();
+    if (!fn) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    cuuint64_t dims[3] = {(cuuint64_t)STEP, (cuuint64_t)TILE, (cuuint64_t)nblk};
+    cuuint64_t strides[2] = {(cuuint64_t)STEP * 2, (cuuint64_t)STEP * TILE * 2};
+    cuuint32_t box[3] = {(cuuint32_t)STEP, (cuuint32_t)TILE, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled (dS) failed (%d)", (int)r);
+    return SSA_OK;
+}
+
+// dS^T blocks per (batch, head): key tile J holds (T - 128 J) / 64 steps.
+size_t ds_blocks_per_bh(int T) {
+    const size_t ntk = (size_t)(T + TILE - 1) / TILE;
+    return ntk * (size_t)(T / STEP) - ntk * (ntk - 1);
+}
+// Heads per launch so that the dS^T buffer stays within a fixed budget.
+constexpr size_t kDsBudgetBytes = size_t(4) << 30;
+int heads_per_chunk(const ssa_params_t& p) {
+    const size_t per = ds_blocks_per_bh(p.T) * (size_t)STEP * TILE * 2;
+    const size_t bh = (size_t)p.B * p.H;
+    size_t hc = kDsBudgetBytes / per;
+    if (hc < 1) hc = 1;
+    if (hc > bh) hc = bh;
+    return (int)hc;
+}
+
 struct TcWs {
     __nv_bfloat16* gf;
     __nv_bfloat16* gs;
     float *lse2, *Df, *Ds;
+    __nv_bfloat16* ds;
 };
 
 TcWs carve(const ssa_params_t& p, void* ws) {
@@ -975,6 +855,7 @@ TcWs carve(const ssa_params_t& p, void* ws) {
     w.lse2 = reinterpret_cast<float*>(b + 2 * big);
     w.Df = reinterpret_cast<float*>(b + 2 * big + small);
     w.Ds = reinterpret_cast<float*>(b + 2 * big + 2 * small);
+    w.ds = reinterpret_cast<__nv_bfloat16*>(b + 2 * big + 3 * small);
     return w;
 }
 
@@ -982,12 +863,13 @@ TcWs carve(const ssa_params_t& p, void* ws) {
 
 bool bwd_tc_supported(const ssa_params_t& p) {
     return p.dtype == SSA_BF16 && p.D == HD && (p.block == 64 || p.block == 128) &&
-           mask_words(p) <= kMaxWords && num_blocks(p) <= kMaxBlocks &&
-           (size_t)p.B * p.H * ((p.T + TILE - 1) / TILE) <= 0x7fffffffull;
+           (size_t)p.B * p.H * ((p.T + TILE - 1) / TILE) <= 0x7fffffffull &&
+           ds_blocks_per_bh(p.T) <= 0x7fffffffull;
 }
 
 size_t bwd_tc_workspace(const ssa_params_t& p) {
-    return 2 * align_up(num_elems(p) * 2, 256) + 3 * align_up(num_rows(p) * 4, 256);
+    return 2 * align_up(num_elems(p) * 2, 256) + 3 * align_up(num_rows(p) * 4, 256) +
+           (size_t)heads_per_chunk(p) * ds_blocks_per_bh(p.T) * STEP * TILE * 2;
 }
 
 int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
@@ -1005,53 +887,64 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     int st = check_launch("bwd_tc_pre_kernel");
     if (st != SSA_OK) return st;
 
-    CUtensorMap k128, v128, q64, gf64, gs64, k64, v64;
-    {
-        const void* srcs[5] = {k, v, q, w.gf, w.gs};
-        CUtensorMap* maps[5] = {&k128, &v128, &q64, &gf64, &gs64};
-        const int rows[5] = {TILE, TILE, STEP, STEP, STEP};
-        for (int i = 0; i < 5 && st == SSA_OK; ++i) st = make_map(maps[i], srcs[i], BH, p.T, rows[i]);
-        if (st == SSA_OK) st = make_map(&k64, k, BH, p.T, STEP);
-        if (st == SSA_OK) st = make_map(&v64, v, BH, p.T, STEP);
-    }
-    if (st != SSA_OK) return st;
-
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
         attr_err = cudaFuncSetAttribute(bwd_dkdv_tc_kernel,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv::SMEM_BYTES);
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(bwd_dq_tc_kernel,
+            attr_err = cudaFuncSetAttribute(bwd_dq_gemm_kernel,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            (int)qk::SMEM_BYTES);
+                                            (int)dq::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess)
         return fail(SSA_ERR_CUDA, "bwd_tc: smem attribute: %s", cudaGetErrorString(attr_err));
 
-    BwdArgs a;
-    a.dq = static_cast<__nv_bfloat16*>(dq);
-    a.dk = static_cast<__nv_bfloat16*>(dk);
-    a.dv = static_cast<__nv_bfloat16*>(dv);
-    a.lse2 = w.lse2;
-    a.Df = w.Df;
-    a.Ds = w.Ds;
-    a.mask = mask;
-    a.BH = BH;
-    a.T = p.T;
-    a.block = p.block;
-    a.words = mask_words(p);
-    a.n_blocks = num_blocks(p);
-    a.scale_log2 = p.sm_scale * kLog2e;
-    a.sm_scale = p.sm_scale;
-    a.timeout_ns = wait_limit_ns();
-    const unsigned grid = (unsigned)((size_t)BH * ((p.T + TILE - 1) / TILE));
-    bwd_dkdv_tc_kernel<<<grid, kv::kThr, kv::SMEM_BYTES, s>>>(k128, v128, q64, gf64, gs64, a);
-    st = check_launch("bwd_dkdv_tc_kernel");
-    if (st != SSA_OK) return st;
-    bwd_dq_tc_kernel<<<grid, qk::kThr, qk::SMEM_BYTES, s>>>(
-        k64, v64, static_cast<const __nv_bfloat16*>(q), w.gf, w.gs, a);
-    return check_launch("bwd_dq_tc_kernel");
+    const int ntile = (p.T + TILE - 1) / TILE;
+    const size_t nb = ds_blocks_per_bh(p.T);
+    const int hc = heads_per_chunk(p);
+    const size_t head_elems = (size_t)p.T * HD;
+    const size_t head_mask = (size_t)num_blocks(p) * mask_words(p);
+    // every (batch, head) is independent: chunks of hc heads share the dS^T buffer
+    for (int h0 = 0; h0 < BH && st == SSA_OK; h0 += hc) {
+        const int nh = BH - h0 < hc ? BH - h0 : hc;
+        auto off = [&](const void* ptr) {
+            return static_cast<const void*>(static_cast<const __nv_bfloat16*>(ptr) + h0 * head_elems);
+        };
+        CUtensorMap k128, q64, gf64, gs64, ds_map;
+        st = make_map(&k128, off(k), nh, p.T, TILE);
+        if (st == SSA_OK) st = make_map(&q64, off(q), nh, p.T, STEP);
+        if (st == SSA_OK) st = make_map(&gf64, off(w.gf), nh, p.T, STEP);
+        if (st == SSA_OK) st = make_map(&gs64, off(w.gs), nh, p.T, STEP);
+        if (st == SSA_OK) st = make_ds_map(&ds_map, w.ds, (size_t)nh * nb);
+        if (st != SSA_OK) break;
+
+        BwdArgs a;
+        a.dq = static_cast<__nv_bfloat16*>(dq) + h0 * head_elems;
+        a.dk = static_cast<__nv_bfloat16*>(dk) + h0 * head_elems;
+        a.dv = static_cast<__nv_bfloat16*>(dv) + h0 * head_elems;
+        a.lse2 = w.lse2 + (size_t)h0 * p.T;
+        a.Df = w.Df + (size_t)h0 * p.T;
+        a.Ds = w.Ds + (size_t)h0 * p.T;
+        a.mask = mask + h0 * head_mask;
+        a.BH = nh;
+        a.T = p.T;
+        a.block = p.block;
+        a.words = mask_words(p);
+        a.n_blocks = num_blocks(p);
+        a.ds_blocks = (int)nb;
+        a.scale_log2 = p.sm_scale * kLog2e;
+        a.sm_scale = p.sm_scale;
+        a.timeout_ns = wait_limit_ns();
+        const unsigned grid = (unsigned)((size_t)nh * ntile);
+        bwd_dkdv_tc_kernel<<<grid, kv::kThr, kv::SMEM_BYTES, s>>>(
+            k128, q64, gf64, gs64, ds_map, static_cast<const __nv_bfloat16*>(off(v)), a);
+        st = check_launch("bwd_dkdv_tc_kernel");
+        if (st != SSA_OK) break;
+        bwd_dq_gemm_kernel<<<grid, dq::kThr, dq::SMEM_BYTES, s>>>(ds_map, k128, a);
+        st = check_launch("bwd_dq_gemm_kernel");
+    }
+    return st;
 }
 
 int bwd_tc_take_status(cudaStream_t) {

@@ -95,6 +95,27 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+// Tiled shared -> global store (bulk-group completion); the source tile must
+// have been made visible to the async proxy (fence.proxy.async) first.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until the source reads of every committed bulk store are done.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until every committed bulk store is complete (writes visible).
+__device__ __forceinline__ void bulk_wait_group0() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -222,11 +243,14 @@ __device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
 }
 
 // Instruction descriptor of kind::f16: bf16 A and B, f32 accumulator.
-// b_mn_major: B stored MN-major (N contiguous) instead of K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+// b_mn_major / a_mn_major: operand stored MN-major (M or N contiguous)
+// instead of K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major,
+                                                      bool a_mn_major = false) {
     return (1u << 4)                        // D format f32
            | (1u << 7)                      // A format bf16
            | (1u << 10)                     // B format bf16
+           | ((a_mn_major ? 1u : 0u) << 15) // A major
            | ((b_mn_major ? 1u : 0u) << 16) // B major
            | ((uint32_t)(N >> 3) << 17)     // N / 8
            | ((uint32_t)(M >> 4) << 24);    // M / 16

@@ -173,7 +173,10 @@ int ssa_align_loss(const ssa_params_t* params, const float* sqdiff_rows,
  * causal key (section 2, "Full Attention Stream").  h_full, h_sparse,
  * lse_full and lse_sparse are the forward's outputs for the same inputs.
  * dh_full / dh_sparse may be NULL (read as zero).  dq, dk, dv are written
- * (not accumulated).  Workspace: SSA_WS_BWD.
+ * (not accumulated).  Workspace: SSA_WS_BWD; on the tensor-core path it
+ * holds the bf16 dS blocks of the causal triangle for up to 4 GiB worth of
+ * (batch, head) pairs at a time (about 2 * T^2 / 2 bytes per pair), so long
+ * sequences are processed a group of heads at a time.
  */
 int ssa_attn_bwd(const ssa_params_t* params, const void* q, const void* k,
                  const void* v, const int32_t* idx, const int32_t* cnt,
