@@ -19,7 +19,8 @@
 //
 // Three kernels, no atomics (bitwise repeatable):
 //   bwd_tc_pre_kernel   one warp per row: G_f, G_s' rounded to bf16, D_f and
-//                       D_s' from the rounded values, lse_full*log2(e).
+//                       D_s' from the rounded values, lse_full*log2(e)
+//                       (the three scalars stored negated).
 //   bwd_dkdv_tc_kernel  CTA = 128 keys; steps of 64 queries.  Per step:
 //                       S^T = K Q^T, dP_f^T = V G_f^T, dP_s^T = V G_s'^T
 //                       (tcgen05 SS, N = 64), the compute warpgroups form
@@ -61,9 +62,9 @@ struct BwdArgs {
     __nv_bfloat16* dq;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
-    const float* lse2;  // lse_full * log2(e)
-    const float* Df;
-    const float* Ds;    // D_s of the c_t-scaled G_s
+    const float* neg_lse2;  // -lse_full * log2(e)
+    const float* neg_Df;    // -D_f
+    const float* neg_Ds;    // -D_s of the c_t-scaled G_s
     const uint32_t* mask;
     int BH, T, block, words, n_blocks;
     int ds_blocks;  // dS^T blocks per (batch, head): one per (key tile, 64-query step)
@@ -160,8 +161,8 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
                   const __nv_bfloat16* __restrict__ dhf, const __nv_bfloat16* __restrict__ dhs,
                   const float* __restrict__ lse_f, const float* __restrict__ lse_s, size_t rows,
                   float cf, float cs, __nv_bfloat16* __restrict__ gf, __nv_bfloat16* __restrict__ gs,
-                  float* __restrict__ lse2, float* __restrict__ Df,
-                  float* __restrict__ Ds) {
+                  float* __restrict__ neg_lse2, float* __restrict__ neg_Df,
+                  float* __restrict__ neg_Ds) {
     const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -204,16 +205,22 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
         sf += __shfl_xor_sync(0xffffffffu, sf, o);
         ss += __shfl_xor_sync(0xffffffffu, ss, o);
     }
-    if (lane == 0) {
-        lse2[row] = lf * kLog2e;
-        Df[row] = sf;
-        Ds[row] = ss;
+    if (lane == 0) {  // negated: the consumers add them
+        neg_lse2[row] = -(lf * kLog2e);
+        neg_Df[row] = -sf;
+        neg_Ds[row] = -ss;
     }
 }
 
 // ============================================================ dK / dV
 #ifndef SSA_KV_WARPGROUPS
 #define SSA_KV_WARPGROUPS 2
+#endif
+#ifndef SSA_KV_POLY_PAIRS
+#define SSA_KV_POLY_PAIRS 0
+#endif
+#ifndef SSA_KV_PACK_CVT
+#define SSA_KV_PACK_CVT 0
 #endif
 namespace kv {
 // K stays in shared memory (A of S^T = K Q^T), V lives in TMEM (A of the dP^T
@@ -225,6 +232,18 @@ namespace kv {
 constexpr int NWG = SSA_KV_WARPGROUPS;  // compute warpgroups; each owns COLS query columns of a step
 static_assert(NWG == 2 || NWG == 4, "2 or 4 compute warpgroups");
 constexpr int COLS = STEP / NWG;
+// of a thread's COLS/2 exponential pairs per step, this many (the last ones)
+// run as a polynomial on the FMA pipe instead of the MUFU unit
+constexpr int kPolyPairs = SSA_KV_POLY_PAIRS;
+static_assert(kPolyPairs >= 0 && kPolyPairs <= COLS / 2 && kPolyPairs % 2 == 0, "whole float4 groups");
+// bf16 packing: integer ALU (add half an ulp, byte permute) or the conversion unit
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+#if SSA_KV_PACK_CVT
+    return pack_bf16(lo, hi);
+#else
+    return pack_bf16_alu(lo, hi);
+#endif
+}
 constexpr int kThr = 128 + 128 * NWG;  // warp 0 TMA, 1 MMA, 2-3 idle, then the compute warps
 constexpr int kComp = 128 * NWG;
 constexpr uint32_t OFF_K = 0;
@@ -237,7 +256,7 @@ constexpr uint32_t T_BYTES = 128 * 128;
 constexpr uint32_t OFF_DS = OFF_STAGE + NSTAGE * STAGE_BYTES;  // dS^T
 constexpr uint32_t OFF_PT = OFF_DS + T_BYTES;                  // P_f^T
 constexpr uint32_t OFF_PST = OFF_PT + T_BYTES;                 // P_s^T on mixed steps
-// per stage, fp32 over the step's 64 queries: lse_full*log2(e) | D_f | D_s
+// per stage, fp32 over the step's 64 queries: -lse_full*log2(e) | -D_f | -D_s
 constexpr uint32_t ROW_BYTES = 3 * STEP * 4;
 constexpr uint32_t OFF_ROWS = OFF_PST + T_BYTES;
 constexpr uint32_t OFF_BAR = OFF_ROWS + NSTAGE * ROW_BYTES;
@@ -365,12 +384,12 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 tma_load_3d(st + ST_Q + BOX_S, &tm_q, BAR(B_FULL + s), 64, t0, bh);
                 tma_load_3d(st + ST_GF, &tm_gf, BAR(B_FULL + s), 0, t0, bh);
                 tma_load_3d(st + ST_GF + BOX_S, &tm_gf, BAR(B_FULL + s), 64, t0, bh);
-                bulk_load(rw, a.lse2 + rowbase + t0, STEP * 4, BAR(B_FULL + s));
-                bulk_load(rw + STEP * 4, a.Df + rowbase + t0, STEP * 4, BAR(B_FULL + s));
+                bulk_load(rw, a.neg_lse2 + rowbase + t0, STEP * 4, BAR(B_FULL + s));
+                bulk_load(rw + STEP * 4, a.neg_Df + rowbase + t0, STEP * 4, BAR(B_FULL + s));
                 if (sp) {  // the sparse stream's operands only where it has work
                     tma_load_3d(st + ST_GS, &tm_gs, BAR(B_FULL + s), 0, t0, bh);
                     tma_load_3d(st + ST_GS + BOX_S, &tm_gs, BAR(B_FULL + s), 64, t0, bh);
-                    bulk_load(rw + 2 * STEP * 4, a.Ds + rowbase + t0, STEP * 4, BAR(B_FULL + s));
+                    bulk_load(rw + 2 * STEP * 4, a.neg_Ds + rowbase + t0, STEP * 4, BAR(B_FULL + s));
                 }
             }
             __syncwarp();
@@ -556,20 +575,34 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 fence_before_sync();
                 mbar_arrive(BAR(B_SFREE));  // S^T may now be overwritten by the next step
                 const float4* L4 = reinterpret_cast<const float4*>(rw + c0);
+                const f32x2 sl2x2 = mk2(sl2, sl2);
 #pragma unroll
                 for (int j4 = 0; j4 < COLS / 4; ++j4) {
-                    const float4 L = L4[j4];
-                    const float lv[4] = {L.x, L.y, L.z, L.w};
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int j = 4 * j4 + h;
-                        float p = ex2(fmaf(__uint_as_float(su[j]), sl2, -lv[h]));
-                        if (diag && t0 + c0 + j < s_tok) p = 0.f;
-                        pf[j] = p;
+                    const float4 L = L4[j4];  // -lse_full * log2(e) of the four queries
+                    const f32x2 x01 = fma2(mk2(__uint_as_float(su[4 * j4]), __uint_as_float(su[4 * j4 + 1])),
+                                           sl2x2, mk2(L.x, L.y));
+                    const f32x2 x23 = fma2(mk2(__uint_as_float(su[4 * j4 + 2]), __uint_as_float(su[4 * j4 + 3])),
+                                           sl2x2, mk2(L.z, L.w));
+                    if (2 * j4 >= COLS / 2 - kPolyPairs) {  // part of the exponentials on the FMA pipe
+                        un2(exp2_poly2(x01), pf[4 * j4], pf[4 * j4 + 1]);
+                        un2(exp2_poly2(x23), pf[4 * j4 + 2], pf[4 * j4 + 3]);
+                    } else {
+                        float x0, x1, x2, x3;
+                        un2(x01, x0, x1);
+                        un2(x23, x2, x3);
+                        pf[4 * j4] = ex2(x0);
+                        pf[4 * j4 + 1] = ex2(x1);
+                        pf[4 * j4 + 2] = ex2(x2);
+                        pf[4 * j4 + 3] = ex2(x3);
                     }
-                    pfk[2 * j4] = pack_bf16_alu(pf[4 * j4], pf[4 * j4 + 1]);
-                    pfk[2 * j4 + 1] = pack_bf16_alu(pf[4 * j4 + 2], pf[4 * j4 + 3]);
                 }
+                if (diag) {  // causal: query t0 + c0 + j sees key s_tok only if t >= s
+#pragma unroll
+                    for (int j = 0; j < COLS; ++j)
+                        if (t0 + c0 + j < s_tok) pf[j] = 0.f;
+                }
+#pragma unroll
+                for (int j2 = 0; j2 < COLS / 2; ++j2) pfk[j2] = pack2(pf[2 * j2], pf[2 * j2 + 1]);
             }
             if (!wait(B_PREADY, i & 1)) {
                 ok = false;
@@ -587,19 +620,27 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const float4* S4 = reinterpret_cast<const float4*>(rw + 2 * STEP + c0);
 #pragma unroll
                 for (int j4 = 0; j4 < COLS / 4; ++j4) {
-                    const float4 F = F4[j4];
-                    const float4 S = use_s ? S4[j4] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float fv[4] = {F.x, F.y, F.z, F.w}, sv[4] = {S.x, S.y, S.z, S.w};
-                    float ds[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int j = 4 * j4 + h;
-                        float g = __uint_as_float(fu[j]) - fv[h];
-                        if (use_s) g += __uint_as_float(pu[j]) - sv[h];
-                        ds[h] = key_ok ? pf[j] * g : 0.f;  // stored dS^T rows past T stay zero
+                    const float4 F = F4[j4];  // -D_f
+                    f32x2 g01 = add2(mk2(__uint_as_float(fu[4 * j4]), __uint_as_float(fu[4 * j4 + 1])),
+                                     mk2(F.x, F.y));
+                    f32x2 g23 = add2(mk2(__uint_as_float(fu[4 * j4 + 2]), __uint_as_float(fu[4 * j4 + 3])),
+                                     mk2(F.z, F.w));
+                    if (use_s) {
+                        const float4 S = S4[j4];  // -D_s'
+                        g01 = add2(g01, add2(mk2(__uint_as_float(pu[4 * j4]), __uint_as_float(pu[4 * j4 + 1])),
+                                             mk2(S.x, S.y)));
+                        g23 = add2(g23, add2(mk2(__uint_as_float(pu[4 * j4 + 2]), __uint_as_float(pu[4 * j4 + 3])),
+                                             mk2(S.z, S.w)));
                     }
-                    dsk[2 * j4] = pack_bf16_alu(ds[0], ds[1]);
-                    dsk[2 * j4 + 1] = pack_bf16_alu(ds[2], ds[3]);
+                    float d0, d1, d2, d3;
+                    un2(mul2(mk2(pf[4 * j4], pf[4 * j4 + 1]), g01), d0, d1);
+                    un2(mul2(mk2(pf[4 * j4 + 2], pf[4 * j4 + 3]), g23), d2, d3);
+                    dsk[2 * j4] = pack2(d0, d1);
+                    dsk[2 * j4 + 1] = pack2(d2, d3);
+                }
+                if (!key_ok) {  // stored dS^T rows past T stay zero (warp-uniform)
+#pragma unroll
+                    for (int e = 0; e < COLS / 2; ++e) dsk[e] = 0u;
                 }
             }
             // the tiles are single-buffered: wait for the previous step's dV / dK MMAs
@@ -841,7 +882,7 @@ int heads_per_chunk(const ssa_params_t& p) {
 struct TcWs {
     __nv_bfloat16* gf;
     __nv_bfloat16* gs;
-    float *lse2, *Df, *Ds;
+    float *neg_lse2, *neg_Df, *neg_Ds;
     __nv_bfloat16* ds;
 };
 
@@ -852,9 +893,9 @@ TcWs carve(const ssa_params_t& p, void* ws) {
     TcWs w;
     w.gf = reinterpret_cast<__nv_bfloat16*>(b);
     w.gs = reinterpret_cast<__nv_bfloat16*>(b + big);
-    w.lse2 = reinterpret_cast<float*>(b + 2 * big);
-    w.Df = reinterpret_cast<float*>(b + 2 * big + small);
-    w.Ds = reinterpret_cast<float*>(b + 2 * big + 2 * small);
+    w.neg_lse2 = reinterpret_cast<float*>(b + 2 * big);
+    w.neg_Df = reinterpret_cast<float*>(b + 2 * big + small);
+    w.neg_Ds = reinterpret_cast<float*>(b + 2 * big + 2 * small);
     w.ds = reinterpret_cast<__nv_bfloat16*>(b + 2 * big + 3 * small);
     return w;
 }
@@ -883,7 +924,7 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     bwd_tc_pre_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(hf), static_cast<const __nv_bfloat16*>(hs),
         static_cast<const __nv_bfloat16*>(dhf), static_cast<const __nv_bfloat16*>(dhs), lf, ls, rows,
-        (float)(w_s * two_over_n), (float)(w_c * two_over_n), w.gf, w.gs, w.lse2, w.Df, w.Ds);
+        (float)(w_s * two_over_n), (float)(w_c * two_over_n), w.gf, w.gs, w.neg_lse2, w.neg_Df, w.neg_Ds);
     int st = check_launch("bwd_tc_pre_kernel");
     if (st != SSA_OK) return st;
 
@@ -923,9 +964,9 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
         a.dq = static_cast<__nv_bfloat16*>(dq) + h0 * head_elems;
         a.dk = static_cast<__nv_bfloat16*>(dk) + h0 * head_elems;
         a.dv = static_cast<__nv_bfloat16*>(dv) + h0 * head_elems;
-        a.lse2 = w.lse2 + (size_t)h0 * p.T;
-        a.Df = w.Df + (size_t)h0 * p.T;
-        a.Ds = w.Ds + (size_t)h0 * p.T;
+        a.neg_lse2 = w.neg_lse2 + (size_t)h0 * p.T;
+        a.neg_Df = w.neg_Df + (size_t)h0 * p.T;
+        a.neg_Ds = w.neg_Ds + (size_t)h0 * p.T;
         a.mask = mask + h0 * head_mask;
         a.BH = nh;
         a.T = p.T;
