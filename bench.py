@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import ctypes
 import json
 import math
 import os
@@ -81,6 +82,23 @@ def step_flops(w, p_full, p_sel):
     f_fwd = 4 * w.D * p_full * BH
     f_bwd = (10 * w.D * p_full + 4 * w.D * p_sel) * BH
     return f_fwd, f_bwd
+
+
+def kernel_flops(w, p_full, p_sel):
+    """Algorithmic FLOPs of each tensor-core kernel of one step.  fwd: S and
+    P V of the full stream (the sparse stream's products are a subset of the
+    same tiles); dK/dV kernel: S^T, dP_f^T, dV, dK per causal pair plus dP_s^T
+    and the sparse dV per selected pair; dQ GEMM: dS K per causal pair."""
+    BH, d = w.B * w.H, w.D
+    return {"fwd_tc_kernel": 4 * d * p_full * BH,
+            "bwd_dkdv_tc_kernel": (8 * d * p_full + 4 * d * p_sel) * BH,
+            "bwd_dq_gemm_kernel": 2 * d * p_full * BH}
+
+
+def ds_blocks_per_bh(T):
+    """[128 keys x 64 queries] dS^T blocks of the causal triangle of one head."""
+    ntk = (T + 127) // 128
+    return ntk * (T // 64) - ntk * (ntk - 1)
 
 
 def source_sha(*names):
@@ -187,7 +205,9 @@ class Layer:
         # select: pool + score; fwd: 1; loss: 2; bwd: pre + dk/dv + dq (either path)
         return 2 + 1 + 2 + 3
 
-    def run(self, stream, events=None):
+    def run(self, stream, events=None, kernel_events=None):
+        """One step; `events` (5) bracket the four ABI calls, `kernel_events`
+        (4, tensor-core path) the kernels inside the backward call."""
         s, ssa, P = stream.cuda_stream, self.ssa, self.p
         ptr = lambda t: t.data_ptr()
         ev = events or [None] * 5
@@ -211,11 +231,16 @@ class Layer:
         ssa.check(st, "loss")
         if ev[3] is not None:
             ev[3].record(stream)
+        if kernel_events is not None:
+            handles = (ctypes.c_void_p * 4)(*[e.cuda_event for e in kernel_events])
+            ssa.check(ssa.ssa_debug_set_kernel_events(handles, 4), "kernel events")
         st = ssa.ssa_attn_bwd(P, ptr(self.q), ptr(self.k), ptr(self.v), None, None,
                               ptr(self.mask), ptr(self.hf), ptr(self.hs), ptr(r["lse_f"]),
                               ptr(r["lse_s"]), ptr(self.dhf), ptr(self.dhs), self.w_s, self.w_c,
                               ptr(self.dq), ptr(self.dk), ptr(self.dv), ptr(self.ws[3]),
                               self.ws[3].numel(), s)
+        if kernel_events is not None:
+            ssa.ssa_debug_set_kernel_events(None, 0)
         ssa.check(st, "bwd")
         if ev[4] is not None:
             ev[4].record(stream)
@@ -241,12 +266,18 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
     per_call = {n: 0.0 for n in names}
     step_ms = []
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    kevs = None
+    if layer.path == 1:  # per-kernel events inside the backward call
+        kevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        for ks in kevs:
+            for e in ks:
+                e.record(stream)  # creates the event so its handle can be passed down
     barrier(world)
     torch.cuda.synchronize(dev)
     with ClockSampler(torch.cuda.current_device()) as clk:
         for i in range(args.steps):
             flush.zero_()  # evict L2 between timed steps (outside the events)
-            layer.run(stream, evs[i])
+            layer.run(stream, evs[i], kevs[i] if kevs else None)
         torch.cuda.synchronize(dev)
     barrier(world)
     layer.ssa.device_status()
@@ -259,28 +290,42 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
     ms_per_step = max_ms / args.steps
     value = whole_job_tflops(f_fwd + f_bwd, world, ms_per_step)
 
-    # dominant ABI call and its roofline
+    # per-kernel times (fwd: the call is its one kernel) and the dominant kernel's roofline
     avg = {n: per_call[n] / args.steps for n in names}
-    dom = max(("fwd", "bwd"), key=lambda n: avg[n])
     sustained = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    kernels = None
     if layer.path == 1:
-        flops = f_fwd if dom == "fwd" else f_bwd
-        achieved = flops / (avg[dom] * 1e-3) / 1e12
-        name = "fwd_tc_kernel" if dom == "fwd" else "bwd_tc (pre + dkdv + dq kernels)"
-        roof = {"kernel": name, "bound": "tensor", "peak": sustained,
-                "unit": "TFLOP/s", "peak_kind": f"{peak_src} bf16 dense, sustained",
-                "traffic": ncu_traffic("fwd_tc_kernel" if dom == "fwd" else "bwd_tc")}
+        kms = {"fwd_tc_kernel": avg["fwd"], "bwd_tc_pre_kernel": 0.0, "bwd_dkdv_tc_kernel": 0.0,
+               "bwd_dq_gemm_kernel": 0.0}
+        for ks in kevs:
+            kms["bwd_tc_pre_kernel"] += ks[0].elapsed_time(ks[1]) / args.steps
+            kms["bwd_dkdv_tc_kernel"] += ks[1].elapsed_time(ks[2]) / args.steps
+            kms["bwd_dq_gemm_kernel"] += ks[2].elapsed_time(ks[3]) / args.steps
+        kfl = kernel_flops(w, p_full, p_sel)
+        kernels = {k: {"ms": round(v, 4)} for k, v in kms.items()}
+        for k, f in kfl.items():
+            kernels[k]["tflops"] = round(f / (kms[k] * 1e-3) / 1e12, 2)
+        # the dQ GEMM streams the stored dS^T blocks: its own bound is HBM
+        dq_bytes = (ds_blocks_per_bh(w.T) * 64 * 128 * 2 + 2 * w.T * w.D * 2) * w.B * w.H
+        kernels["bwd_dq_gemm_kernel"]["hbm_gbs"] = round(dq_bytes / (kms["bwd_dq_gemm_kernel"] * 1e-3) / 1e9, 1)
+        kernels["bwd_dq_gemm_kernel"]["hbm_bytes"] = dq_bytes
+        dom = max(kfl, key=lambda k: kms[k])
+        roof = {"kernel": dom, "bound": "tensor", "peak": sustained, "unit": "TFLOP/s",
+                "peak_kind": f"{peak_src} bf16 dense, sustained", "traffic": ncu_traffic(dom)}
+        flops, dom_ms = kfl[dom], kms[dom]
     else:
+        dom = max(("fwd", "bwd"), key=lambda n: avg[n])
         flops = f_fwd if dom == "fwd" else f_bwd
-        achieved = flops / (avg[dom] * 1e-3) / 1e12
         fp32 = NUM_SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         roof = {"kernel": f"{dom}_simt", "bound": "alu", "peak": round(fp32, 1),
                 "unit": "TFLOP/s", "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock",
                 "traffic": ncu_traffic(f"{dom}_simt")}
+        dom_ms = avg[dom]
+    achieved = flops / (dom_ms * 1e-3) / 1e12
     roof["achieved"] = round(achieved, 2)
     roof["frac"] = round(achieved / roof["peak"], 4)
-    roof["ms_per_launch"] = round(avg[dom], 4)
-    roof["flops_per_launch"] = f_fwd if dom == "fwd" else f_bwd
+    roof["ms_per_launch"] = round(dom_ms, 4)
+    roof["flops_per_launch"] = flops
 
     fwd_tflops = f_fwd / (avg["fwd"] * 1e-3) / 1e12
     out = {
@@ -294,6 +339,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
                    "l2": "flushed before every timed step", "kernel_path": layer.path},
         "roofline": roof,
         "breakdown_ms": {n: round(avg[n], 4) for n in names},
+        "kernels": kernels,
         "fwd_tflops": round(fwd_tflops, 2),
         "fwd_frac_sustained": round(fwd_tflops / sustained, 4),
         "fwd_frac_burst": round(fwd_tflops / peaks.get("bf16_tflops", 1590.0), 4),

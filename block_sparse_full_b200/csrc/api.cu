@@ -15,6 +15,7 @@ namespace {
 thread_local char g_last_error[512] = "";
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<void*> g_kernel_events[kKernelEvents];
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -79,6 +80,11 @@ size_t bwd_workspace(const ssa_params_t& p) {
 }  // namespace
 
 unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
+void mark_kernel_event(int i, cudaStream_t s) {
+    void* e = g_kernel_events[i].load(std::memory_order_relaxed);
+    if (e) cudaEventRecord(static_cast<cudaEvent_t>(e), s);
+}
 
 int fail(int status, const char* fmt, ...) {
     va_list ap;
@@ -239,6 +245,17 @@ int ssa_version(void) { return (1 << 16) | 0; }
 
 void ssa_debug_set_wait_limit_ns(unsigned long long ns) {
     g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs, std::memory_order_relaxed);
+}
+
+int ssa_debug_set_kernel_events(void* const* events, int n) {
+    if (n == 0) {
+        for (auto& e : ssa::g_kernel_events) e.store(nullptr, std::memory_order_relaxed);
+        return SSA_OK;
+    }
+    if (n != ssa::kKernelEvents || !events) return ssa::fail(SSA_ERR_INVALID_ARG, "need %d events", ssa::kKernelEvents);
+    for (int i = 0; i < n; ++i)
+        ssa::g_kernel_events[i].store(events[i], std::memory_order_relaxed);
+    return SSA_OK;
 }
 
 }  // extern "C"

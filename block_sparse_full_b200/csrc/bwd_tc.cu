@@ -921,12 +921,14 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     const TcWs w = carve(p, ws);
     const size_t rows = num_rows(p);
     const double two_over_n = 2.0 / (double)num_elems(p);
+    mark_kernel_event(0, s);
     bwd_tc_pre_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(hf), static_cast<const __nv_bfloat16*>(hs),
         static_cast<const __nv_bfloat16*>(dhf), static_cast<const __nv_bfloat16*>(dhs), lf, ls, rows,
         (float)(w_s * two_over_n), (float)(w_c * two_over_n), w.gf, w.gs, w.neg_lse2, w.neg_Df, w.neg_Ds);
     int st = check_launch("bwd_tc_pre_kernel");
     if (st != SSA_OK) return st;
+    mark_kernel_event(1, s);
 
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -982,8 +984,10 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
             k128, q64, gf64, gs64, ds_map, static_cast<const __nv_bfloat16*>(off(v)), a);
         st = check_launch("bwd_dkdv_tc_kernel");
         if (st != SSA_OK) break;
+        if (h0 == 0) mark_kernel_event(2, s);
         bwd_dq_gemm_kernel<<<grid, dq::kThr, dq::SMEM_BYTES, s>>>(ds_map, k128, a);
         st = check_launch("bwd_dq_gemm_kernel");
+        if (h0 == 0) mark_kernel_event(3, s);
     }
     return st;
 }

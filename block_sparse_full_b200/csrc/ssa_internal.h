@@ -22,6 +22,11 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Wall-clock limit of the kernels' bounded waits (default 2 s; tests shorten it).
 unsigned long long wait_limit_ns();
 
+// Measurement hook (ssa_debug_set_kernel_events): records caller event i on
+// stream s when the hook is enabled, else does nothing.
+constexpr int kKernelEvents = 4;
+void mark_kernel_event(int i, cudaStream_t s);
+
 inline size_t num_rows(const ssa_params_t& p) {
     return (size_t)p.B * p.H * p.T;
 }

@@ -35,7 +35,7 @@ EXPORTS = (
     "ssa_attn_fwd_dual", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
     "ssa_kernel_path", "ssa_selftest_math", "ssa_selftest_wait_timeout",
-    "ssa_debug_set_wait_limit_ns", "ssa_version",
+    "ssa_debug_set_wait_limit_ns", "ssa_debug_set_kernel_events", "ssa_version",
 )
 
 
@@ -77,6 +77,7 @@ _SIGNATURES = {
     "ssa_selftest_math": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "ssa_version": (c_int, []),
     "ssa_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
+    "ssa_debug_set_kernel_events": (c_int, [c_void_p, c_int]),
     "ssa_selftest_wait_timeout": (c_int, [ctypes.c_ulonglong, c_void_p, c_void_p]),
 }
 
@@ -160,6 +161,10 @@ def ssa_selftest_wait_timeout(limit_ns, gave_up, stream):
 
 def ssa_debug_set_wait_limit_ns(ns):
     _lib.ssa_debug_set_wait_limit_ns(ns)
+
+
+def ssa_debug_set_kernel_events(events, n):
+    return _lib.ssa_debug_set_kernel_events(events, n)
 
 
 def ssa_version():

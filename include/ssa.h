@@ -225,6 +225,16 @@ int ssa_selftest_wait_timeout(unsigned long long limit_ns, int* gave_up, void* s
  * Process-wide; not synchronised with calls running on other threads. */
 void ssa_debug_set_wait_limit_ns(unsigned long long ns);
 
+/* Measurement hook: makes later ssa_attn_bwd calls on the tensor-core path
+ * record the caller's CUDA events (cudaEvent_t, passed as void*) on the call's
+ * stream at kernel boundaries: events[0] before the preprocess kernel,
+ * events[1] after it, events[2] after the dK/dV kernel and events[3] after
+ * the dQ GEMM of the first group of heads (the only group unless the dS
+ * buffer is split).  n must be 4 to enable, 0 to disable; the events stay
+ * owned by the caller, who must disable the hook before destroying them.
+ * Returns SSA_OK or SSA_ERR_INVALID_ARG.  Process-wide, like the hook above. */
+int ssa_debug_set_kernel_events(void* const* events, int n);
+
 /* ABI version, (major << 16) | minor. */
 int ssa_version(void);
 
