@@ -213,9 +213,6 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
 }
 
 // ============================================================ dK / dV
-#ifndef SSA_KV_WARPGROUPS
-#define SSA_KV_WARPGROUPS 2
-#endif
 #ifndef SSA_KV_POLY_PAIRS
 #define SSA_KV_POLY_PAIRS 0
 #endif
@@ -223,80 +220,77 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
 #define SSA_KV_PACK_CVT 0
 #endif
 namespace kv {
-// K stays in shared memory (A of S^T = K Q^T), V lives in TMEM (A of the dP^T
-// MMAs, TS form); Q, G_f, G_s' steps stream through a ring.  The compute
-// warps write P^T (and, on mixed steps, the sparse stream's row-masked copy)
-// and dS^T as swizzled bf16 tiles in shared memory: the A operands of
-// dV += P^T G and dK += dS^T Q.  S^T and dP^T are handed over separately as
-// soon as they have been read into registers.
-constexpr int NWG = SSA_KV_WARPGROUPS;  // compute warpgroups; each owns COLS query columns of a step
-static_assert(NWG == 2 || NWG == 4, "2 or 4 compute warpgroups");
-constexpr int COLS = STEP / NWG;
-// of a thread's COLS/2 exponential pairs per step, this many (the last ones)
-// run as a polynomial on the FMA pipe instead of the MUFU unit
+// K and V of the tile live in TMEM: the A operands of S^T = K Q^T and
+// dP^T = V G^T (TS form: only the 64-query B tiles are read from shared
+// memory).  Q, G_f, G_s' steps stream through a ring.  One 64-column TMEM
+// range holds, in turn within a step, S^T, then (on sparse steps) dP_s^T,
+// then the bf16 P^T that feeds dV += P^T G_f (+ the sparse stream's
+// row-masked copy next to it on mixed steps); S^T of the next step is issued
+// behind the dV MMAs.  dS^T goes to a double-buffered swizzled shared tile:
+// the A operand of dK += dS^T Q and the source of its TMA store for the dQ GEMM.
+constexpr int COLS = 32;  // query columns per compute warpgroup (two warpgroups)
+// of a thread's 16 exponential pairs per step, this many (the last ones) run
+// as a polynomial on the FMA pipe instead of the MUFU unit
 constexpr int kPolyPairs = SSA_KV_POLY_PAIRS;
 static_assert(kPolyPairs >= 0 && kPolyPairs <= COLS / 2 && kPolyPairs % 2 == 0, "whole float4 groups");
-// bf16 packing: integer ALU (add half an ulp, byte permute) or the conversion unit
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+// bf16 packing of dS: integer ALU (add half an ulp, byte permute) or the conversion unit
+__device__ __forceinline__ uint32_t pack_ds(float lo, float hi) {
 #if SSA_KV_PACK_CVT
     return pack_bf16(lo, hi);
 #else
     return pack_bf16_alu(lo, hi);
 #endif
 }
-constexpr int kThr = 128 + 128 * NWG;  // warp 0 TMA, 1 MMA, 2-3 idle, then the compute warps
-constexpr int kComp = 128 * NWG;
-constexpr uint32_t OFF_K = 0;
-constexpr uint32_t OFF_STAGE = TILE_BYTES;
+constexpr int kThr = 384;  // warp 0 TMA, 1 MMA, 2 dS^T stores, 3 idle, 4-11 compute
+constexpr int kComp = 256;
+constexpr uint32_t OFF_STAGE = 0;
 constexpr uint32_t ST_Q = 0, ST_GF = STEP_BYTES, ST_GS = 2 * STEP_BYTES;
 constexpr uint32_t STAGE_BYTES = 3 * STEP_BYTES;
 constexpr int NSTAGE = 3;
-// bf16 [128 keys x 64 queries] tiles, K-major with 128-byte swizzle
+// dS^T, bf16 [128 keys x 64 queries], K-major with 128-byte swizzle, x2
 constexpr uint32_t T_BYTES = 128 * 128;
-constexpr uint32_t OFF_DS = OFF_STAGE + NSTAGE * STAGE_BYTES;  // dS^T
-constexpr uint32_t OFF_PT = OFF_DS + T_BYTES;                  // P_f^T
-constexpr uint32_t OFF_PST = OFF_PT + T_BYTES;                 // P_s^T on mixed steps
+constexpr uint32_t OFF_DS = OFF_STAGE + NSTAGE * STAGE_BYTES;
 // per stage, fp32 over the step's 64 queries: -lse_full*log2(e) | -D_f | -D_s
 constexpr uint32_t ROW_BYTES = 3 * STEP * 4;
-constexpr uint32_t OFF_ROWS = OFF_PST + T_BYTES;
+constexpr uint32_t OFF_ROWS = OFF_DS + 2 * T_BYTES;
+constexpr int NBAR = 24;
 constexpr uint32_t OFF_BAR = OFF_ROWS + NSTAGE * ROW_BYTES;
 // TMEM slot, abort flag, then one selection word per stage (bit 0: the step's
 // query block selects key block kb0, bit 1: selects kb1)
-constexpr uint32_t OFF_MISC = OFF_BAR + 16 * 8;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 32;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 32 + 1024;  // + slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "227 KB of shared memory per CTA");
 enum : int {  // barrier indices, derived from the ring depth
     B_FULL = 0, B_EMPTY = B_FULL + NSTAGE,
-    B_K = B_EMPTY + NSTAGE,  // K tile landed
-    B_OPS = B_K + 1,         // V is in TMEM
-    B_SREADY = B_OPS + 1,    // S^T of the step is in TMEM
-    B_PREADY = B_SREADY + 1, // dP_f^T, dP_s^T of the step are in TMEM
-    B_SFREE = B_PREADY + 1,  // the compute warps have read S^T (may be overwritten)
-    B_PFREE = B_SFREE + 1,   // ... and dP^T
-    B_TREADY = B_PFREE + 1,  // P^T / P_s^T / dS^T tiles written
-    B_TFREE = B_TREADY + 1,  // ... and read by the dV / dK MMAs and the dS^T store
-    B_DONE = B_TFREE + 1, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
+    B_OPS = B_EMPTY + NSTAGE,  // K and V are in TMEM
+    B_SREADY = B_OPS + 1,      // S^T of the step is in TMEM
+    B_SFREE = B_SREADY + 1,    // ... and has been read (the range may be overwritten)
+    B_PSREADY = B_SFREE + 1,   // dP_s^T of a sparse step is in the S range
+    B_PTREADY = B_PSREADY + 1, // P^T (bf16) written over the S range
+    B_PREADY = B_PTREADY + 1,  // dP_f^T of the step is in TMEM
+    B_PFREE = B_PREADY + 1,    // ... and has been read
+    B_DSREADY = B_PFREE + 1,   // x2: dS^T buffer written
+    B_TFREE = B_DSREADY + 2,   // x2: dS^T buffer read by the dK MMAs and the store
+    B_DONE = B_TFREE + 2, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
 };
-static_assert(B_COUNT <= 16, "barrier area holds 16");
-constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_S = 256, TM_V = 320, TM_DPF = 384, TM_DPS = 448;
+static_assert(B_COUNT <= NBAR, "barrier area");
+constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_K = 256, TM_V = 320, TM_S = 384, TM_DPF = 448;
+// bf16 P^T of warpgroup w over the first 16 of its 32 S columns, the masked
+// copy in the other 16: TMEM column of the A operand's k-step kk (16 queries)
+__device__ __forceinline__ uint32_t acol(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 }  // namespace kv
 
 __global__ void __launch_bounds__(kv::kThr, 1)
-bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_gf, const __grid_constant__ CUtensorMap tm_gs,
-                   const __grid_constant__ CUtensorMap tm_ds, const __nv_bfloat16* __restrict__ v,
+bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_gf,
+                   const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_ds,
+                   const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                    const BwdArgs a) {
     using namespace kv;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const uint32_t base = smem_u32(smem_raw);
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gbase = smem_raw + (base - raw);
     unsigned int* status = &g_bwd_tc_status;
-    // the swizzled tiles need a 1024-byte aligned base and the layout leaves no
-    // room to realign: refuse (status bit 1) rather than misplace them
-    if (base & 1023u) {
-        if (threadIdx.x == 0) atomicOr(status, 2u);
-        return;
-    }
-    uint8_t* gbase = smem_raw;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_MISC + 4);
     uint32_t* flags = reinterpret_cast<uint32_t*>(gbase + OFF_MISC + 8);
@@ -320,14 +314,17 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             mbar_init(BAR(B_FULL + s), 1);
             mbar_init(BAR(B_EMPTY + s), 1);
         }
-        mbar_init(BAR(B_K), 1);
         mbar_init(BAR(B_OPS), kComp);
         mbar_init(BAR(B_SREADY), 1);
-        mbar_init(BAR(B_PREADY), 1);
         mbar_init(BAR(B_SFREE), kComp);
+        mbar_init(BAR(B_PSREADY), 1);
+        mbar_init(BAR(B_PTREADY), kComp);
+        mbar_init(BAR(B_PREADY), 1);
         mbar_init(BAR(B_PFREE), kComp);
-        mbar_init(BAR(B_TREADY), kComp);
-        mbar_init(BAR(B_TFREE), 2);  // MMA commit + the dS^T store's source read
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR(B_DSREADY + b), kComp);
+            mbar_init(BAR(B_TFREE + b), 2);  // MMA commit + the dS^T store's source read
+        }
         mbar_init(BAR(B_DONE), 1);
         mbar_init(BAR(B_DRAIN), 1);
         *abort_flag = 0;
@@ -351,14 +348,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (warp == 0) {
         // -------------------------------------------- TMA producer (whole warp)
         if (elect_one()) {
-            prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_gf);
             prefetch_tmap(&tm_gs);
             prefetch_tmap(&tm_ds);
-            mbar_expect_tx(BAR(B_K), TILE_BYTES);
-            tma_load_3d(base + OFF_K, &tm_k, BAR(B_K), 0, s0, bh);
-            tma_load_3d(base + OFF_K + BOX_T, &tm_k, BAR(B_K), 64, s0, bh);
         }
         __syncwarp();
         int issued[NSTAGE];
@@ -395,7 +388,6 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             __syncwarp();
             issued[s] = i;
         }
-        wait_drain(BAR(B_K), 0, kDrainLimitNs);
         if (*abort_flag)
             for (int s = 0; s < NSTAGE; ++s)
                 if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
@@ -405,156 +397,170 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             // and its commits are issued by one elected lane
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S^T, dP^T
             constexpr uint32_t id_a = idesc_bf16_f32(TILE, HD, true);     // dV, dK
-            const uint64_t kdesc = smem_desc_sw128(base + OFF_K, 16, 1024);
             const uint64_t st_k0 = smem_desc_sw128(base + OFF_STAGE, 16, 1024);      // K-major
             const uint64_t st_m0 = smem_desc_sw128(base + OFF_STAGE, BOX_S, 1024);   // MN-major
-            const uint64_t dsd = smem_desc_sw128(base + OFF_DS, 16, 1024);           // K-major A
-            const uint64_t ptd = smem_desc_sw128(base + OFF_PT, 16, 1024);
-            const uint64_t pstd = smem_desc_sw128(base + OFF_PST, 16, 1024);
-            auto kq = [](int kk) { return (uint32_t)((kk >> 2) * BOX_T + (kk & 3) * 32); };
+            const uint64_t ds_0 = smem_desc_sw128(base + OFF_DS, 16, 1024);          // K-major A
             auto ks = [](int kk) { return (uint32_t)((kk >> 2) * BOX_S + (kk & 3) * 32); };
-            auto issue_s = [&](int i) {  // S^T = K Q^T
-                const uint64_t qd = desc_add(st_k0, (i % NSTAGE) * STAGE_BYTES + ST_Q);
-                if (elect_one()) {
+            // D (TMEM) += A (TMEM, K or V) x B^T (64 rows of the stage, K-major)
+            auto issue_tn = [&](uint32_t d, uint32_t a_col, uint32_t st_off) {
+                const uint64_t bd = desc_add(st_k0, st_off);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ss(tmem + TM_S, desc_add(kdesc, kq(kk)), desc_add(qd, ks(kk)), id_s, kk > 0);
-                    mma_commit(BAR(B_SREADY));
-                }
-                __syncwarp();
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + d, tmem + a_col + 8 * kk, desc_add(bd, ks(kk)), id_s, kk > 0);
             };
-            auto issue_dp = [&](int i) {  // dP_f^T = V G_f^T, dP_s^T = V G_s'^T (V in TMEM)
-                const uint32_t s = i % NSTAGE;
-                const uint64_t gfd = desc_add(st_k0, s * STAGE_BYTES + ST_GF);
-                const uint64_t gsd = desc_add(st_k0, s * STAGE_BYTES + ST_GS);
-                const bool sp = flags[s] != 0u;
+            auto stage_off = [&](int i) { return (uint32_t)((i % NSTAGE) * STAGE_BYTES); };
+            bool ok = wait(B_OPS, 0) && wait(B_FULL, 0);
+            if (ok) {
                 if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tmem + TM_DPF, tmem + TM_V + 8 * kk, desc_add(gfd, ks(kk)), id_s, kk > 0);
-                    if (sp) {
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_ts(tmem + TM_DPS, tmem + TM_V + 8 * kk, desc_add(gsd, ks(kk)), id_s,
-                                   kk > 0);
-                    }
+                    issue_tn(TM_S, TM_K, stage_off(0) + ST_Q);  // S^T_0
+                    mma_commit(BAR(B_SREADY));
+                    issue_tn(TM_DPF, TM_V, stage_off(0) + ST_GF);  // dP_f^T_0
                     mma_commit(BAR(B_PREADY));
                 }
                 __syncwarp();
-            };
-            auto issue_acc = [&](int i) {  // dV += P_f^T G_f + P_s^T G_s', dK += dS^T Q
-                const uint32_t s = i % NSTAGE;
-                const uint64_t gfm = desc_add(st_m0, s * STAGE_BYTES + ST_GF);
-                const uint64_t gsm = desc_add(st_m0, s * STAGE_BYTES + ST_GS);
-                const uint64_t qm = desc_add(st_m0, s * STAGE_BYTES + ST_Q);
-                const uint32_t fl = flags[s];
-                // P_s^T = P_f^T on selected key rows (c_t is folded into G_s'); the
-                // row-masked copy is needed only when the tile's two key blocks differ
-                const uint64_t psd = (fl == 1u || fl == 2u) ? pstd : ptd;
-                if (elect_one()) {
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + TM_DV, desc_add(ptd, kk * 32), desc_add(gfm, kk * 2048), id_a,
-                               (i > 0 || kk > 0) ? 1u : 0u);
-                    if (fl != 0u) {
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_ss(tmem + TM_DV, desc_add(psd, kk * 32), desc_add(gsm, kk * 2048), id_a, 1u);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tmem + TM_DK, desc_add(dsd, kk * 32), desc_add(qm, kk * 2048), id_a,
-                               (i > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(BAR(B_EMPTY + s));
-                    mma_commit(BAR(B_TFREE));
-                }
-                __syncwarp();
-            };
-            bool ok = wait(B_K, 0) && wait(B_OPS, 0) && wait(B_FULL, 0);
-            if (ok) {
-                issue_s(0);
-                issue_dp(0);
             }
+            int nsp = 0;  // sparse steps so far (phase of B_PSREADY)
             for (int i = 0; ok && i < ns; ++i) {
-                if (i + 1 < ns) {
-                    if (!wait(B_FULL + (i + 1) % NSTAGE, ((i + 1) / NSTAGE) & 1) || !wait(B_SFREE, i & 1)) {
+                const int s = i % NSTAGE, b = i & 1;
+                const uint32_t fl = flags[s];
+                const bool sp = fl != 0u;
+                // (a) dP_s^T into the S range once S^T has been read
+                if (sp) {
+                    if (!wait(B_SFREE, i & 1)) {
                         ok = false;
                         break;
                     }
-                    issue_s(i + 1);
+                    if (elect_one()) {
+                        issue_tn(TM_S, TM_V, stage_off(i) + ST_GS);
+                        mma_commit(BAR(B_PSREADY));
+                    }
+                    __syncwarp();
+                    ++nsp;
+                }
+                // (b) dV += P_f^T G_f (+ P_s^T G_s') once P^T is in TMEM, then S^T of
+                // the next step into the same columns (the MMAs run in issue order)
+                if (!wait(B_PTREADY, i & 1)) {
+                    ok = false;
+                    break;
+                }
+                const bool more = i + 1 < ns;
+                if (more && !wait(B_FULL + (i + 1) % NSTAGE, ((i + 1) / NSTAGE) & 1)) {
+                    ok = false;
+                    break;
+                }
+                // P_s^T = P_f^T on selected key rows (c_t is folded into G_s'); the
+                // row-masked copy is needed only when the tile's two key blocks differ
+                const uint32_t ps_off = (fl == 1u || fl == 2u) ? 16u : 0u;
+                if (elect_one()) {
+                    const uint64_t gfm = desc_add(st_m0, stage_off(i) + ST_GF);
+                    const uint64_t gsm = desc_add(st_m0, stage_off(i) + ST_GS);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tmem + TM_DV, tmem + TM_S + acol(kk), desc_add(gfm, kk * 2048), id_a,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                    if (sp) {
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_ts(tmem + TM_DV, tmem + TM_S + acol(kk) + ps_off, desc_add(gsm, kk * 2048),
+                                   id_a, 1u);
+                    }
+                    if (more) {
+                        issue_tn(TM_S, TM_K, stage_off(i + 1) + ST_Q);
+                        mma_commit(BAR(B_SREADY));
+                    }
+                }
+                __syncwarp();
+                // (c) dP_f^T of the next step once this one's has been read
+                if (more) {
                     if (!wait(B_PFREE, i & 1)) {
                         ok = false;
                         break;
                     }
-                    issue_dp(i + 1);
+                    if (elect_one()) {
+                        issue_tn(TM_DPF, TM_V, stage_off(i + 1) + ST_GF);
+                        mma_commit(BAR(B_PREADY));
+                    }
+                    __syncwarp();
                 }
-                if (!wait(B_TREADY, i & 1)) {
+                // (d) dK += dS^T Q once dS^T is in shared memory
+                if (!wait(B_DSREADY + b, (i >> 1) & 1)) {
                     ok = false;
                     break;
                 }
-                // dS^T of the step to global memory for the dQ GEMM (lane 0 owns the
-                // bulk group), then the dV / dK MMAs on the same tiles
-                if (lane == 0) {
-                    tma_store_3d(&tm_ds, base + OFF_DS, 0, 0, ds_blk0 + i);
-                    bulk_commit_group();
-                }
-                issue_acc(i);
-                if (lane == 0) {
-                    bulk_wait_group_read0();
-                    mbar_arrive(BAR(B_TFREE));
+                if (elect_one()) {
+                    const uint64_t qm = desc_add(st_m0, stage_off(i) + ST_Q);
+                    const uint64_t dd = desc_add(ds_0, b * T_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tmem + TM_DK, desc_add(dd, kk * 32), desc_add(qm, kk * 2048), id_a,
+                               (i > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(BAR(B_EMPTY + s));
+                    mma_commit(BAR(B_TFREE + b));
                 }
                 __syncwarp();
             }
+            (void)nsp;
             if (elect_one()) {
                 mma_commit(BAR(B_DONE));
                 mma_commit(BAR(B_DRAIN));
             }
             __syncwarp();
             wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
-            if (lane == 0) bulk_wait_group0();  // the dS^T stores are complete
         }
+    } else if (warp == 2) {
+        // ------------------------------------------ dS^T stores for the dQ GEMM
+        // (lane 0 owns the bulk group; off the MMA issuer's path)
+        for (int i = 0; i < ns; ++i) {
+            const int b = i & 1;
+            if (!wait(B_DSREADY + b, (i >> 1) & 1)) break;
+            if (lane == 0) {
+                tma_store_3d(&tm_ds, base + OFF_DS + b * T_BYTES, 0, 0, ds_blk0 + i);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+                mbar_arrive(BAR(B_TFREE + b));
+            }
+            __syncwarp();
+        }
+        if (lane == 0) bulk_wait_group0();  // the dS^T stores are complete
+        __syncwarp();
     } else if (warp >= 4) {
-        // ------------------------------------------ compute warpgroups
-        // warpgroup wg handles query columns [COLS wg, COLS wg + COLS) of every step
+        // ------------------------------------------ two compute warpgroups
+        // warpgroup wg handles query columns [32 wg, 32 wg + 32) of every step
         const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
         const int r = sw * 32 + lane;  // key row of the tile == TMEM lane
         const int s_tok = s0 + r;
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
         const float sl2 = a.scale_log2;
         const bool in_kb1 = r >= 64 && a.block == 64;  // warp-uniform
-        const bool key_ok = s_tok < a.T;
+        const bool key_ok = s_tok < a.T;                // warp-uniform (T is a multiple of 64)
         const int c0 = COLS * wg;
         bool ok = true;
-        {  // V rows of the tile (this warpgroup's HD/NWG columns) into TMEM
-            constexpr int W = HD / NWG / 2;  // 32-bit TMEM columns per warpgroup
-            uint32_t u[W];
-            const uint4* p4 = reinterpret_cast<const uint4*>(v + (rowbase + (s_tok < a.T ? s_tok : 0)) * HD +
-                                                             2 * W * wg);
+        {  // K and V rows of the tile (this warpgroup's 64 columns of each) into TMEM
+            const size_t row = rowbase + (key_ok ? s_tok : 0);
+            auto fill = [&](const __nv_bfloat16* src, uint32_t col) {
+                uint32_t u[32];
+                const uint4* p4 = reinterpret_cast<const uint4*>(src + row * HD + 64 * wg);
 #pragma unroll
-            for (int v4 = 0; v4 < W / 4; ++v4) {
-                const uint4 x = s_tok < a.T ? __ldg(p4 + v4) : make_uint4(0u, 0u, 0u, 0u);
-                u[4 * v4] = x.x;
-                u[4 * v4 + 1] = x.y;
-                u[4 * v4 + 2] = x.z;
-                u[4 * v4 + 3] = x.w;
-            }
-            tmem_st<W>(trow + TM_V + W * wg, u);
+                for (int v4 = 0; v4 < 8; ++v4) {
+                    const uint4 x = key_ok ? __ldg(p4 + v4) : make_uint4(0u, 0u, 0u, 0u);
+                    u[4 * v4] = x.x;
+                    u[4 * v4 + 1] = x.y;
+                    u[4 * v4 + 2] = x.z;
+                    u[4 * v4 + 3] = x.w;
+                }
+                tmem_st32(trow + col + 32 * wg, u);
+            };
+            fill(k, TM_K);
+            fill(v, TM_V);
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_OPS));
         }
         const uint32_t rowoff = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
-        auto put_row = [&](uint32_t tile, const uint32_t (&w)[COLS / 2]) {  // swizzled row r
-#pragma unroll
-            for (int q4 = 0; q4 < COLS / 8; ++q4) {
-                const uint32_t chunk = (uint32_t)((c0 >> 3) + q4) ^ (uint32_t)(r & 7);
-                *reinterpret_cast<uint4*>(gbase + tile + rowoff + chunk * 16) =
-                    make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-            }
-        };
+        int nsp = 0;
         for (int i = 0; i < ns; ++i) {
             const int t0 = s0 + STEP * i;
-            const int s = i % NSTAGE;
+            const int s = i % NSTAGE, b = i & 1;
             // the stage's row vectors and selection word (already landed: the MMA
             // warp waited for them before issuing this step's S^T)
             if (!wait(B_FULL + s, (i / NSTAGE) & 1) || !wait(B_SREADY, i & 1)) {
@@ -562,6 +568,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 break;
             }
             const uint32_t fl = flags[s];
+            const bool sp = fl != 0u;
             const bool use_s = in_kb1 ? (fl >> 1) & 1u : fl & 1u;
             const bool mixed = fl == 1u || fl == 2u;
             const bool diag = t0 < s0 + TILE;
@@ -570,10 +577,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             uint32_t pfk[COLS / 2];
             {
                 uint32_t su[COLS];
-                tmem_ld<COLS>(trow + TM_S + c0, su);
+                tmem_ld32(trow + TM_S + c0, su);
                 tmem_wait_ld();
                 fence_before_sync();
-                mbar_arrive(BAR(B_SFREE));  // S^T may now be overwritten by the next step
+                mbar_arrive(BAR(B_SFREE));  // the S range may now take dP_s^T
                 const float4* L4 = reinterpret_cast<const float4*>(rw + c0);
                 const f32x2 sl2x2 = mk2(sl2, sl2);
 #pragma unroll
@@ -583,7 +590,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                                            sl2x2, mk2(L.x, L.y));
                     const f32x2 x23 = fma2(mk2(__uint_as_float(su[4 * j4 + 2]), __uint_as_float(su[4 * j4 + 3])),
                                            sl2x2, mk2(L.z, L.w));
-                    if (2 * j4 >= COLS / 2 - kPolyPairs) {  // part of the exponentials on the FMA pipe
+                    if (2 * j4 >= COLS / 2 - kPolyPairs) {
                         un2(exp2_poly2(x01), pf[4 * j4], pf[4 * j4 + 1]);
                         un2(exp2_poly2(x23), pf[4 * j4 + 2], pf[4 * j4 + 3]);
                     } else {
@@ -602,20 +609,43 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         if (t0 + c0 + j < s_tok) pf[j] = 0.f;
                 }
 #pragma unroll
-                for (int j2 = 0; j2 < COLS / 2; ++j2) pfk[j2] = pack2(pf[2 * j2], pf[2 * j2 + 1]);
+                for (int j2 = 0; j2 < COLS / 2; ++j2) pfk[j2] = pack_bf16_alu(pf[2 * j2], pf[2 * j2 + 1]);
             }
+            // dP_s^T (sparse steps) comes through the S range: read it before P^T
+            // overwrites those columns
+            uint32_t pu[COLS];
+            if (sp) {
+                if (!wait(B_PSREADY, nsp & 1)) {
+                    ok = false;
+                    break;
+                }
+                ++nsp;
+                if (use_s) {
+                    tmem_ld32(trow + TM_S + c0, pu);
+                    tmem_wait_ld();
+                }
+            }
+            tmem_st<16>(trow + TM_S + c0, pfk);
+            if (mixed) {  // the sparse stream's P^T: zero on unselected key rows
+                if (!use_s)
+#pragma unroll
+                    for (int e = 0; e < COLS / 2; ++e) pfk[e] = 0u;
+                tmem_st<16>(trow + TM_S + c0 + 16, pfk);
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            mbar_arrive(BAR(B_PTREADY));
             if (!wait(B_PREADY, i & 1)) {
                 ok = false;
                 break;
             }
             uint32_t dsk[COLS / 2];
             {
-                uint32_t fu[COLS], pu[COLS];
-                tmem_ld<COLS>(trow + TM_DPF + c0, fu);
-                if (use_s) tmem_ld<COLS>(trow + TM_DPS + c0, pu);
+                uint32_t fu[COLS];
+                tmem_ld32(trow + TM_DPF + c0, fu);
                 tmem_wait_ld();
                 fence_before_sync();
-                mbar_arrive(BAR(B_PFREE));  // dP^T may now be overwritten by the next step
+                mbar_arrive(BAR(B_PFREE));  // dP_f^T may now be overwritten by the next step
                 const float4* F4 = reinterpret_cast<const float4*>(rw + STEP + c0);
                 const float4* S4 = reinterpret_cast<const float4*>(rw + 2 * STEP + c0);
 #pragma unroll
@@ -635,37 +665,36 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     float d0, d1, d2, d3;
                     un2(mul2(mk2(pf[4 * j4], pf[4 * j4 + 1]), g01), d0, d1);
                     un2(mul2(mk2(pf[4 * j4 + 2], pf[4 * j4 + 3]), g23), d2, d3);
-                    dsk[2 * j4] = pack2(d0, d1);
-                    dsk[2 * j4 + 1] = pack2(d2, d3);
+                    dsk[2 * j4] = pack_ds(d0, d1);
+                    dsk[2 * j4 + 1] = pack_ds(d2, d3);
                 }
-                if (!key_ok) {  // stored dS^T rows past T stay zero (warp-uniform)
+                if (!key_ok) {  // stored dS^T rows past T stay zero
 #pragma unroll
                     for (int e = 0; e < COLS / 2; ++e) dsk[e] = 0u;
                 }
             }
-            // the tiles are single-buffered: wait for the previous step's dV / dK MMAs
-            if (i > 0 && !wait(B_TFREE, (i - 1) & 1)) {
+            // dS^T row r into buffer b once the dK MMAs and the store of step i-2 read it
+            if (i >= 2 && !wait(B_TFREE + b, ((i >> 1) + 1) & 1)) {
                 ok = false;
                 break;
             }
-            put_row(OFF_PT, pfk);
-            put_row(OFF_DS, dsk);
-            if (mixed) {  // the sparse stream's P^T: zero on unselected key rows
-                if (!use_s)
+            {
+                uint8_t* dsb = gbase + OFF_DS + b * T_BYTES + rowoff;
 #pragma unroll
-                    for (int e = 0; e < COLS / 2; ++e) pfk[e] = 0u;
-                put_row(OFF_PST, pfk);
+                for (int q4 = 0; q4 < COLS / 8; ++q4) {
+                    const uint32_t chunk = (uint32_t)((c0 >> 3) + q4) ^ (uint32_t)(r & 7);
+                    *reinterpret_cast<uint4*>(dsb + chunk * 16) =
+                        make_uint4(dsk[4 * q4], dsk[4 * q4 + 1], dsk[4 * q4 + 2], dsk[4 * q4 + 3]);
+                }
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the MMAs
-            mbar_arrive(BAR(B_TREADY));
+            mbar_arrive(BAR(B_DSREADY + b));
         }
         if (ok) ok = wait(B_DONE, 0);
         if (ok) {
-            const bool valid = s_tok < a.T;
-            const size_t row = rowbase + (valid ? s_tok : 0);
-            constexpr int OC = HD / NWG;  // output columns per warpgroup
-            store_row_cols<OC / 32>(trow + TM_DV + OC * wg, 1.f, a.dv + row * HD + OC * wg, valid);
-            store_row_cols<OC / 32>(trow + TM_DK + OC * wg, a.sm_scale, a.dk + row * HD + OC * wg, valid);
+            const size_t row = rowbase + (key_ok ? s_tok : 0);
+            store_row_cols<2>(trow + TM_DV + 64 * wg, 1.f, a.dv + row * HD + 64 * wg, key_ok);
+            store_row_cols<2>(trow + TM_DK + 64 * wg, a.sm_scale, a.dk + row * HD + 64 * wg, key_ok);
         }
     }
     fence_before_sync();
@@ -981,7 +1010,8 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
         a.timeout_ns = wait_limit_ns();
         const unsigned grid = (unsigned)((size_t)nh * ntile);
         bwd_dkdv_tc_kernel<<<grid, kv::kThr, kv::SMEM_BYTES, s>>>(
-            k128, q64, gf64, gs64, ds_map, static_cast<const __nv_bfloat16*>(off(v)), a);
+            q64, gf64, gs64, ds_map, static_cast<const __nv_bfloat16*>(off(k)),
+            static_cast<const __nv_bfloat16*>(off(v)), a);
         st = check_launch("bwd_dkdv_tc_kernel");
         if (st != SSA_OK) break;
         if (h0 == 0) mark_kernel_event(2, s);
@@ -999,8 +1029,6 @@ int bwd_tc_take_status(cudaStream_t) {
     if (v) {
         const unsigned int zero = 0;
         cudaMemcpyToSymbol(g_bwd_tc_status, &zero, sizeof zero);
-        if (v & 2u)
-            return fail(SSA_ERR_CUDA, "bwd tcgen05 kernels: dynamic shared memory not 1024-byte aligned");
         return fail(SSA_ERR_TIMEOUT, "bwd tcgen05 kernels: a bounded mbarrier wait expired");
     }
     return SSA_OK;
