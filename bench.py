@@ -124,17 +124,45 @@ def ncu_traffic(kernel_key):
 
 
 class ClockSampler:
-    """nvidia-smi samples (200 ms) while the timed region runs."""
+    """SM clock and clock-event reasons while the timed region runs: NVML read
+    every 5 ms from a thread (reads only, no setting is changed), plus
+    nvidia-smi at 200 ms as a second source."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h): sw power cap, hw slowdown, sw/hw thermal
+    NVML_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                 "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
         self.file = None
+        self.nvml = []
+        self._stop = None
+        self._thread = None
+
+    def _nvml_loop(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            while not self._stop.is_set():
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                self.nvml.append((sm, mx, get_reasons(h)))
+                self._stop.wait(0.005)
+            pynvml.nvmlShutdown()
+        except Exception:  # NVML unavailable: nvidia-smi samples only
+            pass
 
     def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._nvml_loop, daemon=True)
+        self._thread.start()
         try:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
@@ -145,6 +173,8 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        self._stop.set()
+        self._thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -153,27 +183,31 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if self.proc is None or self.file is None:
-            return None
-        self.file.flush()
-        with open(self.file.name) as f:
-            rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
-        os.unlink(self.file.name)
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
-            except (ValueError, IndexError):
-                continue
-            for n, v in zip(names, r[4:8]):
-                if v.strip().lower() == "active":
-                    reasons.add(n)
+        for c, m, bits in self.nvml:
+            sm.append(float(c))
+            mx.append(float(m))
+            reasons.update(n for n, bit in self.NVML_BITS.items() if bits & bit)
+        src = "nvml" if sm else None
+        if self.file is not None:
+            self.file.flush()
+            with open(self.file.name) as f:
+                rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+            os.unlink(self.file.name)
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for r in rows:
+                try:
+                    c, m = float(r[1]), float(r[2])
+                except (ValueError, IndexError):
+                    continue
+                sm.append(c)
+                mx.append(m)
+                reasons.update(n for n, v in zip(names, r[4:8]) if v.strip().lower() == "active")
+                src = "nvml+nvidia-smi" if src else "nvidia-smi"
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": src}
 
 
 # ----------------------------------------------------------------------------- our arm
