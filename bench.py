@@ -24,6 +24,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import ctypes
+import dataclasses
 import json
 import math
 import os
@@ -281,7 +282,7 @@ class Layer:
 
 
 def run_ours(args, rank, world, dev, peaks, peak_src):
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     torch.cuda.set_device(dev)
     inp = make_inputs(w)
     grads = upstream_grads(w)
@@ -336,11 +337,16 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
             kms["bwd_dkdv_tc_kernel"] += ks[1].elapsed_time(ks[2]) / args.steps
             kms["bwd_dq_gemm_kernel"] += ks[2].elapsed_time(ks[3]) / args.steps
         kfl = kernel_flops(w, p_full, p_sel)
+        # the events bracket the backward kernels of the first group of heads
+        group = layer.ssa.ssa_bwd_heads_per_group(layer.p) / (w.B * w.H)
+        for k in ("bwd_dkdv_tc_kernel", "bwd_dq_gemm_kernel"):
+            kfl[k] *= group
         kernels = {k: {"ms": round(v, 4)} for k, v in kms.items()}
+        kernels["bwd_heads_per_group"] = layer.ssa.ssa_bwd_heads_per_group(layer.p)
         for k, f in kfl.items():
             kernels[k]["tflops"] = round(f / (kms[k] * 1e-3) / 1e12, 2)
         # the dQ GEMM streams the stored dS^T blocks: its own bound is HBM
-        dq_bytes = (ds_blocks_per_bh(w.T) * 64 * 128 * 2 + 2 * w.T * w.D * 2) * w.B * w.H
+        dq_bytes = round((ds_blocks_per_bh(w.T) * 64 * 128 * 2 + 2 * w.T * w.D * 2) * w.B * w.H * group)
         kernels["bwd_dq_gemm_kernel"]["hbm_gbs"] = round(dq_bytes / (kms["bwd_dq_gemm_kernel"] * 1e-3) / 1e9, 1)
         kernels["bwd_dq_gemm_kernel"]["hbm_bytes"] = dq_bytes
         dom = max(kfl, key=lambda k: kms[k])
@@ -455,7 +461,10 @@ def blas_threads():
         return os.cpu_count()
 
 
-def cpu_baseline(w, inp, grads, slices=8, rows_per_slice=1024):
+def cpu_baseline(w, inp, grads, slices=8):
+    """The oracle on a bounded sample: `slices` runs of query rows at the end
+    of head (0, 0), about 8192 x 8192 row-key pairs in all at any T."""
+    rows_per_slice = min(w.T, 8 * 1024 * 8192 // w.T) // slices
     flops = secs = 0.0
     for s in range(slices):
         hi = w.T - s * rows_per_slice
@@ -469,7 +478,7 @@ def cpu_baseline(w, inp, grads, slices=8, rows_per_slice=1024):
 
 
 def run_reference(args, world):
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     inp = make_inputs(w)
     grads = upstream_grads(w)
     rows = 512
@@ -500,6 +509,16 @@ def run_reference(args, world):
 
 # ----------------------------------------------------------------------------- distributed
 
+def workload(args):
+    """The named workload, with the selection budget overridden by --topk."""
+    w = WORKLOADS[args.workload]
+    if args.topk is None or args.topk == w.topk:
+        return w
+    if args.topk not in (getattr(w, "sweep", None) or ()):
+        raise SystemExit(f"--topk {args.topk}: {w.name} sweeps {getattr(w, 'sweep', None)}")
+    return dataclasses.replace(w, topk=args.topk, name=f"{w.name}_k{args.topk}")
+
+
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
@@ -529,6 +548,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--topk", type=int, default=None,
+                    help="selection budget override (one of the workload's sweep values)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -549,7 +570,7 @@ def main(argv=None):
     out = run_ours(args, rank, world, dev, peaks, src)
     if rank == 0:
         if world == 1 and args.cpu_baseline:
-            w = WORKLOADS[args.workload]
+            w = workload(args)
             out["cpu_baseline"] = cpu_baseline(w, make_inputs(w), upstream_grads(w))
         print(json.dumps(out), flush=True)
     if world > 1:

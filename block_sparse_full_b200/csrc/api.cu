@@ -243,6 +243,11 @@ int ssa_kernel_path(const ssa_params_t* p) {
 
 int ssa_version(void) { return (1 << 16) | 0; }
 
+int ssa_bwd_heads_per_group(const ssa_params_t* p) {
+    if (validate(p) != SSA_OK || !use_tc(*p)) return -1;
+    return ssa::bwd_tc_heads_per_group(*p);
+}
+
 void ssa_debug_set_wait_limit_ns(unsigned long long ns) {
     g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs, std::memory_order_relaxed);
 }

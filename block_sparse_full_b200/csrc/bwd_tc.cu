@@ -931,6 +931,8 @@ TcWs carve(const ssa_params_t& p, void* ws) {
 
 }  // namespace
 
+int bwd_tc_heads_per_group(const ssa_params_t& p) { return heads_per_chunk(p); }
+
 bool bwd_tc_supported(const ssa_params_t& p) {
     return p.dtype == SSA_BF16 && p.D == HD && (p.block == 64 || p.block == 128) &&
            (size_t)p.B * p.H * ((p.T + TILE - 1) / TILE) <= 0x7fffffffull &&

@@ -75,6 +75,7 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
                   const void* dh_sparse, float w_s, float w_c, void* dq, void* dk, void* dv,
                   void* ws, cudaStream_t s);
 int bwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
+int bwd_tc_heads_per_group(const ssa_params_t& p);  // heads sharing the dS workspace
 
 // ---- self-tests (selftest.cu)
 int selftest_take_status();  // SSA_ERR_TIMEOUT if the self-test wait expired

@@ -34,7 +34,7 @@ EXPORTS = (
     "ssa_workspace_size", "ssa_select_blocks", "ssa_select_blocks_noalloc",
     "ssa_attn_fwd_dual", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
-    "ssa_kernel_path", "ssa_selftest_math", "ssa_selftest_wait_timeout",
+    "ssa_kernel_path", "ssa_bwd_heads_per_group", "ssa_selftest_math", "ssa_selftest_wait_timeout",
     "ssa_debug_set_wait_limit_ns", "ssa_debug_set_kernel_events", "ssa_version",
 )
 
@@ -74,6 +74,7 @@ _SIGNATURES = {
     "ssa_status_string": (ctypes.c_char_p, [c_int]),
     "ssa_last_error": (ctypes.c_char_p, []),
     "ssa_kernel_path": (c_int, [_P]),
+    "ssa_bwd_heads_per_group": (c_int, [_P]),
     "ssa_selftest_math": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "ssa_version": (c_int, []),
     "ssa_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
@@ -161,6 +162,10 @@ def ssa_selftest_wait_timeout(limit_ns, gave_up, stream):
 
 def ssa_debug_set_wait_limit_ns(ns):
     _lib.ssa_debug_set_wait_limit_ns(ns)
+
+
+def ssa_bwd_heads_per_group(params):
+    return _lib.ssa_bwd_heads_per_group(ctypes.byref(params))
 
 
 def ssa_debug_set_kernel_events(events, n):

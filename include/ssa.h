@@ -198,6 +198,11 @@ const char* ssa_status_string(int status);
 /* Detail of the last error returned on the calling host thread ("" if none). */
 const char* ssa_last_error(void);
 
+/* Heads per group of the tensor-core backward (the dS workspace holds one
+ * group; the groups run one after another; B*H when all fit), or -1 when
+ * the params are invalid or select the CUDA-core path. */
+int ssa_bwd_heads_per_group(const ssa_params_t* params);
+
 /* Which kernel family the params select: 0 = CUDA-core (SIMT) kernels
  * (float32, bf16 with D = 64, or SSA_FLAG_FORCE_SIMT), 1 = bf16 tcgen05
  * tensor-core kernels (D = 128), -1 = invalid or unsupported params. */
@@ -229,8 +234,8 @@ void ssa_debug_set_wait_limit_ns(unsigned long long ns);
  * record the caller's CUDA events (cudaEvent_t, passed as void*) on the call's
  * stream at kernel boundaries: events[0] before the preprocess kernel,
  * events[1] after it, events[2] after the dK/dV kernel and events[3] after
- * the dQ GEMM of the first group of heads (the only group unless the dS
- * buffer is split).  n must be 4 to enable, 0 to disable; the events stay
+ * the dQ GEMM of the first group of heads (ssa_bwd_heads_per_group; the
+ * only group unless the dS buffer is split).  n must be 4 to enable, 0 to disable; the events stay
  * owned by the caller, who must disable the hook before destroying them.
  * Returns SSA_OK or SSA_ERR_INVALID_ARG.  Process-wide, like the hook above. */
 int ssa_debug_set_kernel_events(void* const* events, int n);

@@ -114,3 +114,23 @@ def test_kernel_path_choice():
     assert ssa.ssa_kernel_path(P(dtype=ssa.SSA_F32)) == 0
     assert ssa.ssa_kernel_path(P(D=64)) == 0
     assert ssa.ssa_kernel_path(P(flags=ssa.SSA_FLAG_FORCE_SIMT)) == 0
+
+
+def test_bwd_head_groups_bound_the_ds_workspace():
+    # the tensor-core backward stores bf16 dS blocks of the causal triangle:
+    # (T - 128 J) / 64 blocks of 16 KB for key tile J, within 4 GiB per group
+    def blocks(T):
+        ntk = (T + 127) // 128
+        return ntk * (T // 64) - ntk * (ntk - 1)
+    assert blocks(192) == 4 and blocks(8192) == 4160
+    bench = P(B=1, H=16, T=8192, block=64, topk=16)
+    assert ssa.ssa_bwd_heads_per_group(bench) == 16
+    sink = P(B=1, H=8, T=65536, block=128, topk=16)
+    assert ssa.ssa_bwd_heads_per_group(sink) == 1
+    train = P(B=4, H=32, T=4096, block=64, topk=8)
+    per_head = blocks(4096) * 16 * 1024
+    assert ssa.ssa_bwd_heads_per_group(train) == min(128, (4 << 30) // per_head)
+    assert ssa.ssa_bwd_heads_per_group(P(dtype=ssa.SSA_F32)) == -1
+    # the workspace holds exactly one group's blocks on top of the row data
+    g = ssa.ssa_bwd_heads_per_group(train)
+    assert ssa.ssa_workspace_size(train, ssa.SSA_WS_BWD) >= g * per_head
