@@ -222,12 +222,14 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
 namespace kv {
 // K and V of the tile live in TMEM: the A operands of S^T = K Q^T and
 // dP^T = V G^T (TS form: only the 64-query B tiles are read from shared
-// memory).  Q, G_f, G_s' steps stream through a ring.  One 64-column TMEM
-// range holds, in turn within a step, S^T, then (on sparse steps) dP_s^T,
-// then the bf16 P^T that feeds dV += P^T G_f (+ the sparse stream's
-// row-masked copy next to it on mixed steps); S^T of the next step is issued
-// behind the dV MMAs.  dS^T goes to a double-buffered swizzled shared tile:
-// the A operand of dK += dS^T Q and the source of its TMA store for the dQ GEMM.
+// memory).  Q, G_f, G_s' steps stream through a ring.  The S range holds S^T
+// and then, on sparse steps, dP_s^T; once the compute warps have read them
+// the next step's S^T goes there.  The dP range holds dP_f^T and then the
+// bf16 P^T that feeds dV += P^T G_f (+ the sparse stream's row-masked copy
+// next to it on mixed steps); the next step's dP_f^T is issued behind the dV
+// MMAs, and is needed only after the next step's exponentials.  dS^T goes
+// to a double-buffered swizzled shared tile: the A operand of dK += dS^T Q
+// and the source of its TMA store for the dQ GEMM.
 constexpr int COLS = 32;  // query columns per compute warpgroup (two warpgroups)
 // of a thread's 16 exponential pairs per step, this many (the last ones) run
 // as a polynomial on the FMA pipe instead of the MUFU unit
@@ -266,16 +268,16 @@ enum : int {  // barrier indices, derived from the ring depth
     B_SREADY = B_OPS + 1,      // S^T of the step is in TMEM
     B_SFREE = B_SREADY + 1,    // ... and has been read (the range may be overwritten)
     B_PSREADY = B_SFREE + 1,   // dP_s^T of a sparse step is in the S range
-    B_PTREADY = B_PSREADY + 1, // P^T (bf16) written over the S range
-    B_PREADY = B_PTREADY + 1,  // dP_f^T of the step is in TMEM
-    B_PFREE = B_PREADY + 1,    // ... and has been read
-    B_DSREADY = B_PFREE + 1,   // x2: dS^T buffer written
+    B_PSFREE = B_PSREADY + 1,  // ... and has been read
+    B_PREADY = B_PSFREE + 1,   // dP_f^T of the step is in the dP range
+    B_PTREADY = B_PREADY + 1,  // ... has been read and P^T (bf16) written over it
+    B_DSREADY = B_PTREADY + 1, // x2: dS^T buffer written
     B_TFREE = B_DSREADY + 2,   // x2: dS^T buffer read by the dK MMAs and the store
     B_DONE = B_TFREE + 2, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
 };
 static_assert(B_COUNT <= NBAR, "barrier area");
 constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_K = 256, TM_V = 320, TM_S = 384, TM_DPF = 448;
-// bf16 P^T of warpgroup w over the first 16 of its 32 S columns, the masked
+// bf16 P^T of warpgroup w over the first 16 of its 32 dP columns, the masked
 // copy in the other 16: TMEM column of the A operand's k-step kk (16 queries)
 __device__ __forceinline__ uint32_t acol(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 }  // namespace kv
@@ -318,9 +320,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         mbar_init(BAR(B_SREADY), 1);
         mbar_init(BAR(B_SFREE), kComp);
         mbar_init(BAR(B_PSREADY), 1);
-        mbar_init(BAR(B_PTREADY), kComp);
+        mbar_init(BAR(B_PSFREE), kComp);
         mbar_init(BAR(B_PREADY), 1);
-        mbar_init(BAR(B_PFREE), kComp);
+        mbar_init(BAR(B_PTREADY), kComp);
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR(B_DSREADY + b), kComp);
             mbar_init(BAR(B_TFREE + b), 2);  // MMA commit + the dS^T store's source read
@@ -419,32 +421,46 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 __syncwarp();
             }
-            int nsp = 0;  // sparse steps so far (phase of B_PSREADY)
+            int nsp = 0;  // sparse steps so far (phase of B_PSREADY / B_PSFREE)
             for (int i = 0; ok && i < ns; ++i) {
                 const int s = i % NSTAGE, b = i & 1;
                 const uint32_t fl = flags[s];
                 const bool sp = fl != 0u;
-                // (a) dP_s^T into the S range once S^T has been read
-                if (sp) {
+                const bool more = i + 1 < ns;
+                // (a) S range: dP_s^T once S^T has been read (sparse steps), then the
+                // next step's S^T once that has been read too
+                if (sp || more) {
                     if (!wait(B_SFREE, i & 1)) {
                         ok = false;
                         break;
                     }
+                }
+                if (sp) {
                     if (elect_one()) {
                         issue_tn(TM_S, TM_V, stage_off(i) + ST_GS);
                         mma_commit(BAR(B_PSREADY));
                     }
                     __syncwarp();
+                    if (more && !wait(B_PSFREE, nsp & 1)) {
+                        ok = false;
+                        break;
+                    }
                     ++nsp;
                 }
-                // (b) dV += P_f^T G_f (+ P_s^T G_s') once P^T is in TMEM, then S^T of
-                // the next step into the same columns (the MMAs run in issue order)
-                if (!wait(B_PTREADY, i & 1)) {
-                    ok = false;
-                    break;
+                if (more) {
+                    if (!wait(B_FULL + (i + 1) % NSTAGE, ((i + 1) / NSTAGE) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    if (elect_one()) {
+                        issue_tn(TM_S, TM_K, stage_off(i + 1) + ST_Q);
+                        mma_commit(BAR(B_SREADY));
+                    }
+                    __syncwarp();
                 }
-                const bool more = i + 1 < ns;
-                if (more && !wait(B_FULL + (i + 1) % NSTAGE, ((i + 1) / NSTAGE) & 1)) {
+                // (b) dP range: dV += P_f^T G_f (+ P_s^T G_s') once P^T has replaced
+                // dP_f^T there, then dP_f^T of the next step (the MMAs run in order)
+                if (!wait(B_PTREADY, i & 1)) {
                     ok = false;
                     break;
                 }
@@ -456,33 +472,21 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const uint64_t gsm = desc_add(st_m0, stage_off(i) + ST_GS);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tmem + TM_DV, tmem + TM_S + acol(kk), desc_add(gfm, kk * 2048), id_a,
+                        mma_ts(tmem + TM_DV, tmem + TM_DPF + acol(kk), desc_add(gfm, kk * 2048), id_a,
                                (i > 0 || kk > 0) ? 1u : 0u);
                     if (sp) {
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_ts(tmem + TM_DV, tmem + TM_S + acol(kk) + ps_off, desc_add(gsm, kk * 2048),
+                            mma_ts(tmem + TM_DV, tmem + TM_DPF + acol(kk) + ps_off, desc_add(gsm, kk * 2048),
                                    id_a, 1u);
                     }
                     if (more) {
-                        issue_tn(TM_S, TM_K, stage_off(i + 1) + ST_Q);
-                        mma_commit(BAR(B_SREADY));
-                    }
-                }
-                __syncwarp();
-                // (c) dP_f^T of the next step once this one's has been read
-                if (more) {
-                    if (!wait(B_PFREE, i & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    if (elect_one()) {
                         issue_tn(TM_DPF, TM_V, stage_off(i + 1) + ST_GF);
                         mma_commit(BAR(B_PREADY));
                     }
-                    __syncwarp();
                 }
-                // (d) dK += dS^T Q once dS^T is in shared memory
+                __syncwarp();
+                // (c) dK += dS^T Q once dS^T is in shared memory
                 if (!wait(B_DSREADY + b, (i >> 1) & 1)) {
                     ok = false;
                     break;
@@ -611,8 +615,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                 for (int j2 = 0; j2 < COLS / 2; ++j2) pfk[j2] = pack_bf16_alu(pf[2 * j2], pf[2 * j2 + 1]);
             }
-            // dP_s^T (sparse steps) comes through the S range: read it before P^T
-            // overwrites those columns
+            // dP_s^T (sparse steps) comes through the S range after S^T
             uint32_t pu[COLS];
             if (sp) {
                 if (!wait(B_PSREADY, nsp & 1)) {
@@ -624,17 +627,9 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tmem_ld32(trow + TM_S + c0, pu);
                     tmem_wait_ld();
                 }
+                fence_before_sync();
+                mbar_arrive(BAR(B_PSFREE));  // the S range may take the next S^T
             }
-            tmem_st<16>(trow + TM_S + c0, pfk);
-            if (mixed) {  // the sparse stream's P^T: zero on unselected key rows
-                if (!use_s)
-#pragma unroll
-                    for (int e = 0; e < COLS / 2; ++e) pfk[e] = 0u;
-                tmem_st<16>(trow + TM_S + c0 + 16, pfk);
-            }
-            tmem_wait_st();
-            fence_before_sync();
-            mbar_arrive(BAR(B_PTREADY));
             if (!wait(B_PREADY, i & 1)) {
                 ok = false;
                 break;
@@ -644,8 +639,18 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 uint32_t fu[COLS];
                 tmem_ld32(trow + TM_DPF + c0, fu);
                 tmem_wait_ld();
+                // P^T (bf16) over this warpgroup's dP_f^T columns, now read; on a mixed
+                // step the sparse stream's copy, zero on unselected key rows, beside it
+                tmem_st<16>(trow + TM_DPF + c0, pfk);
+                if (mixed) {
+                    if (!use_s)
+#pragma unroll
+                        for (int e = 0; e < COLS / 2; ++e) pfk[e] = 0u;
+                    tmem_st<16>(trow + TM_DPF + c0 + 16, pfk);
+                }
+                tmem_wait_st();
                 fence_before_sync();
-                mbar_arrive(BAR(B_PFREE));  // dP_f^T may now be overwritten by the next step
+                mbar_arrive(BAR(B_PTREADY));
                 const float4* F4 = reinterpret_cast<const float4*>(rw + STEP + c0);
                 const float4* S4 = reinterpret_cast<const float4*>(rw + 2 * STEP + c0);
 #pragma unroll
