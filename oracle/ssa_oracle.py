@@ -55,7 +55,7 @@ import numpy as np
 
 __all__ = [
     "f64", "pool_blocks", "block_scores", "select_blocks", "block_selection_matrix",
-    "attn_fwd_dual", "align_loss", "alignment_upstream", "attn_bwd",
+    "attn_fwd_dual", "attn_fwd_sparse", "align_loss", "alignment_upstream", "attn_bwd",
 ]
 
 
@@ -218,6 +218,43 @@ def attn_fwd_dual(q, k, v, idx, cnt, block: int, sm_scale: float, rows=None,
                 for name, val in res.items():
                     out[name][b, h, start:start + step] = val
     return out
+
+
+def attn_fwd_sparse(q, k, v, idx, cnt, block: int, sm_scale: float, rows=None):
+    """The sparse stream alone, as run at inference (section 4 of the technical
+    summaries, "Efficienza": the same operations as MoBA).
+
+    For query t in block i, the keys are gathered explicitly: every key s <= t
+    of every block listed in idx[i, :cnt[i]] (S_i, which always holds block i
+    itself); with x = sm_scale * q_t . k_s over those keys only,
+      h(t) = sum_s softmax(x)_s v_s,   lse(t) = log sum_s e^x.
+    Same quantities as h_sparse / lse_sparse of ``attn_fwd_dual``, formed from
+    the index lists instead of a mask over all causal keys.
+
+    q, k, v: [B, H, T, d]; idx, cnt: [B, H, n, k] / [B, H, n].  ``rows``
+    optionally restricts the query rows.  Returns dict(h, lse).
+    """
+    q, k, v = f64(q), f64(k), f64(v)
+    idx, cnt = np.asarray(idx), np.asarray(cnt)
+    B, H, T, d = q.shape
+    rows = np.arange(T) if rows is None else np.asarray(sorted(rows), dtype=np.int64)
+    h_out = np.zeros((B, H, len(rows), v.shape[-1]))
+    lse_out = np.zeros((B, H, len(rows)))
+    for b in range(B):
+        for h in range(H):
+            for i in np.unique(rows // block):
+                sel = np.flatnonzero(rows // block == i)
+                ts = rows[sel]
+                blocks = np.sort(idx[b, h, i, :cnt[b, h, i]])
+                keys = np.concatenate([np.arange(j * block, (j + 1) * block) for j in blocks])
+                x = sm_scale * (q[b, h, ts] @ k[b, h, keys].T)       # [rows of block i, keys]
+                x = np.where(keys[None, :] <= ts[:, None], x, -np.inf)
+                m = x.max(axis=1, keepdims=True)
+                e = np.exp(x - m)
+                l = e.sum(axis=1)
+                h_out[b, h, sel] = (e @ v[b, h, keys]) / l[:, None]
+                lse_out[b, h, sel] = m[:, 0] + np.log(l)
+    return {"h": h_out, "lse": lse_out}
 
 
 def align_loss(h_full, h_sparse, w_sparsity: float = 1.0, w_commit: float = 1.0):

@@ -35,6 +35,12 @@ MUTATIONS = {
     "bwd_dv_sparse_dropped": ("dv += p_full.T @ g_full[t] + p_sparse.T @ g_sparse[t]",
                               "dv += p_full.T @ g_full[t]"),
     "loss_sum_not_mean": ("L = float(np.mean((hf - hs) ** 2))", "L = float(np.sum((hf - hs) ** 2))"),
+    "sparse_only_no_causal_mask": ("x = np.where(keys[None, :] <= ts[:, None], x, -np.inf)",
+                                   "x = np.where(keys[None, :] <= ts[:, None] + block, x, -np.inf)"),
+    "sparse_only_lse_missing_max": ("lse_out[b, h, sel] = m[:, 0] + np.log(l)",
+                                    "lse_out[b, h, sel] = np.log(l)"),
+    "sparse_only_first_listed_block_dropped": ("blocks = np.sort(idx[b, h, i, :cnt[b, h, i]])",
+                                               "blocks = np.sort(idx[b, h, i, 1:cnt[b, h, i]])"),
 }
 
 PIN_TESTS = [
@@ -50,6 +56,9 @@ PIN_TESTS = [
     lambda: pins.test_align_loss_is_library_mse(),
     lambda: pins.test_bwd_central_finite_differences(40.0, 25.0),
     lambda: pins.test_bwd_matches_library_autograd(),
+    lambda: pins.test_sparse_only_matches_library_attention_on_selected_keys(),
+    lambda: pins.test_sparse_only_diagonal_budget_is_blockwise_causal_attention(),
+    lambda: pins.test_sparse_only_brute_force_tiny(),
 ]
 
 

@@ -334,3 +334,60 @@ def test_bwd_full_budget_is_textbook_attention_backward():
     (h * torch.from_numpy(Rf + Rs)).sum().backward()
     for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
         np.testing.assert_allclose(mine, ref.numpy(), rtol=0, atol=1e-11)
+
+
+# ---------------------------------------------------------------- sparse-only forward (inference)
+
+def test_sparse_only_matches_library_attention_on_selected_keys():
+    # the gathered-key sparse stream equals library attention restricted to
+    # the selected causal keys, for several budgets including the diagonal only
+    B, H, T, d, block = 1, 2, 128, 8, 16
+    for topk, seed in ((1, 7), (3, 8), (T // block, 9)):
+        q, k, v, idx, cnt = _case(B, H, T, d, block, topk=topk, seed=seed)
+        out = O.attn_fwd_sparse(q, k, v, idx, cnt, block, 0.45)
+        _, sel, _ = token_masks(idx, cnt, block, T)
+        np.testing.assert_allclose(out["h"], sdpa(q, k, v, sel, 0.45), rtol=0, atol=1e-12)
+        x = torch.from_numpy(0.45 * np.einsum("bhtd,bhsd->bhts", q, k))
+        ls = torch.logsumexp(x.masked_fill(~torch.from_numpy(sel), -math.inf), -1).numpy()
+        np.testing.assert_allclose(out["lse"], ls, rtol=0, atol=1e-12)
+
+
+def test_sparse_only_diagonal_budget_is_blockwise_causal_attention():
+    # top-1 keeps only the current block: per-block causal attention (library)
+    B, H, T, d, block = 1, 1, 64, 4, 16
+    q, k, v, idx, cnt = _case(B, H, T, d, block, topk=1, seed=11)
+    assert np.all(cnt == 1) and np.all(idx[..., 0] == np.arange(T // block))
+    out = O.attn_fwd_sparse(q, k, v, idx, cnt, block, 0.9)
+    for i in range(T // block):
+        sl = slice(i * block, (i + 1) * block)
+        ref = sdpa(q[..., sl, :], k[..., sl, :], v[..., sl, :],
+                   np.tril(np.ones((block, block), dtype=bool)), 0.9)
+        np.testing.assert_allclose(out["h"][..., sl, :], ref, rtol=0, atol=1e-12)
+
+
+def test_sparse_only_equals_the_dual_forwards_sparse_stream():
+    B, H, T, d, block = 2, 2, 96, 8, 8
+    q, k, v, idx, cnt = _case(B, H, T, d, block, topk=3, seed=13)
+    dual = O.attn_fwd_dual(q, k, v, idx, cnt, block, 0.6)
+    rows = [0, 5, 8, 40, 95]
+    sp = O.attn_fwd_sparse(q, k, v, idx, cnt, block, 0.6, rows=rows)
+    np.testing.assert_allclose(sp["h"], dual["h_sparse"][:, :, rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sp["lse"], dual["lse_sparse"][:, :, rows], rtol=0, atol=1e-12)
+
+
+def test_sparse_only_brute_force_tiny():
+    # T = 4, block 2, one head: keys listed by hand
+    q = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0], [0.5, -1.0]])[None, None]
+    k = np.array([[0.2, 0.1], [0.0, 0.3], [1.0, -1.0], [0.4, 0.4]])[None, None]
+    v = np.array([[1.0, 2.0], [3.0, 4.0], [5.0, 6.0], [7.0, 8.0]])[None, None]
+    idx = np.array([[[[0, -1], [1, -1]]]])  # block 1 selects only itself
+    cnt = np.array([[[1, 1]]])
+    out = O.attn_fwd_sparse(q, k, v, idx, cnt, 2, 1.0)
+    # row 3 sees keys 2 and 3 only: weights e^{q3.k2}, e^{q3.k3}
+    x2, x3 = 0.5 * 1.0 + (-1.0) * (-1.0), 0.5 * 0.4 + (-1.0) * 0.4
+    w2, w3 = math.exp(x2), math.exp(x3)
+    np.testing.assert_allclose(out["h"][0, 0, 3], (w2 * v[0, 0, 2] + w3 * v[0, 0, 3]) / (w2 + w3),
+                               rtol=0, atol=1e-14)
+    np.testing.assert_allclose(out["lse"][0, 0, 3], math.log(w2 + w3), rtol=0, atol=1e-14)
+    # row 0 sees only key 0
+    np.testing.assert_allclose(out["h"][0, 0, 0], v[0, 0, 0], rtol=0, atol=1e-15)
