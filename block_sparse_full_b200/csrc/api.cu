@@ -73,6 +73,13 @@ bool use_tc(const ssa_params_t& p) {
 }
 
 size_t fwd_workspace(const ssa_params_t& p) { return use_tc(p) ? fwd_tc_workspace(p) : 0; }
+// CUDA-core path of the sparse-only forward: the dual kernel's other outputs
+// (h_full in dtype, then delta, lse_full, sqdiff as float32 rows)
+size_t fwd_sparse_workspace(const ssa_params_t& p) {
+    if (use_tc(p)) return 0;
+    const size_t esz = p.dtype == SSA_BF16 ? 2 : 4;
+    return align_up(num_elems(p) * esz, 256) + 3 * align_up(num_rows(p) * 4, 256);
+}
 size_t bwd_workspace(const ssa_params_t& p) {
     return use_tc(p) ? bwd_tc_workspace(p) : bwd_simt_workspace(p);
 }
@@ -119,6 +126,7 @@ size_t ssa_workspace_size(const ssa_params_t* p, int which) {
         case SSA_WS_FWD: return fwd_workspace(*p);
         case SSA_WS_LOSS: return loss_workspace(*p);
         case SSA_WS_BWD: return bwd_workspace(*p);
+        case SSA_WS_FWD_SPARSE: return fwd_sparse_workspace(*p);
         default: fail(SSA_ERR_INVALID_ARG, "unknown workspace id %d", which); return (size_t)-1;
     }
 }
@@ -162,6 +170,36 @@ int ssa_attn_fwd_dual(const ssa_params_t* p, const void* q, const void* k, const
                              sqdiff, ws, s);
     return launch_fwd_simt(*p, q, k, v, mask, h_full, h_sparse, delta, lse_full, lse_sparse,
                            sqdiff, s);
+}
+
+int ssa_attn_fwd_sparse(const ssa_params_t* p, const void* q, const void* k, const void* v,
+                        const int32_t* idx, const int32_t* cnt, const uint32_t* mask,
+                        void* h_sparse, float* lse_sparse, void* ws, size_t ws_bytes, void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(validate(p));
+    SSA_TRY(need_ptr(q, "q"));
+    SSA_TRY(need_ptr(k, "k"));
+    SSA_TRY(need_ptr(v, "v"));
+    SSA_TRY(opt_ptr(idx, "idx"));
+    SSA_TRY(opt_ptr(cnt, "cnt"));
+    SSA_TRY(need_ptr(mask, "mask"));
+    SSA_TRY(need_ptr(h_sparse, "h_sparse"));
+    SSA_TRY(need_ptr(lse_sparse, "lse_sparse"));
+    const size_t need = fwd_sparse_workspace(*p);
+    SSA_TRY(need_ws(ws, ws_bytes, need, "ssa_attn_fwd_sparse"));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (use_tc(*p)) return launch_fwd_sparse_tc(*p, q, k, v, mask, h_sparse, lse_sparse, s);
+    // CUDA-core path: the dual kernel, its full-stream outputs kept in the workspace
+    const size_t esz = p->dtype == SSA_BF16 ? 2 : 4;
+    const size_t rows = align_up(num_rows(*p) * 4, 256);
+    char* w = static_cast<char*>(ws);
+    void* h_full = w;
+    char* r = w + align_up(num_elems(*p) * esz, 256);
+    float* delta = reinterpret_cast<float*>(r);
+    float* lse_full = reinterpret_cast<float*>(r + rows);
+    float* sqdiff = reinterpret_cast<float*>(r + 2 * rows);
+    return launch_fwd_simt(*p, q, k, v, mask, h_full, h_sparse, delta, lse_full, lse_sparse, sqdiff,
+                           s);
 }
 
 int ssa_align_loss(const ssa_params_t* p, const float* sqdiff, float w_s, float w_c,

@@ -115,6 +115,13 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
     return true;
 }
 
+// kSparse = false: the dual forward (both streams).  kSparse = true: the
+// sparse stream alone (inference, the same operations as MoBA): key tiles
+// that neither of the tile's query blocks selects are skipped by every
+// role, the running max is taken over selected keys only, unselected
+// (row, half) pairs get P = 0, one accumulator (O_sel), and the epilogue
+// writes h_sparse and lse_sparse only.
+template <bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
@@ -170,6 +177,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // key tiles the CTA processes (all causal ones for the dual forward); the
+    // diagonal tile is always used (the current block is always selected)
+    auto tile_used = [&](int j) -> bool {
+        if (!kSparse) return true;
+        bool a0, a1, b0, b1;
+        half_sel(mrow, j, I, 0, a.block, ragged1, a0, a1);
+        half_sel(mrow, j, I, 1, a.block, ragged1, b0, b1);
+        return a0 || a1 || b0 || b1;
+    };
 
     // Roles 0 and 1 run their loops with the whole warp (warp-uniform address and
     // descriptor arithmetic); one elected lane issues each TMA / tcgen05 op.
@@ -186,12 +202,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         __syncwarp();
         int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
-        for (int j = 0; j < ntk; ++j) {
-            const int s = j & 1;
-            const uint32_t ph = ((j >> 1) + 1) & 1;
+        for (int j = 0, jj = 0; j < ntk; ++j) {
+            if (!tile_used(j)) continue;
+            const int s = jj & 1;  // ring slot of the jj-th processed tile
+            const uint32_t ph = ((jj >> 1) + 1) & 1;
             const uint32_t kdst = base + OFF_K + s * TILE_BYTES;
             const uint32_t vdst = base + OFF_V + s * TILE_BYTES;
-            if (j >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, status, lim)))
+            if (jj >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, status, lim)))
                 break;
             if (elect_one()) {
                 mbar_expect_tx(BAR(B_KFULL + s), TILE_BYTES);
@@ -199,8 +216,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tma_load_3d(kdst + HALF_BYTES, &tm_k, BAR(B_KFULL + s), 64, j * BN, bh);
             }
             __syncwarp();
-            issued_k[s] = j;
-            if (j >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, status, lim)))
+            issued_k[s] = jj;
+            if (jj >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, status, lim)))
                 break;
             if (elect_one()) {
                 mbar_expect_tx(BAR(B_VFULL + s), TILE_BYTES);
@@ -208,7 +225,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tma_load_3d(vdst + HALF_BYTES, &tm_v, BAR(B_VFULL + s), 64, j * BN, bh);
             }
             __syncwarp();
-            issued_v[s] = j;
+            issued_v[s] = jj;
+            ++jj;
         }
         if (*abort_flag) {  // let copies in flight land before the CTA exits
             for (int s = 0; s < 2; ++s) {
@@ -228,9 +246,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // SBO = 1 KB apart; 16 keys (2 KB) per MMA
         const uint64_t vdesc0 = smem_desc_sw128(base + OFF_V, HALF_BYTES, 1024);
         bool ok = __all_sync(FULL, mbar_wait(BAR(B_QFULL), 0, abort_flag, status, lim));
-        auto issue_pv = [&](int i) -> bool {
-            const int b = i & 1;
-            const uint32_t ph = (i >> 1) & 1;
+        auto issue_pv = [&](int i, int ii) -> bool {  // key tile i, ii-th processed
+            const int b = ii & 1;
+            const uint32_t ph = (ii >> 1) & 1;
             if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY + b), ph, abort_flag, status, lim))) return false;
             if (!__all_sync(FULL, mbar_wait(BAR(B_VFULL + b), ph, abort_flag, status, lim))) return false;
             fence_after_sync();
@@ -248,7 +266,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         // half h's P sits in the first 32 columns of its own S range,
                         // the complementary ("alt") copy of a mixed half in the next 32
                         const uint32_t pa = sb + 64 * h + 8 * kk;
-                        if (s0[h] == s1[h]) {
+                        if (kSparse) {  // rows that do not select the half hold P = 0
+                            if (s0[h] || s1[h]) mma_ts(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
+                        } else if (s0[h] == s1[h]) {
                             mma_ts(tmem + (s0[h] ? TM_OSEL : TM_OUNS), pa, bd, idesc_pv, 1);
                         } else {
                             mma_ts(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
@@ -262,9 +282,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             __syncwarp();
             return true;
         };
+        int jj = 0, jprev = -1;
         for (int j = 0; ok && j < ntk; ++j) {
-            const int s = j & 1;
-            if (!__all_sync(FULL, mbar_wait(BAR(B_KFULL + s), (j >> 1) & 1, abort_flag, status, lim))) {
+            if (!tile_used(j)) continue;
+            const int s = jj & 1;
+            if (!__all_sync(FULL, mbar_wait(BAR(B_KFULL + s), (jj >> 1) & 1, abort_flag, status, lim))) {
                 ok = false;
                 break;
             }
@@ -282,9 +304,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mma_commit(BAR(B_KEMPTY + s));
             }
             __syncwarp();
-            if (j >= 1 && !issue_pv(j - 1)) ok = false;
+            if (jj >= 1 && !issue_pv(jprev, jj - 1)) ok = false;
+            jprev = j;
+            ++jj;
         }
-        if (ok) issue_pv(ntk - 1);
+        if (ok && jj > 0) issue_pv(jprev, jj - 1);
         if (elect_one()) mma_commit(BAR(B_DRAIN));  // all MMAs complete before teardown
         __syncwarp();
         wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
@@ -327,11 +351,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float sl2 = a.scale_log2;
         float m2 = -INFINITY, lsel = 0.f, luns = 0.f;
         bool ok = true;
+        int jj = 0;  // tiles processed so far (ring slot / phase)
         for (int j = 0; j < ntk; ++j) {
-            const int b = j & 1;
+            if (!tile_used(j)) continue;
+            const int b = jj & 1;
             // warp-uniform outcome: the TMEM loads below are warp-collective
             const bool got = __all_sync(
-                0xffffffffu, mbar_wait(BAR(B_SREADY + b), (j >> 1) & 1, abort_flag, status, lim));
+                0xffffffffu, mbar_wait(BAR(B_SREADY + b), (jj >> 1) & 1, abort_flag, status, lim));
             const uint32_t sb = trow + (b ? TM_S1 : TM_S0) + c0;
             float s[64];
             if (got) {
@@ -354,6 +380,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 for (int c = 0; c < 64; ++c)
                     if (c0 + c > r) s[c] = -INFINITY;
             }
+            bool s0, s1;
+            half_sel(mrow, j, I, wg, a.block, ragged1, s0, s1);
+            const bool mixed = s0 != s1;
+            const bool row_sel = mixed ? ((r < 64 || a.block == 128) ? s0 : s1) : s0;
+            if (kSparse && !row_sel) {  // the sparse stream alone: this half is not attended
+#pragma unroll
+                for (int c = 0; c < 64; ++c) s[c] = -INFINITY;
+            }
             float mx8[8];  // independent partial maxima (short dependency chains)
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -364,7 +398,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]),
                             fmaxf(mx8[6], mx8[7]));
-            float* xm = xch + (j & 1) * 256;
+            float* xm = xch + (jj & 1) * 256;
             xm[wg * 128 + r] = mx;
             if (wg_vote(!got || *abort_flag)) {  // a wait expired somewhere: both leave here
                 ok = false;
@@ -372,7 +406,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             mx = fmaxf(mx, xm[(1 - wg) * 128 + r]);
             const float mnew = mx * sl2;
-            if (j == 0) {
+            if (jj == 0) {
                 m2 = mnew;
             } else {
                 const bool need = mnew > m2 + kRescaleThreshold;
@@ -380,7 +414,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 // expires the rescale is skipped and the abort flag ends the loop at
                 // the next vote.
                 if (__any_sync(0xffffffffu, need) &&
-                    __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (j - 1) & 1, abort_flag,
+                    __all_sync(0xffffffffu, mbar_wait(BAR(B_PVDONE), (jj - 1) & 1, abort_flag,
                                                       status, lim))) {
                     fence_after_sync();
                     const float mup = fmaxf(m2, mnew);
@@ -389,7 +423,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     lsel *= alpha;
                     luns *= alpha;
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < (kSparse ? 2 : 4); ++c) {
                         const uint32_t col = (c < 2 ? TM_OSEL : TM_OUNS) + c0 + 32 * (c & 1);
                         uint32_t u[32];
                         tmem_ld32(trow + col, u);
@@ -402,10 +436,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             }
             const float negm = -m2;
-            bool s0, s1;
-            half_sel(mrow, j, I, wg, a.block, ragged1, s0, s1);
-            const bool mixed = s0 != s1;
-            const bool row_sel = mixed ? ((r < 64 || a.block == 128) ? s0 : s1) : s0;
+            // sparse stream alone: rows with no attended key yet, or whose half is not
+            // attended, contribute P = 0 (no exponentials)
+            const bool zero_p = kSparse && (!row_sel || !(m2 > -INFINITY));
             // p = 2^(s*sigma*log2e - m), two columns at a time (packed f32x2).  Off
             // the diagonal a quarter of the pairs take the FMA-pipe exponential so
             // that the MUFU unit is not the limit; on the diagonal every pair uses
@@ -413,7 +446,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const f32x2 sl2x2 = mk2(sl2, sl2), nm2 = mk2(negm, negm);
             f32x2 acc[4] = {mk2(0.f, 0.f), mk2(0.f, 0.f), mk2(0.f, 0.f), mk2(0.f, 0.f)};
             uint32_t pk[32];
-            if (j == I) {
+            if (zero_p) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pk[c] = 0u;
+            } else if (j == I) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     float x0, x1;
@@ -443,7 +479,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             un2(add2(acc[0], acc[1]), a0, a1);
             un2(add2(acc[2], acc[3]), b0, b1);
             const float sum = (a0 + a1) + (b0 + b1);
-            if (!mixed) {
+            if (kSparse || !mixed) {
                 tmem_st32(sb, pk);
             } else {
                 uint32_t main_[32], alt[32];
@@ -460,10 +496,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PREADY + b));
+            ++jj;
         }
         if (ok)
             ok = __all_sync(0xffffffffu,
-                            mbar_wait(BAR(B_PVDONE), (ntk - 1) & 1, abort_flag, status, lim));
+                            mbar_wait(BAR(B_PVDONE), (jj - 1) & 1, abort_flag, status, lim));
         // both warpgroups take the same decision and the same barriers below
         ok = !wg_vote(!ok || *abort_flag);
         float* xl = xch;  // [wg][sel|uns][row] reuses the max exchange area
@@ -471,57 +508,83 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         xl[(wg * 2 + 1) * 128 + r] = luns;
         wg_sync();
         const float Ls = lsel + xl[((1 - wg) * 2) * 128 + r];
-        const float Lu = luns + xl[((1 - wg) * 2 + 1) * 128 + r];
-        float sq = 0.f;
         const int t = t0 + r;
         const bool valid = t < a.T;
         const size_t row = (size_t)bh * a.T + (valid ? t : 0);
-        if (ok) {
-            fence_after_sync();
-            const float l = Ls + Lu;
-            const float inv_l = 1.f / l;
-            const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
+        if constexpr (kSparse) {
+            // the diagonal block holds key t itself, so Ls > 0 on valid rows
+            if (ok) {
+                fence_after_sync();
+                const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
-                uint32_t os[32], ou[32];
-                tmem_ld32(trow + TM_OSEL + c0 + 32 * c, os);
-                tmem_ld32(trow + TM_OUNS + c0 + 32 * c, ou);
-                tmem_wait_ld();
-                uint32_t hf[16], hs[16];
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t os[32];
+                    tmem_ld32(trow + TM_OSEL + c0 + 32 * c, os);
+                    tmem_wait_ld();
+                    uint32_t hs[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float sa = __uint_as_float(os[2 * e]), sb2 = __uint_as_float(os[2 * e + 1]);
-                    const float ua = __uint_as_float(ou[2 * e]), ub = __uint_as_float(ou[2 * e + 1]);
-                    const float fa = (sa + ua) * inv_l, fb = (sb2 + ub) * inv_l;
-                    const float pa = sa * inv_ls, pb = sb2 * inv_ls;
-                    sq = fmaf(fa - pa, fa - pa, sq);
-                    sq = fmaf(fb - pb, fb - pb, sq);
-                    hf[e] = pack_bf16(fa, fb);
-                    hs[e] = pack_bf16(pa, pb);
+                    for (int e = 0; e < 16; ++e)
+                        hs[e] = pack_bf16(__uint_as_float(os[2 * e]) * inv_ls,
+                                          __uint_as_float(os[2 * e + 1]) * inv_ls);
+                    if (valid) {
+                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * HD + c0 + 32 * c);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
+                    }
                 }
-                if (valid) {
-                    uint4* df = reinterpret_cast<uint4*>(a.h_full + row * HD + c0 + 32 * c);
-                    uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * HD + c0 + 32 * c);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        df[v4] = make_uint4(hf[4 * v4], hf[4 * v4 + 1], hf[4 * v4 + 2], hf[4 * v4 + 3]);
-                        ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
+                if (wg == 0 && valid)
+                    a.lse_sparse[row] = Ls > 0.f ? (m2 + log2f(Ls)) * kLn2 : -INFINITY;
+            }
+        } else {
+            const float Lu = luns + xl[((1 - wg) * 2 + 1) * 128 + r];
+            float sq = 0.f;
+            if (ok) {
+                fence_after_sync();
+                const float l = Ls + Lu;
+                const float inv_l = 1.f / l;
+                const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
+    #pragma unroll 1
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t os[32], ou[32];
+                    tmem_ld32(trow + TM_OSEL + c0 + 32 * c, os);
+                    tmem_ld32(trow + TM_OUNS + c0 + 32 * c, ou);
+                    tmem_wait_ld();
+                    uint32_t hf[16], hs[16];
+    #pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float sa = __uint_as_float(os[2 * e]), sb2 = __uint_as_float(os[2 * e + 1]);
+                        const float ua = __uint_as_float(ou[2 * e]), ub = __uint_as_float(ou[2 * e + 1]);
+                        const float fa = (sa + ua) * inv_l, fb = (sb2 + ub) * inv_l;
+                        const float pa = sa * inv_ls, pb = sb2 * inv_ls;
+                        sq = fmaf(fa - pa, fa - pa, sq);
+                        sq = fmaf(fb - pb, fb - pb, sq);
+                        hf[e] = pack_bf16(fa, fb);
+                        hs[e] = pack_bf16(pa, pb);
+                    }
+                    if (valid) {
+                        uint4* df = reinterpret_cast<uint4*>(a.h_full + row * HD + c0 + 32 * c);
+                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * HD + c0 + 32 * c);
+    #pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            df[v4] = make_uint4(hf[4 * v4], hf[4 * v4 + 1], hf[4 * v4 + 2], hf[4 * v4 + 3]);
+                            ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
+                        }
                     }
                 }
             }
-        }
-        float* xs = xch + 512;  // [wg][row] squared-difference partials
-        xs[wg * 128 + r] = sq;
-        wg_sync();
-        if (ok && wg == 0 && valid) {
-            const float l = Ls + Lu;
-            a.delta[row] = Lu / l;
-            a.lse_full[row] = (m2 + log2f(l)) * kLn2;
-            a.lse_sparse[row] = Ls > 0.f ? (m2 + log2f(Ls)) * kLn2 : -INFINITY;
-            a.sqdiff[row] = sq + xs[128 + r];
+            float* xs = xch + 512;  // [wg][row] squared-difference partials
+            xs[wg * 128 + r] = sq;
+            wg_sync();
+            if (ok && wg == 0 && valid) {
+                const float l = Ls + Lu;
+                a.delta[row] = Lu / l;
+                a.lse_full[row] = (m2 + log2f(l)) * kLn2;
+                a.lse_sparse[row] = Ls > 0.f ? (m2 + log2f(Ls)) * kLn2 : -INFINITY;
+                a.sqdiff[row] = sq + xs[128 + r];
+            }
         }
     }
-
     fence_before_sync();
     __syncthreads();
     if (warp == 1) {
@@ -570,9 +633,10 @@ bool fwd_tc_supported(const ssa_params_t& p) {
 
 size_t fwd_tc_workspace(const ssa_params_t&) { return 0; }
 
-int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
-                  const uint32_t* mask, void* hf, void* hs, float* delta, float* lf, float* ls,
-                  float* sq, void*, cudaStream_t s) {
+namespace {
+template <bool kSparse>
+int launch_fwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                       const uint32_t* mask, const FwdArgs& outs, cudaStream_t s) {
     const int BH = p.B * p.H;
     CUtensorMap mq, mk, mv;
     int st = make_map(&mq, q, BH, p.T);
@@ -582,18 +646,12 @@ int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)SMEM_BYTES);
+        attr_err = cudaFuncSetAttribute(fwd_tc_kernel<kSparse>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     });
     if (attr_err != cudaSuccess)
         return fail(SSA_ERR_CUDA, "fwd_tc: smem attribute: %s", cudaGetErrorString(attr_err));
-    FwdArgs a;
-    a.h_full = static_cast<__nv_bfloat16*>(hf);
-    a.h_sparse = static_cast<__nv_bfloat16*>(hs);
-    a.delta = delta;
-    a.lse_full = lf;
-    a.lse_sparse = ls;
-    a.sqdiff = sq;
+    FwdArgs a = outs;
     a.mask = mask;
     a.BH = BH;
     a.T = p.T;
@@ -603,8 +661,30 @@ int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     a.scale_log2 = p.sm_scale * 1.4426950408889634f;
     a.timeout_ns = wait_limit_ns();
     const unsigned grid = (unsigned)((size_t)BH * ((p.T + BM - 1) / BM));
-    fwd_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, a);
-    return check_launch("fwd_tc_kernel");
+    fwd_tc_kernel<kSparse><<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, a);
+    return check_launch(kSparse ? "fwd_tc_kernel<sparse>" : "fwd_tc_kernel");
+}
+}  // namespace
+
+int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                  const uint32_t* mask, void* hf, void* hs, float* delta, float* lf, float* ls,
+                  float* sq, void*, cudaStream_t s) {
+    FwdArgs o{};
+    o.h_full = static_cast<__nv_bfloat16*>(hf);
+    o.h_sparse = static_cast<__nv_bfloat16*>(hs);
+    o.delta = delta;
+    o.lse_full = lf;
+    o.lse_sparse = ls;
+    o.sqdiff = sq;
+    return launch_fwd_tc_impl<false>(p, q, k, v, mask, o, s);
+}
+
+int launch_fwd_sparse_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                         const uint32_t* mask, void* hs, float* ls, cudaStream_t s) {
+    FwdArgs o{};
+    o.h_sparse = static_cast<__nv_bfloat16*>(hs);
+    o.lse_sparse = ls;
+    return launch_fwd_tc_impl<true>(p, q, k, v, mask, o, s);
 }
 
 int fwd_tc_take_status(cudaStream_t) {

@@ -52,6 +52,9 @@ int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
                   float* lse_full, float* lse_sparse, float* sqdiff, void* ws,
                   cudaStream_t s);
 int fwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
+// the sparse stream alone (inference): h_sparse and lse_sparse only
+int launch_fwd_sparse_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                         const uint32_t* mask, void* h_sparse, float* lse_sparse, cudaStream_t s);
 
 // ---- alignment loss (loss.cu)
 size_t loss_workspace(const ssa_params_t& p);

@@ -27,12 +27,12 @@ SSA_OK, SSA_ERR_INVALID_ARG, SSA_ERR_UNSUPPORTED = 0, -1, -2
 SSA_ERR_WORKSPACE, SSA_ERR_CUDA, SSA_ERR_TIMEOUT = -3, -4, -5
 SSA_F32, SSA_BF16 = 0, 1
 SSA_FLAG_FORCE_SINK, SSA_FLAG_FORCE_SIMT = 1, 2
-SSA_WS_SELECT, SSA_WS_FWD, SSA_WS_LOSS, SSA_WS_BWD = 0, 1, 2, 3
+SSA_WS_SELECT, SSA_WS_FWD, SSA_WS_LOSS, SSA_WS_BWD, SSA_WS_FWD_SPARSE = 0, 1, 2, 3, 4
 
 # every symbol include/ssa.h declares
 EXPORTS = (
     "ssa_workspace_size", "ssa_select_blocks", "ssa_select_blocks_noalloc",
-    "ssa_attn_fwd_dual", "ssa_align_loss",
+    "ssa_attn_fwd_dual", "ssa_attn_fwd_sparse", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
     "ssa_kernel_path", "ssa_bwd_heads_per_group", "ssa_selftest_math", "ssa_selftest_wait_timeout",
     "ssa_debug_set_wait_limit_ns", "ssa_debug_set_kernel_events", "ssa_version",
@@ -64,6 +64,8 @@ _SIGNATURES = {
     "ssa_attn_fwd_dual": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_size_t, c_void_p]),
+    "ssa_attn_fwd_sparse": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "ssa_align_loss": (c_int, [_P, c_void_p, c_float, c_float, c_void_p, c_void_p, c_size_t,
                                c_void_p]),
     "ssa_attn_bwd": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -122,6 +124,12 @@ def ssa_attn_fwd_dual(params, q, k, v, idx, cnt, mask, h_full, h_sparse, delta, 
     return _lib.ssa_attn_fwd_dual(ctypes.byref(params), q, k, v, idx, cnt, mask, h_full,
                                   h_sparse, delta, lse_full, lse_sparse, sqdiff_rows, ws,
                                   ws_bytes, stream)
+
+
+def ssa_attn_fwd_sparse(params, q, k, v, idx, cnt, mask, h_sparse, lse_sparse, ws, ws_bytes,
+                        stream):
+    return _lib.ssa_attn_fwd_sparse(ctypes.byref(params), q, k, v, idx, cnt, mask, h_sparse,
+                                    lse_sparse, ws, ws_bytes, stream)
 
 
 def ssa_align_loss(params, sqdiff_rows, w_sparsity, w_commit, loss_out, ws, ws_bytes, stream):
@@ -255,6 +263,22 @@ def attn_fwd_dual(params, q, k, v, mask, idx=None, cnt=None, ws=None, out=None):
                             _ptr(out["delta"]), _ptr(out["lse_full"]),
                             _ptr(out["lse_sparse"]), _ptr(out["sqdiff"]), _ptr(ws),
                             ws.numel(), _stream(dev)), "ssa_attn_fwd_dual")
+    return out
+
+
+def attn_fwd_sparse(params, q, k, v, mask, idx=None, cnt=None, ws=None, out=None):
+    """The sparse stream alone (inference) -> dict(h_sparse, lse_sparse)."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (mask, "mask")):
+        _need(t, nm)
+    dev = q.device
+    if out is None:
+        out = {"h_sparse": torch.empty_like(q),
+               "lse_sparse": torch.empty((params.B, params.H, params.T), dtype=torch.float32,
+                                         device=dev)}
+    ws = workspace(params, SSA_WS_FWD_SPARSE, dev) if ws is None else ws
+    check(ssa_attn_fwd_sparse(params, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt),
+                              _ptr(mask), _ptr(out["h_sparse"]), _ptr(out["lse_sparse"]),
+                              _ptr(ws), ws.numel(), _stream(dev)), "ssa_attn_fwd_sparse")
     return out
 
 

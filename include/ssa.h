@@ -89,7 +89,8 @@ enum {
     SSA_WS_SELECT = 0,
     SSA_WS_FWD = 1,
     SSA_WS_LOSS = 2,
-    SSA_WS_BWD = 3
+    SSA_WS_BWD = 3,
+    SSA_WS_FWD_SPARSE = 4
 };
 
 /* Bytes of scratch the named entry point needs for these params (0 if none,
@@ -151,6 +152,23 @@ int ssa_attn_fwd_dual(const ssa_params_t* params, const void* q, const void* k,
                       const uint32_t* mask, void* h_full, void* h_sparse,
                       float* delta, float* lse_full, float* lse_sparse,
                       float* sqdiff_rows, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The sparse stream alone, as run at inference (section 4, "Efficienza":
+ * at inference SSA runs the same operations as MoBA).  For query t in block
+ * i and the keys s <= t whose block is in S_i (read from `mask`; idx/cnt
+ * may be NULL and are not read), x = sm_scale * q_t . k_s:
+ *   h_sparse = sum_{sel} e^x v_s / sum_{sel} e^x,  lse_sparse = log sum_{sel} e^x
+ * — the same quantities as ssa_attn_fwd_dual's, from a kernel that visits
+ * only the selected key blocks (work proportional to the selected pairs).
+ * h_sparse is [B,H,T,D] in dtype, lse_sparse [B,H,T] float32.  Workspace:
+ * SSA_WS_FWD_SPARSE (0 on the tensor-core path; the CUDA-core path runs the
+ * dual kernel and keeps the full-stream outputs there).
+ */
+int ssa_attn_fwd_sparse(const ssa_params_t* params, const void* q, const void* k,
+                        const void* v, const int32_t* idx, const int32_t* cnt,
+                        const uint32_t* mask, void* h_sparse, float* lse_sparse,
+                        void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Alignment losses (section 2, "Allineamento Bidirezionale"): with
