@@ -232,13 +232,23 @@ class Layer:
                      for k in ("delta", "lse_f", "lse_s", "sqd")}
         self.loss = torch.empty(2, dtype=torch.float32, device=dev)
         self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
-        self.ws = {i: ssa.workspace(self.p, i, dev) for i in range(4)}
+        self.ws = {i: ssa.workspace(self.p, i, dev) for i in range(5)}
+        self.hs_inf = torch.empty_like(self.q)  # sparse-only forward (inference) outputs
+        self.ls_inf = torch.empty((B, H, T), dtype=torch.float32, device=dev)
         self.w_s = self.w_c = 1.0
         self.path = ssa.ssa_kernel_path(self.p)
 
     def launches_per_step(self):
         # select: pool + score; fwd: 1; loss: 2; bwd: pre + dk/dv + dq (either path)
         return 2 + 1 + 2 + 3
+
+    def run_sparse_fwd(self, stream):
+        """The sparse stream alone (inference mode) on the step's selection."""
+        ssa, ptr = self.ssa, (lambda t: t.data_ptr())
+        st = ssa.ssa_attn_fwd_sparse(self.p, ptr(self.q), ptr(self.k), ptr(self.v), None, None,
+                                     ptr(self.mask), ptr(self.hs_inf), ptr(self.ls_inf),
+                                     ptr(self.ws[4]), self.ws[4].numel(), stream.cuda_stream)
+        ssa.check(st, "sparse fwd")
 
     def run(self, stream, events=None, kernel_events=None):
         """One step; `events` (5) bracket the four ABI calls, `kernel_events`
@@ -367,6 +377,27 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
     roof["ms_per_launch"] = round(dom_ms, 4)
     roof["flops_per_launch"] = flops
 
+    # inference mode: the sparse stream alone on the same selection (not part
+    # of the training step; timed after it, L2 flushed before each call)
+    inf_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        layer.run_sparse_fwd(stream)
+        e1.record(stream)
+        if i >= args.warmup:
+            inf_ms.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    layer.ssa.device_status()
+    sparse_ms = sum(a.elapsed_time(b) for a, b in inf_ms) / len(inf_ms)
+    f_sparse = 4 * w.D * p_sel * w.B * w.H
+    inference = {"kernel": "fwd_tc_kernel<sparse>" if layer.path == 1 else "fwd_simt (dual)",
+                 "ms": round(sparse_ms, 4), "flops": f_sparse,
+                 "tflops": round(f_sparse / (sparse_ms * 1e-3) / 1e12, 2),
+                 "dual_fwd_ms": round(avg["fwd"], 4),
+                 "speedup_vs_dual_fwd": round(avg["fwd"] / sparse_ms, 3)}
+
     fwd_tflops = f_fwd / (avg["fwd"] * 1e-3) / 1e12
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
@@ -380,6 +411,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
         "roofline": roof,
         "breakdown_ms": {n: round(avg[n], 4) for n in names},
         "kernels": kernels,
+        "inference_sparse_fwd": inference,
         "fwd_tflops": round(fwd_tflops, 2),
         "fwd_frac_sustained": round(fwd_tflops / sustained, 4),
         "fwd_frac_burst": round(fwd_tflops / peaks.get("bf16_tflops", 1590.0), 4),
