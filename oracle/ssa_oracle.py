@@ -55,7 +55,8 @@ import numpy as np
 
 __all__ = [
     "f64", "pool_blocks", "block_scores", "select_blocks", "block_selection_matrix",
-    "attn_fwd_dual", "attn_fwd_sparse", "align_loss", "alignment_upstream", "attn_bwd",
+    "attn_fwd_dual", "attn_fwd_sparse", "diagnostics", "align_loss", "alignment_upstream",
+    "attn_bwd",
 ]
 
 
@@ -255,6 +256,33 @@ def attn_fwd_sparse(q, k, v, idx, cnt, block: int, sm_scale: float, rows=None):
                 h_out[b, h, sel] = (e @ v[b, h, keys]) / l[:, None]
                 lse_out[b, h, sel] = m[:, 0] + np.log(l)
     return {"h": h_out, "lse": lse_out}
+
+
+def diagnostics(q, k, lse_full, delta, block: int, sm_scale: float):
+    """Attention diagnostics the pages discuss (section 1 of the technical
+    summaries: the approximation error grows with the discarded mass delta;
+    the first block acting as an attention sink; the sparsity of learned
+    attention):
+
+      sink(t)        = full-softmax mass on the keys of block 0:
+                       sum_{s <= t, s < block} exp(sm_scale q_t . k_s - lse_full(t))
+      mean_delta[h]  = mean over t of delta(t)
+      mean_sink[h]   = mean over t of sink(t)
+
+    q, k: [B, H, T, d]; lse_full, delta: [B, H, T] (the forward's outputs).
+    Returns dict(sink [B,H,T], mean_delta [B,H], mean_sink [B,H]).
+    """
+    q, k = f64(q), f64(k)
+    lse, dl = f64(lse_full), f64(delta)
+    B, H, T, d = q.shape
+    sink = np.zeros((B, H, T))
+    keys = np.arange(min(block, T))
+    for b in range(B):
+        for h in range(H):
+            x = sm_scale * (q[b, h] @ k[b, h, keys].T)                    # [T, block]
+            w = np.where(keys[None, :] <= np.arange(T)[:, None], np.exp(x - lse[b, h][:, None]), 0.0)
+            sink[b, h] = w.sum(axis=1)
+    return {"sink": sink, "mean_delta": dl.mean(axis=2), "mean_sink": sink.mean(axis=2)}
 
 
 def align_loss(h_full, h_sparse, w_sparsity: float = 1.0, w_commit: float = 1.0):

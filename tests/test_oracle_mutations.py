@@ -41,6 +41,9 @@ MUTATIONS = {
                                     "lse_out[b, h, sel] = np.log(l)"),
     "sparse_only_first_listed_block_dropped": ("blocks = np.sort(idx[b, h, i, :cnt[b, h, i]])",
                                                "blocks = np.sort(idx[b, h, i, 1:cnt[b, h, i]])"),
+    "sink_mass_strict_causality": ("w = np.where(keys[None, :] <= np.arange(T)[:, None], np.exp(x - lse[b, h][:, None]), 0.0)",
+                                   "w = np.where(keys[None, :] < np.arange(T)[:, None], np.exp(x - lse[b, h][:, None]), 0.0)"),
+    "sink_mass_half_block": ("keys = np.arange(min(block, T))", "keys = np.arange(min(block, T) // 2)"),
 }
 
 PIN_TESTS = [
@@ -59,6 +62,7 @@ PIN_TESTS = [
     lambda: pins.test_sparse_only_matches_library_attention_on_selected_keys(),
     lambda: pins.test_sparse_only_diagonal_budget_is_blockwise_causal_attention(),
     lambda: pins.test_sparse_only_brute_force_tiny(),
+    lambda: pins.test_sink_mass_is_library_softmax_on_block_zero(),
 ]
 
 

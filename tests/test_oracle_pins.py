@@ -391,3 +391,34 @@ def test_sparse_only_brute_force_tiny():
     np.testing.assert_allclose(out["lse"][0, 0, 3], math.log(w2 + w3), rtol=0, atol=1e-14)
     # row 0 sees only key 0
     np.testing.assert_allclose(out["h"][0, 0, 0], v[0, 0, 0], rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------- diagnostics
+
+def test_sink_mass_is_library_softmax_on_block_zero():
+    B, H, T, d, block = 1, 2, 96, 8, 16
+    q, k, v, idx, cnt = _case(B, H, T, d, block, topk=2, seed=17)
+    fwd = O.attn_fwd_dual(q, k, v, idx, cnt, block, 0.8)
+    dg = O.diagnostics(q, k, fwd["lse_full"], fwd["delta"], block, 0.8)
+    x = torch.from_numpy(0.8 * np.einsum("bhtd,bhsd->bhts", q, k))
+    causal = torch.from_numpy(np.tril(np.ones((T, T), dtype=bool)))
+    p = torch.softmax(x.masked_fill(~causal, -math.inf), dim=-1).numpy()
+    np.testing.assert_allclose(dg["sink"], p[..., :block].sum(-1), rtol=0, atol=1e-12)
+    # rows inside block 0 put all their mass there
+    np.testing.assert_allclose(dg["sink"][..., :block], 1.0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dg["mean_sink"], dg["sink"].mean(-1), rtol=0, atol=0)
+    np.testing.assert_allclose(dg["mean_delta"], fwd["delta"].mean(-1), rtol=0, atol=0)
+
+
+def test_sink_mass_rises_with_a_planted_sink():
+    # a large logit boost on block 0 moves almost all mass there
+    B, H, T, d, block = 1, 1, 64, 8, 16
+    q, k, v, idx, cnt = _case(B, H, T, d, block, topk=2, seed=19)
+    base = O.attn_fwd_dual(q, k, v, idx, cnt, block, 1.0)
+    s0 = O.diagnostics(q, k, base["lse_full"], base["delta"], block, 1.0)["sink"]
+    u = np.ones(d) / math.sqrt(d)
+    q2, k2 = q + 3.0 * u, k.copy()
+    k2[..., :block, :] += 3.0 * u
+    fwd = O.attn_fwd_dual(q2, k2, v, idx, cnt, block, 1.0)
+    s1 = O.diagnostics(q2, k2, fwd["lse_full"], fwd["delta"], block, 1.0)["sink"]
+    assert s1[..., block:].mean() > 0.9 > s0[..., block:].mean()
