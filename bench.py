@@ -233,6 +233,8 @@ class Layer:
         self.loss = torch.empty(2, dtype=torch.float32, device=dev)
         self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
         self.ws = {i: ssa.workspace(self.p, i, dev) for i in range(5)}
+        self.sink = torch.empty((B, H, T), dtype=torch.float32, device=dev)  # diagnostics
+        self.head_stats = torch.empty((B, H, 2), dtype=torch.float32, device=dev)
         self.hs_inf = torch.empty_like(self.q)  # sparse-only forward (inference) outputs
         self.ls_inf = torch.empty((B, H, T), dtype=torch.float32, device=dev)
         self.w_s = self.w_c = 1.0
@@ -249,6 +251,14 @@ class Layer:
                                      ptr(self.mask), ptr(self.hs_inf), ptr(self.ls_inf),
                                      ptr(self.ws[4]), self.ws[4].numel(), stream.cuda_stream)
         ssa.check(st, "sparse fwd")
+
+    def run_diagnostics(self, stream):
+        """Sink mass on block 0 and per-head means, from the step's forward outputs."""
+        ssa, ptr, r = self.ssa, (lambda t: t.data_ptr()), self.rows
+        st = ssa.ssa_attn_diagnostics(self.p, ptr(self.q), ptr(self.k), ptr(r["lse_f"]),
+                                      ptr(r["delta"]), ptr(self.sink), ptr(self.head_stats),
+                                      stream.cuda_stream)
+        ssa.check(st, "diagnostics")
 
     def run(self, stream, events=None, kernel_events=None):
         """One step; `events` (5) bracket the four ABI calls, `kernel_events`
@@ -391,6 +401,26 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
     torch.cuda.synchronize(dev)
     layer.ssa.device_status()
     sparse_ms = sum(a.elapsed_time(b) for a, b in inf_ms) / len(inf_ms)
+    diag_ev = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        layer.run_diagnostics(stream)
+        e1.record(stream)
+        if i >= args.warmup:
+            diag_ev.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    layer.ssa.device_status()
+    diag_ms = sum(a.elapsed_time(b) for a, b in diag_ev) / len(diag_ev)
+    # reads Q, block 0 of K, lse_full and delta; writes the sink row vector
+    esz = 2 if w.dtype == "bf16" else 4
+    diag_bytes = w.B * w.H * (w.T * w.D * esz + min(w.block, w.T) * w.D * esz + 3 * w.T * 4)
+    hs = layer.head_stats.cpu().numpy()
+    diagnostics = {"kernels": ["diag_sink_kernel", "diag_head_kernel"], "ms": round(diag_ms, 4),
+                   "hbm_bytes": diag_bytes, "hbm_gbs": round(diag_bytes / (diag_ms * 1e-3) / 1e9, 1),
+                   "mean_delta": round(float(hs[..., 0].mean()), 6),
+                   "mean_sink_mass": round(float(hs[..., 1].mean()), 6)}
     f_sparse = 4 * w.D * p_sel * w.B * w.H
     inference = {"kernel": "fwd_tc_kernel<sparse>" if layer.path == 1 else "fwd_simt (dual)",
                  "ms": round(sparse_ms, 4), "flops": f_sparse,
@@ -412,6 +442,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
         "breakdown_ms": {n: round(avg[n], 4) for n in names},
         "kernels": kernels,
         "inference_sparse_fwd": inference,
+        "diagnostics": diagnostics,
         "fwd_tflops": round(fwd_tflops, 2),
         "fwd_frac_sustained": round(fwd_tflops / sustained, 4),
         "fwd_frac_burst": round(fwd_tflops / peaks.get("bf16_tflops", 1590.0), 4),

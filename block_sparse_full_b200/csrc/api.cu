@@ -202,6 +202,21 @@ int ssa_attn_fwd_sparse(const ssa_params_t* p, const void* q, const void* k, con
                            s);
 }
 
+int ssa_attn_diagnostics(const ssa_params_t* p, const void* q, const void* k,
+                         const float* lse_full, const float* delta, float* sink_rows,
+                         float* head_stats, void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(validate(p));
+    SSA_TRY(need_ptr(q, "q"));
+    SSA_TRY(need_ptr(k, "k"));
+    SSA_TRY(need_ptr(lse_full, "lse_full"));
+    SSA_TRY(need_ptr(delta, "delta"));
+    SSA_TRY(need_ptr(sink_rows, "sink_rows"));
+    SSA_TRY(need_ptr(head_stats, "head_stats"));
+    return launch_diagnostics(*p, q, k, lse_full, delta, sink_rows, head_stats,
+                              static_cast<cudaStream_t>(stream));
+}
+
 int ssa_align_loss(const ssa_params_t* p, const float* sqdiff, float w_s, float w_c,
                    float* loss_out, void* ws, size_t ws_bytes, void* stream) {
     g_last_error[0] = 0;

@@ -56,6 +56,10 @@ int fwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
 int launch_fwd_sparse_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
                          const uint32_t* mask, void* h_sparse, float* lse_sparse, cudaStream_t s);
 
+// ---- attention diagnostics (diag.cu)
+int launch_diagnostics(const ssa_params_t& p, const void* q, const void* k, const float* lse_full,
+                       const float* delta, float* sink, float* stats, cudaStream_t s);
+
 // ---- alignment loss (loss.cu)
 size_t loss_workspace(const ssa_params_t& p);
 int launch_loss(const ssa_params_t& p, const float* sqdiff, float w_s, float w_c,

@@ -32,7 +32,7 @@ SSA_WS_SELECT, SSA_WS_FWD, SSA_WS_LOSS, SSA_WS_BWD, SSA_WS_FWD_SPARSE = 0, 1, 2,
 # every symbol include/ssa.h declares
 EXPORTS = (
     "ssa_workspace_size", "ssa_select_blocks", "ssa_select_blocks_noalloc",
-    "ssa_attn_fwd_dual", "ssa_attn_fwd_sparse", "ssa_align_loss",
+    "ssa_attn_fwd_dual", "ssa_attn_fwd_sparse", "ssa_attn_diagnostics", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
     "ssa_kernel_path", "ssa_bwd_heads_per_group", "ssa_selftest_math", "ssa_selftest_wait_timeout",
     "ssa_debug_set_wait_limit_ns", "ssa_debug_set_kernel_events", "ssa_version",
@@ -66,6 +66,8 @@ _SIGNATURES = {
                                   c_void_p, c_void_p, c_size_t, c_void_p]),
     "ssa_attn_fwd_sparse": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "ssa_attn_diagnostics": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                     c_void_p, c_void_p]),
     "ssa_align_loss": (c_int, [_P, c_void_p, c_float, c_float, c_void_p, c_void_p, c_size_t,
                                c_void_p]),
     "ssa_attn_bwd": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -130,6 +132,11 @@ def ssa_attn_fwd_sparse(params, q, k, v, idx, cnt, mask, h_sparse, lse_sparse, w
                         stream):
     return _lib.ssa_attn_fwd_sparse(ctypes.byref(params), q, k, v, idx, cnt, mask, h_sparse,
                                     lse_sparse, ws, ws_bytes, stream)
+
+
+def ssa_attn_diagnostics(params, q, k, lse_full, delta, sink_rows, head_stats, stream):
+    return _lib.ssa_attn_diagnostics(ctypes.byref(params), q, k, lse_full, delta, sink_rows,
+                                     head_stats, stream)
 
 
 def ssa_align_loss(params, sqdiff_rows, w_sparsity, w_commit, loss_out, ws, ws_bytes, stream):
@@ -280,6 +287,17 @@ def attn_fwd_sparse(params, q, k, v, mask, idx=None, cnt=None, ws=None, out=None
                               _ptr(mask), _ptr(out["h_sparse"]), _ptr(out["lse_sparse"]),
                               _ptr(ws), ws.numel(), _stream(dev)), "ssa_attn_fwd_sparse")
     return out
+
+
+def diagnostics(params, q, k, fwd):
+    """Sink mass per row and per-head means of delta and sink -> dict(sink, head_stats)."""
+    _need(q, "q"), _need(k, "k")
+    dev = q.device
+    sink = torch.empty((params.B, params.H, params.T), dtype=torch.float32, device=dev)
+    stats = torch.empty((params.B, params.H, 2), dtype=torch.float32, device=dev)
+    check(ssa_attn_diagnostics(params, _ptr(q), _ptr(k), _ptr(fwd["lse_full"]), _ptr(fwd["delta"]),
+                               _ptr(sink), _ptr(stats), _stream(dev)), "ssa_attn_diagnostics")
+    return {"sink": sink, "head_stats": stats}
 
 
 def align_loss(params, sqdiff, w_sparsity=1.0, w_commit=1.0, ws=None, out=None):

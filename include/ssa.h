@@ -171,6 +171,20 @@ int ssa_attn_fwd_sparse(const ssa_params_t* params, const void* q, const void* k
                         void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Attention diagnostics (section 1: the sparse approximation error grows
+ * with the discarded mass delta; the pages also discuss the first block as an
+ * attention sink and the sparsity of learned attention), from the dual
+ * forward's lse_full and delta for the same q, k:
+ *   sink_rows[t]  = sum_{s <= t, s < block} exp(sm_scale q_t . k_s - lse_full(t))
+ *                   (full-softmax mass on block 0), float32 [B,H,T];
+ *   head_stats    = float32 [B,H,2]: mean over t of delta, mean over t of sink.
+ * The means are fixed-order float64 sums (bitwise repeatable).  No workspace.
+ */
+int ssa_attn_diagnostics(const ssa_params_t* params, const void* q, const void* k,
+                         const float* lse_full, const float* delta, float* sink_rows,
+                         float* head_stats, void* stream);
+
+/*
  * Alignment losses (section 2, "Allineamento Bidirezionale"): with
  * N = B*H*T*D and L = sum(sqdiff_rows) / N (the mean squared difference of
  * the two outputs), writes loss_out[0] = w_sparsity * L (L_sparsity) and
