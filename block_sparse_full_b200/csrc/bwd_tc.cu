@@ -47,10 +47,9 @@ namespace {
 
 using namespace tc;
 
-constexpr int HD = 128;
 constexpr int TILE = 128;  // keys per dK/dV CTA, queries per dQ CTA
 constexpr int STEP = 64;   // queries per dK/dV step, keys per dQ step
-constexpr uint32_t BOX_T = TILE * 128;  // [128 rows x 64 d] bf16 = 16 KB
+constexpr uint32_t BOX_T = TILE * 128;  // [128 rows x 64 d] bf16 = 16 KB (head dims 64, 128: 1 or 2 boxes)
 constexpr uint32_t BOX_S = STEP * 128;  // [64 rows x 64 d] bf16 = 8 KB
 constexpr uint32_t TILE_BYTES = 2 * BOX_T;
 constexpr uint32_t STEP_BYTES = 2 * BOX_S;
@@ -155,7 +154,8 @@ __device__ __forceinline__ void store_row_cols(uint32_t trow_col, float mul, __n
 }
 
 // ============================================================ preprocess
-// One warp per row, lane owns 4 consecutive columns.
+// One warp per row, lane owns D/32 consecutive columns.
+template <int D>
 __global__ void __launch_bounds__(256)
 bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __restrict__ hs,
                   const __nv_bfloat16* __restrict__ dhf, const __nv_bfloat16* __restrict__ dhs,
@@ -163,29 +163,34 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
                   float cf, float cs, __nv_bfloat16* __restrict__ gf, __nv_bfloat16* __restrict__ gs,
                   float* __restrict__ neg_lse2, float* __restrict__ neg_Df,
                   float* __restrict__ neg_Ds) {
+    constexpr int NP = D / 64;  // bf16 pairs per lane
     const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
-    const size_t e = row * HD + 4 * lane;
-    auto ld4 = [](const __nv_bfloat16* p, float (&o)[4]) {
-        const uint2 u = *reinterpret_cast<const uint2*>(p);
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-        o[0] = __low2float(a); o[1] = __high2float(a); o[2] = __low2float(b); o[3] = __high2float(b);
+    const size_t e = row * D + 2 * NP * lane;
+    auto ld = [](const __nv_bfloat16* p, float (&o)[2 * NP]) {
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+            const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162*>(p)[i];
+            o[2 * i] = __low2float(x);
+            o[2 * i + 1] = __high2float(x);
+        }
     };
     // c_t = exp(lse_full - lse_sparse) carries P_f to P_s on selected pairs; it is
     // folded into G_s here (0 where the sparse stream has no mass)
     const float lf = lse_f[row], ls = lse_s[row];
     const float c = ls > -INFINITY ? expf(lf - ls) : 0.f;
-    float f[4], s[4], uf[4] = {0, 0, 0, 0}, us[4] = {0, 0, 0, 0};
-    ld4(hf + e, f);
-    ld4(hs + e, s);
-    if (dhf) ld4(dhf + e, uf);
-    if (dhs) ld4(dhs + e, us);
-    float sf = 0.f, ss = 0.f;
-    uint32_t pf[2], ps[2];
+    float f[2 * NP], s[2 * NP], uf[2 * NP], us[2 * NP];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2 * NP; ++i) uf[i] = us[i] = 0.f;
+    ld(hf + e, f);
+    ld(hs + e, s);
+    if (dhf) ld(dhf + e, uf);
+    if (dhs) ld(dhs + e, us);
+    float sf = 0.f, ss = 0.f;
+    uint32_t pf[NP], ps[NP];
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
         const float gf0 = uf[2 * i] + cf * (f[2 * i] - s[2 * i]);
         const float gf1 = uf[2 * i + 1] + cf * (f[2 * i + 1] - s[2 * i + 1]);
         const float gs0 = c * (us[2 * i] + cs * (s[2 * i] - f[2 * i]));
@@ -198,8 +203,11 @@ bwd_tc_pre_kernel(const __nv_bfloat16* __restrict__ hf, const __nv_bfloat16* __r
         sf = fmaf(__low2float(rf), f[2 * i], fmaf(__high2float(rf), f[2 * i + 1], sf));
         ss = fmaf(__low2float(rs), s[2 * i], fmaf(__high2float(rs), s[2 * i + 1], ss));
     }
-    *reinterpret_cast<uint2*>(gf + e) = make_uint2(pf[0], pf[1]);
-    *reinterpret_cast<uint2*>(gs + e) = make_uint2(ps[0], ps[1]);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+        reinterpret_cast<uint32_t*>(gf + e)[i] = pf[i];
+        reinterpret_cast<uint32_t*>(gs + e)[i] = ps[i];
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         sf += __shfl_xor_sync(0xffffffffu, sf, o);
@@ -276,18 +284,27 @@ enum : int {  // barrier indices, derived from the ring depth
     B_DONE = B_TFREE + 2, B_DRAIN = B_DONE + 1, B_COUNT = B_DRAIN + 1
 };
 static_assert(B_COUNT <= NBAR, "barrier area");
-constexpr uint32_t TM_DV = 0, TM_DK = 128, TM_K = 256, TM_V = 320, TM_S = 384, TM_DPF = 448;
+// TMEM columns for head dim D: dV | dK (D each) | K | V (bf16, D/2 each) | S | dP (64 each);
+// 512 at D = 128, 320 at D = 64
+template <int D> struct Tm {
+    static constexpr uint32_t DV = 0, DK = D, K = 2 * D, V = 2 * D + D / 2, S = 3 * D, DPF = 3 * D + 64;
+};
 // bf16 P^T of warpgroup w over the first 16 of its 32 dP columns, the masked
 // copy in the other 16: TMEM column of the A operand's k-step kk (16 queries)
 __device__ __forceinline__ uint32_t acol(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 }  // namespace kv
 
+template <int D>
 __global__ void __launch_bounds__(kv::kThr, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_gf,
                    const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_ds,
                    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                    const BwdArgs a) {
     using namespace kv;
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    constexpr uint32_t TM_DV = Tm<D>::DV, TM_DK = Tm<D>::DK, TM_K = Tm<D>::K, TM_V = Tm<D>::V,
+                       TM_S = Tm<D>::S, TM_DPF = Tm<D>::DPF;
+    constexpr uint32_t kStep = STEP * D * 2;  // bytes of one step tile (Q, G_f or G_s')
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -373,17 +390,18 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (elect_one()) {
                 const bool sp = fl != 0u;
                 flags[s] = fl;  // published by the arrive below
-                mbar_expect_tx(BAR(B_FULL + s), 2 * STEP_BYTES + 2 * STEP * 4 +
-                                                    (sp ? STEP_BYTES + STEP * 4 : 0u));
-                tma_load_3d(st + ST_Q, &tm_q, BAR(B_FULL + s), 0, t0, bh);
-                tma_load_3d(st + ST_Q + BOX_S, &tm_q, BAR(B_FULL + s), 64, t0, bh);
-                tma_load_3d(st + ST_GF, &tm_gf, BAR(B_FULL + s), 0, t0, bh);
-                tma_load_3d(st + ST_GF + BOX_S, &tm_gf, BAR(B_FULL + s), 64, t0, bh);
+                mbar_expect_tx(BAR(B_FULL + s), 2 * kStep + 2 * STEP * 4 + (sp ? kStep + STEP * 4 : 0u));
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x) {
+                    tma_load_3d(st + ST_Q + x * BOX_S, &tm_q, BAR(B_FULL + s), 64 * x, t0, bh);
+                    tma_load_3d(st + ST_GF + x * BOX_S, &tm_gf, BAR(B_FULL + s), 64 * x, t0, bh);
+                }
                 bulk_load(rw, a.neg_lse2 + rowbase + t0, STEP * 4, BAR(B_FULL + s));
                 bulk_load(rw + STEP * 4, a.neg_Df + rowbase + t0, STEP * 4, BAR(B_FULL + s));
                 if (sp) {  // the sparse stream's operands only where it has work
-                    tma_load_3d(st + ST_GS, &tm_gs, BAR(B_FULL + s), 0, t0, bh);
-                    tma_load_3d(st + ST_GS + BOX_S, &tm_gs, BAR(B_FULL + s), 64, t0, bh);
+#pragma unroll
+                    for (int x = 0; x < D / 64; ++x)
+                        tma_load_3d(st + ST_GS + x * BOX_S, &tm_gs, BAR(B_FULL + s), 64 * x, t0, bh);
                     bulk_load(rw + 2 * STEP * 4, a.neg_Ds + rowbase + t0, STEP * 4, BAR(B_FULL + s));
                 }
             }
@@ -398,7 +416,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // descriptors formed once, advanced by constant offsets; each MMA group
             // and its commits are issued by one elected lane
             constexpr uint32_t id_s = idesc_bf16_f32(TILE, STEP, false);  // S^T, dP^T
-            constexpr uint32_t id_a = idesc_bf16_f32(TILE, HD, true);     // dV, dK
+            constexpr uint32_t id_a = idesc_bf16_f32(TILE, D, true);      // dV, dK
             const uint64_t st_k0 = smem_desc_sw128(base + OFF_STAGE, 16, 1024);      // K-major
             const uint64_t st_m0 = smem_desc_sw128(base + OFF_STAGE, BOX_S, 1024);   // MN-major
             const uint64_t ds_0 = smem_desc_sw128(base + OFF_DS, 16, 1024);          // K-major A
@@ -407,7 +425,7 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             auto issue_tn = [&](uint32_t d, uint32_t a_col, uint32_t st_off) {
                 const uint64_t bd = desc_add(st_k0, st_off);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
+                for (int kk = 0; kk < D / 16; ++kk)
                     mma_ts(tmem + d, tmem + a_col + 8 * kk, desc_add(bd, ks(kk)), id_s, kk > 0);
             };
             auto stage_off = [&](int i) { return (uint32_t)((i % NSTAGE) * STAGE_BYTES); };
@@ -539,20 +557,21 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const bool key_ok = s_tok < a.T;                // warp-uniform (T is a multiple of 64)
         const int c0 = COLS * wg;
         bool ok = true;
-        {  // K and V rows of the tile (this warpgroup's 64 columns of each) into TMEM
+        {  // K and V rows of the tile (this warpgroup's D/2 columns of each) into TMEM
             const size_t row = rowbase + (key_ok ? s_tok : 0);
+            constexpr int W = D / 4;  // 32-bit TMEM columns per warpgroup and operand
             auto fill = [&](const __nv_bfloat16* src, uint32_t col) {
-                uint32_t u[32];
-                const uint4* p4 = reinterpret_cast<const uint4*>(src + row * HD + 64 * wg);
+                uint32_t u[W];
+                const uint4* p4 = reinterpret_cast<const uint4*>(src + row * D + 2 * W * wg);
 #pragma unroll
-                for (int v4 = 0; v4 < 8; ++v4) {
+                for (int v4 = 0; v4 < W / 4; ++v4) {
                     const uint4 x = key_ok ? __ldg(p4 + v4) : make_uint4(0u, 0u, 0u, 0u);
                     u[4 * v4] = x.x;
                     u[4 * v4 + 1] = x.y;
                     u[4 * v4 + 2] = x.z;
                     u[4 * v4 + 3] = x.w;
                 }
-                tmem_st32(trow + col + 32 * wg, u);
+                tmem_st<W>(trow + col + W * wg, u);
             };
             fill(k, TM_K);
             fill(v, TM_V);
@@ -698,8 +717,10 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (ok) ok = wait(B_DONE, 0);
         if (ok) {
             const size_t row = rowbase + (key_ok ? s_tok : 0);
-            store_row_cols<2>(trow + TM_DV + 64 * wg, 1.f, a.dv + row * HD + 64 * wg, key_ok);
-            store_row_cols<2>(trow + TM_DK + 64 * wg, a.sm_scale, a.dk + row * HD + 64 * wg, key_ok);
+            constexpr int OC = D / 2;  // output columns per warpgroup
+            store_row_cols<OC / 32>(trow + TM_DV + OC * wg, 1.f, a.dv + row * D + OC * wg, key_ok);
+            store_row_cols<OC / 32>(trow + TM_DK + OC * wg, a.sm_scale, a.dk + row * D + OC * wg,
+                                    key_ok);
         }
     }
     fence_before_sync();
@@ -732,6 +753,7 @@ enum : int {
 static_assert(B_COUNT <= 16, "barrier area holds 16");
 }  // namespace dq
 
+template <int D>
 __global__ void __launch_bounds__(dq::kThr, 1)
 bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_k,
                    const BwdArgs a) {
@@ -794,11 +816,12 @@ bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_const
             // blocks of key tile j for query steps 2(I - j) and 2(I - j) + 1
             const int blk = bh * a.ds_blocks + j * (a.T / STEP) - j * (j - 1) + 2 * (I - j);
             if (elect_one()) {
-                mbar_expect_tx(BAR(B_FULL + s), (two ? 2 : 1) * BLK_BYTES + TILE_BYTES);
+                mbar_expect_tx(BAR(B_FULL + s), (two ? 2 : 1) * BLK_BYTES + TILE * D * 2);
                 tma_load_3d(st, &tm_ds, BAR(B_FULL + s), 0, 0, blk);
                 if (two) tma_load_3d(st + BLK_BYTES, &tm_ds, BAR(B_FULL + s), 0, 0, blk + 1);
-                tma_load_3d(st + ST_B, &tm_k, BAR(B_FULL + s), 0, TILE * j, bh);
-                tma_load_3d(st + ST_B + BOX_T, &tm_k, BAR(B_FULL + s), 64, TILE * j, bh);
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x)
+                    tma_load_3d(st + ST_B + x * BOX_T, &tm_k, BAR(B_FULL + s), 64 * x, TILE * j, bh);
             }
             __syncwarp();
             issued[s] = j;
@@ -808,7 +831,7 @@ bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_const
                 if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
     } else if (warp == 1) {
         // ------------------------------------------ MMA issuer (whole warp)
-        constexpr uint32_t id = idesc_bf16_f32(TILE, HD, true, true);  // A and B MN-major
+        constexpr uint32_t id = idesc_bf16_f32(TILE, D, true, true);  // A and B MN-major
         const uint64_t a0 = smem_desc_sw128(base, BLK_BYTES, 1024);
         const uint64_t b0 = smem_desc_sw128(base + ST_B, BOX_T, 1024);
         for (int j = 0; j < nj; ++j) {
@@ -840,7 +863,7 @@ bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_const
         if (__all_sync(FULL, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim))) {
             fence_after_sync();
             const bool valid = t < a.T;
-            store_row_cols<4>(trow, a.sm_scale, a.dq + (rowbase + (valid ? t : 0)) * HD, valid);
+            store_row_cols<D / 32>(trow, a.sm_scale, a.dq + (rowbase + (valid ? t : 0)) * D, valid);
         }
     }
     fence_before_sync();
@@ -866,12 +889,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [BH, T, 128] bf16 as a 3-D tensor (d, t, bh); box 64 d x `rows` t; 128B swizzle.
-int make_map(CUtensorMap* m, const void* ptr, int BH, int T, int rows) {
+// [BH, T, D] bf16 as a 3-D tensor (d, t, bh); box 64 d x `rows` t; 128B swizzle.
+int make_map(CUtensorMap* m, const void* ptr, int BH, int T, int rows, int D) {
     auto fn = encode_fn();
     if (!fn) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)T * HD * 2};
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
@@ -939,7 +962,7 @@ TcWs carve(const ssa_params_t& p, void* ws) {
 int bwd_tc_heads_per_group(const ssa_params_t& p) { return heads_per_chunk(p); }
 
 bool bwd_tc_supported(const ssa_params_t& p) {
-    return p.dtype == SSA_BF16 && p.D == HD && (p.block == 64 || p.block == 128) &&
+    return p.dtype == SSA_BF16 && (p.D == 64 || p.D == 128) && (p.block == 64 || p.block == 128) &&
            (size_t)p.B * p.H * ((p.T + TILE - 1) / TILE) <= 0x7fffffffull &&
            ds_blocks_per_bh(p.T) <= 0x7fffffffull;
 }
@@ -949,16 +972,18 @@ size_t bwd_tc_workspace(const ssa_params_t& p) {
            (size_t)heads_per_chunk(p) * ds_blocks_per_bh(p.T) * STEP * TILE * 2;
 }
 
-int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
-                  const uint32_t* mask, const void* hf, const void* hs, const float* lf,
-                  const float* ls, const void* dhf, const void* dhs, float w_s, float w_c,
-                  void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
+namespace {
+template <int D>
+int launch_bwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                       const void* hf, const void* hs, const float* lf, const float* ls,
+                       const void* dhf, const void* dhs, float w_s, float w_c, const uint32_t* mask,
+                       void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
     const int BH = p.B * p.H;
     const TcWs w = carve(p, ws);
     const size_t rows = num_rows(p);
     const double two_over_n = 2.0 / (double)num_elems(p);
     mark_kernel_event(0, s);
-    bwd_tc_pre_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
+    bwd_tc_pre_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(hf), static_cast<const __nv_bfloat16*>(hs),
         static_cast<const __nv_bfloat16*>(dhf), static_cast<const __nv_bfloat16*>(dhs), lf, ls, rows,
         (float)(w_s * two_over_n), (float)(w_c * two_over_n), w.gf, w.gs, w.neg_lse2, w.neg_Df, w.neg_Ds);
@@ -969,10 +994,10 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(bwd_dkdv_tc_kernel,
+        attr_err = cudaFuncSetAttribute(bwd_dkdv_tc_kernel<D>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kv::SMEM_BYTES);
         if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(bwd_dq_gemm_kernel,
+            attr_err = cudaFuncSetAttribute(bwd_dq_gemm_kernel<D>,
                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)dq::SMEM_BYTES);
     });
@@ -982,7 +1007,7 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     const int ntile = (p.T + TILE - 1) / TILE;
     const size_t nb = ds_blocks_per_bh(p.T);
     const int hc = heads_per_chunk(p);
-    const size_t head_elems = (size_t)p.T * HD;
+    const size_t head_elems = (size_t)p.T * D;
     const size_t head_mask = (size_t)num_blocks(p) * mask_words(p);
     // every (batch, head) is independent: chunks of hc heads share the dS^T buffer
     for (int h0 = 0; h0 < BH && st == SSA_OK; h0 += hc) {
@@ -991,10 +1016,10 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
             return static_cast<const void*>(static_cast<const __nv_bfloat16*>(ptr) + h0 * head_elems);
         };
         CUtensorMap k128, q64, gf64, gs64, ds_map;
-        st = make_map(&k128, off(k), nh, p.T, TILE);
-        if (st == SSA_OK) st = make_map(&q64, off(q), nh, p.T, STEP);
-        if (st == SSA_OK) st = make_map(&gf64, off(w.gf), nh, p.T, STEP);
-        if (st == SSA_OK) st = make_map(&gs64, off(w.gs), nh, p.T, STEP);
+        st = make_map(&k128, off(k), nh, p.T, TILE, D);
+        if (st == SSA_OK) st = make_map(&q64, off(q), nh, p.T, STEP, D);
+        if (st == SSA_OK) st = make_map(&gf64, off(w.gf), nh, p.T, STEP, D);
+        if (st == SSA_OK) st = make_map(&gs64, off(w.gs), nh, p.T, STEP, D);
         if (st == SSA_OK) st = make_ds_map(&ds_map, w.ds, (size_t)nh * nb);
         if (st != SSA_OK) break;
 
@@ -1016,17 +1041,29 @@ int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
         a.sm_scale = p.sm_scale;
         a.timeout_ns = wait_limit_ns();
         const unsigned grid = (unsigned)((size_t)nh * ntile);
-        bwd_dkdv_tc_kernel<<<grid, kv::kThr, kv::SMEM_BYTES, s>>>(
+        bwd_dkdv_tc_kernel<D><<<grid, kv::kThr, kv::SMEM_BYTES, s>>>(
             q64, gf64, gs64, ds_map, static_cast<const __nv_bfloat16*>(off(k)),
             static_cast<const __nv_bfloat16*>(off(v)), a);
         st = check_launch("bwd_dkdv_tc_kernel");
         if (st != SSA_OK) break;
         if (h0 == 0) mark_kernel_event(2, s);
-        bwd_dq_gemm_kernel<<<grid, dq::kThr, dq::SMEM_BYTES, s>>>(ds_map, k128, a);
+        bwd_dq_gemm_kernel<D><<<grid, dq::kThr, dq::SMEM_BYTES, s>>>(ds_map, k128, a);
         st = check_launch("bwd_dq_gemm_kernel");
         if (h0 == 0) mark_kernel_event(3, s);
     }
     return st;
+}
+}  // namespace
+
+int launch_bwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
+                  const uint32_t* mask, const void* hf, const void* hs, const float* lf,
+                  const float* ls, const void* dhf, const void* dhs, float w_s, float w_c,
+                  void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
+    if (p.D == 64)
+        return launch_bwd_tc_impl<64>(p, q, k, v, hf, hs, lf, ls, dhf, dhs, w_s, w_c, mask, dq, dk,
+                                      dv, ws, s);
+    return launch_bwd_tc_impl<128>(p, q, k, v, hf, hs, lf, ls, dhf, dhs, w_s, w_c, mask, dq, dk,
+                                   dv, ws, s);
 }
 
 int bwd_tc_take_status(cudaStream_t) {

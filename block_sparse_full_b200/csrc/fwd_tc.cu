@@ -45,10 +45,10 @@ using namespace tc;
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
-constexpr int HD = 128;  // head dim
+constexpr int HD = 128;  // largest head dim (the shared-memory layout is sized for it)
 constexpr int kThreads = 384;  // warps 0-1 roles, 2-3 idle, 4-11 two softmax warpgroups
 constexpr int kSoftmax = 256;
-constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB
+constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB ring slot (half used at d = 64)
 constexpr uint32_t HALF_BYTES = 128 * 128;    // [128 rows x 64 cols] bf16 box, 16 KB
 constexpr int kMaxWords = 256;                // mask words per query block (n <= 8192)
 
@@ -115,16 +115,20 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
     return true;
 }
 
+// D: head dim, 64 or 128 (one or two 64-column boxes per tile; an S tile
+// takes D/16 MMA k-steps; each softmax warpgroup owns D/2 output columns).
 // kSparse = false: the dual forward (both streams).  kSparse = true: the
 // sparse stream alone (inference, the same operations as MoBA): key tiles
 // that neither of the tile's query blocks selects are skipped by every
 // role, the running max is taken over selected keys only, unselected
 // (row, half) pairs get P = 0, one accumulator (O_sel), and the epilogue
 // writes h_sparse and lse_sparse only.
-template <bool kSparse>
+template <int D, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+    static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    constexpr uint32_t kTileBytes = BM * D * 2;  // bytes a Q / K / V tile load brings
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -196,9 +200,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            mbar_expect_tx(BAR(B_QFULL), TILE_BYTES);
-            tma_load_3d(base + OFF_Q, &tm_q, BAR(B_QFULL), 0, t0, bh);
-            tma_load_3d(base + OFF_Q + HALF_BYTES, &tm_q, BAR(B_QFULL), 64, t0, bh);
+            mbar_expect_tx(BAR(B_QFULL), kTileBytes);
+#pragma unroll
+            for (int x = 0; x < D / 64; ++x)
+                tma_load_3d(base + OFF_Q + x * HALF_BYTES, &tm_q, BAR(B_QFULL), 64 * x, t0, bh);
         }
         __syncwarp();
         int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
@@ -211,18 +216,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (jj >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, status, lim)))
                 break;
             if (elect_one()) {
-                mbar_expect_tx(BAR(B_KFULL + s), TILE_BYTES);
-                tma_load_3d(kdst, &tm_k, BAR(B_KFULL + s), 0, j * BN, bh);
-                tma_load_3d(kdst + HALF_BYTES, &tm_k, BAR(B_KFULL + s), 64, j * BN, bh);
+                mbar_expect_tx(BAR(B_KFULL + s), kTileBytes);
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x)
+                    tma_load_3d(kdst + x * HALF_BYTES, &tm_k, BAR(B_KFULL + s), 64 * x, j * BN, bh);
             }
             __syncwarp();
             issued_k[s] = jj;
             if (jj >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, status, lim)))
                 break;
             if (elect_one()) {
-                mbar_expect_tx(BAR(B_VFULL + s), TILE_BYTES);
-                tma_load_3d(vdst, &tm_v, BAR(B_VFULL + s), 0, j * BN, bh);
-                tma_load_3d(vdst + HALF_BYTES, &tm_v, BAR(B_VFULL + s), 64, j * BN, bh);
+                mbar_expect_tx(BAR(B_VFULL + s), kTileBytes);
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x)
+                    tma_load_3d(vdst + x * HALF_BYTES, &tm_v, BAR(B_VFULL + s), 64 * x, j * BN, bh);
             }
             __syncwarp();
             issued_v[s] = jj;
@@ -239,7 +246,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // Descriptors are formed once and advanced by constant offsets; each group
         // of MMAs (and its commits) is issued by one elected lane.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, HD, true);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
         const uint64_t qdesc = smem_desc_sw128(base + OFF_Q, 16, 1024);          // K-major Q
         const uint64_t kdesc0 = smem_desc_sw128(base + OFF_K, 16, 1024);         // K-major K
         // V is MN-major: 64-wide column boxes LBO = 16 KB apart, 8-key row groups
@@ -295,7 +302,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint32_t sd = tmem + (s ? TM_S1 : TM_S0);
             if (elect_one()) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < D / 16; ++kk) {
                     // K-major, 128B swizzle: 16 bf16 of d = 32 bytes per MMA step
                     const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
                     mma_ss(sd, desc_add(qdesc, off), desc_add(kd, off), idesc_qk, kk > 0 ? 1u : 0u);
@@ -321,7 +328,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
         const int r = sw * 32 + lane;  // row of the tile == TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
-        const int c0 = 64 * wg;
+        const int c0 = 64 * wg;          // this warpgroup's S columns (keys)
+        constexpr int OC = D / 2;        // and its O columns
+        const int oc0 = OC * wg;
         float* xch = reinterpret_cast<float*>(gbase + OFF_XCH);  // [parity][wg][row]
         // named barrier of the two warpgroups; wg_vote also ORs a flag across them so
         // that both always leave the tile loop at the same tile (same barrier count)
@@ -342,10 +351,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             uint32_t z[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) z[i] = 0u;
-            tmem_st32(trow + TM_OSEL + c0, z);
-            tmem_st32(trow + TM_OSEL + c0 + 32, z);
-            tmem_st32(trow + TM_OUNS + c0, z);
-            tmem_st32(trow + TM_OUNS + c0 + 32, z);
+#pragma unroll
+            for (int x = 0; x < OC / 32; ++x) {
+                tmem_st32(trow + TM_OSEL + oc0 + 32 * x, z);
+                tmem_st32(trow + TM_OUNS + oc0 + 32 * x, z);
+            }
             tmem_wait_st();
         }
         const float sl2 = a.scale_log2;
@@ -422,9 +432,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     m2 = mup;
                     lsel *= alpha;
                     luns *= alpha;
+                    constexpr int NCH = OC / 32;  // 32-column chunks per accumulator
 #pragma unroll 1
-                    for (int c = 0; c < (kSparse ? 2 : 4); ++c) {
-                        const uint32_t col = (c < 2 ? TM_OSEL : TM_OUNS) + c0 + 32 * (c & 1);
+                    for (int c = 0; c < (kSparse ? NCH : 2 * NCH); ++c) {
+                        const uint32_t col = (c < NCH ? TM_OSEL : TM_OUNS) + oc0 + 32 * (c % NCH);
                         uint32_t u[32];
                         tmem_ld32(trow + col, u);
                         tmem_wait_ld();
@@ -517,9 +528,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 fence_after_sync();
                 const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
 #pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < OC / 32; ++c) {
                     uint32_t os[32];
-                    tmem_ld32(trow + TM_OSEL + c0 + 32 * c, os);
+                    tmem_ld32(trow + TM_OSEL + oc0 + 32 * c, os);
                     tmem_wait_ld();
                     uint32_t hs[16];
 #pragma unroll
@@ -527,7 +538,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         hs[e] = pack_bf16(__uint_as_float(os[2 * e]) * inv_ls,
                                           __uint_as_float(os[2 * e + 1]) * inv_ls);
                     if (valid) {
-                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * HD + c0 + 32 * c);
+                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * D + oc0 + 32 * c);
 #pragma unroll
                         for (int v4 = 0; v4 < 4; ++v4)
                             ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
@@ -545,10 +556,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const float inv_l = 1.f / l;
                 const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
     #pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < OC / 32; ++c) {
                     uint32_t os[32], ou[32];
-                    tmem_ld32(trow + TM_OSEL + c0 + 32 * c, os);
-                    tmem_ld32(trow + TM_OUNS + c0 + 32 * c, ou);
+                    tmem_ld32(trow + TM_OSEL + oc0 + 32 * c, os);
+                    tmem_ld32(trow + TM_OUNS + oc0 + 32 * c, ou);
                     tmem_wait_ld();
                     uint32_t hf[16], hs[16];
     #pragma unroll
@@ -563,8 +574,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         hs[e] = pack_bf16(pa, pb);
                     }
                     if (valid) {
-                        uint4* df = reinterpret_cast<uint4*>(a.h_full + row * HD + c0 + 32 * c);
-                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * HD + c0 + 32 * c);
+                        uint4* df = reinterpret_cast<uint4*>(a.h_full + row * D + oc0 + 32 * c);
+                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * D + oc0 + 32 * c);
     #pragma unroll
                         for (int v4 = 0; v4 < 4; ++v4) {
                             df[v4] = make_uint4(hf[4 * v4], hf[4 * v4 + 1], hf[4 * v4 + 2], hf[4 * v4 + 3]);
@@ -608,13 +619,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [BH, T, 128] bf16 viewed as a 3-D tensor (d, t, bh); box = 64 d x 128 t,
+// [BH, T, D] bf16 viewed as a 3-D tensor (d, t, bh); box = 64 d x 128 t,
 // 128-byte swizzle; rows past T are zero-filled by the TMA unit.
-int make_map(CUtensorMap* m, const void* ptr, int BH, int T) {
+int make_map(CUtensorMap* m, const void* ptr, int BH, int T, int D) {
     auto fn = encode_fn();
     if (!fn) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)T * HD * 2};
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)BM, 1};
     cuuint32_t es[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
@@ -627,26 +638,26 @@ int make_map(CUtensorMap* m, const void* ptr, int BH, int T) {
 }  // namespace
 
 bool fwd_tc_supported(const ssa_params_t& p) {
-    return p.dtype == SSA_BF16 && p.D == HD && (p.block == 64 || p.block == 128) &&
+    return p.dtype == SSA_BF16 && (p.D == 64 || p.D == 128) && (p.block == 64 || p.block == 128) &&
            mask_words(p) <= kMaxWords && (size_t)p.B * p.H * ((p.T + BM - 1) / BM) <= 0x7fffffffull;
 }
 
 size_t fwd_tc_workspace(const ssa_params_t&) { return 0; }
 
 namespace {
-template <bool kSparse>
+template <int D, bool kSparse>
 int launch_fwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, const void* v,
                        const uint32_t* mask, const FwdArgs& outs, cudaStream_t s) {
     const int BH = p.B * p.H;
     CUtensorMap mq, mk, mv;
-    int st = make_map(&mq, q, BH, p.T);
-    if (st == SSA_OK) st = make_map(&mk, k, BH, p.T);
-    if (st == SSA_OK) st = make_map(&mv, v, BH, p.T);
+    int st = make_map(&mq, q, BH, p.T, D);
+    if (st == SSA_OK) st = make_map(&mk, k, BH, p.T, D);
+    if (st == SSA_OK) st = make_map(&mv, v, BH, p.T, D);
     if (st != SSA_OK) return st;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(fwd_tc_kernel<kSparse>,
+        attr_err = cudaFuncSetAttribute(fwd_tc_kernel<D, kSparse>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     });
     if (attr_err != cudaSuccess)
@@ -661,7 +672,7 @@ int launch_fwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, cons
     a.scale_log2 = p.sm_scale * 1.4426950408889634f;
     a.timeout_ns = wait_limit_ns();
     const unsigned grid = (unsigned)((size_t)BH * ((p.T + BM - 1) / BM));
-    fwd_tc_kernel<kSparse><<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, a);
+    fwd_tc_kernel<D, kSparse><<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, a);
     return check_launch(kSparse ? "fwd_tc_kernel<sparse>" : "fwd_tc_kernel");
 }
 }  // namespace
@@ -676,7 +687,8 @@ int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const voi
     o.lse_full = lf;
     o.lse_sparse = ls;
     o.sqdiff = sq;
-    return launch_fwd_tc_impl<false>(p, q, k, v, mask, o, s);
+    return p.D == 64 ? launch_fwd_tc_impl<64, false>(p, q, k, v, mask, o, s)
+                     : launch_fwd_tc_impl<128, false>(p, q, k, v, mask, o, s);
 }
 
 int launch_fwd_sparse_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
@@ -684,7 +696,8 @@ int launch_fwd_sparse_tc(const ssa_params_t& p, const void* q, const void* k, co
     FwdArgs o{};
     o.h_sparse = static_cast<__nv_bfloat16*>(hs);
     o.lse_sparse = ls;
-    return launch_fwd_tc_impl<true>(p, q, k, v, mask, o, s);
+    return p.D == 64 ? launch_fwd_tc_impl<64, true>(p, q, k, v, mask, o, s)
+                     : launch_fwd_tc_impl<128, true>(p, q, k, v, mask, o, s);
 }
 
 int fwd_tc_take_status(cudaStream_t) {

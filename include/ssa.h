@@ -36,7 +36,7 @@
  *     whose bounded wait expired records SSA_ERR_TIMEOUT in a device status
  *     word that ssa_device_status() reports after synchronising.
  *   - Alignment: every device pointer 16-byte aligned; the bf16 tensor-core
- *     path additionally requires D == 128.
+ *     path takes D == 64 or 128.
  */
 #ifndef SSA_H
 #define SSA_H
@@ -236,8 +236,8 @@ const char* ssa_last_error(void);
 int ssa_bwd_heads_per_group(const ssa_params_t* params);
 
 /* Which kernel family the params select: 0 = CUDA-core (SIMT) kernels
- * (float32, bf16 with D = 64, or SSA_FLAG_FORCE_SIMT), 1 = bf16 tcgen05
- * tensor-core kernels (D = 128), -1 = invalid or unsupported params. */
+ * (float32, or SSA_FLAG_FORCE_SIMT), 1 = bf16 tcgen05 tensor-core kernels
+ * (D = 64 or 128), -1 = invalid or unsupported params. */
 int ssa_kernel_path(const ssa_params_t* params);
 
 /* Self-test of the element-wise arithmetic inside the tensor-core kernels

@@ -112,7 +112,7 @@ def test_workspace_sizes_scale_with_shape():
 
 def test_kernel_path_choice():
     assert ssa.ssa_kernel_path(P(dtype=ssa.SSA_F32)) == 0
-    assert ssa.ssa_kernel_path(P(D=64)) == 0
+    assert ssa.ssa_kernel_path(P(D=64)) == 1   # bf16 d = 64 runs on the tensor cores too
     assert ssa.ssa_kernel_path(P(flags=ssa.SSA_FLAG_FORCE_SIMT)) == 0
 
 

@@ -38,7 +38,7 @@ def _fwd_case(w, flags=0, topk=None, rows=None):
     o_sel = oracle_select(w, inp, topk, flags)
     d = to_dev(inp)
     p = params(w, d["q"], topk, flags)
-    tc_expected = w.dtype == "bf16" and w.D == 128 and not (flags & SIMT)
+    tc_expected = w.dtype == "bf16" and w.D in (64, 128) and not (flags & SIMT)
     assert ssa.ssa_kernel_path(p) == (1 if tc_expected else 0)
     g_sel = ssa.select_blocks(p, d["q"], d["k"])
     excused = assert_selection(g_sel, o_sel)
@@ -197,6 +197,20 @@ def test_train_workload_bwd_head0(mode):
     N = w.B * w.H * w.T * w.D
     ws_ = wc_ = 0.0 if mode == "upstream" else float(N)
     _bwd_case(f"{w.name}/{mode}", w, 0, ws_, wc_, heads=[0])
+
+
+# head dim 64 (Llama-3.2-1B-sized heads) on the tensor-core path
+D64 = Workload("bf16_H8_T4096_d64", B=1, H=8, T=4096, D=64, block=64, topk=16, dtype="bf16",
+               plant="hot", grads=True, seed=16)
+
+
+def test_d64_heads_fwd_sampled_rows_and_bwd():
+    w = D64
+    rows = sample_rows(w.T, w.block, 3, seed=17)
+    inp, d, p, o_sel, out, ref, _ = _fwd_case(w, rows=rows)
+    assert ssa.ssa_kernel_path(p) == 1
+    compare_fwd(w.name, "bf16", out, ref, rows=rows)
+    _bwd_case(w.name + "/bwd", w, 0, 0.0, 0.0, heads=[0, 5])
 
 
 # ------------------------------------------------------------------ robustness
