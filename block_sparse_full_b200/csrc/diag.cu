@@ -5,10 +5,10 @@
 //   sink(t)       = sum_{s <= t, s < block} exp(sigma q_t . k_s - lse_full(t)),
 //                   the full-softmax mass on block 0;
 //   mean_delta[h] = mean over t of delta(t),  mean_sink[h] = mean over t of sink(t).
-// Two launches: diag_sink_kernel (CUDA cores; K of block 0 staged transposed in
-// shared memory, one warp per query row, lane = key) and diag_head_kernel (one
-// CTA per head, fixed-order float64 sums: bitwise repeatable).  HBM-bound: the
-// first pass reads Q once.
+// Two launches: diag_sink_kernel (CUDA cores; block 0 of K and a 64-row slab of
+// Q staged transposed in shared memory, each warp register-tiles 8 rows x its
+// lane's 2 or 4 keys) and diag_head_kernel (one CTA per head, fixed-order
+// float64 sums: bitwise repeatable).  The first pass reads Q once.
 #include "device_util.cuh"
 #include "ssa_internal.h"
 
@@ -18,37 +18,71 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kRowsPerCta = 64;
 
-template <typename T>
+template <typename T, int KPL>  // KPL = keys of block 0 per lane (2 for block 64, 4 for 128)
 __global__ void __launch_bounds__(kThreads)
 diag_sink_kernel(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ lse,
                  int Tn, int D, int nkeys, float scale, float* __restrict__ sink) {
     extern __shared__ float sm[];
-    float* kT = sm;                         // [D][nkeys]: lane j reads column j (no conflicts)
-    float* qs = sm + (size_t)D * nkeys;     // [8 warps][D]
+    constexpr int NK = 32 * KPL;                 // key slots (keys past nkeys are masked)
+    constexpr int RW = kRowsPerCta / (kThreads / 32);  // rows per warp (8)
+    float* kT = sm;                              // [D][NK]: lane reads its KPL keys at once
+    float* qT = sm + (size_t)D * NK;             // [D][kRowsPerCta]: a warp's rows are contiguous
     const size_t bh = blockIdx.y;
+    const int r0 = blockIdx.x * kRowsPerCta;
     const T* kh = k + bh * (size_t)Tn * D;
-    for (int e = threadIdx.x; e < nkeys * D; e += kThreads) {
+    for (int e = threadIdx.x; e < NK * D; e += kThreads) {
         const int s = e / D, c = e % D;
-        kT[c * nkeys + s] = to_f32(kh[(size_t)s * D + c]);
+        kT[c * NK + s] = s < nkeys ? to_f32(kh[(size_t)s * D + c]) : 0.f;
+    }
+    for (int e = threadIdx.x; e < kRowsPerCta * D; e += kThreads) {
+        const int r = e / D, c = e % D;
+        const int t = r0 + r;
+        qT[c * kRowsPerCta + r] = t < Tn ? to_f32(q[(bh * (size_t)Tn + t) * D + c]) : 0.f;
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float* qw = qs + warp * D;
-    const int r0 = blockIdx.x * kRowsPerCta;
-    for (int r = r0 + warp; r < r0 + kRowsPerCta && r < Tn; r += kThreads / 32) {
-        const size_t row = bh * (size_t)Tn + r;
-        for (int c = lane; c < D; c += 32) qw[c] = to_f32(q[row * D + c]);
-        __syncwarp();
-        const float l = lse[row];
-        float acc = 0.f;
-        for (int s = lane; s < nkeys && s <= r; s += 32) {
-            float x = 0.f;
-            for (int c = 0; c < D; ++c) x = fmaf(qw[c], kT[c * nkeys + s], x);
-            acc += expf(scale * x - l);
+    // acc[r][j] = q_(row r of this warp) . k_(key KPL*lane + j)
+    float acc[RW][KPL];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) acc[r][j] = 0.f;
+    const float* qw = qT + RW * warp;
+    for (int c = 0; c < D; ++c) {
+        const float4 qa = *reinterpret_cast<const float4*>(qw + c * kRowsPerCta);
+        const float4 qb = *reinterpret_cast<const float4*>(qw + c * kRowsPerCta + 4);
+        const float qv[RW] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        float kv[KPL];
+        if constexpr (KPL == 2) {
+            const float2 x = *reinterpret_cast<const float2*>(kT + c * NK + 2 * lane);
+            kv[0] = x.x;
+            kv[1] = x.y;
+        } else {
+            const float4 x = *reinterpret_cast<const float4*>(kT + c * NK + 4 * lane);
+            kv[0] = x.x;
+            kv[1] = x.y;
+            kv[2] = x.z;
+            kv[3] = x.w;
         }
-        acc = warp_sum(acc);
-        if (lane == 0) sink[row] = acc;
-        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < RW; ++r)
+#pragma unroll
+            for (int j = 0; j < KPL; ++j) acc[r][j] = fmaf(qv[r], kv[j], acc[r][j]);
+    }
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+        const int t = r0 + RW * warp + r;
+        if (t >= Tn) break;  // warp-uniform
+        const size_t row = bh * (size_t)Tn + t;
+        const float l = lse[row];
+        float m = 0.f;
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) {
+            const int s = KPL * lane + j;
+            if (s < nkeys && s <= t) m += expf(scale * acc[r][j] - l);
+        }
+        m = warp_sum(m);
+        if (lane == 0) sink[row] = m;
     }
 }
 
@@ -86,26 +120,26 @@ int launch_diagnostics(const ssa_params_t& p, const void* q, const void* k, cons
                        const float* delta, float* sink, float* stats, cudaStream_t s) {
     const int BH = p.B * p.H;
     const int nkeys = p.block < p.T ? p.block : p.T;
-    const size_t smem = ((size_t)p.D * nkeys + (kThreads / 32) * (size_t)p.D) * sizeof(float);
+    const int kpl = p.block > 64 ? 4 : 2;
+    const size_t smem = ((size_t)p.D * 32 * kpl + (size_t)p.D * kRowsPerCta) * sizeof(float);
     const dim3 grid((unsigned)((p.T + kRowsPerCta - 1) / kRowsPerCta), (unsigned)BH);
-    cudaError_t e;
+    auto go = [&](auto kernel, auto qp, auto kp) -> int {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "diag: smem attribute: %s", cudaGetErrorString(e));
+        kernel<<<grid, kThreads, smem, s>>>(qp, kp, lse_full, p.T, p.D, nkeys, p.sm_scale, sink);
+        return check_launch("diag_sink_kernel");
+    };
+    int st;
     if (p.dtype == SSA_BF16) {
-        e = cudaFuncSetAttribute(diag_sink_kernel<__nv_bfloat16>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess)
-            diag_sink_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
-                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                lse_full, p.T, p.D, nkeys, p.sm_scale, sink);
+        auto qp = static_cast<const __nv_bfloat16*>(q);
+        auto kp = static_cast<const __nv_bfloat16*>(k);
+        st = kpl == 4 ? go(diag_sink_kernel<__nv_bfloat16, 4>, qp, kp)
+                      : go(diag_sink_kernel<__nv_bfloat16, 2>, qp, kp);
     } else {
-        e = cudaFuncSetAttribute(diag_sink_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e == cudaSuccess)
-            diag_sink_kernel<float><<<grid, kThreads, smem, s>>>(
-                static_cast<const float*>(q), static_cast<const float*>(k), lse_full, p.T, p.D,
-                nkeys, p.sm_scale, sink);
+        auto qp = static_cast<const float*>(q);
+        auto kp = static_cast<const float*>(k);
+        st = kpl == 4 ? go(diag_sink_kernel<float, 4>, qp, kp) : go(diag_sink_kernel<float, 2>, qp, kp);
     }
-    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "diag: smem attribute: %s", cudaGetErrorString(e));
-    int st = check_launch("diag_sink_kernel");
     if (st != SSA_OK) return st;
     diag_head_kernel<<<BH, kThreads, 0, s>>>(delta, sink, p.T, stats);
     return check_launch("diag_head_kernel");
