@@ -55,8 +55,8 @@ import numpy as np
 
 __all__ = [
     "f64", "pool_blocks", "block_scores", "select_blocks", "block_selection_matrix",
-    "attn_fwd_dual", "attn_fwd_sparse", "diagnostics", "align_loss", "alignment_upstream",
-    "attn_bwd",
+    "attn_fwd_dual", "attn_fwd_sparse", "diagnostics", "decode_pool", "decode_step",
+    "align_loss", "alignment_upstream", "attn_bwd",
 ]
 
 
@@ -283,6 +283,55 @@ def diagnostics(q, k, lse_full, delta, block: int, sm_scale: float):
             w = np.where(keys[None, :] <= np.arange(T)[:, None], np.exp(x - lse[b, h][:, None]), 0.0)
             sink[b, h] = w.sum(axis=1)
     return {"sink": sink, "mean_delta": dl.mean(axis=2), "mean_sink": sink.mean(axis=2)}
+
+
+def decode_pool(k_cache, block: int, n_done: int) -> np.ndarray:
+    """Pooled keys of the first ``n_done`` completed blocks of a key cache
+    [B, H, Tcap, d]: Kbar_j = mean of the keys of block j (float64)."""
+    k = f64(k_cache)
+    B, H, _, d = k.shape
+    return k[:, :, : n_done * block].reshape(B, H, n_done, block, d).mean(axis=3)
+
+
+def decode_step(q_t, k_cache, v_cache, t: int, block: int, topk: int, sm_scale: float,
+                force_sink: bool = False):
+    """One generation step of the sparse stream over a key/value cache (the
+    summaries' section 4: at inference SSA runs MoBA's operations; decoding
+    at long context).  The pages do not describe decoding itself; the reading
+    used here is MoBA's inference rule: the current query token q_t (not a
+    query-block mean, whose later members do not exist yet) is scored against
+    the pooled keys of the completed blocks, Kbar_j for j < i = t // block;
+    the current block i is always attended (its keys 0..t) and counts inside
+    the budget k; block 0 is forced only with ``force_sink``; the remaining
+    places go to the best-scoring completed blocks (score descending, index
+    ascending).  Then softmax attention over every key of the selected
+    blocks that is <= t.
+
+    q_t: [B, H, d]; k_cache, v_cache: [B, H, Tcap, d] holding keys 0..t.
+    Returns dict(h [B,H,d], lse [B,H], idx [B,H,k] ascending, -1 padded).
+    """
+    q, K, V = f64(q_t), f64(k_cache), f64(v_cache)
+    B, H, d = q.shape
+    i = t // block
+    kbar = decode_pool(k_cache, block, i)                          # [B, H, i, d]
+    h_out = np.zeros((B, H, V.shape[-1]))
+    lse_out = np.zeros((B, H))
+    idx_out = np.full((B, H, topk), -1, dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            forced = [i] + ([0] if force_sink and i > 0 else [])
+            cand = [j for j in range(i) if j not in forced]
+            score = {j: float(q[b, h] @ kbar[b, h, j]) for j in cand}
+            ranked = sorted(cand, key=lambda j: (-score[j], j))
+            sel = sorted(forced + ranked[: max(topk - len(forced), 0)])
+            idx_out[b, h, : len(sel)] = sel
+            keys = np.concatenate([np.arange(j * block, min((j + 1) * block, t + 1)) for j in sel])
+            x = sm_scale * (K[b, h, keys] @ q[b, h])
+            m = x.max()
+            e = np.exp(x - m)
+            h_out[b, h] = (e @ V[b, h, keys]) / e.sum()
+            lse_out[b, h] = m + np.log(e.sum())
+    return {"h": h_out, "lse": lse_out, "idx": idx_out}
 
 
 def align_loss(h_full, h_sparse, w_sparsity: float = 1.0, w_commit: float = 1.0):

@@ -44,6 +44,12 @@ MUTATIONS = {
     "sink_mass_strict_causality": ("w = np.where(keys[None, :] <= np.arange(T)[:, None], np.exp(x - lse[b, h][:, None]), 0.0)",
                                    "w = np.where(keys[None, :] < np.arange(T)[:, None], np.exp(x - lse[b, h][:, None]), 0.0)"),
     "sink_mass_half_block": ("keys = np.arange(min(block, T))", "keys = np.arange(min(block, T) // 2)"),
+    "decode_current_block_outside_budget": ("sel = sorted(forced + ranked[: max(topk - len(forced), 0)])",
+                                            "sel = sorted(forced + ranked[: max(topk - len(forced) + 1, 0)])"),
+    "decode_ties_to_higher_index": ("ranked = sorted(cand, key=lambda j: (-score[j], j))",
+                                    "ranked = sorted(cand, key=lambda j: (-score[j], -j))"),
+    "decode_future_keys_of_current_block": ("keys = np.concatenate([np.arange(j * block, min((j + 1) * block, t + 1)) for j in sel])",
+                                            "keys = np.concatenate([np.arange(j * block, (j + 1) * block) for j in sel])"),
 }
 
 PIN_TESTS = [
@@ -63,6 +69,9 @@ PIN_TESTS = [
     lambda: pins.test_sparse_only_diagonal_budget_is_blockwise_causal_attention(),
     lambda: pins.test_sparse_only_brute_force_tiny(),
     lambda: pins.test_sink_mass_is_library_softmax_on_block_zero(),
+    lambda: pins.test_decode_full_budget_is_causal_attention_row(),
+    lambda: pins.test_decode_selection_brute_force(),
+    lambda: pins.test_decode_ties_sink_and_first_block(),
 ]
 
 

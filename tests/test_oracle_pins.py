@@ -422,3 +422,73 @@ def test_sink_mass_rises_with_a_planted_sink():
     fwd = O.attn_fwd_dual(q2, k2, v, idx, cnt, block, 1.0)
     s1 = O.diagnostics(q2, k2, fwd["lse_full"], fwd["delta"], block, 1.0)["sink"]
     assert s1[..., block:].mean() > 0.9 > s0[..., block:].mean()
+
+
+# ---------------------------------------------------------------- decode over a KV cache
+
+def test_decode_pool_is_block_mean():
+    r = np.random.default_rng(31)
+    k = r.standard_normal((1, 2, 40, 3))
+    kb = O.decode_pool(k, 8, 4)
+    np.testing.assert_allclose(kb[0, 1, 2], k[0, 1, 16:24].mean(axis=0), rtol=0, atol=1e-15)
+    assert kb.shape == (1, 2, 4, 3)
+
+
+def test_decode_full_budget_is_causal_attention_row():
+    # every block selected: the step is the last row of causal attention (library)
+    r = np.random.default_rng(33)
+    B, H, Tcap, d, block = 1, 2, 80, 8, 16
+    K, V = r.standard_normal((B, H, Tcap, d)), r.standard_normal((B, H, Tcap, d))
+    for t in (0, 15, 16, 47, 79):
+        q = r.standard_normal((B, H, d))
+        out = O.decode_step(q, K, V, t, block, topk=Tcap // block, sm_scale=0.3)
+        ref = sdpa(q[:, :, None], K[:, :, : t + 1], V[:, :, : t + 1],
+                   np.ones((1, t + 1), dtype=bool), 0.3)[:, :, 0]
+        np.testing.assert_allclose(out["h"], ref, rtol=0, atol=1e-12)
+        x = torch.from_numpy(0.3 * np.einsum("bhd,bhsd->bhs", q, K[:, :, : t + 1]))
+        np.testing.assert_allclose(out["lse"], torch.logsumexp(x, -1).numpy(), rtol=0, atol=1e-12)
+        assert (out["idx"][..., : t // block + 1] == np.arange(t // block + 1)).all()
+
+
+def test_decode_selection_brute_force():
+    # the chosen set maximises the summed score among sets holding the current
+    # block (with distinct scores the top-(k-1) completed blocks are that set)
+    r = np.random.default_rng(35)
+    B, H, Tcap, d, block, topk = 1, 3, 96, 4, 8, 4
+    K, V = r.standard_normal((B, H, Tcap, d)), r.standard_normal((B, H, Tcap, d))
+    t = 90
+    q = r.standard_normal((B, H, d))
+    out = O.decode_step(q, K, V, t, block, topk, 1.0)
+    i = t // block
+    kbar = K[:, :, : i * block].reshape(B, H, i, block, d).mean(axis=3)
+    for h in range(H):
+        s = kbar[0, h] @ q[0, h]
+        best = max(itertools.combinations(range(i), topk - 1), key=lambda c: sum(s[list(c)]))
+        assert out["idx"][0, h].tolist() == sorted(list(best) + [i])
+        # attention restricted to those blocks' keys (library)
+        keys = np.concatenate([np.arange(j * block, min((j + 1) * block, t + 1))
+                               for j in out["idx"][0, h]])
+        ref = sdpa(q[0, h][None, None, None], K[0, h][keys][None, None], V[0, h][keys][None, None],
+                   np.ones((1, len(keys)), dtype=bool), 1.0)[0, 0, 0]
+        np.testing.assert_allclose(out["h"][0, h], ref, rtol=0, atol=1e-12)
+
+
+def test_decode_ties_sink_and_first_block():
+    B, H, Tcap, d, block = 1, 1, 48, 2, 8
+    K = np.zeros((B, H, Tcap, d))
+    V = np.arange(Tcap * d, dtype=float).reshape(1, 1, Tcap, d)
+    q = np.array([[[1.0, 0.0]]])
+    # all completed blocks score 0: ties go to the lowest indices
+    out = O.decode_step(q, K, V, 44, block, topk=3, sm_scale=1.0)
+    assert out["idx"][0, 0].tolist() == [0, 1, 5]
+    # block 0 forced by the sink flag even when another block scores higher
+    K2 = K.copy()
+    K2[0, 0, 24:32, 0] = 5.0
+    out = O.decode_step(q, K2, V, 44, block, topk=2, sm_scale=1.0, force_sink=True)
+    assert out["idx"][0, 0].tolist() == [0, 5]
+    out = O.decode_step(q, K2, V, 44, block, topk=2, sm_scale=1.0)
+    assert out["idx"][0, 0].tolist() == [3, 5]
+    # t inside block 0: only the current block's causal keys
+    out = O.decode_step(q, K, V, 3, block, topk=4, sm_scale=1.0)
+    assert out["idx"][0, 0].tolist() == [0, -1, -1, -1]
+    np.testing.assert_allclose(out["h"][0, 0], V[0, 0, :4].mean(axis=0), rtol=0, atol=1e-14)
