@@ -127,6 +127,7 @@ size_t ssa_workspace_size(const ssa_params_t* p, int which) {
         case SSA_WS_LOSS: return loss_workspace(*p);
         case SSA_WS_BWD: return bwd_workspace(*p);
         case SSA_WS_FWD_SPARSE: return fwd_sparse_workspace(*p);
+        case SSA_WS_DECODE: return decode_workspace(*p);
         default: fail(SSA_ERR_INVALID_ARG, "unknown workspace id %d", which); return (size_t)-1;
     }
 }
@@ -200,6 +201,43 @@ int ssa_attn_fwd_sparse(const ssa_params_t* p, const void* q, const void* k, con
     float* sqdiff = reinterpret_cast<float*>(r + 2 * rows);
     return launch_fwd_simt(*p, q, k, v, mask, h_full, h_sparse, delta, lse_full, lse_sparse, sqdiff,
                            s);
+}
+
+static int decode_shape(const ssa_params_t* p) {
+    SSA_TRY(validate(p));
+    if (p->D != 64 && p->D != 128) return fail(SSA_ERR_UNSUPPORTED, "decode: D must be 64 or 128");
+    if (p->topk > 64) return fail(SSA_ERR_UNSUPPORTED, "decode: topk must be <= 64");
+    return SSA_OK;
+}
+
+int ssa_decode_pool(const ssa_params_t* p, int j0, int j1, const void* k_cache, double* kbar,
+                    void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(decode_shape(p));
+    SSA_TRY(need_ptr(k_cache, "k_cache"));
+    SSA_TRY(need_ptr(kbar, "kbar"));
+    if (j0 < 0 || j1 < j0 || j1 > num_blocks(*p))
+        return fail(SSA_ERR_INVALID_ARG, "decode_pool: blocks [%d, %d) outside [0, %d]", j0, j1,
+                    num_blocks(*p));
+    return launch_decode_pool(*p, j0, j1, k_cache, kbar, static_cast<cudaStream_t>(stream));
+}
+
+int ssa_decode_step(const ssa_params_t* p, int t, const void* q, const void* k_cache,
+                    const void* v_cache, const double* kbar, void* h, float* lse, int32_t* idx,
+                    void* ws, size_t ws_bytes, void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(decode_shape(p));
+    if (t < 0 || t >= p->T) return fail(SSA_ERR_INVALID_ARG, "decode_step: t = %d outside [0, %d)", t, p->T);
+    SSA_TRY(need_ptr(q, "q"));
+    SSA_TRY(need_ptr(k_cache, "k_cache"));
+    SSA_TRY(need_ptr(v_cache, "v_cache"));
+    SSA_TRY(need_ptr(kbar, "kbar"));
+    SSA_TRY(need_ptr(h, "h"));
+    SSA_TRY(need_ptr(lse, "lse"));
+    SSA_TRY(opt_ptr(idx, "idx"));
+    SSA_TRY(need_ws(ws, ws_bytes, decode_workspace(*p), "ssa_decode_step"));
+    return launch_decode_step(*p, t, q, k_cache, v_cache, kbar, h, lse, idx, ws,
+                              static_cast<cudaStream_t>(stream));
 }
 
 int ssa_attn_diagnostics(const ssa_params_t* p, const void* q, const void* k,

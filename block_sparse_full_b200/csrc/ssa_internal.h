@@ -56,6 +56,14 @@ int fwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
 int launch_fwd_sparse_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
                          const uint32_t* mask, void* h_sparse, float* lse_sparse, cudaStream_t s);
 
+// ---- decode over a key/value cache (decode.cu)
+size_t decode_workspace(const ssa_params_t& p);
+int launch_decode_pool(const ssa_params_t& p, int j0, int j1, const void* k, double* kbar,
+                       cudaStream_t s);
+int launch_decode_step(const ssa_params_t& p, int t, const void* q, const void* k, const void* v,
+                       const double* kbar, void* h, float* lse, int32_t* idx, void* ws,
+                       cudaStream_t s);
+
 // ---- attention diagnostics (diag.cu)
 int launch_diagnostics(const ssa_params_t& p, const void* q, const void* k, const float* lse_full,
                        const float* delta, float* sink, float* stats, cudaStream_t s);

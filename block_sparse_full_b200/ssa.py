@@ -27,12 +27,13 @@ SSA_OK, SSA_ERR_INVALID_ARG, SSA_ERR_UNSUPPORTED = 0, -1, -2
 SSA_ERR_WORKSPACE, SSA_ERR_CUDA, SSA_ERR_TIMEOUT = -3, -4, -5
 SSA_F32, SSA_BF16 = 0, 1
 SSA_FLAG_FORCE_SINK, SSA_FLAG_FORCE_SIMT = 1, 2
-SSA_WS_SELECT, SSA_WS_FWD, SSA_WS_LOSS, SSA_WS_BWD, SSA_WS_FWD_SPARSE = 0, 1, 2, 3, 4
+SSA_WS_SELECT, SSA_WS_FWD, SSA_WS_LOSS, SSA_WS_BWD, SSA_WS_FWD_SPARSE, SSA_WS_DECODE = range(6)
 
 # every symbol include/ssa.h declares
 EXPORTS = (
     "ssa_workspace_size", "ssa_select_blocks", "ssa_select_blocks_noalloc",
-    "ssa_attn_fwd_dual", "ssa_attn_fwd_sparse", "ssa_attn_diagnostics", "ssa_align_loss",
+    "ssa_attn_fwd_dual", "ssa_attn_fwd_sparse", "ssa_attn_diagnostics", "ssa_decode_pool",
+    "ssa_decode_step", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
     "ssa_kernel_path", "ssa_bwd_heads_per_group", "ssa_selftest_math", "ssa_selftest_wait_timeout",
     "ssa_debug_set_wait_limit_ns", "ssa_debug_set_kernel_events", "ssa_version",
@@ -68,6 +69,9 @@ _SIGNATURES = {
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "ssa_attn_diagnostics": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p]),
+    "ssa_decode_pool": (c_int, [_P, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "ssa_decode_step": (c_int, [_P, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "ssa_align_loss": (c_int, [_P, c_void_p, c_float, c_float, c_void_p, c_void_p, c_size_t,
                                c_void_p]),
     "ssa_attn_bwd": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -137,6 +141,15 @@ def ssa_attn_fwd_sparse(params, q, k, v, idx, cnt, mask, h_sparse, lse_sparse, w
 def ssa_attn_diagnostics(params, q, k, lse_full, delta, sink_rows, head_stats, stream):
     return _lib.ssa_attn_diagnostics(ctypes.byref(params), q, k, lse_full, delta, sink_rows,
                                      head_stats, stream)
+
+
+def ssa_decode_pool(params, j0, j1, k_cache, kbar, stream):
+    return _lib.ssa_decode_pool(ctypes.byref(params), j0, j1, k_cache, kbar, stream)
+
+
+def ssa_decode_step(params, t, q, k_cache, v_cache, kbar, h, lse, idx, ws, ws_bytes, stream):
+    return _lib.ssa_decode_step(ctypes.byref(params), t, q, k_cache, v_cache, kbar, h, lse, idx, ws,
+                                ws_bytes, stream)
 
 
 def ssa_align_loss(params, sqdiff_rows, w_sparsity, w_commit, loss_out, ws, ws_bytes, stream):
@@ -298,6 +311,38 @@ def diagnostics(params, q, k, fwd):
     check(ssa_attn_diagnostics(params, _ptr(q), _ptr(k), _ptr(fwd["lse_full"]), _ptr(fwd["delta"]),
                                _ptr(sink), _ptr(stats), _stream(dev)), "ssa_attn_diagnostics")
     return {"sink": sink, "head_stats": stats}
+
+
+class DecodeCache:
+    """Key/value cache of capacity params.T and the pooled keys of its completed
+    blocks, for ssa_decode_step.  Tensors are allocated on ``device``."""
+
+    def __init__(self, params, device, dtype):
+        B, H, T, D = params.B, params.H, params.T, params.D
+        self.params = params
+        self.k = torch.zeros((B, H, T, D), dtype=dtype, device=device)
+        self.v = torch.zeros_like(self.k)
+        self.kbar = torch.zeros((B, H, T // params.block, D), dtype=torch.float64, device=device)
+        self.pooled = 0  # completed blocks whose pooled keys are in kbar
+        self.ws = workspace(params, SSA_WS_DECODE, device)
+
+    def pool_upto(self, n_blocks):
+        if n_blocks > self.pooled:
+            check(ssa_decode_pool(self.params, self.pooled, n_blocks, _ptr(self.k), _ptr(self.kbar),
+                                  _stream(self.k.device)), "ssa_decode_pool")
+            self.pooled = n_blocks
+
+    def step(self, t, q_t, idx=True):
+        """Attend q_t [B,H,D] at position t (keys/values 0..t already written)."""
+        p = self.params
+        self.pool_upto(t // p.block)
+        h = torch.empty((p.B, p.H, p.D), dtype=self.k.dtype, device=self.k.device)
+        lse = torch.empty((p.B, p.H), dtype=torch.float32, device=self.k.device)
+        ix = torch.empty((p.B, p.H, p.topk), dtype=torch.int32, device=self.k.device) if idx else None
+        check(ssa_decode_step(p, t, _ptr(q_t), _ptr(self.k), _ptr(self.v), _ptr(self.kbar), _ptr(h),
+                              _ptr(lse), _ptr(ix), _ptr(self.ws), self.ws.numel(),
+                              _stream(self.k.device)), "ssa_decode_step")
+        return {"h": h, "lse": lse, "idx": ix}
 
 
 def align_loss(params, sqdiff, w_sparsity=1.0, w_commit=1.0, ws=None, out=None):

@@ -90,7 +90,8 @@ enum {
     SSA_WS_FWD = 1,
     SSA_WS_LOSS = 2,
     SSA_WS_BWD = 3,
-    SSA_WS_FWD_SPARSE = 4
+    SSA_WS_FWD_SPARSE = 4,
+    SSA_WS_DECODE = 5
 };
 
 /* Bytes of scratch the named entry point needs for these params (0 if none,
@@ -169,6 +170,31 @@ int ssa_attn_fwd_sparse(const ssa_params_t* params, const void* q, const void* k
                         const void* v, const int32_t* idx, const int32_t* cnt,
                         const uint32_t* mask, void* h_sparse, float* lse_sparse,
                         void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Decoding over a key/value cache (section 4, "Efficienza": at inference SSA
+ * runs MoBA's operations; the pages do not describe decoding itself, and the
+ * rule below is MoBA's).  params->T is the cache capacity (a multiple of
+ * block); k_cache, v_cache are [B,H,T,D] in dtype, keys 0..t valid; D is 64
+ * or 128 and topk <= 64 here.
+ *
+ * ssa_decode_pool: kbar[b,h,j,:] = mean of the keys of block j, float64, for
+ *   j0 <= j < j1 (call it once a block is complete; kbar is [B,H,T/block,D]).
+ * ssa_decode_step: one step at position t.  i = t / block; the current query
+ *   q_t ([B,H,D]) is scored against kbar_j of the completed blocks j < i in
+ *   float64; S = {i} (+ {0} with SSA_FLAG_FORCE_SINK), plus the best-scoring
+ *   completed blocks (ties to the lower index) up to topk places in all (all
+ *   of them when there are fewer); then h = softmax attention of q_t over
+ *   every key of S that is <= t ([B,H,D] in dtype) and lse its log-sum-exp
+ *   (float32 [B,H]).  idx, if not NULL, receives S ascending, -1 padded
+ *   ([B,H,topk] int32).  kbar must hold blocks 0..i-1.  Workspace:
+ *   SSA_WS_DECODE.
+ */
+int ssa_decode_pool(const ssa_params_t* params, int j0, int j1, const void* k_cache,
+                    double* kbar, void* stream);
+int ssa_decode_step(const ssa_params_t* params, int t, const void* q, const void* k_cache,
+                    const void* v_cache, const double* kbar, void* h, float* lse, int32_t* idx,
+                    void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Attention diagnostics (section 1: the sparse approximation error grows

@@ -1,0 +1,64 @@
+"""GPU parity of the decode step over a key/value cache (the sparse stream at
+generation time, MoBA's inference rule) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_full_b200 import ssa
+from block_sparse_full_b200.inputs import WORKLOADS, make_inputs
+from oracle import ssa_oracle as O
+
+from gpu_parity_util import DEV, TOL, log, params
+from test_gpu_parity import SINK, SMALL
+
+pytestmark = pytest.mark.gpu
+
+
+def _decode(w, ts, flags=0, heads=None, topk=None):
+    inp = make_inputs(w)
+    p = params(w, inp["q"].to(DEV), topk, flags)
+    cache = ssa.DecodeCache(p, DEV, inp["k"].dtype)
+    cache.k.copy_(inp["k"].to(DEV))
+    cache.v.copy_(inp["v"].to(DEV))
+    hs = slice(None) if heads is None else heads
+    tol = TOL[w.dtype]
+    k_eff = topk if topk is not None else w.topk
+    for t in ts:
+        q_t = inp["q"][:, :, t].contiguous()
+        got = cache.step(t, q_t.to(DEV))
+        torch.cuda.synchronize()
+        ssa.device_status()
+        ref = O.decode_step(q_t[:, hs], inp["k"][:, hs], inp["v"][:, hs], t, w.block, k_eff,
+                            w.sm_scale, force_sink=bool(flags & SINK))
+        np.testing.assert_array_equal(got["idx"][:, hs].cpu().numpy(), ref["idx"])
+        h = got["h"][:, hs].float().cpu().numpy()
+        e = float(np.abs(h - ref["h"]).max())
+        scale = float(np.abs(ref["h"]).max())
+        el = float(np.abs(got["lse"][:, hs].cpu().numpy() - ref["lse"]).max())
+        assert e <= tol["h"] and e <= tol["h_rel"] * max(scale, 1.0 if w.dtype == "f32" else scale), (t, e)
+        assert el <= tol["lse"], (t, el)
+        log(f"decode/{w.name}/t{t}", h=e, lse=el)
+    # the pooled keys are exact float64 block means
+    n = cache.pooled
+    want = O.decode_pool(inp["k"], w.block, n)
+    np.testing.assert_array_equal(cache.kbar[:, :, :n].cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("name", ["bf16_T1216_b64", "bf16_T448_d64", "f32_T320_d128",
+                                  "bf16_B2_T640_b128_sink"])
+def test_decode_small(name):
+    w = SMALL[name]
+    T, b = w.T, w.block
+    ts = sorted({0, b - 1, b, 2 * b + 5, T // 2, T - b, T - 1})
+    _decode(w, ts)
+
+
+def test_decode_force_sink_and_full_budget():
+    w = SMALL["bf16_B2_T640_b128_sink"]
+    _decode(w, [130, 383, 639], flags=SINK)
+    _decode(w, [200, 639], topk=w.T // w.block)
+
+
+def test_decode_T65536_sink_last_token():
+    w = WORKLOADS["bf16_T65536_H8_sink"]
+    _decode(w, [w.T - 1, w.T // 2 + 17], heads=[1, 6])
