@@ -413,6 +413,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
     torch.cuda.synchronize(dev)
     layer.ssa.device_status()
     diag_ms = sum(a.elapsed_time(b) for a, b in diag_ev) / len(diag_ev)
+    decode = decode_bench(args, w, layer, stream, flush, dev)
     # reads Q, block 0 of K, lse_full and delta; writes the sink row vector
     esz = 2 if w.dtype == "bf16" else 4
     diag_bytes = w.B * w.H * (w.T * w.D * esz + min(w.block, w.T) * w.D * esz + 3 * w.T * 4)
@@ -443,6 +444,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
         "kernels": kernels,
         "inference_sparse_fwd": inference,
         "diagnostics": diagnostics,
+        "decode_step": decode,
         "fwd_tflops": round(fwd_tflops, 2),
         "fwd_frac_sustained": round(fwd_tflops / sustained, 4),
         "fwd_frac_burst": round(fwd_tflops / peaks.get("bf16_tflops", 1590.0), 4),
@@ -571,6 +573,40 @@ def run_reference(args, world):
 
 
 # ----------------------------------------------------------------------------- distributed
+
+def decode_bench(args, w, layer, stream, flush, dev):
+    """One generation step at the last position of the workload (context T):
+    the sparse stream over a key/value cache holding the step's K and V."""
+    from block_sparse_full_b200 import ssa
+    if w.D not in (64, 128) or w.topk > 64:
+        return None
+    cache = ssa.DecodeCache(layer.p, dev, layer.k.dtype)
+    cache.k.copy_(layer.k)
+    cache.v.copy_(layer.v)
+    t = w.T - 1
+    cache.pool_upto(t // w.block)
+    q_t = layer.q[:, :, t].contiguous()
+    ev = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.step(t, q_t, idx=False)
+        e1.record(stream)
+        if i >= args.warmup:
+            ev.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    ssa.device_status()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    esz = 2 if w.dtype == "bf16" else 4
+    i = t // w.block
+    # keys and values of the selected blocks, the pooled-key scan, q and h
+    per_head = w.topk * w.block * w.D * esz * 2 + i * w.D * 8 + 2 * w.D * esz
+    nbytes = per_head * w.B * w.H
+    return {"kernels": ["decode_select_kernel", "decode_attend_kernel", "decode_combine_kernel"],
+            "context": w.T, "ms": round(ms, 4), "hbm_bytes": nbytes,
+            "hbm_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+
 
 def workload(args):
     """The named workload, with the selection budget overridden by --topk."""
