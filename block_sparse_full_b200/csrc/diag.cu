@@ -30,12 +30,14 @@ diag_sink_kernel(const T* __restrict__ q, const T* __restrict__ k, const float* 
     const size_t bh = blockIdx.y;
     const int r0 = blockIdx.x * kRowsPerCta;
     const T* kh = k + bh * (size_t)Tn * D;
+    // transposed staging, consecutive threads on consecutive shared words (no
+    // bank conflicts); the strided global reads hit the same lines repeatedly (L1)
     for (int e = threadIdx.x; e < NK * D; e += kThreads) {
-        const int s = e / D, c = e % D;
+        const int s = e % NK, c = e / NK;
         kT[c * NK + s] = s < nkeys ? to_f32(kh[(size_t)s * D + c]) : 0.f;
     }
     for (int e = threadIdx.x; e < kRowsPerCta * D; e += kThreads) {
-        const int r = e / D, c = e % D;
+        const int r = e % kRowsPerCta, c = e / kRowsPerCta;
         const int t = r0 + r;
         qT[c * kRowsPerCta + r] = t < Tn ? to_f32(q[(bh * (size_t)Tn + t) * D + c]) : 0.f;
     }
