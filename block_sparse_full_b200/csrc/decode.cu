@@ -12,10 +12,11 @@
 // Launches (CUDA cores: one query per head is matrix-vector work, bound by
 // the key/value bytes it reads):
 //   decode_pool_kernel     Kbar_j = mean of block j's keys (float64, exact)
-//   decode_select_kernel   one CTA per head: scores (warp per block, lanes
-//                          split d), top-k by rounds of a CTA-wide argmax
-//   decode_attend_kernel   one CTA per (head, selected block): online
-//                          softmax over the block's keys (warp per key group)
+//   decode_select_kernel   one CTA per head: scores (thread per block),
+//                          top-k by rounds of a CTA-wide argmax
+//   decode_attend_kernel   one CTA per (head, selected block): scores with a
+//                          thread per key, softmax statistics CTA-wide, then
+//                          P V with threads over (d, key group)
 //   decode_combine_kernel  one warp per head merges the per-block partials
 #include "device_util.cuh"
 #include "ssa_internal.h"
@@ -52,13 +53,17 @@ decode_select_kernel(const T* __restrict__ q, const double* __restrict__ kbar, i
     const size_t bh = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const T* qh = q + bh * D;
-    // scores of the completed blocks (warp per block, lanes split d)
-    for (int j = warp; j < i; j += kThreads / 32) {
-        const double* kb = kbar + (bh * nb + j) * D;
+    // scores of the completed blocks: thread per block, independent loads of its
+    // float64 pooled key (one memory latency for the whole scan)
+    for (int j = threadIdx.x; j < i; j += kThreads) {
+        const double2* kb = reinterpret_cast<const double2*>(kbar + (bh * nb + j) * D);
         double acc = 0.0;
-        for (int c = lane; c < D; c += 32) acc += (double)to_f32(qh[c]) * kb[c];
-        acc = warp_sum(acc);
-        if (lane == 0) score[j] = acc;
+#pragma unroll 8
+        for (int c = 0; c < D / 2; ++c) {
+            const double2 x = kb[c];
+            acc += (double)to_f32(qh[2 * c]) * x.x + (double)to_f32(qh[2 * c + 1]) * x.y;
+        }
+        score[j] = acc;
     }
     __syncthreads();
     int n = 0;
@@ -131,51 +136,78 @@ __global__ void __launch_bounds__(kThreads)
 decode_attend_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const int32_t* __restrict__ sel, int Tcap, int D, int block, int t, int topk,
                      float scale, float* __restrict__ part) {
-    __shared__ float wm[kThreads / 32], wl[kThreads / 32];
-    __shared__ float wo[kThreads / 32][128];
+    __shared__ float qs[128];
+    __shared__ float ps[128];             // scores, then e^{x - m}
+    __shared__ float red[kThreads / 32];
+    __shared__ float og[kThreads];        // [key group][d] partial sums of P V
     const int slot = blockIdx.x;
     const size_t bh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float* out = part + (bh * topk + slot) * (2 + D);
     const int j = sel[bh * topk + slot];
-    const int s_end = j < 0 ? 0 : min((j + 1) * block, t + 1);
-    constexpr int NW = kThreads / 32;
-    const int per = D / 32;  // columns per lane (2 or 4)
-    float qv[4], o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int e = 0; e < per; ++e) qv[e] = to_f32(q[bh * D + lane * per + e]);
-    float m = -INFINITY, l = 0.f;
-    for (int s = (j < 0 ? 0 : j * block) + warp; s < s_end; s += NW) {
-        const T* ks = k + (bh * Tcap + s) * D + lane * per;
-        const T* vs = v + (bh * Tcap + s) * D + lane * per;
-        float x = 0.f;
-        for (int e = 0; e < per; ++e) x = fmaf(qv[e], to_f32(ks[e]), x);
-        x = warp_sum(x) * scale;
-        const float mn = fmaxf(m, x);
-        const float a = expf(m - mn), p = expf(x - mn);  // m = -inf first: a = 0
-        l = l * a + p;
-        for (int e = 0; e < per; ++e) o[e] = o[e] * a + p * to_f32(vs[e]);
-        m = mn;
-    }
-    if (lane == 0) {
-        wm[warp] = m;
-        wl[warp] = l;
-    }
-    for (int e = 0; e < per; ++e) wo[warp][lane * per + e] = o[e];
+    const int s0 = j < 0 ? 0 : j * block;
+    const int nks = j < 0 ? 0 : min((j + 1) * block, t + 1) - s0;  // keys of this block <= t
+    for (int c = threadIdx.x; c < D; c += kThreads) qs[c] = to_f32(q[bh * D + c]);
     __syncthreads();
-    if (warp == 0) {  // merge the warps' partials
-        float M = -INFINITY;
-        for (int w = 0; w < NW; ++w) M = fmaxf(M, wm[w]);
-        float L = 0.f, O[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int w = 0; w < NW; ++w) {
-            const float a = wm[w] > -INFINITY ? expf(wm[w] - M) : 0.f;
-            L += a * wl[w];
-            for (int e = 0; e < per; ++e) O[e] += a * wo[w][lane * per + e];
+    // scores: thread per key, its row read in 16-byte pieces (independent loads)
+    float x = -INFINITY;
+    if (threadIdx.x < nks) {
+        const uint4* kr = reinterpret_cast<const uint4*>(k + (bh * Tcap + s0 + threadIdx.x) * D);
+        constexpr int E = 16 / sizeof(T);  // elements per 16-byte piece
+        float acc = 0.f;
+        for (int c = 0; c < D / E; ++c) {
+            const uint4 u = kr[c];
+            const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+            for (int z = 0; z < E; ++z) acc = fmaf(qs[c * E + z], to_f32(e[z]), acc);
         }
-        if (lane == 0) {
-            out[0] = M;
-            out[1] = L;
-        }
-        for (int e = 0; e < per; ++e) out[2 + lane * per + e] = O[e];
+        x = acc * scale;
+        ps[threadIdx.x] = x;
+    }
+    // m = max over the block's keys, then p = e^{x - m} and l = sum p
+    float mx = warp_max(x);
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    float m = red[0];
+    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+    __syncthreads();
+    float p = 0.f;
+    if (threadIdx.x < nks) {
+        p = expf(x - m);
+        ps[threadIdx.x] = p;
+    }
+    const float ls = warp_sum(p);
+    if (lane == 0) red[warp] = ls;
+    __syncthreads();
+    float l = 0.f;
+    for (int w = 0; w < kThreads / 32; ++w) l += red[w];
+    // o[d] = sum_s p_s v_s[d]: thread (g, d) over keys s = g, g + G, ... (coalesced in d)
+    const int G = kThreads / D;
+    const int d = threadIdx.x % D, g = threadIdx.x / D;
+    // the value loads are independent: unrolled so that many are in flight
+    const T* vcol = v + (bh * Tcap + s0) * D + d;
+    float a4[4] = {0.f, 0.f, 0.f, 0.f};
+    int s = g;
+#pragma unroll 4
+    for (; s + 3 * G < nks; s += 4 * G) {
+        const float x0 = to_f32(vcol[(size_t)s * D]), x1 = to_f32(vcol[(size_t)(s + G) * D]);
+        const float x2 = to_f32(vcol[(size_t)(s + 2 * G) * D]), x3 = to_f32(vcol[(size_t)(s + 3 * G) * D]);
+        a4[0] = fmaf(ps[s], x0, a4[0]);
+        a4[1] = fmaf(ps[s + G], x1, a4[1]);
+        a4[2] = fmaf(ps[s + 2 * G], x2, a4[2]);
+        a4[3] = fmaf(ps[s + 3 * G], x3, a4[3]);
+    }
+    for (; s < nks; s += G) a4[0] = fmaf(ps[s], to_f32(vcol[(size_t)s * D]), a4[0]);
+    og[g * D + d] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    __syncthreads();
+    if (threadIdx.x < D) {
+        float o = 0.f;
+        for (int gg = 0; gg < G; ++gg) o += og[gg * D + threadIdx.x];
+        out[2 + threadIdx.x] = o;
+    }
+    if (threadIdx.x == 0) {
+        out[0] = nks > 0 ? m : -INFINITY;
+        out[1] = l;
     }
 }
 

@@ -5,9 +5,9 @@
 //   sink(t)       = sum_{s <= t, s < block} exp(sigma q_t . k_s - lse_full(t)),
 //                   the full-softmax mass on block 0;
 //   mean_delta[h] = mean over t of delta(t),  mean_sink[h] = mean over t of sink(t).
-// Two launches: diag_sink_kernel (CUDA cores; block 0 of K and a 64-row slab of
-// Q staged transposed in shared memory, each warp register-tiles 8 rows x its
-// lane's 2 or 4 keys) and diag_head_kernel (one CTA per head, fixed-order
+// Two launches: diag_sink_kernel (CUDA cores; block 0 of K staged transposed
+// once per CTA, 64-row slabs of Q staged row-major, each warp register-tiles 8
+// rows x its lane's 2 or 4 keys) and diag_head_kernel (one CTA per head, fixed-order
 // float64 sums: bitwise repeatable).  The first pass reads Q once.
 #include "device_util.cuh"
 #include "ssa_internal.h"
@@ -21,70 +21,80 @@ constexpr int kRowsPerCta = 64;
 template <typename T, int KPL>  // KPL = keys of block 0 per lane (2 for block 64, 4 for 128)
 __global__ void __launch_bounds__(kThreads)
 diag_sink_kernel(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ lse,
-                 int Tn, int D, int nkeys, float scale, float* __restrict__ sink) {
+                 int Tn, int D, int nkeys, float scale, int slabs, float* __restrict__ sink) {
     extern __shared__ float sm[];
     constexpr int NK = 32 * KPL;                 // key slots (keys past nkeys are masked)
     constexpr int RW = kRowsPerCta / (kThreads / 32);  // rows per warp (8)
+    const int QS = D + 4;                        // row stride of the Q slab (16-byte aligned)
     float* kT = sm;                              // [D][NK]: lane reads its KPL keys at once
-    float* qT = sm + (size_t)D * NK;             // [D][kRowsPerCta]: a warp's rows are contiguous
+    float* qs = sm + (size_t)D * NK;             // [kRowsPerCta][D + 4], row-major
     const size_t bh = blockIdx.y;
-    const int r0 = blockIdx.x * kRowsPerCta;
     const T* kh = k + bh * (size_t)Tn * D;
-    // transposed staging, consecutive threads on consecutive shared words (no
-    // bank conflicts); the strided global reads hit the same lines repeatedly (L1)
+    // block 0 of K, transposed once per CTA (consecutive threads on consecutive shared
+    // words; the strided global reads hit the same lines repeatedly in L1)
     for (int e = threadIdx.x; e < NK * D; e += kThreads) {
         const int s = e % NK, c = e / NK;
         kT[c * NK + s] = s < nkeys ? to_f32(kh[(size_t)s * D + c]) : 0.f;
     }
-    for (int e = threadIdx.x; e < kRowsPerCta * D; e += kThreads) {
-        const int r = e % kRowsPerCta, c = e / kRowsPerCta;
-        const int t = r0 + r;
-        qT[c * kRowsPerCta + r] = t < Tn ? to_f32(q[(bh * (size_t)Tn + t) * D + c]) : 0.f;
-    }
-    __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // acc[r][j] = q_(row r of this warp) . k_(key KPL*lane + j)
-    float acc[RW][KPL];
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-#pragma unroll
-        for (int j = 0; j < KPL; ++j) acc[r][j] = 0.f;
-    const float* qw = qT + RW * warp;
-    for (int c = 0; c < D; ++c) {
-        const float4 qa = *reinterpret_cast<const float4*>(qw + c * kRowsPerCta);
-        const float4 qb = *reinterpret_cast<const float4*>(qw + c * kRowsPerCta + 4);
-        const float qv[RW] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-        float kv[KPL];
-        if constexpr (KPL == 2) {
-            const float2 x = *reinterpret_cast<const float2*>(kT + c * NK + 2 * lane);
-            kv[0] = x.x;
-            kv[1] = x.y;
-        } else {
-            const float4 x = *reinterpret_cast<const float4*>(kT + c * NK + 4 * lane);
-            kv[0] = x.x;
-            kv[1] = x.y;
-            kv[2] = x.z;
-            kv[3] = x.w;
+    for (int slab = 0; slab < slabs; ++slab) {
+        const int r0 = (blockIdx.x * slabs + slab) * kRowsPerCta;
+        if (r0 >= Tn) break;  // CTA-uniform
+        __syncthreads();  // previous slab's reads of qs are done (and kT is staged)
+        for (int e = threadIdx.x; e < kRowsPerCta * D; e += kThreads) {
+            const int r = e / D, c = e % D;
+            const int t = r0 + r;
+            qs[r * QS + c] = t < Tn ? to_f32(q[(bh * (size_t)Tn + t) * D + c]) : 0.f;
         }
+        __syncthreads();
+        // acc[r][j] = q_(row r of this warp) . k_(key KPL*lane + j)
+        float acc[RW][KPL];
 #pragma unroll
         for (int r = 0; r < RW; ++r)
 #pragma unroll
-            for (int j = 0; j < KPL; ++j) acc[r][j] = fmaf(qv[r], kv[j], acc[r][j]);
-    }
+            for (int j = 0; j < KPL; ++j) acc[r][j] = 0.f;
+        const float* qw = qs + (RW * warp) * QS;
+        for (int c = 0; c < D; c += 4) {
+            float kv[4][KPL];
 #pragma unroll
-    for (int r = 0; r < RW; ++r) {
-        const int t = r0 + RW * warp + r;
-        if (t >= Tn) break;  // warp-uniform
-        const size_t row = bh * (size_t)Tn + t;
-        const float l = lse[row];
-        float m = 0.f;
+            for (int u = 0; u < 4; ++u) {
+                if constexpr (KPL == 2) {
+                    const float2 x = *reinterpret_cast<const float2*>(kT + (c + u) * NK + 2 * lane);
+                    kv[u][0] = x.x;
+                    kv[u][1] = x.y;
+                } else {
+                    const float4 x = *reinterpret_cast<const float4*>(kT + (c + u) * NK + 4 * lane);
+                    kv[u][0] = x.x;
+                    kv[u][1] = x.y;
+                    kv[u][2] = x.z;
+                    kv[u][3] = x.w;
+                }
+            }
 #pragma unroll
-        for (int j = 0; j < KPL; ++j) {
-            const int s = KPL * lane + j;
-            if (s < nkeys && s <= t) m += expf(scale * acc[r][j] - l);
+            for (int r = 0; r < RW; ++r) {
+                const float4 q4 = *reinterpret_cast<const float4*>(qw + r * QS + c);  // broadcast
+                const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int j = 0; j < KPL; ++j) acc[r][j] = fmaf(qv[u], kv[u][j], acc[r][j]);
+            }
         }
-        m = warp_sum(m);
-        if (lane == 0) sink[row] = m;
+#pragma unroll
+        for (int r = 0; r < RW; ++r) {
+            const int t = r0 + RW * warp + r;
+            if (t >= Tn) break;  // warp-uniform
+            const size_t row = bh * (size_t)Tn + t;
+            const float l = lse[row];
+            float m = 0.f;
+#pragma unroll
+            for (int j = 0; j < KPL; ++j) {
+                const int s = KPL * lane + j;
+                if (s < nkeys && s <= t) m += expf(scale * acc[r][j] - l);
+            }
+            m = warp_sum(m);
+            if (lane == 0) sink[row] = m;
+        }
     }
 }
 
@@ -123,12 +133,18 @@ int launch_diagnostics(const ssa_params_t& p, const void* q, const void* k, cons
     const int BH = p.B * p.H;
     const int nkeys = p.block < p.T ? p.block : p.T;
     const int kpl = p.block > 64 ? 4 : 2;
-    const size_t smem = ((size_t)p.D * 32 * kpl + (size_t)p.D * kRowsPerCta) * sizeof(float);
-    const dim3 grid((unsigned)((p.T + kRowsPerCta - 1) / kRowsPerCta), (unsigned)BH);
+    const size_t smem = ((size_t)p.D * 32 * kpl + (size_t)(p.D + 4) * kRowsPerCta) * sizeof(float);
+    // enough CTAs to cover the SMs a few times; each loops over 64-row slabs
+    // with block 0 of K staged once
+    const int nslab = (p.T + kRowsPerCta - 1) / kRowsPerCta;
+    int per_head = (4 * 148 + BH - 1) / BH;
+    if (per_head > nslab) per_head = nslab;
+    const int slabs = (nslab + per_head - 1) / per_head;
+    const dim3 grid((unsigned)((nslab + slabs - 1) / slabs), (unsigned)BH);
     auto go = [&](auto kernel, auto qp, auto kp) -> int {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "diag: smem attribute: %s", cudaGetErrorString(e));
-        kernel<<<grid, kThreads, smem, s>>>(qp, kp, lse_full, p.T, p.D, nkeys, p.sm_scale, sink);
+        kernel<<<grid, kThreads, smem, s>>>(qp, kp, lse_full, p.T, p.D, nkeys, p.sm_scale, slabs, sink);
         return check_launch("diag_sink_kernel");
     };
     int st;
