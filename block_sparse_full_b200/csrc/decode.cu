@@ -12,12 +12,16 @@
 // Launches (CUDA cores: one query per head is matrix-vector work, bound by
 // the key/value bytes it reads):
 //   decode_pool_kernel     Kbar_j = mean of block j's keys (float64, exact)
-//   decode_select_kernel   one CTA per head: scores (thread per block),
-//                          top-k by rounds of a CTA-wide argmax
+//   decode_select_kernel   one CTA per head: scores (warp per block, lanes
+//                          over d), then one warp fills the free slots by
+//                          warp-argmax rounds and writes the ascending list
 //   decode_attend_kernel   one CTA per (head, selected block): scores with a
-//                          thread per key, softmax statistics CTA-wide, then
-//                          P V with threads over (d, key group)
+//                          warp per group of keys (lanes over d), softmax
+//                          statistics CTA-wide, then P V with threads over
+//                          (d, key group)
 //   decode_combine_kernel  one warp per head merges the per-block partials
+#include <type_traits>
+
 #include "device_util.cuh"
 #include "ssa_internal.h"
 
@@ -41,105 +45,128 @@ decode_pool_kernel(const T* __restrict__ k, int Tcap, int D, int block, int j0,
     }
 }
 
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
-decode_select_kernel(const T* __restrict__ q, const double* __restrict__ kbar, int nb, int D,
-                     int i, int topk, bool force_sink, int32_t* __restrict__ sel,
+decode_select_kernel(const T* __restrict__ q, const double* __restrict__ kbar, int nb, int i,
+                     int topk, bool force_sink, int32_t* __restrict__ sel,
                      int32_t* __restrict__ idx_out) {
-    extern __shared__ double score[];  // [i]
-    __shared__ double best_s[kThreads / 32];
-    __shared__ int best_j[kThreads / 32];
-    __shared__ int chosen[kMaxTopk];
+    constexpr int M = D / 32;  // query columns per lane
+    constexpr int U = 4;       // key blocks in flight per warp
+    extern __shared__ double score[];  // [max(i, 1)], then the set bitmask [i / 32 + 1]
+    uint32_t* bits = reinterpret_cast<uint32_t*>(score + (i > 0 ? i : 1));
     const size_t bh = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const T* qh = q + bh * D;
-    // scores of the completed blocks: thread per block, independent loads of its
-    // float64 pooled key (one memory latency for the whole scan)
-    for (int j = threadIdx.x; j < i; j += kThreads) {
-        const double2* kb = reinterpret_cast<const double2*>(kbar + (bh * nb + j) * D);
-        double acc = 0.0;
-#pragma unroll 8
-        for (int c = 0; c < D / 2; ++c) {
-            const double2 x = kb[c];
-            acc += (double)to_f32(qh[2 * c]) * x.x + (double)to_f32(qh[2 * c + 1]) * x.y;
-        }
-        score[j] = acc;
-    }
-    __syncthreads();
-    int n = 0;
-    if (threadIdx.x == 0) {
-        chosen[n++] = i;
-        if (force_sink && i > 0) {
-            chosen[n++] = 0;
-            score[0] = -INFINITY;  // taken
-        }
-    }
-    __syncthreads();
-    n = (force_sink && i > 0) ? 2 : 1;
-    const int want = topk < i + 1 ? topk : i + 1;  // fewer candidates than places: take all
-    for (; n < want; ++n) {
-        // CTA-wide argmax by (score desc, index asc); taken blocks hold -inf
-        double bs = -INFINITY;
-        int bj = 1 << 30;
-        for (int j = threadIdx.x; j < i; j += kThreads) {
-            const double v = score[j];
-            if (v > bs || (v == bs && j < bj)) {
-                bs = v;
-                bj = j;
-            }
+    const int words = (i >> 5) + 1;  // bits 0 .. i
+    double qr[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) qr[m] = (double)to_f32(q[bh * D + lane + 32 * m]);
+    for (int w = threadIdx.x; w < words; w += kThreads) bits[w] = 0u;
+    // scores of the completed blocks: warp per block, lane l owns columns
+    // l, l + 32, ... (coalesced rows of the float64 pooled keys), U blocks'
+    // loads in flight per warp, fixed butterfly sum
+    const double* kb = kbar + bh * (size_t)nb * D;
+    for (int j0 = warp * U; j0 < i; j0 += (kThreads / 32) * U) {
+        double a[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const double* kr = kb + (size_t)min(j0 + u, i - 1) * D + lane;  // past the end: unused
+            double acc = 0.0;
+#pragma unroll
+            for (int m = 0; m < M; ++m) acc = fma(qr[m], kr[32 * m], acc);
+            a[u] = acc;
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double os = __shfl_xor_sync(0xffffffffu, bs, o);
-            const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-            if (os > bs || (os == bs && oj < bj)) {
-                bs = os;
-                bj = oj;
-            }
-        }
+        for (int u = 0; u < U; ++u) a[u] = warp_sum(a[u]);
         if (lane == 0) {
-            best_s[warp] = bs;
-            best_j[warp] = bj;
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (j0 + u < i) score[j0 + u] = a[u];
         }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            double s = best_s[0];
-            int jb = best_j[0];
-            for (int w = 1; w < kThreads / 32; ++w)
-                if (best_s[w] > s || (best_s[w] == s && best_j[w] < jb)) {
-                    s = best_s[w];
-                    jb = best_j[w];
-                }
-            chosen[n] = jb;
-            score[jb] = -INFINITY;
-        }
-        __syncthreads();
     }
-    if (threadIdx.x == 0) {  // ascending, -1 padded
-        for (int a = 1; a < want; ++a)
-            for (int b = a; b > 0 && chosen[b - 1] > chosen[b]; --b) {
-                const int x = chosen[b];
-                chosen[b] = chosen[b - 1];
-                chosen[b - 1] = x;
-            }
-        for (int a = 0; a < topk; ++a) {
-            const int v = a < want ? chosen[a] : -1;
-            sel[bh * topk + a] = v;
-            if (idx_out) idx_out[bh * topk + a] = v;
+    __syncthreads();
+    if (warp != 0) return;
+    // one warp: forced blocks, the free slots by warp-argmax rounds, then the
+    // ascending index list (-1 padded) from the bitmask by popcount prefix
+    const bool sink = force_sink && i > 0;
+    const int want = topk < i + 1 ? topk : i + 1;  // fewer candidates than places: take all
+    const int first = sink ? 1 : 0;                // candidates are first .. i-1
+    const int r = want - (sink ? 2 : 1);           // free slots (>= 0: a sink needs topk >= 2)
+    if (lane == 0) {
+        bits[i >> 5] |= 1u << (i & 31);
+        if (sink) bits[0] |= 1u;
+    }
+    __syncwarp();
+    if (i - first <= r) {
+        for (int j = first + lane; j < i; j += 32) atomicOr(&bits[j >> 5], 1u << (j & 31));
+    } else {
+        warp_topk_rounds(score, first, i, r, bits, lane);
+    }
+    __syncwarp();
+    int32_t* srow = sel + bh * topk;
+    int32_t* irow = idx_out ? idx_out + bh * topk : nullptr;
+    int base = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+        const int w = w0 + lane;
+        const uint32_t wv = w < words ? bits[w] : 0u;
+        const int c = __popc(wv);
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
         }
+        int pos = base + incl - c;
+        for (uint32_t b = wv; b != 0u; b &= b - 1u, ++pos) {
+            if (pos < topk) {  // NaN scores: stay in bounds
+                const int v = w * 32 + __ffs(b) - 1;
+                srow[pos] = v;
+                if (irow) irow[pos] = v;
+            }
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    for (int p = base + lane; p < topk; p += 32) {
+        srow[p] = -1;
+        if (irow) irow[p] = -1;
+    }
+}
+
+// E consecutive elements of a row, as float, in one vector load (E * sizeof(T)
+// is 4, 8 or 16 bytes and the address a multiple of it)
+template <typename T, int E>
+__device__ __forceinline__ void load_row_piece(const T* p, float (&x)[E]) {
+    constexpr int B = E * (int)sizeof(T);
+    if constexpr (B == 16) {
+        const uint4 u = *reinterpret_cast<const uint4*>(p);
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int z = 0; z < E; ++z) x[z] = to_f32(e[z]);
+    } else if constexpr (B == 8) {
+        const uint2 u = *reinterpret_cast<const uint2*>(p);
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int z = 0; z < E; ++z) x[z] = to_f32(e[z]);
+    } else {
+        static_assert(B == 4, "row piece of 4, 8 or 16 bytes");
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(p);
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int z = 0; z < E; ++z) x[z] = to_f32(e[z]);
     }
 }
 
 // partial of one (head, selected block): m (max of x), l (sum e^{x-m}), o[D]
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 decode_attend_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                     const int32_t* __restrict__ sel, int Tcap, int D, int block, int t, int topk,
+                     const int32_t* __restrict__ sel, int Tcap, int block, int t, int topk,
                      float scale, float* __restrict__ part) {
-    __shared__ float qs[128];
-    __shared__ float ps[128];             // scores, then e^{x - m}
-    __shared__ float red[kThreads / 32];
-    __shared__ float og[kThreads];        // [key group][d] partial sums of P V
+    constexpr int E = D / 32;            // columns per lane
+    constexpr int NW = kThreads / 32;    // warps
+    constexpr int KPW = 128 / NW;        // keys per warp (block <= 128)
+    __shared__ float ps[128];            // scores, then e^{x - m}
+    __shared__ float red[NW];
+    __shared__ float og[kThreads];       // [key group][d] partial sums of P V
     const int slot = blockIdx.x;
     const size_t bh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -147,29 +174,36 @@ decode_attend_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     const int j = sel[bh * topk + slot];
     const int s0 = j < 0 ? 0 : j * block;
     const int nks = j < 0 ? 0 : min((j + 1) * block, t + 1) - s0;  // keys of this block <= t
-    for (int c = threadIdx.x; c < D; c += kThreads) qs[c] = to_f32(q[bh * D + c]);
-    __syncthreads();
-    // scores: thread per key, its row read in 16-byte pieces (independent loads)
-    float x = -INFINITY;
-    if (threadIdx.x < nks) {
-        const uint4* kr = reinterpret_cast<const uint4*>(k + (bh * Tcap + s0 + threadIdx.x) * D);
-        constexpr int E = 16 / sizeof(T);  // elements per 16-byte piece
-        float acc = 0.f;
-        for (int c = 0; c < D / E; ++c) {
-            const uint4 u = kr[c];
-            const T* e = reinterpret_cast<const T*>(&u);
+    // scores: warp w takes keys w, w + NW, ...; lane l reads columns
+    // [E l, E l + E) of each key row (coalesced), all the warp's rows in flight
+    float qv[E];
+    load_row_piece<T, E>(q + bh * D + E * lane, qv);
+    float acc[KPW];
 #pragma unroll
-            for (int z = 0; z < E; ++z) acc = fmaf(qs[c * E + z], to_f32(e[z]), acc);
+    for (int kk = 0; kk < KPW; ++kk) {
+        const int s = warp + NW * kk;
+        acc[kk] = 0.f;
+        if (s < nks) {
+            float x[E];
+            load_row_piece<T, E>(k + (bh * Tcap + s0 + s) * D + E * lane, x);
+#pragma unroll
+            for (int z = 0; z < E; ++z) acc[kk] = fmaf(qv[z], x[z], acc[kk]);
         }
-        x = acc * scale;
-        ps[threadIdx.x] = x;
     }
+#pragma unroll
+    for (int kk = 0; kk < KPW; ++kk) {
+        const int s = warp + NW * kk;
+        const float dot = warp_sum(acc[kk]);
+        if (lane == 0 && s < nks) ps[s] = dot * scale;
+    }
+    __syncthreads();
     // m = max over the block's keys, then p = e^{x - m} and l = sum p
+    const float x = threadIdx.x < nks ? ps[threadIdx.x] : -INFINITY;
     float mx = warp_max(x);
     if (lane == 0) red[warp] = mx;
     __syncthreads();
     float m = red[0];
-    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+    for (int w = 1; w < NW; ++w) m = fmaxf(m, red[w]);
     __syncthreads();
     float p = 0.f;
     if (threadIdx.x < nks) {
@@ -180,7 +214,7 @@ decode_attend_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     if (lane == 0) red[warp] = ls;
     __syncthreads();
     float l = 0.f;
-    for (int w = 0; w < kThreads / 32; ++w) l += red[w];
+    for (int w = 0; w < NW; ++w) l += red[w];
     // o[d] = sum_s p_s v_s[d]: thread (g, d) over keys s = g, g + G, ... (coalesced in d)
     const int G = kThreads / D;
     const int d = threadIdx.x % D, g = threadIdx.x / D;
@@ -211,26 +245,30 @@ decode_attend_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     }
 }
 
+// one warp per head: the partials' weights e^{m_a - M} are formed once
 template <typename T>
 __global__ void __launch_bounds__(32)
 decode_combine_kernel(const float* __restrict__ part, int D, int topk, T* __restrict__ h,
                       float* __restrict__ lse) {
+    __shared__ float wgt[kMaxTopk];
     const size_t bh = blockIdx.x;
     const int lane = threadIdx.x;
     const float* p = part + bh * topk * (2 + D);
     float M = -INFINITY;
-    for (int a = 0; a < topk; ++a) M = fmaxf(M, p[a * (2 + D)]);
+    for (int a = lane; a < topk; a += 32) M = fmaxf(M, p[a * (2 + D)]);
+    M = warp_max(M);
     float L = 0.f;
-    for (int a = 0; a < topk; ++a) {
+    for (int a = lane; a < topk; a += 32) {
         const float ma = p[a * (2 + D)];
-        if (ma > -INFINITY) L += expf(ma - M) * p[a * (2 + D) + 1];
+        const float w = ma > -INFINITY ? expf(ma - M) : 0.f;
+        wgt[a] = w;
+        L += w * p[a * (2 + D) + 1];
     }
+    L = warp_sum(L);
+    __syncwarp();
     for (int c = lane; c < D; c += 32) {
         float acc = 0.f;
-        for (int a = 0; a < topk; ++a) {
-            const float ma = p[a * (2 + D)];
-            if (ma > -INFINITY) acc += expf(ma - M) * p[a * (2 + D) + 2 + c];
-        }
+        for (int a = 0; a < topk; ++a) acc = fmaf(wgt[a], p[a * (2 + D) + 2 + c], acc);
         h[bh * D + c] = from_f32<T>(acc / L);
     }
     if (lane == 0) lse[bh] = M + logf(L);
@@ -265,28 +303,33 @@ int launch_decode_step(const ssa_params_t& p, int t, const void* q, const void* 
     int32_t* sel = static_cast<int32_t*>(ws);
     float* part = reinterpret_cast<float*>(static_cast<char*>(ws) +
                                            align_up((size_t)BH * p.topk * 4, 256));
-    const size_t smem = (size_t)(i > 0 ? i : 1) * sizeof(double);
+    const size_t smem = (size_t)(i > 0 ? i : 1) * sizeof(double) + (size_t)((i >> 5) + 1) * 4;
     const bool sink = (p.flags & SSA_FLAG_FORCE_SINK) != 0;
     const int nb = num_blocks(p);
-    auto run = [&](auto tag) -> int {
+    auto run = [&](auto tag, auto dtag) -> int {
         using T = decltype(tag);
-        auto sk = decode_select_kernel<T>;
+        constexpr int D = decltype(dtag)::value;
+        auto sk = decode_select_kernel<T, D>;
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "decode: smem attribute: %s", cudaGetErrorString(e));
         }
-        sk<<<BH, kThreads, smem, s>>>(static_cast<const T*>(q), kbar, nb, p.D, i, p.topk, sink, sel, idx);
+        sk<<<BH, kThreads, smem, s>>>(static_cast<const T*>(q), kbar, nb, i, p.topk, sink, sel, idx);
         int st = check_launch("decode_select_kernel");
         if (st != SSA_OK) return st;
-        decode_attend_kernel<T><<<dim3((unsigned)p.topk, (unsigned)BH), kThreads, 0, s>>>(
+        decode_attend_kernel<T, D><<<dim3((unsigned)p.topk, (unsigned)BH), kThreads, 0, s>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), sel, p.T,
-            p.D, p.block, t, p.topk, p.sm_scale, part);
+            p.block, t, p.topk, p.sm_scale, part);
         st = check_launch("decode_attend_kernel");
         if (st != SSA_OK) return st;
         decode_combine_kernel<T><<<BH, 32, 0, s>>>(part, p.D, p.topk, static_cast<T*>(h), lse);
         return check_launch("decode_combine_kernel");
     };
-    return p.dtype == SSA_BF16 ? run(__nv_bfloat16{}) : run(float{});
+    using D64 = std::integral_constant<int, 64>;
+    using D128 = std::integral_constant<int, 128>;
+    if (p.dtype == SSA_BF16)
+        return p.D == 64 ? run(__nv_bfloat16{}, D64{}) : run(__nv_bfloat16{}, D128{});
+    return p.D == 64 ? run(float{}, D64{}) : run(float{}, D128{});
 }
 
 }  // namespace ssa

@@ -509,9 +509,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_arrive(BAR(B_PREADY + b));
             ++jj;
         }
-        if (ok)
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(BAR(B_PVDONE), (jj - 1) & 1, abort_flag, status, lim));
+        // Every MMA (the last PV included) has completed once B_DRAIN has.  A
+        // parity wait on B_PVDONE for the last tile is not enough: the softmax
+        // only knows that the PV two tiles back has landed, and a barrier one
+        // phase behind reports the wanted parity as complete.
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_DRAIN), 0, abort_flag, status, lim));
         // both warpgroups take the same decision and the same barriers below
         ok = !wg_vote(!ok || *abort_flag);
         float* xl = xch;  // [wg][sel|uns][row] reuses the max exchange area
