@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from block_sparse_full_b200 import ssa
-from block_sparse_full_b200.inputs import WORKLOADS, make_inputs
+from block_sparse_full_b200.inputs import WORKLOADS, Workload, make_inputs
 from oracle import ssa_oracle as O
 
 from gpu_parity_util import DEV, TOL, log, params
@@ -62,3 +62,16 @@ def test_decode_force_sink_and_full_budget():
 def test_decode_T65536_sink_last_token():
     w = WORKLOADS["bf16_T65536_H8_sink"]
     _decode(w, [w.T - 1, w.T // 2 + 17], heads=[1, 6])
+
+
+def test_decode_f32_d64_workload():
+    w = WORKLOADS["f32_T1024_d64"]
+    _decode(w, [0, 63, 64, 500, w.T - 1])
+
+
+def test_decode_more_than_1024_completed_blocks():
+    # 1100 blocks of 64: the selection bitmask spans 35 words, so the ascending
+    # list is assembled over more than one warp-wide chunk of mask words
+    w = Workload("bf16_T70400_d64_decode", B=1, H=1, T=64 * 1100, D=64, block=64, topk=12,
+                 dtype="bf16", plant="hot", seed=41)
+    _decode(w, [w.T - 1, 64 * 1030 + 3])

@@ -26,7 +26,9 @@ CASES = [
     ("bf16", 64, 128, 40, 12, True),
     ("f32", 128, 128, 45, 7, False),
     ("f32", 64, 64, 130, 64, True),
+    ("f32", 64, 128, 33, 5, False),
     ("bf16", 64, 64, 1100, 16, False),   # rows longer than 1024 blocks: the per-row kernel
+    ("bf16", 128, 64, 1030, 7, True),
     ("bf16", 128, 64, 1024, 9, True),    # the longest rows of the 8-row kernel
 ]
 
