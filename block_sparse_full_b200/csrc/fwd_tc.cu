@@ -7,7 +7,8 @@
 // subset only).
 //
 // CTA = (query tile of 128 rows, batch*head), 256 threads:
-//   warp 0      TMA producer: Q once, then K_j and V_j into 2-stage rings
+//   warps 0, 2  TMA producers: Q once and K_j (warp 0), V_j (warp 2), into
+//               2-stage rings
 //   warp 1      TMEM owner and MMA issuer (one thread):
 //                 S_j = Q K_j^T          (tcgen05 SS, into S buffer j%2)
 //                 O_sel/O_uns += P_j V_j  (tcgen05 TS, P read from TMEM)
@@ -46,7 +47,7 @@ using namespace tc;
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int HD = 128;  // largest head dim (the shared-memory layout is sized for it)
-constexpr int kThreads = 384;  // warps 0-1 roles, 2-3 idle, 4-11 two softmax warpgroups
+constexpr int kThreads = 384;  // warps 0-2 roles, 3 idle, 4-11 two softmax warpgroups
 constexpr int kSoftmax = 256;
 constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB ring slot (half used at d = 64)
 constexpr uint32_t HALF_BYTES = 128 * 128;    // [128 rows x 64 cols] bf16 box, 16 KB
@@ -74,7 +75,10 @@ static_assert(B_COUNT <= NBAR, "barrier area");
 
 constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_OSEL = 256, TM_OUNS = 384;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr int kPolyLane = 3;  // pairs c with c % 4 == 3 use the FMA-pipe exponential
+// pairs c with c % 8 in {1, 4, 6} (three eighths) use the FMA-pipe exponential
+__device__ __forceinline__ bool poly_pair(int c) {
+    return (c & 7) == 1 || (c & 7) == 4 || (c & 7) == 6;
+}
 constexpr float kLn2 = 0.693147180559945309f;
 
 __device__ unsigned int g_fwd_tc_status;
@@ -194,52 +198,48 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // Roles 0 and 1 run their loops with the whole warp (warp-uniform address and
     // descriptor arithmetic); one elected lane issues each TMA / tcgen05 op.
     const unsigned FULL = 0xffffffffu;
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+    if (warp == 0 || warp == 2) {
+        // ------------------------------------------------ TMA producers
+        // warp 0: Q once, then the K ring; warp 2: the V ring.  Separate
+        // producers keep a K load from queueing behind a V slot that waits
+        // for the other warpgroup's PV product.
+        const bool is_k = warp == 0;
+        const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+        const int FULLB = is_k ? B_KFULL : B_VFULL, EMPTYB = is_k ? B_KEMPTY : B_VEMPTY;
+        const uint32_t ring = base + (is_k ? OFF_K : OFF_V);
         if (elect_one()) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_k);
-            prefetch_tmap(&tm_v);
-            mbar_expect_tx(BAR(B_QFULL), kTileBytes);
+            prefetch_tmap(tm);
+            if (is_k) {
+                prefetch_tmap(&tm_q);
+                mbar_expect_tx(BAR(B_QFULL), kTileBytes);
 #pragma unroll
-            for (int x = 0; x < D / 64; ++x)
-                tma_load_3d(base + OFF_Q + x * HALF_BYTES, &tm_q, BAR(B_QFULL), 64 * x, t0, bh);
+                for (int x = 0; x < D / 64; ++x)
+                    tma_load_3d(base + OFF_Q + x * HALF_BYTES, &tm_q, BAR(B_QFULL), 64 * x, t0, bh);
+            }
         }
         __syncwarp();
-        int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
+        int issued[2] = {-1, -1};
         for (int j = 0, jj = 0; j < ntk; ++j) {
             if (!tile_used(j)) continue;
             const int s = jj & 1;  // ring slot of the jj-th processed tile
             const uint32_t ph = ((jj >> 1) + 1) & 1;
-            const uint32_t kdst = base + OFF_K + s * TILE_BYTES;
-            const uint32_t vdst = base + OFF_V + s * TILE_BYTES;
-            if (jj >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_KEMPTY + s), ph, abort_flag, status, lim)))
+            const uint32_t dst = ring + s * TILE_BYTES;
+            if (jj >= 2 && !__all_sync(FULL, mbar_wait(BAR(EMPTYB + s), ph, abort_flag, status, lim)))
                 break;
             if (elect_one()) {
-                mbar_expect_tx(BAR(B_KFULL + s), kTileBytes);
+                mbar_expect_tx(BAR(FULLB + s), kTileBytes);
 #pragma unroll
                 for (int x = 0; x < D / 64; ++x)
-                    tma_load_3d(kdst + x * HALF_BYTES, &tm_k, BAR(B_KFULL + s), 64 * x, j * BN, bh);
+                    tma_load_3d(dst + x * HALF_BYTES, tm, BAR(FULLB + s), 64 * x, j * BN, bh);
             }
             __syncwarp();
-            issued_k[s] = jj;
-            if (jj >= 2 && !__all_sync(FULL, mbar_wait(BAR(B_VEMPTY + s), ph, abort_flag, status, lim)))
-                break;
-            if (elect_one()) {
-                mbar_expect_tx(BAR(B_VFULL + s), kTileBytes);
-#pragma unroll
-                for (int x = 0; x < D / 64; ++x)
-                    tma_load_3d(vdst + x * HALF_BYTES, &tm_v, BAR(B_VFULL + s), 64 * x, j * BN, bh);
-            }
-            __syncwarp();
-            issued_v[s] = jj;
+            if (s == 0) issued[0] = jj;
+            else issued[1] = jj;
             ++jj;
         }
         if (*abort_flag) {  // let copies in flight land before the CTA exits
-            for (int s = 0; s < 2; ++s) {
-                if (issued_k[s] >= 0) wait_drain(BAR(B_KFULL + s), (issued_k[s] >> 1) & 1, kDrainLimitNs);
-                if (issued_v[s] >= 0) wait_drain(BAR(B_VFULL + s), (issued_v[s] >> 1) & 1, kDrainLimitNs);
-            }
+            if (issued[0] >= 0) wait_drain(BAR(FULLB), (issued[0] >> 1) & 1, kDrainLimitNs);
+            if (issued[1] >= 0) wait_drain(BAR(FULLB + 1), (issued[1] >> 1) & 1, kDrainLimitNs);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -451,7 +451,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // attended, contribute P = 0 (no exponentials)
             const bool zero_p = kSparse && (!row_sel || !(m2 > -INFINITY));
             // p = 2^(s*sigma*log2e - m), two columns at a time (packed f32x2).  Off
-            // the diagonal a quarter of the pairs take the FMA-pipe exponential so
+            // the diagonal three eighths of the pairs take the FMA-pipe exponential so
             // that the MUFU unit is not the limit; on the diagonal every pair uses
             // the MUFU, whose 2^-inf = 0 keeps masked keys exact.
             const f32x2 sl2x2 = mk2(sl2, sl2), nm2 = mk2(negm, negm);
@@ -474,7 +474,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 for (int c = 0; c < 32; ++c) {
                     const f32x2 x2 = fma2(mk2(s[2 * c], s[2 * c + 1]), sl2x2, nm2);
                     float p0, p1;
-                    if ((c & 3) == kPolyLane) {
+                    if (poly_pair(c)) {
                         un2(exp2_poly2(x2), p0, p1);
                     } else {
                         float x0, x1;

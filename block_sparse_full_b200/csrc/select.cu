@@ -32,8 +32,8 @@ constexpr int kMaxBlocksPerRow = 4096;  // n = T / block limit (score row in sme
 // consecutive units: every thread first issues all its 16-byte loads (V
 // consecutive columns of rows g, g + G, ... of each unit; a warp covers
 // whole rows, so they coalesce), then the units are reduced one at a time
-// through shared memory in a fixed order.  Each thread keeps at most 16
-// loads in flight; the grid is about one wave for the usual sizes.  The
+// through shared memory in a fixed order.  Each thread keeps 8 to 16 loads
+// in flight.  The
 // base pointers are 16-byte aligned (host-checked).
 template <typename T, int D, int BLOCK>
 struct PoolShape {
@@ -41,7 +41,9 @@ struct PoolShape {
     static constexpr int TPR = D / V;               // threads per row
     static constexpr int G = kPoolThreads / TPR;    // row groups
     static constexpr int PER = BLOCK / G;           // rows per thread per unit
-    static constexpr int U = PER >= 16 ? 1 : 16 / PER;
+    // units per CTA: 8 loads in flight per thread for short rows (more CTAs
+    // per SM), 16 for long ones
+    static constexpr int U = PER >= 16 ? 1 : (PER >= 8 ? 16 / PER : 8 / PER);
     static_assert(BLOCK % G == 0, "block rows must split evenly over row groups");
 };
 
@@ -116,7 +118,8 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
                   int32_t* __restrict__ cnt, uint32_t* __restrict__ mask) {
     constexpr int M = D / 32;
     constexpr int R = kRowsPerCta;
-    constexpr int KPW = 4;  // keys per warp per group
+    constexpr int KPW = 32 / R;                   // keys per warp per group
+    constexpr int GROUP = (kSelThreads / 32) * KPW;  // keys per group
     static_assert(KPW * R == 32, "one partial per lane after the transpose-reduce");
     extern __shared__ double smem[];
     double* sc = smem;                                                      // [R][n]
@@ -150,8 +153,8 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
     if (kend > 0) {
         double kv[KPW][M], kn[KPW][M];
         load_group(0, kv);
-        for (int j0 = 0; j0 < kend; j0 += 32) {
-            if (j0 + 32 < kend) load_group(j0 + 32, kn);
+        for (int j0 = 0; j0 < kend; j0 += GROUP) {
+            if (j0 + GROUP < kend) load_group(j0 + GROUP, kn);
             double v[32];
 #pragma unroll
             for (int kk = 0; kk < KPW; ++kk)
@@ -186,6 +189,7 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
     }
     __syncthreads();  // all rows' scores and cleared bits visible
 
+    if (warp >= R) return;
     const int i = i0 + warp;
     if (i >= n) return;
     const size_t row = bh * n + i;
