@@ -102,6 +102,16 @@ def ds_blocks_per_bh(T):
     return ntk * (T // 64) - ntk * (ntk - 1)
 
 
+def data_description(w):
+    """What the synthetic inputs of workload ``w`` are, for the JSON line."""
+    base = "synthetic (seeded N(0,1)" + ("/sqrt(d)" if w.scale_data else "")
+    if w.plant == "hot":
+        return base + f", {w.n_hot} planted hot key blocks per head)"
+    if w.plant == "sink":
+        return base + ", a planted heavy sink in key block 0)"
+    return base + ")"
+
+
 def source_sha(*names):
     h = hashlib.sha256()
     for n in names:
@@ -110,9 +120,10 @@ def source_sha(*names):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_key):
-    """DRAM bytes per launch recorded from an ncu capture of this kernel,
-    or None when no capture exists or the kernel source changed since."""
+def ncu_traffic(kernel_key, workload):
+    """DRAM bytes per launch recorded from an ncu capture of this kernel on
+    this workload, or None when no such capture exists or the kernel source
+    changed since."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
@@ -120,6 +131,8 @@ def ncu_traffic(kernel_key):
         table = json.load(f)
     e = table.get(kernel_key)
     if not e or e.get("source_sha") != source_sha(*e["sources"]):
+        return None
+    if e.get("workload", "").split(" ")[0] != workload:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -371,7 +384,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
         kernels["bwd_dq_gemm_kernel"]["hbm_bytes"] = dq_bytes
         dom = max(kfl, key=lambda k: kms[k])
         roof = {"kernel": dom, "bound": "tensor", "peak": sustained, "unit": "TFLOP/s",
-                "peak_kind": f"{peak_src} bf16 dense, sustained", "traffic": ncu_traffic(dom)}
+                "peak_kind": f"{peak_src} bf16 dense, sustained", "traffic": ncu_traffic(dom, w.name)}
         flops, dom_ms = kfl[dom], kms[dom]
     else:
         dom = max(("fwd", "bwd"), key=lambda n: avg[n])
@@ -379,7 +392,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
         fp32 = NUM_SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         roof = {"kernel": f"{dom}_simt", "bound": "alu", "peak": round(fp32, 1),
                 "unit": "TFLOP/s", "peak_kind": "fp32 FMA: 148 SMs x 128 lanes x 2 x max SM clock",
-                "traffic": ncu_traffic(f"{dom}_simt")}
+                "traffic": ncu_traffic(f"{dom}_simt", w.name)}
         dom_ms = avg[dom]
     achieved = flops / (dom_ms * 1e-3) / 1e12
     roof["achieved"] = round(achieved, 2)
@@ -433,8 +446,8 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1)/sqrt(d) with planted hot key blocks)",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": data_description(w),
         "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "block": w.block,
                    "topk": w.topk, "global_batch": w.B * world, "seq_len": w.T,
                    "parallelism": f"replicas x{world} (independent batch*head units)",
