@@ -37,3 +37,30 @@ def test_two_rank_max_and_aggregate():
     # each rank did its own 1e12-FLOP step; the job's rate uses the slowest rank
     assert bench.whole_job_tflops(1e12, world, 5.0) == pytest.approx(400.0)
     assert bench.whole_job_tflops(1e12, 1, 5.0) == pytest.approx(200.0)
+
+
+def test_json_labels_follow_the_workload():
+    from block_sparse_full_b200.inputs import WORKLOADS
+    f32 = WORKLOADS["f32_T1024_d64"]
+    assert f32.dtype == "f32"
+    assert "planted" not in bench.data_description(f32)
+    assert "/sqrt(d)" not in bench.data_description(f32)  # config 1 draws plain N(0,1)
+    assert "hot key blocks" in bench.data_description(WORKLOADS["bf16_T8192_H16_hot"])
+    assert "sink" in bench.data_description(WORKLOADS["bf16_T65536_H8_sink"])
+    assert "planted" not in bench.data_description(WORKLOADS["bf16_B4_H32_T4096_train"])
+
+
+def test_ncu_traffic_only_for_the_captured_workload_and_source(tmp_path, monkeypatch):
+    import json
+    table = {"k": {"sources": ["fwd_tc.cu"], "source_sha": bench.source_sha("fwd_tc.cu"),
+                   "dram_bytes_per_launch": 123, "workload": "bf16_T8192_H16_hot (B1 H16 ...)"},
+             "stale": {"sources": ["fwd_tc.cu"], "source_sha": "0" * 16,
+                       "dram_bytes_per_launch": 456, "workload": "bf16_T8192_H16_hot"}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "ncu_traffic.json").write_text(json.dumps(table))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "source_sha", lambda *n: table["k"]["source_sha"])
+    assert bench.ncu_traffic("k", "bf16_T8192_H16_hot") == 123
+    assert bench.ncu_traffic("k", "bf16_T16384_H16_sweep") is None  # another workload
+    assert bench.ncu_traffic("stale", "bf16_T8192_H16_hot") is None  # source changed since
+    assert bench.ncu_traffic("missing", "bf16_T8192_H16_hot") is None
