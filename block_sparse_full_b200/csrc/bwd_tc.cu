@@ -21,16 +21,21 @@
 //   bwd_tc_pre_kernel   one warp per row: G_f, G_s' rounded to bf16, D_f and
 //                       D_s' from the rounded values, lse_full*log2(e)
 //                       (the three scalars stored negated).
-//   bwd_dkdv_tc_kernel  CTA = 128 keys; steps of 64 queries.  Per step:
-//                       S^T = K Q^T, dP_f^T = V G_f^T, dP_s^T = V G_s'^T
-//                       (tcgen05 SS, N = 64), the compute warpgroups form
-//                       P_f^T (bf16, back to TMEM) and dS^T (bf16, to a
-//                       swizzled shared-memory tile), then
-//                       dV += P_f^T G_f + P_s^T G_s' (TS) and dK += dS^T Q (SS).
-//                       TMEM: dV | dK | S^T x2 | dP_f^T | dP_s^T = 512 cols.
-//   bwd_dq_tc_kernel    CTA = 128 queries; steps of 64 keys: S = Q K^T,
-//                       dP_f = G_f V^T, dP_s = G_s' V^T, dS, dQ += dS K.
-//                       TMEM: dQ | S x2 | (dP_f, dP_s) x2 = 512 cols.
+//   bwd_dkdv_tc_kernel  CTA = 128 keys of one head; steps of 64 queries.
+//                       K and V are copied into TMEM once; per step
+//                       S^T = K Q^T and dP_f^T = V G_f^T (TS, N = 64), and
+//                       dP_s^T = V G_s'^T on steps the sparse stream
+//                       touches.  The compute warpgroups form P_f^T (bf16,
+//                       back into TMEM, plus a row-masked copy for the sparse
+//                       stream on mixed steps) and dS^T (bf16, to a swizzled
+//                       shared-memory tile); then dV += P_f^T G_f + P_s^T G_s'
+//                       (TS) and dK += dS^T Q (SS).  Warp 2 stores each dS^T
+//                       tile to the workspace by TMA.
+//                       TMEM: dV | dK | K | V | S range | dP_f^T = 512 cols.
+//   bwd_dq_gemm_kernel  dQ = sigma dS K over the stored dS^T blocks: CTA =
+//                       128 queries of one head, a 3-stage TMA ring of two
+//                       dS^T blocks and a key tile per stage, the
+//                       accumulator in 128 TMEM columns.
 // The sparse-stream MMAs are skipped on steps where no (query block, key
 // block) pair is selected.  Every wait is bounded; an expiry sets a device
 // status word and the CTA drains its tensor-core work and frees TMEM.
