@@ -4,7 +4,9 @@ Two layers, both argument marshalling only:
 
 * ``ssa_*`` functions with the C names and signatures; pointers and the
   stream are plain integers.
-* ``select_blocks``, ``attn_fwd_dual``, ``align_loss``, ``attn_bwd``: take
+* ``select_blocks``, ``attn_fwd_dual``, ``align_loss``, ``attn_bwd``,
+  ``attn_fwd_sparse``, ``diagnostics`` and ``DecodeCache`` (a key/value cache
+  with its pooled keys, for ``ssa_decode_pool`` / ``ssa_decode_step``): take
   torch CUDA tensors, allocate the outputs and the workspace with torch, pass
   raw device pointers and torch's current stream to the C entry point and
   raise ``SsaError`` on a non-zero status.
