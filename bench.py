@@ -102,6 +102,13 @@ def ds_blocks_per_bh(T):
     return ntk * (T // 64) - ntk * (ntk - 1)
 
 
+def workload_config(w, world, parallelism):
+    """The ``config`` object both arms print for workload ``w``."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "block": w.block,
+            "topk": w.topk, "global_batch": w.B * world, "seq_len": w.T,
+            "parallelism": parallelism}
+
+
 def data_description(w):
     """What the synthetic inputs of workload ``w`` are, for the JSON line."""
     base = "synthetic (seeded N(0,1)" + ("/sqrt(d)" if w.scale_data else "")
@@ -448,9 +455,7 @@ def run_ours(args, rank, world, dev, peaks, peak_src):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": data_description(w),
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "block": w.block,
-                   "topk": w.topk, "global_batch": w.B * world, "seq_len": w.T,
-                   "parallelism": f"replicas x{world} (independent batch*head units)",
+        "config": {**workload_config(w, world, f"replicas x{world} (independent batch*head units)"),
                    "l2": "flushed before every timed step", "kernel_path": layer.path},
         "roofline": roof,
         "breakdown_ms": {n: round(avg[n], 4) for n in names},
@@ -607,9 +612,8 @@ def run_reference(args, world):
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs / args.steps * 1e3, 2), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D,
-                   "block": w.block, "topk": w.topk},
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": data_description(w),
+        "config": workload_config(w, 1, "the oracle on one process's host cores"),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,

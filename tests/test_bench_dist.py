@@ -64,3 +64,13 @@ def test_ncu_traffic_only_for_the_captured_workload_and_source(tmp_path, monkeyp
     assert bench.ncu_traffic("k", "bf16_T16384_H16_sweep") is None  # another workload
     assert bench.ncu_traffic("stale", "bf16_T8192_H16_hot") is None  # source changed since
     assert bench.ncu_traffic("missing", "bf16_T8192_H16_hot") is None
+
+
+def test_both_arms_print_the_same_config_keys():
+    from block_sparse_full_b200.inputs import WORKLOADS
+    w = WORKLOADS["bf16_T8192_H16_hot"]
+    ours = bench.workload_config(w, 2, "replicas x2")
+    ref = bench.workload_config(w, 1, "oracle")
+    assert set(ours) == set(ref)
+    assert ours["workload"] == ref["workload"] == w.name
+    assert ours["global_batch"] == 2 * w.B and ref["global_batch"] == w.B
