@@ -3,11 +3,11 @@
 // Sparse Attention Stream = block-sparse attention; section 4, "Efficienza":
 // the same operations as MoBA at inference).
 //
-// Two kernels, both on CUDA cores in float64 (the decision is an integer
-// set, so it is taken in the precision the definition fixes):
+// Two steps, on CUDA cores in float64 (the decision is an integer set, so it
+// is taken in the precision the definition fixes):
 //   pool_kernel       reads Q and K once (HBM-bound) and writes the exact
 //                     float64 block means Qbar, Kbar to the workspace;
-//   score_topk_row_kernel one CTA per 8 query blocks of one (b, h): scores
+//   score_topk_kernel one CTA per 8 query blocks of one (b, h): scores
 //                     s_ij for j < i (register-tiled over 8 rows x 4 keys
 //                     per warp, fixed summation order), then one warp per
 //                     row fills the free slots by warp-argmax rounds under
@@ -33,8 +33,7 @@ constexpr int kMaxBlocksPerRow = 4096;  // n = T / block limit (score row in sme
 // consecutive columns of rows g, g + G, ... of each unit; a warp covers
 // whole rows, so they coalesce), then the units are reduced one at a time
 // through shared memory in a fixed order.  Each thread keeps 8 to 16 loads
-// in flight.  The
-// base pointers are 16-byte aligned (host-checked).
+// in flight.  The base pointers are 16-byte aligned (host-checked).
 template <typename T, int D, int BLOCK>
 struct PoolShape {
     static constexpr int V = 16 / (int)sizeof(T);  // columns per load
