@@ -1,21 +1,23 @@
 // Fused dual-stream forward on the sm_100a tensor cores (bf16 in, fp32
-// accumulate, head dim 128): one pass over the causal K/V of a 128-row query
+// accumulate, head dim 64 or 128): one pass over the causal K/V of a 128-row query
 // tile produces the full-attention output, the block-sparse output, the
 // discarded mass delta(t) and both log-sum-exps ("Sintesi Tecnica: SSA",
 // section 2: the sparse stream and its full-attention counterpart of the
 // same layer; section 1: the sparse stream normalises over the selected
 // subset only).
 //
-// CTA = (query tile of 128 rows, batch*head), 256 threads:
+// CTA = (query tile of 128 rows, batch*head), 384 threads:
 //   warps 0, 2  TMA producers: Q once and K_j (warp 0), V_j (warp 2), into
 //               2-stage rings
 //   warp 1      TMEM owner and MMA issuer (one thread):
 //                 S_j = Q K_j^T          (tcgen05 SS, into S buffer j%2)
 //                 O_sel/O_uns += P_j V_j  (tcgen05 TS, P read from TMEM)
-//   warps 4..7  softmax: thread = query row = TMEM lane.  Reads S_j, keeps
-//               one running max for both streams, splits the row sum into
-//               l_sel / l_uns by the selection mask and writes P_j (bf16)
-//               back into the S buffer for the PV product.
+//   warps 4..11 two softmax warpgroups, warpgroup h taking keys
+//               [64h, 64h + 64) of every tile: thread = query row = TMEM
+//               lane.  They read S_j, keep one running max for both streams
+//               (combined through shared memory once per tile), split the row
+//               sum into l_sel / l_uns by the selection mask and write P_j
+//               (bf16) back into the S buffer for the PV product.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O_sel [256,384) O_uns [384,512).
 //
 // A 128-key tile holds one or two key blocks and the 128 query rows one or
