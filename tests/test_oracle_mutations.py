@@ -48,6 +48,12 @@ MUTATIONS = {
                                             "sel = sorted(forced + ranked[: max(topk - len(forced) + 1, 0)])"),
     "decode_ties_to_higher_index": ("ranked = sorted(cand, key=lambda j: (-score[j], j))",
                                     "ranked = sorted(cand, key=lambda j: (-score[j], -j))"),
+    "sqdiff_mean_not_sum": ("\"sqdiff\": ((h_full - h_sparse) ** 2).sum(axis=1),",
+                            "\"sqdiff\": ((h_full - h_sparse) ** 2).mean(axis=1),"),
+    "decode_pool_sum_not_mean": (".reshape(B, H, n_done, block, d).mean(axis=3)",
+                                 ".reshape(B, H, n_done, block, d).sum(axis=3)"),
+    "decode_lse_missing_max": ("lse_out[b, h] = m + np.log(e.sum())",
+                               "lse_out[b, h] = np.log(e.sum())"),
     "decode_future_keys_of_current_block": ("keys = np.concatenate([np.arange(j * block, min((j + 1) * block, t + 1)) for j in sel])",
                                             "keys = np.concatenate([np.arange(j * block, (j + 1) * block) for j in sel])"),
 }
@@ -69,6 +75,8 @@ PIN_TESTS = [
     lambda: pins.test_sparse_only_diagonal_budget_is_blockwise_causal_attention(),
     lambda: pins.test_sparse_only_brute_force_tiny(),
     lambda: pins.test_sink_mass_is_library_softmax_on_block_zero(),
+    lambda: pins.test_sqdiff_rows_from_library_attention(),
+    lambda: pins.test_decode_pool_is_block_mean(),
     lambda: pins.test_decode_full_budget_is_causal_attention_row(),
     lambda: pins.test_decode_selection_brute_force(),
     lambda: pins.test_decode_ties_sink_and_first_block(),

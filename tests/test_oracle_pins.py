@@ -184,6 +184,22 @@ def test_streams_match_library_attention_with_masks():
     assert np.all(out["delta"][has_uns] > 0.0)
 
 
+def test_sqdiff_rows_from_library_attention():
+    """sqdiff(t) = sum_c (h_full - h_sparse)_c^2, with both outputs from library
+    attention under the causal and the selection masks; its mean over the
+    B*H*T*d elements is the alignment loss."""
+    B, H, T, d, block = 1, 2, 96, 8, 8
+    q, k, v, idx, cnt = _case(B, H, T, d, block, topk=3, seed=17)
+    out = O.attn_fwd_dual(q, k, v, idx, cnt, block, 0.6)
+    causal, sel, _ = token_masks(idx, cnt, block, T)
+    hf = sdpa(q, k, v, causal[None, None], 0.6)
+    hs = sdpa(q, k, v, sel, 0.6)
+    np.testing.assert_allclose(out["sqdiff"], ((hf - hs) ** 2).sum(axis=-1), rtol=1e-10, atol=1e-14)
+    assert np.all(out["sqdiff"][..., :block] == 0.0)  # the first query block sees only itself
+    L, _ = O.align_loss(out["h_full"], out["h_sparse"])
+    assert L == pytest.approx(out["sqdiff"].sum() / (B * H * T * d), rel=1e-12)
+
+
 def test_lse_against_library_logsumexp():
     B, H, T, d, block = 1, 2, 64, 8, 8
     q, k, v, idx, cnt = _case(B, H, T, d, block, topk=2, seed=5)
