@@ -34,6 +34,14 @@ MUTATIONS = {
     "bwd_missing_scale": ("dk += sm_scale * dx.T @ q[t]", "dk += dx.T @ q[t]"),
     "bwd_dv_sparse_dropped": ("dv += p_full.T @ g_full[t] + p_sparse.T @ g_sparse[t]",
                               "dv += p_full.T @ g_full[t]"),
+    "sparsity_gradient_to_wrong_stream": ("g_full = f64(dh_full) + w_s * (2.0 / n_total) * (hf - hs)",
+                                          "g_full = f64(dh_full) + w_s * (2.0 / n_total) * (hs - hf)"),
+    "bwd_sparse_jacobian_row_term_dropped": (
+        "dx += p_sparse * (dp_sparse - (p_sparse * dp_sparse).sum(axis=1, keepdims=True))",
+        "dx += p_sparse * dp_sparse"),
+    "bwd_dq_unscaled": ("dq[t] = sm_scale * dx @ k", "dq[t] = dx @ k"),
+    "bwd_sparse_stream_over_all_causal_keys": (
+        "sel = causal & blocksel[t // block][:, s // block]", "sel = causal"),
     "loss_sum_not_mean": ("L = float(np.mean((hf - hs) ** 2))", "L = float(np.sum((hf - hs) ** 2))"),
     "sparse_only_no_causal_mask": ("x = np.where(keys[None, :] <= ts[:, None], x, -np.inf)",
                                    "x = np.where(keys[None, :] <= ts[:, None] + block, x, -np.inf)"),
