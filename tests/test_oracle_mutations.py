@@ -27,6 +27,10 @@ MUTATIONS = {
                           "return pool_blocks(k, block) @ pool_blocks(q, block).T"),
     "ties_to_higher_index": ("ranked = sorted(cand, key=lambda j: (-s[i, j], j))",
                              "ranked = sorted(cand, key=lambda j: (-s[i, j], -j))"),
+    "margin_always_zero": ("margin[b, h, i] = s[i, ranked[r - 1]] - s[i, ranked[r]]",
+                           "margin[b, h, i] = 0.0"),
+    "margin_from_the_top_block": ("margin[b, h, i] = s[i, ranked[r - 1]] - s[i, ranked[r]]",
+                                  "margin[b, h, i] = s[i, ranked[0]] - s[i, ranked[r]]"),
     "diagonal_outside_budget": ("r = max(topk - len(forced), 0)",
                                 "r = max(topk - len(forced) + 1, 0)"),
     "commit_gradient_sign": ("g_sparse = f64(dh_sparse) + w_c * (2.0 / n_total) * (hs - hf)",
@@ -72,6 +76,7 @@ PIN_TESTS = [
     lambda: pins.test_pooling_closed_forms(),
     lambda: pins.test_scores_are_mean_of_per_query_scores(),
     lambda: pins.test_topk_ties_go_to_lower_block_index(),
+    lambda: pins.test_selection_margin_is_zero_exactly_where_the_best_set_is_not_unique(),
     lambda: pins.test_mask_words_beyond_32_blocks(),
     lambda: pins.test_full_budget_reduces_to_causal_attention(),
     lambda: pins.test_streams_match_library_attention_with_masks(),

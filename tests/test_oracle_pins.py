@@ -121,6 +121,39 @@ def test_topk_against_exhaustive_search(topk, force_sink):
             assert bits == want
 
 
+def test_selection_margin_is_zero_exactly_where_the_best_set_is_not_unique():
+    """The margin the GPU tests use to excuse near-ties: with integer-valued
+    data every block score is exact, so an exhaustive search over the r-subsets
+    of the candidates tells whether the best set is unique; the margin must be
+    0 exactly where it is not, positive where it is, and inf where nothing
+    was rejected."""
+    r = np.random.default_rng(23)
+    B, H, block, n, d = 1, 3, 2, 10, 3
+    q = r.integers(-2, 3, size=(B, H, n * block, d)).astype(np.float64)
+    k = r.integers(-1, 2, size=(B, H, n * block, d)).astype(np.float64)
+    seen_tie = seen_unique = False
+    for topk in (2, 3, 4):
+        _, _, _, margin = O.select_blocks(q, k, block, topk)
+        for h in range(H):
+            s = O.block_scores(q[0, h], k[0, h], block)
+            for i in range(n):
+                cand = list(range(i))
+                rr = topk - 1
+                if rr == 0 or rr >= len(cand):
+                    assert margin[0, h, i] == np.inf
+                    continue
+                sums = [sum(s[i, j] for j in c) for c in itertools.combinations(cand, rr)]
+                best = max(sums)
+                unique = sum(1 for x in sums if x == best) == 1
+                if unique:
+                    assert margin[0, h, i] > 0
+                    seen_unique = True
+                else:
+                    assert margin[0, h, i] == 0
+                    seen_tie = True
+    assert seen_tie and seen_unique
+
+
 def test_topk_ties_go_to_lower_block_index():
     # block = token, q = 1: scores are the key values; blocks 1, 2, 4 tie
     k = np.array([0.0, 5.0, 5.0, 1.0, 5.0, 0.0, 0.0]).reshape(1, 1, 7, 1)
