@@ -413,9 +413,11 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             __syncwarp();
             issued[s] = i;
         }
-        if (*abort_flag)
-            for (int s = 0; s < NSTAGE; ++s)
-                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
+        // every copy issued lands before the CTA exits, also when another role gives
+        // up after this warp left its loop (the last load of each stage; earlier
+        // ones completed before their stage was refilled)
+        for (int s = 0; s < NSTAGE; ++s)
+            if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
     } else if (warp == 1) {
         {  // ------------------------------------------ MMA issuer (whole warp)
             // descriptors formed once, advanced by constant offsets; each MMA group
@@ -831,9 +833,8 @@ bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_const
             __syncwarp();
             issued[s] = j;
         }
-        if (*abort_flag)
-            for (int s = 0; s < NSTAGE; ++s)
-                if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
+        for (int s = 0; s < NSTAGE; ++s)  // every issued copy lands before the CTA exits
+            if (issued[s] >= 0) wait_drain(BAR(B_FULL + s), (issued[s] / NSTAGE) & 1, kDrainLimitNs);
     } else if (warp == 1) {
         // ------------------------------------------ MMA issuer (whole warp)
         constexpr uint32_t id = idesc_bf16_f32(TILE, D, true, true);  // A and B MN-major
@@ -930,12 +931,12 @@ size_t ds_blocks_per_bh(int T) {
     const size_t ntk = (size_t)(T + TILE - 1) / TILE;
     return ntk * (size_t)(T / STEP) - ntk * (ntk - 1);
 }
-// Heads per launch so that the dS^T buffer stays within a fixed budget.
-constexpr size_t kDsBudgetBytes = size_t(4) << 30;
+// Heads per launch so that the dS^T buffer stays within a byte budget
+// (4 GiB unless a test sets another through ssa_debug_set_ds_budget_bytes).
 int heads_per_chunk(const ssa_params_t& p) {
     const size_t per = ds_blocks_per_bh(p.T) * (size_t)STEP * TILE * 2;
     const size_t bh = (size_t)p.B * p.H;
-    size_t hc = kDsBudgetBytes / per;
+    size_t hc = (size_t)ds_budget_bytes() / per;
     if (hc < 1) hc = 1;
     if (hc > bh) hc = bh;
     return (int)hc;

@@ -239,10 +239,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             else issued[1] = jj;
             ++jj;
         }
-        if (*abort_flag) {  // let copies in flight land before the CTA exits
-            if (issued[0] >= 0) wait_drain(BAR(FULLB), (issued[0] >> 1) & 1, kDrainLimitNs);
-            if (issued[1] >= 0) wait_drain(BAR(FULLB + 1), (issued[1] >> 1) & 1, kDrainLimitNs);
-        }
+        // Every copy this warp issued lands before the CTA exits, whether or not a
+        // wait gave up (another role may abort after this warp left its loop): the
+        // Q tile, then the last load of each ring slot (earlier ones completed
+        // before their slot was refilled).  Free on the normal path.
+        if (is_k) wait_drain(BAR(B_QFULL), 0, kDrainLimitNs);
+        if (issued[0] >= 0) wait_drain(BAR(FULLB), (issued[0] >> 1) & 1, kDrainLimitNs);
+        if (issued[1] >= 0) wait_drain(BAR(FULLB + 1), (issued[1] >> 1) & 1, kDrainLimitNs);
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         // Descriptors are formed once and advanced by constant offsets; each group
