@@ -11,9 +11,15 @@
 // loads the library holds until the process exits.
 //
 // Host code cannot use the array's name as a device address (on the host it
-// names a shadow variable), so the device address is looked up once per
-// device with cudaGetSymbolAddress, while that device is current, on the
-// first call made on it.
+// names a shadow variable), so the device address is looked up with
+// cudaGetSymbolAddress while the device is current, on the first call made in
+// each CUDA context, and cached against that context's unique ID: after a
+// cudaDeviceReset the next call runs in a new primary context, where the
+// module (and with it the array) has been loaded again, and looks the address
+// up again instead of using the old one.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "ssa_internal.h"
@@ -27,10 +33,39 @@ static __device__ __align__(256) unsigned char g_select_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+struct Cached {
+    unsigned long long ctx_id;  // 0 = nothing cached
+    void* addr;
+};
+Cached g_cache[kMaxDevices] = {};
 
-// Device address of g_select_scratch on the current device (looked up on
-// first use, then cached).  Returns an SSA status.
+// Unique ID of the calling thread's current CUDA context (0 if none or the
+// driver entry points are unavailable), through the runtime's driver
+// entry-point query so that the library needs no link against libcuda.
+unsigned long long current_context_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of g_select_scratch on the current device, valid in the
+// current context.  Returns an SSA status.
 int scratch_address(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -38,15 +73,17 @@ int scratch_address(void** out) {
     if (dev < 0 || dev >= kMaxDevices)
         return ssa::fail(SSA_ERR_UNSUPPORTED, "device index %d beyond %d", dev, kMaxDevices);
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_addr[dev]) {
+    const unsigned long long id = current_context_id();
+    if (id == 0 || g_cache[dev].ctx_id != id) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_select_scratch);
         if (e != cudaSuccess || !p)
             return ssa::fail(SSA_ERR_CUDA, "cudaGetSymbolAddress(select scratch): %s",
                              cudaGetErrorString(e));
-        g_scratch_addr[dev] = p;
+        // the lookup makes the primary context current if none was; cache under it
+        g_cache[dev] = Cached{id ? id : current_context_id(), p};
     }
-    *out = g_scratch_addr[dev];
+    *out = g_cache[dev].addr;
     return SSA_OK;
 }
 

@@ -127,7 +127,9 @@ int ssa_select_blocks(const ssa_params_t* params, const void* q, const void* k,
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture begins.
+ *     before any stream capture begins.  The address is cached per CUDA
+ *     context: after a cudaDeviceReset the first call in the new context
+ *     looks it up again (so it too should come before any capture).
  *   - All calls share the one array: calls that overlap on the GPU (other
  *     streams, other host threads) race and give undefined results; order
  *     them on one stream.  Nothing in the array needs clearing between calls.
@@ -197,10 +199,12 @@ int ssa_decode_step(const ssa_params_t* params, int t, const void* q, const void
                     void* ws, size_t ws_bytes, void* stream);
 
 /*
- * Attention diagnostics (section 1: the sparse approximation error grows
- * with the discarded mass delta; the pages also discuss the first block as an
- * attention sink and the sparsity of learned attention), from the dual
- * forward's lse_full and delta for the same q, k:
+ * Attention diagnostics, from the dual forward's lse_full and delta for the
+ * same q, k.  The sparse approximation error grows with the discarded mass
+ * delta ("Sintesi Tecnica: SSA", section 1); the paper's abstract (the
+ * chatpaper.ai summary and the arXiv 2511.20102 listing, "Abstract") ties
+ * long-context extrapolation to too much attention going to sink areas, the
+ * first block here, and discusses how sparse learned attention is:
  *   sink_rows[t]  = sum_{s <= t, s < block} exp(sm_scale q_t . k_s - lse_full(t))
  *                   (full-softmax mass on block 0), float32 [B,H,T];
  *   head_stats    = float32 [B,H,2]: mean over t of delta, mean over t of sink.
@@ -287,6 +291,17 @@ int ssa_selftest_wait_timeout(unsigned long long limit_ns, int* gave_up, void* s
  * then reports SSA_ERR_TIMEOUT and the outputs of that call are undefined.
  * Process-wide; not synchronised with calls running on other threads. */
 void ssa_debug_set_wait_limit_ns(unsigned long long ns);
+
+/* Test hook: byte budget of the tensor-core backward's dS workspace, which
+ * sets how many heads form one group (ssa_bwd_heads_per_group: the largest
+ * count whose dS blocks fit, at least 1).  0 restores the default of 4 GiB.
+ * Affects ssa_workspace_size(SSA_WS_BWD), ssa_bwd_heads_per_group and
+ * ssa_attn_bwd calls made after it, so a caller sizes the workspace after
+ * setting it.  A smaller budget makes small problems run the grouped path
+ * (several launches of the dK/dV kernel and the dQ GEMM, one per group)
+ * that otherwise only very long sequences reach.  Process-wide, like the
+ * hook above. */
+void ssa_debug_set_ds_budget_bytes(unsigned long long bytes);
 
 /* Measurement hook: makes later ssa_attn_bwd calls on the tensor-core path
  * record the caller's CUDA events (cudaEvent_t, passed as void*) on the call's

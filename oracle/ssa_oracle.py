@@ -259,10 +259,11 @@ def attn_fwd_sparse(q, k, v, idx, cnt, block: int, sm_scale: float, rows=None):
 
 
 def diagnostics(q, k, lse_full, delta, block: int, sm_scale: float):
-    """Attention diagnostics the pages discuss (section 1 of the technical
-    summaries: the approximation error grows with the discarded mass delta;
-    the first block acting as an attention sink; the sparsity of learned
-    attention):
+    """Attention diagnostics the pages discuss: the approximation error grows
+    with the discarded mass delta (section 1 of the technical summaries);
+    extrapolation suffers when too much attention goes to sink areas, here
+    the first block (the paper's abstract, on the chatpaper.ai summary and the
+    arXiv 2511.20102 listing); how sparse learned attention is (same abstract):
 
       sink(t)        = full-softmax mass on the keys of block 0:
                        sum_{s <= t, s < block} exp(sm_scale q_t . k_s - lse_full(t))
