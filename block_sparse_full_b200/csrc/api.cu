@@ -16,6 +16,8 @@ thread_local char g_last_error[512] = "";
 constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<void*> g_kernel_events[kKernelEvents];
+constexpr unsigned long long kDefaultDsBudget = 4ull << 30;
+std::atomic<unsigned long long> g_ds_budget{kDefaultDsBudget};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -87,6 +89,7 @@ size_t bwd_workspace(const ssa_params_t& p) {
 }  // namespace
 
 unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+unsigned long long ds_budget_bytes() { return g_ds_budget.load(std::memory_order_relaxed); }
 
 void mark_kernel_event(int i, cudaStream_t s) {
     void* e = g_kernel_events[i].load(std::memory_order_relaxed);
@@ -341,6 +344,10 @@ int ssa_bwd_heads_per_group(const ssa_params_t* p) {
 
 void ssa_debug_set_wait_limit_ns(unsigned long long ns) {
     g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs, std::memory_order_relaxed);
+}
+
+void ssa_debug_set_ds_budget_bytes(unsigned long long bytes) {
+    g_ds_budget.store(bytes ? bytes : kDefaultDsBudget, std::memory_order_relaxed);
 }
 
 int ssa_debug_set_kernel_events(void* const* events, int n) {

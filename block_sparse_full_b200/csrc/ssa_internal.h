@@ -22,6 +22,10 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Wall-clock limit of the kernels' bounded waits (default 2 s; tests shorten it).
 unsigned long long wait_limit_ns();
 
+// Byte budget of the tensor-core backward's dS workspace (default 4 GiB;
+// tests shrink it so that small problems run in several head groups).
+unsigned long long ds_budget_bytes();
+
 // Measurement hook (ssa_debug_set_kernel_events): records caller event i on
 // stream s when the hook is enabled, else does nothing.
 constexpr int kKernelEvents = 4;

@@ -38,7 +38,8 @@ EXPORTS = (
     "ssa_decode_step", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
     "ssa_kernel_path", "ssa_bwd_heads_per_group", "ssa_selftest_math", "ssa_selftest_wait_timeout",
-    "ssa_debug_set_wait_limit_ns", "ssa_debug_set_kernel_events", "ssa_version",
+    "ssa_debug_set_wait_limit_ns", "ssa_debug_set_ds_budget_bytes", "ssa_debug_set_kernel_events",
+    "ssa_version",
 )
 
 
@@ -88,6 +89,7 @@ _SIGNATURES = {
     "ssa_selftest_math": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p]),
     "ssa_version": (c_int, []),
     "ssa_debug_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
+    "ssa_debug_set_ds_budget_bytes": (None, [ctypes.c_ulonglong]),
     "ssa_debug_set_kernel_events": (c_int, [c_void_p, c_int]),
     "ssa_selftest_wait_timeout": (c_int, [ctypes.c_ulonglong, c_void_p, c_void_p]),
 }
@@ -192,6 +194,10 @@ def ssa_selftest_wait_timeout(limit_ns, gave_up, stream):
 
 def ssa_debug_set_wait_limit_ns(ns):
     _lib.ssa_debug_set_wait_limit_ns(ns)
+
+
+def ssa_debug_set_ds_budget_bytes(nbytes):
+    _lib.ssa_debug_set_ds_budget_bytes(nbytes)
 
 
 def ssa_bwd_heads_per_group(params):

@@ -62,8 +62,10 @@ def oracle_mask_to_dev(o_mask):
     return torch.from_numpy(o_mask.view(np.int32).copy()).to(DEV)
 
 
-def compare_fwd(case, dtype, gpu, ref, rows=None):
-    """Compare GPU forward outputs (all rows) with oracle outputs (``rows``)."""
+def compare_fwd(case, dtype, gpu, ref, rows=None, ref_abs=None):
+    """Compare GPU forward outputs (all rows) with oracle outputs (``rows``).
+    With ``ref_abs`` (the oracle forward on |v|, same rows) the per-row squared
+    difference is also held to ``sqdiff_budget``."""
     tol = TOL[dtype]
     sl = (slice(None), slice(None), rows) if rows is not None else (slice(None),) * 3
     errs = {}
@@ -85,9 +87,137 @@ def compare_fwd(case, dtype, gpu, ref, rows=None):
         g = gpu[name][sl].cpu().numpy()
         errs[name] = float(np.abs(g - ref[name]).max())
         assert errs[name] <= tol["lse"], f"{case} {name} {errs[name]:.3e}"
-    g = gpu["sqdiff"][sl].cpu().numpy().astype(np.float64)
-    errs["sqdiff_rel"] = float(np.abs(g - ref["sqdiff"]).sum() / max(ref["sqdiff"].sum(), 1e-30))
+    if ref_abs is not None:
+        g = gpu["sqdiff"][sl].cpu().numpy().astype(np.float64)
+        r = ref["sqdiff"]
+        dev = np.abs(g - r)
+        budget = sqdiff_budget(dtype, ref, ref_abs)
+        assert np.isfinite(g).all(), "sqdiff"
+        worst = np.unravel_index(np.argmax(dev - budget), dev.shape)
+        assert (dev <= budget).all(), (f"{case} sqdiff: |gpu - oracle| {dev[worst]:.3e} > budget "
+                                       f"{budget[worst]:.3e} (oracle {r[worst]:.3e}) at {worst}")
+        errs["sqdiff_budget_ratio"] = float((dev / budget).max())
+        errs["sqdiff_rel_max"] = float((dev / np.maximum(r, 1e-30)).max(initial=0.0,
+                                                                        where=r > 0))
     log(case, **errs)
+    return errs
+
+
+def sqdiff_budget(dtype, ref, ref_abs):
+    """Per-row bound on |r_gpu(t) - r_oracle(t)|, r(t) = sum_c (h_full - h_sparse)_c^2,
+    derived from the kernels' arithmetic (both kernels keep O_sel, O_uns and
+    l_sel, l_uns and form h_full = (O_sel + O_uns) / (l_sel + l_uns),
+    h_sparse = O_sel / l_sel, r from the float32 values before rounding).
+
+    The tensor-core path rounds each softmax weight p to bf16 (relative error
+    <= u = 2^-8) before the P.V products but sums l_sel, l_uns from the
+    unrounded weights.  With d = h_full - h_sparse, errors e_sel in O_sel and
+    e_uns in O_uns move d_c by  e_sel,c (1/l - 1/l_sel) + e_uns,c / l,  and
+    since 1/l - 1/l_sel = -delta / l_sel and |e_x,c| <= u sum_x p |v_c|,
+    |dd_c| <= u delta (A_sel,c + A_uns,c), A the softmax-weighted means of |v_c|
+    over the selected / unselected keys (the oracle run on |v|).  An
+    approximate exponential (relative error <= 7.5e-5 < 2^-12) perturbs a
+    weight in O and l alike, which moves d_c by at most
+    2^-12 (delta (A + |h_full| + |h_sparse|) + 2 |d_c|).  The two separate
+    float32 reciprocals and products add 2^-22 (|h_full| + |h_sparse|).  With
+    E_c the sum of these terms, |r_gpu - r| <= sum_c (2 |d_c| E_c + E_c^2).
+    float32 inputs (no weight rounding, float32 sums over at most 2^10 keys
+    per row in the tests) take u = 2^-14 for both terms."""
+    d = np.abs(ref["h_full"] - ref["h_sparse"])
+    A = ref_abs["h_sparse"] + ref_abs["h_unsel"]
+    Hm = np.abs(ref["h_full"]) + np.abs(ref["h_sparse"])
+    delta = ref["delta"][..., None]
+    u, eta = (2.0 ** -8, 2.0 ** -12) if dtype == "bf16" else (2.0 ** -14, 2.0 ** -14)
+    E = delta * (u * A + eta * (A + Hm)) + 2 * eta * d + 2.0 ** -22 * Hm
+    return (2 * d * E + E * E).sum(-1) + 1e-6 * ref["sqdiff"] + 1e-30
+
+
+def oracle_fwd(q, k, v, idx, cnt, block, scale, rows=None, with_abs=True, threads=None):
+    """The oracle forward for every (batch, head) of q, k, v, one (b, h) per
+    task on a thread pool (numpy releases the GIL in its array loops), and,
+    with ``with_abs``, the same forward on |v| (the weighted means of |v| that
+    ``sqdiff_budget`` takes).  Returns (ref, ref_abs)."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    qn, kn, vn = (O.f64(x) for x in (q, k, v))
+    B, H = qn.shape[:2]
+    jobs = [(b, h) for b in range(B) for h in range(H)]
+    vs = [vn] + ([np.abs(vn)] if with_abs else [])
+
+    def one(args):
+        which, (b, h) = args
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        return O.attn_fwd_dual(qn[sl], kn[sl], vs[which][sl], idx[sl], cnt[sl], block, scale,
+                               rows=rows)
+
+    tasks = [(wi, j) for wi in range(len(vs)) for j in jobs]
+    nthr = threads or min(len(tasks), os.cpu_count() or 1, 16)
+    with ThreadPoolExecutor(max_workers=nthr) as ex:
+        res = list(ex.map(one, tasks))
+    outs = []
+    for wi in range(len(vs)):
+        part = res[wi * len(jobs):(wi + 1) * len(jobs)]
+        merged = {}
+        for name in part[0]:
+            arr = np.zeros((B, H) + part[0][name].shape[2:])
+            for (b, h), r in zip(jobs, part):
+                arr[b, h] = r[name][0, 0]
+            merged[name] = arr
+        outs.append(merged)
+    return outs[0], (outs[1] if with_abs else None)
+
+
+def oracle_loss_rows(q, k, v, idx, cnt, block, scale, dtype, threads=None):
+    """Per (batch, head) and on every row: the oracle's alignment loss term
+    (``O.align_loss`` of that head's outputs, a mean over its T x d
+    elements), its per-row squared difference and the ``sqdiff_budget`` of
+    each row.  Heads run on a thread pool and only row vectors are kept, so
+    that whole workloads fit in host memory.  Returns (loss, sqdiff, budget):
+    the mean over heads of the per-head losses (heads have equal sizes, so it
+    is the loss over all B*H*T*d elements) and two [B, H, T] arrays."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    qn, kn, vn = (O.f64(x) for x in (q, k, v))
+    B, H, T = qn.shape[:3]
+    jobs = [(b, h) for b in range(B) for h in range(H)]
+
+    def one(bh):
+        b, h = bh
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        ref = O.attn_fwd_dual(qn[sl], kn[sl], vn[sl], idx[sl], cnt[sl], block, scale)
+        ref_abs = O.attn_fwd_dual(qn[sl], kn[sl], np.abs(vn[sl]), idx[sl], cnt[sl], block, scale)
+        ls, _ = O.align_loss(ref["h_full"], ref["h_sparse"])
+        return ls, ref["sqdiff"][0, 0], sqdiff_budget(dtype, ref, ref_abs)[0, 0]
+
+    nthr = threads or min(len(jobs), os.cpu_count() or 1, 16)
+    with ThreadPoolExecutor(max_workers=nthr) as ex:
+        res = list(ex.map(one, jobs))
+    sq = np.zeros((B, H, T))
+    bud = np.zeros((B, H, T))
+    for (b, h), (_, r, bb) in zip(jobs, res):
+        sq[b, h], bud[b, h] = r, bb
+    return float(np.mean([x[0] for x in res])), sq, bud
+
+
+def compare_loss(case, p, gpu_sqdiff, ref_loss, ref_sq, budget, n_total, w_s=2.0, w_c=3.0):
+    """GPU per-row squared differences (every row) against the oracle's within
+    ``budget``, and the GPU loss kernel against the oracle's loss: within the
+    summed row budgets and within relative 2e-2."""
+    g = gpu_sqdiff.cpu().numpy().astype(np.float64)
+    dev = np.abs(g - ref_sq)
+    worst = np.unravel_index(np.argmax(dev - budget), dev.shape)
+    assert (dev <= budget).all(), (f"{case} sqdiff: {dev[worst]:.3e} > budget {budget[worst]:.3e} "
+                                   f"(oracle {ref_sq[worst]:.3e}) at {worst}")
+    loss = ssa.align_loss(p, gpu_sqdiff, w_s, w_c).cpu().numpy().astype(np.float64)
+    allowed = min(budget.sum() / n_total, TOL["bf16"]["loss_rel"] * ref_loss)
+    errs = {}
+    for i, wgt in enumerate((w_s, w_c)):
+        e = abs(loss[i] / wgt - ref_loss)
+        errs[f"loss{i}_rel"] = e / ref_loss
+        assert e <= allowed, f"{case} loss[{i}]: |{loss[i] / wgt:.6e} - {ref_loss:.6e}| > {allowed:.3e}"
+    errs["sqdiff_budget_ratio"] = float((dev / budget).max())
+    errs["loss_budget"] = budget.sum() / n_total / ref_loss
+    log(case + "/loss", **errs)
     return errs
 
 
@@ -108,13 +238,13 @@ def dq_rounding_budget(q, k, v, idx, cnt, block, scale, dh_full, dh_sparse, w_s,
     return scale * (dDf * np.abs(kbar["h_full"]) + dDs * np.abs(kbar["h_sparse"]))
 
 
-def compare_grads(case, dtype, got, want, dq_budget=None):
-    """max |g - ref| <= tol * max|ref| per tensor; for dq also allow the
-    (elementwise) deviation caused by the bf16 rounding of the forward
+def compare_grads(case, dtype, got, want, dq_budget=None, names=("dq", "dk", "dv")):
+    """max |g - ref| <= tol * max|ref| per tensor; for dq, if given, also allow
+    the (elementwise) deviation caused by the bf16 rounding of the forward
     outputs, ``dq_budget`` from ``dq_rounding_budget``."""
     tol = TOL[dtype]["grad_rel"]
     errs = {}
-    for name, g, r in zip(("dq", "dk", "dv"), got, want):
+    for name, g, r in zip(names, got, want):
         g = g.float().cpu().numpy()
         diff = np.abs(g - r)
         scale = float(np.abs(r).max())

@@ -134,3 +134,21 @@ def test_bwd_head_groups_bound_the_ds_workspace():
     # the workspace holds exactly one group's blocks on top of the row data
     g = ssa.ssa_bwd_heads_per_group(train)
     assert ssa.ssa_workspace_size(train, ssa.SSA_WS_BWD) >= g * per_head
+
+
+def test_ds_budget_hook_sets_the_head_groups():
+    train = P(B=4, H=32, T=4096, block=64, topk=8)
+    ntk = 4096 // 128
+    per_head = (ntk * (4096 // 64) - ntk * (ntk - 1)) * 16 * 1024
+    default = ssa.ssa_bwd_heads_per_group(train)
+    try:
+        ssa.ssa_debug_set_ds_budget_bytes(1)  # below one head: still one head per group
+        assert ssa.ssa_bwd_heads_per_group(train) == 1
+        ssa.ssa_debug_set_ds_budget_bytes(int(2.5 * per_head))
+        assert ssa.ssa_bwd_heads_per_group(train) == 2
+        ws2 = ssa.ssa_workspace_size(train, ssa.SSA_WS_BWD)
+        ssa.ssa_debug_set_ds_budget_bytes(5 * per_head)
+        assert ssa.ssa_workspace_size(train, ssa.SSA_WS_BWD) == ws2 + 3 * per_head
+    finally:
+        ssa.ssa_debug_set_ds_budget_bytes(0)
+    assert ssa.ssa_bwd_heads_per_group(train) == default

@@ -10,8 +10,8 @@ from block_sparse_full_b200.inputs import WORKLOADS, Workload, make_inputs, upst
 from oracle import ssa_oracle as O
 
 from gpu_parity_util import (DEV, TOL, assert_selection, compare_fwd, compare_grads,
-                             dq_rounding_budget, log, oracle_mask_to_dev, oracle_select, params,
-                             sample_rows, to_dev)
+                             compare_loss, dq_rounding_budget, log, oracle_fwd, oracle_loss_rows,
+                             oracle_mask_to_dev, oracle_select, params, sample_rows, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -44,11 +44,11 @@ def _fwd_case(w, flags=0, topk=None, rows=None):
     excused = assert_selection(g_sel, o_sel)
     mask = oracle_mask_to_dev(o_sel[2])
     out = ssa.attn_fwd_dual(p, d["q"], d["k"], d["v"], mask)
-    ref = O.attn_fwd_dual(inp["q"], inp["k"], inp["v"], o_sel[0], o_sel[1], w.block, w.sm_scale,
-                          rows=rows)
+    ref, ref_abs = oracle_fwd(inp["q"], inp["k"], inp["v"], o_sel[0], o_sel[1], w.block,
+                              w.sm_scale, rows=rows)
     torch.cuda.synchronize()
     ssa.device_status()
-    return inp, d, p, o_sel, out, ref, excused
+    return inp, d, p, o_sel, out, (ref, ref_abs), excused
 
 
 # ------------------------------------------------------------------ selection + fwd
@@ -57,21 +57,21 @@ def _fwd_case(w, flags=0, topk=None, rows=None):
 @pytest.mark.parametrize("flags", [0, SIMT])
 def test_fwd_small(name, flags):
     w = SMALL[name]
-    _, _, p, _, out, ref, _ = _fwd_case(w, flags)
-    compare_fwd(f"{name}/flags{flags}", w.dtype, out, ref)
+    _, _, p, _, out, (ref, ref_abs), _ = _fwd_case(w, flags)
+    compare_fwd(f"{name}/flags{flags}", w.dtype, out, ref, ref_abs=ref_abs)
 
 
 def test_fwd_block128_force_sink_flag():
     w = SMALL["bf16_B2_T640_b128_sink"]
-    _, _, _, o_sel, out, ref, _ = _fwd_case(w, SINK)
+    _, _, _, o_sel, out, (ref, ref_abs), _ = _fwd_case(w, SINK)
     assert (o_sel[0][..., 1:, 0] == 0).all()  # block 0 first in every S_i, i > 0
-    compare_fwd("b128/force_sink", w.dtype, out, ref)
+    compare_fwd("b128/force_sink", w.dtype, out, ref, ref_abs=ref_abs)
 
 
 def test_f32_T1024_workload():
     w = WORKLOADS["f32_T1024_d64"]
-    inp, d, p, o_sel, out, ref, _ = _fwd_case(w)
-    compare_fwd(w.name, "f32", out, ref)
+    inp, d, p, o_sel, out, (ref, ref_abs), _ = _fwd_case(w)
+    compare_fwd(w.name, "f32", out, ref, ref_abs=ref_abs)
     loss = ssa.align_loss(p, out["sqdiff"], 1.0, 0.5).cpu().numpy()
     ls, lc = O.align_loss(ref["h_full"], ref["h_sparse"], 1.0, 0.5)
     assert abs(loss[0] - ls) <= TOL["f32"]["loss_rel"] * ls
@@ -82,9 +82,9 @@ def test_f32_T1024_workload():
 def test_T8192_workload_sampled_rows():
     w = WORKLOADS["bf16_T8192_H16_hot"]
     rows = sample_rows(w.T, w.block, 4, seed=1)
-    inp, d, p, o_sel, out, ref, excused = _fwd_case(w, rows=rows)
+    inp, d, p, o_sel, out, (ref, ref_abs), excused = _fwd_case(w, rows=rows)
     assert ssa.ssa_kernel_path(p) == 1
-    compare_fwd(w.name, "bf16", out, ref, rows=rows)
+    compare_fwd(w.name, "bf16", out, ref, rows=rows, ref_abs=ref_abs)
     # planted hot blocks are picked by every later query block
     hot = inp["hot_blocks"].numpy()
     sel = O.block_selection_matrix(o_sel[0], o_sel[1])
@@ -92,11 +92,15 @@ def test_T8192_workload_sampled_rows():
     for h in range(w.H):
         for j in np.flatnonzero(hot[0, h]):
             assert sel[0, h, j + 1:, j].all()
-    # loss: GPU reduction vs fp64 sum of the GPU rows, and rows vs oracle
+    # loss: GPU reduction vs fp64 sum of the GPU rows
     loss = ssa.align_loss(p, out["sqdiff"], 2.0, 3.0).cpu().numpy()
     host = out["sqdiff"].double().sum().item() / (w.B * w.H * w.T * w.D)
     assert abs(loss[0] - 2.0 * host) <= 1e-6 * 2.0 * host
     assert abs(loss[1] - 3.0 * host) <= 1e-6 * 3.0 * host
+    # every row of all 16 heads against the oracle, and the loss against the oracle's
+    ref_loss, ref_sq, budget = oracle_loss_rows(inp["q"], inp["k"], inp["v"], o_sel[0], o_sel[1],
+                                                w.block, w.sm_scale, "bf16")
+    compare_loss(w.name, p, out["sqdiff"], ref_loss, ref_sq, budget, w.B * w.H * w.T * w.D)
 
 
 def test_T16384_budget_sweep():
@@ -113,10 +117,10 @@ def test_T16384_budget_sweep():
         out = ssa.attn_fwd_dual(p, d["q"], d["k"], d["v"], oracle_mask_to_dev(o_sel[2]))
         loss = ssa.align_loss(p, out["sqdiff"]).cpu().numpy()
         sub = {n: inp[n][:, heads] for n in "qkv"}
-        ref = O.attn_fwd_dual(sub["q"], sub["k"], sub["v"], o_sel[0][:, heads],
-                              o_sel[1][:, heads], w.block, w.sm_scale, rows=rows)
+        ref, ref_abs = oracle_fwd(sub["q"], sub["k"], sub["v"], o_sel[0][:, heads],
+                                  o_sel[1][:, heads], w.block, w.sm_scale, rows=rows)
         gsub = {n: t[:, heads] for n, t in out.items()}
-        compare_fwd(f"{w.name}/k{k}", "bf16", gsub, ref, rows=rows)
+        compare_fwd(f"{w.name}/k{k}", "bf16", gsub, ref, rows=rows, ref_abs=ref_abs)
         delta = out["delta"].cpu().numpy()
         assert (delta >= -1e-6).all() and (delta <= 1 + 1e-6).all()
         if prev_delta is not None:  # nested budgets: discarded mass cannot grow
@@ -146,20 +150,30 @@ def test_T65536_sink_workload():
     out = ssa.attn_fwd_dual(p, d["q"], d["k"], d["v"], oracle_mask_to_dev(o_sel[2]))
     rows = np.unique(np.concatenate([sample_rows(w.T, 4096, 8, seed=5), [w.T - 1]]))
     heads = [0, 5]
-    ref = O.attn_fwd_dual(inp["q"][:, heads], inp["k"][:, heads], inp["v"][:, heads],
-                          o_sel[0][:, heads], o_sel[1][:, heads], w.block, w.sm_scale, rows=rows)
-    compare_fwd(w.name, "bf16", {n: t[:, heads] for n, t in out.items()}, ref, rows=rows)
+    ref, ref_abs = oracle_fwd(inp["q"][:, heads], inp["k"][:, heads], inp["v"][:, heads],
+                              o_sel[0][:, heads], o_sel[1][:, heads], w.block, w.sm_scale,
+                              rows=rows)
+    compare_fwd(w.name, "bf16", {n: t[:, heads] for n, t in out.items()}, ref, rows=rows,
+                ref_abs=ref_abs)
 
 
 # ------------------------------------------------------------------ backward
 
-def _bwd_case(case, w, flags, ws_, wc_, heads=None):
+def _bwd_case(case, w, flags, ws_, wc_, heads=None, rows=None):
+    """GPU selection (checked bit-exact against the oracle) -> forward ->
+    backward, and dq, dk, dv of ``heads`` against the oracle.  With ``rows``
+    only dq of those query rows is compared (dq_t depends on row t alone).
+    The tensor-core path is held to the plain 2e-2 x max|g| bound; the
+    CUDA-core path's dq also gets the budget for the bf16 rounding of the
+    forward outputs (``dq_rounding_budget``)."""
     inp = make_inputs(w)
     g = upstream_grads(w) if ws_ == 0 and wc_ == 0 else None
     d = to_dev(inp)
     o_sel = oracle_select(w, inp)
     p = params(w, d["q"], flags=flags)
-    mask = oracle_mask_to_dev(o_sel[2])
+    g_sel = ssa.select_blocks(p, d["q"], d["k"])
+    assert_selection(g_sel, o_sel)
+    mask = g_sel[2]
     fwd = ssa.attn_fwd_dual(p, d["q"], d["k"], d["v"], mask)
     dhf = g["dh_full"].to(DEV) if g else None
     dhs = g["dh_sparse"].to(DEV) if g else None
@@ -171,9 +185,15 @@ def _bwd_case(case, w, flags, ws_, wc_, heads=None):
     args = (inp["q"][:, hs], inp["k"][:, hs], inp["v"][:, hs], o_sel[0][:, hs], o_sel[1][:, hs],
             w.block, w.sm_scale, g["dh_full"][:, hs] if g else zeros,
             g["dh_sparse"][:, hs] if g else zeros, ws_, wc_)
+    if rows is not None:
+        dq, _, _ = O.attn_bwd(*args, n_total=inp["q"].numel(), rows=rows)
+        got_dq = got[0][:, hs][:, :, rows]
+        compare_grads(case, w.dtype, [got_dq], [dq[:, :, rows]], names=("dq",))
+        return
     want = O.attn_bwd(*args, n_total=inp["q"].numel())
+    simt = ssa.ssa_kernel_path(p) == 0
     budget = dq_rounding_budget(*(O.f64(a) if isinstance(a, torch.Tensor) else a for a in args),
-                                n_total=inp["q"].numel()) if w.dtype == "bf16" else None
+                                n_total=inp["q"].numel()) if w.dtype == "bf16" and simt else None
     compare_grads(case, w.dtype, [t[:, hs] for t in got], want, dq_budget=budget)
 
 
@@ -199,6 +219,32 @@ def test_train_workload_bwd_head0(mode):
     _bwd_case(f"{w.name}/{mode}", w, 0, ws_, wc_, heads=[0])
 
 
+def test_train_workload_selection_fwd_and_loss():
+    """The training workload (B4 H32 T4096): selection of all 128 heads bit
+    exact, the forward outputs of head 0 of every batch on every row, the
+    per-row squared difference of every row and the loss against the
+    oracle's."""
+    w = WORKLOADS["bf16_B4_H32_T4096_train"]
+    inp = make_inputs(w)
+    d = to_dev(inp)
+    o_sel = oracle_select(w, inp)
+    p = params(w, d["q"])
+    assert ssa.ssa_kernel_path(p) == 1
+    g_sel = ssa.select_blocks(p, d["q"], d["k"])
+    assert_selection(g_sel, o_sel)
+    out = ssa.attn_fwd_dual(p, d["q"], d["k"], d["v"], g_sel[2])
+    torch.cuda.synchronize()
+    ssa.device_status()
+    heads = [0]
+    ref, ref_abs = oracle_fwd(inp["q"][:, heads], inp["k"][:, heads], inp["v"][:, heads],
+                              o_sel[0][:, heads], o_sel[1][:, heads], w.block, w.sm_scale)
+    compare_fwd(w.name + "/head0", "bf16", {n: t[:, heads] for n, t in out.items()}, ref,
+                ref_abs=ref_abs)
+    ref_loss, ref_sq, budget = oracle_loss_rows(inp["q"], inp["k"], inp["v"], o_sel[0], o_sel[1],
+                                                w.block, w.sm_scale, "bf16")
+    compare_loss(w.name, p, out["sqdiff"], ref_loss, ref_sq, budget, w.B * w.H * w.T * w.D)
+
+
 # head dim 64 (Llama-3.2-1B-sized heads) on the tensor-core path
 D64 = Workload("bf16_H8_T4096_d64", B=1, H=8, T=4096, D=64, block=64, topk=16, dtype="bf16",
                plant="hot", grads=True, seed=16)
@@ -207,9 +253,9 @@ D64 = Workload("bf16_H8_T4096_d64", B=1, H=8, T=4096, D=64, block=64, topk=16, d
 def test_d64_heads_fwd_sampled_rows_and_bwd():
     w = D64
     rows = sample_rows(w.T, w.block, 3, seed=17)
-    inp, d, p, o_sel, out, ref, _ = _fwd_case(w, rows=rows)
+    inp, d, p, o_sel, out, (ref, ref_abs), _ = _fwd_case(w, rows=rows)
     assert ssa.ssa_kernel_path(p) == 1
-    compare_fwd(w.name, "bf16", out, ref, rows=rows)
+    compare_fwd(w.name, "bf16", out, ref, rows=rows, ref_abs=ref_abs)
     _bwd_case(w.name + "/bwd", w, 0, 0.0, 0.0, heads=[0, 5])
 
 
