@@ -74,3 +74,17 @@ def test_both_arms_print_the_same_config_keys():
     assert set(ours) == set(ref)
     assert ours["workload"] == ref["workload"] == w.name
     assert ours["global_batch"] == 2 * w.B and ref["global_batch"] == w.B
+
+
+def test_roofline_peak_follows_the_timed_region():
+    # a short region runs at the clocks of the burst GEMM measurement, a long
+    # one under the power cap like the sustained loop
+    assert bench.roofline_peak(26.0, 1645.6, 1387.7)[0] == 1645.6
+    assert "burst" in bench.roofline_peak(26.0, 1645.6, 1387.7)[1]
+    assert bench.roofline_peak(2500.0, 1645.6, 1387.7)[0] == 1387.7
+
+
+def test_gpus_flag_must_match_the_launch(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    with pytest.raises(SystemExit):
+        bench.main(["--gpus", "2", "--impl", "reference"])
