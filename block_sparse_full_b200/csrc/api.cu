@@ -171,9 +171,42 @@ int ssa_attn_fwd_dual(const ssa_params_t* p, const void* q, const void* k, const
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (use_tc(*p))
         return launch_fwd_tc(*p, q, k, v, mask, h_full, h_sparse, delta, lse_full, lse_sparse,
-                             sqdiff, ws, s);
+                             sqdiff, nullptr, ws, s);
     return launch_fwd_simt(*p, q, k, v, mask, h_full, h_sparse, delta, lse_full, lse_sparse,
                            sqdiff, s);
+}
+
+int ssa_attn_fwd_dual_diag(const ssa_params_t* p, const void* q, const void* k, const void* v,
+                           const int32_t* idx, const int32_t* cnt, const uint32_t* mask,
+                           void* h_full, void* h_sparse, float* delta, float* lse_full,
+                           float* lse_sparse, float* sqdiff, float* sink_rows, float* head_stats,
+                           void* ws, size_t ws_bytes, void* stream) {
+    g_last_error[0] = 0;
+    SSA_TRY(validate(p));
+    SSA_TRY(need_ptr(sink_rows, "sink_rows"));
+    SSA_TRY(need_ptr(head_stats, "head_stats"));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!use_tc(*p)) {  // CUDA-core path: the dual forward, then the diagnostics pass
+        SSA_TRY(ssa_attn_fwd_dual(p, q, k, v, idx, cnt, mask, h_full, h_sparse, delta, lse_full,
+                                  lse_sparse, sqdiff, ws, ws_bytes, stream));
+        return launch_diagnostics(*p, q, k, lse_full, delta, sink_rows, head_stats, s);
+    }
+    SSA_TRY(need_ptr(q, "q"));
+    SSA_TRY(need_ptr(k, "k"));
+    SSA_TRY(need_ptr(v, "v"));
+    SSA_TRY(opt_ptr(idx, "idx"));
+    SSA_TRY(opt_ptr(cnt, "cnt"));
+    SSA_TRY(need_ptr(mask, "mask"));
+    SSA_TRY(need_ptr(h_full, "h_full"));
+    SSA_TRY(need_ptr(h_sparse, "h_sparse"));
+    SSA_TRY(need_ptr(delta, "delta"));
+    SSA_TRY(need_ptr(lse_full, "lse_full"));
+    SSA_TRY(need_ptr(lse_sparse, "lse_sparse"));
+    SSA_TRY(need_ptr(sqdiff, "sqdiff_rows"));
+    SSA_TRY(need_ws(ws, ws_bytes, fwd_workspace(*p), "ssa_attn_fwd_dual_diag"));
+    SSA_TRY(launch_fwd_tc(*p, q, k, v, mask, h_full, h_sparse, delta, lse_full, lse_sparse, sqdiff,
+                          sink_rows, ws, s));
+    return launch_diag_heads(*p, delta, sink_rows, head_stats, s);
 }
 
 int ssa_attn_fwd_sparse(const ssa_params_t* p, const void* q, const void* k, const void* v,

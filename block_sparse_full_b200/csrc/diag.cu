@@ -159,7 +159,12 @@ int launch_diagnostics(const ssa_params_t& p, const void* q, const void* k, cons
         st = kpl == 4 ? go(diag_sink_kernel<float, 4>, qp, kp) : go(diag_sink_kernel<float, 2>, qp, kp);
     }
     if (st != SSA_OK) return st;
-    diag_head_kernel<<<BH, kThreads, 0, s>>>(delta, sink, p.T, stats);
+    return launch_diag_heads(p, delta, sink, stats, s);
+}
+
+int launch_diag_heads(const ssa_params_t& p, const float* delta, const float* sink, float* stats,
+                      cudaStream_t s) {
+    diag_head_kernel<<<p.B * p.H, kThreads, 0, s>>>(delta, sink, p.T, stats);
     return check_launch("diag_head_kernel");
 }
 

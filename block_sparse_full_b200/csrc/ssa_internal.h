@@ -53,8 +53,8 @@ bool fwd_tc_supported(const ssa_params_t& p);
 size_t fwd_tc_workspace(const ssa_params_t& p);
 int launch_fwd_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
                   const uint32_t* mask, void* h_full, void* h_sparse, float* delta,
-                  float* lse_full, float* lse_sparse, float* sqdiff, void* ws,
-                  cudaStream_t s);
+                  float* lse_full, float* lse_sparse, float* sqdiff, float* sink, void* ws,
+                  cudaStream_t s);  // sink: optional block-0 mass per row
 int fwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
 // the sparse stream alone (inference): h_sparse and lse_sparse only
 int launch_fwd_sparse_tc(const ssa_params_t& p, const void* q, const void* k, const void* v,
@@ -71,6 +71,9 @@ int launch_decode_step(const ssa_params_t& p, int t, const void* q, const void* 
 // ---- attention diagnostics (diag.cu)
 int launch_diagnostics(const ssa_params_t& p, const void* q, const void* k, const float* lse_full,
                        const float* delta, float* sink, float* stats, cudaStream_t s);
+// per-head means of delta and of the sink mass from the row vectors (fixed-order float64)
+int launch_diag_heads(const ssa_params_t& p, const float* delta, const float* sink, float* stats,
+                      cudaStream_t s);
 
 // ---- alignment loss (loss.cu)
 size_t loss_workspace(const ssa_params_t& p);

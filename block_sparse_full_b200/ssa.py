@@ -34,7 +34,8 @@ SSA_WS_SELECT, SSA_WS_FWD, SSA_WS_LOSS, SSA_WS_BWD, SSA_WS_FWD_SPARSE, SSA_WS_DE
 # every symbol include/ssa.h declares
 EXPORTS = (
     "ssa_workspace_size", "ssa_select_blocks", "ssa_select_blocks_noalloc",
-    "ssa_attn_fwd_dual", "ssa_attn_fwd_sparse", "ssa_attn_diagnostics", "ssa_decode_pool",
+    "ssa_attn_fwd_dual", "ssa_attn_fwd_sparse", "ssa_attn_diagnostics", "ssa_attn_fwd_dual_diag",
+    "ssa_decode_pool",
     "ssa_decode_step", "ssa_align_loss",
     "ssa_attn_bwd", "ssa_device_status", "ssa_status_string", "ssa_last_error",
     "ssa_kernel_path", "ssa_bwd_heads_per_group", "ssa_selftest_math", "ssa_selftest_wait_timeout",
@@ -72,6 +73,10 @@ _SIGNATURES = {
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "ssa_attn_diagnostics": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                      c_void_p, c_void_p]),
+    "ssa_attn_fwd_dual_diag": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                       c_void_p]),
     "ssa_decode_pool": (c_int, [_P, c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "ssa_decode_step": (c_int, [_P, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -145,6 +150,13 @@ def ssa_attn_fwd_sparse(params, q, k, v, idx, cnt, mask, h_sparse, lse_sparse, w
 def ssa_attn_diagnostics(params, q, k, lse_full, delta, sink_rows, head_stats, stream):
     return _lib.ssa_attn_diagnostics(ctypes.byref(params), q, k, lse_full, delta, sink_rows,
                                      head_stats, stream)
+
+
+def ssa_attn_fwd_dual_diag(params, q, k, v, idx, cnt, mask, h_full, h_sparse, delta, lse_full,
+                           lse_sparse, sqdiff_rows, sink_rows, head_stats, ws, ws_bytes, stream):
+    return _lib.ssa_attn_fwd_dual_diag(ctypes.byref(params), q, k, v, idx, cnt, mask, h_full,
+                                       h_sparse, delta, lse_full, lse_sparse, sqdiff_rows,
+                                       sink_rows, head_stats, ws, ws_bytes, stream)
 
 
 def ssa_decode_pool(params, j0, j1, k_cache, kbar, stream):
@@ -319,6 +331,30 @@ def diagnostics(params, q, k, fwd):
     check(ssa_attn_diagnostics(params, _ptr(q), _ptr(k), _ptr(fwd["lse_full"]), _ptr(fwd["delta"]),
                                _ptr(sink), _ptr(stats), _stream(dev)), "ssa_attn_diagnostics")
     return {"sink": sink, "head_stats": stats}
+
+
+def attn_fwd_dual_diag(params, q, k, v, mask, idx=None, cnt=None, ws=None, out=None):
+    """Both streams plus the diagnostics in one call -> the dict of
+    ``attn_fwd_dual`` with ``sink`` [B,H,T] and ``head_stats`` [B,H,2] added."""
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (mask, "mask")):
+        _need(t, nm)
+    dev = q.device
+    rows = (params.B, params.H, params.T)
+    if out is None:
+        out = {
+            "h_full": torch.empty_like(q), "h_sparse": torch.empty_like(q),
+            **{nm: torch.empty(rows, dtype=torch.float32, device=dev)
+               for nm in ("delta", "lse_full", "lse_sparse", "sqdiff", "sink")},
+            "head_stats": torch.empty((params.B, params.H, 2), dtype=torch.float32, device=dev),
+        }
+    ws = workspace(params, SSA_WS_FWD, dev) if ws is None else ws
+    check(ssa_attn_fwd_dual_diag(params, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt),
+                                 _ptr(mask), _ptr(out["h_full"]), _ptr(out["h_sparse"]),
+                                 _ptr(out["delta"]), _ptr(out["lse_full"]),
+                                 _ptr(out["lse_sparse"]), _ptr(out["sqdiff"]), _ptr(out["sink"]),
+                                 _ptr(out["head_stats"]), _ptr(ws), ws.numel(), _stream(dev)),
+          "ssa_attn_fwd_dual_diag")
+    return out
 
 
 class DecodeCache:

@@ -215,6 +215,23 @@ int ssa_attn_diagnostics(const ssa_params_t* params, const void* q, const void* 
                          float* head_stats, void* stream);
 
 /*
+ * ssa_attn_fwd_dual and ssa_attn_diagnostics in one call: the same outputs
+ * as the first (same arguments and workspace, SSA_WS_FWD) plus sink_rows and
+ * head_stats as the second defines them.  On the tensor-core path the
+ * forward kernel accumulates each row's weight on block 0 while it walks key
+ * tile 0 (rescaled with the running max like the row sums) and divides by
+ * the full normaliser at the end, so q and block 0 of k are not read again;
+ * one small kernel then forms the per-head means.  On the CUDA-core path it
+ * runs the two calls one after the other.
+ */
+int ssa_attn_fwd_dual_diag(const ssa_params_t* params, const void* q, const void* k,
+                           const void* v, const int32_t* idx, const int32_t* cnt,
+                           const uint32_t* mask, void* h_full, void* h_sparse, float* delta,
+                           float* lse_full, float* lse_sparse, float* sqdiff_rows,
+                           float* sink_rows, float* head_stats, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/*
  * Alignment losses (section 2, "Allineamento Bidirezionale"): with
  * N = B*H*T*D and L = sum(sqdiff_rows) / N (the mean squared difference of
  * the two outputs), writes loss_out[0] = w_sparsity * L (L_sparsity) and

@@ -221,17 +221,21 @@ def compare_loss(case, p, gpu_sqdiff, ref_loss, ref_sq, budget, n_total, w_s=2.0
     return errs
 
 
-def dq_rounding_budget(q, k, v, idx, cnt, block, scale, dh_full, dh_sparse, w_s, w_c, n_total):
+def dq_rounding_budget(q, k, v, idx, cnt, block, scale, dh_full, dh_sparse, w_s, w_c, n_total,
+                       rows=None):
     """Elementwise bound on the dq deviation that rounding the forward outputs
     to bf16 alone causes.  The backward takes D_f = G_f . h_full and
     D_s = G_s . h_sparse from the stored (bf16) outputs; a perturbation dD
     of D enters dq_t as -sigma * dD(t) * sum_s P(t,s) k_s, and that
     softmax-weighted mean key is the attention output with v := k.  All
-    values come from the oracle; the bf16 rounding is torch's on the host."""
-    ref = O.attn_fwd_dual(q, k, v, idx, cnt, block, scale)
-    kbar = O.attn_fwd_dual(q, k, k, idx, cnt, block, scale)
+    values come from the oracle; the bf16 rounding is torch's on the host.
+    ``rows`` restricts it to those query rows (each row's bound is its own)."""
+    ref = O.attn_fwd_dual(q, k, v, idx, cnt, block, scale, rows=rows)
+    kbar = O.attn_fwd_dual(q, k, k, idx, cnt, block, scale, rows=rows)
     hf, hs = ref["h_full"], ref["h_sparse"]
     r16 = lambda a: torch.from_numpy(a).to(torch.bfloat16).double().numpy()
+    if rows is not None:
+        dh_full, dh_sparse = dh_full[:, :, rows], dh_sparse[:, :, rows]
     g_f, g_s = O.alignment_upstream(hf, hs, dh_full, dh_sparse, w_s, w_c, n_total)
     dDf = (np.abs(g_f) * np.abs(hf - r16(hf))).sum(-1, keepdims=True)
     dDs = (np.abs(g_s) * np.abs(hs - r16(hs))).sum(-1, keepdims=True)
@@ -254,6 +258,7 @@ def compare_grads(case, dtype, got, want, dq_budget=None, names=("dq", "dk", "dv
         if name == "dq" and dq_budget is not None:
             allowed = allowed + 1.25 * dq_budget
             errs["dq_budget_ratio"] = float((diff / allowed).max())
+            errs["dq_plain_ratio"] = float(diff.max() / (tol * scale))  # against 2e-2 x max alone
         ok = diff <= allowed
         assert ok.all(), (f"{case} {name}: max err {diff.max():.3e} (tol {tol} x {scale:.3e}); "
                           f"worst at {np.unravel_index(np.argmax(diff - allowed), diff.shape)}")

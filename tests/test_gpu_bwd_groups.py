@@ -17,8 +17,8 @@ from block_sparse_full_b200 import ssa
 from block_sparse_full_b200.inputs import Workload, make_inputs, upstream_grads
 from oracle import ssa_oracle as O
 
-from gpu_parity_util import (DEV, assert_selection, compare_grads, oracle_select, params,
-                             sample_rows, to_dev)
+from gpu_parity_util import (DEV, assert_selection, compare_grads, dq_rounding_budget,
+                             oracle_select, params, sample_rows, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -62,9 +62,12 @@ def test_small_problem_in_head_groups(budget_heads, groups):
     inp, g, o_sel, hc, got, ws_, wc_ = _run(w, budget_heads, align=budget_heads == 2.5)
     assert hc == int(budget_heads)
     assert -(-w.B * w.H // hc) == groups
-    want = O.attn_bwd(inp["q"], inp["k"], inp["v"], o_sel[0], o_sel[1], w.block, w.sm_scale,
-                      g["dh_full"], g["dh_sparse"], ws_, wc_, n_total=inp["q"].numel())
-    compare_grads(f"bwd_groups/{groups}", "bf16", got, want)
+    args = (inp["q"], inp["k"], inp["v"], o_sel[0], o_sel[1], w.block, w.sm_scale,
+            g["dh_full"], g["dh_sparse"], ws_, wc_)
+    want = O.attn_bwd(*args, n_total=inp["q"].numel())
+    budget = dq_rounding_budget(*(O.f64(a) if isinstance(a, torch.Tensor) else a for a in args),
+                                n_total=inp["q"].numel())
+    compare_grads(f"bwd_groups/{groups}", "bf16", got, want, dq_budget=budget)
 
 
 def test_grouped_results_equal_one_group():
@@ -88,8 +91,10 @@ def test_real_grouped_shape_T32768():
     n = inp["q"].numel()
     rows = sample_rows(w.T, 4096, 6, seed=43)
     dq, _, _ = O.attn_bwd(*args, n_total=n, rows=rows)
+    budget = dq_rounding_budget(*(O.f64(a) if isinstance(a, torch.Tensor) else a for a in args),
+                                n_total=n, rows=rows)
     compare_grads("bwd_groups/T32768/dq_rows", "bf16", [sub(got[0])[:, :, rows]],
-                  [dq[:, :, rows]], names=("dq",))
+                  [dq[:, :, rows]], dq_budget=budget, names=("dq",))
     tail = np.arange(w.T - 256, w.T)  # keys that only the last 256 query rows see
     _, dk, dv = O.attn_bwd(*args, n_total=n, rows=tail)
     compare_grads("bwd_groups/T32768/dkdv_tail", "bf16",
