@@ -6,21 +6,18 @@
 // same layer; section 1: the sparse stream normalises over the selected
 // subset only).
 //
-// CTA = (query tile of 128 rows, batch*head), 640 threads:
+// CTA = (query tile of 128 rows, batch*head), 384 threads:
 //   warps 0, 2  TMA producers: Q once and K_j (warp 0), V_j (warp 2), into
 //               2-stage rings
 //   warp 1      TMEM owner and MMA issuer (one thread):
 //                 S_j = Q K_j^T          (tcgen05 SS, into S buffer j%2)
-//                 O_sel/O_uns += P_j V_j  (tcgen05 TS, P read from TMEM), the
-//                 MMAs of each 64-key half issued as soon as that half's P is in
-//   warps 4..19 four softmax warpgroups, warpgroup g taking keys
-//               [32g, 32g + 32) of every tile and output columns
-//               [g D/4, (g+1) D/4): thread = query row = TMEM lane.  They read
-//               S_j, keep one running max for both streams (combined through
-//               shared memory once per tile), split the row sum into l_sel /
-//               l_uns by the selection mask and write P_j (bf16) back into
-//               the S buffer for the PV product.  Four warps per scheduler
-//               hide the latency of the exponentials and the TMEM traffic.
+//                 O_sel/O_uns += P_j V_j  (tcgen05 TS, P read from TMEM)
+//   warps 4..11 two softmax warpgroups, warpgroup h taking keys
+//               [64h, 64h + 64) of every tile: thread = query row = TMEM
+//               lane.  They read S_j, keep one running max for both streams
+//               (combined through shared memory once per tile), split the row
+//               sum into l_sel / l_uns by the selection mask and write P_j
+//               (bf16) back into the S buffer for the PV product.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O_sel [256,384) O_uns [384,512).
 //
 // A 128-key tile holds one or two key blocks and the 128 query rows one or
@@ -32,6 +29,10 @@
 // The running max is only raised (and O rescaled) when a row's tile max
 // exceeds it by more than 2^8; the final normalisation divides by sums taken
 // against the same stale max, so the result is unchanged.
+//
+// Optionally (ssa_attn_fwd_dual_diag) each row's weight on block 0 is summed
+// while key tile 0 is processed, rescaled with the row sums, and divided by
+// the full normaliser in the epilogue: the attention-sink mass.
 //
 // Every mbarrier wait is bounded (wall-clock limit); on expiry the kernel
 // records SSA_ERR_TIMEOUT in a device status word, the other roles stop,
@@ -52,10 +53,8 @@ using namespace tc;
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
 constexpr int HD = 128;  // largest head dim (the shared-memory layout is sized for it)
-constexpr int kNWG = 4;                      // softmax warpgroups
-constexpr int kKW = BN / kNWG;               // keys of a tile per warpgroup (32)
-constexpr int kSoftmax = 128 * kNWG;         // softmax threads (512)
-constexpr int kThreads = 128 + kSoftmax;     // warps 0-2 roles, 3 idle, 4-19 softmax
+constexpr int kThreads = 384;  // warps 0-2 roles, 3 idle, 4-11 two softmax warpgroups
+constexpr int kSoftmax = 256;
 constexpr uint32_t TILE_BYTES = BM * HD * 2;  // 32 KB ring slot (half used at d = 64)
 constexpr uint32_t HALF_BYTES = 128 * 128;    // [128 rows x 64 cols] bf16 box, 16 KB
 constexpr int kMaxWords = 256;                // mask words per query block (n <= 8192)
@@ -64,20 +63,19 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + TILE_BYTES;
 constexpr uint32_t OFF_V = OFF_K + 2 * TILE_BYTES;
 constexpr uint32_t OFF_BAR = OFF_V + 2 * TILE_BYTES;
-constexpr int NBAR = 24;
+constexpr int NBAR = 16;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;  // [0] tmem base, [1] abort flag
 constexpr uint32_t OFF_MASK = OFF_MISC + 16;       // mask rows of the two query blocks
-// warpgroup exchange area, 2048 f32: row maxima [parity][wg][row] (1024), then in
-// the epilogue l_sel/l_uns [wg][2][row] (1024) and squared-difference sums
-// [wg][row] at offset 1024 (512)
+// warpgroup exchange area, 1024 f32: row maxima [parity][wg][row] (512), then in
+// the epilogue l_sel/l_uns [wg][2][row] (512), squared-difference sums [wg][row]
+// at offset 512 (256) and block-0 weights [wg][row] at offset 768 (256)
 constexpr uint32_t OFF_XCH = OFF_MASK + 2 * kMaxWords * 4;
-constexpr uint32_t SMEM_USED = OFF_XCH + 2048 * 4;
+constexpr uint32_t SMEM_USED = OFF_XCH + 1024 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 
-enum : int {  // barrier indices (two-stage K / V rings, two S buffers; P ready per
-              // S buffer and 64-key half: B_PREADY + 2 b + h)
+enum : int {  // barrier indices (two-stage K / V rings, two S buffers)
     B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7,
-    B_SREADY = 9, B_PREADY = 11, B_PVDONE = 15, B_DRAIN = 16, B_COUNT = 17
+    B_SREADY = 9, B_PREADY = 11, B_PVDONE = 13, B_DRAIN = 14, B_COUNT = 15
 };
 static_assert(B_COUNT <= NBAR, "barrier area");
 
@@ -129,7 +127,7 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
 }
 
 // D: head dim, 64 or 128 (one or two 64-column boxes per tile; an S tile
-// takes D/16 MMA k-steps; each softmax warpgroup owns D/4 output columns).
+// takes D/16 MMA k-steps; each softmax warpgroup owns D/2 output columns).
 // kSparse = false: the dual forward (both streams).  kSparse = true: the
 // sparse stream alone (inference, the same operations as MoBA): key tiles
 // that neither of the tile's query blocks selects are skipped by every
@@ -171,8 +169,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mbar_init(BAR(B_VFULL + s), 1);
             mbar_init(BAR(B_VEMPTY + s), 1);
             mbar_init(BAR(B_SREADY + s), 1);
-            mbar_init(BAR(B_PREADY + 2 * s), kSoftmax / 2);      // warpgroups 0, 1
-            mbar_init(BAR(B_PREADY + 2 * s + 1), kSoftmax / 2);  // warpgroups 2, 3
+            mbar_init(BAR(B_PREADY + s), kSoftmax);
         }
         mbar_init(BAR(B_PVDONE), 1);
         mbar_init(BAR(B_DRAIN), 1);
@@ -269,17 +266,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         auto issue_pv = [&](int i, int ii) -> bool {  // key tile i, ii-th processed
             const int b = ii & 1;
             const uint32_t ph = (ii >> 1) & 1;
+            if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY + b), ph, abort_flag, status, lim))) return false;
             if (!__all_sync(FULL, mbar_wait(BAR(B_VFULL + b), ph, abort_flag, status, lim))) return false;
+            fence_after_sync();
             const uint64_t vd = desc_add(vdesc0, b * TILE_BYTES);
             const uint32_t sb = tmem + (b ? TM_S1 : TM_S0);
+            bool s0[2], s1[2];
+            half_sel(mrow, i, I, 0, a.block, ragged1, s0[0], s1[0]);
+            half_sel(mrow, i, I, 1, a.block, ragged1, s0[1], s1[1]);
+            if (elect_one()) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {  // each half as soon as its two warpgroups wrote P
-                if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY + 2 * b + h), ph, abort_flag, status, lim)))
-                    return false;
-                fence_after_sync();
-                bool s0, s1;
-                half_sel(mrow, i, I, h, a.block, ragged1, s0, s1);
-                if (elect_one()) {
+                for (int h = 0; h < 2; ++h) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t bd = desc_add(vd, (4 * h + kk) * 2048);
@@ -287,21 +284,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         // the complementary ("alt") copy of a mixed half in the next 32
                         const uint32_t pa = sb + 64 * h + 8 * kk;
                         if (kSparse) {  // rows that do not select the half hold P = 0
-                            if (s0 || s1) mma_ts(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
-                        } else if (s0 == s1) {
-                            mma_ts(tmem + (s0 ? TM_OSEL : TM_OUNS), pa, bd, idesc_pv, 1);
+                            if (s0[h] || s1[h]) mma_ts(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
+                        } else if (s0[h] == s1[h]) {
+                            mma_ts(tmem + (s0[h] ? TM_OSEL : TM_OUNS), pa, bd, idesc_pv, 1);
                         } else {
                             mma_ts(tmem + TM_OSEL, pa, bd, idesc_pv, 1);
                             mma_ts(tmem + TM_OUNS, pa + 32, bd, idesc_pv, 1);
                         }
                     }
-                    if (h == 1) {
-                        mma_commit(BAR(B_VEMPTY + b));
-                        mma_commit(BAR(B_PVDONE));
-                    }
                 }
-                __syncwarp();
+                mma_commit(BAR(B_VEMPTY + b));
+                mma_commit(BAR(B_PVDONE));
             }
+            __syncwarp();
             return true;
         };
         int jj = 0, jprev = -1;
@@ -335,43 +330,42 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         __syncwarp();
         wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
     } else if (warp >= 4) {
-        // ------------------------------------------ four softmax warpgroups
-        // Warpgroup g owns keys [32g, 32g + 32) of every tile (inside 64-key half
-        // hh = g / 2) and columns [g OC, (g+1) OC) of O_sel / O_uns.  The row max
-        // is combined through shared memory once per tile; l_sel / l_uns and the
-        // squared difference are combined in the epilogue.
+        // ------------------------------------------- two softmax warpgroups
+        // Warpgroup h (= wg) owns keys [64h, 64h+64) of every tile and the
+        // columns [64h, 64h+64) of O_sel / O_uns.  The row max is combined
+        // through shared memory once per tile; l_sel / l_uns and the squared
+        // difference are combined in the epilogue.
         const int wg = (warp - 4) >> 2, sw = (warp - 4) & 3;
         const int r = sw * 32 + lane;  // row of the tile == TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
-        const int hh = wg >> 1;              // the 64-key half this warpgroup's keys lie in
-        const int c0 = kKW * wg;             // this warpgroup's S columns (keys)
-        // its bf16 P columns: half hh's P takes the first 32 columns of the half's
-        // 64-column S range (16 per warpgroup), the alt copy of a mixed half the next 32
-        const uint32_t pcol = 64u * hh + 16u * (wg & 1);
-        constexpr int OC = D / kNWG;         // and its O columns (32 or 16)
+        const int c0 = 64 * wg;          // this warpgroup's S columns (keys)
+        constexpr int OC = D / 2;        // and its O columns
         const int oc0 = OC * wg;
         float* xch = reinterpret_cast<float*>(gbase + OFF_XCH);  // [parity][wg][row]
-        // named barrier of the softmax warpgroups; wg_vote also ORs a flag across them
-        // so that all always leave the tile loop at the same tile (same barrier count)
-        auto wg_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kSoftmax) : "memory"); };
+        // named barrier of the two warpgroups; wg_vote also ORs a flag across them so
+        // that both always leave the tile loop at the same tile (same barrier count)
+        auto wg_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
         auto wg_vote = [](bool flag) -> bool {
             uint32_t out;
             asm volatile(
                 "{\n\t.reg .pred p, q;\n\t"
                 "setp.ne.u32 q, %1, 0;\n\t"
-                "bar.red.or.pred p, 1, %2, q;\n\t"
+                "bar.red.or.pred p, 1, 256, q;\n\t"
                 "selp.u32 %0, 1, 0, p;\n\t}"
                 : "=r"(out)
-                : "r"((uint32_t)flag), "n"(kSoftmax)
+                : "r"((uint32_t)flag)
                 : "memory");
             return out != 0;
         };
         {
-            uint32_t z[OC];
+            uint32_t z[32];
 #pragma unroll
-            for (int i = 0; i < OC; ++i) z[i] = 0u;
-            tmem_st<OC>(trow + TM_OSEL + oc0, z);
-            tmem_st<OC>(trow + TM_OUNS + oc0, z);
+            for (int i = 0; i < 32; ++i) z[i] = 0u;
+#pragma unroll
+            for (int x = 0; x < OC / 32; ++x) {
+                tmem_st32(trow + TM_OSEL + oc0 + 32 * x, z);
+                tmem_st32(trow + TM_OUNS + oc0 + 32 * x, z);
+            }
             tmem_wait_st();
         }
         const float sl2 = a.scale_log2;
@@ -388,51 +382,53 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // warp-uniform outcome: the TMEM loads below are warp-collective
             const bool got = __all_sync(
                 0xffffffffu, mbar_wait(BAR(B_SREADY + b), (jj >> 1) & 1, abort_flag, status, lim));
-            const uint32_t sbase = trow + (b ? TM_S1 : TM_S0);
-            float s[kKW];
+            const uint32_t sb = trow + (b ? TM_S1 : TM_S0) + c0;
+            float s[64];
             if (got) {
                 fence_after_sync();
-                uint32_t u[kKW];
-                tmem_ld32(sbase + c0, u);
+                uint32_t u0[32], u1[32];
+                tmem_ld32(sb, u0);
+                tmem_ld32(sb + 32, u1);
                 tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < kKW; ++c) s[c] = __uint_as_float(u[c]);
+                for (int c = 0; c < 32; ++c) {
+                    s[c] = __uint_as_float(u0[c]);
+                    s[32 + c] = __uint_as_float(u1[c]);
+                }
             } else {
 #pragma unroll
-                for (int c = 0; c < kKW; ++c) s[c] = 0.f;
+                for (int c = 0; c < 64; ++c) s[c] = 0.f;
             }
             if (j == I) {  // diagonal tile: keys after the row are masked (and keys >= T)
 #pragma unroll
-                for (int c = 0; c < kKW; ++c)
+                for (int c = 0; c < 64; ++c)
                     if (c0 + c > r) s[c] = -INFINITY;
             }
             bool s0, s1;
-            half_sel(mrow, j, I, hh, a.block, ragged1, s0, s1);
+            half_sel(mrow, j, I, wg, a.block, ragged1, s0, s1);
             const bool mixed = s0 != s1;
             const bool row_sel = mixed ? ((r < 64 || a.block == 128) ? s0 : s1) : s0;
             if (kSparse && !row_sel) {  // the sparse stream alone: this half is not attended
 #pragma unroll
-                for (int c = 0; c < kKW; ++c) s[c] = -INFINITY;
+                for (int c = 0; c < 64; ++c) s[c] = -INFINITY;
             }
             float mx8[8];  // independent partial maxima (short dependency chains)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mx8[k] = max3(s[k], s[8 + k], fmaxf(s[16 + k], s[24 + k]));
+            for (int k = 0; k < 8; ++k) {
+                mx8[k] = max3(s[k], s[8 + k], s[16 + k]);
+                mx8[k] = max3(mx8[k], s[24 + k], s[32 + k]);
+                mx8[k] = max3(mx8[k], s[40 + k], s[48 + k]);
+                mx8[k] = fmaxf(mx8[k], s[56 + k]);
+            }
             float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]),
                             fmaxf(mx8[6], mx8[7]));
-            float* xm = xch + (jj & 1) * (kNWG * 128);
+            float* xm = xch + (jj & 1) * 256;
             xm[wg * 128 + r] = mx;
-            // The vote is also the point after which P may be written: every
-            // warpgroup has its S columns in registers (a mixed half's alt copy
-            // goes over the S columns of the half's other warpgroup).
-            fence_before_sync();
-            if (wg_vote(!got || *abort_flag)) {  // a wait expired somewhere: all leave here
+            if (wg_vote(!got || *abort_flag)) {  // a wait expired somewhere: both leave here
                 ok = false;
                 break;
             }
-            fence_after_sync();
-#pragma unroll
-            for (int g = 0; g < kNWG; ++g)
-                if (g != wg) mx = fmaxf(mx, xm[g * 128 + r]);
+            mx = fmaxf(mx, xm[(1 - wg) * 128 + r]);
             const float mnew = mx * sl2;
             if (jj == 0) {
                 m2 = mnew;
@@ -451,15 +447,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     lsel *= alpha;
                     luns *= alpha;
                     lsink *= alpha;
+                    constexpr int NCH = OC / 32;  // 32-column chunks per accumulator
 #pragma unroll 1
-                    for (int c = 0; c < (kSparse ? 1 : 2); ++c) {
-                        const uint32_t col = (c == 0 ? TM_OSEL : TM_OUNS) + oc0;
-                        uint32_t u[OC];
-                        tmem_ld<OC>(trow + col, u);
+                    for (int c = 0; c < (kSparse ? NCH : 2 * NCH); ++c) {
+                        const uint32_t col = (c < NCH ? TM_OSEL : TM_OUNS) + oc0 + 32 * (c % NCH);
+                        uint32_t u[32];
+                        tmem_ld32(trow + col, u);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < OC; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-                        tmem_st<OC>(trow + col, u);
+                        for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+                        tmem_st32(trow + col, u);
                     }
                     tmem_wait_st();
                 }
@@ -474,13 +471,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             // the MUFU, whose 2^-inf = 0 keeps masked keys exact.
             const f32x2 sl2x2 = mk2(sl2, sl2), nm2 = mk2(negm, negm);
             f32x2 acc[4] = {mk2(0.f, 0.f), mk2(0.f, 0.f), mk2(0.f, 0.f), mk2(0.f, 0.f)};
-            uint32_t pk[kKW / 2];
+            uint32_t pk[32];
             if (zero_p) {
 #pragma unroll
-                for (int c = 0; c < kKW / 2; ++c) pk[c] = 0u;
+                for (int c = 0; c < 32; ++c) pk[c] = 0u;
             } else if (j == I) {
 #pragma unroll
-                for (int c = 0; c < kKW / 2; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     float x0, x1;
                     un2(fma2(mk2(s[2 * c], s[2 * c + 1]), sl2x2, nm2), x0, x1);
                     const float p0 = ex2(x0), p1 = ex2(x1);
@@ -489,7 +486,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < kKW / 2; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     const f32x2 x2 = fma2(mk2(s[2 * c], s[2 * c + 1]), sl2x2, nm2);
                     float p0, p1;
                     if (poly_pair(c)) {
@@ -509,23 +506,23 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             un2(add2(acc[2], acc[3]), b0, b1);
             const float sum = (a0 + a1) + (b0 + b1);
             if (kSparse || !mixed) {
-                tmem_st<kKW / 2>(sbase + pcol, pk);
+                tmem_st32(sb, pk);
             } else {
-                uint32_t main_[kKW / 2], alt[kKW / 2];
+                uint32_t main_[32], alt[32];
 #pragma unroll
-                for (int c = 0; c < kKW / 2; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     main_[c] = row_sel ? pk[c] : 0u;
                     alt[c] = row_sel ? 0u : pk[c];
                 }
-                tmem_st<kKW / 2>(sbase + pcol, main_);
-                tmem_st<kKW / 2>(sbase + pcol + 32, alt);
+                tmem_st32(sb, main_);
+                tmem_st32(sb + 32, alt);
             }
             if (row_sel) lsel += sum;
             else luns += sum;
             if (j == 0 && sink_keys) lsink = sum;
             tmem_wait_st();
             fence_before_sync();
-            mbar_arrive(BAR(B_PREADY + 2 * b + hh));
+            mbar_arrive(BAR(B_PREADY + b));
             ++jj;
         }
         // Every MMA (the last PV included) has completed once B_DRAIN has.  A
@@ -533,95 +530,90 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // only knows that the PV two tiles back has landed, and a barrier one
         // phase behind reports the wanted parity as complete.
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(BAR(B_DRAIN), 0, abort_flag, status, lim));
-        // all warpgroups take the same decision and the same barriers below
+        // both warpgroups take the same decision and the same barriers below
         ok = !wg_vote(!ok || *abort_flag);
         float* xl = xch;  // [wg][sel|uns][row] reuses the max exchange area
         xl[(wg * 2) * 128 + r] = lsel;
         xl[(wg * 2 + 1) * 128 + r] = luns;
         wg_sync();
-        float Ls = 0.f, Lu = 0.f;
-#pragma unroll
-        for (int g = 0; g < kNWG; ++g) {  // the same order in every warpgroup
-            Ls += xl[(g * 2) * 128 + r];
-            Lu += xl[(g * 2 + 1) * 128 + r];
-        }
+        const float Ls = lsel + xl[((1 - wg) * 2) * 128 + r];
         const int t = t0 + r;
         const bool valid = t < a.T;
         const size_t row = (size_t)bh * a.T + (valid ? t : 0);
-        constexpr int NV4 = OC / 8;  // 16-byte stores per output row segment
         if constexpr (kSparse) {
             // the diagonal block holds key t itself, so Ls > 0 on valid rows
             if (ok) {
                 fence_after_sync();
                 const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
-                uint32_t os[OC];
-                tmem_ld<OC>(trow + TM_OSEL + oc0, os);
-                tmem_wait_ld();
-                uint32_t hs[OC / 2];
+#pragma unroll 1
+                for (int c = 0; c < OC / 32; ++c) {
+                    uint32_t os[32];
+                    tmem_ld32(trow + TM_OSEL + oc0 + 32 * c, os);
+                    tmem_wait_ld();
+                    uint32_t hs[16];
 #pragma unroll
-                for (int e = 0; e < OC / 2; ++e)
-                    hs[e] = pack_bf16(__uint_as_float(os[2 * e]) * inv_ls,
-                                      __uint_as_float(os[2 * e + 1]) * inv_ls);
-                if (valid) {
-                    uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * D + oc0);
+                    for (int e = 0; e < 16; ++e)
+                        hs[e] = pack_bf16(__uint_as_float(os[2 * e]) * inv_ls,
+                                          __uint_as_float(os[2 * e + 1]) * inv_ls);
+                    if (valid) {
+                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * D + oc0 + 32 * c);
 #pragma unroll
-                    for (int v4 = 0; v4 < NV4; ++v4)
-                        ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
+                    }
                 }
                 if (wg == 0 && valid)
                     a.lse_sparse[row] = Ls > 0.f ? (m2 + log2f(Ls)) * kLn2 : -INFINITY;
             }
         } else {
+            const float Lu = luns + xl[((1 - wg) * 2 + 1) * 128 + r];
             float sq = 0.f;
             if (ok) {
                 fence_after_sync();
                 const float l = Ls + Lu;
                 const float inv_l = 1.f / l;
                 const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
-                uint32_t os[OC], ou[OC];
-                tmem_ld<OC>(trow + TM_OSEL + oc0, os);
-                tmem_ld<OC>(trow + TM_OUNS + oc0, ou);
-                tmem_wait_ld();
-                uint32_t hf[OC / 2], hs[OC / 2];
-#pragma unroll
-                for (int e = 0; e < OC / 2; ++e) {
-                    const float sa = __uint_as_float(os[2 * e]), sb2 = __uint_as_float(os[2 * e + 1]);
-                    const float ua = __uint_as_float(ou[2 * e]), ub = __uint_as_float(ou[2 * e + 1]);
-                    const float fa = (sa + ua) * inv_l, fb = (sb2 + ub) * inv_l;
-                    const float pa = sa * inv_ls, pb = sb2 * inv_ls;
-                    sq = fmaf(fa - pa, fa - pa, sq);
-                    sq = fmaf(fb - pb, fb - pb, sq);
-                    hf[e] = pack_bf16(fa, fb);
-                    hs[e] = pack_bf16(pa, pb);
-                }
-                if (valid) {
-                    uint4* df = reinterpret_cast<uint4*>(a.h_full + row * D + oc0);
-                    uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * D + oc0);
-#pragma unroll
-                    for (int v4 = 0; v4 < NV4; ++v4) {
-                        df[v4] = make_uint4(hf[4 * v4], hf[4 * v4 + 1], hf[4 * v4 + 2], hf[4 * v4 + 3]);
-                        ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
+    #pragma unroll 1
+                for (int c = 0; c < OC / 32; ++c) {
+                    uint32_t os[32], ou[32];
+                    tmem_ld32(trow + TM_OSEL + oc0 + 32 * c, os);
+                    tmem_ld32(trow + TM_OUNS + oc0 + 32 * c, ou);
+                    tmem_wait_ld();
+                    uint32_t hf[16], hs[16];
+    #pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float sa = __uint_as_float(os[2 * e]), sb2 = __uint_as_float(os[2 * e + 1]);
+                        const float ua = __uint_as_float(ou[2 * e]), ub = __uint_as_float(ou[2 * e + 1]);
+                        const float fa = (sa + ua) * inv_l, fb = (sb2 + ub) * inv_l;
+                        const float pa = sa * inv_ls, pb = sb2 * inv_ls;
+                        sq = fmaf(fa - pa, fa - pa, sq);
+                        sq = fmaf(fb - pb, fb - pb, sq);
+                        hf[e] = pack_bf16(fa, fb);
+                        hs[e] = pack_bf16(pa, pb);
+                    }
+                    if (valid) {
+                        uint4* df = reinterpret_cast<uint4*>(a.h_full + row * D + oc0 + 32 * c);
+                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * D + oc0 + 32 * c);
+    #pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            df[v4] = make_uint4(hf[4 * v4], hf[4 * v4 + 1], hf[4 * v4 + 2], hf[4 * v4 + 3]);
+                            ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
+                        }
                     }
                 }
             }
-            float* xs = xch + 2 * kNWG * 128;  // [wg][row] squared-difference partials
-            float* xk = xs + kNWG * 128;       // [wg][row] block-0 weight partials
+            float* xs = xch + 512;  // [wg][row] squared-difference partials
+            float* xk = xch + 768;  // [wg][row] block-0 weight partials
             xs[wg * 128 + r] = sq;
             xk[wg * 128 + r] = lsink;
             wg_sync();
             if (ok && wg == 0 && valid) {
                 const float l = Ls + Lu;
-                float sqt = 0.f, snk = 0.f;
-#pragma unroll
-                for (int g = 0; g < kNWG; ++g) {
-                    sqt += xs[g * 128 + r];
-                    snk += xk[g * 128 + r];
-                }
                 a.delta[row] = Lu / l;
                 a.lse_full[row] = (m2 + log2f(l)) * kLn2;
                 a.lse_sparse[row] = Ls > 0.f ? (m2 + log2f(Ls)) * kLn2 : -INFINITY;
-                a.sqdiff[row] = sqt;
-                if (a.sink) a.sink[row] = snk / l;
+                a.sqdiff[row] = sq + xs[128 + r];
+                if (a.sink) a.sink[row] = (lsink + xk[128 + r]) / l;
             }
         }
     }

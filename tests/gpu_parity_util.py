@@ -96,6 +96,9 @@ def compare_fwd(case, dtype, gpu, ref, rows=None, ref_abs=None):
         worst = np.unravel_index(np.argmax(dev - budget), dev.shape)
         assert (dev <= budget).all(), (f"{case} sqdiff: |gpu - oracle| {dev[worst]:.3e} > budget "
                                        f"{budget[worst]:.3e} (oracle {r[worst]:.3e}) at {worst}")
+        # and the losses' relative tolerance, row by row (float32 resolution as the floor)
+        rel = tol["loss_rel"] * r + 1e-12 * max(float(r.max()), 1e-30)
+        assert (dev <= rel).all(), f"{case} sqdiff: relative error above {tol['loss_rel']}"
         errs["sqdiff_budget_ratio"] = float((dev / budget).max())
         errs["sqdiff_rel_max"] = float((dev / np.maximum(r, 1e-30)).max(initial=0.0,
                                                                         where=r > 0))
@@ -208,6 +211,8 @@ def compare_loss(case, p, gpu_sqdiff, ref_loss, ref_sq, budget, n_total, w_s=2.0
     worst = np.unravel_index(np.argmax(dev - budget), dev.shape)
     assert (dev <= budget).all(), (f"{case} sqdiff: {dev[worst]:.3e} > budget {budget[worst]:.3e} "
                                    f"(oracle {ref_sq[worst]:.3e}) at {worst}")
+    rel = TOL["bf16"]["loss_rel"] * ref_sq + 1e-12 * max(float(ref_sq.max()), 1e-30)
+    assert (dev <= rel).all(), f"{case} sqdiff: relative error above {TOL['bf16']['loss_rel']}"
     loss = ssa.align_loss(p, gpu_sqdiff, w_s, w_c).cpu().numpy().astype(np.float64)
     allowed = min(budget.sum() / n_total, TOL["bf16"]["loss_rel"] * ref_loss)
     errs = {}
