@@ -137,7 +137,8 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
 template <int D, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const FwdArgs a) {
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_hf,
+              const __grid_constant__ CUtensorMap tm_hs, const FwdArgs a) {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
     constexpr uint32_t kTileBytes = BM * D * 2;  // bytes a Q / K / V tile load brings
     extern __shared__ uint8_t smem_raw[];
@@ -342,9 +343,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         constexpr int OC = D / 2;        // and its O columns
         const int oc0 = OC * wg;
         float* xch = reinterpret_cast<float*>(gbase + OFF_XCH);  // [parity][wg][row]
-        // named barrier of the two warpgroups; wg_vote also ORs a flag across them so
-        // that both always leave the tile loop at the same tile (same barrier count)
+        // named barrier of the two warpgroups; the votes also OR a flag across the
+        // warps they join, so that they leave the tile loop at the same tile (same
+        // barrier counts)
         auto wg_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+        // the per-tile row-max exchange only needs the two warps that hold the same
+        // 32 rows (warps 4 + sw and 8 + sw, on the same scheduler): barrier 2 + sw
+        auto pair_vote = [sw](bool flag) -> bool {
+            uint32_t out;
+            asm volatile(
+                "{\n\t.reg .pred p, q;\n\t"
+                "setp.ne.u32 q, %1, 0;\n\t"
+                "bar.red.or.pred p, %2, 64, q;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(out)
+                : "r"((uint32_t)flag), "r"(2 + sw)
+                : "memory");
+            return out != 0;
+        };
         auto wg_vote = [](bool flag) -> bool {
             uint32_t out;
             asm volatile(
@@ -424,7 +440,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                             fmaxf(mx8[6], mx8[7]));
             float* xm = xch + (jj & 1) * 256;
             xm[wg * 128 + r] = mx;
-            if (wg_vote(!got || *abort_flag)) {  // a wait expired somewhere: both leave here
+            if (pair_vote(!got || *abort_flag)) {  // a wait expired somewhere: both leave here
                 ok = false;
                 break;
             }
@@ -482,7 +498,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     un2(fma2(mk2(s[2 * c], s[2 * c + 1]), sl2x2, nm2), x0, x1);
                     const float p0 = ex2(x0), p1 = ex2(x1);
                     acc[c & 3] = add2(acc[c & 3], mk2(p0, p1));
-                    pk[c] = pack_bf16_alu(p0, p1);
+                    pk[c] = pack_bf16(p0, p1);
                 }
             } else {
 #pragma unroll
@@ -498,7 +514,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         p1 = ex2(x1);
                     }
                     acc[c & 3] = add2(acc[c & 3], mk2(p0, p1));
-                    pk[c] = pack_bf16_alu(p0, p1);
+                    pk[c] = pack_bf16(p0, p1);
                 }
             }
             float a0, a1, b0, b1;
@@ -540,6 +556,38 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int t = t0 + r;
         const bool valid = t < a.T;
         const size_t row = (size_t)bh * a.T + (valid ? t : 0);
+        // The output tiles go through shared memory (the K ring, free once every
+        // MMA has completed) in the 128-byte-swizzled [128 rows x 64 columns]
+        // boxes of the output tensor maps, and leave by TMA stores: a thread owns
+        // a row, so direct stores would scatter each warp's writes over 32 rows.
+        // Rows past T are clipped by the tensor map.
+        uint8_t* stage = gbase + OFF_K;  // h_sparse boxes, then h_full boxes (dual)
+        constexpr uint32_t kOutBytes = BM * D * 2;
+        const uint32_t rowoff = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
+        // 16-byte chunk v (8 columns) of output columns [col0, col0 + 32): box col/64
+        auto put = [&](uint8_t* tile, int col0, const uint32_t (&h)[16]) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int col = col0 + 8 * v;
+                const uint32_t chunk = (uint32_t)((col & 63) >> 3) ^ (uint32_t)(r & 7);
+                *reinterpret_cast<uint4*>(tile + (col >> 6) * HALF_BYTES + rowoff + chunk * 16) =
+                    make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+            }
+        };
+        // one thread stores the staged tile(s) once every row is written
+        auto store_tiles = [&](bool dual) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            wg_sync();
+            if (warp == 4 && lane == 0 && ok) {
+#pragma unroll
+                for (int x = 0; x < D / 64; ++x) {
+                    tma_store_3d(&tm_hs, base + OFF_K + x * HALF_BYTES, 64 * x, t0, bh);
+                    if (dual) tma_store_3d(&tm_hf, base + OFF_K + kOutBytes + x * HALF_BYTES, 64 * x, t0, bh);
+                }
+                bulk_commit_group();
+                bulk_wait_group_read0();  // the staging area stays valid until read
+            }
+        };
         if constexpr (kSparse) {
             // the diagonal block holds key t itself, so Ls > 0 on valid rows
             if (ok) {
@@ -555,16 +603,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     for (int e = 0; e < 16; ++e)
                         hs[e] = pack_bf16(__uint_as_float(os[2 * e]) * inv_ls,
                                           __uint_as_float(os[2 * e + 1]) * inv_ls);
-                    if (valid) {
-                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * D + oc0 + 32 * c);
-#pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4)
-                            ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
-                    }
+                    put(stage, oc0 + 32 * c, hs);
                 }
                 if (wg == 0 && valid)
                     a.lse_sparse[row] = Ls > 0.f ? (m2 + log2f(Ls)) * kLn2 : -INFINITY;
             }
+            store_tiles(false);
         } else {
             const float Lu = luns + xl[((1 - wg) * 2 + 1) * 128 + r];
             float sq = 0.f;
@@ -573,14 +617,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 const float l = Ls + Lu;
                 const float inv_l = 1.f / l;
                 const float inv_ls = Ls > 0.f ? 1.f / Ls : 0.f;
-    #pragma unroll 1
+#pragma unroll 1
                 for (int c = 0; c < OC / 32; ++c) {
                     uint32_t os[32], ou[32];
                     tmem_ld32(trow + TM_OSEL + oc0 + 32 * c, os);
                     tmem_ld32(trow + TM_OUNS + oc0 + 32 * c, ou);
                     tmem_wait_ld();
                     uint32_t hf[16], hs[16];
-    #pragma unroll
+#pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const float sa = __uint_as_float(os[2 * e]), sb2 = __uint_as_float(os[2 * e + 1]);
                         const float ua = __uint_as_float(ou[2 * e]), ub = __uint_as_float(ou[2 * e + 1]);
@@ -591,22 +635,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         hf[e] = pack_bf16(fa, fb);
                         hs[e] = pack_bf16(pa, pb);
                     }
-                    if (valid) {
-                        uint4* df = reinterpret_cast<uint4*>(a.h_full + row * D + oc0 + 32 * c);
-                        uint4* ds = reinterpret_cast<uint4*>(a.h_sparse + row * D + oc0 + 32 * c);
-    #pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4) {
-                            df[v4] = make_uint4(hf[4 * v4], hf[4 * v4 + 1], hf[4 * v4 + 2], hf[4 * v4 + 3]);
-                            ds[v4] = make_uint4(hs[4 * v4], hs[4 * v4 + 1], hs[4 * v4 + 2], hs[4 * v4 + 3]);
-                        }
-                    }
+                    put(stage, oc0 + 32 * c, hs);
+                    put(stage + kOutBytes, oc0 + 32 * c, hf);
                 }
             }
             float* xs = xch + 512;  // [wg][row] squared-difference partials
             float* xk = xch + 768;  // [wg][row] block-0 weight partials
             xs[wg * 128 + r] = sq;
             xk[wg * 128 + r] = lsink;
-            wg_sync();
+            store_tiles(true);  // (its barrier also publishes xs, xk)
             if (ok && wg == 0 && valid) {
                 const float l = Ls + Lu;
                 a.delta[row] = Lu / l;
@@ -670,10 +707,13 @@ template <int D, bool kSparse>
 int launch_fwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, const void* v,
                        const uint32_t* mask, const FwdArgs& outs, cudaStream_t s) {
     const int BH = p.B * p.H;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mhf, mhs;
     int st = make_map(&mq, q, BH, p.T, D);
     if (st == SSA_OK) st = make_map(&mk, k, BH, p.T, D);
     if (st == SSA_OK) st = make_map(&mv, v, BH, p.T, D);
+    if (st == SSA_OK) st = make_map(&mhs, outs.h_sparse, BH, p.T, D);
+    // the sparse-only kernel writes h_sparse alone (the h_full map is not used)
+    if (st == SSA_OK) st = make_map(&mhf, kSparse ? outs.h_sparse : outs.h_full, BH, p.T, D);
     if (st != SSA_OK) return st;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -693,7 +733,7 @@ int launch_fwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, cons
     a.scale_log2 = p.sm_scale * 1.4426950408889634f;
     a.timeout_ns = wait_limit_ns();
     const unsigned grid = (unsigned)((size_t)BH * ((p.T + BM - 1) / BM));
-    fwd_tc_kernel<D, kSparse><<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, a);
+    fwd_tc_kernel<D, kSparse><<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mhf, mhs, a);
     return check_launch(kSparse ? "fwd_tc_kernel<sparse>" : "fwd_tc_kernel");
 }
 }  // namespace
