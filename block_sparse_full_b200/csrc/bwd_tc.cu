@@ -96,29 +96,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
-// Writes 32*NCH fp32 columns of a TMEM accumulator row (from `trow_col`)
-// scaled by `mul` as bf16 to global memory at dst.
-template <int NCH>
-__device__ __forceinline__ void store_row_cols(uint32_t trow_col, float mul, __nv_bfloat16* dst,
-                                               bool valid) {
-#pragma unroll 1
-    for (int c = 0; c < NCH; ++c) {
-        uint32_t u[32];
-        tmem_ld32(trow_col + 32 * c, u);
-        tmem_wait_ld();
-        uint32_t o[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-            o[e] = pack_bf16(__uint_as_float(u[2 * e]) * mul, __uint_as_float(u[2 * e + 1]) * mul);
-        if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-                d4[v4] = make_uint4(o[4 * v4], o[4 * v4 + 1], o[4 * v4 + 2], o[4 * v4 + 3]);
-        }
-    }
-}
-
 // ============================================================ preprocess
 // One warp per row, lane owns D/32 consecutive columns.
 template <int D>
@@ -264,6 +241,7 @@ template <int D>
 __global__ void __launch_bounds__(kv::kThr, 1)
 bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_gf,
                    const __grid_constant__ CUtensorMap tm_gs, const __grid_constant__ CUtensorMap tm_ds,
+                   const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                    const BwdArgs a) {
     using namespace kv;
@@ -683,12 +661,28 @@ bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_arrive(BAR(B_DSREADY + b));
         }
         if (ok) ok = wait(B_DONE, 0);
-        if (ok) {
-            const size_t row = rowbase + (key_ok ? s_tok : 0);
+        // dV and dK leave through shared memory (the stage ring, idle once every
+        // MMA has completed) and TMA stores: a thread owns a key row, so direct
+        // stores would scatter each warp's writes over 32 rows.  Rows past T are
+        // clipped by the tensor maps.
+        const bool all_ok = bar_and(ok, 1, kComp);
+        uint8_t* stage = gbase + OFF_STAGE;
+        constexpr uint32_t kOutBytes = TILE * D * 2;
+        if (all_ok) {
             constexpr int OC = D / 2;  // output columns per warpgroup
-            store_row_cols<OC / 32>(trow + TM_DV + OC * wg, 1.f, a.dv + row * D + OC * wg, key_ok);
-            store_row_cols<OC / 32>(trow + TM_DK + OC * wg, a.sm_scale, a.dk + row * D + OC * wg,
-                                    key_ok);
+            stage_row_cols<OC / 32>(trow + TM_DV + OC * wg, 1.f, stage, OC * wg, r);
+            stage_row_cols<OC / 32>(trow + TM_DK + OC * wg, a.sm_scale, stage + kOutBytes, OC * wg, r);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        bar_sync(1, kComp);
+        if (all_ok && warp == 4 && lane == 0) {
+#pragma unroll
+            for (int x = 0; x < D / 64; ++x) {
+                tma_store_3d(&tm_dv, base + OFF_STAGE + x * BOX_T, 64 * x, s0, bh);
+                tma_store_3d(&tm_dk, base + OFF_STAGE + kOutBytes + x * BOX_T, 64 * x, s0, bh);
+            }
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging area stays valid until read
         }
     }
     fence_before_sync();
@@ -724,7 +718,7 @@ static_assert(B_COUNT <= 16, "barrier area holds 16");
 template <int D>
 __global__ void __launch_bounds__(dq::kThr, 1)
 bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_k,
-                   const BwdArgs a) {
+                   const __grid_constant__ CUtensorMap tm_dq, const BwdArgs a) {
     using namespace dq;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -743,7 +737,6 @@ bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_const
     const bool two = t0 + 64 < a.T;  // the tile's second 64-query step exists
     const int nj = I + 1;            // key tiles 0..I
     auto BAR = [&](int i) { return base + OFF_BAR + 8u * (uint32_t)i; };
-    const size_t rowbase = (size_t)bh * a.T;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
@@ -825,12 +818,22 @@ bwd_dq_gemm_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_const
         // ------------------------------------------ epilogue: warps 2-5 cover TMEM lanes
         const int sw = warp & 3;
         const int r = sw * 32 + lane;
-        const int t = t0 + r;
         const uint32_t trow = tmem + ((uint32_t)(sw * 32) << 16);
-        if (__all_sync(FULL, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim))) {
+        // dQ leaves through shared memory (the ring, idle once every MMA has
+        // completed) and TMA stores; rows past T are clipped by the tensor map
+        const bool ok = __all_sync(FULL, mbar_wait(BAR(B_DONE), 0, abort_flag, status, lim));
+        const bool all_ok = bar_and(ok, 1, 128);
+        if (all_ok) {
             fence_after_sync();
-            const bool valid = t < a.T;
-            store_row_cols<D / 32>(trow, a.sm_scale, a.dq + (rowbase + (valid ? t : 0)) * D, valid);
+            stage_row_cols<D / 32>(trow, a.sm_scale, gbase, 0, r);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        bar_sync(1, 128);
+        if (all_ok && warp == 2 && lane == 0) {
+#pragma unroll
+            for (int x = 0; x < D / 64; ++x) tma_store_3d(&tm_dq, base + x * BOX_T, 64 * x, t0, bh);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging area stays valid until read
         }
     }
     fence_before_sync();
@@ -982,8 +985,11 @@ int launch_bwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, cons
         auto off = [&](const void* ptr) {
             return static_cast<const void*>(static_cast<const __nv_bfloat16*>(ptr) + h0 * head_elems);
         };
-        CUtensorMap k128, q64, gf64, gs64, ds_map;
+        CUtensorMap k128, q64, gf64, gs64, ds_map, dq128, dk128, dv128;
         st = make_map(&k128, off(k), nh, p.T, TILE, D);
+        if (st == SSA_OK) st = make_map(&dq128, off(dq), nh, p.T, TILE, D);
+        if (st == SSA_OK) st = make_map(&dk128, off(dk), nh, p.T, TILE, D);
+        if (st == SSA_OK) st = make_map(&dv128, off(dv), nh, p.T, TILE, D);
         if (st == SSA_OK) st = make_map(&q64, off(q), nh, p.T, STEP, D);
         if (st == SSA_OK) st = make_map(&gf64, off(w.gf), nh, p.T, STEP, D);
         if (st == SSA_OK) st = make_map(&gs64, off(w.gs), nh, p.T, STEP, D);
@@ -1009,12 +1015,12 @@ int launch_bwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, cons
         a.timeout_ns = wait_limit_ns();
         const unsigned grid = (unsigned)((size_t)nh * ntile);
         bwd_dkdv_tc_kernel<D><<<grid, kv::kThr, kv::SMEM_BYTES, s>>>(
-            q64, gf64, gs64, ds_map, static_cast<const __nv_bfloat16*>(off(k)),
+            q64, gf64, gs64, ds_map, dk128, dv128, static_cast<const __nv_bfloat16*>(off(k)),
             static_cast<const __nv_bfloat16*>(off(v)), a);
         st = check_launch("bwd_dkdv_tc_kernel");
         if (st != SSA_OK) break;
         if (h0 == 0) mark_kernel_event(2, s);
-        bwd_dq_gemm_kernel<D><<<grid, dq::kThr, dq::SMEM_BYTES, s>>>(ds_map, k128, a);
+        bwd_dq_gemm_kernel<D><<<grid, dq::kThr, dq::SMEM_BYTES, s>>>(ds_map, k128, dq128, a);
         st = check_launch("bwd_dq_gemm_kernel");
         if (h0 == 0) mark_kernel_event(3, s);
     }

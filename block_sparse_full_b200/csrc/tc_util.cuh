@@ -318,6 +318,53 @@ __device__ __forceinline__ uint32_t pack_bf16_alu(float lo, float hi) {
     return r;
 }
 
+// bar.red.and over `count` threads of named barrier `id`: true iff every
+// participating thread passed true.
+__device__ __forceinline__ bool bar_and(bool flag, uint32_t id, uint32_t count) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(out)
+        : "r"((uint32_t)flag), "r"(id), "r"(count)
+        : "memory");
+    return out != 0;
+}
+__device__ __forceinline__ void bar_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Staged output tile for a TMA store: a [128 rows x D columns] bf16 tile kept
+// as [128 rows x 64 columns] boxes (16 KB apart) in the 128-byte-swizzled
+// layout of the tensor maps (row r at (r/8)*1024 + (r%8)*128, 16-byte chunk c
+// of the row at chunk c ^ (r%8)).  Writes 32*NCH float32 TMEM columns of row r
+// (from trow_col), scaled by mul and rounded to bf16, as output columns
+// [col0, col0 + 32*NCH).  Distinct rows of a warp land in distinct banks.
+template <int NCH>
+__device__ __forceinline__ void stage_row_cols(uint32_t trow_col, float mul, uint8_t* tile,
+                                               int col0, int r) {
+    const uint32_t rowoff = (uint32_t)(r >> 3) * 1024 + (uint32_t)(r & 7) * 128;
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c) {
+        uint32_t u[32];
+        tmem_ld32(trow_col + 32 * c, u);
+        tmem_wait_ld();
+        uint32_t o[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            o[e] = pack_bf16(__uint_as_float(u[2 * e]) * mul, __uint_as_float(u[2 * e + 1]) * mul);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int col = col0 + 32 * c + 8 * v;
+            const uint32_t chunk = (uint32_t)((col & 63) >> 3) ^ (uint32_t)(r & 7);
+            *reinterpret_cast<uint4*>(tile + (col >> 6) * (128 * 128) + rowoff + chunk * 16) =
+                make_uint4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- packed f32x2
 typedef unsigned long long f32x2;
 __device__ __forceinline__ f32x2 mk2(float a, float b) {
