@@ -10,16 +10,20 @@
 // the selected blocks up to t.
 //
 // Launches (CUDA cores: one query per head is matrix-vector work, bound by
-// the key/value bytes it reads):
+// the key/value bytes it reads and by latency):
 //   decode_pool_kernel     Kbar_j = mean of block j's keys (float64, exact)
-//   decode_select_kernel   one CTA per head: scores (warp per block, lanes
-//                          over d), then one warp fills the free slots by
-//                          warp-argmax rounds and writes the ascending list
-//   decode_attend_kernel   one CTA per (head, selected block): scores with a
+//   decode_select_kernel   CTA per (32 completed blocks, head): scores (warp
+//                          per block, lanes over d) to the workspace; the
+//                          head's last CTA to finish (a counter in the
+//                          workspace) fills the free slots by warp-argmax
+//                          rounds and writes the ascending list
+//   decode_attend_kernel   CTA per (head, selected block): scores with a
 //                          warp per group of keys (lanes over d), softmax
 //                          statistics CTA-wide, then P V with threads over
-//                          (d, key group)
-//   decode_combine_kernel  one warp per head merges the per-block partials
+//                          (d, key group); the head's last CTA to finish
+//                          merges the per-block partials into h and lse
+// The counters are cleared before each step (one memset) and by the CTA that
+// consumes them.
 #include <type_traits>
 
 #include "device_util.cuh"
@@ -48,41 +52,57 @@ decode_pool_kernel(const T* __restrict__ k, int Tcap, int D, int block, int j0,
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 decode_select_kernel(const T* __restrict__ q, const double* __restrict__ kbar, int nb, int i,
-                     int topk, bool force_sink, int32_t* __restrict__ sel,
+                     int topk, bool force_sink, double* __restrict__ score_g,
+                     unsigned int* __restrict__ counter, int32_t* __restrict__ sel,
                      int32_t* __restrict__ idx_out) {
     constexpr int M = D / 32;  // query columns per lane
     constexpr int U = 4;       // key blocks in flight per warp
+    constexpr int CHUNK = (kThreads / 32) * U;  // completed blocks per CTA
     extern __shared__ double score[];  // [max(i, 1)], then the set bitmask [i / 32 + 1]
+    __shared__ int is_last;
     uint32_t* bits = reinterpret_cast<uint32_t*>(score + (i > 0 ? i : 1));
-    const size_t bh = blockIdx.x;
+    const size_t bh = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int words = (i >> 5) + 1;  // bits 0 .. i
-    double qr[M];
+    double* sg = score_g + bh * (size_t)nb;
+    // scores of this CTA's completed blocks: warp per block, lane l owns columns
+    // l, l + 32, ... (coalesced rows of the float64 pooled keys), U blocks' loads
+    // in flight per warp, fixed butterfly sum
+    {
+        double qr[M];
 #pragma unroll
-    for (int m = 0; m < M; ++m) qr[m] = (double)to_f32(q[bh * D + lane + 32 * m]);
-    for (int w = threadIdx.x; w < words; w += kThreads) bits[w] = 0u;
-    // scores of the completed blocks: warp per block, lane l owns columns
-    // l, l + 32, ... (coalesced rows of the float64 pooled keys), U blocks'
-    // loads in flight per warp, fixed butterfly sum
-    const double* kb = kbar + bh * (size_t)nb * D;
-    for (int j0 = warp * U; j0 < i; j0 += (kThreads / 32) * U) {
-        double a[U];
+        for (int m = 0; m < M; ++m) qr[m] = (double)to_f32(q[bh * D + lane + 32 * m]);
+        const double* kb = kbar + bh * (size_t)nb * D;
+        const int j0 = CHUNK * blockIdx.x + U * warp;
+        if (j0 < i) {
+            double a[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const double* kr = kb + (size_t)min(j0 + u, i - 1) * D + lane;  // past the end: unused
-            double acc = 0.0;
+            for (int u = 0; u < U; ++u) {
+                const double* kr = kb + (size_t)min(j0 + u, i - 1) * D + lane;  // past the end: unused
+                double acc = 0.0;
 #pragma unroll
-            for (int m = 0; m < M; ++m) acc = fma(qr[m], kr[32 * m], acc);
-            a[u] = acc;
-        }
+                for (int m = 0; m < M; ++m) acc = fma(qr[m], kr[32 * m], acc);
+                a[u] = acc;
+            }
 #pragma unroll
-        for (int u = 0; u < U; ++u) a[u] = warp_sum(a[u]);
-        if (lane == 0) {
+            for (int u = 0; u < U; ++u) a[u] = warp_sum(a[u]);
+            if (lane == 0) {
 #pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (j0 + u < i) score[j0 + u] = a[u];
+                for (int u = 0; u < U; ++u)
+                    if (j0 + u < i) sg[j0 + u] = a[u];
+            }
         }
     }
+    // the head's last CTA to finish takes the selection
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(&counter[bh], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    for (int j = threadIdx.x; j < i; j += kThreads) score[j] = __ldcg(sg + j);
+    for (int w = threadIdx.x; w < words; w += kThreads) bits[w] = 0u;
+    if (threadIdx.x == 0) counter[bh] = 0u;  // ready for the next step
     __syncthreads();
     if (warp != 0) return;
     // one warp: forced blocks, the free slots by warp-argmax rounds, then the
@@ -160,7 +180,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
 decode_attend_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const int32_t* __restrict__ sel, int Tcap, int block, int t, int topk,
-                     float scale, float* __restrict__ part) {
+                     float scale, float* __restrict__ part, unsigned int* __restrict__ counter,
+                     T* __restrict__ h, float* __restrict__ lse) {
     constexpr int E = D / 32;            // columns per lane
     constexpr int NW = kThreads / 32;    // warps
     constexpr int KPW = 128 / NW;        // keys per warp (block <= 128)
@@ -243,42 +264,51 @@ decode_attend_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
         out[0] = nks > 0 ? m : -INFINITY;
         out[1] = l;
     }
-}
-
-// one warp per head: the partials' weights e^{m_a - M} are formed once
-template <typename T>
-__global__ void __launch_bounds__(32)
-decode_combine_kernel(const float* __restrict__ part, int D, int topk, T* __restrict__ h,
-                      float* __restrict__ lse) {
+    // the head's last CTA to finish merges the partials: weights e^{m_a - M}
+    __shared__ int is_last;
     __shared__ float wgt[kMaxTopk];
-    const size_t bh = blockIdx.x;
-    const int lane = threadIdx.x;
-    const float* p = part + bh * topk * (2 + D);
-    float M = -INFINITY;
-    for (int a = lane; a < topk; a += 32) M = fmaxf(M, p[a * (2 + D)]);
-    M = warp_max(M);
-    float L = 0.f;
-    for (int a = lane; a < topk; a += 32) {
-        const float ma = p[a * (2 + D)];
-        const float w = ma > -INFINITY ? expf(ma - M) : 0.f;
-        wgt[a] = w;
-        L += w * p[a * (2 + D) + 1];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) is_last = atomicAdd(&counter[bh], 1u) == (unsigned)topk - 1u;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    const float* pp = part + bh * topk * (2 + D);
+    if (warp == 0) {
+        float Mx = -INFINITY;
+        for (int a = lane; a < topk; a += 32) Mx = fmaxf(Mx, __ldcg(pp + a * (2 + D)));
+        Mx = warp_max(Mx);
+        float L = 0.f;
+        for (int a = lane; a < topk; a += 32) {
+            const float ma = __ldcg(pp + a * (2 + D));
+            const float w = ma > -INFINITY ? expf(ma - Mx) : 0.f;
+            wgt[a] = w;
+            L += w * __ldcg(pp + a * (2 + D) + 1);
+        }
+        L = warp_sum(L);
+        if (lane == 0) {
+            red[0] = L;
+            lse[bh] = Mx + logf(L);
+            counter[bh] = 0u;  // ready for the next step
+        }
     }
-    L = warp_sum(L);
-    __syncwarp();
-    for (int c = lane; c < D; c += 32) {
+    __syncthreads();
+    const float inv_L = 1.f / red[0];
+    for (int c = threadIdx.x; c < D; c += kThreads) {
         float acc = 0.f;
-        for (int a = 0; a < topk; ++a) acc = fmaf(wgt[a], p[a * (2 + D) + 2 + c], acc);
-        h[bh * D + c] = from_f32<T>(acc / L);
+        for (int a = 0; a < topk; ++a) acc = fmaf(wgt[a], __ldcg(pp + a * (2 + D) + 2 + c), acc);
+        h[bh * D + c] = from_f32<T>(acc * inv_L);
     }
-    if (lane == 0) lse[bh] = M + logf(L);
 }
 
 }  // namespace
 
+// selected indices [BH, topk] i32 | partials [BH, topk, 2 + D] f32 | scores
+// [BH, n] f64 | two counters per head
 size_t decode_workspace(const ssa_params_t& p) {
     const size_t bh = (size_t)p.B * p.H;
-    return align_up(bh * p.topk * 4, 256) + align_up(bh * p.topk * (2 + p.D) * 4, 256);
+    return align_up(bh * p.topk * 4, 256) + align_up(bh * p.topk * (2 + p.D) * 4, 256) +
+           align_up(bh * (size_t)num_blocks(p) * 8, 256) + align_up(bh * 2 * 4, 256);
 }
 
 int launch_decode_pool(const ssa_params_t& p, int j0, int j1, const void* k, double* kbar,
@@ -300,9 +330,16 @@ int launch_decode_step(const ssa_params_t& p, int t, const void* q, const void* 
                        cudaStream_t s) {
     const int BH = p.B * p.H;
     const int i = t / p.block;
-    int32_t* sel = static_cast<int32_t*>(ws);
-    float* part = reinterpret_cast<float*>(static_cast<char*>(ws) +
-                                           align_up((size_t)BH * p.topk * 4, 256));
+    char* w = static_cast<char*>(ws);
+    int32_t* sel = reinterpret_cast<int32_t*>(w);
+    w += align_up((size_t)BH * p.topk * 4, 256);
+    float* part = reinterpret_cast<float*>(w);
+    w += align_up((size_t)BH * p.topk * (2 + p.D) * 4, 256);
+    double* score_g = reinterpret_cast<double*>(w);
+    w += align_up((size_t)BH * num_blocks(p) * 8, 256);
+    unsigned int* counters = reinterpret_cast<unsigned int*>(w);  // [2][BH]
+    cudaError_t me = cudaMemsetAsync(counters, 0, (size_t)BH * 2 * 4, s);
+    if (me != cudaSuccess) return fail(SSA_ERR_CUDA, "decode: counters: %s", cudaGetErrorString(me));
     const size_t smem = (size_t)(i > 0 ? i : 1) * sizeof(double) + (size_t)((i >> 5) + 1) * 4;
     const bool sink = (p.flags & SSA_FLAG_FORCE_SINK) != 0;
     const int nb = num_blocks(p);
@@ -314,16 +351,16 @@ int launch_decode_step(const ssa_params_t& p, int t, const void* q, const void* 
             cudaError_t e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "decode: smem attribute: %s", cudaGetErrorString(e));
         }
-        sk<<<BH, kThreads, smem, s>>>(static_cast<const T*>(q), kbar, nb, i, p.topk, sink, sel, idx);
+        constexpr int kChunk = (kThreads / 32) * 4;  // completed blocks per select CTA
+        const unsigned chunks = (unsigned)(i > 0 ? (i + kChunk - 1) / kChunk : 1);
+        sk<<<dim3(chunks, (unsigned)BH), kThreads, smem, s>>>(
+            static_cast<const T*>(q), kbar, nb, i, p.topk, sink, score_g, counters, sel, idx);
         int st = check_launch("decode_select_kernel");
         if (st != SSA_OK) return st;
         decode_attend_kernel<T, D><<<dim3((unsigned)p.topk, (unsigned)BH), kThreads, 0, s>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), sel, p.T,
-            p.block, t, p.topk, p.sm_scale, part);
-        st = check_launch("decode_attend_kernel");
-        if (st != SSA_OK) return st;
-        decode_combine_kernel<T><<<BH, 32, 0, s>>>(part, p.D, p.topk, static_cast<T*>(h), lse);
-        return check_launch("decode_combine_kernel");
+            p.block, t, p.topk, p.sm_scale, part, counters + BH, static_cast<T*>(h), lse);
+        return check_launch("decode_attend_kernel");
     };
     using D64 = std::integral_constant<int, 64>;
     using D128 = std::integral_constant<int, 128>;
