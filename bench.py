@@ -703,7 +703,7 @@ def decode_bench(args, w, layer, stream, flush, dev):
     per_head = w.topk * w.block * w.D * esz * 2 + i * w.D * 8 + 2 * w.D * esz
     nbytes = per_head * w.B * w.H
     del graph
-    return {"kernels": ["decode_select_kernel", "decode_attend_kernel", "decode_combine_kernel"],
+    return {"kernels": ["decode_step_kernel"],
             "timed_as": "CUDA graph replay", "context": w.T, "ms": round(ms, 4), "hbm_bytes": nbytes,
             "hbm_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
 
