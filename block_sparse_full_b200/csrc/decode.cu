@@ -12,7 +12,7 @@
 // Launches (CUDA cores: one query per head is matrix-vector work, bound by
 // the key/value bytes it reads and, at this size, by latency):
 //   decode_pool_kernel   Kbar_j = mean of block j's keys (float64, exact)
-//   decode_step_kernel   one cluster of 8 CTAs per head; distributed shared
+//   decode_step_kernel   one cluster of 8 (or 4) CTAs per head; distributed shared
 //                        memory carries every hand-off, so the step is one
 //                        launch with no global round trips:
 //     1. every CTA scores its share of the completed blocks (warp per block,
@@ -80,7 +80,6 @@ __device__ __forceinline__ void load_row_piece(const T* p, float (&x)[E]) {
     }
 }
 
-constexpr int kCluster = 8;       // CTAs per head
 constexpr int kStepThreads = 512; // two halves of 8 warps: two selected blocks at a time
 
 // Shared memory of the step kernel (every CTA has the same layout; only the
@@ -94,7 +93,8 @@ struct StepSmem {
     }
 };
 
-template <typename T, int D>
+// kCluster: CTAs per head, 8 or 4 (chosen by the host from the head count)
+template <typename T, int D, int kCluster>
 __global__ void __launch_bounds__(kStepThreads, 1)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const double* __restrict__ kbar, int nb, int Tcap, int block, int t, int topk,
@@ -130,8 +130,8 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     int32_t* sel_l = cluster.map_shared_rank(sel, 0);
     float* part_l = cluster.map_shared_rank(part, 0);
 
-    // 1. scores of the completed blocks j < i: block j goes to CTA j % 8, warp
-    // (j / 8) % 16; lane l owns columns l, l + 32, ... (coalesced rows of the
+    // 1. scores of the completed blocks j < i: block j goes to CTA j % kCluster,
+    // warp (j / kCluster) % 16; lane l owns columns l, l + 32, ... (coalesced rows of the
     // float64 pooled keys), U blocks' loads in flight per warp
     {
         double qr[M];
@@ -224,7 +224,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     }
     cluster.sync();
 
-    // 3. slots rank, rank + 8, ... of the list: half hf (8 warps) of the CTA takes
+    // 3. slots rank, rank + kCluster, ... of the list: half hf (8 warps) of the CTA takes
     // every other one, so that two blocks' loads are in flight at once.  Per
     // block: keys and values loaded together (16-byte value loads; thread
     // (8-column chunk c8, key group g)), scores by a warp per group of keys,
@@ -380,10 +380,15 @@ int launch_decode_step(const ssa_params_t& p, int t, const void* q, const void* 
     const int nb = num_blocks(p);
     const bool sink = (p.flags & SSA_FLAG_FORCE_SINK) != 0;
     const size_t smem = StepSmem::bytes(nb, p.topk, p.D);
-    auto run = [&](auto tag, auto dtag) -> int {
+    // 8 CTAs per head while every head's cluster fits in one wave (a cluster of
+    // 8 CTAs of 512 threads takes 8 SMs of one GPC; measured: 8 clusters at a
+    // time), else 4 (two selected blocks per half then run one after the other)
+    const int cl = BH <= 8 ? 8 : 4;
+    auto run = [&](auto tag, auto dtag, auto ctag) -> int {
         using T = decltype(tag);
         constexpr int D = decltype(dtag)::value;
-        auto kern = decode_step_kernel<T, D>;
+        constexpr int kCluster = decltype(ctag)::value;
+        auto kern = decode_step_kernel<T, D, kCluster>;
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "decode: smem attribute: %s", cudaGetErrorString(e));
@@ -408,9 +413,14 @@ int launch_decode_step(const ssa_params_t& p, int t, const void* q, const void* 
     };
     using D64 = std::integral_constant<int, 64>;
     using D128 = std::integral_constant<int, 128>;
+    using C4 = std::integral_constant<int, 4>;
+    using C8 = std::integral_constant<int, 8>;
+    auto with_cluster = [&](auto tag, auto dtag) -> int {
+        return cl == 8 ? run(tag, dtag, C8{}) : run(tag, dtag, C4{});
+    };
     if (p.dtype == SSA_BF16)
-        return p.D == 64 ? run(__nv_bfloat16{}, D64{}) : run(__nv_bfloat16{}, D128{});
-    return p.D == 64 ? run(float{}, D64{}) : run(float{}, D128{});
+        return p.D == 64 ? with_cluster(__nv_bfloat16{}, D64{}) : with_cluster(__nv_bfloat16{}, D128{});
+    return p.D == 64 ? with_cluster(float{}, D64{}) : with_cluster(float{}, D128{});
 }
 
 }  // namespace ssa
