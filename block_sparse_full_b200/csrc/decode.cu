@@ -389,10 +389,12 @@ int launch_decode_step(const ssa_params_t& p, int t, const void* q, const void* 
         constexpr int D = decltype(dtag)::value;
         constexpr int kCluster = decltype(ctag)::value;
         auto kern = decode_step_kernel<T, D, kCluster>;
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "decode: smem attribute: %s", cudaGetErrorString(e));
-        }
+        size_t limit = 0;
+        int st = opt_in_max_smem<decode_step_kernel<T, D, kCluster>>("decode_step_kernel", &limit);
+        if (st != SSA_OK) return st;
+        if (smem > limit)
+            return fail(SSA_ERR_UNSUPPORTED, "decode: T/block = %d blocks need %zu bytes of shared memory (limit %zu)",
+                        nb, smem, limit);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)kCluster, (unsigned)BH);
         cfg.blockDim = dim3(kStepThreads);

@@ -7,8 +7,8 @@
 // is taken in the precision the definition fixes):
 //   pool_kernel       reads Q and K once (HBM-bound) and writes the exact
 //                     float64 block means Qbar, Kbar to the workspace;
-//   score_topk_kernel one CTA per 8 query blocks of one (b, h): scores
-//                     s_ij for j < i (register-tiled over 8 rows x 4 keys
+//   score_topk_kernel one CTA per 8 query blocks of one (b, h), two CTAs per
+//                     SM: scores s_ij for j < i (tiled over 8 rows x 4 keys
 //                     per warp, fixed summation order), then one warp per
 //                     row fills the free slots by warp-argmax rounds under
 //                     (score desc, index asc) and writes the ascending
@@ -99,19 +99,20 @@ pool_kernel(const T* __restrict__ q, const T* __restrict__ k, double* __restrict
 
 // Rows of R = 8 consecutive query blocks i0 .. i0+7 of one (b, h) per CTA
 // (n <= kRowsKernelMaxN).  Scores: warp w takes keys j0 + 4w .. j0 + 4w + 3
-// of each group of 32 for all 8 rows at once; lane l holds columns l, l+32,
-// ... of the 8 query block means in registers, so one read of a key block
-// mean serves 8 rows.  The 32 partial dot products of a lane (4 keys x 8
-// rows) are summed over the warp by a transpose-reduce (31 double
-// exchanges), after which lane l owns one complete score.  The next group's
-// key means are loaded before the current group is reduced.  Top-k: warp w
-// alone handles row i0 + w (selection, index list, mask, count), with no
-// CTA-wide barrier.  dynamic smem: scores [8][n] f64, bits [8][32] u32.
+// of each group of 32 for all 8 rows at once; the 8 query block means sit in
+// shared memory (lane l reads columns l, l+32, ...), so one read of a key
+// block mean serves 8 rows, and ~120 registers leave room for two CTAs per SM
+// (twice the warps to hide the float64 latencies).  The 32 partial dot
+// products of a lane (4 keys x 8 rows) are summed over the warp by a
+// transpose-reduce (31 double exchanges), after which lane l owns one
+// complete score.  Top-k: warp w alone handles row i0 + w (selection, index
+// list, mask, count), with no CTA-wide barrier.  dynamic smem: scores [8][n]
+// f64, bits [8][32] u32; static: the 8 query block means.
 constexpr int kRowsPerCta = 8;
 constexpr int kRowsKernelMaxN = 1024;
 
 template <int D>
-__global__ void __launch_bounds__(kSelThreads, 1)
+__global__ void __launch_bounds__(kSelThreads, 2)
 score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar, int n,
                   int topk, int force_sink, int words, int32_t* __restrict__ idx,
                   int32_t* __restrict__ cnt, uint32_t* __restrict__ mask) {
@@ -131,13 +132,12 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
     const double* kb = kbar + bh * (size_t)n * D;
     const int kend = min(i0 + R, n) - 1;  // keys j < kend cover every row's j < i
 
-    double qr[R][M];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-        const int i = min(i0 + r, n - 1);
-#pragma unroll
-        for (int m = 0; m < M; ++m) qr[r][m] = qbar[(bh * n + i) * D + lane + 32 * m];
+    __shared__ double qs[R * D];  // the R query-block means
+    for (int e = threadIdx.x; e < R * D; e += kSelThreads) {
+        const int r = e / D, c = e % D;
+        qs[e] = qbar[(bh * n + min(i0 + r, n - 1)) * D + c];
     }
+    __syncthreads();
     for (int t = threadIdx.x; t < R * 32; t += kSelThreads) bits_all[t] = 0u;
 
     auto load_group = [&](int j0, double (&kv)[KPW][M]) {
@@ -150,10 +150,9 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
         }
     };
     if (kend > 0) {
-        double kv[KPW][M], kn[KPW][M];
-        load_group(0, kv);
+        double kv[KPW][M];
         for (int j0 = 0; j0 < kend; j0 += GROUP) {
-            if (j0 + GROUP < kend) load_group(j0 + GROUP, kn);
+            load_group(j0, kv);
             double v[32];
 #pragma unroll
             for (int kk = 0; kk < KPW; ++kk)
@@ -161,7 +160,7 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
                 for (int r = 0; r < R; ++r) {
                     double acc = 0.0;
 #pragma unroll
-                    for (int m = 0; m < M; ++m) acc = fma(qr[r][m], kv[kk][m], acc);
+                    for (int m = 0; m < M; ++m) acc = fma(qs[r * D + lane + 32 * m], kv[kk][m], acc);
                     v[kk * R + r] = acc;
                 }
             // transpose-reduce: after the step of width s, v[t] (t < s) holds
@@ -180,10 +179,6 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
             const int kk = lane / R, r = lane % R;
             const int j = j0 + KPW * warp + kk;
             if (j < kend) sc[(size_t)r * n + j] = v[0];
-#pragma unroll
-            for (int kk2 = 0; kk2 < KPW; ++kk2)
-#pragma unroll
-                for (int m = 0; m < M; ++m) kv[kk2][m] = kn[kk2][m];
         }
     }
     __syncthreads();  // all rows' scores and cleared bits visible
@@ -344,22 +339,16 @@ int launch_score(const ssa_params_t& p, const double* qbar, const double* kbar, 
     const int sink = (p.flags & SSA_FLAG_FORCE_SINK) ? 1 : 0;
     if (n <= kRowsKernelMaxN) {
         const size_t smem = (size_t)kRowsPerCta * n * 8 + kRowsPerCta * 32 * 4;
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(score_topk_kernel<D>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "select: smem attribute: %s", cudaGetErrorString(e));
-        }
+        int st = opt_in_max_smem<score_topk_kernel<D>>("score_topk_kernel");
+        if (st != SSA_OK) return st;
         const size_t grid = (size_t)p.B * p.H * ((n + kRowsPerCta - 1) / kRowsPerCta);
         score_topk_kernel<D><<<(unsigned)grid, kSelThreads, smem, s>>>(qbar, kbar, n, p.topk, sink,
                                                                        words, idx, cnt, mask);
         return check_launch("score_topk_kernel");
     }
     const size_t smem = (size_t)n * 8 + (size_t)words * 4 + (size_t)(words + 1) * 4;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(score_topk_row_kernel<D>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "select: smem attribute: %s", cudaGetErrorString(e));
-    }
+    int st = opt_in_max_smem<score_topk_row_kernel<D>>("score_topk_row_kernel");
+    if (st != SSA_OK) return st;
     score_topk_row_kernel<D><<<(unsigned)rows, kSelThreads, smem, s>>>(qbar, kbar, n, p.topk, sink,
                                                                        words, idx, cnt, mask);
     return check_launch("score_topk_row_kernel");

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "ssa.h"
 
 namespace ssa {
@@ -18,6 +20,31 @@ int fail(int status, const char* fmt, ...);
 int check_launch(const char* what);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Shared memory a CTA may hold on sm_100 (227 KB).
+constexpr size_t kMaxSmemPerCta = 232448;
+
+// Lets kernel K take dynamic shared memory up to the per-CTA maximum less its
+// static shared memory (once per process; launches above the default 48 KB
+// of dynamic plus static shared memory fail without it).  Call it before any
+// stream capture.  Returns an SSA status; *dyn_limit receives the limit.
+template <auto K>
+int opt_in_max_smem(const char* what, size_t* dyn_limit = nullptr) {
+    static std::once_flag once;
+    static cudaError_t err = cudaSuccess;
+    static size_t limit = 0;
+    std::call_once(once, [] {
+        cudaFuncAttributes fa;
+        err = cudaFuncGetAttributes(&fa, K);
+        if (err == cudaSuccess) {
+            limit = kMaxSmemPerCta - fa.sharedSizeBytes;
+            err = cudaFuncSetAttribute(K, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)limit);
+        }
+    });
+    if (dyn_limit) *dyn_limit = limit;
+    if (err != cudaSuccess) return fail(SSA_ERR_CUDA, "%s: shared memory attribute: %s", what, cudaGetErrorString(err));
+    return SSA_OK;
+}
 
 // Wall-clock limit of the kernels' bounded waits (default 2 s; tests shorten it).
 unsigned long long wait_limit_ns();

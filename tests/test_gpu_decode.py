@@ -75,3 +75,19 @@ def test_decode_more_than_1024_completed_blocks():
     w = Workload("bf16_T70400_d64_decode", B=1, H=1, T=64 * 1100, D=64, block=64, topk=12,
                  dtype="bf16", plant="hot", seed=41)
     _decode(w, [w.T - 1, 64 * 1030 + 3])
+
+
+def test_decode_topk64_d128_many_heads():
+    # the largest budget the decode step takes (64 places) at d = 128: its
+    # shared memory passes the default 48 KB per CTA, and with 16 heads the
+    # clusters of 4 CTAs take several selected blocks per half of a CTA
+    w = Workload("bf16_H16_T16384_k64_decode", B=1, H=16, T=16384, D=128, block=64, topk=64,
+                 dtype="bf16", plant="hot", seed=43)
+    _decode(w, [w.T - 1, 64 * 70 + 9], heads=[0, 9])
+
+
+def test_decode_few_heads_cluster_of_eight():
+    # eight heads or fewer: clusters of 8 CTAs per head
+    w = Workload("bf16_H4_T8192_decode", B=2, H=2, T=8192, D=128, block=128, topk=16,
+                 dtype="bf16", plant="sink", seed=44)
+    _decode(w, [w.T - 1, 4000])
