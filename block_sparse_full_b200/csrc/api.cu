@@ -345,6 +345,7 @@ int ssa_device_status(void* stream) {
     int st = fwd_tc_take_status(s);
     if (st == SSA_OK) st = bwd_tc_take_status(s);
     if (st == SSA_OK) st = selftest_take_status();
+    if (st == SSA_OK) st = decode_take_status();
     if (st != SSA_OK) return st;
     return check_launch("pending");
 }

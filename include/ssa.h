@@ -190,9 +190,13 @@ int ssa_attn_fwd_sparse(const ssa_params_t* params, const void* q, const void* k
  *   every key of S that is <= t ([B,H,D] in dtype) and lse its log-sum-exp
  *   (float32 [B,H]).  idx, if not NULL, receives S ascending, -1 padded
  *   ([B,H,topk] int32).  kbar must hold blocks 0..i-1.  Workspace:
- *   SSA_WS_DECODE (0 bytes: the step runs as one launch of a cluster of 8
- *   CTAs per head whose hand-offs stay in shared memory; the argument is kept
- *   so that callers need no change if a later version needs scratch).
+ *   SSA_WS_DECODE (0 bytes: the step runs as one launch of a cluster of 4 or
+ *   8 CTAs per head whose hand-offs stay in shared memory; the argument is
+ *   kept so that callers need no change if a later version needs scratch).
+ *   k_cache and v_cache must be 16-byte aligned (the selected blocks are
+ *   copied with bulk copies).  A bulk copy or a hand-off that does not
+ *   complete within the wait limit makes ssa_device_status return
+ *   SSA_ERR_TIMEOUT.
  */
 int ssa_decode_pool(const ssa_params_t* params, int j0, int j1, const void* k_cache,
                     double* kbar, void* stream);

@@ -91,3 +91,31 @@ def test_decode_few_heads_cluster_of_eight():
     w = Workload("bf16_H4_T8192_decode", B=2, H=2, T=8192, D=128, block=128, topk=16,
                  dtype="bf16", plant="sink", seed=44)
     _decode(w, [w.T - 1, 4000])
+
+
+def test_decode_f32_block128_several_passes():
+    # float32 blocks of 128 keys at d = 128 take 128 KB of keys and values each:
+    # one fits in a CTA's shared memory, so the two selected blocks of each CTA
+    # of a 4-CTA cluster (12 heads) stream in one pass after the other
+    w = Workload("f32_H12_T2048_b128_decode", B=1, H=12, T=2048, D=128, block=128, topk=8,
+                 dtype="f32", plant="hot", seed=45)
+    _decode(w, [w.T - 1, 128 * 9 + 100, 128 * 3 + 1], heads=[0, 5, 11])
+
+
+def test_decode_step_is_repeatable():
+    # the same step twice gives the same bits (fixed reduction orders)
+    w = SMALL["bf16_T1216_b64"]
+    inp = make_inputs(w)
+    p = params(w, inp["q"].to(DEV))
+    cache = ssa.DecodeCache(p, DEV, inp["k"].dtype)
+    cache.k.copy_(inp["k"].to(DEV))
+    cache.v.copy_(inp["v"].to(DEV))
+    t = w.T - 1
+    q_t = inp["q"][:, :, t].contiguous().to(DEV)
+    a = cache.step(t, q_t)
+    a = {n: x.clone() for n, x in a.items()}
+    b = cache.step(t, q_t)
+    torch.cuda.synchronize()
+    ssa.device_status()
+    for n in a:
+        assert torch.equal(a[n], b[n]), n
