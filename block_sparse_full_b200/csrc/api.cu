@@ -346,6 +346,7 @@ int ssa_device_status(void* stream) {
     if (st == SSA_OK) st = bwd_tc_take_status(s);
     if (st == SSA_OK) st = selftest_take_status();
     if (st == SSA_OK) st = decode_take_status();
+    if (st == SSA_OK) st = select_take_status();
     if (st != SSA_OK) return st;
     return check_launch("pending");
 }

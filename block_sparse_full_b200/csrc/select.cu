@@ -5,20 +5,25 @@
 //
 // Two steps, on CUDA cores in float64 (the decision is an integer set, so it
 // is taken in the precision the definition fixes):
-//   pool_kernel       reads Q and K once (HBM-bound) and writes the exact
-//                     float64 block means Qbar, Kbar to the workspace;
+//   pool_ring_kernel  (bf16; pool_kernel for f32) reads Q and K once
+//                     (HBM-bound) and writes the exact float64 block means
+//                     Qbar, Kbar to the workspace;
 //   score_topk_kernel one CTA per 8 query blocks of one (b, h), two CTAs per
-//                     SM: scores s_ij for j < i (tiled over 8 rows x 4 keys
-//                     per warp, fixed summation order), then one warp per
-//                     row fills the free slots by warp-argmax rounds under
-//                     (score desc, index asc) and writes the ascending
-//                     index list by popcount prefix of the set bitmask;
+//                     SM: scores s_ij for j < i on the float64 tensor cores
+//                     (8 rows x 8 keys per DMMA tile, fixed summation
+//                     order), then one warp per row fills the free slots by
+//                     warp rounds under (score desc, index asc) and writes
+//                     the ascending index list by popcount prefix of the
+//                     set bitmask;
 //   score_topk_row_kernel the same selection one CTA per query block, for
 //                     rows longer than 1024 blocks.
+#include <algorithm>
 #include <cstdio>
+#include <mutex>
 
 #include "device_util.cuh"
 #include "ssa_internal.h"
+#include "tc_util.cuh"
 
 namespace ssa {
 namespace {
@@ -97,17 +102,172 @@ pool_kernel(const T* __restrict__ q, const T* __restrict__ k, double* __restrict
     }
 }
 
+using tc::fence_mbar_init;
+using tc::kDrainLimitNs;
+using tc::mbar_expect_tx;
+using tc::mbar_init;
+using tc::mbar_try_wait;
+using tc::smem_u32;
+using tc::globaltimer;
+
+// one-dimensional bulk copy global -> this CTA's shared memory, completing on `bar`
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
+}
+// wait for the phase of parity `parity` (wall-clock bound); false if it expired
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > limit_ns) return false;
+    return true;
+}
+
+__device__ unsigned int g_select_status;
+
+// bf16 pooling as a persistent stream: CTA c takes units c, c + G, ... (G =
+// grid size); one thread keeps NS units in flight with bulk copies (a unit is
+// BLOCK contiguous rows, 8 to 32 KB) into a ring of shared-memory stages, and
+// all threads reduce each landed unit: thread (column pair, row group) sums its
+// rows in float64, the row groups are added in a fixed order.  The copies of
+// the next units overlap the conversions of this one, so HBM stays busy.
+template <int D, int BLOCK>
+struct RingShape {
+    static constexpr int UB = BLOCK * D * 2;                     // bytes per unit
+    static constexpr int NS = UB <= 16384 ? 6 : 3;               // stages in flight
+    static constexpr int CP = D / 2;                             // column pairs
+    static constexpr int RG = kPoolThreads / CP;                 // row groups
+    static constexpr size_t SMEM = (size_t)NS * UB + 2 * (size_t)RG * D * 8 + 1024;
+};
+
+template <int D, int BLOCK>
+__global__ void __launch_bounds__(kPoolThreads, 2)
+pool_ring_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                 double* __restrict__ qbar, double* __restrict__ kbar, int units_q, int total,
+                 unsigned long long limit_ns) {
+    using S = RingShape<D, BLOCK>;
+    constexpr int UB = S::UB, NS = S::NS, CP = S::CP, RG = S::RG;
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ __align__(8) uint64_t full[NS];
+    double* part = reinterpret_cast<double*>(sm + (size_t)NS * UB);  // [2][RG][D]
+    const int tid = threadIdx.x;
+    const int G = gridDim.x;
+    const int mine = blockIdx.x < total ? (total - 1 - (int)blockIdx.x) / G + 1 : 0;
+    auto src_of = [&](int l) -> const void* {
+        const int u = (int)blockIdx.x + l * G;
+        return u < units_q ? (const void*)(q + (size_t)u * BLOCK * D)
+                           : (const void*)(k + (size_t)(u - units_q) * BLOCK * D);
+    };
+    if (tid == 0) {
+        for (int st = 0; st < NS; ++st) mbar_init(smem_u32(&full[st]), 1);
+        fence_mbar_init();
+        for (int l = 0; l < NS && l < mine; ++l) {
+            mbar_expect_tx(smem_u32(&full[l]), UB);
+            bulk_load_1d(smem_u32(sm + (size_t)l * UB), src_of(l), UB, smem_u32(&full[l]));
+        }
+    }
+    __syncthreads();
+    const int cp = tid % CP, rg = tid / CP;
+    int l = 0;
+    for (; l < mine; ++l) {
+        const int st = l % NS;
+        if (!__syncthreads_and(mbar_wait_bounded(smem_u32(&full[st]), (l / NS) & 1, limit_ns))) {
+            atomicOr(&g_select_status, 1u);
+            break;
+        }
+        const uint32_t* unit = reinterpret_cast<const uint32_t*>(sm + (size_t)st * UB);
+        double a0 = 0.0, a1 = 0.0;
+#pragma unroll 8
+        for (int r = rg; r < BLOCK; r += RG) {
+            const uint32_t w = unit[r * CP + cp];  // columns 2 cp, 2 cp + 1 of row r
+            a0 += (double)__uint_as_float(w << 16);
+            a1 += (double)__uint_as_float(w & 0xffff0000u);
+        }
+        double* pp = part + (size_t)(l & 1) * RG * D;
+        pp[rg * D + 2 * cp] = a0;
+        pp[rg * D + 2 * cp + 1] = a1;
+        __syncthreads();  // the stage is read and the partials are written
+        if (tid == 0 && l + NS < mine) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_expect_tx(smem_u32(&full[st]), UB);
+            bulk_load_1d(smem_u32(sm + (size_t)st * UB), src_of(l + NS), UB, smem_u32(&full[st]));
+        }
+        if (tid < D) {
+            double sum = 0.0;
+#pragma unroll
+            for (int g = 0; g < RG; ++g) sum += pp[g * D + tid];
+            const int u = (int)blockIdx.x + l * G;
+            double* dst = u < units_q ? qbar + (size_t)u * D : kbar + (size_t)(u - units_q) * D;
+            dst[tid] = sum / (double)BLOCK;  // block is a power of two: exact
+        }
+    }
+    if (l < mine && tid == 0) {
+        // a wait expired: let the copies already issued land before the CTA exits
+        for (int l2 = l; l2 < mine && l2 < l + NS; ++l2)
+            mbar_wait_bounded(smem_u32(&full[l2 % NS]), (l2 / NS) & 1, kDrainLimitNs);
+    }
+}
+
+// The selection order (score desc, index asc) on integers: the float64 score
+// mapped to a u64 whose unsigned order is the score's order (-0 taken as +0,
+// so that equal scores give equal keys).
+__device__ __forceinline__ uint64_t order_key(double x) {
+    const uint64_t b = (uint64_t)__double_as_longlong(x == 0.0 ? 0.0 : x);
+    return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+// Top r of the candidates first .. i-1 of one row (order keys in shared memory)
+// by warp rounds: each lane holds its best remaining candidate; a round finds
+// the largest key with two warp max-reductions (high and low word) and the
+// lowest index holding it with a min-reduction; the winner's lane rescans its
+// own candidates for the best one below the winner.
+__device__ __forceinline__ void warp_topk_keys(const uint64_t* key, int first, int i, int r,
+                                               uint32_t* bits, int lane) {
+    uint64_t bk = 0;
+    int bj = -1;
+    for (int j = first + lane; j < i; j += 32) {
+        const uint64_t x = key[j];
+        if (bj < 0 || x > bk) {  // ascending j: equal keys keep the lower index
+            bk = x;
+            bj = j;
+        }
+    }
+    for (int round = 0; round < r; ++round) {
+        const uint32_t hi = bj < 0 ? 0u : (uint32_t)(bk >> 32);
+        const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+        const bool top = bj >= 0 && hi == mhi;
+        const uint32_t mlo = __reduce_max_sync(0xffffffffu, top ? (uint32_t)bk : 0u);
+        const bool win = top && (uint32_t)bk == mlo;
+        const uint32_t wj = __reduce_min_sync(0xffffffffu, win ? (uint32_t)bj : 0xffffffffu);
+        if (wj == 0xffffffffu) break;  // no candidate left
+        if ((uint32_t)bj == wj) {
+            atomicOr(&bits[wj >> 5], 1u << (wj & 31));
+            const uint64_t wk = bk;
+            bj = -1;
+            for (int j = first + lane; j < i; j += 32) {
+                const uint64_t x = key[j];
+                if (!(x < wk || (x == wk && j > (int)wj))) continue;  // taken already
+                if (bj < 0 || x > bk) {
+                    bk = x;
+                    bj = j;
+                }
+            }
+        }
+    }
+}
+
 // Rows of R = 8 consecutive query blocks i0 .. i0+7 of one (b, h) per CTA
-// (n <= kRowsKernelMaxN).  Scores: warp w takes keys j0 + 4w .. j0 + 4w + 3
-// of each group of 32 for all 8 rows at once; the 8 query block means sit in
-// shared memory (lane l reads columns l, l+32, ...), so one read of a key
-// block mean serves 8 rows, and ~120 registers leave room for two CTAs per SM
-// (twice the warps to hide the float64 latencies).  The 32 partial dot
-// products of a lane (4 keys x 8 rows) are summed over the warp by a
-// transpose-reduce (31 double exchanges), after which lane l owns one
-// complete score.  Top-k: warp w alone handles row i0 + w (selection, index
-// list, mask, count), with no CTA-wide barrier.  dynamic smem: scores [8][n]
-// f64, bits [8][32] u32; static: the 8 query block means.
+// (n <= kRowsKernelMaxN).  Scores on the float64 tensor cores: warp w takes
+// the 8-key tiles j0 = 8 w, 8 (w + 8), ...; one DMMA (m8n8k4) per 4 columns
+// with A = the 8 query-block means (shared memory, rows padded to D + 4
+// doubles) and B = the tile's 8 key-block means (read from L2), so C holds
+// the tile's 8 x 8 scores, summed over the columns in a fixed order; their
+// order keys go to shared memory.  Top-k: warp w alone handles row i0 + w
+// (selection, index list, mask, count), with no CTA-wide barrier.  dynamic
+// smem: keys [8][n] u64, bits [8][32] u32; static: the 8 query block means.
 constexpr int kRowsPerCta = 8;
 constexpr int kRowsKernelMaxN = 1024;
 
@@ -116,13 +276,12 @@ __global__ void __launch_bounds__(kSelThreads, 2)
 score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar, int n,
                   int topk, int force_sink, int words, int32_t* __restrict__ idx,
                   int32_t* __restrict__ cnt, uint32_t* __restrict__ mask) {
-    constexpr int M = D / 32;
     constexpr int R = kRowsPerCta;
-    constexpr int KPW = 32 / R;                   // keys per warp per group
-    constexpr int GROUP = (kSelThreads / 32) * KPW;  // keys per group
-    static_assert(KPW * R == 32, "one partial per lane after the transpose-reduce");
-    extern __shared__ double smem[];
-    double* sc = smem;                                                      // [R][n]
+    constexpr int NW = kSelThreads / 32;
+    constexpr int QS = D + 4;  // padded row of the query-block means
+    static_assert(R == 8, "the DMMA tile has 8 rows");
+    extern __shared__ uint64_t smem_u64[];
+    uint64_t* sc = smem_u64;                                                // [R][n]
     uint32_t* bits_all = reinterpret_cast<uint32_t*>(sc + (size_t)R * n);  // [R][32]
 
     const int nrb = (n + R - 1) / R;
@@ -132,62 +291,40 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
     const double* kb = kbar + bh * (size_t)n * D;
     const int kend = min(i0 + R, n) - 1;  // keys j < kend cover every row's j < i
 
-    __shared__ double qs[R * D];  // the R query-block means
+    __shared__ double qs[R * QS];  // the R query-block means
     for (int e = threadIdx.x; e < R * D; e += kSelThreads) {
         const int r = e / D, c = e % D;
-        qs[e] = qbar[(bh * n + min(i0 + r, n - 1)) * D + c];
+        qs[r * QS + c] = qbar[(bh * n + min(i0 + r, n - 1)) * D + c];
     }
-    __syncthreads();
     for (int t = threadIdx.x; t < R * 32; t += kSelThreads) bits_all[t] = 0u;
+    __syncthreads();
 
-    auto load_group = [&](int j0, double (&kv)[KPW][M]) {
-#pragma unroll
-        for (int kk = 0; kk < KPW; ++kk) {
-            const int j = max(min(j0 + KPW * warp + kk, kend - 1), 0);  // past the end: result unused
-            const double* kr = kb + (size_t)j * D + lane;
-#pragma unroll
-            for (int m = 0; m < M; ++m) kv[kk][m] = kr[32 * m];
-        }
-    };
-    if (kend > 0) {
-        double kv[KPW][M];
-        for (int j0 = 0; j0 < kend; j0 += GROUP) {
-            load_group(j0, kv);
-            double v[32];
-#pragma unroll
-            for (int kk = 0; kk < KPW; ++kk)
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    double acc = 0.0;
-#pragma unroll
-                    for (int m = 0; m < M; ++m) acc = fma(qs[r * D + lane + 32 * m], kv[kk][m], acc);
-                    v[kk * R + r] = acc;
-                }
-            // transpose-reduce: after the step of width s, v[t] (t < s) holds
-            // entry t + s * (lane bit s) + (the bits kept before), summed
-            // over the lanes that differ in that bit
-#pragma unroll
-            for (int s = 16; s >= 1; s >>= 1) {
-                const bool upper = (lane & s) != 0;
-#pragma unroll
-                for (int t = 0; t < s; ++t) {
-                    const double send = upper ? v[t] : v[t + s];
-                    const double keep = upper ? v[t + s] : v[t];
-                    v[t] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-                }
+    {
+        const int g = lane >> 2, t = lane & 3;  // fragment row / column of the DMMA
+        for (int j0 = 8 * warp; j0 < kend; j0 += 8 * NW) {
+            const double* kr = kb + (size_t)min(j0 + g, kend - 1) * D + t;  // past the end: unused
+            const double* qr = qs + g * QS + t;
+            double c0 = 0.0, c1 = 0.0;
+#pragma unroll 8
+            for (int s4 = 0; s4 < D / 4; ++s4) {
+                const double av = qr[4 * s4];
+                const double bv = kr[4 * s4];
+                asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                             : "+d"(c0), "+d"(c1)
+                             : "d"(av), "d"(bv));
             }
-            const int kk = lane / R, r = lane % R;
-            const int j = j0 + KPW * warp + kk;
-            if (j < kend) sc[(size_t)r * n + j] = v[0];
+            const int j = j0 + 2 * t;  // C[g][2t], C[g][2t + 1]: row i0 + g, keys j, j + 1
+            if (j < kend) sc[(size_t)g * n + j] = order_key(c0);
+            if (j + 1 < kend) sc[(size_t)g * n + j + 1] = order_key(c1);
         }
     }
-    __syncthreads();  // all rows' scores and cleared bits visible
+    __syncthreads();  // all rows' keys visible
 
     if (warp >= R) return;
     const int i = i0 + warp;
     if (i >= n) return;
     const size_t row = bh * n + i;
-    const double* srow = sc + (size_t)warp * n;
+    const uint64_t* srow = sc + (size_t)warp * n;
     uint32_t* bits = bits_all + warp * 32;
     const bool sink = force_sink && i > 0;
     if (lane == 0) {
@@ -201,7 +338,7 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
     if (ncand <= r) {
         for (int j = first + lane; j < i; j += 32) atomicOr(&bits[j >> 5], 1u << (j & 31));
     } else {
-        warp_topk_rounds(srow, first, i, r, bits, lane);
+        warp_topk_keys(srow, first, i, r, bits, lane);
     }
     __syncwarp();
     // ascending index list: lane l owns mask word l (words <= 32)
@@ -321,14 +458,43 @@ int launch_pool(const void* q, const void* k, double* qbar, double* kbar, size_t
     return check_launch("pool_kernel");
 }
 
+template <int D, int BLOCK>
+int launch_pool_ring(const void* q, const void* k, double* qbar, double* kbar, size_t units_q,
+                     cudaStream_t s) {
+    using S = RingShape<D, BLOCK>;
+    static int sms = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    });
+    int st = opt_in_max_smem<pool_ring_kernel<D, BLOCK>>("pool_ring_kernel");
+    if (st != SSA_OK) return st;
+    const size_t total = 2 * units_q;
+    const size_t grid = std::min(total, (size_t)(sms > 0 ? sms : 148) * 2);
+    pool_ring_kernel<D, BLOCK><<<(unsigned)grid, kPoolThreads, S::SMEM, s>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbar,
+        (int)units_q, (int)total, wait_limit_ns());
+    return check_launch("pool_ring_kernel");
+}
+
 template <typename T>
 int launch_pool_t(const ssa_params_t& p, const void* q, const void* k, double* qbar, double* kbar,
                   size_t units_q, cudaStream_t s) {
-    if (p.D == 64)
-        return p.block == 64 ? launch_pool<T, 64, 64>(q, k, qbar, kbar, units_q, s)
-                             : launch_pool<T, 64, 128>(q, k, qbar, kbar, units_q, s);
-    return p.block == 64 ? launch_pool<T, 128, 64>(q, k, qbar, kbar, units_q, s)
-                         : launch_pool<T, 128, 128>(q, k, qbar, kbar, units_q, s);
+    if constexpr (sizeof(T) == 2) {
+        if (p.D == 64)
+            return p.block == 64 ? launch_pool_ring<64, 64>(q, k, qbar, kbar, units_q, s)
+                                 : launch_pool_ring<64, 128>(q, k, qbar, kbar, units_q, s);
+        return p.block == 64 ? launch_pool_ring<128, 64>(q, k, qbar, kbar, units_q, s)
+                             : launch_pool_ring<128, 128>(q, k, qbar, kbar, units_q, s);
+    } else {
+        if (p.D == 64)
+            return p.block == 64 ? launch_pool<T, 64, 64>(q, k, qbar, kbar, units_q, s)
+                                 : launch_pool<T, 64, 128>(q, k, qbar, kbar, units_q, s);
+        return p.block == 64 ? launch_pool<T, 128, 64>(q, k, qbar, kbar, units_q, s)
+                             : launch_pool<T, 128, 128>(q, k, qbar, kbar, units_q, s);
+    }
 }
 
 template <int D>
@@ -355,6 +521,18 @@ int launch_score(const ssa_params_t& p, const double* qbar, const double* kbar, 
 }
 
 }  // namespace
+
+int select_take_status() {
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_select_status, sizeof v);
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (v != 0) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_select_status, &zero, sizeof zero);
+        return fail(SSA_ERR_TIMEOUT, "pooling: a wait for a bulk copy expired");
+    }
+    return SSA_OK;
+}
 
 size_t select_workspace(const ssa_params_t& p) {
     // Qbar and Kbar, float64 [B, H, n, D] each

@@ -127,6 +127,7 @@ int bwd_tc_take_status(cudaStream_t s);  // SSA_ERR_TIMEOUT if a wait expired
 int bwd_tc_heads_per_group(const ssa_params_t& p);  // heads sharing the dS workspace
 
 // ---- self-tests (selftest.cu)
+int select_take_status();  // SSA_ERR_TIMEOUT if a pooling wait expired
 int decode_take_status();  // SSA_ERR_TIMEOUT if a decode-step wait expired
 int selftest_take_status();  // SSA_ERR_TIMEOUT if the self-test wait expired
 

@@ -119,3 +119,15 @@ def test_decode_step_is_repeatable():
     ssa.device_status()
     for n in a:
         assert torch.equal(a[n], b[n]), n
+
+
+def test_decode_sixteen_heads_clusters_of_eight_small_ctas():
+    # 16 heads at top-k 16: clusters of 8 CTAs of 256 threads
+    w = WORKLOADS["bf16_T8192_H16_hot"]
+    _decode(w, [w.T - 1, 3000], heads=[0, 7, 15])
+
+
+def test_decode_many_heads_small_ctas():
+    # 128 heads: clusters of 4 CTAs of 256 threads
+    w = WORKLOADS["bf16_B4_H32_T4096_train"]
+    _decode(w, [w.T - 1, 1500], heads=[0, 31])

@@ -68,3 +68,51 @@ def test_selection_all_keys_equal_takes_lowest_indices():
         want = list(range(min(i, topk - 1))) + [i]
         assert cnt[0, 0, i] == len(want)
         assert idx[0, 0, i, : len(want)].tolist() == want
+
+
+@pytest.mark.parametrize("D,block,n,topk,B,H", [(128, 64, 70, 16, 2, 8), (64, 128, 40, 12, 2, 16),
+                                                (128, 128, 36, 8, 4, 8)])
+def test_selection_many_heads(D, block, n, topk, B, H):
+    # more blocks than the pooling grid holds CTAs: every CTA streams several
+    # blocks through its ring of stages
+    q, k, (dq, dk) = _data("bf16", D, block, n, seed=n + H, B=B, H=H)
+    p = ssa.params_for(dq, block, topk)
+    got = ssa.select_blocks(p, dq, dk)
+    want = O.select_blocks(q, k, block, topk)
+    torch.cuda.synchronize()
+    ssa.device_status()
+    assert assert_selection(got, want, margin_tol=-1.0) == 0
+
+
+@pytest.mark.parametrize("D,block", [(128, 64), (64, 128)])
+def test_pooled_means_exact_over_the_bf16_range(D, block):
+    # the float64 block means the selection ranks by are exact: values spread
+    # over 36 binades with zeros and both signs (block sums still exact in
+    # float64, so any summation order gives the oracle's value), and a block of
+    # bf16 subnormals, pool to the oracle's means bit for bit.  The workspace
+    # holds Qbar then Kbar, float64 [B, H, n, D] each, at 256-byte aligned offsets.
+    B, H, n = 1, 3, 9
+    T = n * block
+    rng = np.random.default_rng(D + block)
+    shape = (2, B, H, T, D)
+    x = rng.choice([-1.0, 1.0], size=shape) * rng.integers(1, 256, size=shape) * 2.0 ** rng.integers(-18, 19, size=shape)
+    x[rng.random(shape) < 0.05] = 0.0
+    sub = slice(2 * block, 3 * block)  # block 2: subnormals and zeros only
+    x[..., sub, :] = rng.integers(-127, 128, size=x[..., sub, :].shape) * 2.0 ** -133
+    t = torch.from_numpy(x).to(torch.bfloat16)
+    back = t.to(torch.float64).numpy()  # the values the GPU sees
+    assert np.array_equal(back, x)
+    dq, dk = t[0].to(DEV), t[1].to(DEV)
+    p = ssa.params_for(dq, block, 4)
+    ws = ssa.workspace(p, ssa.SSA_WS_SELECT, DEV)
+    ssa.select_blocks(p, dq, dk, ws=ws)
+    torch.cuda.synchronize()
+    ssa.device_status()
+    m = B * H * n * D
+    half = (m * 8 + 255) // 256 * 256
+    qbar = ws[: m * 8].view(torch.float64).cpu().numpy().reshape(B, H, n, D)
+    kbar = ws[half: half + m * 8].view(torch.float64).cpu().numpy().reshape(B, H, n, D)
+    for b in range(B):
+        for h in range(H):
+            np.testing.assert_array_equal(qbar[b, h], O.pool_blocks(back[0, b, h], block))
+            np.testing.assert_array_equal(kbar[b, h], O.pool_blocks(back[1, b, h], block))
