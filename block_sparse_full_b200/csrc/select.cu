@@ -3,12 +3,12 @@
 // Sparse Attention Stream = block-sparse attention; section 4, "Efficienza":
 // the same operations as MoBA at inference).
 //
-// Two steps, on CUDA cores in float64 (the decision is an integer set, so it
-// is taken in the precision the definition fixes):
+// Two steps in float64 (the decision is an integer set, so it is taken in the
+// precision the definition fixes):
 //   pool_ring_kernel  (bf16; pool_kernel for f32) reads Q and K once
 //                     (HBM-bound) and writes the exact float64 block means
 //                     Qbar, Kbar to the workspace;
-//   score_topk_kernel one CTA per 8 query blocks of one (b, h), two CTAs per
+//   score_topk_kernel one CTA per 8 query blocks of one (b, h), four CTAs per
 //                     SM: scores s_ij for j < i on the float64 tensor cores
 //                     (8 rows x 8 keys per DMMA tile, fixed summation
 //                     order), then one warp per row fills the free slots by
@@ -219,6 +219,77 @@ __device__ __forceinline__ uint64_t order_key(double x) {
     return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
+__device__ __forceinline__ void dmma8(double (&c)[2], double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(c[0]), "+d"(c[1])
+                 : "d"(a), "d"(b));
+}
+
+// (key, index) a ranks ahead of b: larger key, or equal key and lower index
+__device__ __forceinline__ bool ahead(uint64_t ka, int ja, uint64_t kb, int jb) {
+    return ka > kb || (ka == kb && ja < jb);
+}
+
+// Top r of at most 128 candidates first .. i-1 of one row: each lane holds
+// its (up to four) candidates sorted in registers; a round takes the largest
+// head with one warp max-reduction of the high key words when that maximum
+// is held by one lane (the common case), else by the full (high, low, index)
+// reductions; the winning lane shifts its list.
+__device__ __forceinline__ void warp_topk_keys_small(const uint64_t* key, int first, int i, int r,
+                                                     uint32_t* bits, int lane) {
+    uint64_t k4[4];
+    int j4[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int j = first + lane + 32 * m;
+        j4[m] = j < i ? j : 0x7fffffff;
+        k4[m] = j < i ? key[j] : 0ull;
+    }
+    auto cswap = [&](int a, int b) {  // sorting network step: list order (key desc, index asc)
+        if (ahead(k4[b], j4[b], k4[a], j4[a])) {
+            const uint64_t tk = k4[a];
+            k4[a] = k4[b];
+            k4[b] = tk;
+            const int tj = j4[a];
+            j4[a] = j4[b];
+            j4[b] = tj;
+        }
+    };
+    cswap(0, 1);
+    cswap(2, 3);
+    cswap(0, 2);
+    cswap(1, 3);
+    cswap(1, 2);
+    for (int round = 0; round < r; ++round) {
+        const bool have = j4[0] != 0x7fffffff;
+        const uint32_t hi = have ? (uint32_t)(k4[0] >> 32) : 0u;
+        const uint32_t mhi = __reduce_max_sync(0xffffffffu, hi);
+        const uint32_t tie = __ballot_sync(0xffffffffu, have && hi == mhi);
+        if (tie == 0u) break;  // no candidate left
+        int wl;
+        if (__popc(tie) == 1) {
+            wl = __ffs(tie) - 1;
+        } else {
+            const bool top = (tie >> lane) & 1u;
+            const uint32_t mlo = __reduce_max_sync(0xffffffffu, top ? (uint32_t)k4[0] : 0u);
+            const bool win = top && (uint32_t)k4[0] == mlo;
+            const uint32_t wj = __reduce_min_sync(0xffffffffu, win ? (uint32_t)j4[0] : 0xffffffffu);
+            wl = __ffs(__ballot_sync(0xffffffffu, win && (uint32_t)j4[0] == wj)) - 1;
+        }
+        if (lane == wl) {
+            atomicOr(&bits[j4[0] >> 5], 1u << (j4[0] & 31));
+            k4[0] = k4[1];
+            j4[0] = j4[1];
+            k4[1] = k4[2];
+            j4[1] = j4[2];
+            k4[2] = k4[3];
+            j4[2] = j4[3];
+            k4[3] = 0ull;
+            j4[3] = 0x7fffffff;
+        }
+    }
+}
+
 // Top r of the candidates first .. i-1 of one row (order keys in shared memory)
 // by warp rounds: each lane holds its best remaining candidate; a round finds
 // the largest key with two warp max-reductions (high and low word) and the
@@ -264,15 +335,18 @@ __device__ __forceinline__ void warp_topk_keys(const uint64_t* key, int first, i
 // the 8-key tiles j0 = 8 w, 8 (w + 8), ...; one DMMA (m8n8k4) per 4 columns
 // with A = the 8 query-block means (shared memory, rows padded to D + 4
 // doubles) and B = the tile's 8 key-block means (read from L2), so C holds
-// the tile's 8 x 8 scores, summed over the columns in a fixed order; their
+// the tile's 8 x 8 scores.  The column steps go to four accumulator chains
+// (step mod 4, added pairwise at the end: a fixed order) so that a tile's
+// MMAs overlap; 64 registers leave room for four CTAs per SM.  The scores'
 // order keys go to shared memory.  Top-k: warp w alone handles row i0 + w
-// (selection, index list, mask, count), with no CTA-wide barrier.  dynamic
-// smem: keys [8][n] u64, bits [8][32] u32; static: the 8 query block means.
+// (selection, index list, mask, count), with no CTA-wide barrier; rows of at
+// most 128 candidates keep them sorted in registers.  dynamic smem: keys
+// [8][n] u64, bits [8][32] u32; static: the 8 query block means.
 constexpr int kRowsPerCta = 8;
 constexpr int kRowsKernelMaxN = 1024;
 
 template <int D>
-__global__ void __launch_bounds__(kSelThreads, 2)
+__global__ void __launch_bounds__(kSelThreads, 4)
 score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kbar, int n,
                   int topk, int force_sink, int words, int32_t* __restrict__ idx,
                   int32_t* __restrict__ cnt, uint32_t* __restrict__ mask) {
@@ -301,21 +375,17 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
 
     {
         const int g = lane >> 2, t = lane & 3;  // fragment row / column of the DMMA
+        const double* qr = qs + g * QS + t;
+        // one tile at a time, summed in four chains (column steps s mod 4) so
+        // that the float64 MMAs of a tile overlap
         for (int j0 = 8 * warp; j0 < kend; j0 += 8 * NW) {
             const double* kr = kb + (size_t)min(j0 + g, kend - 1) * D + t;  // past the end: unused
-            const double* qr = qs + g * QS + t;
-            double c0 = 0.0, c1 = 0.0;
-#pragma unroll 8
-            for (int s4 = 0; s4 < D / 4; ++s4) {
-                const double av = qr[4 * s4];
-                const double bv = kr[4 * s4];
-                asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-                             : "+d"(c0), "+d"(c1)
-                             : "d"(av), "d"(bv));
-            }
+            double c[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
+#pragma unroll 16
+            for (int s4 = 0; s4 < D / 4; ++s4) dmma8(c[s4 & 3], qr[4 * s4], kr[4 * s4]);
             const int j = j0 + 2 * t;  // C[g][2t], C[g][2t + 1]: row i0 + g, keys j, j + 1
-            if (j < kend) sc[(size_t)g * n + j] = order_key(c0);
-            if (j + 1 < kend) sc[(size_t)g * n + j + 1] = order_key(c1);
+            if (j < kend) sc[(size_t)g * n + j] = order_key((c[0][0] + c[1][0]) + (c[2][0] + c[3][0]));
+            if (j + 1 < kend) sc[(size_t)g * n + j + 1] = order_key((c[0][1] + c[1][1]) + (c[2][1] + c[3][1]));
         }
     }
     __syncthreads();  // all rows' keys visible
@@ -337,6 +407,8 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
     const int r = topk - (sink ? 2 : 1);     // free slots (>= 0, host-checked)
     if (ncand <= r) {
         for (int j = first + lane; j < i; j += 32) atomicOr(&bits[j >> 5], 1u << (j & 31));
+    } else if (ncand <= 128) {
+        warp_topk_keys_small(srow, first, i, r, bits, lane);
     } else {
         warp_topk_keys(srow, first, i, r, bits, lane);
     }
