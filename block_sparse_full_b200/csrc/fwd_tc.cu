@@ -70,7 +70,13 @@ constexpr uint32_t OFF_MASK = OFF_MISC + 16;       // mask rows of the two query
 // the epilogue l_sel/l_uns [wg][2][row] (512), squared-difference sums [wg][row]
 // at offset 512 (256) and block-0 weights [wg][row] at offset 768 (256)
 constexpr uint32_t OFF_XCH = OFF_MASK + 2 * kMaxWords * 4;
-constexpr uint32_t SMEM_USED = OFF_XCH + 1024 * 4;
+// sparse-only forward: the key tiles the CTA uses, ascending (int16), and the
+// per-warp counts of the list compaction
+constexpr int kMaxTiles = kMaxWords * 32 * 128 / BN;  // T <= kMaxWords * 32 blocks of 128
+constexpr uint32_t OFF_LIST = OFF_XCH + 1024 * 4;
+constexpr uint32_t OFF_LCNT = OFF_LIST + kMaxTiles * 2;
+constexpr uint32_t SMEM_USED = OFF_LCNT + 16 * 4;
+static_assert(SMEM_USED + 1024 <= 232448, "shared memory per CTA");
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 
 enum : int {  // barrier indices (two-stage K / V rings, two S buffers)
@@ -112,7 +118,7 @@ __device__ __forceinline__ bool bit(const uint32_t* row, int j) {
 // none of the half's keys (diagonal tile, block 64, h = 1) and rows past T.
 __device__ __forceinline__ void half_sel(const uint32_t* mrow, int J, int I, int h, int block,
                                          bool ragged1, bool& s0, bool& s1) {
-    const int kb = (J * BN + 64 * h) / block;
+    const int kb = (J * BN + 64 * h) >> (block == 64 ? 6 : 7);  // block is 64 or 128
     s0 = bit(mrow, kb);
     s1 = bit(mrow + kMaxWords, kb);
     if (block == 64 && J == I && h == 1) s0 = s1;
@@ -193,15 +199,41 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    // key tiles the CTA processes (all causal ones for the dual forward); the
-    // diagonal tile is always used (the current block is always selected)
-    auto tile_used = [&](int j) -> bool {
-        if (!kSparse) return true;
-        bool a0, a1, b0, b1;
-        half_sel(mrow, j, I, 0, a.block, ragged1, a0, a1);
-        half_sel(mrow, j, I, 1, a.block, ragged1, b0, b1);
-        return a0 || a1 || b0 || b1;
-    };
+    // key tiles the CTA processes: every causal one for the dual forward; for
+    // the sparse stream alone the tiles that either query block selects (the
+    // diagonal tile always: the current block is always selected), listed
+    // once, ascending, by a ballot compaction, so that no role walks the
+    // unselected tiles
+    int16_t* tlist = reinterpret_cast<int16_t*>(gbase + OFF_LIST);
+    int ntiles = ntk;
+    if constexpr (kSparse) {
+        int* lcnt = reinterpret_cast<int*>(gbase + OFF_LCNT);
+        int total = 0;
+        for (int c = 0; c < ntk; c += kThreads) {  // the same trip count in every thread
+            const int j = c + (int)threadIdx.x;
+            bool used = false;
+            if (j < ntk) {
+                bool a0, a1, b0, b1;
+                half_sel(mrow, j, I, 0, a.block, ragged1, a0, a1);
+                half_sel(mrow, j, I, 1, a.block, ragged1, b0, b1);
+                used = a0 || a1 || b0 || b1;
+            }
+            const uint32_t bal = __ballot_sync(0xffffffffu, used);
+            if (lane == 0) lcnt[warp] = __popc(bal);
+            __syncthreads();
+            int before = 0, all = 0;
+            for (int w = 0; w < kThreads / 32; ++w) {
+                const int cw = lcnt[w];
+                before += w < warp ? cw : 0;
+                all += cw;
+            }
+            if (used) tlist[total + before + __popc(bal & ((1u << lane) - 1u))] = (int16_t)j;
+            total += all;
+            __syncthreads();  // lcnt is reused by the next chunk; the list is complete after the last
+        }
+        ntiles = total;
+    }
+    auto tile_at = [&](int jj) -> int { return kSparse ? (int)tlist[jj] : jj; };
 
     // Roles 0 and 1 run their loops with the whole warp (warp-uniform address and
     // descriptor arithmetic); one elected lane issues each TMA / tcgen05 op.
@@ -227,8 +259,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
         __syncwarp();
         int issued[2] = {-1, -1};
-        for (int j = 0, jj = 0; j < ntk; ++j) {
-            if (!tile_used(j)) continue;
+        for (int jj = 0; jj < ntiles; ++jj) {
+            const int j = tile_at(jj);
             const int s = jj & 1;  // ring slot of the jj-th processed tile
             const uint32_t ph = ((jj >> 1) + 1) & 1;
             const uint32_t dst = ring + s * TILE_BYTES;
@@ -243,7 +275,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             __syncwarp();
             if (s == 0) issued[0] = jj;
             else issued[1] = jj;
-            ++jj;
         }
         // Every copy this warp issued lands before the CTA exits, whether or not a
         // wait gave up (another role may abort after this warp left its loop): the
@@ -301,8 +332,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             return true;
         };
         int jj = 0, jprev = -1;
-        for (int j = 0; ok && j < ntk; ++j) {
-            if (!tile_used(j)) continue;
+        for (; ok && jj < ntiles; ++jj) {
+            const int j = tile_at(jj);
             const int s = jj & 1;
             if (!__all_sync(FULL, mbar_wait(BAR(B_KFULL + s), (jj >> 1) & 1, abort_flag, status, lim))) {
                 ok = false;
@@ -324,7 +355,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             __syncwarp();
             if (jj >= 1 && !issue_pv(jprev, jj - 1)) ok = false;
             jprev = j;
-            ++jj;
         }
         if (ok && jj > 0) issue_pv(jprev, jj - 1);
         if (elect_one()) mma_commit(BAR(B_DRAIN));  // all MMAs complete before teardown
@@ -391,9 +421,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         float lsink = 0.f;
         const bool sink_keys = !kSparse && a.sink != nullptr && c0 < a.block;
         bool ok = true;
-        int jj = 0;  // tiles processed so far (ring slot / phase)
-        for (int j = 0; j < ntk; ++j) {
-            if (!tile_used(j)) continue;
+        for (int jj = 0; jj < ntiles; ++jj) {  // jj: tiles processed so far (ring slot / phase)
+            const int j = tile_at(jj);
             const int b = jj & 1;
             // warp-uniform outcome: the TMEM loads below are warp-collective
             const bool got = __all_sync(
@@ -539,7 +568,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tmem_wait_st();
             fence_before_sync();
             mbar_arrive(BAR(B_PREADY + b));
-            ++jj;
         }
         // Every MMA (the last PV included) has completed once B_DRAIN has.  A
         // parity wait on B_PVDONE for the last tile is not enough: the softmax
