@@ -24,8 +24,9 @@ namespace ssa {
 namespace {
 
 constexpr int kTile = 32;
-constexpr int kThreads = 128;
+constexpr int kThreads = 512;  // 16 warps of 2 rows: the rows' dependency chains overlap
 constexpr int kRowsPerWarp = kTile / (kThreads / 32);
+constexpr int kPreThreads = 128;  // preprocess: a warp per row
 
 struct BwdWs {
     float* gf;
@@ -43,10 +44,10 @@ BwdWs carve(const ssa_params_t& p, void* ws) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kPreThreads)
 bwd_pre_kernel(const T* __restrict__ hf, const T* __restrict__ hs, const T* __restrict__ dhf,
                const T* __restrict__ dhs, size_t rows, int D, float cf, float cs, BwdWs w) {
-    const size_t row = (size_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const size_t row = (size_t)blockIdx.x * (kPreThreads / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
     float sf = 0.f, ss = 0.f;
@@ -269,7 +270,7 @@ int launch_typed(const ssa_params_t& p, const void* q, const void* k, const void
     const BwdWs w = carve(p, ws);
     const size_t rows = num_rows(p);
     const double two_over_n = 2.0 / (double)num_elems(p);
-    bwd_pre_kernel<T><<<(unsigned)((rows + 3) / 4), kThreads, 0, s>>>(
+    bwd_pre_kernel<T><<<(unsigned)((rows + kPreThreads / 32 - 1) / (kPreThreads / 32)), kPreThreads, 0, s>>>(
         static_cast<const T*>(hf), static_cast<const T*>(hs), static_cast<const T*>(dhf),
         static_cast<const T*>(dhs), rows, D, (float)(w_s * two_over_n), (float)(w_c * two_over_n), w);
     int st = check_launch("bwd_pre_kernel");

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 from block_sparse_full_b200 import ssa
-from block_sparse_full_b200.inputs import WORKLOADS, make_inputs
+from block_sparse_full_b200.inputs import WORKLOADS, Workload, make_inputs
 from oracle import ssa_oracle as O
 
 from gpu_parity_util import (DEV, TOL, log, oracle_mask_to_dev, oracle_select, params,
@@ -90,6 +90,17 @@ def test_sparse_fwd_T65536_sink_sampled_rows():
     w = WORKLOADS["bf16_T65536_H8_sink"]
     rows = np.unique(np.concatenate([sample_rows(w.T, 4096, 8, seed=23), [w.T - 1]]))
     _, _, p, _, out, ref = _case(w, rows=rows, heads=[2, 7])
+    compare_sparse(w.name + "/sparse", "bf16", out, ref, rows=rows)
+
+
+def test_sparse_fwd_T131072_sampled_rows():
+    # 1024 key tiles per head at the last query tile: the CTA's list of
+    # selected tiles is compacted over several 384-tile chunks
+    w = Workload("bf16_T131072_H2_sink", B=1, H=2, T=131072, D=128, block=128, topk=16,
+                 dtype="bf16", plant="sink", seed=47)
+    rows = np.unique(np.concatenate([sample_rows(w.T, 16384, 6, seed=29), [w.T - 1]]))
+    _, _, p, _, out, ref = _case(w, rows=rows)
+    assert ssa.ssa_kernel_path(p) == 1
     compare_sparse(w.name + "/sparse", "bf16", out, ref, rows=rows)
 
 
