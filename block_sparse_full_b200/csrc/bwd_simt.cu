@@ -1,6 +1,5 @@
 // Backward through both SSA attention streams on CUDA cores (float32
-// arithmetic).  Used for float32 inputs, bf16 with D = 64 and under
-// SSA_FLAG_FORCE_SIMT.
+// arithmetic).  Used for float32 inputs and under SSA_FLAG_FORCE_SIMT.
 //
 // Upstream reaching each output ("Sintesi Tecnica: SSA", section 2: the
 // full stream gives gradient to every token; L_sparsity pulls h_full toward

@@ -1,7 +1,6 @@
 // Dual-stream forward on CUDA cores (float32 arithmetic): the exact-fp32
 // path for float32 inputs (where tf32 tensor cores would miss a 1e-4
-// tolerance), bf16 with D = 64, and the comparator behind
-// SSA_FLAG_FORCE_SIMT.
+// tolerance) and the comparator behind SSA_FLAG_FORCE_SIMT.
 //
 // One CTA = 32 query rows of one (b, h), 16 warps x 2 rows (a row's logit,
 // softmax and P V chains are serial, so more warps with fewer rows each
