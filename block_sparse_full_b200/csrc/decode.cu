@@ -89,20 +89,21 @@ __device__ unsigned int g_decode_status;
 
 // Shared memory of the step kernel, the same layout in every CTA of a cluster:
 //   order keys [nb] u64 (every CTA holds all of them) | set bitmask [nb / 32 + 1] u32 |
-//   selected blocks [topk] i32 | partials [cluster][2 + D] f32 (the leader's
+//   selected blocks [topk] i32 | popcount prefix of the bitmask words [nb / 32 + 2] i32 | partials [cluster][2 + D] f32 (the leader's
 //   are used) | scores [nbuf * block] f32 | p [nbuf * block] bf16 | o partial
 //   sums [KG][D] f32 | mbarriers (copies, partials) | keys [nbuf][block][D] T
 //   (bf16: per block, D / 64 tiles [block][64] in the 128-byte swizzle) |
 //   values likewise.
 struct StepSmem {
-    size_t score, bits, sel, part, ps, pb, og, bar, kbuf, vbuf, total;
+    size_t score, bits, sel, wpre, part, ps, pb, og, bar, kbuf, vbuf, total;
     __host__ __device__ StepSmem(int nb, int topk, int D, int cluster, int nbuf, int block, int esize,
                                  int threads) {
         auto up = [](size_t x, size_t a) { return (x + a - 1) / a * a; };
         score = 0;
         bits = score + (size_t)nb * 8;
         sel = bits + ((size_t)nb / 32 + 1) * 4;
-        part = up(sel + (size_t)topk * 4, 16);
+        wpre = sel + (size_t)topk * 4;
+        part = up(wpre + ((size_t)nb / 32 + 2) * 4, 16);
         ps = part + (size_t)cluster * (2 + D) * 4;
         pb = ps + (size_t)nbuf * block * 4;
         og = up(pb + (size_t)nbuf * block * 2, 16);
@@ -213,6 +214,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     uint64_t* key = reinterpret_cast<uint64_t*>(sm + L.score);
     uint32_t* bits = reinterpret_cast<uint32_t*>(sm + L.bits);
     int32_t* sel = reinterpret_cast<int32_t*>(sm + L.sel);
+    int32_t* wpre = reinterpret_cast<int32_t*>(sm + L.wpre);
     float* part = reinterpret_cast<float*>(sm + L.part);
     float* ps = reinterpret_cast<float*>(sm + L.ps);
     __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(sm + L.pb);
@@ -267,7 +269,9 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     // lanes of a warp count for one candidate, each over every nseg-th rival, four
     // rivals per iteration.  Past kSplitRankMin candidates the CTAs of the cluster
     // split them (CTA rank counts for candidates rank, rank + kCluster, ...) and
-    // set the kept bits in every CTA.
+    // OR their bitmask words into every other CTA (one remote reduction per word
+    // and CTA, all in flight at once).  Then every thread places the set bits it
+    // owns by a popcount prefix of the words: the ascending list.
     {
         const bool sink = force_sink && i > 0;
         const int want = topk < i + 1 ? topk : i + 1;  // fewer candidates than places: take all
@@ -309,46 +313,48 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 }
                 int ahead = (a0 + a1) + (a2 + a3);
                 for (int off = nseg >> 1; off > 0; off >>= 1) ahead += __shfl_xor_sync(0xffffffffu, ahead, off);
-                if (live && seg == 0 && ahead < r) {
-                    const uint32_t bitv = 1u << (j & 31);
-                    atomicOr(&bits[j >> 5], bitv);
-                    if (split)
-                        for (int q2 = 1; q2 < kCluster; ++q2)
-                            atomicOr(cluster.map_shared_rank(bits, (rank + q2) % kCluster) + (j >> 5), bitv);
-                }
+                if (live && seg == 0 && ahead < r) atomicOr(&bits[j >> 5], 1u << (j & 31));
             }
         }
-        if (split)
+        __syncthreads();  // this CTA's bits are complete
+        if (split) {
+            for (int e = tid; e < words * (kCluster - 1); e += NT) {
+                const int w = e % words, q2 = 1 + e / words;
+                const uint32_t wv = bits[w];
+                if (wv != 0u) atomicOr(cluster.map_shared_rank(bits, (rank + q2) % kCluster) + w, wv);
+            }
             cluster.sync();  // every CTA's kept bits are in every CTA
-        else
-            __syncthreads();
-        if (warp == 0) {  // the ascending list (-1 padded) by popcount prefix
-            int32_t* irow = (idx_out && rank == 0) ? idx_out + bh * topk : nullptr;
+        }
+        if (warp == 0) {  // popcount prefix of the words, 32 at a time
             int basep = 0;
             for (int w0 = 0; w0 < words; w0 += 32) {
                 const int w = w0 + lane;
-                const uint32_t wv = w < words ? bits[w] : 0u;
-                const int c = __popc(wv);
+                const int c = w < words ? __popc(bits[w]) : 0;
                 int incl = c;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
                     const int o = __shfl_up_sync(0xffffffffu, incl, off);
                     if (lane >= off) incl += o;
                 }
-                int pos = basep + incl - c;
-                for (uint32_t b = wv; b != 0u; b &= b - 1u, ++pos) {
-                    if (pos < topk) {  // NaN scores: stay in bounds
-                        const int vv = w * 32 + __ffs(b) - 1;
-                        sel[pos] = vv;
-                        if (irow) irow[pos] = vv;
-                    }
-                }
+                if (w < words) wpre[w] = basep + incl - c;
                 basep += __shfl_sync(0xffffffffu, incl, 31);
             }
-            if (irow)
-                for (int pp = basep + lane; pp < topk; pp += 32) irow[pp] = -1;
             if (lane == 0) nsel_s = basep < topk ? basep : topk;
         }
+        __syncthreads();
+        int32_t* irow = (idx_out && rank == 0) ? idx_out + bh * topk : nullptr;
+        for (int j = tid; j <= i; j += NT) {
+            const uint32_t wv = bits[j >> 5];
+            if ((wv >> (j & 31)) & 1u) {
+                const int pos = wpre[j >> 5] + __popc(wv & ((1u << (j & 31)) - 1u));
+                if (pos < topk) {  // NaN scores: stay in bounds
+                    sel[pos] = j;
+                    if (irow) irow[pos] = j;
+                }
+            }
+        }
+        if (irow)
+            for (int pp = nsel_s + tid; pp < topk; pp += NT) irow[pp] = -1;
         __syncthreads();
     }
 

@@ -424,9 +424,15 @@ score_topk_kernel(const double* __restrict__ qbar, const double* __restrict__ kb
     }
     const int total = __shfl_sync(0xffffffffu, incl, 31);
     int32_t* irow = idx + row * topk;
-    int pos = incl - c;
-    for (uint32_t b = wv; b != 0u; b &= b - 1u, ++pos)
-        if (pos < topk) irow[pos] = lane * 32 + __ffs(b) - 1;  // NaN scores: stay in bounds
+    // word by word, lane l places bit l: no lane walks its word's bits one by one
+    for (int w = 0; w <= (i >> 5); ++w) {
+        const uint32_t ww = __shfl_sync(0xffffffffu, wv, w);
+        const int before = __shfl_sync(0xffffffffu, incl - c, w);
+        if ((ww >> lane) & 1u) {
+            const int pos = before + __popc(ww & ((1u << lane) - 1u));
+            if (pos < topk) irow[pos] = w * 32 + lane;  // NaN scores: stay in bounds
+        }
+    }
     for (int p = total + lane; p < topk; p += 32) irow[p] = -1;
     if (lane < words) mask[row * words + lane] = wv;
     if (lane == 0) cnt[row] = total < topk ? total : topk;
