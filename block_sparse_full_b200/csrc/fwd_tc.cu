@@ -135,15 +135,17 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity, uint64
 // D: head dim, 64 or 128 (one or two 64-column boxes per tile; an S tile
 // takes D/16 MMA k-steps; each softmax warpgroup owns D/2 output columns).
 // kSparse = false: the dual forward (both streams).  kSparse = true: the
-// sparse stream alone (inference, the same operations as MoBA): key tiles
-// that neither of the tile's query blocks selects are skipped by every
-// role, the running max is taken over selected keys only, unselected
-// (row, half) pairs get P = 0, one accumulator (O_sel), and the epilogue
-// writes h_sparse and lse_sparse only.
+// sparse stream alone (inference, the same operations as MoBA): every role
+// walks only the CTA's list of selected keys (with blocks of 64, the
+// off-diagonal selected blocks packed two to a tile, each half loaded as its
+// own 64-row box), the running max is taken over selected keys only,
+// unselected (row, half) pairs get P = 0, one accumulator (O_sel), and the
+// epilogue writes h_sparse and lse_sparse only.
 template <int D, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_hf,
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k64,
+              const __grid_constant__ CUtensorMap tm_v64, const __grid_constant__ CUtensorMap tm_hf,
               const __grid_constant__ CUtensorMap tm_hs, const FwdArgs a) {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
     constexpr uint32_t kTileBytes = BM * D * 2;  // bytes a Q / K / V tile load brings
@@ -199,24 +201,34 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    // key tiles the CTA processes: every causal one for the dual forward; for
-    // the sparse stream alone the tiles that either query block selects (the
-    // diagonal tile always: the current block is always selected), listed
-    // once, ascending, by a ballot compaction, so that no role walks the
-    // unselected tiles
+    // key tiles the CTA processes: every causal one for the dual forward.  For
+    // the sparse stream alone, blocks of 128 keys: the tiles that the query
+    // block selects (the diagonal tile always: the current block is always
+    // selected).  Blocks of 64 keys: the off-diagonal key blocks that either
+    // query block selects, paired in ascending order into tiles of two
+    // 64-key halves (a last odd block leaves its second half empty), then the
+    // diagonal tile.  Either list is built once, ascending, by a ballot
+    // compaction over all threads, so that no role walks unselected tiles.
     int16_t* tlist = reinterpret_cast<int16_t*>(gbase + OFF_LIST);
     int ntiles = ntk;
+    const bool packed = kSparse && a.block == 64;
+    int nsel_off = 0;  // packed: selected off-diagonal key blocks
     if constexpr (kSparse) {
         int* lcnt = reinterpret_cast<int*>(gbase + OFF_LCNT);
+        const int nitems = packed ? 2 * I : ntk;  // key blocks below the diagonal, or tiles
         int total = 0;
-        for (int c = 0; c < ntk; c += kThreads) {  // the same trip count in every thread
+        for (int c = 0; c < nitems; c += kThreads) {  // the same trip count in every thread
             const int j = c + (int)threadIdx.x;
             bool used = false;
-            if (j < ntk) {
-                bool a0, a1, b0, b1;
-                half_sel(mrow, j, I, 0, a.block, ragged1, a0, a1);
-                half_sel(mrow, j, I, 1, a.block, ragged1, b0, b1);
-                used = a0 || a1 || b0 || b1;
+            if (j < nitems) {
+                if (packed) {
+                    used = bit(mrow, j) || bit(mrow + kMaxWords, j);
+                } else {
+                    bool a0, a1, b0, b1;
+                    half_sel(mrow, j, I, 0, a.block, ragged1, a0, a1);
+                    half_sel(mrow, j, I, 1, a.block, ragged1, b0, b1);
+                    used = a0 || a1 || b0 || b1;
+                }
             }
             const uint32_t bal = __ballot_sync(0xffffffffu, used);
             if (lane == 0) lcnt[warp] = __popc(bal);
@@ -231,9 +243,36 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             total += all;
             __syncthreads();  // lcnt is reused by the next chunk; the list is complete after the last
         }
-        ntiles = total;
+        if (packed) {
+            nsel_off = total;
+            ntiles = (total + 1) / 2 + 1;
+        } else {
+            ntiles = total;
+        }
     }
-    auto tile_at = [&](int jj) -> int { return kSparse ? (int)tlist[jj] : jj; };
+    // tile jj: natural key tile j (j >= 0), or (packed) the key blocks kb0, kb1
+    // of its two halves (kb1 = -1: empty half)
+    struct TileDesc {
+        int j, kb0, kb1;
+    };
+    auto tile_desc = [&](int jj) -> TileDesc {
+        if (kSparse && packed) {
+            if (jj == ntiles - 1) return {I, 0, 0};
+            return {-1, (int)tlist[2 * jj], 2 * jj + 1 < nsel_off ? (int)tlist[2 * jj + 1] : -1};
+        }
+        return {kSparse ? (int)tlist[jj] : jj, 0, 0};
+    };
+    // selection of half h of a tile by the tile's two query blocks
+    auto sel_half = [&](const TileDesc& td, int h, bool& s0, bool& s1) {
+        if (td.j >= 0) {
+            half_sel(mrow, td.j, I, h, a.block, ragged1, s0, s1);
+            return;
+        }
+        const int kb = h ? td.kb1 : td.kb0;
+        s0 = kb >= 0 && bit(mrow, kb);
+        s1 = kb >= 0 && bit(mrow + kMaxWords, kb);
+        if (ragged1) s1 = s0;
+    };
 
     // Roles 0 and 1 run their loops with the whole warp (warp-uniform address and
     // descriptor arithmetic); one elected lane issues each TMA / tcgen05 op.
@@ -245,6 +284,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // for the other warpgroup's PV product.
         const bool is_k = warp == 0;
         const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+        const CUtensorMap* tm64 = is_k ? &tm_k64 : &tm_v64;  // 64-row boxes: packed halves
         const int FULLB = is_k ? B_KFULL : B_VFULL, EMPTYB = is_k ? B_KEMPTY : B_VEMPTY;
         const uint32_t ring = base + (is_k ? OFF_K : OFF_V);
         if (elect_one()) {
@@ -260,7 +300,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         __syncwarp();
         int issued[2] = {-1, -1};
         for (int jj = 0; jj < ntiles; ++jj) {
-            const int j = tile_at(jj);
+            const TileDesc td = tile_desc(jj);
             const int s = jj & 1;  // ring slot of the jj-th processed tile
             const uint32_t ph = ((jj >> 1) + 1) & 1;
             const uint32_t dst = ring + s * TILE_BYTES;
@@ -268,9 +308,23 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 break;
             if (elect_one()) {
                 mbar_expect_tx(BAR(FULLB + s), kTileBytes);
+                if (td.j >= 0) {
 #pragma unroll
-                for (int x = 0; x < D / 64; ++x)
-                    tma_load_3d(dst + x * HALF_BYTES, tm, BAR(FULLB + s), 64 * x, j * BN, bh);
+                    for (int x = 0; x < D / 64; ++x)
+                        tma_load_3d(dst + x * HALF_BYTES, tm, BAR(FULLB + s), 64 * x, td.j * BN, bh);
+                } else {
+                    // two 64-row boxes per 64-column box: the same swizzled layout as
+                    // one 128-row box; an empty half repeats the first block (its
+                    // selection bits are clear, so it takes no part)
+#pragma unroll
+                    for (int x = 0; x < D / 64; ++x)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int kb = (h && td.kb1 >= 0) ? td.kb1 : td.kb0;
+                            tma_load_3d(dst + x * HALF_BYTES + h * (64 * 128), tm64, BAR(FULLB + s), 64 * x,
+                                        kb * 64, bh);
+                        }
+                }
             }
             __syncwarp();
             if (s == 0) issued[0] = jj;
@@ -295,7 +349,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // SBO = 1 KB apart; 16 keys (2 KB) per MMA
         const uint64_t vdesc0 = smem_desc_sw128(base + OFF_V, HALF_BYTES, 1024);
         bool ok = __all_sync(FULL, mbar_wait(BAR(B_QFULL), 0, abort_flag, status, lim));
-        auto issue_pv = [&](int i, int ii) -> bool {  // key tile i, ii-th processed
+        auto issue_pv = [&](const TileDesc& td, int ii) -> bool {  // the ii-th processed tile
             const int b = ii & 1;
             const uint32_t ph = (ii >> 1) & 1;
             if (!__all_sync(FULL, mbar_wait(BAR(B_PREADY + b), ph, abort_flag, status, lim))) return false;
@@ -304,8 +358,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const uint64_t vd = desc_add(vdesc0, b * TILE_BYTES);
             const uint32_t sb = tmem + (b ? TM_S1 : TM_S0);
             bool s0[2], s1[2];
-            half_sel(mrow, i, I, 0, a.block, ragged1, s0[0], s1[0]);
-            half_sel(mrow, i, I, 1, a.block, ragged1, s0[1], s1[1]);
+            sel_half(td, 0, s0[0], s1[0]);
+            sel_half(td, 1, s0[1], s1[1]);
             if (elect_one()) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -331,9 +385,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             __syncwarp();
             return true;
         };
-        int jj = 0, jprev = -1;
+        int jj = 0;
+        TileDesc tdprev = {0, 0, 0};
         for (; ok && jj < ntiles; ++jj) {
-            const int j = tile_at(jj);
+            const TileDesc td = tile_desc(jj);
             const int s = jj & 1;
             if (!__all_sync(FULL, mbar_wait(BAR(B_KFULL + s), (jj >> 1) & 1, abort_flag, status, lim))) {
                 ok = false;
@@ -353,10 +408,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 mma_commit(BAR(B_KEMPTY + s));
             }
             __syncwarp();
-            if (jj >= 1 && !issue_pv(jprev, jj - 1)) ok = false;
-            jprev = j;
+            if (jj >= 1 && !issue_pv(tdprev, jj - 1)) ok = false;
+            tdprev = td;
         }
-        if (ok && jj > 0) issue_pv(jprev, jj - 1);
+        if (ok && jj > 0) issue_pv(tdprev, jj - 1);
         if (elect_one()) mma_commit(BAR(B_DRAIN));  // all MMAs complete before teardown
         __syncwarp();
         wait_drain(BAR(B_DRAIN), 0, kDrainLimitNs);
@@ -422,7 +477,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const bool sink_keys = !kSparse && a.sink != nullptr && c0 < a.block;
         bool ok = true;
         for (int jj = 0; jj < ntiles; ++jj) {  // jj: tiles processed so far (ring slot / phase)
-            const int j = tile_at(jj);
+            const TileDesc td = tile_desc(jj);
+            const int j = td.j;  // -1 for a packed tile (never the diagonal)
             const int b = jj & 1;
             // warp-uniform outcome: the TMEM loads below are warp-collective
             const bool got = __all_sync(
@@ -450,7 +506,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (c0 + c > r) s[c] = -INFINITY;
             }
             bool s0, s1;
-            half_sel(mrow, j, I, wg, a.block, ragged1, s0, s1);
+            sel_half(td, wg, s0, s1);
             const bool mixed = s0 != s1;
             const bool row_sel = mixed ? ((r < 64 || a.block == 128) ? s0 : s1) : s0;
             if (kSparse && !row_sel) {  // the sparse stream alone: this half is not attended
@@ -705,14 +761,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [BH, T, D] bf16 viewed as a 3-D tensor (d, t, bh); box = 64 d x 128 t,
-// 128-byte swizzle; rows past T are zero-filled by the TMA unit.
-int make_map(CUtensorMap* m, const void* ptr, int BH, int T, int D) {
+// [BH, T, D] bf16 viewed as a 3-D tensor (d, t, bh); box = 64 d x `rows` t
+// (128 by default), 128-byte swizzle; rows past T are zero-filled by the TMA
+// unit.
+int make_map(CUtensorMap* m, const void* ptr, int BH, int T, int D, int rows = BM) {
     auto fn = encode_fn();
     if (!fn) return fail(SSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)T, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)T * D * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)BM, 1};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -735,10 +792,13 @@ template <int D, bool kSparse>
 int launch_fwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, const void* v,
                        const uint32_t* mask, const FwdArgs& outs, cudaStream_t s) {
     const int BH = p.B * p.H;
-    CUtensorMap mq, mk, mv, mhf, mhs;
+    CUtensorMap mq, mk, mv, mk64, mv64, mhf, mhs;
     int st = make_map(&mq, q, BH, p.T, D);
     if (st == SSA_OK) st = make_map(&mk, k, BH, p.T, D);
     if (st == SSA_OK) st = make_map(&mv, v, BH, p.T, D);
+    // 64-row boxes: the halves of the sparse-only forward's packed tiles
+    if (st == SSA_OK) st = make_map(&mk64, k, BH, p.T, D, 64);
+    if (st == SSA_OK) st = make_map(&mv64, v, BH, p.T, D, 64);
     if (st == SSA_OK) st = make_map(&mhs, outs.h_sparse, BH, p.T, D);
     // the sparse-only kernel writes h_sparse alone (the h_full map is not used)
     if (st == SSA_OK) st = make_map(&mhf, kSparse ? outs.h_sparse : outs.h_full, BH, p.T, D);
@@ -761,7 +821,7 @@ int launch_fwd_tc_impl(const ssa_params_t& p, const void* q, const void* k, cons
     a.scale_log2 = p.sm_scale * 1.4426950408889634f;
     a.timeout_ns = wait_limit_ns();
     const unsigned grid = (unsigned)((size_t)BH * ((p.T + BM - 1) / BM));
-    fwd_tc_kernel<D, kSparse><<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mhf, mhs, a);
+    fwd_tc_kernel<D, kSparse><<<grid, kThreads, SMEM_BYTES, s>>>(mq, mk, mv, mk64, mv64, mhf, mhs, a);
     return check_launch(kSparse ? "fwd_tc_kernel<sparse>" : "fwd_tc_kernel");
 }
 }  // namespace
