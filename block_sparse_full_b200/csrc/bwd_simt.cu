@@ -22,9 +22,10 @@
 namespace ssa {
 namespace {
 
-constexpr int kTile = 32;
-constexpr int kThreads = 512;  // 16 warps of 2 rows: the rows' dependency chains overlap
-constexpr int kRowsPerWarp = kTile / (kThreads / 32);
+constexpr int kRowsB = 16;   // rows per CTA: queries (dq) or keys (dk/dv)
+constexpr int kChunk = 32;   // keys (dq) or queries (dk/dv) per streamed chunk: lane j owns chunk row j
+constexpr int kThreads = 512;  // a warp per row: the rows' dependency chains overlap
+constexpr int kRowsPerWarp = kRowsB / (kThreads / 32);
 constexpr int kPreThreads = 128;  // preprocess: a warp per row
 
 struct BwdWs {
@@ -70,9 +71,9 @@ bwd_pre_kernel(const T* __restrict__ hf, const T* __restrict__ hs, const T* __re
 
 template <int D>
 struct DqSmem {
-    float q[kTile][D], gf[kTile][D], gs[kTile][D];
-    float k[kTile][D + 1], v[kTile][D + 1];
-    float lf[kTile], ls[kTile], df[kTile], ds[kTile];
+    float q[kRowsB][D], gf[kRowsB][D], gs[kRowsB][D];
+    float k[kChunk][D + 1], v[kChunk][D + 1];
+    float lf[kRowsB], ls[kRowsB], df[kRowsB], ds[kRowsB];
     uint32_t mrow[256];
 };
 
@@ -85,21 +86,21 @@ bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
     constexpr int DPL = D / 32;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     DqSmem<D>& sm = *reinterpret_cast<DqSmem<D>*>(smem_raw);
-    const int ntiles = T_ / kTile;
+    const int ntiles = T_ / kRowsB;
     const int tile = ntiles - 1 - (int)(blockIdx.x / BH);
     const size_t bh = blockIdx.x % BH;
-    const int t0 = tile * kTile;
+    const int t0 = tile * kRowsB;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t base = bh * (size_t)T_ * D;
     const size_t rbase = bh * (size_t)T_ + t0;
 
-    for (int e = tid; e < kTile * D; e += kThreads) {
+    for (int e = tid; e < kRowsB * D; e += kThreads) {
         const size_t g = base + (size_t)t0 * D + e;
         sm.q[e / D][e % D] = to_f32(q[g]);
         sm.gf[e / D][e % D] = w.gf[g];
         sm.gs[e / D][e % D] = w.gs[g];
     }
-    if (tid < kTile) {
+    if (tid < kRowsB) {
         sm.lf[tid] = lse_f[rbase + tid];
         sm.ls[tid] = lse_s[rbase + tid];
         sm.df[tid] = w.df[rbase + tid];
@@ -114,9 +115,11 @@ bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 #pragma unroll
         for (int u = 0; u < DPL; ++u) acc[r][u] = 0.f;
 
-    for (int s0 = 0; s0 < t0 + kTile; s0 += kTile) {
+    // chunks of 32 keys from 0 (a chunk lies inside one key block; keys past a
+    // row are masked)
+    for (int s0 = 0; s0 < t0 + kRowsB; s0 += kChunk) {
         __syncthreads();
-        for (int e = tid; e < kTile * D; e += kThreads) {
+        for (int e = tid; e < kChunk * D; e += kThreads) {
             const size_t g = base + (size_t)s0 * D + e;
             sm.k[e / D][e % D] = to_f32(k[g]);
             sm.v[e / D][e % D] = to_f32(v[g]);
@@ -145,7 +148,7 @@ bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
                 dsv += ps * (dps - sm.ds[rr]);
             }
 #pragma unroll 8
-            for (int j = 0; j < kTile; ++j) {
+            for (int j = 0; j < kChunk; ++j) {
                 const float dj = __shfl_sync(0xffffffffu, dsv, j);
 #pragma unroll
                 for (int u = 0; u < DPL; ++u) acc[r][u] = fmaf(dj, sm.k[j][lane + 32 * u], acc[r][u]);
@@ -162,9 +165,9 @@ bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
 
 template <int D>
 struct DkvSmem {
-    float k[kTile][D], v[kTile][D];
-    float q[kTile][D + 1], gf[kTile][D + 1], gs[kTile][D + 1];
-    float lf[kTile], ls[kTile], df[kTile], ds[kTile];
+    float k[kRowsB][D], v[kRowsB][D];
+    float q[kChunk][D + 1], gf[kChunk][D + 1], gs[kChunk][D + 1];
+    float lf[kChunk], ls[kChunk], df[kChunk], ds[kChunk];
 };
 
 template <typename T, int D>
@@ -178,13 +181,13 @@ bwd_dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     DkvSmem<D>& sm = *reinterpret_cast<DkvSmem<D>*>(smem_raw);
     const int tile = (int)(blockIdx.x / BH);  // key tile 0 sees every query: first
     const size_t bh = blockIdx.x % BH;
-    const int s_base = tile * kTile;
+    const int s_base = tile * kRowsB;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t base = bh * (size_t)T_ * D;
     const int n = T_ / block;
     const int kblk = s_base / block;
 
-    for (int e = tid; e < kTile * D; e += kThreads) {
+    for (int e = tid; e < kRowsB * D; e += kThreads) {
         const size_t g = base + (size_t)s_base * D + e;
         sm.k[e / D][e % D] = to_f32(k[g]);
         sm.v[e / D][e % D] = to_f32(v[g]);
@@ -195,15 +198,17 @@ bwd_dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
 #pragma unroll
         for (int u = 0; u < DPL; ++u) adk[r][u] = adv[r][u] = 0.f;
 
-    for (int t0 = s_base; t0 < T_; t0 += kTile) {
+    // chunks of 32 queries from the 32-aligned chunk holding the first key (a
+    // chunk lies inside one query block; queries before a key are masked)
+    for (int t0 = s_base & ~(kChunk - 1); t0 < T_; t0 += kChunk) {
         __syncthreads();
-        for (int e = tid; e < kTile * D; e += kThreads) {
+        for (int e = tid; e < kChunk * D; e += kThreads) {
             const size_t g = base + (size_t)t0 * D + e;
             sm.q[e / D][e % D] = to_f32(q[g]);
             sm.gf[e / D][e % D] = w.gf[g];
             sm.gs[e / D][e % D] = w.gs[g];
         }
-        if (tid < kTile) {
+        if (tid < kChunk) {
             const size_t rr = bh * (size_t)T_ + t0 + tid;
             sm.lf[tid] = lse_f[rr];
             sm.ls[tid] = lse_s[rr];
@@ -237,7 +242,7 @@ bwd_dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
                 dsv += ps * (dps - sm.ds[lane]);
             }
 #pragma unroll 4
-            for (int j = 0; j < kTile; ++j) {
+            for (int j = 0; j < kChunk; ++j) {
                 const float pfj = __shfl_sync(0xffffffffu, pf, j);
                 const float psj = __shfl_sync(0xffffffffu, ps, j);
                 const float dj = __shfl_sync(0xffffffffu, dsv, j);
@@ -276,7 +281,7 @@ int launch_typed(const ssa_params_t& p, const void* q, const void* k, const void
     if (st != SSA_OK) return st;
 
     const int BH = p.B * p.H;
-    const unsigned grid = (unsigned)((size_t)BH * (p.T / kTile));
+    const unsigned grid = (unsigned)((size_t)BH * (p.T / kRowsB));
     size_t smem = sizeof(DqSmem<D>);
     cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -309,7 +314,7 @@ int launch_bwd_simt(const ssa_params_t& p, const void* q, const void* k, const v
                     const float* ls, const void* dhf, const void* dhs, float w_s, float w_c,
                     void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
     if (mask_words(p) > 256) return fail(SSA_ERR_UNSUPPORTED, "bwd_simt: more than 8192 blocks");
-    if ((size_t)p.B * p.H * (p.T / kTile) > 0x7fffffffull)
+    if ((size_t)p.B * p.H * (p.T / kRowsB) > 0x7fffffffull)
         return fail(SSA_ERR_UNSUPPORTED, "bwd_simt: grid too large");
     const bool bf = p.dtype == SSA_BF16;
 #define SSA_BWD_ARGS p, q, k, v, mask, hf, hs, lf, ls, dhf, dhs, w_s, w_c, dq, dk, dv, ws, s

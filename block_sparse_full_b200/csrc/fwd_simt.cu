@@ -2,9 +2,9 @@
 // path for float32 inputs (where tf32 tensor cores would miss a 1e-4
 // tolerance) and the comparator behind SSA_FLAG_FORCE_SIMT.
 //
-// One CTA = 32 query rows of one (b, h), 16 warps x 2 rows (a row's logit,
-// softmax and P V chains are serial, so more warps with fewer rows each
-// overlap them).  K/V stream
+// One CTA = 16 query rows of one (b, h), a warp per row (a row's logit,
+// softmax and P V chains are serial, so many warps with one row each overlap
+// them, and small problems still give the GPU many CTAs).  K/V stream
 // through shared memory in chunks of 32 keys; lane j owns key j of the chunk
 // for the logits and dimension lane + 32u of the accumulators.  A chunk lies
 // inside one key block and the CTA's rows inside one query block, so the
@@ -21,9 +21,9 @@
 namespace ssa {
 namespace {
 
-constexpr int kRows = 32;  // query rows per CTA
+constexpr int kRows = 16;  // query rows per CTA
 constexpr int kKeys = 32;  // keys per chunk
-constexpr int kThreads = 512;  // 16 warps of 2 rows: the rows' dependency chains overlap
+constexpr int kThreads = 512;  // 16 warps of 1 row: the rows' dependency chains overlap
 constexpr int kRowsPerWarp = kRows / (kThreads / 32);
 
 template <int D>

@@ -308,10 +308,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 break;
             if (elect_one()) {
                 mbar_expect_tx(BAR(FULLB + s), kTileBytes);
-                if (td.j >= 0) {
+                if (td.j >= 0 || (td.kb1 == td.kb0 + 1 && (td.kb0 & 1) == 0)) {
+                    // a natural key tile (or a packed pair that is one): one 128-row box
+                    const int row0 = td.j >= 0 ? td.j * BN : td.kb0 * 64;
 #pragma unroll
                     for (int x = 0; x < D / 64; ++x)
-                        tma_load_3d(dst + x * HALF_BYTES, tm, BAR(FULLB + s), 64 * x, td.j * BN, bh);
+                        tma_load_3d(dst + x * HALF_BYTES, tm, BAR(FULLB + s), 64 * x, row0, bh);
                 } else {
                     // two 64-row boxes per 64-column box: the same swizzled layout as
                     // one 128-row box; an empty half repeats the first block (its
