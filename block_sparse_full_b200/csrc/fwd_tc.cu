@@ -525,17 +525,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             float mx = max3(max3(mx8[0], mx8[1], mx8[2]), max3(mx8[3], mx8[4], mx8[5]),
                             fmaxf(mx8[6], mx8[7]));
-            float* xm = xch + (jj & 1) * 256;
-            xm[wg * 128 + r] = mx;
-            if (pair_vote(!got || *abort_flag)) {  // a wait expired somewhere: both leave here
-                ok = false;
-                break;
-            }
-            mx = fmaxf(mx, xm[(1 - wg) * 128 + r]);
-            const float mnew = mx * sl2;
-            if (jj == 0) {
-                m2 = mnew;
-            } else {
+            // The two warps holding these rows exchange their halves' maxima only
+            // when the running max must move: on the first tile, or when either
+            // half of some row exceeds it by more than the lazy-rescale threshold
+            // (the same rows rescale as with an exchange on every tile, since
+            // max(a, b) > t exactly when a > t or b > t).
+            const bool moved = jj == 0 || mx * sl2 > m2 + kRescaleThreshold;
+            if (pair_vote(moved || !got || *abort_flag)) {
+                float* xm = xch + (jj & 1) * 256;
+                xm[wg * 128 + r] = mx;
+                if (pair_vote(!got || *abort_flag)) {  // a wait expired somewhere: both leave here
+                    ok = false;
+                    break;
+                }
+                mx = fmaxf(mx, xm[(1 - wg) * 128 + r]);
+                const float mnew = mx * sl2;
+                if (jj == 0) {
+                    m2 = mnew;
+                } else {
                 const bool need = mnew > m2 + kRescaleThreshold;
                 // PV_{j-1} must have landed in O before it is rescaled.  If that wait
                 // expires the rescale is skipped and the abort flag ends the loop at
@@ -562,6 +569,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         tmem_st32(trow + col, u);
                     }
                     tmem_wait_st();
+                }
                 }
             }
             const float negm = -m2;
