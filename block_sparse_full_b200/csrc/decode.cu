@@ -88,19 +88,20 @@ constexpr int kSplitRankMin = 192;
 __device__ unsigned int g_decode_status;
 
 // Shared memory of the step kernel, the same layout in every CTA of a cluster:
-//   order keys [nb] u64 (every CTA holds all of them) | set bitmask [nb / 32 + 1] u32 |
-//   selected blocks [topk] i32 | popcount prefix of the bitmask words [nb / 32 + 2] i32 | partials [cluster][2 + D] f32 (the leader's
-//   are used) | scores [nbuf * block] f32 | p [nbuf * block] bf16 | o partial
-//   sums [KG][D] f32 | mbarriers (copies, partials) | keys [nbuf][block][D] T
-//   (bf16: per block, D / 64 tiles [block][64] in the 128-byte swizzle) |
-//   values likewise.
+//   order keys of the block scores [nb] u64 (every CTA holds all of them) |
+//   set bitmask [nb / 32 + 1] u32 | selected blocks [topk] i32 | popcount
+//   prefix of the bitmask words [nb / 32 + 2] i32 | partials [cluster][2 + D]
+//   f32 (the leader's are used) | attention scores [nbuf * block] f32 |
+//   p [nbuf * block] bf16 | o partial sums [KG][D] f32 | mbarriers (copies,
+//   partials) | keys [nbuf][block][D] T (bf16: per block, D / 64 tiles
+//   [block][64] in the 128-byte swizzle) | values likewise.
 struct StepSmem {
-    size_t score, bits, sel, wpre, part, ps, pb, og, bar, kbuf, vbuf, total;
+    size_t key, bits, sel, wpre, part, ps, pb, og, bar, kbuf, vbuf, total;
     __host__ __device__ StepSmem(int nb, int topk, int D, int cluster, int nbuf, int block, int esize,
                                  int threads) {
         auto up = [](size_t x, size_t a) { return (x + a - 1) / a * a; };
-        score = 0;
-        bits = score + (size_t)nb * 8;
+        key = 0;
+        bits = key + (size_t)nb * 8;
         sel = bits + ((size_t)nb / 32 + 1) * 4;
         wpre = sel + (size_t)topk * 4;
         part = up(wpre + ((size_t)nb / 32 + 2) * 4, 16);
@@ -211,7 +212,7 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     // the 128-byte swizzle of the TMA tiles follows address bits 7-9: the
     // layout starts on a 1024-byte boundary (the same offset in every CTA)
     unsigned char* sm = sm_raw + ((1024u - (smem_u32(sm_raw) & 1023u)) & 1023u);
-    uint64_t* key = reinterpret_cast<uint64_t*>(sm + L.score);
+    uint64_t* key = reinterpret_cast<uint64_t*>(sm + L.key);
     uint32_t* bits = reinterpret_cast<uint32_t*>(sm + L.bits);
     int32_t* sel = reinterpret_cast<int32_t*>(sm + L.sel);
     int32_t* wpre = reinterpret_cast<int32_t*>(sm + L.wpre);
