@@ -607,7 +607,16 @@ decode_step_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
     // 4. the leader merges the partials once the other CTAs' have arrived:
     // weights e^{m_r - M}
-    if (!__syncthreads_and(wait_phase(bar_part, 0, true, limit_ns))) return;
+    if (!__syncthreads_and(wait_phase(bar_part, 0, true, limit_ns))) {
+        // The others write their partials into this CTA's shared memory before
+        // they arrive, so it must not exit while one may still write.  Each of
+        // them gives up after at most one expired wait per pass (this CTA has
+        // the most passes) and one drain: wait that long again (bounded), then
+        // leave with the status already recorded and no output.
+        const int npass = (mine + nbuf - 1) / nbuf;
+        wait_phase(bar_part, 0, true, (uint64_t)(npass + 1) * limit_ns + kDrainLimitNs);
+        return;
+    }
     __shared__ float wgt[8];
     if (warp == 0) {
         const float mr = lane < kCluster ? part[lane * (2 + D)] : -INFINITY;

@@ -67,3 +67,38 @@ def test_short_kernel_wait_limit_keeps_context_usable():
     for name in ("h_full", "h_sparse"):
         err = np.abs(out[name].float().cpu().numpy() - ref[name]).max()
         assert err <= 1e-2 * np.abs(ref[name]).max()
+
+
+def test_short_wait_limit_in_the_decode_step():
+    # The decode step's waits (its copies, and the leader's wait for the other
+    # CTAs' partials) expire under a 100 ns limit; the leader then waits for
+    # the partials that are still being written into its shared memory before
+    # it leaves.  The context stays usable and the next step is exact.
+    w = Workload("fail_bf16_decode", B=1, H=4, T=8192, D=128, block=64, topk=16, dtype="bf16",
+                 plant="hot", seed=32)
+    inp = make_inputs(w)
+    p = ssa.params_for(inp["q"].cuda(), w.block, w.topk, w.sm_scale)
+    cache = ssa.DecodeCache(p, "cuda", inp["k"].dtype)
+    cache.k.copy_(inp["k"].cuda())
+    cache.v.copy_(inp["v"].cuda())
+    t = w.T - 1
+    q_t = inp["q"][:, :, t].contiguous()
+    good = cache.step(t, q_t.cuda())
+    good = {n: x.clone() for n, x in good.items()}
+    torch.cuda.synchronize()
+    assert ssa.ssa_device_status(_stream()) == ssa.SSA_OK
+    ssa.ssa_debug_set_wait_limit_ns(100)
+    try:
+        cache.step(t, q_t.cuda())
+        assert ssa.ssa_device_status(_stream()) in (ssa.SSA_OK, ssa.SSA_ERR_TIMEOUT)
+    finally:
+        ssa.ssa_debug_set_wait_limit_ns(0)
+    out = cache.step(t, q_t.cuda())
+    torch.cuda.synchronize()
+    assert ssa.ssa_device_status(_stream()) == ssa.SSA_OK
+    for name in good:
+        assert torch.equal(out[name], good[name]), name
+    ref = O.decode_step(q_t, inp["k"], inp["v"], t, w.block, w.topk, w.sm_scale)
+    np.testing.assert_array_equal(out["idx"].cpu().numpy(), ref["idx"])
+    err = np.abs(out["h"].float().cpu().numpy() - ref["h"]).max()
+    assert err <= 1e-2 * np.abs(ref["h"]).max()
