@@ -262,8 +262,9 @@ class Layer:
         self.path = ssa.ssa_kernel_path(self.p)
 
     def launches_per_step(self):
-        # select: pool + score; fwd: 1; loss: 2; bwd: pre + dk/dv + dq (either path)
-        return 2 + 1 + 2 + 3
+        # select: pool + score; fwd: 1; loss: 2; bwd: pre + dk/dv + dq on the
+        # tensor-core path, pre + one dq-and-dk/dv grid on the CUDA-core path
+        return 2 + 1 + 2 + (3 if self.path == 1 else 2)
 
     def run_sparse_fwd(self, stream):
         """The sparse stream alone (inference mode) on the step's selection."""

@@ -13,9 +13,10 @@
 //   with D_f = G_f.h_full and D_s = G_s.h_sparse (row dots),
 //   dq_t = sigma sum_s dS k_s,  dk_s = sigma sum_t dS q_t,
 //   dv_s = sum_t P_f G_f(t) + [sel] P_s G_s(t).
-// Three kernels: a row preprocess (G_f, G_s, D_f, D_s into the workspace), a
-// dq kernel over query tiles and a dk/dv kernel over key tiles; no atomics,
-// so results are bitwise repeatable.
+// Two launches: a row preprocess (G_f, G_s, D_f, D_s into the workspace),
+// then one grid whose CTAs take either a query tile (dq) or a key tile
+// (dk/dv), the two kinds interleaved; no atomics, so results are bitwise
+// repeatable.
 #include "device_util.cuh"
 #include "ssa_internal.h"
 
@@ -77,18 +78,21 @@ struct DqSmem {
     uint32_t mrow[256];
 };
 
+// dq of query tile L's 16 rows (tiles in longest-first order)
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
-bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-              const uint32_t* __restrict__ mask, const float* __restrict__ lse_f,
-              const float* __restrict__ lse_s, BwdWs w, int BH, int T_, int block, int words,
-              float sm_scale, T* __restrict__ dq) {
+__device__ __forceinline__ void dq_tile(DqSmem<D>& sm, int L, const T* __restrict__ q,
+                                        const T* __restrict__ k, const T* __restrict__ v,
+                                        const uint32_t* __restrict__ mask,
+                                        const float* __restrict__ lse_f,
+                                        const float* __restrict__ lse_s, const BwdWs& w, int BH,
+                                        int T_, int block, int words, float sm_scale,
+                                        T* __restrict__ dq) {
     constexpr int DPL = D / 32;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    DqSmem<D>& sm = *reinterpret_cast<DqSmem<D>*>(smem_raw);
+    constexpr int kNE = kChunk * D / kThreads;  // elements per thread of a chunk operand
+    static_assert(kNE * kThreads == kChunk * D, "whole chunks per CTA");
     const int ntiles = T_ / kRowsB;
-    const int tile = ntiles - 1 - (int)(blockIdx.x / BH);
-    const size_t bh = blockIdx.x % BH;
+    const int tile = ntiles - 1 - L / BH;
+    const size_t bh = L % BH;
     const int t0 = tile * kRowsB;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t base = bh * (size_t)T_ * D;
@@ -116,15 +120,29 @@ bwd_dq_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restr
         for (int u = 0; u < DPL; ++u) acc[r][u] = 0.f;
 
     // chunks of 32 keys from 0 (a chunk lies inside one key block; keys past a
-    // row are masked)
-    for (int s0 = 0; s0 < t0 + kRowsB; s0 += kChunk) {
+    // row are masked); chunk c + 1 is loaded into registers while chunk c is
+    // computed
+    T kn[kNE], vn[kNE];
+    auto fetch = [&](int s0) {
+#pragma unroll
+        for (int x = 0; x < kNE; ++x) {
+            const size_t g = base + (size_t)s0 * D + tid + x * kThreads;
+            kn[x] = k[g];
+            vn[x] = v[g];
+        }
+    };
+    const int send = t0 + kRowsB;  // chunks starting below send end at or before T
+    fetch(0);
+    for (int s0 = 0; s0 < send; s0 += kChunk) {
         __syncthreads();
-        for (int e = tid; e < kChunk * D; e += kThreads) {
-            const size_t g = base + (size_t)s0 * D + e;
-            sm.k[e / D][e % D] = to_f32(k[g]);
-            sm.v[e / D][e % D] = to_f32(v[g]);
+#pragma unroll
+        for (int x = 0; x < kNE; ++x) {
+            const int e = tid + x * kThreads;
+            sm.k[e / D][e % D] = to_f32(kn[x]);
+            sm.v[e / D][e % D] = to_f32(vn[x]);
         }
         __syncthreads();
+        if (s0 + kChunk < send) fetch(s0 + kChunk);
         const bool sel = mask_bit(sm.mrow, s0 / block);
 #pragma unroll 1
         for (int r = 0; r < kRowsPerWarp; ++r) {
@@ -170,17 +188,20 @@ struct DkvSmem {
     float lf[kChunk], ls[kChunk], df[kChunk], ds[kChunk];
 };
 
+// dk, dv of key tile L's 16 rows (key tile 0 sees every query: first)
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads)
-bwd_dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                const uint32_t* __restrict__ mask, const float* __restrict__ lse_f,
-                const float* __restrict__ lse_s, BwdWs w, int BH, int T_, int block, int words,
-                float sm_scale, T* __restrict__ dk, T* __restrict__ dv) {
+__device__ __forceinline__ void dkdv_tile(DkvSmem<D>& sm, int L, const T* __restrict__ q,
+                                          const T* __restrict__ k, const T* __restrict__ v,
+                                          const uint32_t* __restrict__ mask,
+                                          const float* __restrict__ lse_f,
+                                          const float* __restrict__ lse_s, const BwdWs& w, int BH,
+                                          int T_, int block, int words, float sm_scale,
+                                          T* __restrict__ dk, T* __restrict__ dv) {
     constexpr int DPL = D / 32;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    DkvSmem<D>& sm = *reinterpret_cast<DkvSmem<D>*>(smem_raw);
-    const int tile = (int)(blockIdx.x / BH);  // key tile 0 sees every query: first
-    const size_t bh = blockIdx.x % BH;
+    constexpr int kNE = kChunk * D / kThreads;  // elements per thread of a chunk operand
+    static_assert(kNE * kThreads == kChunk * D, "whole chunks per CTA");
+    const int tile = L / BH;
+    const size_t bh = L % BH;
     const int s_base = tile * kRowsB;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const size_t base = bh * (size_t)T_ * D;
@@ -199,23 +220,45 @@ bwd_dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         for (int u = 0; u < DPL; ++u) adk[r][u] = adv[r][u] = 0.f;
 
     // chunks of 32 queries from the 32-aligned chunk holding the first key (a
-    // chunk lies inside one query block; queries before a key are masked)
-    for (int t0 = s_base & ~(kChunk - 1); t0 < T_; t0 += kChunk) {
-        __syncthreads();
-        for (int e = tid; e < kChunk * D; e += kThreads) {
-            const size_t g = base + (size_t)t0 * D + e;
-            sm.q[e / D][e % D] = to_f32(q[g]);
-            sm.gf[e / D][e % D] = w.gf[g];
-            sm.gs[e / D][e % D] = w.gs[g];
+    // chunk lies inside one query block; queries before a key are masked);
+    // chunk c + 1 is loaded into registers while chunk c is computed
+    T qn[kNE];
+    float gfn[kNE], gsn[kNE], lfn = 0.f, lsn = 0.f, dfn = 0.f, dsn = 0.f;
+    auto fetch = [&](int t0) {
+#pragma unroll
+        for (int x = 0; x < kNE; ++x) {
+            const size_t g = base + (size_t)t0 * D + tid + x * kThreads;
+            qn[x] = q[g];
+            gfn[x] = w.gf[g];
+            gsn[x] = w.gs[g];
         }
         if (tid < kChunk) {
             const size_t rr = bh * (size_t)T_ + t0 + tid;
-            sm.lf[tid] = lse_f[rr];
-            sm.ls[tid] = lse_s[rr];
-            sm.df[tid] = w.df[rr];
-            sm.ds[tid] = w.ds[rr];
+            lfn = lse_f[rr];
+            lsn = lse_s[rr];
+            dfn = w.df[rr];
+            dsn = w.ds[rr];
+        }
+    };
+    const int tbeg = s_base & ~(kChunk - 1);  // T is a multiple of 64: chunks end at or before T
+    fetch(tbeg);
+    for (int t0 = tbeg; t0 < T_; t0 += kChunk) {
+        __syncthreads();
+#pragma unroll
+        for (int x = 0; x < kNE; ++x) {
+            const int e = tid + x * kThreads;
+            sm.q[e / D][e % D] = to_f32(qn[x]);
+            sm.gf[e / D][e % D] = gfn[x];
+            sm.gs[e / D][e % D] = gsn[x];
+        }
+        if (tid < kChunk) {
+            sm.lf[tid] = lfn;
+            sm.ls[tid] = lsn;
+            sm.df[tid] = dfn;
+            sm.ds[tid] = dsn;
         }
         __syncthreads();
+        if (t0 + kChunk < T_) fetch(t0 + kChunk);
         const uint32_t* mrow = mask + (bh * n + t0 / block) * (size_t)words;
         const bool sel = mask_bit(mrow, kblk);
         const int t = t0 + lane;
@@ -266,6 +309,31 @@ bwd_dkdv_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
     }
 }
 
+// dq and dk/dv in one grid: even CTAs take dk/dv key tiles, odd ones dq query
+// tiles, each role in its own longest-first order, so the two run side by
+// side instead of one after the other.
+template <int D>
+union BwdSmem {
+    DqSmem<D> dq;
+    DkvSmem<D> kv;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+bwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                const uint32_t* __restrict__ mask, const float* __restrict__ lse_f,
+                const float* __restrict__ lse_s, BwdWs w, int BH, int T_, int block, int words,
+                float sm_scale, T* __restrict__ dq, T* __restrict__ dk, T* __restrict__ dv) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    BwdSmem<D>& sm = *reinterpret_cast<BwdSmem<D>*>(smem_raw);
+    const int L = (int)(blockIdx.x >> 1);
+    if (blockIdx.x & 1u)
+        dq_tile<T, D>(sm.dq, L, q, k, v, mask, lse_f, lse_s, w, BH, T_, block, words, sm_scale, dq);
+    else
+        dkdv_tile<T, D>(sm.kv, L, q, k, v, mask, lse_f, lse_s, w, BH, T_, block, words, sm_scale, dk,
+                        dv);
+}
+
 template <typename T, int D>
 int launch_typed(const ssa_params_t& p, const void* q, const void* k, const void* v,
                  const uint32_t* mask, const void* hf, const void* hs, const float* lf,
@@ -281,25 +349,16 @@ int launch_typed(const ssa_params_t& p, const void* q, const void* k, const void
     if (st != SSA_OK) return st;
 
     const int BH = p.B * p.H;
-    const unsigned grid = (unsigned)((size_t)BH * (p.T / kRowsB));
-    size_t smem = sizeof(DqSmem<D>);
-    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<T, D>,
+    const unsigned grid = (unsigned)(2 * (size_t)BH * (p.T / kRowsB));  // dk/dv and dq tiles
+    const size_t smem = sizeof(BwdSmem<D>);
+    cudaError_t e = cudaFuncSetAttribute(bwd_simt_kernel<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "bwd_dq: smem attribute: %s", cudaGetErrorString(e));
-    bwd_dq_kernel<T, D><<<grid, kThreads, smem, s>>>(
+    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "bwd_simt: smem attribute: %s", cudaGetErrorString(e));
+    bwd_simt_kernel<T, D><<<grid, kThreads, smem, s>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), mask, lf, ls,
-        w, BH, p.T, p.block, mask_words(p), p.sm_scale, static_cast<T*>(dq));
-    st = check_launch("bwd_dq_kernel");
-    if (st != SSA_OK) return st;
-
-    smem = sizeof(DkvSmem<D>);
-    e = cudaFuncSetAttribute(bwd_dkdv_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return fail(SSA_ERR_CUDA, "bwd_dkdv: smem attribute: %s", cudaGetErrorString(e));
-    bwd_dkdv_kernel<T, D><<<grid, kThreads, smem, s>>>(
-        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), mask, lf, ls,
-        w, BH, p.T, p.block, mask_words(p), p.sm_scale, static_cast<T*>(dk), static_cast<T*>(dv));
-    return check_launch("bwd_dkdv_kernel");
+        w, BH, p.T, p.block, mask_words(p), p.sm_scale, static_cast<T*>(dq), static_cast<T*>(dk),
+        static_cast<T*>(dv));
+    return check_launch("bwd_simt_kernel");
 }
 
 }  // namespace
@@ -314,7 +373,7 @@ int launch_bwd_simt(const ssa_params_t& p, const void* q, const void* k, const v
                     const float* ls, const void* dhf, const void* dhs, float w_s, float w_c,
                     void* dq, void* dk, void* dv, void* ws, cudaStream_t s) {
     if (mask_words(p) > 256) return fail(SSA_ERR_UNSUPPORTED, "bwd_simt: more than 8192 blocks");
-    if ((size_t)p.B * p.H * (p.T / kRowsB) > 0x7fffffffull)
+    if (2 * (size_t)p.B * p.H * (p.T / kRowsB) > 0x7fffffffull)
         return fail(SSA_ERR_UNSUPPORTED, "bwd_simt: grid too large");
     const bool bf = p.dtype == SSA_BF16;
 #define SSA_BWD_ARGS p, q, k, v, mask, hf, hs, lf, ls, dhf, dhs, w_s, w_c, dq, dk, dv, ws, s

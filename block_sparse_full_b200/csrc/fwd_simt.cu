@@ -8,7 +8,8 @@
 // through shared memory in chunks of 32 keys; lane j owns key j of the chunk
 // for the logits and dimension lane + 32u of the accumulators.  A chunk lies
 // inside one key block and the CTA's rows inside one query block, so the
-// selection test (sparse stream or not) is one mask bit per chunk.  Online
+// selection test (sparse stream or not) is one mask bit per chunk.  The next
+// chunk's loads are in flight while a chunk is computed.  Online
 // softmax with one running max shared by both streams:
 //   l_sel, l_uns  running sums over selected / unselected keys,
 //   O_sel, O_uns  running weighted sums of v,
@@ -70,14 +71,31 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         for (int u = 0; u < DPL; ++u) osel[r][u] = ouns[r][u] = 0.f;
     }
 
-    for (int s0 = 0; s0 < t0 + kRows; s0 += kKeys) {
+    // chunk c + 1's keys and values are loaded into registers while chunk c
+    // is computed, and stored to shared memory after it
+    constexpr int NE = kKeys * D / kThreads;  // elements per thread per chunk and operand
+    static_assert(NE * kThreads == kKeys * D, "whole chunks per CTA");
+    T kn[NE], vn[NE];
+    auto fetch = [&](int s0) {
+#pragma unroll
+        for (int x = 0; x < NE; ++x) {
+            const size_t g = base + (size_t)s0 * D + tid + x * kThreads;
+            kn[x] = k[g];
+            vn[x] = v[g];
+        }
+    };
+    const int send = t0 + kRows;  // chunks [s0, s0 + 32) with s0 < send end at or before T
+    fetch(0);
+    for (int s0 = 0; s0 < send; s0 += kKeys) {
         __syncthreads();
-        for (int e = tid; e < kKeys * D; e += kThreads) {
-            const size_t g = base + (size_t)s0 * D + e;
-            sm.k[e / D][e % D] = to_f32(k[g]);
-            sm.v[e / D][e % D] = to_f32(v[g]);
+#pragma unroll
+        for (int x = 0; x < NE; ++x) {
+            const int e = tid + x * kThreads;
+            sm.k[e / D][e % D] = to_f32(kn[x]);
+            sm.v[e / D][e % D] = to_f32(vn[x]);
         }
         __syncthreads();
+        if (s0 + kKeys < send) fetch(s0 + kKeys);
         const bool chunk_sel = mask_bit(sm.mrow, s0 / block);
 #pragma unroll
         for (int r = 0; r < kRowsPerWarp; ++r) {
