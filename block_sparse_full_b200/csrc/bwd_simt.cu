@@ -70,10 +70,47 @@ bwd_pre_kernel(const T* __restrict__ hf, const T* __restrict__ hs, const T* __re
     }
 }
 
+// a + x[0] y[0] + x[1] y[1] + ... + x[D-1] y[D-1], one fused multiply-add per
+// column in column order (the rounding of a plain loop), four columns per
+// shared-memory load; x and y are 16-byte aligned.
+template <int D>
+__device__ __forceinline__ float dot_seq(const float* x, const float* y, float a) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* y4 = reinterpret_cast<const float4*>(y);
+#pragma unroll 4
+    for (int c = 0; c < D / 4; ++c) {
+        const float4 p = x4[c], q = y4[c];
+        a = fmaf(p.x, q.x, a);
+        a = fmaf(p.y, q.y, a);
+        a = fmaf(p.z, q.z, a);
+        a = fmaf(p.w, q.w, a);
+    }
+    return a;
+}
+// two such sums side by side (independent chains, the same order in each)
+template <int D>
+__device__ __forceinline__ void dot2_seq(const float* x0, const float* y0, float& a0, const float* x1,
+                                         const float* y1, float& a1) {
+    const float4 *p4 = reinterpret_cast<const float4*>(x0), *q4 = reinterpret_cast<const float4*>(y0);
+    const float4 *r4 = reinterpret_cast<const float4*>(x1), *s4 = reinterpret_cast<const float4*>(y1);
+#pragma unroll 4
+    for (int c = 0; c < D / 4; ++c) {
+        const float4 p = p4[c], q = q4[c], r = r4[c], s = s4[c];
+        a0 = fmaf(p.x, q.x, a0);
+        a1 = fmaf(r.x, s.x, a1);
+        a0 = fmaf(p.y, q.y, a0);
+        a1 = fmaf(r.y, s.y, a1);
+        a0 = fmaf(p.z, q.z, a0);
+        a1 = fmaf(r.z, s.z, a1);
+        a0 = fmaf(p.w, q.w, a0);
+        a1 = fmaf(r.w, s.w, a1);
+    }
+}
+
 template <int D>
 struct DqSmem {
     float q[kRowsB][D], gf[kRowsB][D], gs[kRowsB][D];
-    float k[kChunk][D + 1], v[kChunk][D + 1];
+    float k[kChunk][D + 4], v[kChunk][D + 4];  // +4: 16-byte rows, conflict-free per lane
     float lf[kRowsB], ls[kRowsB], df[kRowsB], ds[kRowsB];
     uint32_t mrow[256];
 };
@@ -150,17 +187,12 @@ __device__ __forceinline__ void dq_tile(DqSmem<D>& sm, int L, const T* __restric
             const int t = t0 + rr;
             const bool valid = s0 + lane <= t;
             float x = 0.f, dpf = 0.f, dps = 0.f;
-#pragma unroll 16
-            for (int c = 0; c < D; ++c) {
-                x = fmaf(sm.q[rr][c], sm.k[lane][c], x);
-                dpf = fmaf(sm.gf[rr][c], sm.v[lane][c], dpf);
-            }
+            dot2_seq<D>(sm.q[rr], sm.k[lane], x, sm.gf[rr], sm.v[lane], dpf);
             x *= sm_scale;
             const float pf = valid ? expf(x - sm.lf[rr]) : 0.f;
             float dsv = pf * (dpf - sm.df[rr]);
             if (sel) {
-#pragma unroll 16
-                for (int c = 0; c < D; ++c) dps = fmaf(sm.gs[rr][c], sm.v[lane][c], dps);
+                dps = dot_seq<D>(sm.gs[rr], sm.v[lane], dps);
                 const float lsr = sm.ls[rr];
                 const float ps = (valid && lsr > -INFINITY) ? expf(x - lsr) : 0.f;
                 dsv += ps * (dps - sm.ds[rr]);
@@ -184,7 +216,7 @@ __device__ __forceinline__ void dq_tile(DqSmem<D>& sm, int L, const T* __restric
 template <int D>
 struct DkvSmem {
     float k[kRowsB][D], v[kRowsB][D];
-    float q[kChunk][D + 1], gf[kChunk][D + 1], gs[kChunk][D + 1];
+    float q[kChunk][D + 4], gf[kChunk][D + 4], gs[kChunk][D + 4];  // as above
     float lf[kChunk], ls[kChunk], df[kChunk], ds[kChunk];
 };
 
@@ -268,18 +300,13 @@ __device__ __forceinline__ void dkdv_tile(DkvSmem<D>& sm, int L, const T* __rest
             const int s = s_base + rr;
             const bool valid = t >= s;
             float x = 0.f, dpf = 0.f, dps = 0.f;
-#pragma unroll 16
-            for (int c = 0; c < D; ++c) {
-                x = fmaf(sm.q[lane][c], sm.k[rr][c], x);
-                dpf = fmaf(sm.gf[lane][c], sm.v[rr][c], dpf);
-            }
+            dot2_seq<D>(sm.q[lane], sm.k[rr], x, sm.gf[lane], sm.v[rr], dpf);
             x *= sm_scale;
             const float pf = valid ? expf(x - sm.lf[lane]) : 0.f;
             float dsv = pf * (dpf - sm.df[lane]);
             float ps = 0.f;
             if (sel) {
-#pragma unroll 16
-                for (int c = 0; c < D; ++c) dps = fmaf(sm.gs[lane][c], sm.v[rr][c], dps);
+                dps = dot_seq<D>(sm.gs[lane], sm.v[rr], dps);
                 const float lsr = sm.ls[lane];
                 ps = (valid && lsr > -INFINITY) ? expf(x - lsr) : 0.f;
                 dsv += ps * (dps - sm.ds[lane]);

@@ -30,10 +30,28 @@ constexpr int kRowsPerWarp = kRows / (kThreads / 32);
 template <int D>
 struct FwdSmem {
     float q[kRows][D];
-    float k[kKeys][D + 1];  // +1: lane j reads row j, conflict-free
+    float k[kKeys][D + 4];  // +4: lane j reads row j 16 bytes at a time, conflict-free
     float v[kKeys][D];
     uint32_t mrow[256];     // mask words of this CTA's query block
 };
+
+// a + x[0] y[0] + x[1] y[1] + ... + x[D-1] y[D-1], one fused multiply-add per
+// column in column order (the rounding of a plain loop), four columns per
+// shared-memory load; x and y are 16-byte aligned.
+template <int D>
+__device__ __forceinline__ float dot_seq(const float* x, const float* y, float a) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* y4 = reinterpret_cast<const float4*>(y);
+#pragma unroll 4
+    for (int c = 0; c < D / 4; ++c) {
+        const float4 p = x4[c], q = y4[c];
+        a = fmaf(p.x, q.x, a);
+        a = fmaf(p.y, q.y, a);
+        a = fmaf(p.z, q.z, a);
+        a = fmaf(p.w, q.w, a);
+    }
+    return a;
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
@@ -101,9 +119,7 @@ fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __res
         for (int r = 0; r < kRowsPerWarp; ++r) {
             const int rr = warp * kRowsPerWarp + r;
             const int t = t0 + rr;
-            float x = 0.f;
-#pragma unroll 16
-            for (int c = 0; c < D; ++c) x = fmaf(sm.q[rr][c], sm.k[lane][c], x);
+            float x = dot_seq<D>(sm.q[rr], sm.k[lane], 0.f);
             const bool valid = s0 + lane <= t;
             x = valid ? x * sm_scale : -INFINITY;
             const float mnew = fmaxf(m[r], warp_max(x));  // key s0 <= t always valid
