@@ -27,6 +27,43 @@ def test_header_declarations_are_exported():
     assert sorted(ssa.EXPORTS) == names
 
 
+def _prototypes():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return {name: args.strip()
+            for name, args in re.findall(r"\b(ssa_\w+)\s*\(([^;{)]*)\)\s*;", src)}
+
+
+def _ctype_class(c_decl):
+    # the ctypes argument class a C parameter declaration needs
+    t = re.sub(r"\b(const|restrict)\b", "", c_decl).strip()
+    if "ssa_params_t" in t:
+        return "params"
+    if "*" in t or t.startswith("cudaStream_t"):
+        return "pointer"
+    base = t.split()[:-1] if len(t.split()) > 1 else t.split()
+    base = " ".join(base)
+    # size_t and unsigned long long are both unsigned 64-bit here (and one
+    # ctypes type on LP64)
+    return {"int": "int", "size_t": "u64", "float": "float", "unsigned long long": "u64"}[base]
+
+
+def test_binding_signatures_match_the_header():
+    # every prototype's parameter list, argument by argument, against the
+    # ctypes signature the binding installs: a drift between the two would pass
+    # wrong-width arguments silently
+    cls = {ctypes.c_void_p: "pointer", ctypes.c_int: "int", ctypes.c_size_t: "u64",
+           ctypes.c_float: "float", ctypes.c_ulonglong: "u64"}
+    assert ctypes.sizeof(ctypes.c_size_t) == ctypes.sizeof(ctypes.c_ulonglong) == 8
+    protos = _prototypes()
+    assert sorted(protos) == declared_functions()
+    for name, args in protos.items():
+        want = [] if args in ("", "void") else [_ctype_class(a) for a in args.split(",")]
+        got = [("params" if a is ssa._P else cls[a]) for a in ssa._SIGNATURES[name][1]]
+        assert got == want, (name, got, want)
+
+
 def test_exports_are_c_symbols():
     # plain C names, no C++ mangling
     out = os.popen(f"nm -D --defined-only {ssa.LIB_PATH}").read()
