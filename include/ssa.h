@@ -196,8 +196,9 @@ int ssa_attn_fwd_sparse(const ssa_params_t* params, const void* q, const void* k
  *   k_cache and v_cache must be 16-byte aligned (the selected blocks are
  *   copied with bulk copies).  A bulk copy or a hand-off that does not
  *   complete within the wait limit makes ssa_device_status return
- *   SSA_ERR_TIMEOUT; h and lse of the heads concerned are then not written
- *   (idx is), and the launch still ends only after every CTA of each
+ *   SSA_ERR_TIMEOUT; h and lse of the heads concerned are then undefined
+ *   (left unwritten, or formed without the blocks whose copies expired; idx
+ *   is still exact), and the launch still ends only after every CTA of each
  *   cluster has stopped writing into the others' shared memory.
  */
 int ssa_decode_pool(const ssa_params_t* params, int j0, int j1, const void* k_cache,
