@@ -35,8 +35,9 @@
  *     anything is launched; launch errors return SSA_ERR_CUDA.  A kernel
  *     whose bounded wait expired records SSA_ERR_TIMEOUT in a device status
  *     word that ssa_device_status() reports after synchronising; the outputs
- *     of the calls made since the last check are then undefined (inputs and
- *     workspaces are not corrupted, and later calls run normally).
+ *     of the calls made since the last check are then undefined (nothing
+ *     outside their outputs and workspaces is written, and later calls run
+ *     normally).
  *   - Alignment: every device pointer 16-byte aligned; the bf16 tensor-core
  *     path takes D == 64 or 128.
  */
